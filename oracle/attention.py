@@ -1,0 +1,202 @@
+"""Plain float64 CPU oracle for decode attention and chunked-prefill attention.
+
+TEST INFRASTRUCTURE ONLY. Nothing on the product path imports this module: only the
+tests, ``__graft_entry__.smoke()`` and ``bench.py`` (its CPU-baseline leg and its
+``--impl reference`` arm) may call it. It shares no code with the CUDA library.
+
+Sources (web pages, cited by title and section):
+
+* "大语言模型长序列推理优化：ChunkedPrefill与FlashDecoding技术解析"
+  (LLM long-sequence inference: ChunkedPrefill and FlashDecoding), below "ChunkedPrefill page".
+  §2.1 gives chunk attention: scores = q·Kᵀ/√d_head over the cache with the chunk's own
+  K/V appended first, under a causal mask. §3.1 gives decode attention as a
+  softmax-weighted sum of V rows computed block by block with an online softmax.
+* "大模型推理加速FlashDecoding算法原理与多GPU并行解码实战"
+  (FlashDecoding algorithm and multi-GPU decoding), below "FlashDecoding page".
+  Section "FlashDecoding算法原理与标准注意力机制对比" fixes the shapes
+  Q [batch, heads, 1, head_dim], K/V [batch, heads, seq_len, head_dim] and the scaled
+  score q·kᵀ/√head_dim; section "多GPU张量并行扩展下的FlashDecoding实现" masks keys at
+  positions >= cache_lens; section "部署落地的工程细节" item 3 maps the query heads of a
+  GQA group onto one KV head.
+
+What is computed (the plain definition; FlashDecoding reaches exactly this result up to
+rounding, so the oracle is the definition itself with no splitting):
+
+    for each batch row b and query head h, with kv = h // G (G = Hq / Hkv), n = len_b:
+        s_j  = (q_h · k_j) * scale            j < n,   scale = 1/sqrt(D) by default
+        M    = max_j s_j
+        O    = sum_j exp(s_j - M) v_j / sum_j exp(s_j - M)
+        LSE  = M + ln sum_j exp(s_j - M)              (natural log of the scaled scores)
+
+Readings where the pages are silent (each is listed in the design doc):
+
+* n = 0 gives O = 0 and LSE = -inf.
+* A cache length outside [0, S_cap] is clamped into that range (the CUDA side clamps too
+  and raises a status flag).
+* A chunk row i of request b sees keys j <= prefix_len_b + i (bottom-right causal
+  alignment: the chunk's K/V already sit in the cache at [prefix, prefix + chunk_len)).
+
+Inputs are numpy arrays: float32 / float64 values, or uint16 arrays holding the raw bits of
+bf16 values. Every value is widened exactly to float64 before any arithmetic.
+"""
+
+from __future__ import annotations
+
+import math
+from typing import Iterable, Optional, Sequence, Tuple
+
+import numpy as np
+
+__all__ = [
+    "widen",
+    "decode_attention",
+    "chunk_prefill_attention",
+    "attention_rows",
+]
+
+
+def widen(x: np.ndarray) -> np.ndarray:
+    """Exact float64 copy of ``x``.
+
+    uint16 arrays are bf16 bit patterns: a bf16 number is the upper 16 bits of an IEEE
+    binary32, so shifting the bits up by 16 gives the binary32 with the same value, and
+    binary32 -> binary64 is exact.
+    """
+    x = np.asarray(x)
+    if x.dtype == np.uint16:
+        return (x.astype(np.uint32) << np.uint32(16)).view(np.float32).astype(np.float64)
+    if x.dtype in (np.float32, np.float64):
+        return x.astype(np.float64)
+    raise TypeError(f"oracle: unsupported input dtype {x.dtype}")
+
+
+def attention_rows(q_rows: np.ndarray, keys: np.ndarray, values: np.ndarray,
+                   n_visible: Sequence[int], scale: float) -> Tuple[np.ndarray, np.ndarray]:
+    """Softmax attention of several query rows over a prefix of one key/value sequence.
+
+    q_rows [R, D] float64, keys/values [N, D] float64, n_visible[r] = number of leading keys
+    row r may see. Returns (O [R, D], LSE [R]) in float64. This is the definition written out
+    once per row: scores, max, exponentials, normalised weighted sum, log-sum-exp.
+    """
+    R, D = q_rows.shape
+    out = np.zeros((R, D), dtype=np.float64)
+    lse = np.full((R,), -np.inf, dtype=np.float64)
+    for r in range(R):
+        n = int(n_visible[r])
+        if n <= 0:
+            continue  # no visible key: O = 0, LSE = -inf
+        s = (keys[:n] @ q_rows[r]) * scale          # s_j = q·k_j * scale
+        m = s.max()                                 # M = max_j s_j
+        e = np.exp(s - m)                           # exp(s_j - M)
+        z = e.sum()                                 # sum_j exp(s_j - M)
+        out[r] = (e @ values[:n]) / z               # sum_j exp(s_j - M) v_j / z
+        lse[r] = m + math.log(z)                    # M + ln z
+    return out, lse
+
+
+def _clamp_len(n: int, cap: int) -> int:
+    return max(0, min(int(n), int(cap)))
+
+
+def decode_attention(q: np.ndarray, k_cache: np.ndarray, v_cache: np.ndarray,
+                     cache_lens: Sequence[int], scale: Optional[float] = None,
+                     rows: Optional[Iterable[Tuple[int, int]]] = None
+                     ) -> Tuple[np.ndarray, np.ndarray]:
+    """Decode attention (one query token per sequence) against a contiguous KV cache.
+
+    q [B, Hq, D]; k_cache, v_cache [B, Hkv, S_cap, D]; cache_lens [B].
+    Returns out [B, Hq, D] and lse [B, Hq], both float64. With ``rows`` (an iterable of
+    (b, h) pairs) only those outputs are computed; the rest are NaN.
+
+    Source: FlashDecoding page, section "FlashDecoding算法原理与标准注意力机制对比" (shapes,
+    scaled scores) and section "多GPU张量并行扩展下的FlashDecoding实现" (keys at positions
+    >= cache_lens are masked); GQA head mapping from section "部署落地的工程细节" item 3.
+    """
+    B, Hq, D = q.shape
+    Bk, Hkv, S_cap, Dk = k_cache.shape
+    if Bk != B or Dk != D or v_cache.shape != k_cache.shape:
+        raise ValueError("oracle: shape mismatch")
+    if Hq % Hkv != 0:
+        raise ValueError("oracle: Hq must be a multiple of Hkv")
+    G = Hq // Hkv
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    out = np.full((B, Hq, D), np.nan, dtype=np.float64)
+    lse = np.full((B, Hq), np.nan, dtype=np.float64)
+    if rows is None:
+        rows = [(b, h) for b in range(B) for h in range(Hq)]
+    # Group the requested rows by (b, kv head) so each key/value slab is widened once.
+    groups = {}
+    for b, h in rows:
+        groups.setdefault((int(b), int(h) // G), []).append(int(h))
+    for (b, kv), heads in sorted(groups.items()):
+        n = _clamp_len(cache_lens[b], S_cap)
+        keys = widen(k_cache[b, kv, :n])
+        values = widen(v_cache[b, kv, :n])
+        qr = widen(q[b, heads])
+        o, l = attention_rows(qr, keys, values, [n] * len(heads), scale)
+        out[b, heads] = o
+        lse[b, heads] = l
+    return out, lse
+
+
+def chunk_prefill_attention(q_chunk: np.ndarray, k_cache: np.ndarray, v_cache: np.ndarray,
+                            prefix_lens: Sequence[int], chunk_lens: Sequence[int],
+                            scale: Optional[float] = None,
+                            rows: Optional[Iterable[Tuple[int, int]]] = None
+                            ) -> Tuple[np.ndarray, np.ndarray]:
+    """Causal attention of packed query chunks against their cached prefix plus themselves.
+
+    q_chunk [sum(chunk_lens), Hq, D], packed request by request; k_cache, v_cache
+    [B, Hkv, S_cap, D] already hold each request's prefix and its chunk at
+    [prefix_len_b, prefix_len_b + chunk_len_b). Row i of request b sees keys
+    j <= prefix_len_b + i. Returns out [sum(chunk_lens), Hq, D] and lse [sum(chunk_lens), Hq].
+    ``rows`` selects (packed row, h) pairs; the rest are NaN.
+
+    Source: ChunkedPrefill page §2.1 (the chunk's K/V are appended to the cache, then
+    scores against the whole cache under a causal mask) and its list of three requirements
+    (persist each chunk's KV; a token sees only itself and earlier tokens); prefix reuse from
+    "Chunked-Prefills分块预填充机制：破解大模型推理的吞吐与延迟困局" §三.2 (KV cache reuse).
+    A request with chunk_len = 1 and prefix_len = len - 1 is plain decode over len keys.
+    """
+    total, Hq, D = q_chunk.shape
+    B, Hkv, S_cap, Dk = k_cache.shape
+    if Dk != D or v_cache.shape != k_cache.shape:
+        raise ValueError("oracle: shape mismatch")
+    if len(prefix_lens) != B or len(chunk_lens) != B:
+        raise ValueError("oracle: prefix_lens / chunk_lens must have one entry per request")
+    if int(sum(int(c) for c in chunk_lens)) != total:
+        raise ValueError("oracle: q_chunk rows must equal sum(chunk_lens)")
+    if Hq % Hkv != 0:
+        raise ValueError("oracle: Hq must be a multiple of Hkv")
+    G = Hq // Hkv
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    row_req = np.zeros(total, dtype=np.int64)
+    row_pos = np.zeros(total, dtype=np.int64)
+    off = 0
+    for b in range(B):
+        c = int(chunk_lens[b])
+        row_req[off:off + c] = b
+        row_pos[off:off + c] = np.arange(c)
+        off += c
+    out = np.full((total, Hq, D), np.nan, dtype=np.float64)
+    lse = np.full((total, Hq), np.nan, dtype=np.float64)
+    if rows is None:
+        rows = [(p, h) for p in range(total) for h in range(Hq)]
+    groups = {}
+    for p, h in rows:
+        p = int(p)
+        groups.setdefault((int(row_req[p]), int(h) // G), []).append((p, int(h)))
+    for (b, kv), items in sorted(groups.items()):
+        limit = _clamp_len(int(prefix_lens[b]) + int(chunk_lens[b]), S_cap)
+        keys = widen(k_cache[b, kv, :limit])
+        values = widen(v_cache[b, kv, :limit])
+        qr = np.stack([widen(q_chunk[p, h]) for p, h in items])
+        # row i of the chunk sees prefix_len + i + 1 keys, clamped to the cache capacity
+        n_vis = [_clamp_len(int(prefix_lens[b]) + int(row_pos[p]) + 1, S_cap) for p, _ in items]
+        o, l = attention_rows(qr, keys, values, n_vis, scale)
+        for r, (p, h) in enumerate(items):
+            out[p, h] = o[r]
+            lse[p, h] = l[r]
+    return out, lse

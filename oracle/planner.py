@@ -1,0 +1,152 @@
+"""Plain-Python split planner oracle.
+
+TEST INFRASTRUCTURE ONLY (see ``oracle/attention.py``). The CUDA library plans its split-KV
+work on the host (``fd_split_plan``) and on the device; the tests require both to equal this
+plan exactly, integer for integer.
+
+Source: "大模型推理加速FlashDecoding算法原理与多GPU并行解码实战" (FlashDecoding algorithm and
+multi-GPU decoding), section "Variable-Length序列动态切分策略": a greedy allocator fills
+workers up to target = ceil(total tokens / workers) with pieces of at most max_chunk = 1024
+tokens, never leaves a piece under min_chunk = 128 on its own, and exists so that short
+sequences do not leave workers idle. Section "性能压测与瓶颈分析" adds that pieces under about
+256 tokens lose to launch overhead. The ChunkedPrefill page ("大语言模型长序列推理优化：
+ChunkedPrefill与FlashDecoding技术解析", §3.1) gives the tile range 256-1024 tokens, and the
+Chunked-Prefills page ("Chunked-Prefills分块预填充机制：破解大模型推理的吞吐与延迟困局",
+§四.1) gives the rule chunk_size = min(MAX_CHUNK_SIZE, input_length / NUM_CHUNKS).
+
+Reading used on one GPU (the workers are the persistent CTAs, one per SM):
+
+1. total = sum of the clamped cache lengths.
+2. chunk = clamp(ceil(total * Hkv / (WAVES * num_ctas)), 256, 1024) tokens.
+3. n_b = max(1, ceil(len_b / chunk)) splits for sequence b.
+4. Split s of sequence b is [floor(s * len_b / n_b), floor((s + 1) * len_b / n_b)): the offset
+   restarts at 0 for every sequence and no token is dropped (the printed allocator never
+   resets its offset between sequences and drops tokens once the workers run out).
+5. With equal splits every split of a multi-split sequence has more than chunk / 2 >= 128
+   tokens, so the printed "merge a piece under min_chunk into the previous one" rule never
+   fires; the tests check that bound.
+6. Items are ordered longest first (LPT list scheduling over the persistent CTAs): sequences
+   by their longest split, descending, ties by index; within a sequence by KV head, then split.
+
+A fixed split count (num_splits > 0) instead gives every sequence num_splits splits of
+chunk_b = ceil(len_b / num_splits) tokens, split s = [min(s * chunk_b, len_b),
+min((s + 1) * chunk_b, len_b)) (the FlashDecoding page's chunk_size rule); trailing splits
+may be empty.
+
+Chunked prefill (``chunk_plan``): a request with chunk_len = 1 is a decode row over
+prefix_len + 1 keys and is planned as above. A request with a longer chunk is cut into query
+tiles of 128 rows; tile t sees at most K_t = min(prefix + min(chunk_len, 128 (t + 1)), S_cap)
+keys, which are cut into n_t = max(1, ceil(K_t / CHUNK_KV_SPLIT)) equal splits the same way.
+Every row of the tile owns n_t partial slots.
+"""
+
+from __future__ import annotations
+
+from dataclasses import dataclass, field
+from typing import List, Sequence, Tuple
+
+__all__ = [
+    "MIN_CHUNK", "MAX_CHUNK", "WAVES", "Q_TILE", "CHUNK_KV_SPLIT",
+    "DecodePlan", "decode_plan", "ChunkPlan", "chunk_plan",
+]
+
+MIN_CHUNK = 256        # launch-overhead floor, FlashDecoding page "性能压测与瓶颈分析"
+MAX_CHUNK = 1024       # max_chunk of the allocator / top of the 256-1024 tile range
+MIN_PIECE = 128        # min_chunk of the allocator
+WAVES = 8              # target items per persistent CTA
+Q_TILE = 128           # query rows per chunked-prefill tile
+CHUNK_KV_SPLIT = 2048  # keys per split for a chunked-prefill query tile
+
+
+def _cdiv(a: int, b: int) -> int:
+    return -(-a // b)
+
+
+@dataclass
+class DecodePlan:
+    chunk_tokens: int
+    splits_per_seq: List[int]
+    # (b, kv_head, split, start, end) in execution order
+    items: List[Tuple[int, int, int, int, int]] = field(default_factory=list)
+
+    @property
+    def total_items(self) -> int:
+        return len(self.items)
+
+    @property
+    def max_splits_per_seq(self) -> int:
+        return max(self.splits_per_seq) if self.splits_per_seq else 0
+
+
+def _split_bounds_equal(n_tok: int, n_split: int) -> List[Tuple[int, int]]:
+    return [((s * n_tok) // n_split, ((s + 1) * n_tok) // n_split) for s in range(n_split)]
+
+
+def _split_bounds_fixed(n_tok: int, n_split: int) -> List[Tuple[int, int]]:
+    c = _cdiv(n_tok, n_split) if n_tok > 0 else 0
+    return [(min(s * c, n_tok), min((s + 1) * c, n_tok)) for s in range(n_split)]
+
+
+def decode_plan(cache_lens: Sequence[int], num_kv_heads: int, cache_capacity: int,
+                num_ctas: int, num_splits: int = 0) -> DecodePlan:
+    """Plan the split-KV work of one decode call (see the module docstring)."""
+    lens = [max(0, min(int(x), int(cache_capacity))) for x in cache_lens]
+    B = len(lens)
+    if num_splits > 0:
+        bounds = [_split_bounds_fixed(n, num_splits) for n in lens]
+        chunk = 0
+        keys = [_cdiv(n, num_splits) for n in lens]
+    else:
+        total = sum(lens)
+        chunk = _cdiv(total * num_kv_heads, WAVES * max(1, num_ctas))
+        chunk = max(MIN_CHUNK, min(MAX_CHUNK, chunk))
+        counts = [max(1, _cdiv(n, chunk)) for n in lens]
+        bounds = [_split_bounds_equal(n, c) for n, c in zip(lens, counts)]
+        keys = [_cdiv(n, c) for n, c in zip(lens, counts)]
+    order = sorted(range(B), key=lambda b: (-keys[b], b))
+    items = []
+    for b in order:
+        for h in range(num_kv_heads):
+            for s, (t0, t1) in enumerate(bounds[b]):
+                items.append((b, h, s, t0, t1))
+    return DecodePlan(chunk_tokens=chunk, splits_per_seq=[len(x) for x in bounds], items=items)
+
+
+@dataclass
+class ChunkPlan:
+    decode: DecodePlan                     # plan over the chunk_len == 1 requests (indexed by request)
+    decode_requests: List[int]             # request index of each decode row, in request order
+    # (b, q_tile, q_head, split, key_start, key_end) in execution order
+    tile_items: List[Tuple[int, int, int, int, int, int]] = field(default_factory=list)
+    row_splits: List[int] = field(default_factory=list)      # partial slots per packed row
+
+
+def chunk_plan(prefix_lens: Sequence[int], chunk_lens: Sequence[int], num_q_heads: int,
+               num_kv_heads: int, cache_capacity: int, num_ctas: int) -> ChunkPlan:
+    """Plan a chunked-prefill call: decode rows via ``decode_plan``, longer chunks by tiles."""
+    B = len(chunk_lens)
+    dec_req = [b for b in range(B) if int(chunk_lens[b]) == 1]
+    dec_lens = [int(prefix_lens[b]) + 1 for b in dec_req]
+    dec = decode_plan(dec_lens, num_kv_heads, cache_capacity, num_ctas, 0)
+    # express decode items by request index
+    dec.items = [(dec_req[i], h, s, t0, t1) for (i, h, s, t0, t1) in dec.items]
+    row_splits: List[int] = []
+    tiles = []
+    for b in range(B):
+        c = int(chunk_lens[b])
+        if c == 1:
+            row_splits.append(dec.splits_per_seq[dec_req.index(b)])
+            continue
+        p = int(prefix_lens[b])
+        for t in range(_cdiv(c, Q_TILE)):
+            k_t = max(0, min(p + min(c, Q_TILE * (t + 1)), int(cache_capacity)))
+            n_t = max(1, _cdiv(k_t, CHUNK_KV_SPLIT))
+            rows_in_tile = min(Q_TILE, c - Q_TILE * t)
+            row_splits.extend([n_t] * rows_in_tile)
+            for h in range(num_q_heads):
+                for s, (k0, k1) in enumerate(_split_bounds_equal(k_t, n_t)):
+                    tiles.append((b, t, h, s, k0, k1))
+    # longest work first: by key count of the split, descending; ties keep generation order
+    order = sorted(range(len(tiles)), key=lambda i: (-(tiles[i][5] - tiles[i][4]), i))
+    return ChunkPlan(decode=dec, decode_requests=dec_req,
+                     tile_items=[tiles[i] for i in order], row_splits=row_splits)

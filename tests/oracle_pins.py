@@ -1,0 +1,323 @@
+"""Checks that pin the float64 oracle to things other than itself.
+
+Each ``pin_*`` takes the oracle's attention module (``oracle.attention`` or a deliberately
+mutated copy of it) and raises AssertionError when the module disagrees with:
+
+* hand-derived closed-form fixtures under tests/golden/ (decode and causal chunk);
+* closed forms: q = 0 gives the mean of the visible V rows and LSE = ln n; n = 1 gives v_0 and
+  LSE = s_0; two keys give sigmoid weights; a dominant score selects one V row; equal scores
+  give the mean;
+* library routines computed independently on the CPU: torch.softmax / torch.logsumexp in
+  float64 followed by a matmul, and torch's scaled_dot_product_attention with a causal mask;
+* invariants: any split of the keys merged by log-sum-exp equals no split; jointly permuting K
+  and V rows changes nothing; the pages' sequential online softmax and split-then-merge
+  algorithms (oracle/formulations.py) give the same result.
+
+tests/test_oracle_pins.py runs them on the real oracle; tests/test_oracle_mutations.py plants
+mistakes in a copy of the oracle and checks that some pin catches each one.
+"""
+
+from __future__ import annotations
+
+import json
+import math
+import os
+
+import numpy as np
+import torch
+
+from oracle import formulations
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+TOL = 1e-12
+
+
+def _close(a, b, tol=TOL, what=""):
+    a = np.asarray(a, dtype=np.float64)
+    b = np.asarray(b, dtype=np.float64)
+    assert a.shape == b.shape, f"{what}: shape {a.shape} vs {b.shape}"
+    both_inf = np.isinf(a) & np.isinf(b) & (np.sign(a) == np.sign(b))
+    err = np.where(both_inf, 0.0, np.abs(a - b))
+    assert np.all(np.isfinite(err)), f"{what}: non-finite mismatch"
+    m = float(err.max()) if err.size else 0.0
+    assert m <= tol * max(1.0, float(np.abs(np.where(both_inf, 0, b)).max() if b.size else 1.0)), \
+        f"{what}: max abs err {m:.3e}"
+
+
+def _rand(shape, seed, scale=1.0):
+    return np.random.default_rng(seed).standard_normal(shape) * scale
+
+
+def _torch_reference(q, k, v, lens, scale):
+    """softmax(q·Kᵀ·scale)·V and logsumexp with torch float64 library routines, head h -> kv h//G."""
+    B, Hq, D = q.shape
+    Hkv = k.shape[1]
+    G = Hq // Hkv
+    out = np.zeros((B, Hq, D))
+    lse = np.zeros((B, Hq))
+    for b in range(B):
+        n = int(lens[b])
+        for h in range(Hq):
+            if n == 0:
+                out[b, h] = 0.0
+                lse[b, h] = -math.inf
+                continue
+            K = torch.from_numpy(np.ascontiguousarray(k[b, h // G, :n], dtype=np.float64))
+            V = torch.from_numpy(np.ascontiguousarray(v[b, h // G, :n], dtype=np.float64))
+            qq = torch.from_numpy(np.ascontiguousarray(q[b, h], dtype=np.float64))
+            s = torch.mv(K, qq) * scale
+            out[b, h] = (torch.softmax(s, dim=0) @ V).numpy()
+            lse[b, h] = float(torch.logsumexp(s, dim=0))
+    return out, lse
+
+
+# ---- fixtures -------------------------------------------------------------------------------
+
+def pin_golden_decode(att):
+    with open(os.path.join(GOLDEN, "decode_two_keys_exact.json")) as f:
+        g = json.load(f)
+    q = np.array(g["q"])
+    k = np.array(g["k_cache"])
+    v = np.array(g["v_cache"])
+    out, lse = att.decode_attention(q, k, v, g["cache_lens"])
+    _close(out, g["expected_out"], g["tolerance"], "golden decode O")
+    _close(lse, g["expected_lse"], g["tolerance"], "golden decode LSE")
+
+
+def pin_golden_chunk(att):
+    with open(os.path.join(GOLDEN, "chunk_causal_exact.json")) as f:
+        g = json.load(f)
+    out, lse = att.chunk_prefill_attention(np.array(g["q_chunk"]), np.array(g["k_cache"]),
+                                           np.array(g["v_cache"]), g["prefix_lens"],
+                                           g["chunk_lens"])
+    _close(out, g["expected_out"], g["tolerance"], "golden chunk O")
+    _close(lse, g["expected_lse"], g["tolerance"], "golden chunk LSE")
+
+
+# ---- closed forms ---------------------------------------------------------------------------
+
+def pin_zero_query_is_mean(att):
+    # GQA G = 2, distinct V per KV head, ragged lengths: O = mean of the visible V rows.
+    B, Hq, Hkv, S, D = 2, 4, 2, 9, 8
+    q = np.zeros((B, Hq, D))
+    k = _rand((B, Hkv, S, D), 1)
+    v = _rand((B, Hkv, S, D), 2)
+    lens = [5, 9]
+    out, lse = att.decode_attention(q, k, v, lens)
+    for b in range(B):
+        for h in range(Hq):
+            _close(out[b, h], v[b, h // 2, :lens[b]].mean(axis=0), what="q=0 mean")
+            _close(lse[b, h], math.log(lens[b]), what="q=0 LSE")
+
+
+def pin_single_key(att):
+    B, Hq, Hkv, S, D = 1, 2, 1, 4, 16
+    q = _rand((B, Hq, D), 3)
+    k = _rand((B, Hkv, S, D), 4)
+    v = _rand((B, Hkv, S, D), 5)
+    out, lse = att.decode_attention(q, k, v, [1])
+    for h in range(Hq):
+        s0 = math.fsum(float(a) * float(c) for a, c in zip(q[0, h], k[0, 0, 0])) / math.sqrt(D)
+        _close(out[0, h], v[0, 0, 0], what="n=1 O")
+        _close(lse[0, h], s0, what="n=1 LSE")
+
+
+def pin_two_keys_sigmoid(att):
+    D = 8
+    q = _rand((1, 1, D), 6)
+    k = _rand((1, 1, 2, D), 7)
+    v = _rand((1, 1, 2, D), 8)
+    out, lse = att.decode_attention(q, k, v, [2])
+    s = [math.fsum(float(a) * float(c) for a, c in zip(q[0, 0], k[0, 0, j])) / math.sqrt(D)
+         for j in range(2)]
+    sig = lambda x: 1.0 / (1.0 + math.exp(-x))
+    expect = sig(s[0] - s[1]) * v[0, 0, 0] + sig(s[1] - s[0]) * v[0, 0, 1]
+    _close(out[0, 0], expect, what="two-key O")
+    hi, lo = max(s), min(s)
+    _close(lse[0, 0], hi + math.log1p(math.exp(lo - hi)), what="two-key LSE")
+
+
+def pin_one_hot(att):
+    # Orthogonal query heads; each head has its own key that beats every other score by
+    # hundreds of nats, so O is that key's V row to float64 precision.
+    B, Hq, Hkv, S, D = 1, 4, 2, 12, 16
+    q = np.zeros((B, Hq, D))
+    for h in range(Hq):
+        q[0, h, h] = 3.0
+    k = _rand((B, Hkv, S, D), 10, scale=1e-3)
+    v = _rand((B, Hkv, S, D), 11)
+    hot = {0: 3, 1: 7, 2: 1, 3: 10}
+    for h, j in hot.items():
+        k[0, h // 2, j, h] = 400.0
+    out, lse = att.decode_attention(q, k, v, [S])
+    for h, j in hot.items():
+        _close(out[0, h], v[0, h // 2, j], what=f"one-hot head {h}")
+        _close(lse[0, h], float(q[0, h] @ k[0, h // 2, j]) / 4.0, 1e-9, f"one-hot LSE {h}")
+
+
+def pin_equal_scores(att):
+    B, Hq, Hkv, S, D = 1, 2, 1, 7, 8
+    q = _rand((B, Hq, D), 12)
+    row = _rand((D,), 13)
+    k = np.broadcast_to(row, (B, Hkv, S, D)).copy()
+    v = _rand((B, Hkv, S, D), 14)
+    out, lse = att.decode_attention(q, k, v, [6])
+    for h in range(Hq):
+        s = math.fsum(float(a) * float(c) for a, c in zip(q[0, h], row)) / math.sqrt(D)
+        _close(out[0, h], v[0, 0, :6].mean(axis=0), what="equal scores O")
+        _close(lse[0, h], s + math.log(6), what="equal scores LSE")
+
+
+def pin_empty_and_clamp(att):
+    B, Hq, Hkv, S, D = 3, 2, 1, 5, 4
+    q = _rand((B, Hq, D), 15)
+    k = _rand((B, Hkv, S, D), 16)
+    v = _rand((B, Hkv, S, D), 17)
+    out, lse = att.decode_attention(q, k, v, [0, 99, -3])
+    assert np.all(out[0] == 0.0) and np.all(lse[0] == -math.inf), "len 0: O = 0, LSE = -inf"
+    assert np.all(out[2] == 0.0) and np.all(lse[2] == -math.inf), "negative len clamps to 0"
+    ref, rl = att.decode_attention(q, k, v, [0, S, 0])
+    _close(out[1], ref[1], what="len > capacity clamps")
+    _close(lse[1], rl[1], what="len > capacity clamps (LSE)")
+
+
+# ---- library routines -----------------------------------------------------------------------
+
+def pin_torch_softmax(att):
+    B, Hq, Hkv, S, D = 3, 8, 2, 37, 16
+    q = _rand((B, Hq, D), 20, 2.0)
+    k = _rand((B, Hkv, S, D), 21)
+    v = _rand((B, Hkv, S, D), 22)
+    lens = [37, 1, 20]
+    out, lse = att.decode_attention(q, k, v, lens)
+    ro, rl = _torch_reference(q, k, v, lens, 1.0 / math.sqrt(D))
+    _close(out, ro, 1e-11, "torch softmax O")
+    _close(lse, rl, 1e-11, "torch logsumexp")
+
+
+def _sdpa_causal(q, k, v, scale):
+    """q/k/v [H, L, D] float64 -> (O [H, L, D], LSE [H, L]) with a square causal mask."""
+    Q, K, V = (torch.from_numpy(np.ascontiguousarray(x)) for x in (q, k, v))
+    O = torch.nn.functional.scaled_dot_product_attention(Q, K, V, is_causal=True, scale=scale)
+    s = (Q @ K.transpose(-1, -2)) * scale
+    L = s.shape[-1]
+    s = s.masked_fill(torch.ones(L, L, dtype=torch.bool).triu(1), -math.inf)
+    return O.numpy(), torch.logsumexp(s, dim=-1).numpy()
+
+
+def pin_chunk_equals_full_causal(att):
+    # A sequence of 23 tokens: chunked prefill of rows [prefix, prefix + chunk) over a cache
+    # that already holds all 23 K/V rows must equal rows of full causal attention.
+    H, L, D = 2, 23, 8
+    q = _rand((H, L, D), 30)
+    k = _rand((H, L, D), 31)
+    v = _rand((H, L, D), 32)
+    scale = 1.0 / math.sqrt(D)
+    full_o, full_l = _sdpa_causal(q, k, v, scale)
+    cache_k = k[None]
+    cache_v = v[None]
+    for prefix, chunk in [(0, 23), (5, 7), (10, 13), (22, 1)]:
+        qc = np.transpose(q[:, prefix:prefix + chunk], (1, 0, 2))
+        o, l = att.chunk_prefill_attention(qc, cache_k, cache_v, [prefix], [chunk])
+        _close(o, np.transpose(full_o[:, prefix:prefix + chunk], (1, 0, 2)), 1e-11,
+               f"chunk ({prefix},{chunk}) O")
+        _close(l, full_l[:, prefix:prefix + chunk].T, 1e-11, f"chunk ({prefix},{chunk}) LSE")
+    # decode over len keys equals the last row of full causal attention over len tokens
+    for n in (1, 9, 23):
+        o, l = att.decode_attention(q[None, :, n - 1], cache_k, cache_v, [n])
+        _close(o[0], full_o[:, n - 1], 1e-11, "decode = last causal row")
+        _close(l[0], full_l[:, n - 1], 1e-11, "decode LSE = last causal row")
+
+
+def pin_chunk_batch_gqa(att):
+    # Several packed requests with GQA against torch softmax per row.
+    Hq, Hkv, S, D = 4, 2, 40, 8
+    prefix = [0, 17, 30]
+    chunk = [5, 1, 10]
+    B = 3
+    total = sum(chunk)
+    q = _rand((total, Hq, D), 40)
+    k = _rand((B, Hkv, S, D), 41)
+    v = _rand((B, Hkv, S, D), 42)
+    out, lse = att.chunk_prefill_attention(q, k, v, prefix, chunk)
+    p = 0
+    for b in range(B):
+        for i in range(chunk[b]):
+            n = prefix[b] + i + 1
+            ro, rl = _torch_reference(q[p][None], k[b:b + 1], v[b:b + 1], [n], 1 / math.sqrt(D))
+            _close(out[p], ro[0], 1e-11, "packed chunk O")
+            _close(lse[p], rl[0], 1e-11, "packed chunk LSE")
+            p += 1
+
+
+# ---- invariants -----------------------------------------------------------------------------
+
+def pin_split_invariance(att):
+    B, Hq, Hkv, S, D = 1, 2, 1, 50, 16
+    q = _rand((B, Hq, D), 50, 3.0)
+    k = _rand((B, Hkv, S, D), 51)
+    v = _rand((B, Hkv, S, D), 52)
+    n = 47
+    full_o, full_l = att.decode_attention(q, k, v, [n])
+    for cuts in ([20], [1, 2, 46], [10, 20, 30, 40], [0, 47]):
+        bounds = [0] + cuts + [n]
+        outs, lses = [], []
+        for a, c in zip(bounds[:-1], bounds[1:]):
+            o, l = att.decode_attention(q, k[:, :, a:], v[:, :, a:], [c - a])
+            outs.append(o)
+            lses.append(l)
+        for h in range(Hq):
+            mo, ml = formulations.merge_partials([o[0, h] for o in outs],
+                                                 [float(l[0, h]) for l in lses])
+            _close(mo, full_o[0, h], 1e-12, f"split {cuts} O")
+            _close(ml, full_l[0, h], 1e-12, f"split {cuts} LSE")
+
+
+def pin_permutation_invariance(att):
+    B, Hq, Hkv, S, D = 1, 2, 1, 30, 8
+    q = _rand((B, Hq, D), 60)
+    k = _rand((B, Hkv, S, D), 61)
+    v = _rand((B, Hkv, S, D), 62)
+    perm = np.random.default_rng(63).permutation(S)
+    o1, l1 = att.decode_attention(q, k, v, [S])
+    o2, l2 = att.decode_attention(q, k[:, :, perm], v[:, :, perm], [S])
+    _close(o1, o2, 1e-12, "permuted O")
+    _close(l1, l2, 1e-12, "permuted LSE")
+
+
+def pin_page_formulations(att):
+    B, Hq, Hkv, S, D = 1, 3, 1, 301, 16
+    q = _rand((B, Hq, D), 70, 2.0)
+    k = _rand((B, Hkv, S, D), 71)
+    v = _rand((B, Hkv, S, D), 72)
+    n = 289
+    out, lse = att.decode_attention(q, k, v, [n])
+    scale = 1.0 / math.sqrt(D)
+    for h in range(Hq):
+        for block in (1, 7, 64, 256, 1000):
+            o, l = formulations.online_softmax_row(q[0, h], k[0, 0], v[0, 0], n, scale, block)
+            _close(o, out[0, h], 1e-12, f"online block {block} O")
+            _close(l, lse[0, h], 1e-12, f"online block {block} LSE")
+        for chunks in (1, 2, 3, 8, 289, 400):
+            o, l = formulations.split_merge_row(q[0, h], k[0, 0], v[0, 0], n, scale, chunks)
+            _close(o, out[0, h], 1e-12, f"split-merge {chunks} O")
+            _close(l, lse[0, h], 1e-12, f"split-merge {chunks} LSE")
+
+
+def pin_bf16_widening(att):
+    # bf16 bit patterns must widen to exactly the values torch gives them.
+    x = torch.randn(1000, dtype=torch.float32).to(torch.bfloat16)
+    bits = x.view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(att.widen(bits), x.to(torch.float64).numpy()), "bf16 widening"
+    special = torch.tensor([0.0, -0.0, 1e38, -1e-38, float("inf")], dtype=torch.bfloat16)
+    sb = special.view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(att.widen(sb), special.to(torch.float64).numpy()), "bf16 specials"
+
+
+ALL_PINS = [
+    pin_golden_decode, pin_golden_chunk, pin_zero_query_is_mean, pin_single_key,
+    pin_two_keys_sigmoid, pin_one_hot, pin_equal_scores, pin_empty_and_clamp,
+    pin_torch_softmax, pin_chunk_equals_full_causal, pin_chunk_batch_gqa,
+    pin_split_invariance, pin_permutation_invariance, pin_page_formulations,
+    pin_bf16_widening,
+]

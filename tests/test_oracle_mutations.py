@@ -1,0 +1,58 @@
+"""Plant plausible mistakes in a copy of the oracle (on the CPU) and check the pins catch each.
+
+Each mutation rewrites one expression of oracle/attention.py: a dropped term, a wrong sign,
+a wrong index or head mapping, a swapped operand, an off-by-one in the causal limit. The
+mutated source is executed as a throw-away module; at least one pin must then fail.
+"""
+
+import math
+import os
+import types
+
+import pytest
+
+from oracle_pins import ALL_PINS
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+SRC = open(os.path.join(ROOT, "oracle", "attention.py")).read()
+
+MUTATIONS = {
+    "scale_dropped_sqrt": ("scale = 1.0 / math.sqrt(D)", "scale = 1.0 / D"),
+    "lse_drops_max": ("lse[r] = m + math.log(z)", "lse[r] = math.log(z)"),
+    "lse_wrong_sign": ("lse[r] = m + math.log(z)", "lse[r] = m - math.log(z)"),
+    "no_normalisation": ("out[r] = (e @ values[:n]) / z", "out[r] = (e @ values[:n])"),
+    "exp_wrong_sign": ("e = np.exp(s - m)", "e = np.exp(m - s)"),
+    "k_v_swapped": ("s = (keys[:n] @ q_rows[r]) * scale", "s = (values[:n] @ q_rows[r]) * scale"),
+    "gqa_mod_mapping": ("groups.setdefault((int(b), int(h) // G), []).append(int(h))",
+                        "groups.setdefault((int(b), int(h) % Hkv), []).append(int(h))"),
+    "ignores_cache_len": ("n = _clamp_len(cache_lens[b], S_cap)", "n = S_cap"),
+    "len_off_by_one": ("n = _clamp_len(cache_lens[b], S_cap)",
+                       "n = _clamp_len(cache_lens[b] - 1, S_cap)"),
+    "causal_off_by_one": ("_clamp_len(int(prefix_lens[b]) + int(row_pos[p]) + 1, S_cap)",
+                          "_clamp_len(int(prefix_lens[b]) + int(row_pos[p]), S_cap)"),
+    "causal_top_left": ("_clamp_len(int(prefix_lens[b]) + int(row_pos[p]) + 1, S_cap)",
+                        "_clamp_len(int(row_pos[p]) + 1, S_cap)"),
+    "bf16_widen_shift": ("<< np.uint32(16)", "<< np.uint32(15)"),
+    "empty_lse_zero": ("lse = np.full((R,), -np.inf, dtype=np.float64)",
+                       "lse = np.full((R,), 0.0, dtype=np.float64)"),
+}
+
+
+def _mutant(name):
+    old, new = MUTATIONS[name]
+    assert SRC.count(old) >= 1, f"mutation anchor for {name} missing"
+    mod = types.ModuleType(f"oracle_mutant_{name}")
+    exec(compile(SRC.replace(old, new), f"<mutant {name}>", "exec"), mod.__dict__)
+    return mod
+
+
+@pytest.mark.parametrize("name", sorted(MUTATIONS))
+def test_pins_catch_mutation(name):
+    mod = _mutant(name)
+    failed = []
+    for pin in ALL_PINS:
+        try:
+            pin(mod)
+        except (AssertionError, ValueError, IndexError, FloatingPointError, OverflowError):
+            failed.append(pin.__name__)
+    assert failed, f"no pin caught mutation {name}"

@@ -1,0 +1,121 @@
+"""The planner oracle against hand-worked plans and its coverage / bound properties.
+
+Parity of the planner is pinned by properties rather than by the pages' allocator, which
+targets whole GPUs and drops tokens: every sequence's splits tile [0, len) in order with no gap
+or overlap, no split exceeds the chunk, a split of a multi-split sequence never falls under
+the allocator's min_chunk of 128, items come longest first, and the item count stays under the
+bound the CUDA library uses to size its workspace.
+"""
+
+import random
+
+import pytest
+
+from oracle import planner as P
+
+
+def _bound(B, Hkv, cap, ctas, num_splits):
+    if num_splits > 0:
+        return Hkv * B * num_splits
+    return Hkv * B + max(P.WAVES * ctas, -(-Hkv * B * cap // P.MAX_CHUNK))
+
+
+def test_fixed_even():
+    # one sequence of 1024 keys, 4 fixed splits -> 256 keys each, for every KV head
+    p = P.decode_plan([1024], 8, 1024, 148, num_splits=4)
+    assert p.splits_per_seq == [4]
+    assert p.total_items == 32
+    assert sorted({(t0, t1) for (_, _, _, t0, t1) in p.items}) == [
+        (0, 256), (256, 512), (512, 768), (768, 1024)]
+
+
+def test_fixed_ragged_and_empty():
+    # chunk_size = ceil(10 / 4) = 3 -> [0,3) [3,6) [6,9) [9,10); len 2 -> [0,1) [1,2) then empties
+    p = P.decode_plan([10, 2], 1, 16, 148, num_splits=4)
+    got = {b: [] for b in range(2)}
+    for b, h, s, t0, t1 in p.items:
+        got[b].append((s, t0, t1))
+    assert got[0] == [(0, 0, 3), (1, 3, 6), (2, 6, 9), (3, 9, 10)]
+    assert got[1] == [(0, 0, 1), (1, 1, 2), (2, 2, 2), (3, 2, 2)]
+
+
+def test_auto_hand_worked_13b_shape():
+    # 4 x 16384 keys, 40 KV heads, 148 CTAs: ceil(65536*40 / (8*148)) = 2215 -> clamp 1024
+    p = P.decode_plan([16384] * 4, 40, 16384, 148)
+    assert p.chunk_tokens == 1024
+    assert p.splits_per_seq == [16, 16, 16, 16]
+    assert p.total_items == 4 * 40 * 16
+
+
+def test_auto_hand_worked_small():
+    # total 1300 tokens, 1 KV head: ceil(1300 / 1184) = 2 -> clamp up to 256
+    p = P.decode_plan([1000, 300, 0], 1, 4096, 148)
+    assert p.chunk_tokens == 256
+    assert p.splits_per_seq == [4, 2, 1]
+    assert p.items == [(0, 0, 0, 0, 250), (0, 0, 1, 250, 500), (0, 0, 2, 500, 750),
+                       (0, 0, 3, 750, 1000), (1, 0, 0, 0, 150), (1, 0, 1, 150, 300),
+                       (2, 0, 0, 0, 0)]
+
+
+def test_auto_clamps_lengths():
+    p = P.decode_plan([-5, 10**9], 2, 3000, 148)
+    assert p.splits_per_seq[0] == 1
+    spans = [(t0, t1) for (b, h, s, t0, t1) in p.items if b == 1 and h == 0]
+    assert spans[0][0] == 0 and spans[-1][1] == 3000
+
+
+@pytest.mark.parametrize("seed", range(40))
+def test_properties_random(seed):
+    rng = random.Random(seed)
+    B = rng.choice([1, 2, 3, 7, 32, 100])
+    Hkv = rng.choice([1, 2, 8, 40])
+    cap = rng.choice([1, 63, 64, 65, 257, 1024, 4096, 32768])
+    ctas = rng.choice([1, 8, 148])
+    num_splits = rng.choice([0, 0, 0, 1, 3, 8, 40])
+    lens = [rng.choice([0, 1, cap - 1, cap, rng.randint(0, cap)]) for _ in range(B)]
+    p = P.decode_plan(lens, Hkv, cap, ctas, num_splits)
+    again = P.decode_plan(lens, Hkv, cap, ctas, num_splits)
+    assert p == again, "deterministic"
+    assert p.total_items == Hkv * sum(p.splits_per_seq)
+    assert p.total_items <= _bound(B, Hkv, cap, ctas, num_splits)
+    if num_splits == 0:
+        assert P.MIN_CHUNK <= p.chunk_tokens <= P.MAX_CHUNK
+    per = {}
+    for b, h, s, t0, t1 in p.items:
+        per.setdefault((b, h), []).append((s, t0, t1))
+    keys = []
+    for b in range(B):
+        n = max(0, min(lens[b], cap))
+        for h in range(Hkv):
+            sp = per[(b, h)]
+            assert [s for s, _, _ in sp] == list(range(len(sp)))
+            assert sp[0][1] == 0 and sp[-1][2] == n, "splits cover [0, len)"
+            for (_, a0, a1), (_, c0, c1) in zip(sp, sp[1:]):
+                assert a1 == c0, "no gap, no overlap"
+            for _, t0, t1 in sp:
+                assert 0 <= t0 <= t1 <= n
+                if num_splits == 0:
+                    assert t1 - t0 <= p.chunk_tokens
+                    if len(sp) > 1:
+                        assert t1 - t0 >= 128, "no piece under min_chunk"
+        keys.append(max(t1 - t0 for _, t0, t1 in per[(b, 0)]))
+    # longest-first order over sequences
+    order = []
+    for b, h, s, t0, t1 in p.items:
+        if not order or order[-1] != b:
+            order.append(b)
+    assert len(order) == B, "a sequence's items are contiguous"
+    ks = [keys[b] for b in order]
+    assert ks == sorted(ks, reverse=True)
+
+
+def test_chunk_plan_hand_worked():
+    # request 0: chunk 300 at prefix 5000, 2 heads; request 1: decode row over 70 keys
+    cp = P.chunk_plan([5000, 69], [300, 1], 2, 2, 8192, 148)
+    assert cp.decode_requests == [1]
+    assert cp.decode.splits_per_seq == [1]
+    # tiles: rows 0-127 see <= 5128 keys -> 3 splits; 128-255 -> 5256 -> 3; 256-299 -> 5300 -> 3
+    assert cp.row_splits == [3] * 300 + [1]
+    spans = sorted({(t, s, k0, k1) for (b, t, h, s, k0, k1) in cp.tile_items if t == 0})
+    assert spans == [(0, 0, 0, 1709), (0, 1, 1709, 3418), (0, 2, 3418, 5128)]
+    assert len(cp.tile_items) == 3 * 2 * 3

@@ -1,0 +1,163 @@
+"""Seeded synthetic inputs shared by the oracle tests, the CUDA parity tests and bench.py.
+
+This module only draws random numbers and casts them; it holds none of the attention
+arithmetic. Every tensor is drawn on the CPU from ``torch.Generator`` seeds so that the same
+bytes reach the oracle and the GPU.
+
+Recipe (values i.i.d. N(0, 1) drawn in float32, then cast to the storage dtype with
+round-to-nearest-even):
+
+* q first, in one draw of shape [B, Hq, D];
+* then K: for b in batch order, for each KV head, one draw of [len_b, D] (valid rows only);
+* then V in the same order. Rows at positions >= len_b hold ``pad_fill`` (0 by default; the
+  bounds tests use NaN so any read past the cache length poisons the result);
+* "peaked" K (long-context workload): per (b, KV head), ``peaked_rows`` row indices below len_b
+  are drawn without replacement from numpy's default_rng(seed + 200) and those K rows are
+  multiplied by ``peak_scale`` in float32 before the cast;
+* cache lengths drawn uniformly, both ends inclusive, with numpy default_rng(seed).
+
+The named workloads are the five benchmark shapes of this project (decode MHA fp32, decode
+MHA bf16 13B-like, decode GQA bf16 70B-like, long-context GQA, mixed chunked-prefill step);
+tensor seed = 1000 + index, length seed = 1100 + index.
+"""
+
+from __future__ import annotations
+
+from dataclasses import dataclass
+from typing import Dict, List, Optional
+
+import numpy as np
+import torch
+
+__all__ = [
+    "DecodeInputs", "ChunkInputs", "uniform_lens", "make_decode_inputs", "make_chunk_inputs",
+    "WORKLOADS", "workload", "to_numpy_exact",
+]
+
+
+@dataclass
+class DecodeInputs:
+    q: torch.Tensor            # [B, Hq, D]
+    k_cache: torch.Tensor      # [B, Hkv, S_cap, D]
+    v_cache: torch.Tensor      # [B, Hkv, S_cap, D]
+    cache_lens: torch.Tensor   # int32 [B]
+    num_splits: int = 0
+    name: str = ""
+
+
+@dataclass
+class ChunkInputs:
+    q_chunk: torch.Tensor      # [sum(chunk_lens), Hq, D]
+    k_cache: torch.Tensor      # [B, Hkv, S_cap, D]
+    v_cache: torch.Tensor
+    prefix_lens: torch.Tensor  # int32 [B]
+    chunk_lens: torch.Tensor   # int32 [B]
+    name: str = ""
+
+
+def uniform_lens(seed: int, batch: int, lo: int, hi: int) -> List[int]:
+    """Integer lengths uniform on [lo, hi], both ends inclusive."""
+    return [int(x) for x in np.random.default_rng(seed).integers(lo, hi + 1, size=batch)]
+
+
+def _fill_cache(gen: torch.Generator, B: int, H: int, S_cap: int, D: int, lens: List[int],
+                dtype: torch.dtype, pad_fill: float,
+                peak_rows: Optional[Dict[tuple, np.ndarray]] = None,
+                peak_scale: float = 8.0) -> torch.Tensor:
+    cache = torch.full((B, H, S_cap, D), float(pad_fill), dtype=dtype)
+    for b in range(B):
+        n = max(0, min(int(lens[b]), S_cap))
+        for h in range(H):
+            if n == 0:
+                continue
+            x = torch.randn((n, D), generator=gen, dtype=torch.float32)
+            if peak_rows is not None and (b, h) in peak_rows:
+                idx = torch.from_numpy(peak_rows[(b, h)].astype(np.int64))
+                x[idx] *= peak_scale
+            cache[b, h, :n] = x.to(dtype)
+    return cache
+
+
+def make_decode_inputs(batch: int, q_heads: int, kv_heads: int, head_dim: int, capacity: int,
+                       lens: List[int], dtype: torch.dtype, seed: int, num_splits: int = 0,
+                       pad_fill: float = 0.0, peaked_rows: int = 0, peak_scale: float = 8.0,
+                       name: str = "") -> DecodeInputs:
+    gen = torch.Generator().manual_seed(seed)
+    q = torch.randn((batch, q_heads, head_dim), generator=gen, dtype=torch.float32).to(dtype)
+    peaks = None
+    if peaked_rows > 0:
+        rng = np.random.default_rng(seed + 200)
+        peaks = {}
+        for b in range(batch):
+            n = max(0, min(int(lens[b]), capacity))
+            for h in range(kv_heads):
+                peaks[(b, h)] = rng.choice(n, size=min(peaked_rows, n), replace=False)
+    k = _fill_cache(gen, batch, kv_heads, capacity, head_dim, lens, dtype, pad_fill, peaks,
+                    peak_scale)
+    v = _fill_cache(gen, batch, kv_heads, capacity, head_dim, lens, dtype, pad_fill)
+    return DecodeInputs(q=q, k_cache=k, v_cache=v,
+                        cache_lens=torch.tensor(lens, dtype=torch.int32),
+                        num_splits=num_splits, name=name)
+
+
+def make_chunk_inputs(prefix_lens: List[int], chunk_lens: List[int], q_heads: int,
+                      kv_heads: int, head_dim: int, capacity: int, dtype: torch.dtype,
+                      seed: int, pad_fill: float = 0.0, name: str = "") -> ChunkInputs:
+    """Packed query chunks plus a cache holding each request's prefix and chunk K/V."""
+    gen = torch.Generator().manual_seed(seed)
+    total = int(sum(chunk_lens))
+    q = torch.randn((total, q_heads, head_dim), generator=gen, dtype=torch.float32).to(dtype)
+    lens = [int(p) + int(c) for p, c in zip(prefix_lens, chunk_lens)]
+    B = len(chunk_lens)
+    k = _fill_cache(gen, B, kv_heads, capacity, head_dim, lens, dtype, pad_fill)
+    v = _fill_cache(gen, B, kv_heads, capacity, head_dim, lens, dtype, pad_fill)
+    return ChunkInputs(q_chunk=q, k_cache=k, v_cache=v,
+                       prefix_lens=torch.tensor(prefix_lens, dtype=torch.int32),
+                       chunk_lens=torch.tensor(chunk_lens, dtype=torch.int32), name=name)
+
+
+# ---- the five named workloads --------------------------------------------------------------
+
+WORKLOADS = {
+    1: "decode_mha_fp32_b1_h8_d64_len1024_splits4",
+    2: "decode_mha_bf16_b4_h40_d128_len16384",
+    3: "decode_gqa_bf16_b32_hq64_hkv8_d128_lenU1024-32768",
+    4: "longctx_gqa_bf16_hq64_hkv8_d128_len32768_peaked",
+    5: "mixed_chunk512_prefix15872_plus31decode_h32_d128",
+}
+
+
+def workload(index: int, batch: Optional[int] = None, pad_fill: float = 0.0):
+    """Build one of the five named workloads (index 1..5) at its full size."""
+    seed = 1000 + index
+    lseed = 1100 + index
+    if index == 1:
+        return make_decode_inputs(1, 8, 8, 64, 1024, [1024], torch.float32, seed,
+                                  num_splits=4, pad_fill=pad_fill, name=WORKLOADS[1])
+    if index == 2:
+        return make_decode_inputs(4, 40, 40, 128, 16384, [16384] * 4, torch.bfloat16, seed,
+                                  pad_fill=pad_fill, name=WORKLOADS[2])
+    if index == 3:
+        lens = uniform_lens(lseed, 32, 1024, 32768)
+        return make_decode_inputs(32, 64, 8, 128, 32768, lens, torch.bfloat16, seed,
+                                  pad_fill=pad_fill, name=WORKLOADS[3])
+    if index == 4:
+        b = 1 if batch is None else int(batch)
+        return make_decode_inputs(b, 64, 8, 128, 32768, [32768] * b, torch.bfloat16,
+                                  seed, peaked_rows=8, peak_scale=8.0,
+                                  pad_fill=pad_fill, name=f"{WORKLOADS[4]}_b{b}")
+    if index == 5:
+        dec = uniform_lens(lseed, 31, 512, 8192)
+        prefix = [15872] + [n - 1 for n in dec]
+        chunk = [512] + [1] * 31
+        return make_chunk_inputs(prefix, chunk, 32, 32, 128, 16384, torch.bfloat16, seed,
+                                 pad_fill=pad_fill, name=WORKLOADS[5])
+    raise ValueError(f"unknown workload {index}")
+
+
+def to_numpy_exact(t: torch.Tensor) -> np.ndarray:
+    """CPU numpy view of a tensor with no value change: bf16 becomes its uint16 bit pattern."""
+    t = t.detach().cpu().contiguous()
+    if t.dtype == torch.bfloat16:
+        return t.view(torch.int16).numpy().view(np.uint16)
+    return t.numpy()
