@@ -1,0 +1,401 @@
+#!/usr/bin/env python
+"""Decode-attention benchmark: µs per call and achieved HBM GB/s.
+
+Default workload: decode GQA bf16, Llama-3-70B-like shape (batch 32, 64 query / 8 KV heads,
+head_dim 128, cache lengths uniform in [1024, 32768], capacity 32768, planner splits). One step is
+one fd_decode_attention call (device planner + split kernel + LSE combine) over resident inputs.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl fd|reference] [--workload 1-4]
+
+Prints one JSON line on rank 0. `value` is the whole-job GB/s: the algorithmic bytes every rank
+processed (K+V bytes of the valid keys plus the Q bytes) over the slowest rank's device time.
+With N > 1 (torchrun) every rank runs an independent replica: the path has no exchange step.
+`--impl reference` times the float64 CPU oracle on a bounded sample of the same workload.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "decode-attn µs/call and achieved HBM GB/s vs 8 TB/s peak (Llama-3-70B GQA)"
+FALLBACK_HBM_GBS = 6650.0
+L2_BYTES = 126 * 1024 * 1024
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=3000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["fd", "reference"], default="fd")
+    ap.add_argument("--workload", type=int, default=3, choices=[1, 2, 3, 4])
+    ap.add_argument("--batch", type=int, default=None, help="batch of the long-context workload")
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--cpu-seconds", type=float, default=15.0,
+                    help="host-time budget of the oracle CPU baseline sample")
+    return ap.parse_args()
+
+
+# ------------------------------------------------------------------------------ helpers -------
+
+def log(*a):
+    print(*a, file=sys.stderr, flush=True)
+
+
+def algorithmic_bytes(inp) -> int:
+    """K+V bytes of the valid keys (each read once) plus the Q bytes."""
+    B, hkv, cap, d = inp.k_cache.shape
+    es = inp.k_cache.element_size()
+    lens = [max(0, min(int(x), cap)) for x in inp.cache_lens.tolist()]
+    return 2 * sum(lens) * hkv * d * es + inp.q.numel() * inp.q.element_size()
+
+
+def measured_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            j = json.load(f)
+        return float(j["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_source_sha(name: str) -> str:
+    path = os.path.join(ROOT, "split_kv_decode_flashdecoding_b200", "csrc", name)
+    h = hashlib.sha256()
+    for f in sorted([path, os.path.join(os.path.dirname(path), "common.cuh")]):
+        with open(f, "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def traffic_from_profiles(kernel_file: str, workload: str):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on this source."""
+    path = os.path.join(ROOT, "profiles", "dram_traffic.json")
+    try:
+        with open(path) as f:
+            j = json.load(f)
+        e = j[workload]
+        if e.get("source_sha") == kernel_source_sha(kernel_file):
+            return float(e["bytes_per_launch"])
+    except Exception:
+        pass
+    return None
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples while the timed region runs."""
+
+    QUERY = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.path = tempfile.mktemp(prefix="fd_clocks_", suffix=".csv")
+        self.proc = None
+        self.gpu = gpu_index
+
+    def start(self):
+        try:
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=self.fh, stderr=subprocess.DEVNULL)
+            time.sleep(0.5)
+        except Exception as e:  # no nvidia-smi: report that instead of clocks
+            log(f"clock sampler unavailable: {e}")
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.15)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.fh.close()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                p = [x.strip() for x in line.split(",")]
+                if len(p) < 10:
+                    continue
+                try:
+                    sm.append(float(p[2]))
+                    smax.append(float(p[3]))
+                except ValueError:
+                    continue
+                for n, v in zip(names, p[6:10]):
+                    if v.lower().startswith("active"):
+                        reasons.add(n)
+        os.unlink(self.path)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def cpu_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [int(x.get("num_threads", 1)) for x in threadpool_info() if x.get("user_api") == "blas"]
+        if n:
+            return max(n)
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+def oracle_sample(inp, seconds: float, seed: int = 0):
+    """Time the oracle on whole (b, KV head) groups of the workload, in a seeded order, until
+    `seconds` of host time are spent. Returns (bytes/s, description, groups, elapsed)."""
+    from oracle import attention as oracle
+    from workloads import to_numpy_exact
+    q = to_numpy_exact(inp.q)
+    k = to_numpy_exact(inp.k_cache)
+    v = to_numpy_exact(inp.v_cache)
+    B, hq, d = q.shape
+    hkv = k.shape[1]
+    g = hq // hkv
+    lens = inp.cache_lens.tolist()
+    es = inp.k_cache.element_size()
+    order = np.random.default_rng(seed).permutation(B * hkv)
+    done, nbytes = 0, 0
+    t0 = time.perf_counter()
+    for idx in order:
+        b, h = divmod(int(idx), hkv)
+        rows = [(b, h * g + j) for j in range(g)]
+        oracle.decode_attention(q, k, v, lens, rows=rows)
+        n = max(0, min(int(lens[b]), k.shape[2]))
+        nbytes += 2 * n * d * es + g * d * inp.q.element_size()
+        done += 1
+        if time.perf_counter() - t0 >= seconds:
+            break
+    el = time.perf_counter() - t0
+    desc = (f"{done} of {B * hkv} (batch, KV head) groups of the workload, all {g} query heads "
+            f"each, seeded order; float64 numpy")
+    return nbytes / el, desc, done, el
+
+
+def load_workload(args):
+    from workloads import WORKLOADS, workload
+    t0 = time.time()
+    inp = workload(args.workload, batch=args.batch)
+    log(f"generated {inp.name} in {time.time() - t0:.1f}s")
+    return inp
+
+
+# ------------------------------------------------------------------------------ arms ----------
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return 0
+    inp = load_workload(args)
+    per_step = max(0.2, min(5.0, 120.0 / max(1, args.steps + args.warmup)))
+    for _ in range(args.warmup):
+        oracle_sample(inp, per_step / 4, seed=1)
+    rates = []
+    t0 = time.perf_counter()
+    total_bytes = 0
+    for s in range(args.steps):
+        r, desc, groups, el = oracle_sample(inp, per_step, seed=100 + s)
+        rates.append(r)
+        total_bytes += r * el
+    el = time.perf_counter() - t0
+    value = total_bytes / el / 1e9
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(1e3 * el / max(1, args.steps), 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": inp.name},
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": cpu_threads(),
+                         "kind": "oracle",
+                         "sample": f"per step: {per_step:.2f}s of host time over whole (batch, KV head) groups"},
+        "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_fd(args, rank, world, local_rank):
+    import split_kv_decode_flashdecoding_b200 as fd
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    inp = load_workload(args)
+    alg = algorithmic_bytes(inp)
+    B, hq, d = inp.q.shape
+    hkv = inp.k_cache.shape[1]
+    g = hq // hkv
+    q = inp.q.to(dev)
+    k = inp.k_cache.to(dev)
+    v = inp.v_cache.to(dev)
+    lens = inp.cache_lens.to(dev)
+    out = torch.empty_like(q)
+    lse = torch.empty((B, hq), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    ns = inp.num_splits
+    input_bytes = sum(t.numel() * t.element_size() for t in (q, k, v))
+    l2_policy = ("inputs larger than L2 (valid K/V bytes per call exceed the 126 MB L2)"
+                 if alg > 2 * L2_BYTES else "inputs smaller than L2: measured with warm L2")
+
+    def step():
+        fd.fd_decode_attention(q, k, v, lens, ns, out=out, lse=lse, stream=stream)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+
+    # ---- timed region: K calls, CUDA events on the launching stream ----
+    sampler = ClockSampler(local_rank) if rank == 0 else None
+    if sampler:
+        sampler.start()
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    clocks = sampler.stop() if sampler else None
+    ms_total = e0.elapsed_time(e1)
+    t = torch.tensor([ms_total], dtype=torch.float64, device=dev)
+    if world > 1:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    ms_max = float(t.item())
+    ms_per_step = ms_max / args.steps
+    value = world * alg * args.steps / (ms_max * 1e-3) / 1e9
+
+    # ---- per-kernel durations (same calls, with events between the launches) ----
+    nprof = min(args.steps, 200)
+    fd.fd_profile_begin(nprof)
+    for _ in range(nprof):
+        step()
+    torch.cuda.synchronize()
+    prof = fd.fd_profile_end(nprof)
+    plan_ms = statistics.mean(p[0] for p in prof)
+    split_ms = statistics.mean(p[1] for p in prof)
+    comb_ms = statistics.mean(p[2] for p in prof)
+    peak, peak_kind = measured_peak()
+    use_tc = inp.q.dtype == torch.bfloat16 and d == 128 and 2 <= g <= 16
+    kfile = "decode_tc.cu" if use_tc else "decode_simt.cu"
+    achieved = alg / (split_ms * 1e-3) / 1e9
+
+    # ---- end to end: host buffers, copies inside the timed region ----
+    e2e = None
+    if args.e2e_steps > 0:
+        hq_ = inp.q.pin_memory()
+        hk = inp.k_cache.pin_memory()
+        hv = inp.v_cache.pin_memory()
+        hl = inp.cache_lens.pin_memory()
+        ho = torch.empty_like(inp.q).pin_memory()
+        hlse = torch.empty((B, hq), dtype=torch.float32).pin_memory()
+        h2d = sum(x.numel() * x.element_size() for x in (hq_, hk, hv, hl))
+        d2h = ho.numel() * ho.element_size() + hlse.numel() * 4
+
+        def e2e_step():
+            q.copy_(hq_, non_blocking=True)
+            k.copy_(hk, non_blocking=True)
+            v.copy_(hv, non_blocking=True)
+            lens.copy_(hl, non_blocking=True)
+            step()
+            ho.copy_(out, non_blocking=True)
+            hlse.copy_(lse, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        if world > 1:
+            torch.distributed.barrier()
+        a0 = torch.cuda.Event(enable_timing=True)
+        a1 = torch.cuda.Event(enable_timing=True)
+        a0.record(stream)
+        for _ in range(args.e2e_steps):
+            e2e_step()
+        a1.record(stream)
+        torch.cuda.synchronize()
+        te = torch.tensor([a0.elapsed_time(a1)], dtype=torch.float64, device=dev)
+        if world > 1:
+            torch.distributed.all_reduce(te, op=torch.distributed.ReduceOp.MAX)
+        e2e = {"value": round(world * alg * args.e2e_steps / (float(te.item()) * 1e-3) / 1e9, 3),
+               "unit": "GB/s", "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+               "steps": args.e2e_steps,
+               "note": "full cache tensors copied host->device every step"}
+
+    cpu = None
+    if rank == 0 and world == 1 and args.cpu_seconds > 0:
+        rate, desc, groups, el = oracle_sample(inp, args.cpu_seconds)
+        cpu = {"value": round(rate / 1e9, 4), "unit": "GB/s", "cores": cpu_threads(),
+               "kind": "oracle", "sample": f"{desc}; {el:.1f}s"}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
+            "steps": args.steps, "warmup": max(3, args.warmup),
+            "ms_per_step": round(ms_per_step, 5), "us_per_call": round(ms_per_step * 1e3, 2),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16"
+            if inp.q.dtype == torch.bfloat16 else "f32", "data": "synthetic",
+            "config": {"workload": inp.name, "batch": B, "q_heads": hq, "kv_heads": hkv,
+                       "head_dim": d, "cache_capacity": int(inp.k_cache.shape[2]),
+                       "sum_cache_len": int(sum(inp.cache_lens.tolist())),
+                       "num_splits": "planner" if ns == 0 else ns,
+                       "algorithmic_bytes_per_call": alg, "input_bytes_resident": input_bytes,
+                       "l2": l2_policy, "parallelism": f"replicas x{world}"},
+            "roofline": {"bound": "hbm", "kernel": kfile.replace(".cu", "_kernel"),
+                         "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                         "frac": round(achieved / peak, 4), "peak_kind": f"{peak_kind} copy bandwidth",
+                         "traffic": traffic_from_profiles(kfile, inp.name),
+                         "kernel_ms": {"planner": round(plan_ms, 5), "split": round(split_ms, 5),
+                                       "combine": round(comb_ms, 5)}},
+            "clocks": clocks,
+            "e2e": e2e,
+            "gpu_launches": 3 * args.steps,
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    args = parse_args()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        return run_reference(args, rank, world)
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local_rank)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    try:
+        return run_fd(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    sys.exit(main())

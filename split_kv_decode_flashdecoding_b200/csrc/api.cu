@@ -1,0 +1,611 @@
+// C ABI of the library (include/fd.h): argument validation, the per-(device, stream) workspace,
+// tensor-map construction, kernel dispatch and optional per-launch timing.
+#include <algorithm>
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <map>
+#include <mutex>
+#include <string>
+#include <utility>
+#include <vector>
+
+#include "common.cuh"
+#include "internal.h"
+
+using namespace fd;
+
+namespace {
+
+// ---------------------------------------------------------------------------- errors ---------
+thread_local std::string g_last_error;
+
+fd_status fail(fd_status s, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return s;
+}
+
+fd_status cuda_fail(cudaError_t e, const char* what) {
+  return fail(FD_ERR_CUDA, "%s: %s (%s)", what, cudaGetErrorName(e), cudaGetErrorString(e));
+}
+
+#define FD_CUDA(call, what)                       \
+  do {                                            \
+    cudaError_t e_ = (call);                      \
+    if (e_ != cudaSuccess) return cuda_fail(e_, what); \
+  } while (0)
+
+// ---------------------------------------------------------------------------- workspace ------
+struct Workspace {
+  void* ptr = nullptr;
+  size_t bytes = 0;
+};
+std::mutex g_mu;
+std::map<std::pair<int, uintptr_t>, Workspace> g_ws;
+
+fd_status get_workspace(cudaStream_t stream, size_t need, void** out) {
+  int dev = 0;
+  FD_CUDA(cudaGetDevice(&dev), "cudaGetDevice");
+  std::lock_guard<std::mutex> lock(g_mu);
+  Workspace& w = g_ws[{dev, reinterpret_cast<uintptr_t>(stream)}];
+  if (w.ptr && w.bytes >= need) {
+    *out = w.ptr;
+    return FD_OK;
+  }
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  FD_CUDA(cudaStreamIsCapturing(stream, &cs), "cudaStreamIsCapturing");
+  if (cs != cudaStreamCaptureStatusNone)
+    return fail(FD_ERR_WORKSPACE,
+                "workspace of this stream holds %zu bytes but the call needs %zu; reserve it with "
+                "fd_reserve_workspace before capturing",
+                w.bytes, need);
+  uint32_t old_status = 0;
+  if (w.ptr) {
+    FD_CUDA(cudaStreamSynchronize(stream), "cudaStreamSynchronize");
+    FD_CUDA(cudaMemcpy(&old_status, w.ptr, sizeof(uint32_t), cudaMemcpyDeviceToHost), "read status");
+    FD_CUDA(cudaFree(w.ptr), "cudaFree(workspace)");
+    w.ptr = nullptr;
+    w.bytes = 0;
+  }
+  size_t nb = std::max(need, static_cast<size_t>(1) << 20);
+  nb = (nb + (2u << 20) - 1) / (2u << 20) * (2u << 20);
+  void* p = nullptr;
+  cudaError_t e = cudaMalloc(&p, nb);
+  if (e != cudaSuccess) {
+    (void)cudaGetLastError();
+    return fail(FD_ERR_WORKSPACE, "cudaMalloc of %zu workspace bytes failed: %s", nb,
+                cudaGetErrorString(e));
+  }
+  WsHeader h;
+  std::memset(&h, 0, sizeof(h));
+  h.status = old_status;
+  FD_CUDA(cudaMemcpyAsync(p, &h, sizeof(h), cudaMemcpyHostToDevice, stream), "init workspace");
+  FD_CUDA(cudaStreamSynchronize(stream), "cudaStreamSynchronize");
+  w.ptr = p;
+  w.bytes = nb;
+  *out = p;
+  return FD_OK;
+}
+
+// ---------------------------------------------------------------------------- devices --------
+int sm_count(int dev) {
+  static std::mutex mu;
+  static std::map<int, int> cache;
+  std::lock_guard<std::mutex> lock(mu);
+  auto it = cache.find(dev);
+  if (it != cache.end()) return it->second;
+  int n = 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) n = 0;
+  cache[dev] = n;
+  return n;
+}
+
+// ---------------------------------------------------------------------------- tensor maps ----
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static std::once_flag once;
+  static EncodeTiledFn fn = nullptr;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &f, 12000, cudaEnableDefault,
+                                         &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(f);
+  });
+  return fn;
+}
+
+// bf16 tensor map, 128-byte swizzle, 64-element inner box; dims/strides innermost first.
+fd_status make_tmap(CUtensorMap* map, const void* base, int rank, const uint64_t* dims,
+                    const uint64_t* strides_bytes, const uint32_t* box, const char* what) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return fail(FD_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  cuuint64_t d[5], s[4];
+  cuuint32_t b[5], es[5];
+  for (int i = 0; i < rank; ++i) {
+    d[i] = dims[i];
+    b[i] = box[i];
+    es[i] = 1;
+    if (i > 0) s[i - 1] = strides_bytes[i - 1];
+  }
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(base), d, s, b,
+                  es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(FD_ERR_CUDA, "cuTensorMapEncodeTiled(%s) failed: %d", what, (int)r);
+  return FD_OK;
+}
+
+// ---------------------------------------------------------------------------- profiling ------
+struct Profiler {
+  std::mutex mu;
+  std::vector<cudaEvent_t> ev;  // 4 per call
+  int max_calls = 0;
+  int calls = 0;
+  bool active = false;
+} g_prof;
+
+// Returns the 4 events of the next profiled call, or nullptr.
+cudaEvent_t* prof_next() {
+  std::lock_guard<std::mutex> lock(g_prof.mu);
+  if (!g_prof.active || g_prof.calls >= g_prof.max_calls) return nullptr;
+  return &g_prof.ev[4 * static_cast<size_t>(g_prof.calls++)];
+}
+
+// ---------------------------------------------------------------------------- validation -----
+size_t elem_size(int dtype) { return dtype == FD_F32 ? 4 : 2; }
+
+fd_status check_tensor(const fd_tensor* t, const char* name, int ndim) {
+  if (!t) return fail(FD_ERR_INVALID_ARGUMENT, "%s is NULL", name);
+  if (t->ndim != ndim) return fail(FD_ERR_INVALID_ARGUMENT, "%s must have %d dimensions, got %d", name, ndim, t->ndim);
+  if (t->dtype != FD_F32 && t->dtype != FD_BF16)
+    return fail(FD_ERR_UNSUPPORTED, "%s: dtype %d is not FD_F32 or FD_BF16", name, t->dtype);
+  for (int i = 0; i < ndim; ++i) {
+    if (t->shape[i] < 0) return fail(FD_ERR_INVALID_ARGUMENT, "%s: negative shape[%d]", name, i);
+    if (t->shape[i] > INT32_MAX) return fail(FD_ERR_UNSUPPORTED, "%s: shape[%d] exceeds int32", name, i);
+    if (t->stride[i] < 0) return fail(FD_ERR_UNSUPPORTED, "%s: negative stride[%d]", name, i);
+  }
+  if (t->stride[ndim - 1] != 1)
+    return fail(FD_ERR_UNSUPPORTED, "%s: the last dimension must be contiguous (stride 1)", name);
+  return FD_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool stride16(int64_t stride_elems, int dtype) { return (stride_elems * static_cast<int64_t>(elem_size(dtype))) % 16 == 0; }
+
+struct DecodeShape {
+  int B, hq, hkv, g, d, cap, dtype;
+  bool use_tc;
+  int nctas;
+};
+
+fd_status check_kv(const fd_tensor* k, const fd_tensor* v, int dtype, int B, int d) {
+  fd_status s;
+  if ((s = check_tensor(k, "k_cache", 4)) != FD_OK) return s;
+  if ((s = check_tensor(v, "v_cache", 4)) != FD_OK) return s;
+  if (k->dtype != dtype || v->dtype != dtype) return fail(FD_ERR_INVALID_ARGUMENT, "k_cache / v_cache dtype differs from q");
+  for (int i = 0; i < 4; ++i) {
+    if (k->shape[i] != v->shape[i]) return fail(FD_ERR_INVALID_ARGUMENT, "k_cache and v_cache shapes differ");
+    if (k->stride[i] != v->stride[i]) return fail(FD_ERR_UNSUPPORTED, "k_cache and v_cache must share strides");
+  }
+  if (k->shape[0] != B) return fail(FD_ERR_INVALID_ARGUMENT, "k_cache batch %lld != %d", (long long)k->shape[0], B);
+  if (k->shape[3] != d) return fail(FD_ERR_INVALID_ARGUMENT, "k_cache head_dim %lld != q head_dim %d", (long long)k->shape[3], d);
+  if (k->shape[1] < 1) return fail(FD_ERR_INVALID_ARGUMENT, "k_cache needs at least one KV head");
+  if (k->shape[2] < 1) return fail(FD_ERR_INVALID_ARGUMENT, "k_cache capacity (dim 2) must be >= 1");
+  if (k->stride[2] != d) return fail(FD_ERR_UNSUPPORTED, "token rows of the cache must be contiguous (stride[2] == head_dim)");
+  if (B > 0 && (!k->data || !v->data)) return fail(FD_ERR_INVALID_ARGUMENT, "k_cache / v_cache data is NULL");
+  if (!aligned16(k->data) || !aligned16(v->data) || !stride16(k->stride[0], dtype) || !stride16(k->stride[1], dtype))
+    return fail(FD_ERR_UNSUPPORTED, "cache data and strides must be 16-byte aligned");
+  return FD_OK;
+}
+
+fd_status check_q_out(const fd_tensor* q, const fd_tensor* out, const char* qn) {
+  fd_status s;
+  if ((s = check_tensor(q, qn, 3)) != FD_OK) return s;
+  if ((s = check_tensor(out, "out", 3)) != FD_OK) return s;
+  if (out->dtype != q->dtype) return fail(FD_ERR_INVALID_ARGUMENT, "out dtype differs from %s", qn);
+  for (int i = 0; i < 3; ++i)
+    if (out->shape[i] != q->shape[i]) return fail(FD_ERR_INVALID_ARGUMENT, "out shape differs from %s", qn);
+  if (q->shape[0] > 0 && (!q->data || !out->data)) return fail(FD_ERR_INVALID_ARGUMENT, "%s / out data is NULL", qn);
+  if (!aligned16(q->data) || !stride16(q->stride[0], q->dtype) || !stride16(q->stride[1], q->dtype))
+    return fail(FD_ERR_UNSUPPORTED, "%s data and strides must be 16-byte aligned", qn);
+  return FD_OK;
+}
+
+fd_status resolve_decode(const fd_tensor* q, const fd_tensor* k, const fd_tensor* v,
+                         const fd_tensor* out, DecodeShape* sh) {
+  fd_status s;
+  if ((s = check_q_out(q, out, "q")) != FD_OK) return s;
+  sh->B = static_cast<int>(q->shape[0]);
+  sh->hq = static_cast<int>(q->shape[1]);
+  sh->d = static_cast<int>(q->shape[2]);
+  sh->dtype = q->dtype;
+  if (sh->d != 64 && sh->d != 128) return fail(FD_ERR_UNSUPPORTED, "head_dim %d: only 64 and 128 are supported", sh->d);
+  if ((s = check_kv(k, v, sh->dtype, sh->B, sh->d)) != FD_OK) return s;
+  sh->hkv = static_cast<int>(k->shape[1]);
+  sh->cap = static_cast<int>(k->shape[2]);
+  if (sh->hq < 1 || sh->hq % sh->hkv != 0)
+    return fail(FD_ERR_INVALID_ARGUMENT, "q heads (%d) must be a positive multiple of KV heads (%d)", sh->hq, sh->hkv);
+  sh->g = sh->hq / sh->hkv;
+  if (sh->B > kMaxPlanBatch) return fail(FD_ERR_UNSUPPORTED, "batch %d exceeds %d", sh->B, kMaxPlanBatch);
+  sh->use_tc = sh->dtype == FD_BF16 && sh->d == 128 && sh->g >= 2 && sh->g <= 16;
+  if (!sh->use_tc && sh->g > 8)
+    return fail(FD_ERR_UNSUPPORTED, "group size %d needs bf16 with head_dim 128 (tensor-core kernel)", sh->g);
+  return FD_OK;
+}
+
+int decode_ctas(int dev, bool use_tc) {
+  const int n = sm_count(dev);
+  return use_tc ? n : n * simt_ctas_per_sm();
+}
+
+size_t decode_ws_bytes(int B, int hq, int hkv, int cap, int d, int fixed, int nctas) {
+  const int64_t items = decode_max_items(B, hkv, cap, fixed, nctas);
+  const int64_t slots = (items + hkv - 1) / hkv;
+  return ws_layout(items, 0, B, slots, hq, d).total;
+}
+
+// ---------------------------------------------------------------------------- host planner ---
+struct HostPlan {
+  int32_t chunk = 0;
+  std::vector<int32_t> lens, nsplit, order;
+  int64_t total_items = 0;
+};
+
+void host_plan(const int32_t* lens_in, int B, int hkv, int cap, int fixed, int nctas, HostPlan* hp) {
+  hp->lens.resize(B);
+  hp->nsplit.resize(B);
+  int64_t total = 0;
+  for (int b = 0; b < B; ++b) {
+    hp->lens[b] = clamp_len(lens_in[b], cap);
+    total += hp->lens[b];
+  }
+  hp->chunk = fixed > 0 ? 0 : plan_chunk_tokens(total, hkv, nctas);
+  std::vector<int32_t> key(B);
+  hp->total_items = 0;
+  for (int b = 0; b < B; ++b) {
+    hp->nsplit[b] = plan_num_splits(hp->lens[b], hp->chunk, fixed);
+    key[b] = plan_sort_key(hp->lens[b], hp->nsplit[b]);
+    hp->total_items += static_cast<int64_t>(hp->nsplit[b]) * hkv;
+  }
+  hp->order.resize(B);
+  for (int b = 0; b < B; ++b) hp->order[b] = b;
+  std::stable_sort(hp->order.begin(), hp->order.end(), [&](int a, int c) { return key[a] > key[c]; });
+}
+
+void end_profile_events(cudaEvent_t* ev, int slot, cudaStream_t stream) {
+  if (ev) cudaEventRecord(ev[slot], stream);
+}
+
+}  // namespace
+
+// ================================================================================ ABI ========
+extern "C" {
+
+const char* fd_status_string(fd_status s) {
+  switch (s) {
+    case FD_OK: return "FD_OK";
+    case FD_ERR_INVALID_ARGUMENT: return "FD_ERR_INVALID_ARGUMENT";
+    case FD_ERR_UNSUPPORTED: return "FD_ERR_UNSUPPORTED";
+    case FD_ERR_CUDA: return "FD_ERR_CUDA";
+    case FD_ERR_WORKSPACE: return "FD_ERR_WORKSPACE";
+  }
+  return "FD_UNKNOWN_STATUS";
+}
+
+const char* fd_last_error_message(void) { return g_last_error.c_str(); }
+
+int32_t fd_decode_num_ctas(int32_t device, int32_t dtype, int32_t group_size, int32_t head_dim) {
+  const bool tc = dtype == FD_BF16 && head_dim == 128 && group_size >= 2 && group_size <= 16;
+  return decode_ctas(device, tc);
+}
+
+size_t fd_decode_workspace_bytes(int32_t batch, int32_t num_q_heads, int32_t num_kv_heads,
+                                 int32_t cache_capacity, int32_t head_dim, int32_t num_splits,
+                                 int32_t num_ctas) {
+  if (batch < 0 || num_q_heads < 1 || num_kv_heads < 1 || cache_capacity < 0 || head_dim < 1 || num_splits < 0)
+    return 0;
+  return decode_ws_bytes(batch, num_q_heads, num_kv_heads, cache_capacity, head_dim, num_splits,
+                         num_ctas);
+}
+
+fd_status fd_split_plan(const int32_t* cache_lens_host, int32_t batch, int32_t num_kv_heads,
+                        int32_t cache_capacity, int32_t num_splits, int32_t num_ctas,
+                        int32_t* splits_per_seq_host, int32_t* items_host,
+                        int32_t items_capacity, fd_plan_info* info) {
+  if (!info) return fail(FD_ERR_INVALID_ARGUMENT, "info is NULL");
+  if (batch < 0) return fail(FD_ERR_INVALID_ARGUMENT, "batch must be >= 0");
+  if (batch > 0 && !cache_lens_host) return fail(FD_ERR_INVALID_ARGUMENT, "cache_lens_host is NULL");
+  if (num_kv_heads < 1) return fail(FD_ERR_INVALID_ARGUMENT, "num_kv_heads must be >= 1");
+  if (cache_capacity < 0) return fail(FD_ERR_INVALID_ARGUMENT, "cache_capacity must be >= 0");
+  if (num_splits < 0) return fail(FD_ERR_INVALID_ARGUMENT, "num_splits must be >= 0");
+  if (num_ctas < 1) return fail(FD_ERR_INVALID_ARGUMENT, "num_ctas must be >= 1");
+  if (items_host && items_capacity < 0) return fail(FD_ERR_INVALID_ARGUMENT, "items_capacity must be >= 0");
+  HostPlan hp;
+  host_plan(cache_lens_host, batch, num_kv_heads, cache_capacity, num_splits, num_ctas, &hp);
+  if (hp.total_items > INT32_MAX) return fail(FD_ERR_UNSUPPORTED, "plan has more than 2^31 items");
+  int32_t maxs = 0;
+  for (int b = 0; b < batch; ++b) {
+    if (splits_per_seq_host) splits_per_seq_host[b] = hp.nsplit[b];
+    maxs = std::max(maxs, hp.nsplit[b]);
+  }
+  if (items_host) {
+    int64_t i = 0;
+    for (int r = 0; r < batch && i < items_capacity; ++r) {
+      const int b = hp.order[r];
+      const int n = hp.nsplit[b];
+      for (int h = 0; h < num_kv_heads && i < items_capacity; ++h)
+        for (int s = 0; s < n && i < items_capacity; ++s, ++i) {
+          int32_t t0, t1;
+          plan_split_range(hp.lens[b], n, s, num_splits, &t0, &t1);
+          int32_t* o = items_host + 5 * i;
+          o[0] = b; o[1] = h; o[2] = s; o[3] = t0; o[4] = t1;
+        }
+    }
+  }
+  info->chunk_tokens = hp.chunk;
+  info->total_items = static_cast<int32_t>(hp.total_items);
+  info->max_splits_per_seq = maxs;
+  info->num_ctas = num_ctas;
+  // plan tables only: header, items and the per-row split tables
+  info->workspace_bytes = ws_layout(hp.total_items, 0, batch, 0, 1, 1).total;
+  return FD_OK;
+}
+
+fd_status fd_split_plan_device(const int32_t* cache_lens, int32_t batch, int32_t num_kv_heads,
+                               int32_t cache_capacity, int32_t num_splits, int32_t num_ctas,
+                               int32_t* splits_per_seq_dev, int32_t* items_dev,
+                               int32_t items_capacity, int32_t* total_items_dev, void* stream_) {
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+  if (batch < 0 || batch > kMaxPlanBatch) return fail(FD_ERR_INVALID_ARGUMENT, "batch must be in [0, %d]", kMaxPlanBatch);
+  if (batch > 0 && (!cache_lens || !splits_per_seq_dev)) return fail(FD_ERR_INVALID_ARGUMENT, "NULL device pointer");
+  if (!total_items_dev) return fail(FD_ERR_INVALID_ARGUMENT, "total_items_dev is NULL");
+  if (num_kv_heads < 1 || cache_capacity < 0 || num_splits < 0 || num_ctas < 1)
+    return fail(FD_ERR_INVALID_ARGUMENT, "bad plan arguments");
+  if (items_dev && items_capacity < 0) return fail(FD_ERR_INVALID_ARGUMENT, "items_capacity must be >= 0");
+  const int64_t items = decode_max_items(batch, num_kv_heads, cache_capacity, num_splits, num_ctas);
+  const WsLayout L = ws_layout(items, 0, batch, 0, 1, 1);
+  void* ws = nullptr;
+  fd_status s = get_workspace(stream, L.total, &ws);
+  if (s != FD_OK) return s;
+  char* base = static_cast<char*>(ws);
+  PlanParams pp{};
+  pp.lens = cache_lens;
+  pp.B = batch;
+  pp.hkv = num_kv_heads;
+  pp.hq = num_kv_heads;
+  pp.cap = cache_capacity;
+  pp.fixed = num_splits;
+  pp.nctas = num_ctas;
+  pp.max_dec_items = items;
+  pp.hdr = reinterpret_cast<WsHeader*>(base);
+  pp.items = reinterpret_cast<DecodeItem*>(base + L.dec_items);
+  pp.row_nsplit = reinterpret_cast<int32_t*>(base + L.row_nsplit);
+  pp.row_base = reinterpret_cast<int32_t*>(base + L.row_base);
+  pp.out_splits = splits_per_seq_dev;
+  pp.out_items = items_dev;
+  pp.out_cap = items_dev ? items_capacity : 0;
+  pp.out_total = total_items_dev;
+  FD_CUDA(launch_plan_decode(pp, stream), "plan kernel launch");
+  return FD_OK;
+}
+
+fd_status fd_decode_attention(const fd_tensor* q, const fd_tensor* k_cache,
+                              const fd_tensor* v_cache, const int32_t* cache_lens,
+                              int32_t num_splits, fd_tensor* out, float* lse, void* stream_) {
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+  DecodeShape sh{};
+  fd_status s = resolve_decode(q, k_cache, v_cache, out, &sh);
+  if (s != FD_OK) return s;
+  if (num_splits < 0) return fail(FD_ERR_INVALID_ARGUMENT, "num_splits must be >= 0");
+  if (num_splits > 65536) return fail(FD_ERR_UNSUPPORTED, "num_splits above 65536");
+  if (sh.B == 0) return FD_OK;
+  if (!cache_lens) return fail(FD_ERR_INVALID_ARGUMENT, "cache_lens is NULL");
+  if (!lse) return fail(FD_ERR_INVALID_ARGUMENT, "lse is NULL");
+  int dev = 0;
+  FD_CUDA(cudaGetDevice(&dev), "cudaGetDevice");
+  const int nctas = decode_ctas(dev, sh.use_tc);
+  if (nctas < 1) return fail(FD_ERR_CUDA, "no multiprocessors reported for device %d", dev);
+
+  const int64_t max_items = decode_max_items(sh.B, sh.hkv, sh.cap, num_splits, nctas);
+  const int64_t max_slots = (max_items + sh.hkv - 1) / sh.hkv;
+  const WsLayout L = ws_layout(max_items, 0, sh.B, max_slots, sh.hq, sh.d);
+  void* ws = nullptr;
+  if ((s = get_workspace(stream, L.total, &ws)) != FD_OK) return s;
+  char* base = static_cast<char*>(ws);
+  WsHeader* hdr = reinterpret_cast<WsHeader*>(base);
+  DecodeItem* items = reinterpret_cast<DecodeItem*>(base + L.dec_items);
+  int32_t* row_nsplit = reinterpret_cast<int32_t*>(base + L.row_nsplit);
+  int32_t* row_base = reinterpret_cast<int32_t*>(base + L.row_base);
+  float* part_o = reinterpret_cast<float*>(base + L.part_o);
+  float* part_lse = reinterpret_cast<float*>(base + L.part_lse);
+
+  DecodeParams dp{};
+  dp.q = q->data;
+  dp.q_sr = q->stride[0];
+  dp.q_sh = q->stride[1];
+  dp.k = k_cache->data;
+  dp.v = v_cache->data;
+  dp.kv_sb = k_cache->stride[0];
+  dp.kv_sh = k_cache->stride[1];
+  dp.out = out->data;
+  dp.o_sr = out->stride[0];
+  dp.o_sh = out->stride[1];
+  dp.lse = lse;
+  dp.hq = sh.hq;
+  dp.hkv = sh.hkv;
+  dp.g = sh.g;
+  dp.d = sh.d;
+  dp.cap = sh.cap;
+  dp.q_box_rows = std::min(16, sh.hq);
+  dp.kv_box_rows = std::min(128, sh.cap);
+  dp.scale_log2 = static_cast<float>(1.0 / std::sqrt(static_cast<double>(sh.d)) * 1.4426950408889634);
+  dp.hdr = hdr;
+  dp.items = items;
+  dp.row_base = row_base;
+  dp.part_o = part_o;
+  dp.part_lse = part_lse;
+
+  CUtensorMap tq, tk, tv;
+  if (sh.use_tc) {
+    const uint64_t qd[3] = {static_cast<uint64_t>(sh.d), static_cast<uint64_t>(sh.hq), static_cast<uint64_t>(sh.B)};
+    const uint64_t qs[2] = {static_cast<uint64_t>(q->stride[1]) * 2, static_cast<uint64_t>(q->stride[0]) * 2};
+    const uint32_t qb[3] = {64, static_cast<uint32_t>(dp.q_box_rows), 1};
+    if ((s = make_tmap(&tq, q->data, 3, qd, qs, qb, "q")) != FD_OK) return s;
+    const uint64_t kd[4] = {static_cast<uint64_t>(sh.d), static_cast<uint64_t>(sh.cap), static_cast<uint64_t>(sh.hkv), static_cast<uint64_t>(sh.B)};
+    const uint64_t ks[3] = {static_cast<uint64_t>(k_cache->stride[2]) * 2, static_cast<uint64_t>(k_cache->stride[1]) * 2,
+                            static_cast<uint64_t>(k_cache->stride[0]) * 2};
+    const uint32_t kb[4] = {64, static_cast<uint32_t>(dp.kv_box_rows), 1, 1};
+    if ((s = make_tmap(&tk, k_cache->data, 4, kd, ks, kb, "k_cache")) != FD_OK) return s;
+    if ((s = make_tmap(&tv, v_cache->data, 4, kd, ks, kb, "v_cache")) != FD_OK) return s;
+  }
+
+  PlanParams pp{};
+  pp.lens = cache_lens;
+  pp.B = sh.B;
+  pp.hkv = sh.hkv;
+  pp.hq = sh.hq;
+  pp.cap = sh.cap;
+  pp.fixed = num_splits;
+  pp.nctas = nctas;
+  pp.max_dec_items = max_items;
+  pp.hdr = hdr;
+  pp.items = items;
+  pp.row_nsplit = row_nsplit;
+  pp.row_base = row_base;
+
+  CombineParams cp{};
+  cp.row_nsplit = row_nsplit;
+  cp.row_base = row_base;
+  cp.part_o = part_o;
+  cp.part_lse = part_lse;
+  cp.out = out->data;
+  cp.o_sr = out->stride[0];
+  cp.o_sh = out->stride[1];
+  cp.lse = lse;
+  cp.rows = sh.B;
+  cp.hq = sh.hq;
+  cp.d = sh.d;
+  cp.dtype = sh.dtype;
+
+  cudaEvent_t* ev = prof_next();
+  end_profile_events(ev, 0, stream);
+  FD_CUDA(launch_plan_decode(pp, stream), "plan kernel launch");
+  end_profile_events(ev, 1, stream);
+  if (sh.use_tc) {
+    FD_CUDA(launch_decode_tc(dp, tq, tk, tv, nctas, stream), "tensor-core split kernel launch");
+  } else {
+    FD_CUDA(launch_decode_simt(dp, sh.dtype, nctas, stream), "split kernel launch");
+  }
+  end_profile_events(ev, 2, stream);
+  FD_CUDA(launch_combine(cp, stream), "combine kernel launch");
+  end_profile_events(ev, 3, stream);
+  return FD_OK;
+}
+
+fd_status fd_chunk_prefill_attention(const fd_tensor* q_chunk, const fd_tensor* k_cache,
+                                     const fd_tensor* v_cache, const int32_t* prefix_lens,
+                                     const int32_t* chunk_lens, fd_tensor* out, float* lse,
+                                     void* stream) {
+  (void)q_chunk; (void)k_cache; (void)v_cache; (void)prefix_lens; (void)chunk_lens;
+  (void)out; (void)lse; (void)stream;
+  return fail(FD_ERR_UNSUPPORTED, "chunked prefill is not built yet");
+}
+
+size_t fd_chunk_workspace_bytes(int32_t batch, int32_t total_rows, int32_t num_q_heads,
+                                int32_t num_kv_heads, int32_t cache_capacity, int32_t head_dim,
+                                int32_t num_ctas) {
+  (void)batch; (void)total_rows; (void)num_q_heads; (void)num_kv_heads; (void)cache_capacity;
+  (void)head_dim; (void)num_ctas;
+  return 0;
+}
+
+fd_status fd_reserve_workspace(size_t bytes, void* stream_) {
+  void* ws = nullptr;
+  return get_workspace(static_cast<cudaStream_t>(stream_), std::max(bytes, sizeof(WsHeader)), &ws);
+}
+
+fd_status fd_poll_status(void* stream_, uint32_t* flags) {
+  if (!flags) return fail(FD_ERR_INVALID_ARGUMENT, "flags is NULL");
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+  *flags = 0;
+  int dev = 0;
+  FD_CUDA(cudaGetDevice(&dev), "cudaGetDevice");
+  FD_CUDA(cudaStreamSynchronize(stream), "cudaStreamSynchronize");
+  void* ptr = nullptr;
+  {
+    std::lock_guard<std::mutex> lock(g_mu);
+    auto it = g_ws.find({dev, reinterpret_cast<uintptr_t>(stream)});
+    if (it != g_ws.end()) ptr = it->second.ptr;
+  }
+  if (!ptr) return FD_OK;
+  uint32_t v = 0;
+  FD_CUDA(cudaMemcpy(&v, ptr, sizeof(v), cudaMemcpyDeviceToHost), "read status");
+  const uint32_t zero = 0;
+  FD_CUDA(cudaMemcpy(ptr, &zero, sizeof(zero), cudaMemcpyHostToDevice), "clear status");
+  *flags = v;
+  return FD_OK;
+}
+
+fd_status fd_profile_begin(int32_t max_calls) {
+  if (max_calls < 1) return fail(FD_ERR_INVALID_ARGUMENT, "max_calls must be >= 1");
+  std::lock_guard<std::mutex> lock(g_prof.mu);
+  for (cudaEvent_t e : g_prof.ev) cudaEventDestroy(e);
+  g_prof.ev.assign(4 * static_cast<size_t>(max_calls), nullptr);
+  for (auto& e : g_prof.ev) FD_CUDA(cudaEventCreate(&e), "cudaEventCreate");
+  g_prof.max_calls = max_calls;
+  g_prof.calls = 0;
+  g_prof.active = true;
+  return FD_OK;
+}
+
+fd_status fd_profile_end(float* ms, int32_t max_calls, int32_t* n_calls) {
+  if (!ms || !n_calls) return fail(FD_ERR_INVALID_ARGUMENT, "NULL output");
+  std::lock_guard<std::mutex> lock(g_prof.mu);
+  if (!g_prof.active) return fail(FD_ERR_INVALID_ARGUMENT, "profiling was not started");
+  const int n = std::min(g_prof.calls, max_calls);
+  for (int i = 0; i < n; ++i) {
+    cudaEvent_t* e = &g_prof.ev[4 * static_cast<size_t>(i)];
+    FD_CUDA(cudaEventSynchronize(e[3]), "cudaEventSynchronize");
+    for (int j = 0; j < 3; ++j) FD_CUDA(cudaEventElapsedTime(&ms[3 * i + j], e[j], e[j + 1]), "cudaEventElapsedTime");
+  }
+  *n_calls = n;
+  for (cudaEvent_t e : g_prof.ev) cudaEventDestroy(e);
+  g_prof.ev.clear();
+  g_prof.active = false;
+  g_prof.calls = 0;
+  return FD_OK;
+}
+
+void fd_shutdown(void) {
+  {
+    std::lock_guard<std::mutex> lock(g_mu);
+    for (auto& kv : g_ws) {
+      if (kv.second.ptr) {
+        int cur = 0;
+        cudaGetDevice(&cur);
+        cudaSetDevice(kv.first.first);
+        cudaDeviceSynchronize();
+        cudaFree(kv.second.ptr);
+        cudaSetDevice(cur);
+      }
+    }
+    g_ws.clear();
+  }
+  std::lock_guard<std::mutex> lock(g_prof.mu);
+  for (cudaEvent_t e : g_prof.ev) cudaEventDestroy(e);
+  g_prof.ev.clear();
+  g_prof.active = false;
+}
+
+}  // extern "C"

@@ -1,0 +1,97 @@
+// Kernel parameter blocks and launcher declarations shared inside the library.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "plan.h"
+
+namespace fd {
+
+// Device planner for a decode call (or the decode rows of a chunked-prefill call).
+struct PlanParams {
+  const int32_t* lens;      // [B] cache lengths (decode) or prefix lengths (chunk mode)
+  const int32_t* chunk_lens;  // chunk mode only: [B] chunk lengths; nullptr for decode
+  int32_t B, hkv, hq, cap, fixed, nctas;
+  int64_t max_dec_items, max_tile_items, max_rows, max_slots;
+  WsHeader* hdr;
+  DecodeItem* items;
+  TileItem* tiles;
+  int32_t* row_nsplit;
+  int32_t* row_base;
+  // optional export of the decode plan (fd_split_plan_device)
+  int32_t* out_splits;
+  int32_t* out_items;
+  int32_t out_cap;
+  int32_t* out_total;
+};
+
+// Split pass of decode items (both the CUDA-core and the tensor-core kernels).
+struct DecodeParams {
+  const void* q;     // [rows, Hq, D]
+  int64_t q_sr, q_sh;  // element strides of row and head
+  const void* k;     // [B, Hkv, S_cap, D], token rows contiguous
+  const void* v;
+  int64_t kv_sb, kv_sh;  // element strides of batch and head (same for k and v)
+  void* out;         // [rows, Hq, D]
+  int64_t o_sr, o_sh;
+  float* lse;        // [rows, Hq] contiguous
+  int32_t hq, hkv, g, d, cap;
+  int32_t q_box_rows;   // rows of one Q tensor-map box (tensor-core kernel): min(16, Hq)
+  int32_t kv_box_rows;  // rows of one K/V tensor-map box (tensor-core kernel): min(128, S_cap)
+  float scale_log2;  // softmax scale * log2(e)
+  WsHeader* hdr;
+  const DecodeItem* items;
+  const int32_t* row_base;
+  float* part_o;     // [slots, Hq, D]
+  float* part_lse;   // [slots, Hq] (log2 domain)
+};
+
+// Chunked-prefill tiles.
+struct TileParams {
+  const void* q;
+  int64_t q_sr, q_sh;
+  void* out;
+  int64_t o_sr, o_sh;
+  float* lse;
+  int32_t hq, hkv, g, d, cap;
+  float scale_log2;
+  WsHeader* hdr;
+  const TileItem* tiles;
+  float* part_o;
+  float* part_lse;
+};
+
+// LSE merge of the partials of rows with more than one split.
+struct CombineParams {
+  const int32_t* row_nsplit;
+  const int32_t* row_base;
+  const float* part_o;
+  const float* part_lse;
+  void* out;
+  int64_t o_sr, o_sh;
+  float* lse;
+  int32_t rows, hq, d, dtype;
+};
+
+cudaError_t launch_plan_decode(const PlanParams& p, cudaStream_t stream);
+cudaError_t launch_plan_chunk(const PlanParams& p, cudaStream_t stream);
+
+// CUDA-core split kernel: any dtype, D in {64,128}, G <= 8.
+int simt_ctas_per_sm();
+cudaError_t launch_decode_simt(const DecodeParams& p, int dtype, int nctas, cudaStream_t stream);
+
+// tcgen05 split kernel: bf16, D == 128, 2 <= G <= 16.
+cudaError_t launch_decode_tc(const DecodeParams& p, const CUtensorMap& tmap_q,
+                             const CUtensorMap& tmap_k, const CUtensorMap& tmap_v, int nctas,
+                             cudaStream_t stream);
+
+// tcgen05 chunked-prefill tile kernel: bf16, D == 128.
+cudaError_t launch_chunk_tc(const TileParams& p, const CUtensorMap& tmap_q,
+                            const CUtensorMap& tmap_k, const CUtensorMap& tmap_v, int nctas,
+                            cudaStream_t stream);
+
+cudaError_t launch_combine(const CombineParams& p, cudaStream_t stream);
+
+}  // namespace fd

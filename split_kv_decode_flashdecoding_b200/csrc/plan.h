@@ -1,0 +1,147 @@
+// Split planning shared by the host planner (fd_split_plan) and the device planner kernel, plus
+// the work-item formats and the workspace layout the kernels read.
+//
+// Source: "大模型推理加速FlashDecoding算法原理与多GPU并行解码实战" (FlashDecoding algorithm and
+// multi-GPU decoding), section "Variable-Length序列动态切分策略": a greedy allocator that fills
+// each worker up to ceil(total tokens / workers) with pieces of at most max_chunk = 1024 tokens
+// and never leaves a piece under min_chunk = 128 alone; section "性能压测与瓶颈分析": pieces
+// under ~256 tokens lose to launch overhead. On one GPU the workers are persistent CTAs; the
+// plan below gives every sequence equal splits sized so that about kWaves items exist per CTA,
+// restarts the offset for every sequence and drops no token.
+#pragma once
+
+#include <stddef.h>
+#include <stdint.h>
+
+#include "../../include/fd.h"
+
+#if defined(__CUDACC__)
+#define FD_HD __host__ __device__ __forceinline__
+#else
+#define FD_HD inline
+#endif
+
+namespace fd {
+
+constexpr int32_t kMinChunk = 256;        // launch-overhead floor ("性能压测与瓶颈分析")
+constexpr int32_t kMaxChunk = 1024;       // allocator max_chunk / top of the 256-1024 tile range
+constexpr int32_t kWaves = 8;             // target work items per persistent CTA
+constexpr int32_t kQTile = 128;           // chunked-prefill query rows per tile
+constexpr int32_t kChunkKvSplit = 2048;   // keys per split of a chunked-prefill query tile
+constexpr int32_t kMaxPlanBatch = 4096;   // largest batch the one-CTA device planner accepts
+
+// One split of one (sequence, KV head): keys [t0, t1) of cache row b, output row `row`.
+struct DecodeItem {
+  int32_t row;     // output row: b for decode, the packed query row for chunked prefill
+  int32_t b;       // cache batch index
+  int32_t h;       // KV head
+  int32_t split;   // split index within the sequence
+  int32_t t0, t1;  // key range
+  int32_t nsplit;  // splits of this sequence (1: write the final output directly)
+  int32_t seqlen;  // clamped sequence length (keys at >= seqlen may hold anything)
+};
+static_assert(sizeof(DecodeItem) == 32, "DecodeItem is 32 bytes");
+
+// One key split of one 128-row query tile of one head of a chunked-prefill request.
+struct TileItem {
+  int32_t b, h, split, nsplit;
+  int32_t k0, k1;    // key range of the split
+  int32_t row0;      // packed query row of the tile's first row
+  int32_t pos0;      // chunk position of the tile's first row
+  int32_t rows;      // valid rows in the tile (<= kQTile)
+  int32_t prefix;    // prefix length: row at chunk position i sees keys <= prefix + i
+  int32_t slot0;     // partial slot of (row0, split 0); row r uses slot0 + r * nsplit + split
+  int32_t pad[5];
+};
+static_assert(sizeof(TileItem) == 64, "TileItem is 64 bytes");
+
+// Header at the start of every workspace.
+struct WsHeader {
+  uint32_t status;          // FD_FLAG_* bits, sticky until fd_poll_status
+  int32_t num_dec_items;    // decode items planned by the last call
+  int32_t num_tile_items;   // tile items planned by the last call
+  int32_t dec_counter;      // dynamic scheduler cursor (reset by the planner every call)
+  int32_t tile_counter;
+  int32_t pad[59];
+};
+static_assert(sizeof(WsHeader) == 256, "WsHeader is 256 bytes");
+
+FD_HD int64_t cdiv64(int64_t a, int64_t b) { return (a + b - 1) / b; }
+FD_HD size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+FD_HD int32_t clamp_len(int64_t len, int32_t cap) {
+  return len < 0 ? 0 : (len > cap ? cap : static_cast<int32_t>(len));
+}
+
+// chunk = clamp(ceil(total * Hkv / (kWaves * nctas)), kMinChunk, kMaxChunk)
+FD_HD int32_t plan_chunk_tokens(int64_t total, int32_t hkv, int32_t nctas) {
+  int64_t c = cdiv64(total * hkv, static_cast<int64_t>(kWaves) * (nctas > 0 ? nctas : 1));
+  if (c < kMinChunk) c = kMinChunk;
+  if (c > kMaxChunk) c = kMaxChunk;
+  return static_cast<int32_t>(c);
+}
+
+// Splits of a sequence: the fixed count, else max(1, ceil(len / chunk)).
+FD_HD int32_t plan_num_splits(int32_t len, int32_t chunk, int32_t fixed) {
+  if (fixed > 0) return fixed;
+  int32_t n = static_cast<int32_t>(cdiv64(len, chunk));
+  return n < 1 ? 1 : n;
+}
+
+// Key range of split s. Fixed mode: [min(s*c, len), min((s+1)*c, len)) with c = ceil(len/n)
+// (the FlashDecoding page's chunk_size rule); planner mode: equal splits
+// [floor(s*len/n), floor((s+1)*len/n)).
+FD_HD void plan_split_range(int32_t len, int32_t n, int32_t s, int32_t fixed, int32_t* t0,
+                            int32_t* t1) {
+  if (fixed > 0) {
+    int64_t c = cdiv64(len, n);
+    int64_t a = s * c, e = (s + 1) * c;
+    *t0 = static_cast<int32_t>(a < len ? a : len);
+    *t1 = static_cast<int32_t>(e < len ? e : len);
+  } else {
+    *t0 = static_cast<int32_t>((static_cast<int64_t>(s) * len) / n);
+    *t1 = static_cast<int32_t>((static_cast<int64_t>(s + 1) * len) / n);
+  }
+}
+
+// Longest-first ordering key of a sequence: its longest split.
+FD_HD int32_t plan_sort_key(int32_t len, int32_t n) {
+  return static_cast<int32_t>(cdiv64(len, n));
+}
+
+// Upper bound of the decode items of any plan of this shape (any lengths), used to size the
+// workspace: sum_b n_b < B + max(kWaves * nctas / Hkv, B * S_cap / kMaxChunk).
+FD_HD int64_t decode_max_items(int64_t B, int64_t hkv, int64_t cap, int32_t fixed,
+                               int32_t nctas) {
+  if (fixed > 0) return B * hkv * fixed;
+  int64_t a = static_cast<int64_t>(kWaves) * (nctas > 0 ? nctas : 1);
+  int64_t b = cdiv64(hkv * B * cap, kMaxChunk);
+  return hkv * B + (a > b ? a : b);
+}
+
+// Workspace layout (byte offsets, 256-byte aligned sections).
+struct WsLayout {
+  size_t dec_items, tile_items, row_nsplit, row_base, part_o, part_lse, total;
+};
+
+FD_HD WsLayout ws_layout(int64_t max_dec_items, int64_t max_tile_items, int64_t rows,
+                         int64_t max_slots, int32_t hq, int32_t d) {
+  WsLayout L;
+  size_t off = sizeof(WsHeader);
+  L.dec_items = off;
+  off = align_up(off + static_cast<size_t>(max_dec_items) * sizeof(DecodeItem), 256);
+  L.tile_items = off;
+  off = align_up(off + static_cast<size_t>(max_tile_items) * sizeof(TileItem), 256);
+  L.row_nsplit = off;
+  off = align_up(off + static_cast<size_t>(rows) * 4, 256);
+  L.row_base = off;
+  off = align_up(off + static_cast<size_t>(rows) * 4, 256);
+  L.part_o = off;
+  off = align_up(off + static_cast<size_t>(max_slots) * hq * d * 4, 256);
+  L.part_lse = off;
+  off = align_up(off + static_cast<size_t>(max_slots) * hq * 4, 256);
+  L.total = off;
+  return L;
+}
+
+}  // namespace fd

@@ -1,0 +1,158 @@
+"""CPU checks of the C ABI: the library loads, exports every function include/fd.h declares, its
+host planner equals the planner oracle integer for integer, and bad arguments are rejected on
+the host before anything touches a GPU. No test here runs a kernel."""
+
+import ctypes
+import os
+import random
+import re
+
+import pytest
+
+import split_kv_decode_flashdecoding_b200 as fd
+from oracle import planner as P
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "fd.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(fd_[a-z_0-9]+)\s*\(", src)))
+
+
+def test_every_declared_symbol_is_exported_and_bound():
+    names = _declared()
+    assert "fd_decode_attention" in names and "fd_split_plan" in names
+    assert "fd_chunk_prefill_attention" in names
+    for n in names:
+        assert hasattr(fd.lib, n), f"{n} not exported by libfd.so"
+        assert n in fd.ABI_FUNCTIONS, f"{n} has no binding"
+
+
+def test_status_strings():
+    for s, name in enumerate(["FD_OK", "FD_ERR_INVALID_ARGUMENT", "FD_ERR_UNSUPPORTED",
+                              "FD_ERR_CUDA", "FD_ERR_WORKSPACE"]):
+        assert fd.fd_status_string(s) == name
+    assert fd.fd_status_string(99) == "FD_UNKNOWN_STATUS"
+
+
+@pytest.mark.parametrize("seed", range(60))
+def test_host_plan_equals_oracle(seed):
+    rng = random.Random(1000 + seed)
+    B = rng.choice([1, 2, 3, 5, 32, 64, 200])
+    hkv = rng.choice([1, 2, 8, 40])
+    cap = rng.choice([1, 16, 63, 64, 65, 257, 1024, 16384, 32768])
+    ctas = rng.choice([1, 7, 148, 296])
+    fixed = rng.choice([0, 0, 0, 1, 4, 9])
+    lens = [rng.choice([0, 1, cap - 1, cap, cap + 5, -2, rng.randint(0, cap)]) for _ in range(B)]
+    info, splits, items = fd.fd_split_plan(lens, hkv, cap, fixed, ctas)
+    ref = P.decode_plan(lens, hkv, cap, ctas, fixed)
+    assert info["chunk_tokens"] == ref.chunk_tokens
+    assert splits == ref.splits_per_seq
+    assert info["total_items"] == ref.total_items
+    assert info["max_splits_per_seq"] == ref.max_splits_per_seq
+    assert [tuple(x) for x in items] == ref.items
+
+
+def test_host_plan_workload_shapes():
+    from workloads import uniform_lens
+    lens = uniform_lens(1103, 32, 1024, 32768)
+    info, splits, items = fd.fd_split_plan(lens, 8, 32768, 0, 148)
+    ref = P.decode_plan(lens, 8, 32768, 148, 0)
+    assert info["chunk_tokens"] == 1024 == ref.chunk_tokens
+    assert [tuple(x) for x in items] == ref.items
+    assert info["total_items"] <= P.MAX_CHUNK * 0 + 8 * 32 + max(8 * 148, 8 * 32 * 32)
+
+
+def test_plan_rejects_bad_arguments():
+    info = fd.FdPlanInfo()
+    lens = (ctypes.c_int32 * 2)(5, 6)
+    assert fd.lib.fd_split_plan(lens, -1, 1, 8, 0, 1, None, None, 0, ctypes.byref(info)) == 1
+    assert fd.lib.fd_split_plan(lens, 2, 0, 8, 0, 1, None, None, 0, ctypes.byref(info)) == 1
+    assert fd.lib.fd_split_plan(lens, 2, 1, 8, -1, 1, None, None, 0, ctypes.byref(info)) == 1
+    assert fd.lib.fd_split_plan(lens, 2, 1, 8, 0, 0, None, None, 0, ctypes.byref(info)) == 1
+    assert fd.lib.fd_split_plan(None, 2, 1, 8, 0, 1, None, None, 0, ctypes.byref(info)) == 1
+    assert fd.lib.fd_split_plan(lens, 2, 1, 8, 0, 1, None, None, 0, None) == 1
+    assert "info" in fd.lib.fd_last_error_message().decode()
+
+
+def _fake(shape, dtype=fd.FD_BF16, strides=None, ptr=0x100000):
+    t = fd.FdTensor()
+    t.data = ptr
+    t.dtype = dtype
+    t.ndim = len(shape)
+    if strides is None:
+        strides, s = [], 1
+        for n in reversed(shape):
+            strides.insert(0, s)
+            s *= n
+    for i, (n, st) in enumerate(zip(shape, strides)):
+        t.shape[i] = n
+        t.stride[i] = st
+    return t
+
+
+def _decode(q, k, v, out, lens=0x200000, lse=0x300000, splits=0):
+    lp = ctypes.cast(ctypes.c_void_p(lens), ctypes.POINTER(ctypes.c_int32)) if lens else None
+    sp = ctypes.cast(ctypes.c_void_p(lse), ctypes.POINTER(ctypes.c_float)) if lse else None
+    return fd.lib.fd_decode_attention(ctypes.byref(q) if q else None, ctypes.byref(k),
+                                      ctypes.byref(v), lp, splits,
+                                      ctypes.byref(out) if out else None, sp, None)
+
+
+def test_decode_rejects_bad_arguments_on_host():
+    B, Hq, Hkv, S, D = 2, 8, 2, 64, 128
+    q, o = _fake([B, Hq, D]), _fake([B, Hq, D])
+    k, v = _fake([B, Hkv, S, D]), _fake([B, Hkv, S, D])
+    assert _decode(None, k, v, o) == fd.FD_ERR_INVALID_ARGUMENT
+    assert _decode(q, k, v, None) == fd.FD_ERR_INVALID_ARGUMENT
+    assert _decode(q, k, v, o, lens=0) == fd.FD_ERR_INVALID_ARGUMENT
+    assert _decode(q, k, v, o, lse=0) == fd.FD_ERR_INVALID_ARGUMENT
+    assert _decode(q, k, v, o, splits=-1) == fd.FD_ERR_INVALID_ARGUMENT
+    # Hq not a multiple of Hkv
+    q3, o3 = _fake([B, 6, D]), _fake([B, 6, D])
+    k4, v4 = _fake([B, 4, S, D]), _fake([B, 4, S, D])
+    assert _decode(q3, k4, v4, o3) == fd.FD_ERR_INVALID_ARGUMENT
+    # head_dim 96 unsupported
+    q96, o96 = _fake([B, Hq, 96]), _fake([B, Hq, 96])
+    k96, v96 = _fake([B, Hkv, S, 96]), _fake([B, Hkv, S, 96])
+    assert _decode(q96, k96, v96, o96) == fd.FD_ERR_UNSUPPORTED
+    # mismatched dtype, mismatched strides, non-contiguous token rows
+    assert _decode(q, _fake([B, Hkv, S, D], fd.FD_F32), _fake([B, Hkv, S, D], fd.FD_F32), o) == 1
+    kt = _fake([B, Hkv, S, D], strides=[Hkv * S * D, S * D, D, 1])
+    vt = _fake([B, Hkv, S, D], strides=[Hkv * S * D * 2, S * D, D, 1])
+    assert _decode(q, kt, vt, o) == fd.FD_ERR_UNSUPPORTED
+    kr = _fake([B, Hkv, S, D], strides=[Hkv * S * 2 * D, S * 2 * D, 2 * D, 1])
+    assert _decode(q, kr, kr, o) == fd.FD_ERR_UNSUPPORTED
+    # last dim not contiguous
+    qs = _fake([B, Hq, D], strides=[Hq * D * 2, D * 2, 2])
+    assert _decode(qs, k, v, o) == fd.FD_ERR_UNSUPPORTED
+    # unaligned data pointer
+    assert _decode(_fake([B, Hq, D], ptr=0x100002), k, v, o) == fd.FD_ERR_UNSUPPORTED
+    # unknown dtype
+    assert _decode(_fake([B, Hq, D], dtype=7), k, v, o) == fd.FD_ERR_UNSUPPORTED
+    # out shape differs
+    assert _decode(q, k, v, _fake([B, Hq + 1, D])) == fd.FD_ERR_INVALID_ARGUMENT
+    # group size above 16 is unsupported
+    q32, o32 = _fake([B, 32, D]), _fake([B, 32, D])
+    k1, v1 = _fake([B, 1, S, D]), _fake([B, 1, S, D])
+    assert _decode(q32, k1, v1, o32) == fd.FD_ERR_UNSUPPORTED
+    # batch 0 is a no-op, before any device work
+    q0, o0 = _fake([0, Hq, D]), _fake([0, Hq, D])
+    k0, v0 = _fake([0, Hkv, S, D]), _fake([0, Hkv, S, D])
+    assert _decode(q0, k0, v0, o0) == fd.FD_OK
+
+
+def test_workspace_bound_covers_plan():
+    for B, hkv, cap, fixed, ctas in [(32, 8, 32768, 0, 148), (1, 8, 32768, 0, 148),
+                                     (4, 40, 16384, 0, 296), (1, 8, 1024, 4, 296),
+                                     (3, 2, 100, 0, 1)]:
+        ws = fd.fd_decode_workspace_bytes(B, hkv * 8, hkv, cap, 128, fixed, ctas)
+        assert ws > 0
+        for lens in ([cap] * B, [0] * B, [1] * B, [cap // 3 + 1] * B):
+            ref = P.decode_plan(lens, hkv, cap, ctas, fixed)
+            # every item's slot and the item list fit the sizes the workspace was laid out for
+            items_bound = (hkv * B * fixed if fixed else
+                           hkv * B + max(P.WAVES * ctas, -(-hkv * B * cap // P.MAX_CHUNK)))
+            assert ref.total_items <= items_bound
