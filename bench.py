@@ -45,6 +45,8 @@ def parse_args():
     ap.add_argument("--workload", type=int, default=3, choices=[1, 2, 3, 4])
     ap.add_argument("--batch", type=int, default=None, help="batch of the long-context workload")
     ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--profile-calls", type=int, default=200,
+                    help="calls timed with per-kernel events after the timed region (0: skip)")
     ap.add_argument("--cpu-seconds", type=float, default=15.0,
                     help="host-time budget of the oracle CPU baseline sample")
     return ap.parse_args()
@@ -229,7 +231,8 @@ def run_reference(args, rank, world):
         "config": {"workload": inp.name},
         "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": cpu_threads(),
                          "kind": "oracle",
-                         "sample": f"per step: {per_step:.2f}s of host time over whole (batch, KV head) groups"},
+                         "sample": f"per step: whole (batch, KV head) groups of the workload in a "
+                                   f"seeded order until {per_step:.2f}s of host time (or all groups)"},
         "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
@@ -291,19 +294,22 @@ def run_fd(args, rank, world, local_rank):
     value = world * alg * args.steps / (ms_max * 1e-3) / 1e9
 
     # ---- per-kernel durations (same calls, with events between the launches) ----
-    nprof = min(args.steps, 200)
-    fd.fd_profile_begin(nprof)
-    for _ in range(nprof):
-        step()
-    torch.cuda.synchronize()
-    prof = fd.fd_profile_end(nprof)
-    plan_ms = statistics.mean(p[0] for p in prof)
-    split_ms = statistics.mean(p[1] for p in prof)
-    comb_ms = statistics.mean(p[2] for p in prof)
+    nprof = min(args.steps, args.profile_calls)
+    prof = [(float("nan"),) * 3]
+    if nprof > 0:
+        fd.fd_profile_begin(nprof)
+        for _ in range(nprof):
+            step()
+        torch.cuda.synchronize()
+        prof = fd.fd_profile_end(nprof)
+    def _mean(i):
+        v = statistics.mean(p[i] for p in prof)
+        return None if v != v else v
+    plan_ms, split_ms, comb_ms = _mean(0), _mean(1), _mean(2)
     peak, peak_kind = measured_peak()
     use_tc = inp.q.dtype == torch.bfloat16 and d == 128 and 2 <= g <= 16
     kfile = "decode_tc.cu" if use_tc else "decode_simt.cu"
-    achieved = alg / (split_ms * 1e-3) / 1e9
+    achieved = alg / (split_ms * 1e-3) / 1e9 if split_ms else None
 
     # ---- end to end: host buffers, copies inside the timed region ----
     e2e = None
@@ -365,11 +371,13 @@ def run_fd(args, rank, world, local_rank):
                        "algorithmic_bytes_per_call": alg, "input_bytes_resident": input_bytes,
                        "l2": l2_policy, "parallelism": f"replicas x{world}"},
             "roofline": {"bound": "hbm", "kernel": kfile.replace(".cu", "_kernel"),
-                         "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
-                         "frac": round(achieved / peak, 4), "peak_kind": f"{peak_kind} copy bandwidth",
+                         "achieved": round(achieved, 1) if achieved else None, "peak": peak,
+                         "unit": "GB/s", "frac": round(achieved / peak, 4) if achieved else None,
+                         "peak_kind": f"{peak_kind} copy bandwidth",
                          "traffic": traffic_from_profiles(kfile, inp.name),
-                         "kernel_ms": {"planner": round(plan_ms, 5), "split": round(split_ms, 5),
-                                       "combine": round(comb_ms, 5)}},
+                         "kernel_ms": {k: (round(v, 5) if v is not None else None) for k, v in
+                                       (("planner", plan_ms), ("split", split_ms),
+                                        ("combine", comb_ms))}},
             "clocks": clocks,
             "e2e": e2e,
             "gpu_launches": 3 * args.steps,

@@ -1,6 +1,7 @@
 """Build the C-ABI library libfd.so in-tree with nvcc for sm_100a.
 
-Usage: python -m split_kv_decode_flashdecoding_b200.build [--force] [-v]
+Usage: python split_kv_decode_flashdecoding_b200/build.py [--force] [-v]
+(run by path: importing the package needs the library already built)
 
 The CUDA runtime is linked statically and the driver entry points the library needs are
 fetched at run time, so the library loads on a machine without a GPU driver (its attention
