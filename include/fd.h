@@ -177,6 +177,35 @@ fd_status fd_chunk_prefill_attention(const fd_tensor* q_chunk, const fd_tensor* 
                                      const int32_t* chunk_lens, fd_tensor* out, float* lse,
                                      void* stream);
 
+/* Size of the device array that holds the scratch of fd_decode_attention_static (64 MiB). */
+#define FD_STATIC_SCRATCH_BYTES (64u * 1024u * 1024u)
+
+/*
+ * fd_decode_attention_static — fd_decode_attention for callers that cannot allocate device memory.
+ *
+ * The pages have no counterpart: this is a deployment variant of the same call. Some callers
+ * cannot call cudaMalloc when they attend: serving engines that hand nearly all HBM to their own
+ * KV-cache pool (a late allocation would fail or fragment it), plugin hosts that only give a
+ * plugin buffers they allocated themselves, and latency-critical loops that cannot afford the
+ * implicit device synchronisation of cudaMalloc / cudaFree. This entry point takes the same
+ * arguments and computes the same result with the same kernels, but keeps its scratch (split plan,
+ * work items, per-split partials) in one file-scope device array of FD_STATIC_SCRATCH_BYTES and
+ * allocates nothing; the caller still passes every input and output.
+ *  - Every GPU that loads the library holds that array until the process exits.
+ *  - The first call on a device looks up the array's device address (cudaGetSymbolAddress) with
+ *    that device current; make that first call before any stream capture begins.
+ *  - All calls share the array and it keeps the last call's contents: calls that overlap on the GPU
+ *    (different streams, or host threads without ordering between their calls) race on it and give
+ *    wrong results. Each call clears, on its stream, the header that must start at zero.
+ *  - A shape whose worst-case scratch (fd_decode_workspace_bytes) exceeds FD_STATIC_SCRATCH_BYTES
+ *    returns FD_ERR_UNSUPPORTED before anything is enqueued.
+ *  - Device status flags of these kernels are not reported by fd_poll_status.
+ */
+fd_status fd_decode_attention_static(const fd_tensor* q, const fd_tensor* k_cache,
+                                     const fd_tensor* v_cache, const int32_t* cache_lens,
+                                     int32_t num_splits, fd_tensor* out, float* lse,
+                                     void* stream);
+
 /* Human-readable name of a status code (static string). */
 const char* fd_status_string(fd_status s);
 

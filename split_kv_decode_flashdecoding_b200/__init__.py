@@ -2,7 +2,7 @@
 
 Argument marshalling only: every step of the attention path runs in the CUDA kernels of
 libfd.so. PyTorch supplies device memory and streams. Importing this package fails loudly when
-libfd.so has not been built (``python -m split_kv_decode_flashdecoding_b200.build``); there is no
+libfd.so has not been built (``python split_kv_decode_flashdecoding_b200/build.py``); there is no
 CPU fallback.
 
 Functions keep the C names:
@@ -23,7 +23,8 @@ from typing import List, Optional, Sequence, Tuple
 import torch
 
 __all__ = [
-    "FdError", "LIB_PATH", "lib", "fd_decode_attention", "fd_chunk_prefill_attention",
+    "FdError", "LIB_PATH", "lib", "fd_decode_attention", "fd_decode_attention_static",
+    "fd_chunk_prefill_attention",
     "fd_split_plan", "fd_split_plan_device", "fd_decode_num_ctas", "fd_decode_workspace_bytes",
     "fd_chunk_workspace_bytes", "fd_reserve_workspace", "fd_poll_status", "fd_profile_begin",
     "fd_profile_end", "fd_shutdown", "fd_status_string", "FD_F32", "FD_BF16",
@@ -61,7 +62,7 @@ class FdError(RuntimeError):
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(
-        f"{LIB_PATH} is missing: build it with `python -m split_kv_decode_flashdecoding_b200.build`"
+        f"{LIB_PATH} is missing: build it with `python split_kv_decode_flashdecoding_b200/build.py`"
         " (there is no fallback implementation)")
 
 lib = ctypes.CDLL(LIB_PATH)
@@ -70,6 +71,7 @@ _TP = ctypes.POINTER(FdTensor)
 # name -> (restype, argtypes); the same names as include/fd.h
 ABI_FUNCTIONS = {
     "fd_decode_attention": (c_i32, [_TP, _TP, _TP, c_i32p, c_i32, _TP, c_f32p, c_vp]),
+    "fd_decode_attention_static": (c_i32, [_TP, _TP, _TP, c_i32p, c_i32, _TP, c_f32p, c_vp]),
     "fd_split_plan": (c_i32, [c_i32p, c_i32, c_i32, c_i32, c_i32, c_i32, c_i32p, c_i32p, c_i32,
                               ctypes.POINTER(FdPlanInfo)]),
     "fd_split_plan_device": (c_i32, [c_i32p, c_i32, c_i32, c_i32, c_i32, c_i32, c_i32p, c_i32p,
@@ -148,6 +150,22 @@ def fd_decode_attention(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.T
                                      int(num_splits), ctypes.byref(_tensor(out)),
                                      _ptr(lse, ctypes.c_float), _stream(stream, q.device))
     _check(st, "fd_decode_attention")
+    return out, lse
+
+
+def fd_decode_attention_static(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
+                               cache_lens: torch.Tensor, num_splits: int, out: torch.Tensor,
+                               lse: torch.Tensor, stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Same as fd_decode_attention, for callers that cannot allocate device memory: the library
+    keeps this call's scratch in a fixed device array (FD_STATIC_SCRATCH_BYTES) and allocates
+    nothing, so `out` and `lse` must be passed in. Calls that overlap on the GPU share that array
+    and race; the first call on a device should come before any stream capture."""
+    with torch.cuda.device(q.device):
+        st = lib.fd_decode_attention_static(
+            ctypes.byref(_tensor(q)), ctypes.byref(_tensor(k_cache)), ctypes.byref(_tensor(v_cache)),
+            _ptr(cache_lens, c_i32), int(num_splits), ctypes.byref(_tensor(out)),
+            _ptr(lse, ctypes.c_float), _stream(stream, q.device))
+    _check(st, "fd_decode_attention_static")
     return out, lse
 
 

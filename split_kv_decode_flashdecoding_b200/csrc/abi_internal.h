@@ -1,0 +1,35 @@
+// Host-side helpers of the C ABI shared by its source files: error reporting, decode-call
+// validation, tensor maps and launch geometry (defined in api.cu).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "../../include/fd.h"
+
+namespace fd_abi {
+
+// Record a formatted message for fd_last_error_message() and return `s`.
+fd_status fail(fd_status s, const char* fmt, ...);
+fd_status cuda_fail(cudaError_t e, const char* what);
+
+struct DecodeShape {
+  int B, hq, hkv, g, d, cap, dtype;
+  bool use_tc;
+  int nctas;
+};
+
+// Validate a decode call's tensors and choose its split kernel.
+fd_status resolve_decode(const fd_tensor* q, const fd_tensor* k, const fd_tensor* v,
+                         const fd_tensor* out, DecodeShape* sh);
+
+// Persistent CTAs of the split kernel on device `dev`.
+int decode_ctas(int dev, bool use_tc);
+
+// bf16 tensor map with 128-byte swizzle; dims / strides innermost first.
+fd_status make_tmap(CUtensorMap* map, const void* base, int rank, const uint64_t* dims,
+                    const uint64_t* strides_bytes, const uint32_t* box, const char* what);
+
+}  // namespace fd_abi

@@ -11,12 +11,14 @@
 #include <utility>
 #include <vector>
 
+#include "abi_internal.h"
 #include "common.cuh"
 #include "internal.h"
 
 using namespace fd;
 
-namespace {
+// Helpers shared with the other C-ABI source files of the library (abi_internal.h).
+namespace fd_abi {
 
 // ---------------------------------------------------------------------------- errors ---------
 thread_local std::string g_last_error;
@@ -183,12 +185,6 @@ fd_status check_tensor(const fd_tensor* t, const char* name, int ndim) {
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 bool stride16(int64_t stride_elems, int dtype) { return (stride_elems * static_cast<int64_t>(elem_size(dtype))) % 16 == 0; }
 
-struct DecodeShape {
-  int B, hq, hkv, g, d, cap, dtype;
-  bool use_tc;
-  int nctas;
-};
-
 fd_status check_kv(const fd_tensor* k, const fd_tensor* v, int dtype, int B, int d) {
   fd_status s;
   if ((s = check_tensor(k, "k_cache", 4)) != FD_OK) return s;
@@ -287,7 +283,9 @@ void end_profile_events(cudaEvent_t* ev, int slot, cudaStream_t stream) {
   if (ev) cudaEventRecord(ev[slot], stream);
 }
 
-}  // namespace
+}  // namespace fd_abi
+
+using namespace fd_abi;
 
 // ================================================================================ ABI ========
 extern "C" {
