@@ -34,10 +34,14 @@ min((s + 1) * chunk_b, len_b)) (the FlashDecoding page's chunk_size rule); trail
 may be empty.
 
 Chunked prefill (``chunk_plan``): a request with chunk_len = 1 is a decode row over
-prefix_len + 1 keys and is planned as above. A request with a longer chunk is cut into query
-tiles of 128 rows; tile t sees at most K_t = min(prefix + min(chunk_len, 128 (t + 1)), S_cap)
-keys, which are cut into n_t = max(1, ceil(K_t / CHUNK_KV_SPLIT)) equal splits the same way.
-Every row of the tile owns n_t partial slots.
+prefix_len + 1 keys and is planned as above (over the decode requests only). A request with a
+longer chunk is cut into query tiles of 128 rows; tile t sees at most
+K_t = min(prefix + min(chunk_len, 128 (t + 1)), S_cap) keys, cut on a fixed grid of
+CHUNK_KV_SPLIT keys: split s = [CHUNK_KV_SPLIT s, min(CHUNK_KV_SPLIT (s + 1), K_t)) for
+s < n_t = max(1, ceil(K_t / CHUNK_KV_SPLIT)). The grid is the same for every tile of a request, so
+the tiles of one head read the same K/V ranges. Every row of a tile owns n_t partial slots. Tile
+items run in the order (request, query head, split, tile): the tiles sharing a split's keys are
+adjacent, so they run at the same time and share those keys in L2.
 """
 
 from __future__ import annotations
@@ -138,15 +142,16 @@ def chunk_plan(prefix_lens: Sequence[int], chunk_lens: Sequence[int], num_q_head
             row_splits.append(dec.splits_per_seq[dec_req.index(b)])
             continue
         p = int(prefix_lens[b])
-        for t in range(_cdiv(c, Q_TILE)):
-            k_t = max(0, min(p + min(c, Q_TILE * (t + 1)), int(cache_capacity)))
-            n_t = max(1, _cdiv(k_t, CHUNK_KV_SPLIT))
-            rows_in_tile = min(Q_TILE, c - Q_TILE * t)
-            row_splits.extend([n_t] * rows_in_tile)
-            for h in range(num_q_heads):
-                for s, (k0, k1) in enumerate(_split_bounds_equal(k_t, n_t)):
-                    tiles.append((b, t, h, s, k0, k1))
-    # longest work first: by key count of the split, descending; ties keep generation order
-    order = sorted(range(len(tiles)), key=lambda i: (-(tiles[i][5] - tiles[i][4]), i))
-    return ChunkPlan(decode=dec, decode_requests=dec_req,
-                     tile_items=[tiles[i] for i in order], row_splits=row_splits)
+        n_tiles = _cdiv(c, Q_TILE)
+        k_t = [max(0, min(p + min(c, Q_TILE * (t + 1)), int(cache_capacity))) for t in range(n_tiles)]
+        n_t = [max(1, _cdiv(k, CHUNK_KV_SPLIT)) for k in k_t]
+        for t in range(n_tiles):
+            row_splits.extend([n_t[t]] * min(Q_TILE, c - Q_TILE * t))
+        for h in range(num_q_heads):
+            for s in range(max(n_t)):
+                for t in range(n_tiles):
+                    if s < n_t[t]:
+                        k0 = min(CHUNK_KV_SPLIT * s, k_t[t])
+                        k1 = min(CHUNK_KV_SPLIT * (s + 1), k_t[t])
+                        tiles.append((b, t, h, s, k0, k1))
+    return ChunkPlan(decode=dec, decode_requests=dec_req, tile_items=tiles, row_splits=row_splits)

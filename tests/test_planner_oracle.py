@@ -114,8 +114,19 @@ def test_chunk_plan_hand_worked():
     cp = P.chunk_plan([5000, 69], [300, 1], 2, 2, 8192, 148)
     assert cp.decode_requests == [1]
     assert cp.decode.splits_per_seq == [1]
-    # tiles: rows 0-127 see <= 5128 keys -> 3 splits; 128-255 -> 5256 -> 3; 256-299 -> 5300 -> 3
+    # tiles see <= 5128, 5256, 5300 keys -> 3 splits each on the 2048-key grid
     assert cp.row_splits == [3] * 300 + [1]
     spans = sorted({(t, s, k0, k1) for (b, t, h, s, k0, k1) in cp.tile_items if t == 0})
-    assert spans == [(0, 0, 0, 1709), (0, 1, 1709, 3418), (0, 2, 3418, 5128)]
+    assert spans == [(0, 0, 0, 2048), (0, 1, 2048, 4096), (0, 2, 4096, 5128)]
     assert len(cp.tile_items) == 3 * 2 * 3
+    # order: head, split, tile
+    assert [(h, s, t) for (b, t, h, s, k0, k1) in cp.tile_items[:4]] == [
+        (0, 0, 0), (0, 0, 1), (0, 0, 2), (0, 1, 0)]
+
+
+def test_chunk_plan_tiles_with_fewer_splits():
+    # a 300-row chunk at prefix 1900: tile 0 sees <= 2028 keys (1 split), tiles 1-2 see more (2)
+    cp = P.chunk_plan([1900], [300], 1, 1, 4096, 148)
+    assert cp.row_splits == [1] * 128 + [2] * 172
+    assert [(t, s, k0, k1) for (b, t, h, s, k0, k1) in cp.tile_items] == [
+        (0, 0, 0, 2028), (1, 0, 0, 2048), (2, 0, 0, 2048), (1, 1, 2048, 2156), (2, 1, 2048, 2200)]
