@@ -168,8 +168,10 @@ fd_status fd_split_plan_device(const int32_t* cache_lens, int32_t batch, int32_t
  *  q_chunk     [T, Hq, D] with T = sum(chunk_lens), packed request by request; D == 128, bf16.
  *  k_cache,    [B, Hkv, S_cap, D] bf16, holding each request's keys/values at
  *  v_cache     [0, prefix_lens[b] + chunk_lens[b]). Same layout rules as fd_decode_attention.
- *  prefix_lens [B] int32 (device), chunk_lens [B] int32 (device, each >= 1, summing to T).
- *              prefix + chunk is clamped to S_cap on the device (status flag).
+ *  prefix_lens [B] int32 (device), chunk_lens [B] int32 (device, each >= 0, summing to T).
+ *              prefix + chunk is clamped to S_cap on the device (status flag). If the chunk
+ *              lengths do not sum to T nothing is computed, `out` / `lse` are left unchanged and
+ *              FD_FLAG_LEN_CLAMPED is raised.
  *  out         [T, Hq, D] bf16 (written); lse [T, Hq] float32 (device, written, natural log).
  */
 fd_status fd_chunk_prefill_attention(const fd_tensor* q_chunk, const fd_tensor* k_cache,
@@ -189,7 +191,7 @@ fd_status fd_chunk_prefill_attention(const fd_tensor* q_chunk, const fd_tensor* 
  * plugin buffers they allocated themselves, and latency-critical loops that cannot afford the
  * implicit device synchronisation of cudaMalloc / cudaFree. This entry point takes the same
  * arguments and computes the same result with the same kernels, but keeps its scratch (split plan,
- * work items, per-split partials) in one file-scope device array of FD_STATIC_SCRATCH_BYTES and
+ * work items, per-split partials, merge counters) in one file-scope device array of FD_STATIC_SCRATCH_BYTES and
  * allocates nothing; the caller still passes every input and output.
  *  - Every GPU that loads the library holds that array until the process exits.
  *  - The first call on a device looks up the array's device address (cudaGetSymbolAddress) with

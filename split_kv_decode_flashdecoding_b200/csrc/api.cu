@@ -247,8 +247,7 @@ int decode_ctas(int dev, bool use_tc) {
 
 size_t decode_ws_bytes(int B, int hq, int hkv, int cap, int d, int fixed, int nctas) {
   const int64_t items = decode_max_items(B, hkv, cap, fixed, nctas);
-  const int64_t slots = (items + hkv - 1) / hkv;
-  return ws_layout(items, 0, B, slots, hq, d).total;
+  return ws_layout(items, 0, B, items, hq, d, hkv).total;
 }
 
 // ---------------------------------------------------------------------------- host planner ---
@@ -372,7 +371,7 @@ fd_status fd_split_plan_device(const int32_t* cache_lens, int32_t batch, int32_t
     return fail(FD_ERR_INVALID_ARGUMENT, "bad plan arguments");
   if (items_dev && items_capacity < 0) return fail(FD_ERR_INVALID_ARGUMENT, "items_capacity must be >= 0");
   const int64_t items = decode_max_items(batch, num_kv_heads, cache_capacity, num_splits, num_ctas);
-  const WsLayout L = ws_layout(items, 0, batch, 0, 1, 1);
+  const WsLayout L = ws_layout(items, 0, batch, 0, 1, 1, num_kv_heads);
   void* ws = nullptr;
   fd_status s = get_workspace(stream, L.total, &ws);
   if (s != FD_OK) return s;
@@ -390,6 +389,7 @@ fd_status fd_split_plan_device(const int32_t* cache_lens, int32_t batch, int32_t
   pp.items = reinterpret_cast<DecodeItem*>(base + L.dec_items);
   pp.row_nsplit = reinterpret_cast<int32_t*>(base + L.row_nsplit);
   pp.row_base = reinterpret_cast<int32_t*>(base + L.row_base);
+  pp.arrivals = reinterpret_cast<int32_t*>(base + L.arrivals);
   pp.out_splits = splits_per_seq_dev;
   pp.out_items = items_dev;
   pp.out_cap = items_dev ? items_capacity : 0;
@@ -416,8 +416,8 @@ fd_status fd_decode_attention(const fd_tensor* q, const fd_tensor* k_cache,
   if (nctas < 1) return fail(FD_ERR_CUDA, "no multiprocessors reported for device %d", dev);
 
   const int64_t max_items = decode_max_items(sh.B, sh.hkv, sh.cap, num_splits, nctas);
-  const int64_t max_slots = (max_items + sh.hkv - 1) / sh.hkv;
-  const WsLayout L = ws_layout(max_items, 0, sh.B, max_slots, sh.hq, sh.d);
+  const int64_t max_slots = max_items;  // one partial slot (G heads) per split item
+  const WsLayout L = ws_layout(max_items, 0, sh.B, max_slots, sh.hq, sh.d, sh.hkv);
   void* ws = nullptr;
   if ((s = get_workspace(stream, L.total, &ws)) != FD_OK) return s;
   char* base = static_cast<char*>(ws);
@@ -427,6 +427,7 @@ fd_status fd_decode_attention(const fd_tensor* q, const fd_tensor* k_cache,
   int32_t* row_base = reinterpret_cast<int32_t*>(base + L.row_base);
   float* part_o = reinterpret_cast<float*>(base + L.part_o);
   float* part_lse = reinterpret_cast<float*>(base + L.part_lse);
+  int32_t* arrivals = reinterpret_cast<int32_t*>(base + L.arrivals);
 
   DecodeParams dp{};
   dp.q = q->data;
@@ -453,6 +454,7 @@ fd_status fd_decode_attention(const fd_tensor* q, const fd_tensor* k_cache,
   dp.row_base = row_base;
   dp.part_o = part_o;
   dp.part_lse = part_lse;
+  dp.arrivals = arrivals;
 
   CUtensorMap tq, tk, tv;
   if (sh.use_tc) {
@@ -481,6 +483,7 @@ fd_status fd_decode_attention(const fd_tensor* q, const fd_tensor* k_cache,
   pp.items = items;
   pp.row_nsplit = row_nsplit;
   pp.row_base = row_base;
+  pp.arrivals = arrivals;
 
   CombineParams cp{};
   cp.row_nsplit = row_nsplit;
@@ -493,8 +496,11 @@ fd_status fd_decode_attention(const fd_tensor* q, const fd_tensor* k_cache,
   cp.lse = lse;
   cp.rows = sh.B;
   cp.hq = sh.hq;
+  cp.hkv = sh.hkv;
+  cp.g = sh.g;
   cp.d = sh.d;
   cp.dtype = sh.dtype;
+
 
   cudaEvent_t* ev = prof_next();
   end_profile_events(ev, 0, stream);
@@ -506,7 +512,9 @@ fd_status fd_decode_attention(const fd_tensor* q, const fd_tensor* k_cache,
     FD_CUDA(launch_decode_simt(dp, sh.dtype, nctas, stream), "split kernel launch");
   }
   end_profile_events(ev, 2, stream);
-  FD_CUDA(launch_combine(cp, stream), "combine kernel launch");
+  // the CUDA-core kernel merges each group's partials itself; the tensor-core kernel leaves them
+  // to the combine kernel
+  if (sh.use_tc) FD_CUDA(launch_combine(cp, stream), "combine kernel launch");
   end_profile_events(ev, 3, stream);
   return FD_OK;
 }
@@ -514,18 +522,178 @@ fd_status fd_decode_attention(const fd_tensor* q, const fd_tensor* k_cache,
 fd_status fd_chunk_prefill_attention(const fd_tensor* q_chunk, const fd_tensor* k_cache,
                                      const fd_tensor* v_cache, const int32_t* prefix_lens,
                                      const int32_t* chunk_lens, fd_tensor* out, float* lse,
-                                     void* stream) {
-  (void)q_chunk; (void)k_cache; (void)v_cache; (void)prefix_lens; (void)chunk_lens;
-  (void)out; (void)lse; (void)stream;
-  return fail(FD_ERR_UNSUPPORTED, "chunked prefill is not built yet");
+                                     void* stream_) {
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+  fd_status s;
+  if ((s = check_q_out(q_chunk, out, "q_chunk")) != FD_OK) return s;
+  const int T = static_cast<int>(q_chunk->shape[0]);
+  const int hq = static_cast<int>(q_chunk->shape[1]);
+  const int d = static_cast<int>(q_chunk->shape[2]);
+  if (q_chunk->dtype != FD_BF16) return fail(FD_ERR_UNSUPPORTED, "chunked prefill needs bf16 tensors");
+  if (d != 128) return fail(FD_ERR_UNSUPPORTED, "chunked prefill supports head_dim 128, got %d", d);
+  if (!k_cache) return fail(FD_ERR_INVALID_ARGUMENT, "k_cache is NULL");
+  const int B = static_cast<int>(k_cache->shape[0]);
+  if ((s = check_kv(k_cache, v_cache, FD_BF16, B, d)) != FD_OK) return s;
+  const int hkv = static_cast<int>(k_cache->shape[1]);
+  const int cap = static_cast<int>(k_cache->shape[2]);
+  if (hq < 1 || hq % hkv != 0)
+    return fail(FD_ERR_INVALID_ARGUMENT, "q heads (%d) must be a positive multiple of KV heads (%d)", hq, hkv);
+  const int g = hq / hkv;
+  if (g > 16) return fail(FD_ERR_UNSUPPORTED, "group size %d above 16", g);
+  if (B > kMaxPlanBatch) return fail(FD_ERR_UNSUPPORTED, "batch %d exceeds %d", B, kMaxPlanBatch);
+  if (T == 0) return FD_OK;
+  if (B == 0) return fail(FD_ERR_INVALID_ARGUMENT, "q_chunk has %d rows but the cache has no request", T);
+  if (!prefix_lens || !chunk_lens) return fail(FD_ERR_INVALID_ARGUMENT, "prefix_lens / chunk_lens is NULL");
+  if (!lse) return fail(FD_ERR_INVALID_ARGUMENT, "lse is NULL");
+  int dev = 0;
+  FD_CUDA(cudaGetDevice(&dev), "cudaGetDevice");
+  const bool dec_tc = g >= 2;  // decode rows of a group >= 2 use the tensor-core decode kernel
+  const int dec_ctas = decode_ctas(dev, dec_tc);
+  const int tile_ctas = sm_count(dev);
+  if (dec_ctas < 1 || tile_ctas < 1) return fail(FD_ERR_CUDA, "no multiprocessors reported for device %d", dev);
+
+  const int64_t max_dec = decode_max_items(B, hkv, cap, 0, dec_ctas);
+  const int64_t max_tiles = chunk_max_tile_items(B, T, hq, cap);
+  const int64_t max_slots = chunk_max_slots(B, T, hkv, cap, dec_ctas);
+  const WsLayout L = ws_layout(max_dec, max_tiles, static_cast<int64_t>(T) + 1, max_slots, hq, d, hkv);
+  void* ws = nullptr;
+  if ((s = get_workspace(stream, L.total, &ws)) != FD_OK) return s;
+  char* base = static_cast<char*>(ws);
+  WsHeader* hdr = reinterpret_cast<WsHeader*>(base);
+  DecodeItem* items = reinterpret_cast<DecodeItem*>(base + L.dec_items);
+  TileItem* tiles = reinterpret_cast<TileItem*>(base + L.tile_items);
+  int32_t* row_nsplit = reinterpret_cast<int32_t*>(base + L.row_nsplit);
+  int32_t* row_base = reinterpret_cast<int32_t*>(base + L.row_base);
+  int32_t* arrivals = reinterpret_cast<int32_t*>(base + L.arrivals);
+  float* part_o = reinterpret_cast<float*>(base + L.part_o);
+  float* part_lse = reinterpret_cast<float*>(base + L.part_lse);
+  const float scale_log2 = static_cast<float>(1.0 / std::sqrt(static_cast<double>(d)) * 1.4426950408889634);
+
+  PlanParams pp{};
+  pp.lens = prefix_lens;
+  pp.chunk_lens = chunk_lens;
+  pp.B = B;
+  pp.hkv = hkv;
+  pp.hq = hq;
+  pp.cap = cap;
+  pp.nctas = dec_ctas;
+  pp.max_dec_items = max_dec;
+  pp.max_tile_items = max_tiles;
+  pp.hdr = hdr;
+  pp.items = items;
+  pp.tiles = tiles;
+  pp.row_nsplit = row_nsplit;
+  pp.row_base = row_base;
+  pp.arrivals = arrivals;
+  pp.total_rows = T;
+  pp.decode_merged_in_kernel = dec_tc ? 0 : 1;
+
+  DecodeParams dp{};
+  dp.q = q_chunk->data;
+  dp.q_sr = q_chunk->stride[0];
+  dp.q_sh = q_chunk->stride[1];
+  dp.k = k_cache->data;
+  dp.v = v_cache->data;
+  dp.kv_sb = k_cache->stride[0];
+  dp.kv_sh = k_cache->stride[1];
+  dp.out = out->data;
+  dp.o_sr = out->stride[0];
+  dp.o_sh = out->stride[1];
+  dp.lse = lse;
+  dp.hq = hq;
+  dp.hkv = hkv;
+  dp.g = g;
+  dp.d = d;
+  dp.cap = cap;
+  dp.q_box_rows = std::min(16, hq);
+  dp.kv_box_rows = std::min(128, cap);
+  dp.scale_log2 = scale_log2;
+  dp.hdr = hdr;
+  dp.items = items;
+  dp.row_base = row_base;
+  dp.part_o = part_o;
+  dp.part_lse = part_lse;
+  dp.arrivals = arrivals;
+
+  TileParams tp{};
+  tp.q = q_chunk->data;
+  tp.q_sr = q_chunk->stride[0];
+  tp.q_sh = q_chunk->stride[1];
+  tp.out = out->data;
+  tp.o_sr = out->stride[0];
+  tp.o_sh = out->stride[1];
+  tp.lse = lse;
+  tp.hq = hq;
+  tp.hkv = hkv;
+  tp.g = g;
+  tp.d = d;
+  tp.cap = cap;
+  tp.q_box_rows = std::min(128, T);
+  tp.kv_box_rows = std::min(128, cap);
+  tp.scale_log2 = scale_log2;
+  tp.hdr = hdr;
+  tp.tiles = tiles;
+  tp.part_o = part_o;
+  tp.part_lse = part_lse;
+
+  CombineParams cp{};
+  cp.row_nsplit = row_nsplit;
+  cp.row_base = row_base;
+  cp.part_o = part_o;
+  cp.part_lse = part_lse;
+  cp.out = out->data;
+  cp.o_sr = out->stride[0];
+  cp.o_sh = out->stride[1];
+  cp.lse = lse;
+  cp.rows = T;
+  cp.hq = hq;
+  cp.hkv = hkv;
+  cp.g = g;
+  cp.d = d;
+  cp.dtype = FD_BF16;
+
+  // tensor maps: q as (D, Hq, T); caches as (D, S_cap, Hkv, B)
+  CUtensorMap tq_dec, tq_tile, tk, tv;
+  const uint64_t qd[3] = {static_cast<uint64_t>(d), static_cast<uint64_t>(hq), static_cast<uint64_t>(T)};
+  const uint64_t qs[2] = {static_cast<uint64_t>(q_chunk->stride[1]) * 2, static_cast<uint64_t>(q_chunk->stride[0]) * 2};
+  const uint32_t qb_dec[3] = {64, static_cast<uint32_t>(dp.q_box_rows), 1};
+  const uint32_t qb_tile[3] = {64, 1, static_cast<uint32_t>(tp.q_box_rows)};
+  if ((s = make_tmap(&tq_tile, q_chunk->data, 3, qd, qs, qb_tile, "q_chunk")) != FD_OK) return s;
+  const uint64_t kd[4] = {static_cast<uint64_t>(d), static_cast<uint64_t>(cap), static_cast<uint64_t>(hkv), static_cast<uint64_t>(B)};
+  const uint64_t ks[3] = {static_cast<uint64_t>(k_cache->stride[2]) * 2, static_cast<uint64_t>(k_cache->stride[1]) * 2,
+                          static_cast<uint64_t>(k_cache->stride[0]) * 2};
+  const uint32_t kb[4] = {64, static_cast<uint32_t>(dp.kv_box_rows), 1, 1};
+  if ((s = make_tmap(&tk, k_cache->data, 4, kd, ks, kb, "k_cache")) != FD_OK) return s;
+  if ((s = make_tmap(&tv, v_cache->data, 4, kd, ks, kb, "v_cache")) != FD_OK) return s;
+  if (dec_tc && (s = make_tmap(&tq_dec, q_chunk->data, 3, qd, qs, qb_dec, "q_chunk (decode rows)")) != FD_OK) return s;
+
+  cudaEvent_t* ev = prof_next();
+  end_profile_events(ev, 0, stream);
+  FD_CUDA(launch_plan_chunk(pp, stream), "chunk plan kernel launch");
+  end_profile_events(ev, 1, stream);
+  if (dec_tc) {
+    FD_CUDA(launch_decode_tc(dp, tq_dec, tk, tv, dec_ctas, stream), "decode-row split kernel launch");
+  } else {
+    FD_CUDA(launch_decode_simt(dp, FD_BF16, dec_ctas, stream), "decode-row split kernel launch");
+  }
+  FD_CUDA(launch_chunk_tc(tp, tq_tile, tk, tv, tile_ctas, stream), "chunk tile kernel launch");
+  end_profile_events(ev, 2, stream);
+  FD_CUDA(launch_combine(cp, stream), "combine kernel launch");
+  end_profile_events(ev, 3, stream);
+  return FD_OK;
 }
 
 size_t fd_chunk_workspace_bytes(int32_t batch, int32_t total_rows, int32_t num_q_heads,
                                 int32_t num_kv_heads, int32_t cache_capacity, int32_t head_dim,
                                 int32_t num_ctas) {
-  (void)batch; (void)total_rows; (void)num_q_heads; (void)num_kv_heads; (void)cache_capacity;
-  (void)head_dim; (void)num_ctas;
-  return 0;
+  if (batch < 0 || total_rows < 0 || num_q_heads < 1 || num_kv_heads < 1 || cache_capacity < 0 ||
+      head_dim < 1 || num_ctas < 1)
+    return 0;
+  const int64_t max_dec = decode_max_items(batch, num_kv_heads, cache_capacity, 0, num_ctas);
+  const int64_t max_tiles = chunk_max_tile_items(batch, total_rows, num_q_heads, cache_capacity);
+  const int64_t max_slots = chunk_max_slots(batch, total_rows, num_kv_heads, cache_capacity, num_ctas);
+  return ws_layout(max_dec, max_tiles, static_cast<int64_t>(total_rows) + 1, max_slots,
+                   num_q_heads, head_dim, num_kv_heads).total;
 }
 
 fd_status fd_reserve_workspace(size_t bytes, void* stream_) {

@@ -11,6 +11,12 @@
 // fp32, so no term underflows unless it is negligible. Splits with LSE_s = -inf (no visible key)
 // get weight 0; a row whose splits are all empty gets O = 0 and LSE = -inf. The merge order is
 // fixed (split 0 first), so results are bitwise reproducible.
+//
+// Partials of one (row, KV head) group are consecutive slots of G query heads each:
+// slot = row_base[row] * Hkv + h * n_row + split, O at [slot][g][d], LSE at [slot][g]. The K/V
+// stream is loaded with an L2 evict-first policy, so these partials are normally still in L2.
+// Launched with programmatic dependent launch: the CTAs become resident while the split kernel
+// runs and wait for its completion before reading anything.
 #include "common.cuh"
 #include "internal.h"
 
@@ -19,10 +25,12 @@ namespace fd {
 namespace {
 
 constexpr int kCombineWarps = 8;
+constexpr int kBatch = 8;  // splits whose loads are in flight together
 
 template <typename T, int D>
 __global__ void __launch_bounds__(kCombineWarps * 32) combine_kernel(CombineParams p) {
   constexpr int kVec = D / 32;  // elements per lane
+  pdl_wait_prerequisites();
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int64_t pair = static_cast<int64_t>(blockIdx.x) * kCombineWarps + warp;
@@ -31,10 +39,15 @@ __global__ void __launch_bounds__(kCombineWarps * 32) combine_kernel(CombinePara
   const int hq = static_cast<int>(pair - static_cast<int64_t>(row) * p.hq);
   const int n = p.row_nsplit[row];
   if (n <= 1) return;  // single split: the split kernel wrote the output directly
-  const int64_t base = p.row_base[row];
+  const int h = hq / p.g, g = hq - h * p.g;
+  const int64_t slot0 = static_cast<int64_t>(p.row_base[row]) * p.hkv + static_cast<int64_t>(h) * n;
+  const float* lse_base = p.part_lse + slot0 * p.g + g;
+  const float* o_base = p.part_o + (slot0 * p.g + g) * D + lane * kVec;
+  const int64_t lse_step = p.g;
+  const int64_t o_step = static_cast<int64_t>(p.g) * D;
 
   float mx = -INFINITY;
-  for (int s = lane; s < n; s += 32) mx = fmaxf(mx, p.part_lse[(base + s) * p.hq + hq]);
+  for (int s = lane; s < n; s += 32) mx = fmaxf(mx, lse_base[s * lse_step]);
   mx = warp_max_f32(mx);
 
   float acc[kVec];
@@ -42,21 +55,33 @@ __global__ void __launch_bounds__(kCombineWarps * 32) combine_kernel(CombinePara
   for (int e = 0; e < kVec; ++e) acc[e] = 0.f;
   float wsum = 0.f;
   if (mx != -INFINITY) {
-    for (int s = 0; s < n; ++s) {
-      const int64_t slot = base + s;
-      const float l = p.part_lse[slot * p.hq + hq];
-      const float w = fast_exp2(l - mx);  // 0 for l = -inf
-      wsum += w;
-      const float* o = p.part_o + (slot * p.hq + hq) * D + lane * kVec;
-      if (kVec == 4) {
-        const float4 x = *reinterpret_cast<const float4*>(o);
-        acc[0] = fmaf(w, x.x, acc[0]);
-        acc[1] = fmaf(w, x.y, acc[1]);
-        acc[2] = fmaf(w, x.z, acc[2]);
-        acc[3] = fmaf(w, x.w, acc[3]);
-      } else {
+    for (int s0 = 0; s0 < n; s0 += kBatch) {
+      float l[kBatch];
+      float x[kBatch][kVec];
 #pragma unroll
-        for (int e = 0; e < kVec; ++e) acc[e] = fmaf(w, o[e], acc[e]);
+      for (int j = 0; j < kBatch; ++j) {
+        const int s = s0 + j;
+        l[j] = -INFINITY;
+#pragma unroll
+        for (int e = 0; e < kVec; ++e) x[j][e] = 0.f;
+        if (s < n) {
+          l[j] = lse_base[s * lse_step];
+          const float* o = o_base + s * o_step;
+          if constexpr (kVec == 4) {
+            const float4 v = *reinterpret_cast<const float4*>(o);
+            x[j][0] = v.x; x[j][1] = v.y; x[j][2] = v.z; x[j][3] = v.w;
+          } else {
+            const float2 v = *reinterpret_cast<const float2*>(o);
+            x[j][0] = v.x; x[j][1] = v.y;
+          }
+        }
+      }
+#pragma unroll
+      for (int j = 0; j < kBatch; ++j) {
+        const float w = fast_exp2(l[j] - mx);  // 0 for l = -inf
+        wsum += w;
+#pragma unroll
+        for (int e = 0; e < kVec; ++e) acc[e] = fmaf(w, x[j][e], acc[e]);
       }
     }
   }
@@ -68,20 +93,32 @@ __global__ void __launch_bounds__(kCombineWarps * 32) combine_kernel(CombinePara
     p.lse[static_cast<int64_t>(row) * p.hq + hq] = wsum > 0.f ? (mx + log2f(wsum)) * kLn2 : -INFINITY;
 }
 
+template <typename T, int D>
+cudaError_t launch_combine_t(const CombineParams& p, unsigned grid, cudaStream_t stream) {
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kCombineWarps * 32);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, combine_kernel<T, D>, p);
+}
+
 }  // namespace
 
 cudaError_t launch_combine(const CombineParams& p, cudaStream_t stream) {
   const int64_t pairs = static_cast<int64_t>(p.rows) * p.hq;
   if (pairs == 0) return cudaSuccess;
   const unsigned grid = static_cast<unsigned>((pairs + kCombineWarps - 1) / kCombineWarps);
-  if (p.dtype == FD_F32) {
-    if (p.d == 64) combine_kernel<float, 64><<<grid, kCombineWarps * 32, 0, stream>>>(p);
-    else combine_kernel<float, 128><<<grid, kCombineWarps * 32, 0, stream>>>(p);
-  } else {
-    if (p.d == 64) combine_kernel<__nv_bfloat16, 64><<<grid, kCombineWarps * 32, 0, stream>>>(p);
-    else combine_kernel<__nv_bfloat16, 128><<<grid, kCombineWarps * 32, 0, stream>>>(p);
-  }
-  return cudaGetLastError();
+  if (p.dtype == FD_F32)
+    return p.d == 64 ? launch_combine_t<float, 64>(p, grid, stream)
+                     : launch_combine_t<float, 128>(p, grid, stream);
+  return p.d == 64 ? launch_combine_t<__nv_bfloat16, 64>(p, grid, stream)
+                   : launch_combine_t<__nv_bfloat16, 128>(p, grid, stream);
 }
 
 }  // namespace fd

@@ -128,6 +128,33 @@ __device__ __forceinline__ void tma_load_4d(void* dst, const CUtensorMap* map, u
       : "memory");
 }
 
+// L2 policy for data read exactly once (the K/V stream): evict it first, so that it does not
+// push out the partial results and query rows that are read again soon.
+__device__ __forceinline__ uint64_t l2_evict_first_policy() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+
+__device__ __forceinline__ void bulk_load_stream(void* dst, const void* src, uint32_t bytes,
+                                                 uint64_t* bar, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1], %2, [%3], %4;" ::"r"(smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar)), "l"(policy)
+      : "memory");
+}
+
+__device__ __forceinline__ void tma_load_4d_stream(void* dst, const CUtensorMap* map,
+                                                   uint64_t* bar, int32_t c0, int32_t c1,
+                                                   int32_t c2, int32_t c3, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      ".L2::cache_hint [%0], [%1, {%3, %4, %5, %6}], [%2], %7;" ::"r"(smem_u32(dst)),
+      "l"(map), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "l"(policy)
+      : "memory");
+}
+
 __device__ __forceinline__ void prefetch_tensor_map(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(map) : "memory");
 }
@@ -257,6 +284,17 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool a_mn, b
          (static_cast<uint32_t>(M >> 4) << 24);
 }
 
+// ---- programmatic dependent launch ---------------------------------------------------------------
+
+// Let the next kernel of the stream (launched with programmatic stream serialization) start.
+__device__ __forceinline__ void pdl_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+// Wait until the previous kernel of the stream has completed and its writes are visible.
+__device__ __forceinline__ void pdl_wait_prerequisites() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
 // ---- numerics -------------------------------------------------------------------------------
 
 // 2^x with the hardware approximation (relative error ~2^-22); ex2(-inf) = 0.
@@ -301,6 +339,108 @@ __device__ __forceinline__ float from_f32<float>(float x) {
 template <>
 __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) {
   return __float2bfloat16_rn(x);
+}
+
+// ---- in-kernel LSE merge of the splits of one (row, KV head) group ------------------------------
+
+// Where split partials live and where merged results go.
+struct MergeTarget {
+  const float* part_o;   // [slots][G][D] fp32, the slots of one group consecutive
+  const float* part_lse; // [slots][G] base-2 log-sum-exp
+  int32_t* arrivals;     // [rows][Hkv] splits completed so far in this call
+  void* out;             // [rows][Hq][D]
+  int64_t o_sr, o_sh;
+  float* lse;            // [rows][Hq] natural log
+  int32_t hq, hkv, g, d;
+};
+
+constexpr int kMergeThreads = 128;  // the role group that writes partials and merges
+constexpr int kMergeLseCap = 512;   // floats of shared memory holding one chunk of split LSEs
+
+// Called by the kMergeThreads threads of named barrier `bar` right after they stored this CTA's
+// partial (O_s, LSE_s) of one split of group (row, h). The split is counted on a device-scope
+// arrival counter; the CTA that completes the group's last split merges all of its partials,
+//   M = max_s LSE_s;  w_s = 2^(LSE_s - M);  O = sum_s w_s O_s / sum_s w_s;  LSE = M + log2 sum_s w_s
+// (the merge of "大模型推理加速FlashDecoding算法原理与多GPU并行解码实战",
+// "多GPU张量并行扩展下的FlashDecoding实现", with the per-split sums folded into w_s), in a fixed
+// split order, while the partials are still in L2. Splits whose LSE is -inf weigh nothing; a group
+// with no visible key gets O = 0 and LSE = -inf. EPT = elements of the G x D output per thread.
+template <typename T, int EPT>
+__device__ __forceinline__ void finish_split_and_merge(const MergeTarget& t, int row, int h,
+                                                       int nsplit, int64_t slot0, int tid,
+                                                       int bar, volatile int* s_flag,
+                                                       float* s_lse) {
+  __threadfence();  // this thread's partial stores, visible device-wide before the count
+  named_bar_sync(bar, kMergeThreads);
+  if (tid == 0) *s_flag = atomicAdd(&t.arrivals[row * t.hkv + h], 1);
+  named_bar_sync(bar, kMergeThreads);
+  if (*s_flag != nsplit - 1) return;  // the same value for every thread of the group
+  __threadfence();
+  const int G = t.g, D = t.d, GD = G * D;
+  float acc[EPT], wsum[EPT], mx[EPT];
+#pragma unroll
+  for (int k = 0; k < EPT; ++k) { acc[k] = 0.f; wsum[k] = 0.f; mx[k] = -INFINITY; }
+  const int chunk = kMergeLseCap / G;  // splits whose LSEs fit the shared buffer
+  for (int c0 = 0; c0 < nsplit; c0 += chunk) {
+    const int cn = min(chunk, nsplit - c0);
+    const float* lsrc = t.part_lse + (slot0 + c0) * G;
+    for (int i = tid; i < cn * G; i += kMergeThreads) s_lse[i] = __ldcg(lsrc + i);
+    named_bar_sync(bar, kMergeThreads);
+    // running maximum per element's head, rescaling what was accumulated so far
+#pragma unroll
+    for (int k = 0; k < EPT; ++k) {
+      const int e = tid + k * kMergeThreads;
+      if (e < GD) {
+        const int g = e / D;
+        float cm = -INFINITY;
+        for (int s = 0; s < cn; ++s) cm = fmaxf(cm, s_lse[s * G + g]);
+        const float nm = fmaxf(mx[k], cm);
+        const float sc = (nm == -INFINITY) ? 1.f : fast_exp2(mx[k] - nm);
+        acc[k] *= sc;
+        wsum[k] *= sc;
+        mx[k] = nm;
+      }
+    }
+    // weighted sum, kB splits per round with all their loads (kB x EPT <= 32) in flight
+    constexpr int kB = EPT >= 32 ? 1 : 32 / EPT;
+    const float* osrc = t.part_o + (slot0 + c0) * static_cast<int64_t>(GD);
+    for (int s0 = 0; s0 < cn; s0 += kB) {
+      float x[kB][EPT];
+#pragma unroll
+      for (int j = 0; j < kB; ++j)
+#pragma unroll
+        for (int k = 0; k < EPT; ++k) {
+          const int e = tid + k * kMergeThreads;
+          x[j][k] = (s0 + j < cn && e < GD) ? __ldcg(osrc + static_cast<int64_t>(s0 + j) * GD + e) : 0.f;
+        }
+#pragma unroll
+      for (int j = 0; j < kB; ++j)
+#pragma unroll
+        for (int k = 0; k < EPT; ++k) {
+          const int e = tid + k * kMergeThreads;
+          if (s0 + j < cn && e < GD && mx[k] != -INFINITY) {
+            const float w = fast_exp2(s_lse[(s0 + j) * G + e / D] - mx[k]);
+            acc[k] = fmaf(w, x[j][k], acc[k]);
+            wsum[k] += w;
+          }
+        }
+    }
+    named_bar_sync(bar, kMergeThreads);  // s_lse is reused by the next chunk
+  }
+#pragma unroll
+  for (int k = 0; k < EPT; ++k) {
+    const int e = tid + k * kMergeThreads;
+    if (e < GD) {
+      const int g = e / D, d = e - g * D;
+      const int hq = h * G + g;
+      T* o = static_cast<T*>(t.out) + static_cast<int64_t>(row) * t.o_sr + static_cast<int64_t>(hq) * t.o_sh;
+      o[d] = from_f32<T>(wsum[k] > 0.f ? acc[k] / wsum[k] : 0.f);
+      if (d == 0)
+        t.lse[static_cast<int64_t>(row) * t.hq + hq] =
+            wsum[k] > 0.f ? (mx[k] + log2f(wsum[k])) * kLn2 : -INFINITY;
+    }
+  }
+  if (tid == 0) t.arrivals[row * t.hkv + h] = 0;  // ready for the next call on this workspace
 }
 
 }  // namespace fd

@@ -44,12 +44,16 @@ struct __align__(128) SimtSmem {
   using C = SimtCfg<T, D, GP>;
   T k[kSimtStages][C::kTile * D];
   T v[kSimtStages][C::kTile * D];
+  T qs[kSimtStages][GP * D];       // the item's query rows, loaded with its first tile
   float sc[2][GP][C::kTile];       // scores, then probabilities, of the current tile
   float wmax[2][kSimtConsumerWarps][GP];
   float red[kSimtConsumerWarps][GP][D];
   float lsum[GP * C::kTile > kSimtConsumers ? GP * C::kTile : kSimtConsumers];
   float lfin[GP];
+  float mlse[kMergeLseCap];        // split LSEs of a group being merged
+  int mflag;
   int32_t meta[kSimtStages][4];    // item index (-1: stop), tile start, valid keys, flags
+  DecodeItem item[kSimtStages];    // descriptor of the stage's item
   uint64_t full[kSimtStages];
   uint64_t empty[kSimtStages];
   int abort_flag;
@@ -103,23 +107,35 @@ __global__ void __launch_bounds__(kSimtThreads) decode_simt_kernel(DecodeParams 
   }
   __syncthreads();
   const WaitCtx ctx{&S.abort_flag, &p.hdr->status};
+  // the barrier set-up above overlapped the planner (programmatic dependent launch)
+  pdl_wait_prerequisites();
+  pdl_launch_dependents();
   const T* kbase = static_cast<const T*>(p.k);
   const T* vbase = static_cast<const T*>(p.v);
+  const T* qbase = static_cast<const T*>(p.q);
 
   if (warp == kSimtConsumerWarps) {
     // ---------------- producer: one thread streams K/V tiles ----------------
     if (lane != 0) return;
     const int n_items = *reinterpret_cast<volatile int32_t*>(&p.hdr->num_dec_items);
+    const uint64_t pol = l2_evict_first_policy();
     uint32_t J = 0;
     bool ok = true;
-    while (ok) {
-      const int idx = atomicAdd(&p.hdr->dec_counter, 1);
-      if (idx >= n_items) break;
-      const DecodeItem it = p.items[idx];
+    // The next item is claimed three tiles before the current one ends and its descriptor is
+    // read one tile later: both global round trips then overlap the ring's lookahead instead of
+    // stalling the stream at every item boundary.
+    int idx = atomicAdd(&p.hdr->dec_counter, 1);
+    DecodeItem it{};
+    if (idx < n_items) it = p.items[idx];
+    while (ok && idx < n_items) {
+      int nidx = n_items;
+      DecodeItem nit{};
       const int len = it.t1 - it.t0;
       const int ntile = len > 0 ? (len + C::kTile - 1) / C::kTile : 1;
+      const int claim_j = max(0, ntile - 3), read_j = max(0, ntile - 2);
       const int64_t off = static_cast<int64_t>(it.b) * p.kv_sb + static_cast<int64_t>(it.h) * p.kv_sh;
       for (int j = 0; j < ntile; ++j, ++J) {
+        if (j == claim_j) nidx = atomicAdd(&p.hdr->dec_counter, 1);
         const int st = J % kSimtStages;
         if (!mbar_wait(&S.empty[st], ((J / kSimtStages) & 1u) ^ 1u, ctx)) { ok = false; break; }
         const int t = it.t0 + j * C::kTile;
@@ -128,15 +144,28 @@ __global__ void __launch_bounds__(kSimtThreads) decode_simt_kernel(DecodeParams 
         S.meta[st][1] = t;
         S.meta[st][2] = valid;
         S.meta[st][3] = (j == 0 ? kFirstTile : 0) | (j == ntile - 1 ? kLastTile : 0);
-        if (valid > 0) {
-          const uint32_t bytes = static_cast<uint32_t>(valid) * D * sizeof(T);
-          mbar_arrive_expect_tx(&S.full[st], 2u * bytes);
-          bulk_load(S.k[st], kbase + off + static_cast<int64_t>(t) * D, bytes, &S.full[st]);
-          bulk_load(S.v[st], vbase + off + static_cast<int64_t>(t) * D, bytes, &S.full[st]);
+        S.item[st] = it;
+        const uint32_t bytes = static_cast<uint32_t>(valid) * D * sizeof(T);
+        const uint32_t qbytes = j == 0 ? static_cast<uint32_t>(p.g) * D * sizeof(T) : 0u;
+        if (bytes + qbytes > 0) {
+          mbar_arrive_expect_tx(&S.full[st], 2u * bytes + qbytes);
+          if (qbytes) {
+            const T* qrow = qbase + static_cast<int64_t>(it.row) * p.q_sr;
+            for (int g = 0; g < p.g; ++g)
+              bulk_load(S.qs[st] + g * D, qrow + static_cast<int64_t>(it.h * p.g + g) * p.q_sh,
+                        D * sizeof(T), &S.full[st]);
+          }
+          if (bytes) {
+            bulk_load(S.k[st], kbase + off + static_cast<int64_t>(t) * D, bytes, &S.full[st]);
+            bulk_load(S.v[st], vbase + off + static_cast<int64_t>(t) * D, bytes, &S.full[st]);
+          }
         } else {
           mbar_arrive(&S.full[st]);
         }
+        if (j == read_j && nidx < n_items) nit = p.items[nidx];
       }
+      idx = nidx;
+      it = nit;
     }
     if (ok) {
       const int st = J % kSimtStages;
@@ -173,12 +202,11 @@ __global__ void __launch_bounds__(kSimtThreads) decode_simt_kernel(DecodeParams 
     const T* vs = S.v[st];
 
     if (flags & kFirstTile) {
-      it = p.items[idx];
-      const T* qrow = static_cast<const T*>(p.q) + static_cast<int64_t>(it.row) * p.q_sr;
+      it = S.item[st];
 #pragma unroll
       for (int g = 0; g < GP; ++g) {
         if (g < p.g) {
-          const T* qh = qrow + static_cast<int64_t>(it.h * p.g + g) * p.q_sh;
+          const T* qh = S.qs[st] + g * D;
 #pragma unroll
           for (int j = 0; j < C::kChunksPerLane; ++j) {
             const int c = (lane % C::kLpt) + j * C::kLpt;
@@ -308,7 +336,7 @@ __global__ void __launch_bounds__(kSimtThreads) decode_simt_kernel(DecodeParams 
       }
       named_bar_sync(1, kSimtConsumers);
       const bool direct = it.nsplit == 1;
-      const int64_t slot = direct ? 0 : static_cast<int64_t>(p.row_base[it.row] + it.split);
+      const int64_t slot = direct ? 0 : static_cast<int64_t>(it.slot);
       for (int i3 = tid; i3 < p.g * D; i3 += kSimtConsumers) {
         const int g = i3 / D;
         const int d = i3 - g * D;
@@ -328,10 +356,14 @@ __global__ void __launch_bounds__(kSimtThreads) decode_simt_kernel(DecodeParams 
           out[d] = from_f32<T>(ov);
           if (d == 0) p.lse[static_cast<int64_t>(it.row) * p.hq + hq] = lse2 * kLn2;
         } else {
-          p.part_o[(slot * p.hq + hq) * D + d] = ov;
-          if (d == 0) p.part_lse[slot * p.hq + hq] = lse2;
+          p.part_o[(slot * p.g + g) * D + d] = ov;
+          if (d == 0) p.part_lse[slot * p.g + g] = lse2;
         }
       }
+      if (!direct)
+        finish_split_and_merge<T, (GP * D + 127) / 128>(merge_target(p), it.row, it.h, it.nsplit,
+                                                        it.slot - it.split, tid, 1, &S.mflag,
+                                                        S.mlse);
       named_bar_sync(1, kSimtConsumers);
     }
     ++J;
@@ -345,8 +377,17 @@ cudaError_t launch_simt_t(const DecodeParams& p, int nctas, cudaStream_t stream)
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  decode_simt_kernel<T, D, GP><<<nctas, kSimtThreads, smem, stream>>>(p);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(nctas);
+  cfg.blockDim = dim3(kSimtThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, decode_simt_kernel<T, D, GP>, p);
 }
 
 template <typename T, int D>

@@ -79,8 +79,8 @@ extern "C" fd_status fd_decode_attention_static(const fd_tensor* q, const fd_ten
   if (nctas < 1) return fail(FD_ERR_CUDA, "no multiprocessors reported for device %d", dev);
 
   const int64_t max_items = decode_max_items(sh.B, sh.hkv, sh.cap, num_splits, nctas);
-  const int64_t max_slots = (max_items + sh.hkv - 1) / sh.hkv;
-  const WsLayout L = ws_layout(max_items, 0, sh.B, max_slots, sh.hq, sh.d);
+  const int64_t max_slots = max_items;  // one partial slot (G heads) per split item
+  const WsLayout L = ws_layout(max_items, 0, sh.B, max_slots, sh.hq, sh.d, sh.hkv);
   if (L.total > static_cast<size_t>(FD_STATIC_SCRATCH_BYTES))
     return fail(FD_ERR_UNSUPPORTED,
                 "this decode shape needs up to %zu bytes of scratch, more than the %zu-byte static "
@@ -96,6 +96,7 @@ extern "C" fd_status fd_decode_attention_static(const fd_tensor* q, const fd_ten
   int32_t* row_base = reinterpret_cast<int32_t*>(base + L.row_base);
   float* part_o = reinterpret_cast<float*>(base + L.part_o);
   float* part_lse = reinterpret_cast<float*>(base + L.part_lse);
+  int32_t* arrivals = reinterpret_cast<int32_t*>(base + L.arrivals);
 
   DecodeParams dp{};
   dp.q = q->data;
@@ -122,6 +123,7 @@ extern "C" fd_status fd_decode_attention_static(const fd_tensor* q, const fd_ten
   dp.row_base = row_base;
   dp.part_o = part_o;
   dp.part_lse = part_lse;
+  dp.arrivals = arrivals;
 
   CUtensorMap tq, tk, tv;
   if (sh.use_tc) {
@@ -152,6 +154,7 @@ extern "C" fd_status fd_decode_attention_static(const fd_tensor* q, const fd_ten
   pp.items = items;
   pp.row_nsplit = row_nsplit;
   pp.row_base = row_base;
+  pp.arrivals = arrivals;
 
   CombineParams cp{};
   cp.row_nsplit = row_nsplit;
@@ -164,6 +167,8 @@ extern "C" fd_status fd_decode_attention_static(const fd_tensor* q, const fd_ten
   cp.lse = lse;
   cp.rows = sh.B;
   cp.hq = sh.hq;
+  cp.hkv = sh.hkv;
+  cp.g = sh.g;
   cp.d = sh.d;
   cp.dtype = sh.dtype;
 
@@ -175,7 +180,9 @@ extern "C" fd_status fd_decode_attention_static(const fd_tensor* q, const fd_ten
   ce = sh.use_tc ? launch_decode_tc(dp, tq, tk, tv, nctas, stream)
                  : launch_decode_simt(dp, sh.dtype, nctas, stream);
   if (ce != cudaSuccess) return cuda_fail(ce, "split kernel launch");
-  ce = launch_combine(cp, stream);
-  if (ce != cudaSuccess) return cuda_fail(ce, "combine kernel launch");
+  if (sh.use_tc) {
+    ce = launch_combine(cp, stream);
+    if (ce != cudaSuccess) return cuda_fail(ce, "combine kernel launch");
+  }
   return FD_OK;
 }

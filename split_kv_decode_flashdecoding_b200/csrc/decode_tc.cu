@@ -48,6 +48,7 @@ struct __align__(1024) TcSmem {
   float lred[4][GPAD];
   int32_t meta[kTcStages][2];                    // tile start, valid keys
   int32_t item_slot[2][2];                       // item index (-1: stop), tiles
+  DecodeItem item[2];                            // the item's descriptor (by item parity)
   uint64_t kfull[kTcStages], vfull[kTcStages], empty[kTcStages];
   uint64_t qfull[2], qempty[2], sfull[2], sempty[2], pfull[2], pempty[2], ofull[2], oempty[2];
   uint64_t drain;
@@ -103,27 +104,42 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   tc_fence_after();
   const uint32_t tmem = S.tmem_base;
   const WaitCtx ctx{&S.abort_flag, &p.hdr->status};
+  // Everything above overlapped the planner (programmatic dependent launch); the plan it wrote
+  // is read below. The combine kernel may launch now: it waits for this grid the same way.
+  pdl_wait_prerequisites();
+  pdl_launch_dependents();
 
   if (warp == kProducerWarp) {
     // ======================= TMA producer =======================
     if (lane == 0) {
       const int n_items = *reinterpret_cast<volatile int32_t*>(&p.hdr->num_dec_items);
+      const uint64_t pol = l2_evict_first_policy();
       uint32_t J = 0, K = 0;
       bool ok = true;
-      while (ok) {
-        const int idx = atomicAdd(&p.hdr->dec_counter, 1);
-        if (idx >= n_items) break;
-        const DecodeItem it = p.items[idx];
+      // The next item is claimed (atomic on the work cursor) when three tiles of the current one
+      // remain and its descriptor is read one tile later, so both round trips overlap the ring's
+      // lookahead: under full HBM load a dependent global access takes microseconds, and the
+      // ring would drain waiting for it at every item boundary. Claiming no earlier keeps the
+      // tail short (a CTA never sits on an item it cannot start soon).
+      int idx = atomicAdd(&p.hdr->dec_counter, 1);
+      DecodeItem it{};
+      if (idx < n_items) it = p.items[idx];
+      while (ok && idx < n_items) {
+        int nidx = n_items;
+        DecodeItem nit{};
         const int len = it.t1 - it.t0;
         const int ntile = len > 0 ? (len + kTcKeys - 1) / kTcKeys : 1;
         const int ps = K & 1;
         if (!mbar_wait(&S.qempty[ps], ((K >> 1) & 1u) ^ 1u, ctx)) { ok = false; break; }
         S.item_slot[ps][0] = idx;
         S.item_slot[ps][1] = ntile;
+        S.item[ps] = it;
         mbar_arrive_expect_tx(&S.qfull[ps], 2u * 128u * static_cast<uint32_t>(p.q_box_rows));
         tma_load_3d(S.q[ps][0], &tmap_q, &S.qfull[ps], 0, it.h * p.g, it.row);
         tma_load_3d(S.q[ps][1], &tmap_q, &S.qfull[ps], 64, it.h * p.g, it.row);
+        const int claim_j = max(0, ntile - 3), read_j = max(0, ntile - 2);
         for (int j = 0; j < ntile; ++j, ++J) {
+          if (j == claim_j) nidx = atomicAdd(&p.hdr->dec_counter, 1);
           const int st = J % kTcStages;
           if (!mbar_wait(&S.empty[st], ((J / kTcStages) & 1u) ^ 1u, ctx)) { ok = false; break; }
           const int t = it.t0 + j * kTcKeys;
@@ -133,17 +149,20 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           if (valid > 0) {
             const uint32_t tx = 2u * 128u * static_cast<uint32_t>(p.kv_box_rows);
             mbar_arrive_expect_tx(&S.kfull[st], tx);
-            tma_load_4d(S.k[st][0], &tmap_k, &S.kfull[st], 0, t, it.h, it.b);
-            tma_load_4d(S.k[st][1], &tmap_k, &S.kfull[st], 64, t, it.h, it.b);
+            tma_load_4d_stream(S.k[st][0], &tmap_k, &S.kfull[st], 0, t, it.h, it.b, pol);
+            tma_load_4d_stream(S.k[st][1], &tmap_k, &S.kfull[st], 64, t, it.h, it.b, pol);
             mbar_arrive_expect_tx(&S.vfull[st], tx);
-            tma_load_4d(S.v[st][0], &tmap_v, &S.vfull[st], 0, t, it.h, it.b);
-            tma_load_4d(S.v[st][1], &tmap_v, &S.vfull[st], 64, t, it.h, it.b);
+            tma_load_4d_stream(S.v[st][0], &tmap_v, &S.vfull[st], 0, t, it.h, it.b, pol);
+            tma_load_4d_stream(S.v[st][1], &tmap_v, &S.vfull[st], 64, t, it.h, it.b, pol);
           } else {
             mbar_arrive(&S.kfull[st]);
             mbar_arrive(&S.vfull[st]);
           }
+          if (j == read_j && nidx < n_items) nit = p.items[nidx];
         }
         ++K;
+        idx = nidx;
+        it = nit;
       }
       if (ok) {
         const int ps = K & 1;
@@ -276,10 +295,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       if (!mbar_wait(&S.qfull[ps], (K >> 1) & 1u, ctx)) break;
       const int idx = S.item_slot[ps][0];
       const int ntile = S.item_slot[ps][1];
+      const DecodeItem it = S.item[ps];
       __syncwarp();
       if (lane == 0) mbar_arrive(&S.qempty[ps]);
       if (idx < 0) break;
-      const DecodeItem it = p.items[idx];
 #pragma unroll
       for (int g = 0; g < GPAD; ++g) { m[g] = -INFINITY; lp[g] = 0.f; oacc[g] = 0.f; alpha_prev[g] = 1.f; }
       int prev_valid = 0;
@@ -373,7 +392,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       }
       named_bar_sync(1, kSoftmaxThreads);
       const bool direct = it.nsplit == 1;
-      const int64_t slot = direct ? 0 : static_cast<int64_t>(p.row_base[it.row] + it.split);
+      const int64_t slot = direct ? 0 : static_cast<int64_t>(it.slot);
 #pragma unroll
       for (int g = 0; g < GPAD; ++g) {
         if (g < p.g) {
@@ -387,8 +406,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             out[tid] = __float2bfloat16_rn(ov);
             if (tid == 0) p.lse[static_cast<int64_t>(it.row) * p.hq + hq] = lse2 * kLn2;
           } else {
-            p.part_o[(slot * p.hq + hq) * kTcD + tid] = ov;
-            if (tid == 0) p.part_lse[slot * p.hq + hq] = lse2;
+            p.part_o[(slot * p.g + g) * kTcD + tid] = ov;
+            if (tid == 0) p.part_lse[slot * p.g + g] = lse2;
           }
         }
       }
@@ -411,8 +430,17 @@ cudaError_t launch_tc_t(const DecodeParams& p, const CUtensorMap& tq, const CUte
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  decode_tc_kernel<GPAD><<<nctas, kTcThreads, smem, stream>>>(p, tq, tk, tv);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(nctas);
+  cfg.blockDim = dim3(kTcThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, decode_tc_kernel<GPAD>, p, tq, tk, tv);
 }
 
 }  // namespace

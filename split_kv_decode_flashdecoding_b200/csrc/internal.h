@@ -5,6 +5,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "common.cuh"
 #include "plan.h"
 
 namespace fd {
@@ -20,6 +21,9 @@ struct PlanParams {
   TileItem* tiles;
   int32_t* row_nsplit;
   int32_t* row_base;
+  int32_t* arrivals;        // [rows * Hkv] split-completion counters of the in-kernel merge
+  int32_t total_rows;       // chunk mode: packed query rows T (= sum of chunk lengths)
+  int32_t decode_merged_in_kernel;  // chunk mode: decode rows merge inside their split kernel
   // optional export of the decode plan (fd_split_plan_device)
   int32_t* out_splits;
   int32_t* out_items;
@@ -44,18 +48,37 @@ struct DecodeParams {
   WsHeader* hdr;
   const DecodeItem* items;
   const int32_t* row_base;
-  float* part_o;     // [slots, Hq, D]
-  float* part_lse;   // [slots, Hq] (log2 domain)
+  float* part_o;     // [slots, G, D], the slots of one (row, KV head) group consecutive
+  float* part_lse;   // [slots, G] (log2 domain)
+  int32_t* arrivals; // [rows, Hkv] split-completion counters of the in-kernel merge
 };
+
+__device__ __forceinline__ MergeTarget merge_target(const DecodeParams& p) {
+  MergeTarget t;
+  t.part_o = p.part_o;
+  t.part_lse = p.part_lse;
+  t.arrivals = p.arrivals;
+  t.out = p.out;
+  t.o_sr = p.o_sr;
+  t.o_sh = p.o_sh;
+  t.lse = p.lse;
+  t.hq = p.hq;
+  t.hkv = p.hkv;
+  t.g = p.g;
+  t.d = p.d;
+  return t;
+}
 
 // Chunked-prefill tiles.
 struct TileParams {
-  const void* q;
+  const void* q;     // [T, Hq, D] packed query chunks
   int64_t q_sr, q_sh;
   void* out;
   int64_t o_sr, o_sh;
   float* lse;
   int32_t hq, hkv, g, d, cap;
+  int32_t q_box_rows;   // rows of one Q tensor-map box: min(128, T)
+  int32_t kv_box_rows;  // rows of one K/V tensor-map box: min(128, S_cap)
   float scale_log2;
   WsHeader* hdr;
   const TileItem* tiles;
@@ -72,7 +95,7 @@ struct CombineParams {
   void* out;
   int64_t o_sr, o_sh;
   float* lse;
-  int32_t rows, hq, d, dtype;
+  int32_t rows, hq, hkv, g, d, dtype;
 };
 
 cudaError_t launch_plan_decode(const PlanParams& p, cudaStream_t stream);
@@ -92,6 +115,8 @@ cudaError_t launch_chunk_tc(const TileParams& p, const CUtensorMap& tmap_q,
                             const CUtensorMap& tmap_k, const CUtensorMap& tmap_v, int nctas,
                             cudaStream_t stream);
 
+// Launched with programmatic dependent launch after a split kernel (tensor-core decode path; the
+// CUDA-core kernel merges its own groups in-kernel).
 cudaError_t launch_combine(const CombineParams& p, cudaStream_t stream);
 
 }  // namespace fd

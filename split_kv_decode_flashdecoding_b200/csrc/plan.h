@@ -38,7 +38,8 @@ struct DecodeItem {
   int32_t split;   // split index within the sequence
   int32_t t0, t1;  // key range
   int32_t nsplit;  // splits of this sequence (1: write the final output directly)
-  int32_t seqlen;  // clamped sequence length (keys at >= seqlen may hold anything)
+  int32_t slot;    // partial slot of this split; the slots of one (row, KV head) group are
+                   // consecutive: row_base[row] * Hkv + h * nsplit + split
 };
 static_assert(sizeof(DecodeItem) == 32, "DecodeItem is 32 bytes");
 
@@ -99,8 +100,14 @@ FD_HD void plan_split_range(int32_t len, int32_t n, int32_t s, int32_t fixed, in
     *t0 = static_cast<int32_t>(a < len ? a : len);
     *t1 = static_cast<int32_t>(e < len ? e : len);
   } else {
-    *t0 = static_cast<int32_t>((static_cast<int64_t>(s) * len) / n);
-    *t1 = static_cast<int32_t>((static_cast<int64_t>(s + 1) * len) / n);
+    const int64_t a = static_cast<int64_t>(s) * len, e = static_cast<int64_t>(s + 1) * len;
+    if (e <= INT32_MAX) {  // 32-bit division when the products fit (the common case)
+      *t0 = static_cast<int32_t>(a) / n;
+      *t1 = static_cast<int32_t>(e) / n;
+    } else {
+      *t0 = static_cast<int32_t>(a / n);
+      *t1 = static_cast<int32_t>(e / n);
+    }
   }
 }
 
@@ -119,13 +126,37 @@ FD_HD int64_t decode_max_items(int64_t B, int64_t hkv, int64_t cap, int32_t fixe
   return hkv * B + (a > b ? a : b);
 }
 
+// Chunked prefill: keys seen by query tile t of a chunk of c rows at prefix p (clamped to S_cap),
+// and the number of kChunkKvSplit-key splits they are cut into.
+FD_HD int32_t chunk_tile_keys(int32_t prefix, int32_t c, int32_t t, int32_t cap) {
+  const int64_t last = static_cast<int64_t>(t + 1) * kQTile;
+  const int64_t k = static_cast<int64_t>(prefix) + (last < c ? last : c);
+  return k < 0 ? 0 : (k > cap ? cap : static_cast<int32_t>(k));
+}
+FD_HD int32_t chunk_tile_splits(int32_t keys) {
+  const int32_t n = static_cast<int32_t>(cdiv64(keys, kChunkKvSplit));
+  return n < 1 ? 1 : n;
+}
+
+// Upper bounds for a chunked-prefill call of T packed rows over B requests (any lengths).
+FD_HD int64_t chunk_max_tile_items(int64_t B, int64_t T, int64_t hq, int64_t cap) {
+  return (cdiv64(T, kQTile) + B) * cdiv64(cap > 0 ? cap : 1, kChunkKvSplit) * hq;
+}
+FD_HD int64_t chunk_max_slots(int64_t B, int64_t T, int64_t hkv, int64_t cap, int32_t nctas) {
+  // decode rows: at most decode_max_items / Hkv splits; tile rows: ceil(S_cap / split) each
+  const int64_t dec = decode_max_items(B, hkv, cap, 0, nctas) / hkv + 1;
+  return (dec + T * cdiv64(cap > 0 ? cap : 1, kChunkKvSplit)) * hkv;
+}
+
 // Workspace layout (byte offsets, 256-byte aligned sections).
 struct WsLayout {
-  size_t dec_items, tile_items, row_nsplit, row_base, part_o, part_lse, total;
+  size_t dec_items, tile_items, row_nsplit, row_base, arrivals, part_o, part_lse, total;
 };
 
+// Partial slots hold the G = Hq / Hkv query heads of one KV head: [slot][G][D] fp32 outputs and
+// [slot][G] base-2 LSEs, so `max_slots` counts (row, KV head, split) triples.
 FD_HD WsLayout ws_layout(int64_t max_dec_items, int64_t max_tile_items, int64_t rows,
-                         int64_t max_slots, int32_t hq, int32_t d) {
+                         int64_t max_slots, int32_t hq, int32_t d, int32_t hkv = 1) {
   WsLayout L;
   size_t off = sizeof(WsHeader);
   L.dec_items = off;
@@ -136,10 +167,13 @@ FD_HD WsLayout ws_layout(int64_t max_dec_items, int64_t max_tile_items, int64_t 
   off = align_up(off + static_cast<size_t>(rows) * 4, 256);
   L.row_base = off;
   off = align_up(off + static_cast<size_t>(rows) * 4, 256);
+  L.arrivals = off;
+  off = align_up(off + static_cast<size_t>(rows) * hkv * 4, 256);
+  const int64_t g = hq / (hkv > 0 ? hkv : 1);
   L.part_o = off;
-  off = align_up(off + static_cast<size_t>(max_slots) * hq * d * 4, 256);
+  off = align_up(off + static_cast<size_t>(max_slots) * g * d * 4, 256);
   L.part_lse = off;
-  off = align_up(off + static_cast<size_t>(max_slots) * hq * 4, 256);
+  off = align_up(off + static_cast<size_t>(max_slots) * g * 4, 256);
   L.total = off;
   return L;
 }

@@ -8,7 +8,9 @@ namespace fd {
 
 namespace {
 
-constexpr int kPlanThreads = 1024;
+constexpr int kMaxPlanThreads = 1024;
+
+__device__ __forceinline__ int plan_threads() { return static_cast<int>(blockDim.x); }
 
 __device__ __forceinline__ long long warp_sum_i64(long long v) {
 #pragma unroll
@@ -26,10 +28,11 @@ __device__ __forceinline__ int warp_incl_scan(int v) {
 }
 
 // Exclusive prefix sum of in[0..n) into out[0..n], out[n] = total. All threads of the CTA call
-// it; `scratch` holds 33 ints of shared memory. n <= 4 * kPlanThreads.
+// it; `scratch` holds 33 ints of shared memory.
 __device__ void block_exclusive_scan(const int32_t* in, int32_t* out, int n, int* scratch) {
   const int tid = threadIdx.x;
-  const int per = (n + kPlanThreads - 1) / kPlanThreads;
+  const int nthr = plan_threads();
+  const int per = (n + nthr - 1) / nthr;
   const int lo = tid * per;
   int local = 0;
   for (int i = 0; i < per; ++i)
@@ -39,7 +42,7 @@ __device__ void block_exclusive_scan(const int32_t* in, int32_t* out, int n, int
   if (lane_id() == 31) scratch[warp] = incl;
   __syncthreads();
   if (warp == 0) {
-    int w = (lane_id() < kPlanThreads / 32) ? scratch[lane_id()] : 0;
+    int w = (lane_id() < static_cast<uint32_t>(nthr / 32)) ? scratch[lane_id()] : 0;
     int wi = warp_incl_scan(w);
     scratch[lane_id()] = wi - w;  // exclusive warp offsets
     if (lane_id() == 31) scratch[32] = wi;
@@ -60,14 +63,16 @@ __device__ void block_exclusive_scan(const int32_t* in, int32_t* out, int n, int
 // `row_of` maps sequence index -> output row (identity for decode calls).
 __device__ void plan_decode_body(const PlanParams& p, const int32_t* len_src, int B,
                                  const int32_t* row_of, uint32_t* s_flags) {
+  // shared memory sized by the batch: 7 * B + 2 ints
   extern __shared__ int32_t smem[];
   int32_t* s_len = smem;
-  int32_t* s_n = s_len + kMaxPlanBatch;
-  int32_t* s_key = s_n + kMaxPlanBatch;
-  int32_t* s_order = s_key + kMaxPlanBatch;
-  int32_t* s_ioff = s_order + kMaxPlanBatch;        // kMaxPlanBatch + 1
-  int32_t* s_tmp = s_ioff + kMaxPlanBatch + 1;      // kMaxPlanBatch
-  int32_t* s_rbase = s_tmp + kMaxPlanBatch;         // kMaxPlanBatch + 1
+  int32_t* s_n = s_len + B;
+  int32_t* s_key = s_n + B;
+  int32_t* s_order = s_key + B;
+  int32_t* s_ioff = s_order + B;        // B + 1
+  int32_t* s_tmp = s_ioff + B + 1;      // B
+  int32_t* s_rbase = s_tmp + B;         // B + 1
+  const int kPlanThreads = plan_threads();
   __shared__ int s_scan[33];
   __shared__ unsigned long long s_total;
   const int tid = threadIdx.x;
@@ -128,40 +133,48 @@ __device__ void plan_decode_body(const PlanParams& p, const int32_t* len_src, in
     p.row_base[row] = s_rbase[b];
     if (p.out_splits) p.out_splits[b] = s_n[b];
   }
-  for (int i = tid; i < total_items; i += kPlanThreads) {
-    // the sequence whose item range holds i: largest r with s_ioff[r] <= i
-    int lo = 0, hi = B - 1;
-    while (lo < hi) {
-      const int mid = (lo + hi + 1) >> 1;
-      if (s_ioff[mid] <= i) lo = mid; else hi = mid - 1;
-    }
-    const int b = s_order[lo];
+  // One warp per sequence (in rank order) writes that sequence's items; lanes take splits, so each
+  // key range is computed once and written for every KV head (no per-item search or division).
+  const int warp = tid >> 5;
+  const int lane = static_cast<int>(lane_id());
+  for (int r = warp; r < B; r += kPlanThreads / 32) {
+    const int b = s_order[r];
     const int32_t n = s_n[b];
-    const int32_t local_i = i - s_ioff[lo];
-    const int32_t h = local_i / n;
-    const int32_t s = local_i - h * n;
-    int32_t t0, t1;
-    plan_split_range(s_len[b], n, s, p.fixed, &t0, &t1);
-    if (!overflow) {
-      DecodeItem it;
-      it.row = row_of ? row_of[b] : b;
-      it.b = b;
-      it.h = h;
-      it.split = s;
-      it.t0 = t0;
-      it.t1 = t1;
-      it.nsplit = n;
-      it.seqlen = s_len[b];
-      p.items[i] = it;
-    }
-    if (p.out_items && i < p.out_cap) {
-      int32_t* o = p.out_items + 5 * static_cast<int64_t>(i);
-      o[0] = b; o[1] = h; o[2] = s; o[3] = t0; o[4] = t1;
+    const int32_t L = s_len[b];
+    const int32_t first = s_ioff[r];
+    const int32_t rbase = s_rbase[b];
+    const int row = row_of ? row_of[b] : b;
+    for (int32_t s = lane; s < n; s += 32) {
+      int32_t t0, t1;
+      plan_split_range(L, n, s, p.fixed, &t0, &t1);
+      for (int32_t h = 0; h < p.hkv; ++h) {
+        const int32_t i = first + h * n + s;
+        if (!overflow) {
+          // two 16-byte stores per 32-byte item: scalar stores from lanes 32 bytes apart would
+          // throttle this single CTA's load/store unit on partial-sector writes
+          int4* dst = reinterpret_cast<int4*>(p.items + i);
+          dst[0] = make_int4(row, b, h, s);
+          dst[1] = make_int4(t0, t1, n, rbase * p.hkv + h * n + s);
+        }
+        if (p.out_items && i < p.out_cap) {
+          int32_t* o = p.out_items + 5 * static_cast<int64_t>(i);
+          o[0] = b; o[1] = h; o[2] = s; o[3] = t0; o[4] = t1;
+        }
+      }
     }
   }
+  // arrival counters of the in-kernel merge start every call at zero
+  if (p.arrivals)
+    for (int i = tid; i < B * p.hkv; i += kPlanThreads) {
+      const int row = row_of ? row_of[i / p.hkv] : i / p.hkv;
+      p.arrivals[row * p.hkv + i % p.hkv] = 0;
+    }
 }
 
-__global__ void __launch_bounds__(kPlanThreads, 1) plan_decode_kernel(PlanParams p) {
+__global__ void __launch_bounds__(kMaxPlanThreads, 1) plan_decode_kernel(PlanParams p) {
+  // the split kernel may launch now (programmatic dependent launch); it waits for this grid's
+  // completion before it reads the plan
+  pdl_launch_dependents();
   __shared__ uint32_t s_flags;
   if (threadIdx.x == 0) s_flags = 0;
   __syncthreads();
@@ -170,17 +183,203 @@ __global__ void __launch_bounds__(kPlanThreads, 1) plan_decode_kernel(PlanParams
   if (threadIdx.x == 0 && s_flags) atomicOr(&p.hdr->status, s_flags);
 }
 
+// Chunked-prefill plan (one CTA): requests with chunk_len == 1 are decode rows over
+// prefix + 1 keys, planned like a decode call over those requests; longer chunks become query
+// tiles of kQTile rows whose keys are cut on a fixed kChunkKvSplit grid, items ordered
+// (request, query head, split, tile). One exclusive scan over all packed rows gives every row
+// its partial slots, so the same combine merges decode rows and tile rows.
+__global__ void __launch_bounds__(kMaxPlanThreads, 1) plan_chunk_kernel(PlanParams p) {
+  pdl_launch_dependents();
+  extern __shared__ int32_t smem[];
+  const int B = p.B;
+  const int T = p.total_rows;
+  const int nthr = plan_threads();
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5;
+  const int lane = static_cast<int>(lane_id());
+  int32_t* s_c = smem;                 // chunk rows (>= 0)
+  int32_t* s_p = s_c + B;              // prefix, clamped to [0, S_cap]
+  int32_t* s_dlen = s_p + B;           // decode length (0 for tile requests)
+  int32_t* s_n = s_dlen + B;           // decode splits
+  int32_t* s_key = s_n + B;            // decode ordering key
+  int32_t* s_order = s_key + B;        // decode requests, longest first
+  int32_t* s_tcnt = s_order + B;       // tile items per request
+  int32_t* s_tmp = s_tcnt + B;
+  int32_t* s_roff = s_tmp + B;         // B + 1: first packed row of each request
+  int32_t* s_dioff = s_roff + B + 1;   // B + 1: decode item offsets (rank order)
+  int32_t* s_tioff = s_dioff + B + 1;  // B + 1: tile item offsets (request order)
+  __shared__ int s_scan[33];
+  __shared__ unsigned long long s_total;
+  __shared__ uint32_t s_flags;
+  __shared__ int s_ndec;
+  if (tid == 0) { s_total = 0ull; s_flags = 0u; s_ndec = 0; }
+  __syncthreads();
+
+  long long local = 0;
+  int ndec = 0;
+  for (int b = tid; b < B; b += nthr) {
+    const int32_t raw_p = p.lens[b], raw_c = p.chunk_lens[b];
+    const int32_t c = raw_c < 0 ? 0 : raw_c;
+    const int32_t pp = clamp_len(raw_p, p.cap);
+    if (raw_c < 0 || pp != raw_p || static_cast<int64_t>(pp) + c > p.cap)
+      atomicOr(&s_flags, FD_FLAG_LEN_CLAMPED);
+    const int32_t dlen = c == 1 ? clamp_len(static_cast<int64_t>(pp) + 1, p.cap) : 0;
+    s_c[b] = c;
+    s_p[b] = pp;
+    s_dlen[b] = dlen;
+    local += dlen;
+    ndec += c == 1 ? 1 : 0;
+  }
+  local = warp_sum_i64(local);
+  if (lane_id() == 0 && local != 0) atomicAdd(&s_total, static_cast<unsigned long long>(local));
+  if (ndec) atomicAdd(&s_ndec, ndec);
+  __syncthreads();
+
+  const int32_t chunk = plan_chunk_tokens(static_cast<int64_t>(s_total), p.hkv, p.nctas);
+  for (int b = tid; b < B; b += nthr) {
+    const int32_t c = s_c[b];
+    if (c == 1) {
+      const int32_t n = plan_num_splits(s_dlen[b], chunk, 0);
+      s_n[b] = n;
+      s_key[b] = plan_sort_key(s_dlen[b], n);
+      s_tcnt[b] = 0;
+    } else {
+      s_n[b] = 0;
+      s_key[b] = -1;
+      int32_t cnt = 0;
+      for (int32_t t = 0; t * kQTile < c; ++t) {
+        const int32_t kt = chunk_tile_keys(s_p[b], c, t, p.cap);
+        cnt += chunk_tile_splits(kt);
+      }
+      s_tcnt[b] = cnt * p.hq;
+    }
+  }
+  __syncthreads();
+  block_exclusive_scan(s_c, s_roff, B, s_scan);
+  // decode requests longest first (stable counting rank among decode requests)
+  for (int b = tid; b < B; b += nthr) {
+    if (s_c[b] != 1) continue;
+    const int32_t kb = s_key[b];
+    int r = 0;
+    for (int j = 0; j < B; ++j) {
+      const int32_t kj = s_key[j];
+      r += (s_c[j] == 1 && (kj > kb || (kj == kb && j < b))) ? 1 : 0;
+    }
+    s_order[r] = b;
+  }
+  __syncthreads();
+  const int nd = s_ndec;
+  for (int r = tid; r < nd; r += nthr) s_tmp[r] = s_n[s_order[r]] * p.hkv;
+  __syncthreads();
+  block_exclusive_scan(s_tmp, s_dioff, nd, s_scan);
+  block_exclusive_scan(s_tcnt, s_tioff, B, s_scan);
+  // chunk lengths that do not add up to the packed rows of q_chunk: nothing is computed (the
+  // outputs are left as they were) and the status word says why
+  const bool inconsistent = s_roff[B] != T;
+  if (tid == 0 && inconsistent) atomicOr(&s_flags, FD_FLAG_LEN_CLAMPED);
+
+  // partial slots per packed row, then their exclusive scan (global memory)
+  for (int b = warp; b < B && !inconsistent; b += nthr / 32) {
+    const int32_t c = s_c[b];
+    const int32_t r0 = s_roff[b];
+    for (int32_t r = lane; r < c; r += 32)
+      p.row_nsplit[r0 + r] = c == 1 ? s_n[b] : chunk_tile_splits(chunk_tile_keys(s_p[b], c, r / kQTile, p.cap));
+  }
+  if (inconsistent)
+    for (int32_t row = tid; row < T; row += nthr) p.row_nsplit[row] = 0;
+  __syncthreads();
+  block_exclusive_scan(p.row_nsplit, p.row_base, T, s_scan);
+
+  const int32_t n_dec_items = s_dioff[nd];
+  const int32_t n_tile_items = s_tioff[B];
+  const bool overflow =
+      inconsistent || n_dec_items > p.max_dec_items || n_tile_items > p.max_tile_items;
+  // decode items: one warp per decode request, lanes over splits
+  for (int r = warp; r < nd && !overflow; r += nthr / 32) {
+    const int b = s_order[r];
+    const int32_t row = s_roff[b];
+    const int32_t n = s_n[b], L = s_dlen[b], first = s_dioff[r];
+    const int32_t rbase = p.row_base[row];
+    for (int32_t s = lane; s < n; s += 32) {
+      int32_t t0, t1;
+      plan_split_range(L, n, s, 0, &t0, &t1);
+      for (int32_t h = 0; h < p.hkv; ++h) {
+        int4* dst = reinterpret_cast<int4*>(p.items + first + h * n + s);
+        dst[0] = make_int4(row, b, h, s);
+        dst[1] = make_int4(t0, t1, n, rbase * p.hkv + h * n + s);
+      }
+    }
+  }
+  // tile items: one warp per request, lanes over query heads, (split, tile) order per head
+  for (int b = warp; b < B && !overflow; b += nthr / 32) {
+    const int32_t c = s_c[b];
+    if (c < 2) continue;
+    const int32_t pp = s_p[b], r0 = s_roff[b];
+    const int32_t ntiles = (c + kQTile - 1) / kQTile;
+    const int32_t per_head = s_tcnt[b] / p.hq;
+    const int32_t nmax = chunk_tile_splits(chunk_tile_keys(pp, c, ntiles - 1, p.cap));
+    for (int32_t h = lane; h < p.hq; h += 32) {
+      int32_t i = s_tioff[b] + h * per_head;
+      for (int32_t s = 0; s < nmax; ++s) {
+        for (int32_t t = 0; t < ntiles; ++t) {
+          const int32_t kt = chunk_tile_keys(pp, c, t, p.cap);
+          const int32_t nt = chunk_tile_splits(kt);
+          if (s >= nt) continue;
+          const int32_t row0 = r0 + t * kQTile;
+          const int32_t rows = min(kQTile, c - t * kQTile);
+          const int32_t k0 = min(s * kChunkKvSplit, kt), k1 = min((s + 1) * kChunkKvSplit, kt);
+          const int32_t slot0 = p.row_base[row0] * p.hkv;
+          int4* dst = reinterpret_cast<int4*>(p.tiles + i);
+          dst[0] = make_int4(b, h, s, nt);
+          dst[1] = make_int4(k0, k1, row0, t * kQTile);
+          dst[2] = make_int4(rows, pp, slot0, 0);
+          dst[3] = make_int4(0, 0, 0, 0);
+          ++i;
+        }
+      }
+    }
+  }
+  __syncthreads();
+  // decode rows merged inside their split kernel: the combine skips them; their counters reset
+  for (int r = tid; r < nd && !inconsistent; r += nthr) {
+    const int32_t row = s_roff[s_order[r]];
+    if (p.decode_merged_in_kernel) p.row_nsplit[row] = 1;
+    for (int32_t h = 0; h < p.hkv; ++h) p.arrivals[row * p.hkv + h] = 0;
+  }
+  if (tid == 0) {
+    p.hdr->num_dec_items = overflow ? 0 : n_dec_items;
+    p.hdr->num_tile_items = overflow ? 0 : n_tile_items;
+    p.hdr->dec_counter = 0;
+    p.hdr->tile_counter = 0;
+    uint32_t f = s_flags | (overflow ? FD_FLAG_PLAN_OVERFLOW : 0u);
+    if (f) atomicOr(&p.hdr->status, f);
+  }
+}
+
 }  // namespace
 
-size_t plan_smem_bytes() { return sizeof(int32_t) * (7 * static_cast<size_t>(kMaxPlanBatch) + 2); }
+cudaError_t launch_plan_chunk(const PlanParams& p, cudaStream_t stream) {
+  const size_t smem = sizeof(int32_t) * (11 * static_cast<size_t>(p.B) + 3);
+  if (smem > 48 * 1024) {
+    cudaError_t e = cudaFuncSetAttribute(plan_chunk_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+  }
+  plan_chunk_kernel<<<1, kMaxPlanThreads, smem, stream>>>(p);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_plan_decode(const PlanParams& p, cudaStream_t stream) {
-  const size_t smem = plan_smem_bytes();
-  cudaError_t e = cudaFuncSetAttribute(plan_decode_kernel,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(smem));
-  if (e != cudaSuccess) return e;
-  plan_decode_kernel<<<1, kPlanThreads, smem, stream>>>(p);
+  const size_t smem = sizeof(int32_t) * (7 * static_cast<size_t>(p.B) + 2);
+  const int threads = kMaxPlanThreads;
+  if (smem > 48 * 1024) {
+    cudaError_t e = cudaFuncSetAttribute(plan_decode_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+  }
+  plan_decode_kernel<<<1, threads, smem, stream>>>(p);
   return cudaGetLastError();
 }
 

@@ -1,0 +1,104 @@
+"""GPU parity of fd_chunk_prefill_attention against the float64 oracle, through the C ABI.
+
+Caches hold NaN past every request's prefix + chunk, so a read beyond the causal limit poisons
+the result; outputs sit inside guard bands that must stay untouched.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import attention as oracle
+from parity import check_lse, check_out, sample_rows
+from workloads import make_chunk_inputs, to_numpy_exact, workload
+
+pytestmark = pytest.mark.gpu
+
+NAN = float("nan")
+
+
+def _run(inp, guard=True):
+    import split_kv_decode_flashdecoding_b200 as fd
+    dev = torch.device("cuda", 0)
+    q = inp.q_chunk.to(dev)
+    T, Hq, D = q.shape
+    if guard:
+        big = torch.full((T + 2, Hq, D), 4321.0, dtype=q.dtype, device=dev)
+        out = big[1:T + 1]
+        lbig = torch.full((T * Hq + 64,), 555.0, dtype=torch.float32, device=dev)
+        lse = lbig[32:32 + T * Hq].view(T, Hq)
+    else:
+        out = torch.empty_like(q)
+        lse = torch.empty((T, Hq), dtype=torch.float32, device=dev)
+    fd.fd_chunk_prefill_attention(q, inp.k_cache.to(dev), inp.v_cache.to(dev),
+                                  inp.prefix_lens.to(dev), inp.chunk_lens.to(dev), out=out, lse=lse)
+    torch.cuda.synchronize()
+    if guard:
+        assert bool((big[0] == 4321.0).all()) and bool((big[T + 1] == 4321.0).all()), "out guard band"
+        assert bool((lbig[:32] == 555.0).all()) and bool((lbig[32 + T * Hq:] == 555.0).all()), "lse guard"
+    flags = fd.fd_poll_status()
+    assert flags & fd.FD_FLAG_WAIT_TIMEOUT == 0 and flags & fd.FD_FLAG_PLAN_OVERFLOW == 0, hex(flags)
+    return out, lse
+
+
+def _oracle(inp, rows=None):
+    return oracle.chunk_prefill_attention(
+        to_numpy_exact(inp.q_chunk), to_numpy_exact(inp.k_cache), to_numpy_exact(inp.v_cache),
+        inp.prefix_lens.tolist(), inp.chunk_lens.tolist(), rows=rows)
+
+
+CASES = [
+    # (prefix_lens, chunk_lens, Hq, Hkv, cap)
+    ([0], [5], 2, 2, 64),                          # tiny chunk, no prefix
+    ([300], [130], 2, 2, 512),                     # two tiles, ragged second tile
+    ([1900], [300], 2, 2, 4096),                   # tile 0 one split, tiles 1-2 two splits
+    ([2500, 10, 0, 700, 33], [200, 1, 1, 1, 0], 4, 4, 4096),  # chunk + decode rows + empty
+    ([1000, 77, 4000], [129, 1, 1], 16, 2, 4200),  # GQA (G = 8): decode rows on tensor cores
+    ([64], [64], 4, 1, 128),                       # GQA G = 4, capacity = prefix + chunk
+]
+
+
+@pytest.mark.parametrize("case", range(len(CASES)))
+def test_small_chunks(case):
+    prefix, chunk, hq, hkv, cap = CASES[case]
+    inp = make_chunk_inputs(prefix, chunk, hq, hkv, 128, cap, torch.bfloat16, seed=300 + case,
+                            pad_fill=NAN)
+    out, lse = _run(inp)
+    ro, rl = _oracle(inp)
+    check_out(out, ro, "chunk out")
+    check_lse(lse, rl, "chunk lse")
+
+
+def test_chunk_equals_decode_rows():
+    # a chunk of 3 rows at prefix p gives, row by row, the decode results over p + i + 1 keys
+    import split_kv_decode_flashdecoding_b200 as fd
+    inp = make_chunk_inputs([777], [3], 8, 8, 128, 1024, torch.bfloat16, seed=41)
+    out, lse = _run(inp)
+    dev = torch.device("cuda", 0)
+    for i in range(3):
+        q = inp.q_chunk[i:i + 1].to(dev)
+        lens = torch.tensor([778 + i], dtype=torch.int32, device=dev)
+        o2, l2 = fd.fd_decode_attention(q, inp.k_cache.to(dev), inp.v_cache.to(dev), lens)
+        torch.cuda.synchronize()
+        check_out(out[i:i + 1], o2.float().cpu().numpy().astype(np.float64), "chunk row vs decode")
+        check_lse(lse[i:i + 1], l2.cpu().numpy().astype(np.float64), "chunk row vs decode lse")
+
+
+def test_full_mixed_workload_sampled():
+    inp = workload(5)
+    out, lse = _run(inp, guard=False)
+    assert bool(torch.isfinite(out.float()).all()) and bool(torch.isfinite(lse).all())
+    T, Hq, _ = inp.q_chunk.shape
+    must = [(0, 0), (1, 5), (127, 31), (128, 7), (255, 3), (256, 0), (383, 12), (511, 31),
+            (512, 0), (520, 9), (T - 1, Hq - 1)]
+    rows = sample_rows(T, Hq, 40, seed=5, must=must)
+    ro, rl = _oracle(inp, rows=rows)
+    check_out(out, ro, "mixed out")
+    check_lse(lse, rl, "mixed lse")
+
+
+def test_chunk_deterministic():
+    inp = make_chunk_inputs([1500, 3], [260, 1], 4, 4, 128, 2048, torch.bfloat16, seed=51)
+    o1, l1 = _run(inp)
+    o2, l2 = _run(inp)
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)

@@ -144,14 +144,19 @@ def test_deterministic_and_stream():
 
 def test_device_plan_equals_host_plan():
     fd = _fd()
+    from workloads import uniform_lens
     rng = np.random.default_rng(0)
-    for trial in range(12):
-        B = int(rng.choice([1, 3, 32, 100, 1000]))
-        cap = int(rng.choice([64, 1024, 32768]))
-        hkv = int(rng.choice([1, 8, 40]))
-        fixed = int(rng.choice([0, 0, 4]))
-        nctas = int(rng.choice([148, 296]))
-        lens = [int(x) for x in rng.integers(-3, cap + 3, size=B)]
+    for trial in range(13):
+        if trial == 0:   # the 70B-like decode workload's plan first
+            B, cap, hkv, fixed, nctas = 32, 32768, 8, 0, 148
+            lens = uniform_lens(1103, 32, 1024, 32768)
+        else:
+            B = int(rng.choice([1, 3, 32, 100, 1000]))
+            cap = int(rng.choice([64, 1024, 32768]))
+            hkv = int(rng.choice([1, 8, 40]))
+            fixed = int(rng.choice([0, 0, 4]))
+            nctas = int(rng.choice([148, 296]))
+            lens = [int(x) for x in rng.integers(-3, cap + 3, size=B)]
         info, splits, items = fd.fd_split_plan(lens, hkv, cap, fixed, nctas)
         ref = oplan.decode_plan(lens, hkv, cap, nctas, fixed)
         dl = torch.tensor(lens, dtype=torch.int32, device="cuda")

@@ -139,8 +139,10 @@ def workload(index: int, batch: Optional[int] = None, pad_fill: float = 0.0):
                                   pad_fill=pad_fill, name=WORKLOADS[2])
     if index == 3:
         lens = uniform_lens(lseed, 32, 1024, 32768)
-        return make_decode_inputs(32, 64, 8, 128, 32768, lens, torch.bfloat16, seed,
-                                  pad_fill=pad_fill, name=WORKLOADS[3])
+        b = 32 if batch is None else int(batch)   # a smaller batch keeps the first b sequences
+        name = WORKLOADS[3] if b == 32 else f"{WORKLOADS[3]}_first{b}"
+        return make_decode_inputs(b, 64, 8, 128, 32768, lens[:b], torch.bfloat16, seed,
+                                  pad_fill=pad_fill, name=name)
     if index == 4:
         b = 1 if batch is None else int(batch)
         return make_decode_inputs(b, 64, 8, 128, 32768, [32768] * b, torch.bfloat16,
