@@ -192,7 +192,10 @@ __global__ void __launch_bounds__(kSimtThreads) decode_simt_kernel(DecodeParams 
   uint32_t J = 0;
   while (true) {
     const int st = J % kSimtStages;
-    if (!mbar_wait(&S.full[st], (J / kSimtStages) & 1u, ctx)) break;
+    // The consumer warps meet at named barriers below, which have no time limit; a warp whose
+    // wait timed out must not leave alone, so they vote and leave together.
+    const bool ok = mbar_wait(&S.full[st], (J / kSimtStages) & 1u, ctx);
+    if (named_bar_or(1, kSimtConsumers, !ok)) break;
     const int idx = S.meta[st][0];
     if (idx < 0) break;
     const int valid = S.meta[st][2];

@@ -8,17 +8,21 @@
 //   p = 2^(s*scale*log2e - m')  per key lane, split into bf16 hi + lo parts (P ≈ P_hi + P_lo)
 //   Oᵀ[128 d x 2·GPAD] = V_tileᵀ · [P_hi | P_lo]ᵀ                UMMA M=128 N=2·GPAD, MN-major A/B
 //
-// Sᵀ and Oᵀ live in tensor memory, double-buffered; the softmax warps read them with tcgen05.ld,
-// keep the running max m, the running sums l (per key lane) and the output accumulator (per d
-// lane) in registers, and rescale by 2^(m - m') as the online softmax of
-// "大语言模型长序列推理优化：ChunkedPrefill与FlashDecoding技术解析" §3.1 does. Splitting P into two
-// bf16 terms keeps ~16 bits of each weight in the P·V product at no visible cost: the tensor
-// pipe is far from busy in this memory-bound loop, and N must be a multiple of 16 anyway.
+// Sᵀ lives in tensor memory, double-buffered; the softmax warps read it with tcgen05.ld and keep
+// the running max m and the running sums l (per key lane) in registers. O accumulates in tensor
+// memory across the item's tiles (one accumulator per item parity) and is rescaled by 2^(m - m')
+// only when the running max grows by more than 2^8, the online softmax of
+// "大语言模型长序列推理优化：ChunkedPrefill与FlashDecoding技术解析" §3.1 with a lazy correction.
+// Splitting P into two bf16 terms keeps ~16 bits of each weight in the P·V product at no visible
+// cost: the tensor pipe is far from busy in this memory-bound loop, and N must be a multiple of
+// 16 anyway.
 //
-// Warp roles: 0-3 softmax / correction / epilogue (one thread per TMEM lane), 4 TMA producer,
-// 5 MMA issuer and TMEM owner. K/V tiles arrive by 4-D TMA with 128-byte swizzle into a 3-stage
-// ring; keys past the sequence end inside the last tile are masked to p = 0 and their V rows are
-// zeroed in shared memory before the P·V product, so stale or poisoned cache rows never leak.
+// Warp roles: 0-3 softmax (one thread per key lane); 4 TMA producer of Q and K; 5 MMA issuer and
+// TMEM owner; 6-9 epilogue (one thread per d lane: O / l, partial or final output); 10 TMA
+// producer of V. K/V tiles arrive by 4-D TMA with 128-byte swizzle into a 3-stage ring whose K
+// and V halves are refilled independently; keys past the sequence end inside the last tile are
+// masked to p = 0 and their V rows are zeroed in shared memory before the P·V product, so stale
+// or poisoned cache rows never leak. The epilogue of an item overlaps the next item's tiles.
 #include "common.cuh"
 #include "internal.h"
 
@@ -29,9 +33,11 @@ namespace {
 constexpr int kTcKeys = 128;           // keys per tile = UMMA M of the Sᵀ product
 constexpr int kTcD = 128;              // head dim = UMMA M of the Oᵀ product
 constexpr int kTcStages = 3;
-constexpr int kTcThreads = 192;
-constexpr int kProducerWarp = 4;
+constexpr int kProducerWarp = 4;     // Q and K
 constexpr int kMmaWarp = 5;
+constexpr int kEpilogueWarp0 = 6;    // warps 6-9; warp w reads TMEM lanes 32 (w mod 4) + [0, 32)
+constexpr int kVProducerWarp = 10;
+constexpr int kTcThreads = 11 * 32;
 constexpr int kSoftmaxThreads = 128;
 constexpr uint32_t kTmemCols = 128;
 constexpr uint32_t kHalfBytes = kTcKeys * 64 * 2;   // one 64-column half of a K or V tile
@@ -45,16 +51,30 @@ struct __align__(1024) TcSmem {
   __nv_bfloat16 q[2][2][16 * 64];                // [item parity][d half], SW128
   __nv_bfloat16 p[2][kPGroups * kTcKeys * 8];    // [tile parity], MN-major core matrices
   float wmax[2][4][GPAD];
-  float lred[4][GPAD];
-  int32_t meta[kTcStages][2];                    // tile start, valid keys
+  // hand-off to the epilogue warps, by item parity
+  float lred[2][4][GPAD];                        // per softmax warp: sum of its key lanes' l
+  float mfin[2][GPAD];                           // final running max
+  int32_t epi[2][4];                             // row (-1: stop), KV head, splits, slot
+  int32_t meta[kTcStages][2];                    // per stage: tile start, valid keys (MMA warp)
   int32_t item_slot[2][2];                       // item index (-1: stop), tiles
   DecodeItem item[2];                            // the item's descriptor (by item parity)
-  uint64_t kfull[kTcStages], vfull[kTcStages], empty[kTcStages];
-  uint64_t qfull[2], qempty[2], sfull[2], sempty[2], pfull[2], pempty[2], ofull[2], oempty[2];
+  // K and V of a stage are released separately: K once the Sᵀ product has read it, V once the
+  // P·V product has, so the next K copy starts while the current tile is still in softmax.
+  uint64_t kfull[kTcStages], vfull[kTcStages], kempty[kTcStages], vempty[kTcStages];
+  uint64_t qfull[2], qempty[2], sfull[2], sempty[2], pfull[2], pempty[2];
+  uint64_t ofull[2];   // by tile parity: that tile's P·V product has completed
+  uint64_t ofin[2];    // by item parity: the item's last P·V product has completed
+  uint64_t oempty[2];  // by item parity: the epilogue has read that item's O accumulator
+  uint64_t lready[2], lfree[2];  // by item parity: hand-off written / read
   uint64_t drain;
   uint32_t tmem_base;
   int abort_flag;
 };
+
+// log2 of the growth of the running maximum that forces a rescale. Below it the weights
+// 2^(x - m) of a tile stay under 2^8, which fp32 sums and the bf16 hi/lo split of P carry
+// without loss, so most tiles skip the exact cross-warp maximum and leave O untouched.
+constexpr float kRescaleThreshold = 8.f;
 
 template <int GPAD>
 __global__ void __launch_bounds__(kTcThreads, 1)
@@ -63,6 +83,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                      const __grid_constant__ CUtensorMap tmap_v) {
   using Smem = TcSmem<GPAD>;
   constexpr int kNO = Smem::kNO;
+  constexpr uint32_t kColO = 32;  // Sᵀ buffers at columns [0, 32), O accumulators after them
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   // dynamic shared memory is only guaranteed 16-byte aligned: round up to 1024 for SW128
   Smem& S = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -74,17 +95,21 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     for (int s = 0; s < kTcStages; ++s) {
       mbar_init(&S.kfull[s], 1);
       mbar_init(&S.vfull[s], 1);
-      mbar_init(&S.empty[s], 1);
+      mbar_init(&S.kempty[s], 1);
+      mbar_init(&S.vempty[s], 1);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&S.qfull[i], 1);
-      mbar_init(&S.qempty[i], 1 + 4);
+      mbar_init(&S.qempty[i], 1 + 4 + 1);  // MMA, softmax warps, V producer
       mbar_init(&S.sfull[i], 1);
       mbar_init(&S.sempty[i], 4);
       mbar_init(&S.pfull[i], 4);
       mbar_init(&S.pempty[i], 1);
       mbar_init(&S.ofull[i], 1);
+      mbar_init(&S.ofin[i], 1);
       mbar_init(&S.oempty[i], 4);
+      mbar_init(&S.lready[i], 4);
+      mbar_init(&S.lfree[i], 4);
     }
     mbar_init(&S.drain, 1);
     S.abort_flag = 0;
@@ -141,22 +166,19 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         for (int j = 0; j < ntile; ++j, ++J) {
           if (j == claim_j) nidx = atomicAdd(&p.hdr->dec_counter, 1);
           const int st = J % kTcStages;
-          if (!mbar_wait(&S.empty[st], ((J / kTcStages) & 1u) ^ 1u, ctx)) { ok = false; break; }
+          const uint32_t free_parity = ((J / kTcStages) & 1u) ^ 1u;
           const int t = it.t0 + j * kTcKeys;
           const int valid = max(0, min(kTcKeys, it.t1 - t));
+          const uint32_t tx = 2u * 128u * static_cast<uint32_t>(p.kv_box_rows);
+          if (!mbar_wait(&S.kempty[st], free_parity, ctx)) { ok = false; break; }
           S.meta[st][0] = t;
           S.meta[st][1] = valid;
           if (valid > 0) {
-            const uint32_t tx = 2u * 128u * static_cast<uint32_t>(p.kv_box_rows);
             mbar_arrive_expect_tx(&S.kfull[st], tx);
             tma_load_4d_stream(S.k[st][0], &tmap_k, &S.kfull[st], 0, t, it.h, it.b, pol);
             tma_load_4d_stream(S.k[st][1], &tmap_k, &S.kfull[st], 64, t, it.h, it.b, pol);
-            mbar_arrive_expect_tx(&S.vfull[st], tx);
-            tma_load_4d_stream(S.v[st][0], &tmap_v, &S.vfull[st], 0, t, it.h, it.b, pol);
-            tma_load_4d_stream(S.v[st][1], &tmap_v, &S.vfull[st], 64, t, it.h, it.b, pol);
           } else {
             mbar_arrive(&S.kfull[st]);
-            mbar_arrive(&S.vfull[st]);
           }
           if (j == read_j && nidx < n_items) nit = p.items[nidx];
         }
@@ -177,6 +199,45 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         for (uint32_t back = 1; back <= kTcStages && back <= J; ++back) {
           const uint32_t jj = J - back;
           mbar_drain(&S.kfull[jj % kTcStages], (jj / kTcStages) & 1u);
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp == kVProducerWarp) {
+    // ======================= TMA producer of V =======================
+    // Follows the items the Q/K producer publishes; a V stage is refilled once the P·V product
+    // of its previous tile has completed, independently of the K half.
+    if (lane == 0) {
+      const uint64_t pol = l2_evict_first_policy();
+      const uint32_t tx = 2u * 128u * static_cast<uint32_t>(p.kv_box_rows);
+      uint32_t J = 0, K = 0;
+      bool ok = true;
+      while (ok) {
+        const int ps = K & 1;
+        if (!mbar_wait(&S.qfull[ps], (K >> 1) & 1u, ctx)) { ok = false; break; }
+        const int idx = S.item_slot[ps][0];
+        const int ntile = S.item_slot[ps][1];
+        const DecodeItem it = S.item[ps];
+        mbar_arrive(&S.qempty[ps]);
+        if (idx < 0) break;
+        for (int j = 0; j < ntile; ++j, ++J) {
+          const int st = J % kTcStages;
+          const int t = it.t0 + j * kTcKeys;
+          const int valid = max(0, min(kTcKeys, it.t1 - t));
+          if (!mbar_wait(&S.vempty[st], ((J / kTcStages) & 1u) ^ 1u, ctx)) { ok = false; break; }
+          if (valid > 0) {
+            mbar_arrive_expect_tx(&S.vfull[st], tx);
+            tma_load_4d_stream(S.v[st][0], &tmap_v, &S.vfull[st], 0, t, it.h, it.b, pol);
+            tma_load_4d_stream(S.v[st][1], &tmap_v, &S.vfull[st], 64, t, it.h, it.b, pol);
+          } else {
+            mbar_arrive(&S.vfull[st]);
+          }
+        }
+        ++K;
+      }
+      if (S.abort_flag) {
+        for (uint32_t back = 1; back <= kTcStages && back <= J; ++back) {
+          const uint32_t jj = J - back;
           mbar_drain(&S.vfull[jj % kTcStages], (jj / kTcStages) & 1u);
         }
       }
@@ -189,26 +250,31 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       const uint32_t idesc_o = idesc_bf16_f32(kTcD, kNO, true, true);
       uint32_t J = 0, K = 0;
       bool ok = true;
+      // the P·V product of a tile is issued after the Sᵀ product of the next one, so the tensor
+      // pipe computes Sᵀ(J + 1) while the softmax warps work on tile J
+      struct Pending { int st, valid; uint32_t jt, item; bool first, last; };
+      Pending prev{};
       bool have_prev = false;
-      int prev_st = 0, prev_valid = 0;
-      uint32_t prev_J = 0;
-      auto issue_pv = [&](int st, int valid, uint32_t jt) -> bool {
-        const int ob = jt & 1;
-        if (!mbar_wait(&S.vfull[st], (jt / kTcStages) & 1u, ctx)) return false;
-        if (!mbar_wait(&S.pfull[ob], (jt >> 1) & 1u, ctx)) return false;
-        if (!mbar_wait(&S.oempty[ob], ((jt >> 1) & 1u) ^ 1u, ctx)) return false;
+      auto issue_pv = [&](const Pending& pv) -> bool {
+        const int pb = pv.jt & 1;
+        const int ob = pv.item & 1;
+        if (!mbar_wait(&S.vfull[pv.st], (pv.jt / kTcStages) & 1u, ctx)) return false;
+        if (!mbar_wait(&S.pfull[pb], (pv.jt >> 1) & 1u, ctx)) return false;
+        // the first product of an item overwrites the accumulator the item two back used
+        if (pv.first && !mbar_wait(&S.oempty[ob], ((pv.item >> 1) & 1u) ^ 1u, ctx)) return false;
         tc_fence_after();
-        const int nk = (valid + 15) / 16;
-        const uint32_t vaddr = smem_u32(S.v[st][0]);
-        const uint32_t paddr = smem_u32(S.p[ob]);
+        const int nk = (pv.valid + 15) / 16;
+        const uint32_t vaddr = smem_u32(S.v[pv.st][0]);
+        const uint32_t paddr = smem_u32(S.p[pb]);
         for (int kk = 0; kk < nk; ++kk) {
           const uint64_t ad = smem_desc(vaddr + kk * 2048, kHalfBytes, 1024, kLayoutSW128);
           const uint64_t bd = smem_desc(paddr + kk * 256, 128, 2048, kLayoutNone);
-          umma_bf16_ss(tmem + 32 + ob * kNO, ad, bd, idesc_o, kk > 0 ? 1u : 0u);
+          umma_bf16_ss(tmem + kColO + ob * kNO, ad, bd, idesc_o, (pv.first && kk == 0) ? 0u : 1u);
         }
-        umma_commit(&S.ofull[ob]);
-        umma_commit(&S.pempty[ob]);
-        umma_commit(&S.empty[st]);
+        umma_commit(&S.ofull[pb]);
+        if (pv.last) umma_commit(&S.ofin[ob]);
+        umma_commit(&S.pempty[pb]);
+        umma_commit(&S.vempty[pv.st]);
         return true;
       };
       while (ok) {
@@ -238,108 +304,130 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             }
           }
           umma_commit(&S.sfull[sb]);
+          umma_commit(&S.kempty[st]);
           if (j == ntile - 1) umma_commit(&S.qempty[ps]);
-          if (have_prev && !issue_pv(prev_st, prev_valid, prev_J)) { ok = false; break; }
+          if (have_prev && !issue_pv(prev)) { ok = false; break; }
           have_prev = true;
-          prev_st = st;
-          prev_valid = valid;
-          prev_J = J;
+          prev = Pending{st, valid, J, K, j == 0, j == ntile - 1};
         }
         if (!ok) break;
         ++K;
       }
-      if (ok && have_prev) ok = issue_pv(prev_st, prev_valid, prev_J);
+      if (ok && have_prev) ok = issue_pv(prev);
       // every MMA this thread issued has completed once `drain` flips
       umma_commit(&S.drain);
       mbar_drain(&S.drain, 0);
     }
     __syncwarp();
-  } else {
-    // ======================= softmax / correction / epilogue =======================
+  } else if (warp < 4) {
+    // ======================= softmax and O correction =======================
+    // A timed-out wait never makes one of these warps leave on its own: the others would wait
+    // for it at a named barrier, which has no time limit. Each warp notes the failure in `ok`,
+    // skips the work that depended on the wait and keeps meeting the barriers; the barriers
+    // themselves vote on the failure, so all four warps leave at the same point.
     const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
-    float m[GPAD], lp[GPAD], oacc[GPAD], alpha_prev[GPAD];
+    float m[GPAD], lp[GPAD];
     uint32_t J = 0, K = 0;
     bool ok = true;
-    auto accumulate = [&](uint32_t jt, int valid, const float* a) -> bool {
-      const int ob = jt & 1;
-      if (!mbar_wait(&S.ofull[ob], (jt >> 1) & 1u, ctx)) return false;
-      tc_fence_after();
-      float hi[GPAD], lo[GPAD];
-      if (valid > 0) {
-        if constexpr (kNO == 16) {
-          uint32_t r[16];
-          tmem_ld16(tmem + lane_base + 32 + ob * kNO, r);
-          tmem_wait_ld();
-#pragma unroll
-          for (int g = 0; g < GPAD; ++g) { hi[g] = __uint_as_float(r[g]); lo[g] = __uint_as_float(r[GPAD + g]); }
-        } else {
-          uint32_t r[32];
-          tmem_ld32(tmem + lane_base + 32 + ob * kNO, r);
-          tmem_wait_ld();
-#pragma unroll
-          for (int g = 0; g < GPAD; ++g) { hi[g] = __uint_as_float(r[g]); lo[g] = __uint_as_float(r[GPAD + g]); }
-        }
-      } else {
-#pragma unroll
-        for (int g = 0; g < GPAD; ++g) { hi[g] = 0.f; lo[g] = 0.f; }
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&S.oempty[ob]);
-#pragma unroll
-      for (int g = 0; g < GPAD; ++g) oacc[g] = fmaf(oacc[g], a[g], hi[g] + lo[g]);
-      return true;
+    // O of the current item (thread = d lane): columns [0, GPAD) the P_hi part, [GPAD, 2 GPAD)
+    // the P_lo part
+    auto load_o = [&](uint32_t ob, uint32_t (&r)[kNO]) {
+      if constexpr (kNO == 16) tmem_ld16(tmem + lane_base + kColO + ob * kNO, r);
+      else tmem_ld32(tmem + lane_base + kColO + ob * kNO, r);
+      tmem_wait_ld();
     };
-    while (ok) {
+    for (;;) {
       const int ps = K & 1;
-      if (!mbar_wait(&S.qfull[ps], (K >> 1) & 1u, ctx)) break;
+      ok = ok && mbar_wait(&S.qfull[ps], (K >> 1) & 1u, ctx);
+      if (named_bar_or(1, kSoftmaxThreads, !ok)) break;
       const int idx = S.item_slot[ps][0];
       const int ntile = S.item_slot[ps][1];
       const DecodeItem it = S.item[ps];
       __syncwarp();
       if (lane == 0) mbar_arrive(&S.qempty[ps]);
-      if (idx < 0) break;
+      const uint32_t ob = K & 1;
+      if (idx < 0) {
+        // tell the epilogue warps to stop
+        if (mbar_wait(&S.lfree[ob], ((K >> 1) & 1u) ^ 1u, ctx)) {
+          if (tid == 0) S.epi[ob][0] = -1;
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&S.lready[ob]);
+        }
+        break;
+      }
 #pragma unroll
-      for (int g = 0; g < GPAD; ++g) { m[g] = -INFINITY; lp[g] = 0.f; oacc[g] = 0.f; alpha_prev[g] = 1.f; }
-      int prev_valid = 0;
+      for (int g = 0; g < GPAD; ++g) { m[g] = -INFINITY; lp[g] = 0.f; }
+      bool abort_item = false;
       for (int j = 0; j < ntile; ++j, ++J) {
         const int st = J % kTcStages;
         const int sb = J & 1;
-        if (!mbar_wait(&S.sfull[sb], (J >> 1) & 1u, ctx)) { ok = false; break; }
-        // the stage's metadata was published with the producer's arrival on kfull
-        if (!mbar_wait(&S.kfull[st], (J / kTcStages) & 1u, ctx)) { ok = false; break; }
+        ok = ok && mbar_wait(&S.sfull[sb], (J >> 1) & 1u, ctx);
         tc_fence_after();
-        const int valid = S.meta[st][1];
+        // Keys of this tile, from the item descriptor. (Not from the stage's kfull barrier: K is
+        // released as soon as Sᵀ has read it, so kfull may already be a phase further on.)
+        const int valid = max(0, min(kTcKeys, it.t1 - (it.t0 + j * kTcKeys)));
         uint32_t sr[16];
-        if (valid > 0) {
+        if (ok && valid > 0) {
           tmem_ld16(tmem + lane_base + sb * 16, sr);
           tmem_wait_ld();
         }
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&S.sempty[sb]);
+        if (lane == 0 && ok) mbar_arrive(&S.sempty[sb]);
 
-        const bool in = tid < valid;
+        const bool in = ok && tid < valid;
         float x[GPAD];
+        bool grow = false;
 #pragma unroll
-        for (int g = 0; g < GPAD; ++g)
+        for (int g = 0; g < GPAD; ++g) {
           x[g] = (in && g < p.g) ? __uint_as_float(sr[g]) * p.scale_log2 : -INFINITY;
-#pragma unroll
-        for (int g = 0; g < GPAD; ++g) {
-          const float wm = warp_max_f32(x[g]);
-          if (lane == 0) S.wmax[sb][warp][g] = wm;
+          grow |= x[g] > m[g] + kRescaleThreshold;
         }
-        named_bar_sync(1, kSoftmaxThreads);
-        float alpha[GPAD], pr[GPAD];
+        // One barrier per tile, which also tells every thread whether any key of the tile lies
+        // more than the threshold above the running maximum (always so on an item's first tile)
+        // or whether a wait has failed.
+        if (named_bar_or(1, kSoftmaxThreads, grow || !ok)) {
+          // exact new maximum over the 128 keys, per query head
+#pragma unroll
+          for (int g = 0; g < GPAD; ++g) {
+            const float wm = warp_max_f32(x[g]);
+            if (lane == 0) S.wmax[sb][warp][g] = wm;
+          }
+          if (named_bar_or(1, kSoftmaxThreads, !ok)) { abort_item = true; break; }
+          float alpha[GPAD];
+#pragma unroll
+          for (int g = 0; g < GPAD; ++g) {
+            const float tmx = fmaxf(fmaxf(S.wmax[sb][0][g], S.wmax[sb][1][g]),
+                                    fmaxf(S.wmax[sb][2][g], S.wmax[sb][3][g]));
+            const float mn = fmaxf(m[g], tmx);
+            alpha[g] = (m[g] == -INFINITY) ? 0.f : fast_exp2(m[g] - mn);
+            lp[g] *= alpha[g];
+            m[g] = mn;
+          }
+          if (j > 0) {
+            // O holds the item's earlier tiles: wait for the last of their products, scale it
+            const uint32_t jp = J - 1;
+            ok = ok && mbar_wait(&S.ofull[jp & 1], (jp >> 1) & 1u, ctx);
+            tc_fence_after();
+            if (ok) {
+              uint32_t o[kNO];
+              load_o(ob, o);
+#pragma unroll
+              for (int g = 0; g < GPAD; ++g) {
+                o[g] = __float_as_uint(__uint_as_float(o[g]) * alpha[g]);
+                o[GPAD + g] = __float_as_uint(__uint_as_float(o[GPAD + g]) * alpha[g]);
+              }
+              if constexpr (kNO == 16) tmem_st16(tmem + lane_base + kColO + ob * kNO, o);
+              else tmem_st32(tmem + lane_base + kColO + ob * kNO, o);
+              tmem_wait_st();
+            }
+          }
+        }
+        float pr[GPAD];
 #pragma unroll
         for (int g = 0; g < GPAD; ++g) {
-          const float tmx = fmaxf(fmaxf(S.wmax[sb][0][g], S.wmax[sb][1][g]),
-                                  fmaxf(S.wmax[sb][2][g], S.wmax[sb][3][g]));
-          const float mn = fmaxf(m[g], tmx);
-          alpha[g] = (mn == -INFINITY) ? 1.f : fast_exp2(m[g] - mn);
-          pr[g] = (mn == -INFINITY) ? 0.f : fast_exp2(x[g] - mn);
-          lp[g] = fmaf(lp[g], alpha[g], pr[g]);
-          m[g] = mn;
+          pr[g] = (m[g] == -INFINITY) ? 0.f : fast_exp2(x[g] - m[g]);
+          lp[g] += pr[g];
         }
         // P_hi / P_lo for this key lane
         uint32_t hw[GPAD / 2], lw[GPAD / 2];
@@ -351,13 +439,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           hw[g / 2] = *reinterpret_cast<const uint32_t*>(&h2);
           lw[g / 2] = *reinterpret_cast<const uint32_t*>(&l2);
         }
-        if (!mbar_wait(&S.pempty[sb], ((J >> 1) & 1u) ^ 1u, ctx)) { ok = false; break; }
+        ok = ok && mbar_wait(&S.pempty[sb], ((J >> 1) & 1u) ^ 1u, ctx);
         if ((valid & 15) != 0) {
           // zero V rows [valid, next multiple of 16): they may lie past the sequence end
-          if (!mbar_wait(&S.vfull[st], (J / kTcStages) & 1u, ctx)) { ok = false; break; }
+          ok = ok && mbar_wait(&S.vfull[st], (J / kTcStages) & 1u, ctx);
           const int r0 = valid, r1 = (valid + 15) & ~15;
           const int nchunks = (r1 - r0) * 2 * 8;
-          for (int c = tid; c < nchunks; c += kSoftmaxThreads) {
+          for (int c = tid; ok && c < nchunks; c += kSoftmaxThreads) {
             const int row = r0 + c / 16;
             const int half = (c / 8) & 1;
             const int ch = c & 7;
@@ -365,54 +453,92 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 make_uint4(0u, 0u, 0u, 0u);
           }
         }
-        unsigned char* pb = reinterpret_cast<unsigned char*>(S.p[sb]);
+        if (ok) {
+          unsigned char* pb = reinterpret_cast<unsigned char*>(S.p[sb]);
 #pragma unroll
-        for (int grp = 0; grp < GPAD / 8; ++grp) {
-          *reinterpret_cast<uint4*>(pb + grp * 2048 + tid * 16) =
-              make_uint4(hw[grp * 4 + 0], hw[grp * 4 + 1], hw[grp * 4 + 2], hw[grp * 4 + 3]);
-          *reinterpret_cast<uint4*>(pb + (GPAD / 8 + grp) * 2048 + tid * 16) =
-              make_uint4(lw[grp * 4 + 0], lw[grp * 4 + 1], lw[grp * 4 + 2], lw[grp * 4 + 3]);
+          for (int grp = 0; grp < GPAD / 8; ++grp) {
+            *reinterpret_cast<uint4*>(pb + grp * 2048 + tid * 16) =
+                make_uint4(hw[grp * 4 + 0], hw[grp * 4 + 1], hw[grp * 4 + 2], hw[grp * 4 + 3]);
+            *reinterpret_cast<uint4*>(pb + (GPAD / 8 + grp) * 2048 + tid * 16) =
+                make_uint4(lw[grp * 4 + 0], lw[grp * 4 + 1], lw[grp * 4 + 2], lw[grp * 4 + 3]);
+          }
         }
         fence_proxy_async_smem();
+        tc_fence_before();  // orders a rescale's tcgen05.st before the P·V product
         __syncwarp();
-        if (lane == 0) mbar_arrive(&S.pfull[sb]);
-        if (j > 0 && !accumulate(J - 1, prev_valid, alpha_prev)) { ok = false; break; }
-#pragma unroll
-        for (int g = 0; g < GPAD; ++g) alpha_prev[g] = alpha[g];
-        prev_valid = valid;
+        if (lane == 0 && ok) mbar_arrive(&S.pfull[sb]);
       }
-      if (!ok) break;
-      if (!accumulate(J - 1, prev_valid, alpha_prev)) break;
+      if (abort_item) break;
 
-      // ---- epilogue: l = sum over key lanes; O = acc / l ----
+      // ---- hand the item to the epilogue warps: per-warp sums of l, the running max ----
+      ok = ok && mbar_wait(&S.lfree[ob], ((K >> 1) & 1u) ^ 1u, ctx);
 #pragma unroll
       for (int g = 0; g < GPAD; ++g) {
-        const float s = warp_sum_f32(lp[g]);
-        if (lane == 0) S.lred[warp][g] = s;
+        const float sum = warp_sum_f32(lp[g]);
+        if (lane == 0 && ok) S.lred[ob][warp][g] = sum;
       }
-      named_bar_sync(1, kSoftmaxThreads);
-      const bool direct = it.nsplit == 1;
-      const int64_t slot = direct ? 0 : static_cast<int64_t>(it.slot);
+      if (tid == 0 && ok) {
+#pragma unroll
+        for (int g = 0; g < GPAD; ++g) S.mfin[ob][g] = m[g];
+        S.epi[ob][0] = it.row;
+        S.epi[ob][1] = it.h;
+        S.epi[ob][2] = it.nsplit;
+        S.epi[ob][3] = it.slot;
+      }
+      __syncwarp();
+      if (lane == 0 && ok) mbar_arrive(&S.lready[ob]);
+      ++K;
+    }
+  } else {
+    // ======================= epilogue: O = (O_hi + O_lo) / l =======================
+    // Runs while the softmax warps already work on the next item; its O accumulator is the other
+    // item parity's, so the two never touch the same columns.
+    const int quad = warp & 3;
+    const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
+    const int d = quad * 32 + lane;
+    for (uint32_t K = 0;; ++K) {
+      const uint32_t ob = K & 1;
+      if (!mbar_wait(&S.lready[ob], (K >> 1) & 1u, ctx)) break;
+      const int row = S.epi[ob][0];
+      if (row < 0) break;
+      const int h = S.epi[ob][1];
+      const bool direct = S.epi[ob][2] == 1;
+      const int64_t slot = direct ? 0 : static_cast<int64_t>(S.epi[ob][3]);
+      float mf[GPAD], l[GPAD];
+#pragma unroll
+      for (int g = 0; g < GPAD; ++g) {
+        mf[g] = S.mfin[ob][g];
+        l[g] = S.lred[ob][0][g] + S.lred[ob][1][g] + S.lred[ob][2][g] + S.lred[ob][3][g];
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&S.lfree[ob]);
+      if (!mbar_wait(&S.ofin[ob], (K >> 1) & 1u, ctx)) break;
+      tc_fence_after();
+      uint32_t o[kNO];
+      if constexpr (kNO == 16) tmem_ld16(tmem + lane_base + kColO + ob * kNO, o);
+      else tmem_ld32(tmem + lane_base + kColO + ob * kNO, o);
+      tmem_wait_ld();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&S.oempty[ob]);
 #pragma unroll
       for (int g = 0; g < GPAD; ++g) {
         if (g < p.g) {
-          const float l = S.lred[0][g] + S.lred[1][g] + S.lred[2][g] + S.lred[3][g];
-          const float ov = l > 0.f ? oacc[g] / l : 0.f;
-          const float lse2 = l > 0.f ? m[g] + log2f(l) : -INFINITY;
-          const int hq = it.h * p.g + g;
+          const float acc = __uint_as_float(o[g]) + __uint_as_float(o[GPAD + g]);
+          const float ov = l[g] > 0.f ? acc / l[g] : 0.f;
+          const float lse2 = l[g] > 0.f ? mf[g] + log2f(l[g]) : -INFINITY;
+          const int hq = h * p.g + g;
           if (direct) {
             __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out) +
-                                 static_cast<int64_t>(it.row) * p.o_sr + static_cast<int64_t>(hq) * p.o_sh;
-            out[tid] = __float2bfloat16_rn(ov);
-            if (tid == 0) p.lse[static_cast<int64_t>(it.row) * p.hq + hq] = lse2 * kLn2;
+                                 static_cast<int64_t>(row) * p.o_sr + static_cast<int64_t>(hq) * p.o_sh;
+            out[d] = __float2bfloat16_rn(ov);
+            if (d == 0) p.lse[static_cast<int64_t>(row) * p.hq + hq] = lse2 * kLn2;
           } else {
-            p.part_o[(slot * p.g + g) * kTcD + tid] = ov;
-            if (tid == 0) p.part_lse[slot * p.g + g] = lse2;
+            p.part_o[(slot * p.g + g) * kTcD + d] = ov;
+            if (d == 0) p.part_lse[slot * p.g + g] = lse2;
           }
         }
       }
-      named_bar_sync(1, kSoftmaxThreads);
-      ++K;
     }
   }
 
