@@ -4,8 +4,9 @@
 Default workload: decode GQA bf16, Llama-3-70B-like shape (batch 32, 64 query / 8 KV heads,
 head_dim 128, cache lengths uniform in [1024, 32768], capacity 32768, planner splits). One step is
 one fd_decode_attention call (device planner + split kernel + LSE combine) over resident inputs.
+Workload 5 (mixed chunked-prefill step) times one fd_chunk_prefill_attention call instead.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl fd|reference] [--workload 1-4]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl fd|reference] [--workload 1-5]
 
 Prints one JSON line on rank 0. `value` is the whole-job GB/s: the algorithmic bytes every rank
 processed (K+V bytes of the valid keys plus the Q bytes) over the slowest rank's device time.
@@ -33,6 +34,7 @@ sys.path.insert(0, ROOT)
 
 METRIC = "decode-attn µs/call and achieved HBM GB/s vs 8 TB/s peak (Llama-3-70B GQA)"
 FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
 L2_BYTES = 126 * 1024 * 1024
 
 
@@ -42,7 +44,7 @@ def parse_args():
     ap.add_argument("--steps", type=int, default=3000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["fd", "reference"], default="fd")
-    ap.add_argument("--workload", type=int, default=3, choices=[1, 2, 3, 4])
+    ap.add_argument("--workload", type=int, default=3, choices=[1, 2, 3, 4, 5])
     ap.add_argument("--batch", type=int, default=None, help="batch of the long-context workload")
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--profile-calls", type=int, default=200,
@@ -58,22 +60,52 @@ def log(*a):
     print(*a, file=sys.stderr, flush=True)
 
 
+def is_chunk(inp) -> bool:
+    return hasattr(inp, "q_chunk")
+
+
+def key_lens(inp):
+    """Valid keys per request: cache_lens, or prefix + chunk for a chunked-prefill step."""
+    cap = inp.k_cache.shape[2]
+    if is_chunk(inp):
+        raw = [int(p) + int(c) for p, c in zip(inp.prefix_lens.tolist(), inp.chunk_lens.tolist())]
+    else:
+        raw = inp.cache_lens.tolist()
+    return [max(0, min(int(x), cap)) for x in raw]
+
+
+def queries(inp):
+    return inp.q_chunk if is_chunk(inp) else inp.q
+
+
 def algorithmic_bytes(inp) -> int:
     """K+V bytes of the valid keys (each read once) plus the Q bytes."""
     B, hkv, cap, d = inp.k_cache.shape
     es = inp.k_cache.element_size()
-    lens = [max(0, min(int(x), cap)) for x in inp.cache_lens.tolist()]
-    return 2 * sum(lens) * hkv * d * es + inp.q.numel() * inp.q.element_size()
+    q = queries(inp)
+    return 2 * sum(key_lens(inp)) * hkv * d * es + q.numel() * q.element_size()
 
 
-def measured_peak():
+def chunk_tile_flops(inp) -> int:
+    """Algorithmic FLOPs of the chunked-prefill tile rows (chunk_len > 1): per (row, query head),
+    2 D for q.k and 2 D for p.v per visible key; row i of a request sees prefix + i + 1 keys."""
+    cap = inp.k_cache.shape[2]
+    hq, d = inp.q_chunk.shape[1], inp.q_chunk.shape[2]
+    keys = 0
+    for p, c in zip(inp.prefix_lens.tolist(), inp.chunk_lens.tolist()):
+        if int(c) > 1:
+            keys += sum(min(int(p) + i + 1, cap) for i in range(int(c)))
+    return 4 * d * hq * keys
+
+
+def measured_peak(key: str = "hbm_gbs"):
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
         with open(path) as f:
             j = json.load(f)
-        return float(j["hbm_gbs"]), "measured"
+        return float(j[key]), "measured"
     except Exception:
-        return FALLBACK_HBM_GBS, "fallback"
+        return (FALLBACK_HBM_GBS if key == "hbm_gbs" else FALLBACK_BF16_TFLOPS), "fallback"
 
 
 def kernel_source_sha(name: str) -> str:
@@ -167,33 +199,46 @@ def cpu_threads() -> int:
 
 
 def oracle_sample(inp, seconds: float, seed: int = 0):
-    """Time the oracle on whole (b, KV head) groups of the workload, in a seeded order, until
-    `seconds` of host time are spent. Returns (bytes/s, description, groups, elapsed)."""
+    """Time the oracle on whole (query row, KV head) groups of the workload, all G query heads
+    each, in a seeded order, until `seconds` of host time are spent.
+    Returns (bytes/s, description, groups, elapsed)."""
     from oracle import attention as oracle
     from workloads import to_numpy_exact
-    q = to_numpy_exact(inp.q)
+    q = to_numpy_exact(queries(inp))
     k = to_numpy_exact(inp.k_cache)
     v = to_numpy_exact(inp.v_cache)
-    B, hq, d = q.shape
+    R, hq, d = q.shape
     hkv = k.shape[1]
     g = hq // hkv
-    lens = inp.cache_lens.tolist()
     es = inp.k_cache.element_size()
-    order = np.random.default_rng(seed).permutation(B * hkv)
+    vis = []
+    if is_chunk(inp):
+        prefix, chunk = inp.prefix_lens.tolist(), inp.chunk_lens.tolist()
+        cap = k.shape[2]
+        for p, c in zip(prefix, chunk):
+            vis.extend(min(int(p) + i + 1, cap) for i in range(int(c)))
+
+        def run(rows):
+            oracle.chunk_prefill_attention(q, k, v, prefix, chunk, rows=rows)
+    else:
+        lens = inp.cache_lens.tolist()
+        vis = key_lens(inp)
+
+        def run(rows):
+            oracle.decode_attention(q, k, v, lens, rows=rows)
+    order = np.random.default_rng(seed).permutation(R * hkv)
     done, nbytes = 0, 0
     t0 = time.perf_counter()
     for idx in order:
-        b, h = divmod(int(idx), hkv)
-        rows = [(b, h * g + j) for j in range(g)]
-        oracle.decode_attention(q, k, v, lens, rows=rows)
-        n = max(0, min(int(lens[b]), k.shape[2]))
-        nbytes += 2 * n * d * es + g * d * inp.q.element_size()
+        r, h = divmod(int(idx), hkv)
+        run([(r, h * g + j) for j in range(g)])
+        nbytes += 2 * vis[r] * d * es + g * d * queries(inp).element_size()
         done += 1
         if time.perf_counter() - t0 >= seconds:
             break
     el = time.perf_counter() - t0
-    desc = (f"{done} of {B * hkv} (batch, KV head) groups of the workload, all {g} query heads "
-            f"each, seeded order; float64 numpy")
+    desc = (f"{done} of {R * hkv} (query row, KV head) groups of the workload, all {g} query "
+            f"heads each, seeded order; float64 numpy")
     return nbytes / el, desc, done, el
 
 
@@ -231,7 +276,7 @@ def run_reference(args, rank, world):
         "config": {"workload": inp.name},
         "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": cpu_threads(),
                          "kind": "oracle",
-                         "sample": f"per step: whole (batch, KV head) groups of the workload in a "
+                         "sample": f"per step: whole (query row, KV head) groups of the workload in a "
                                    f"seeded order until {per_step:.2f}s of host time (or all groups)"},
         "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
@@ -245,24 +290,39 @@ def run_fd(args, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
     inp = load_workload(args)
+    chunk = is_chunk(inp)
     alg = algorithmic_bytes(inp)
-    B, hq, d = inp.q.shape
-    hkv = inp.k_cache.shape[1]
+    R, hq, d = queries(inp).shape
+    B, hkv = inp.k_cache.shape[:2]
     g = hq // hkv
-    q = inp.q.to(dev)
+    q = queries(inp).to(dev)
     k = inp.k_cache.to(dev)
     v = inp.v_cache.to(dev)
-    lens = inp.cache_lens.to(dev)
+    if chunk:
+        lens_h = [inp.prefix_lens, inp.chunk_lens]
+    else:
+        lens_h = [inp.cache_lens]
+    lens = [t.to(dev) for t in lens_h]
     out = torch.empty_like(q)
-    lse = torch.empty((B, hq), dtype=torch.float32, device=dev)
+    lse = torch.empty((R, hq), dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev)
-    ns = inp.num_splits
+    ns = 0 if chunk else inp.num_splits
     input_bytes = sum(t.numel() * t.element_size() for t in (q, k, v))
     l2_policy = ("inputs larger than L2 (valid K/V bytes per call exceed the 126 MB L2)"
                  if alg > 2 * L2_BYTES else "inputs smaller than L2: measured with warm L2")
+    use_tc = inp.k_cache.dtype == torch.bfloat16 and d == 128 and 2 <= g <= 16
+    if chunk:
+        # planner, decode-row split kernel, chunk tile kernel, combine
+        launches_per_step = 4
 
-    def step():
-        fd.fd_decode_attention(q, k, v, lens, ns, out=out, lse=lse, stream=stream)
+        def step():
+            fd.fd_chunk_prefill_attention(q, k, v, lens[0], lens[1], out=out, lse=lse, stream=stream)
+    else:
+        # planner, split kernel and, after the tensor-core split kernel, the combine kernel
+        launches_per_step = 3 if use_tc else 2
+
+        def step():
+            fd.fd_decode_attention(q, k, v, lens[0], ns, out=out, lse=lse, stream=stream)
 
     for _ in range(max(3, args.warmup)):
         step()
@@ -295,39 +355,66 @@ def run_fd(args, rank, world, local_rank):
 
     # ---- per-kernel durations (same calls, with events between the launches) ----
     nprof = min(args.steps, args.profile_calls)
-    prof = [(float("nan"),) * 3]
+    prof = [(float("nan"),) * 4]
     if nprof > 0:
         fd.fd_profile_begin(nprof)
         for _ in range(nprof):
             step()
         torch.cuda.synchronize()
         prof = fd.fd_profile_end(nprof)
+
     def _mean(i):
-        v = statistics.mean(p[i] for p in prof)
-        return None if v != v else v
-    plan_ms, split_ms, comb_ms = _mean(0), _mean(1), _mean(2)
-    peak, peak_kind = measured_peak()
-    use_tc = inp.q.dtype == torch.bfloat16 and d == 128 and 2 <= g <= 16
+        x = statistics.mean(p[i] for p in prof)
+        return None if x != x else x
+    plan_ms, split_ms, tile_ms, comb_ms = _mean(0), _mean(1), _mean(2), _mean(3)
+    peak, peak_kind = measured_peak("hbm_gbs")
     kfile = "decode_tc.cu" if use_tc else "decode_simt.cu"
-    achieved = alg / (split_ms * 1e-3) / 1e9 if split_ms else None
+    split_bytes = alg
+    if chunk:
+        # the decode-row split kernel streams the decode rows' K/V; the tile kernel the rest
+        dec_keys = sum(n for n, c in zip(key_lens(inp), inp.chunk_lens.tolist()) if int(c) == 1)
+        split_bytes = 2 * dec_keys * hkv * d * inp.k_cache.element_size()
+    achieved = split_bytes / (split_ms * 1e-3) / 1e9 if split_ms else None
+    roofline = {"bound": "hbm", "kernel": kfile.replace(".cu", "_kernel"),
+                "achieved": round(achieved, 1) if achieved else None, "peak": peak,
+                "unit": "GB/s", "frac": round(achieved / peak, 4) if achieved else None,
+                "peak_kind": f"{peak_kind} copy bandwidth",
+                "algorithmic_bytes_per_launch": split_bytes,
+                "traffic": traffic_from_profiles(kfile, inp.name),
+                "kernel_ms": {k_: (round(x, 5) if x is not None else None) for k_, x in
+                              (("planner", plan_ms), ("split", split_ms),
+                               ("chunk_tiles", tile_ms), ("combine", comb_ms))}}
+    roofline_tiles = None
+    if chunk and tile_ms:
+        flops = chunk_tile_flops(inp)
+        tpeak, tkind = measured_peak("bf16_tflops")
+        ach = flops / (tile_ms * 1e-3) / 1e12
+        roofline_tiles = {"bound": "tensor", "kernel": "chunk_tc_kernel", "achieved": round(ach, 2),
+                          "peak": tpeak, "unit": "TFLOP/s", "frac": round(ach / tpeak, 4),
+                          "peak_kind": f"{tkind} dense bf16 (burst)",
+                          "algorithmic_flops_per_launch": flops,
+                          "traffic": traffic_from_profiles("chunk_tc.cu", inp.name)}
+        if tile_ms > split_ms:
+            roofline, roofline_tiles = roofline_tiles, roofline
 
     # ---- end to end: host buffers, copies inside the timed region ----
     e2e = None
     if args.e2e_steps > 0:
-        hq_ = inp.q.pin_memory()
+        hq_ = queries(inp).pin_memory()
         hk = inp.k_cache.pin_memory()
         hv = inp.v_cache.pin_memory()
-        hl = inp.cache_lens.pin_memory()
-        ho = torch.empty_like(inp.q).pin_memory()
-        hlse = torch.empty((B, hq), dtype=torch.float32).pin_memory()
-        h2d = sum(x.numel() * x.element_size() for x in (hq_, hk, hv, hl))
+        hl = [t.pin_memory() for t in lens_h]
+        ho = torch.empty_like(queries(inp)).pin_memory()
+        hlse = torch.empty((R, hq), dtype=torch.float32).pin_memory()
+        h2d = sum(x.numel() * x.element_size() for x in [hq_, hk, hv] + hl)
         d2h = ho.numel() * ho.element_size() + hlse.numel() * 4
 
         def e2e_step():
             q.copy_(hq_, non_blocking=True)
             k.copy_(hk, non_blocking=True)
             v.copy_(hv, non_blocking=True)
-            lens.copy_(hl, non_blocking=True)
+            for dst, src in zip(lens, hl):
+                dst.copy_(src, non_blocking=True)
             step()
             ho.copy_(out, non_blocking=True)
             hlse.copy_(lse, non_blocking=True)
@@ -358,31 +445,30 @@ def run_fd(args, rank, world, local_rank):
                "kind": "oracle", "sample": f"{desc}; {el:.1f}s"}
 
     if rank == 0:
+        config = {"workload": inp.name, "batch": B, "q_heads": hq, "kv_heads": hkv,
+                  "head_dim": d, "cache_capacity": int(inp.k_cache.shape[2]),
+                  "sum_key_len": int(sum(key_lens(inp))),
+                  "num_splits": "planner" if ns == 0 else ns,
+                  "algorithmic_bytes_per_call": alg, "input_bytes_resident": input_bytes,
+                  "l2": l2_policy, "parallelism": f"replicas x{world}"}
+        if chunk:
+            config["chunk_rows"] = int(R)
+            config["chunk_tile_flops_per_call"] = chunk_tile_flops(inp)
         line = {
             "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
             "steps": args.steps, "warmup": max(3, args.warmup),
             "ms_per_step": round(ms_per_step, 5), "us_per_call": round(ms_per_step * 1e3, 2),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16"
-            if inp.q.dtype == torch.bfloat16 else "f32", "data": "synthetic",
-            "config": {"workload": inp.name, "batch": B, "q_heads": hq, "kv_heads": hkv,
-                       "head_dim": d, "cache_capacity": int(inp.k_cache.shape[2]),
-                       "sum_cache_len": int(sum(inp.cache_lens.tolist())),
-                       "num_splits": "planner" if ns == 0 else ns,
-                       "algorithmic_bytes_per_call": alg, "input_bytes_resident": input_bytes,
-                       "l2": l2_policy, "parallelism": f"replicas x{world}"},
-            "roofline": {"bound": "hbm", "kernel": kfile.replace(".cu", "_kernel"),
-                         "achieved": round(achieved, 1) if achieved else None, "peak": peak,
-                         "unit": "GB/s", "frac": round(achieved / peak, 4) if achieved else None,
-                         "peak_kind": f"{peak_kind} copy bandwidth",
-                         "traffic": traffic_from_profiles(kfile, inp.name),
-                         "kernel_ms": {k: (round(v, 5) if v is not None else None) for k, v in
-                                       (("planner", plan_ms), ("split", split_ms),
-                                        ("combine", comb_ms))}},
+            if inp.k_cache.dtype == torch.bfloat16 else "f32", "data": "synthetic",
+            "config": config,
+            "roofline": roofline,
             "clocks": clocks,
             "e2e": e2e,
-            "gpu_launches": 3 * args.steps,
+            "gpu_launches": launches_per_step * args.steps,
             "cpu_baseline": cpu,
         }
+        if roofline_tiles is not None:
+            line["roofline_secondary"] = roofline_tiles
         print(json.dumps(line), flush=True)
     return 0
 

@@ -238,9 +238,10 @@ fd_status fd_poll_status(void* stream, uint32_t* flags);
 
 /* Kernel timing for measurement. fd_profile_begin(n) makes the next n attention calls record a
  * CUDA event before and after each of their kernel launches; fd_profile_end synchronises and
- * writes, per profiled call, the milliseconds of its [planner, split/tile kernels, combine]
- * launches into ms[3*i + 0..2] (ms has room for 3*max_calls floats) and the call count into
- * *n_calls. Profiling adds event records between launches; it is off by default. */
+ * writes, per profiled call, the milliseconds of its [planner, decode split kernel, chunk tile
+ * kernel, combine] launches into ms[4*i + 0..3] (ms has room for 4*max_calls floats; a segment
+ * a call does not launch reads about 0) and the call count into *n_calls. Profiling adds event
+ * records between launches, which also keeps them from overlapping; it is off by default. */
 fd_status fd_profile_begin(int32_t max_calls);
 fd_status fd_profile_end(float* ms, int32_t max_calls, int32_t* n_calls);
 

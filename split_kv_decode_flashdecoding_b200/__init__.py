@@ -261,12 +261,12 @@ def fd_profile_begin(max_calls: int) -> None:
     _check(lib.fd_profile_begin(int(max_calls)), "fd_profile_begin")
 
 
-def fd_profile_end(max_calls: int) -> List[Tuple[float, float, float]]:
-    """Per profiled call: (planner ms, split kernels ms, combine ms)."""
-    ms = (ctypes.c_float * (3 * max_calls))()
+def fd_profile_end(max_calls: int) -> List[Tuple[float, float, float, float]]:
+    """Per profiled call: (planner ms, decode split ms, chunk tile ms, combine ms)."""
+    ms = (ctypes.c_float * (4 * max_calls))()
     n = c_i32(0)
     _check(lib.fd_profile_end(ms, int(max_calls), ctypes.byref(n)), "fd_profile_end")
-    return [(ms[3 * i], ms[3 * i + 1], ms[3 * i + 2]) for i in range(n.value)]
+    return [tuple(ms[4 * i + j] for j in range(4)) for i in range(n.value)]
 
 
 def fd_shutdown() -> None:

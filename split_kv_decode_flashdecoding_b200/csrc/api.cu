@@ -149,19 +149,23 @@ fd_status make_tmap(CUtensorMap* map, const void* base, int rank, const uint64_t
 }
 
 // ---------------------------------------------------------------------------- profiling ------
+// Per profiled call: events around the planner, the decode split kernel, the chunk tile kernel
+// (nothing for a decode call) and the combine kernel.
+constexpr int kProfSegments = 4;
+constexpr int kProfEvents = kProfSegments + 1;
 struct Profiler {
   std::mutex mu;
-  std::vector<cudaEvent_t> ev;  // 4 per call
+  std::vector<cudaEvent_t> ev;  // kProfEvents per call
   int max_calls = 0;
   int calls = 0;
   bool active = false;
 } g_prof;
 
-// Returns the 4 events of the next profiled call, or nullptr.
+// Returns the events of the next profiled call, or nullptr.
 cudaEvent_t* prof_next() {
   std::lock_guard<std::mutex> lock(g_prof.mu);
   if (!g_prof.active || g_prof.calls >= g_prof.max_calls) return nullptr;
-  return &g_prof.ev[4 * static_cast<size_t>(g_prof.calls++)];
+  return &g_prof.ev[kProfEvents * static_cast<size_t>(g_prof.calls++)];
 }
 
 // ---------------------------------------------------------------------------- validation -----
@@ -502,9 +506,23 @@ fd_status fd_decode_attention(const fd_tensor* q, const fd_tensor* k_cache,
   cp.dtype = sh.dtype;
 
 
+  // The tensor-core kernel plans small batches itself (every CTA computes the plan in shared
+  // memory, CTA 0 writes the combine's row tables): no planner launch, no items in memory.
+  const bool fused_plan = sh.use_tc && sh.B <= kFusedPlanMaxBatch;
+  if (fused_plan) {
+    dp.items = nullptr;
+    dp.lens = cache_lens;
+    dp.B = sh.B;
+    dp.fixed = num_splits;
+    dp.plan_ctas = nctas;
+    dp.max_items = static_cast<int32_t>(std::min<int64_t>(max_items, INT32_MAX));
+    dp.row_nsplit_out = row_nsplit;
+    dp.row_base_out = row_base;
+  }
+
   cudaEvent_t* ev = prof_next();
   end_profile_events(ev, 0, stream);
-  FD_CUDA(launch_plan_decode(pp, stream), "plan kernel launch");
+  if (!fused_plan) FD_CUDA(launch_plan_decode(pp, stream), "plan kernel launch");
   end_profile_events(ev, 1, stream);
   if (sh.use_tc) {
     FD_CUDA(launch_decode_tc(dp, tq, tk, tv, nctas, stream), "tensor-core split kernel launch");
@@ -512,10 +530,11 @@ fd_status fd_decode_attention(const fd_tensor* q, const fd_tensor* k_cache,
     FD_CUDA(launch_decode_simt(dp, sh.dtype, nctas, stream), "split kernel launch");
   }
   end_profile_events(ev, 2, stream);
+  end_profile_events(ev, 3, stream);  // no chunk tiles in a decode call
   // the CUDA-core kernel merges each group's partials itself; the tensor-core kernel leaves them
   // to the combine kernel
   if (sh.use_tc) FD_CUDA(launch_combine(cp, stream), "combine kernel launch");
-  end_profile_events(ev, 3, stream);
+  end_profile_events(ev, 4, stream);
   return FD_OK;
 }
 
@@ -676,10 +695,11 @@ fd_status fd_chunk_prefill_attention(const fd_tensor* q_chunk, const fd_tensor* 
   } else {
     FD_CUDA(launch_decode_simt(dp, FD_BF16, dec_ctas, stream), "decode-row split kernel launch");
   }
-  FD_CUDA(launch_chunk_tc(tp, tq_tile, tk, tv, tile_ctas, stream), "chunk tile kernel launch");
   end_profile_events(ev, 2, stream);
-  FD_CUDA(launch_combine(cp, stream), "combine kernel launch");
+  FD_CUDA(launch_chunk_tc(tp, tq_tile, tk, tv, tile_ctas, stream), "chunk tile kernel launch");
   end_profile_events(ev, 3, stream);
+  FD_CUDA(launch_combine(cp, stream), "combine kernel launch");
+  end_profile_events(ev, 4, stream);
   return FD_OK;
 }
 
@@ -727,7 +747,7 @@ fd_status fd_profile_begin(int32_t max_calls) {
   if (max_calls < 1) return fail(FD_ERR_INVALID_ARGUMENT, "max_calls must be >= 1");
   std::lock_guard<std::mutex> lock(g_prof.mu);
   for (cudaEvent_t e : g_prof.ev) cudaEventDestroy(e);
-  g_prof.ev.assign(4 * static_cast<size_t>(max_calls), nullptr);
+  g_prof.ev.assign(kProfEvents * static_cast<size_t>(max_calls), nullptr);
   for (auto& e : g_prof.ev) FD_CUDA(cudaEventCreate(&e), "cudaEventCreate");
   g_prof.max_calls = max_calls;
   g_prof.calls = 0;
@@ -741,9 +761,10 @@ fd_status fd_profile_end(float* ms, int32_t max_calls, int32_t* n_calls) {
   if (!g_prof.active) return fail(FD_ERR_INVALID_ARGUMENT, "profiling was not started");
   const int n = std::min(g_prof.calls, max_calls);
   for (int i = 0; i < n; ++i) {
-    cudaEvent_t* e = &g_prof.ev[4 * static_cast<size_t>(i)];
-    FD_CUDA(cudaEventSynchronize(e[3]), "cudaEventSynchronize");
-    for (int j = 0; j < 3; ++j) FD_CUDA(cudaEventElapsedTime(&ms[3 * i + j], e[j], e[j + 1]), "cudaEventElapsedTime");
+    cudaEvent_t* e = &g_prof.ev[kProfEvents * static_cast<size_t>(i)];
+    FD_CUDA(cudaEventSynchronize(e[kProfSegments]), "cudaEventSynchronize");
+    for (int j = 0; j < kProfSegments; ++j)
+      FD_CUDA(cudaEventElapsedTime(&ms[kProfSegments * i + j], e[j], e[j + 1]), "cudaEventElapsedTime");
   }
   *n_calls = n;
   for (cudaEvent_t e : g_prof.ev) cudaEventDestroy(e);

@@ -92,6 +92,17 @@ __device__ __forceinline__ void mbar_drain(uint64_t* bar, uint32_t parity) {
   }
 }
 
+// Called by one thread per CTA once the CTA has made its last claim on the work cursor `counter`:
+// the CTA that arrives last puts the cursor and the arrival count back to zero, so every call
+// starts from zero without a separate reset.
+__device__ __forceinline__ void release_work_cursor(int32_t* counter, int32_t* exits) {
+  __threadfence();
+  if (atomicAdd(exits, 1) == static_cast<int>(gridDim.x) - 1) {
+    atomicExch(counter, 0);
+    atomicExch(exits, 0);
+  }
+}
+
 // ---- named barriers (a subset of the CTA's warps) -----------------------------------------------
 
 __device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t nthreads) {

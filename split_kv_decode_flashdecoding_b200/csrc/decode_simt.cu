@@ -172,6 +172,7 @@ __global__ void __launch_bounds__(kSimtThreads) decode_simt_kernel(DecodeParams 
       if (mbar_wait(&S.empty[st], ((J / kSimtStages) & 1u) ^ 1u, ctx)) {
         S.meta[st][0] = -1;
         mbar_arrive(&S.full[st]);
+        release_work_cursor(&p.hdr->dec_counter, &p.hdr->dec_exit);
         return;
       }
     }
@@ -180,6 +181,7 @@ __global__ void __launch_bounds__(kSimtThreads) decode_simt_kernel(DecodeParams 
       const uint32_t jj = J - back;
       mbar_drain(&S.full[jj % kSimtStages], (jj / kSimtStages) & 1u);
     }
+    release_work_cursor(&p.hdr->dec_counter, &p.hdr->dec_exit);
     return;
   }
 

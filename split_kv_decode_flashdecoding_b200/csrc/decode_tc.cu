@@ -56,6 +56,13 @@ struct __align__(1024) TcSmem {
   float mfin[2][GPAD];                           // final running max
   int32_t epi[2][4];                             // row (-1: stop), KV head, splits, slot
   int32_t meta[kTcStages][2];                    // per stage: tile start, valid keys (MMA warp)
+  // in-kernel plan: lengths, split counts, rank order, partial-slot bases (row order) and item
+  // offsets (rank order, B + 1 entries)
+  int32_t plan_len[kFusedPlanMaxBatch], plan_n[kFusedPlanMaxBatch];
+  int32_t plan_order[kFusedPlanMaxBatch], plan_rbase[kFusedPlanMaxBatch];
+  int32_t plan_ioff[kFusedPlanMaxBatch + 1];
+  long long plan_red[kTcThreads / 32];
+  int32_t plan_clamped;
   int32_t item_slot[2][2];                       // item index (-1: stop), tiles
   DecodeItem item[2];                            // the item's descriptor (by item parity)
   // K and V of a stage are released separately: K once the Sᵀ product has read it, V once the
@@ -70,6 +77,35 @@ struct __align__(1024) TcSmem {
   uint32_t tmem_base;
   int abort_flag;
 };
+
+// dynamic shared memory per CTA, plus the 1024 bytes of alignment slack the kernel may use
+static_assert(sizeof(TcSmem<8>) + 1024 <= 227 * 1024, "tensor-core decode smem (G <= 8)");
+static_assert(sizeof(TcSmem<16>) + 1024 <= 227 * 1024, "tensor-core decode smem (G <= 16)");
+
+// Exclusive prefix sum over i < n (n <= 32 * 8 here) by one warp: out[i] = sum_{j<i} val(j),
+// out[n] = the total.
+template <typename F>
+__device__ __forceinline__ void warp_exclusive_scan(int n, F val, int32_t* out) {
+  const int lane = threadIdx.x & 31;
+  const int per = (n + 31) / 32;
+  const int lo = lane * per;
+  int32_t local = 0;
+  for (int i = 0; i < per; ++i)
+    if (lo + i < n) local += val(lo + i);
+  int32_t incl = local;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  int32_t run = incl - local;
+  for (int i = 0; i < per; ++i)
+    if (lo + i < n) {
+      out[lo + i] = run;
+      run += val(lo + i);
+    }
+  if (lane == 31) out[n] = incl;
+}
 
 // log2 of the growth of the running maximum that forces a rescale. Below it the weights
 // 2^(x - m) of a tile stay under 2^8, which fp32 sums and the bf16 hi/lo split of P carry
@@ -129,15 +165,100 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   tc_fence_after();
   const uint32_t tmem = S.tmem_base;
   const WaitCtx ctx{&S.abort_flag, &p.hdr->status};
-  // Everything above overlapped the planner (programmatic dependent launch); the plan it wrote
-  // is read below. The combine kernel may launch now: it waits for this grid the same way.
+  const bool fused = p.items == nullptr;
+  if (fused) {
+    // ---- the split plan, computed by every CTA in shared memory (the planner's arithmetic):
+    // clamped lengths and their sum, the chunk size, split counts, longest-first ranks, item
+    // offsets in rank order and partial-slot bases in row order. Only the lengths are read from
+    // global memory; they are an input of this call, so this may run before the wait below.
+    const int B = p.B;
+    long long local = 0;
+    bool clamped = false;
+    for (int b = tid; b < B; b += kTcThreads) {
+      const int32_t raw = p.lens[b];
+      const int32_t L = clamp_len(raw, p.cap);
+      clamped |= L != raw;
+      S.plan_len[b] = L;
+      local += L;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) local += __shfl_xor_sync(0xffffffffu, local, o);
+    clamped = __any_sync(0xffffffffu, clamped);
+    if (lane == 0) S.plan_red[warp] = local;
+    if (tid == 0) S.plan_clamped = 0;
+    __syncthreads();
+    if (lane == 0 && clamped) S.plan_clamped = 1;
+    long long total = 0;
+#pragma unroll
+    for (int w = 0; w < kTcThreads / 32; ++w) total += S.plan_red[w];
+    const int32_t chunk = p.fixed > 0 ? 0 : plan_chunk_tokens(total, p.hkv, p.plan_ctas);
+    for (int b = tid; b < B; b += kTcThreads) {
+      const int32_t n = plan_num_splits(S.plan_len[b], chunk, p.fixed);
+      S.plan_n[b] = n;
+      S.plan_ioff[b] = plan_sort_key(S.plan_len[b], n);  // sort keys until the scan below
+    }
+    __syncthreads();
+    // longest first: rank = sequences with a larger key, or an equal key and a smaller index
+    for (int b = tid; b < B; b += kTcThreads) {
+      const int32_t kb = S.plan_ioff[b];
+      int r = 0;
+      for (int j = 0; j < B; ++j) {
+        const int32_t kj = S.plan_ioff[j];
+        r += (kj > kb || (kj == kb && j < b)) ? 1 : 0;
+      }
+      S.plan_order[r] = b;
+    }
+    __syncthreads();
+    if (warp == 0)
+      warp_exclusive_scan(B, [&](int r) { return S.plan_n[S.plan_order[r]] * p.hkv; }, S.plan_ioff);
+    else if (warp == 1)
+      warp_exclusive_scan(B, [&](int b) { return S.plan_n[b]; }, S.plan_rbase);
+    __syncthreads();
+  }
+  // Everything above overlapped the kernel before this one (programmatic dependent launch);
+  // workspace and outputs are touched only below. The combine kernel may launch now: it waits
+  // for this grid the same way.
   pdl_wait_prerequisites();
   pdl_launch_dependents();
+  const int32_t fused_items = fused ? S.plan_ioff[p.B] : 0;
+  const bool fused_overflow = fused && fused_items > p.max_items;
+  if (fused && blockIdx.x == 0) {
+    // the combine kernel's row tables, and the status flags the planner would raise
+    for (int b = tid; b < p.B; b += kTcThreads) {
+      p.row_nsplit_out[b] = S.plan_n[b];
+      p.row_base_out[b] = S.plan_rbase[b];
+    }
+    if (tid == 0 && S.plan_clamped) atomicOr(&p.hdr->status, FD_FLAG_LEN_CLAMPED);
+    if (tid == 0 && fused_overflow) atomicOr(&p.hdr->status, FD_FLAG_PLAN_OVERFLOW);
+  }
+  // item idx of the in-kernel plan: sequence of rank r (largest r with ioff[r] <= idx), then
+  // KV head and split, exactly as the planner lays items out
+  auto fused_item = [&](int idx) {
+    int lo = 0, hi = p.B;
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (S.plan_ioff[mid] <= idx) lo = mid; else hi = mid;
+    }
+    const int b = S.plan_order[lo];
+    const int n = S.plan_n[b];
+    const int local = idx - S.plan_ioff[lo];
+    const int h = local / n, s = local - h * n;
+    DecodeItem it;
+    it.row = b;
+    it.b = b;
+    it.h = h;
+    it.split = s;
+    plan_split_range(S.plan_len[b], n, s, p.fixed, &it.t0, &it.t1);
+    it.nsplit = n;
+    it.slot = S.plan_rbase[b] * p.hkv + h * n + s;
+    return it;
+  };
 
   if (warp == kProducerWarp) {
     // ======================= TMA producer =======================
     if (lane == 0) {
-      const int n_items = *reinterpret_cast<volatile int32_t*>(&p.hdr->num_dec_items);
+      const int n_items = fused ? (fused_overflow ? 0 : fused_items)
+                                : *reinterpret_cast<volatile int32_t*>(&p.hdr->num_dec_items);
       const uint64_t pol = l2_evict_first_policy();
       uint32_t J = 0, K = 0;
       bool ok = true;
@@ -148,7 +269,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       // tail short (a CTA never sits on an item it cannot start soon).
       int idx = atomicAdd(&p.hdr->dec_counter, 1);
       DecodeItem it{};
-      if (idx < n_items) it = p.items[idx];
+      if (idx < n_items) it = fused ? fused_item(idx) : p.items[idx];
       while (ok && idx < n_items) {
         int nidx = n_items;
         DecodeItem nit{};
@@ -180,7 +301,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           } else {
             mbar_arrive(&S.kfull[st]);
           }
-          if (j == read_j && nidx < n_items) nit = p.items[nidx];
+          if (j == read_j && nidx < n_items) nit = fused ? fused_item(nidx) : p.items[nidx];
         }
         ++K;
         idx = nidx;
@@ -546,6 +667,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   __syncthreads();
   tc_fence_after();
   if (warp == kMmaWarp) tmem_dealloc(tmem, kTmemCols);
+  if (tid == 0) release_work_cursor(&p.hdr->dec_counter, &p.hdr->dec_exit);
 }
 
 template <int GPAD>

@@ -46,11 +46,17 @@ struct DecodeParams {
   int32_t kv_box_rows;  // rows of one K/V tensor-map box (tensor-core kernel): min(128, S_cap)
   float scale_log2;  // softmax scale * log2(e)
   WsHeader* hdr;
-  const DecodeItem* items;
+  const DecodeItem* items;  // planner output; nullptr: the tensor-core kernel plans itself
   const int32_t* row_base;
   float* part_o;     // [slots, G, D], the slots of one (row, KV head) group consecutive
   float* part_lse;   // [slots, G] (log2 domain)
   int32_t* arrivals; // [rows, Hkv] split-completion counters of the in-kernel merge
+  // in-kernel plan (items == nullptr, tensor-core kernel, B <= kFusedPlanMaxBatch): the inputs of
+  // the planner and the row tables the combine kernel reads
+  const int32_t* lens;
+  int32_t B, fixed, plan_ctas, max_items;
+  int32_t* row_nsplit_out;
+  int32_t* row_base_out;
 };
 
 __device__ __forceinline__ MergeTarget merge_target(const DecodeParams& p) {

@@ -29,6 +29,7 @@ constexpr int32_t kWaves = 8;             // target work items per persistent CT
 constexpr int32_t kQTile = 128;           // chunked-prefill query rows per tile
 constexpr int32_t kChunkKvSplit = 2048;   // keys per split of a chunked-prefill query tile
 constexpr int32_t kMaxPlanBatch = 4096;   // largest batch the one-CTA device planner accepts
+constexpr int32_t kFusedPlanMaxBatch = 256;  // largest batch the tensor-core split kernel plans itself
 
 // One split of one (sequence, KV head): keys [t0, t1) of cache row b, output row `row`.
 struct DecodeItem {
@@ -61,9 +62,12 @@ struct WsHeader {
   uint32_t status;          // FD_FLAG_* bits, sticky until fd_poll_status
   int32_t num_dec_items;    // decode items planned by the last call
   int32_t num_tile_items;   // tile items planned by the last call
-  int32_t dec_counter;      // dynamic scheduler cursor (reset by the planner every call)
+  int32_t dec_counter;      // dynamic scheduler cursor: zero between calls (the planner zeroes
+                            // it; the tensor-core split kernel's last CTA zeroes it on exit)
   int32_t tile_counter;
-  int32_t pad[59];
+  int32_t dec_exit;         // CTAs of the tensor-core split kernel that have finished (zero
+                            // between calls)
+  int32_t pad[58];
 };
 static_assert(sizeof(WsHeader) == 256, "WsHeader is 256 bytes");
 

@@ -218,3 +218,57 @@ def test_cuda_graph_replay_new_lengths():
         check_out(out, ro)
         check_lse(lse, rl)
     del g
+
+
+@pytest.mark.parametrize("B", [255, 256, 257])
+def test_batch_around_in_kernel_plan_limit(B):
+    # up to 256 sequences the tensor-core kernel plans the call itself; above, the planner kernel
+    # does: both must give the oracle's result
+    rng = np.random.default_rng(900 + B)
+    lens = [int(x) for x in rng.integers(0, 321, size=B)]
+    inp = make_decode_inputs(B, 16, 2, 128, 320, lens, torch.bfloat16, seed=900 + B,
+                             pad_fill=NAN)
+    out, lse = _run(inp)
+    rows = sample_rows(B, 16, 48, seed=B, must=[(0, 0), (B - 1, 15), (B // 2, 7)])
+    ro, rl = _oracle(inp, rows=rows)
+    check_out(out, ro, "out")
+    check_lse(lse, rl, "lse")
+
+
+def test_paths_share_workspace_cursor():
+    # CUDA-core, tensor-core and chunked-prefill calls on one stream share one workspace and its
+    # work cursor; every kernel that claims from the cursor leaves it at zero for the next call
+    fd = _fd()
+    from workloads import make_chunk_inputs
+    dev = torch.device("cuda", 0)
+    mha = make_decode_inputs(3, 8, 8, 128, 700, [700, 3, 333], torch.bfloat16, seed=71,
+                             pad_fill=NAN)
+    gqa = make_decode_inputs(4, 64, 8, 128, 1500, [1500, 17, 900, 256], torch.bfloat16, seed=72,
+                             pad_fill=NAN)
+    chk = make_chunk_inputs([400, 90], [140, 1], 8, 2, 128, 600, torch.bfloat16, seed=73,
+                            pad_fill=NAN)
+    s = torch.cuda.Stream()
+
+    def chunk_call():
+        q = chk.q_chunk.to(dev)
+        out, lse = fd.fd_chunk_prefill_attention(q, chk.k_cache.to(dev), chk.v_cache.to(dev),
+                                                 chk.prefix_lens.to(dev), chk.chunk_lens.to(dev),
+                                                 stream=s)
+        torch.cuda.synchronize()
+        ro, rl = oracle.chunk_prefill_attention(
+            to_numpy_exact(chk.q_chunk), to_numpy_exact(chk.k_cache), to_numpy_exact(chk.v_cache),
+            chk.prefix_lens.tolist(), chk.chunk_lens.tolist())
+        check_out(out, ro, "chunk out")
+        check_lse(lse, rl, "chunk lse")
+
+    def decode_call(inp):
+        with torch.cuda.stream(s):
+            out, lse = _run(inp, stream=s)
+        ro, rl = _oracle(inp)
+        check_out(out, ro, "out")
+        check_lse(lse, rl, "lse")
+
+    for step in (lambda: decode_call(mha), lambda: decode_call(gqa), chunk_call,
+                 lambda: decode_call(gqa), lambda: decode_call(mha), lambda: decode_call(gqa)):
+        step()
+    assert fd.fd_poll_status(stream=s) & (fd.FD_FLAG_WAIT_TIMEOUT | fd.FD_FLAG_PLAN_OVERFLOW) == 0
