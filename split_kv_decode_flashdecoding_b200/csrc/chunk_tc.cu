@@ -13,16 +13,18 @@
 //   O[128 x 128] += P_hi · V_tile + P_lo · V_tile      UMMA M=128 N=128, A from TMEM, V MN-major
 //
 // S is double-buffered in TMEM and P is written back over the S buffer it came from (per
-// 32-key chunk: 16 words of hi pairs, then 16 words of lo pairs, so a chunk's writes only cover
-// columns already read), so P is double-buffered too; O has one buffer. The reference maximum m
-// moves only when a row's maximum grows by more than 2^8, so O (in TMEM) is rescaled rarely —
-// only then does the softmax wait for the previous P·V product; p <= 2^8 is exact enough in
-// fp32 and in the hi/lo split.
-// At the end of the split the row's O / l and LSE = m + log2 l are written: the final output
-// when the tile has a single split, else a partial for the combine kernel.
+// 32-key chunk: 16 words of hi pairs, then 16 words of lo pairs), so P is double-buffered too; O
+// has one accumulator per item parity, so an item's epilogue overlaps the next item's tiles. The
+// reference maximum m moves only when a row's maximum grows by more than 2^8, so O is rescaled
+// rarely — only then does the softmax wait for the previous P·V product; p <= 2^8 is exact enough
+// in fp32 and in the hi/lo split. At the end of the split the epilogue writes O / l and
+// LSE = m + log2 l: the final output when the tile has a single split, else a partial for the
+// combine kernel.
 //
-// Warp roles as in the decode kernel: 0-3 softmax / epilogue (thread = TMEM lane = query row),
-// 4 TMA producer (K/V tiles through a 2-stage ring, the next item's Q prefetched), 5 MMA issuer.
+// Warp roles: 0-3 softmax (thread = TMEM lane = query row); 4 TMA producer of Q and K (2-stage
+// K ring, the next item's Q prefetched); 5 MMA issuer and TMEM owner; 6-9 epilogue (warp w reads
+// TMEM lanes 32 (w mod 4) + [0, 32)); 10 TMA producer of V (2-stage ring). K and V stages are
+// released separately: K once S has read it, V once P·V has.
 #include "common.cuh"
 #include "internal.h"
 
@@ -33,34 +35,41 @@ namespace {
 constexpr int kCkRows = 128;   // query rows per tile = UMMA M
 constexpr int kCkKeys = 128;   // keys per key tile = N of S, K of P·V
 constexpr int kCkD = 128;      // head dim = K of S, N of P·V
-constexpr int kCkStages = 2;
-constexpr int kCkThreads = 192;
-constexpr int kCkProducer = 4;
+constexpr int kCkKStages = 2;
+constexpr int kCkVStages = 2;
+constexpr int kCkProducer = 4;     // Q and K
 constexpr int kCkMma = 5;
-constexpr int kCkSoftmax = 128;
+constexpr int kCkVProducer = 10;
+constexpr int kCkThreads = 11 * 32;
 constexpr uint32_t kCkTmemCols = 512;
-constexpr uint32_t kColS0 = 0, kColO = 256;   // S/P buffers at 0 and 128, O at 256
-constexpr uint32_t kCkHalf = kCkRows * 64 * 2;              // one 64-column half of a 128-row tile
-constexpr float kRescaleThreshold = 8.0f;                   // log2 units
+constexpr uint32_t kColS0 = 0, kColO0 = 256;   // S/P buffers at 0 and 128, O at 256 and 384
+constexpr uint32_t kCkHalf = kCkRows * 64 * 2;  // one 64-column half of a 128-row tile
+constexpr float kRescaleThreshold = 8.0f;       // log2 units
 
 struct __align__(1024) CkSmem {
-  __nv_bfloat16 q[2][2][kCkRows * 64];          // [item parity][d half], SW128
-  __nv_bfloat16 k[kCkStages][2][kCkKeys * 64];  // [stage][d half], SW128
-  __nv_bfloat16 v[kCkStages][2][kCkKeys * 64];
-  int32_t meta[kCkStages][2];                   // key tile start, valid keys
-  int32_t item_slot[2][2];                      // item index (-1: stop), key tiles
+  __nv_bfloat16 q[2][2][kCkRows * 64];           // [item parity][d half], SW128
+  __nv_bfloat16 k[kCkKStages][2][kCkKeys * 64];  // [stage][d half], SW128
+  __nv_bfloat16 v[kCkVStages][2][kCkKeys * 64];
+  int32_t meta[kCkKStages];                      // valid keys of the K stage (MMA warp)
+  int32_t item_slot[2][2];                       // item index (-1: stop), key tiles
   TileItem item[2];
-  uint64_t kfull[kCkStages], vfull[kCkStages], empty[kCkStages];
-  uint64_t qfull[2], qempty[2], sfull[2], sempty[2];
-  // P(J) ready, one barrier per tile parity: with a single barrier of four warp arrivals a fast
-  // warp could arrive for tile J+1 before a slow one arrived for tile J and complete the phase
-  // early; on pfull[J & 1] its next arrival needs S(J+2), which needs P·V(J), which needs the
-  // whole phase of tile J.
+  // hand-off to the epilogue warps, by item parity: per-row running max and sum, the item
+  float mfin[2][kCkRows], lfin[2][kCkRows];
+  TileItem epi[2];
+  int32_t epi_stop[2];
+  uint64_t kfull[kCkKStages], kempty[kCkKStages], vfull[kCkVStages], vempty[kCkVStages];
+  uint64_t qfull[2], qempty[2], sfull[2];
+  uint64_t sfree[2];   // S/P buffer free again: the P·V product that read its P has completed
+  // P(J) ready, one barrier per tile parity: a fast warp's next arrival on pfull[J & 1] is for
+  // tile J + 2, whose S needs P·V(J), which needs the whole phase of tile J
   uint64_t pfull[2];
-  uint64_t pfree, ofin, oempty, drain;
+  uint64_t pfree;      // every P·V product (the softmax waits for the previous one to rescale O)
+  uint64_t ofin[2], oempty[2], lready[2], lfree[2];  // by item parity
+  uint64_t drain;
   uint32_t tmem_base;
   int abort_flag;
 };
+static_assert(sizeof(CkSmem) + 1024 <= 227 * 1024, "chunk tile kernel shared memory");
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
   const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
@@ -78,22 +87,26 @@ __global__ void __launch_bounds__(kCkThreads, 1)
   const int lane = tid & 31;
 
   if (tid == 0) {
-    for (int s = 0; s < kCkStages; ++s) {
+    for (int s = 0; s < kCkKStages; ++s) {
       mbar_init(&S.kfull[s], 1);
+      mbar_init(&S.kempty[s], 1);
+    }
+    for (int s = 0; s < kCkVStages; ++s) {
       mbar_init(&S.vfull[s], 1);
-      mbar_init(&S.empty[s], 1);
+      mbar_init(&S.vempty[s], 1);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&S.qfull[i], 1);
-      mbar_init(&S.qempty[i], 1 + 4);
+      mbar_init(&S.qempty[i], 1 + 4 + 1);  // MMA, softmax warps, V producer
       mbar_init(&S.sfull[i], 1);
-      mbar_init(&S.sempty[i], 1);
+      mbar_init(&S.sfree[i], 1);
+      mbar_init(&S.pfull[i], 4);
+      mbar_init(&S.ofin[i], 1);
+      mbar_init(&S.oempty[i], 4);
+      mbar_init(&S.lready[i], 4);
+      mbar_init(&S.lfree[i], 4);
     }
-    mbar_init(&S.pfull[0], 4);
-    mbar_init(&S.pfull[1], 4);
     mbar_init(&S.pfree, 1);
-    mbar_init(&S.ofin, 1);
-    mbar_init(&S.oempty, 4);
     mbar_init(&S.drain, 1);
     S.abort_flag = 0;
     fence_mbar_init();
@@ -114,9 +127,10 @@ __global__ void __launch_bounds__(kCkThreads, 1)
   const WaitCtx ctx{&S.abort_flag, &p.hdr->status};
   pdl_wait_prerequisites();
   pdl_launch_dependents();
+  const uint32_t kv_tx = 2u * 128u * static_cast<uint32_t>(p.kv_box_rows);
 
   if (warp == kCkProducer) {
-    // ======================= TMA producer =======================
+    // ======================= TMA producer of Q and K =======================
     if (lane == 0) {
       const int n_items = *reinterpret_cast<volatile int32_t*>(&p.hdr->num_tile_items);
       const uint64_t pol = l2_evict_first_policy();
@@ -142,23 +156,17 @@ __global__ void __launch_bounds__(kCkThreads, 1)
         const int hkv = it.h / p.g;
         for (int j = 0; j < ntile; ++j, ++J) {
           if (j == claim_j) nidx = atomicAdd(&p.hdr->tile_counter, 1);
-          const int st = J % kCkStages;
-          if (!mbar_wait(&S.empty[st], ((J / kCkStages) & 1u) ^ 1u, ctx)) { ok = false; break; }
+          const int st = J % kCkKStages;
+          if (!mbar_wait(&S.kempty[st], ((J / kCkKStages) & 1u) ^ 1u, ctx)) { ok = false; break; }
           const int t = it.k0 + j * kCkKeys;
           const int valid = max(0, min(kCkKeys, it.k1 - t));
-          S.meta[st][0] = t;
-          S.meta[st][1] = valid;
+          S.meta[st] = valid;
           if (valid > 0) {
-            const uint32_t tx = 2u * 128u * static_cast<uint32_t>(p.kv_box_rows);
-            mbar_arrive_expect_tx(&S.kfull[st], tx);
+            mbar_arrive_expect_tx(&S.kfull[st], kv_tx);
             tma_load_4d_stream(S.k[st][0], &tmap_k, &S.kfull[st], 0, t, hkv, it.b, pol);
             tma_load_4d_stream(S.k[st][1], &tmap_k, &S.kfull[st], 64, t, hkv, it.b, pol);
-            mbar_arrive_expect_tx(&S.vfull[st], tx);
-            tma_load_4d_stream(S.v[st][0], &tmap_v, &S.vfull[st], 0, t, hkv, it.b, pol);
-            tma_load_4d_stream(S.v[st][1], &tmap_v, &S.vfull[st], 64, t, hkv, it.b, pol);
           } else {
             mbar_arrive(&S.kfull[st]);
-            mbar_arrive(&S.vfull[st]);
           }
           if (j == read_j && nidx < n_items) nit = p.tiles[nidx];
         }
@@ -175,10 +183,47 @@ __global__ void __launch_bounds__(kCkThreads, 1)
         }
       }
       if (S.abort_flag) {
-        for (uint32_t back = 1; back <= kCkStages && back <= J; ++back) {
+        for (uint32_t back = 1; back <= kCkKStages && back <= J; ++back) {
           const uint32_t jj = J - back;
-          mbar_drain(&S.kfull[jj % kCkStages], (jj / kCkStages) & 1u);
-          mbar_drain(&S.vfull[jj % kCkStages], (jj / kCkStages) & 1u);
+          mbar_drain(&S.kfull[jj % kCkKStages], (jj / kCkKStages) & 1u);
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp == kCkVProducer) {
+    // ======================= TMA producer of V =======================
+    if (lane == 0) {
+      const uint64_t pol = l2_evict_first_policy();
+      uint32_t J = 0, K = 0;
+      bool ok = true;
+      while (ok) {
+        const int ps = K & 1;
+        if (!mbar_wait(&S.qfull[ps], (K >> 1) & 1u, ctx)) { ok = false; break; }
+        const int idx = S.item_slot[ps][0];
+        const int ntile = S.item_slot[ps][1];
+        const TileItem it = S.item[ps];
+        mbar_arrive(&S.qempty[ps]);
+        if (idx < 0) break;
+        const int hkv = it.h / p.g;
+        for (int j = 0; j < ntile; ++j, ++J) {
+          const int st = J % kCkVStages;
+          if (!mbar_wait(&S.vempty[st], ((J / kCkVStages) & 1u) ^ 1u, ctx)) { ok = false; break; }
+          const int t = it.k0 + j * kCkKeys;
+          const int valid = max(0, min(kCkKeys, it.k1 - t));
+          if (valid > 0) {
+            mbar_arrive_expect_tx(&S.vfull[st], kv_tx);
+            tma_load_4d_stream(S.v[st][0], &tmap_v, &S.vfull[st], 0, t, hkv, it.b, pol);
+            tma_load_4d_stream(S.v[st][1], &tmap_v, &S.vfull[st], 64, t, hkv, it.b, pol);
+          } else {
+            mbar_arrive(&S.vfull[st]);
+          }
+        }
+        ++K;
+      }
+      if (S.abort_flag) {
+        for (uint32_t back = 1; back <= kCkVStages && back <= J; ++back) {
+          const uint32_t jj = J - back;
+          mbar_drain(&S.vfull[jj % kCkVStages], (jj / kCkVStages) & 1u);
         }
       }
     }
@@ -190,32 +235,35 @@ __global__ void __launch_bounds__(kCkThreads, 1)
       const uint32_t idesc_o = idesc_bf16_f32(kCkRows, kCkD, false, true);
       uint32_t J = 0, K = 0;
       bool ok = true;
+      // the P·V product of a tile is issued after the S product of the next one
+      struct Pending { int valid; uint32_t jt, item; bool first, last; };
+      Pending prev{};
       bool have_prev = false;
-      int prev_st = 0, prev_valid = 0;
-      bool prev_first = false, prev_last = false;
-      uint32_t prev_J = 0, prev_K = 0;
-      auto issue_pv = [&](int st, int valid, uint32_t jt, bool first, bool last, uint32_t kt) -> bool {
-        if (!mbar_wait(&S.vfull[st], (jt / kCkStages) & 1u, ctx)) return false;
-        if (!mbar_wait(&S.pfull[jt & 1], (jt >> 1) & 1u, ctx)) return false;
-        // the item's first product overwrites O: the previous item's O must have been read
-        if (first && kt > 0 && !mbar_wait(&S.oempty, (kt - 1) & 1u, ctx)) return false;
+      auto issue_pv = [&](const Pending& pv) -> bool {
+        const int vs = pv.jt % kCkVStages;
+        const int ob = pv.item & 1;
+        if (!mbar_wait(&S.vfull[vs], (pv.jt / kCkVStages) & 1u, ctx)) return false;
+        if (!mbar_wait(&S.pfull[pv.jt & 1], (pv.jt >> 1) & 1u, ctx)) return false;
+        // the item's first product overwrites the accumulator the item two back used
+        if (pv.first && !mbar_wait(&S.oempty[ob], ((pv.item >> 1) & 1u) ^ 1u, ctx)) return false;
         tc_fence_after();
-        const int nk = (valid + 15) / 16;
-        const uint32_t vaddr = smem_u32(S.v[st][0]);
-        const uint32_t pcol = kColS0 + (jt & 1) * 128;  // P of this tile, over its S buffer
-        bool acc = !first;
+        const int nk = (pv.valid + 15) / 16;
+        const uint32_t vaddr = smem_u32(S.v[vs][0]);
+        const uint32_t pcol = kColS0 + (pv.jt & 1) * 128;  // P of this tile, over its S buffer
+        const uint32_t ocol = kColO0 + ob * 128;
+        bool acc = !pv.first;
         for (int part = 0; part < 2; ++part) {
           for (int kk = 0; kk < nk; ++kk) {
             const uint64_t bd = smem_desc(vaddr + kk * 2048, kCkHalf, 1024, kLayoutSW128);
             const uint32_t acol = pcol + 32 * (kk >> 1) + 16 * part + 8 * (kk & 1);
-            umma_bf16_ts(tmem + kColO, tmem + acol, bd, idesc_o, acc ? 1u : 0u);
+            umma_bf16_ts(tmem + ocol, tmem + acol, bd, idesc_o, acc ? 1u : 0u);
             acc = true;
           }
         }
         umma_commit(&S.pfree);
-        umma_commit(&S.sempty[jt & 1]);
-        umma_commit(&S.empty[st]);
-        if (last) umma_commit(&S.ofin);
+        umma_commit(&S.sfree[pv.jt & 1]);
+        umma_commit(&S.vempty[vs]);
+        if (pv.last) umma_commit(&S.ofin[ob]);
         return true;
       };
       while (ok) {
@@ -227,12 +275,12 @@ __global__ void __launch_bounds__(kCkThreads, 1)
         const uint32_t q0 = smem_u32(S.q[ps][0]);
         const uint32_t q1 = smem_u32(S.q[ps][1]);
         for (int j = 0; j < ntile; ++j, ++J) {
-          const int st = J % kCkStages;
+          const int st = J % kCkKStages;
           const int sb = J & 1;
-          if (!mbar_wait(&S.kfull[st], (J / kCkStages) & 1u, ctx)) { ok = false; break; }
-          if (!mbar_wait(&S.sempty[sb], ((J >> 1) & 1u) ^ 1u, ctx)) { ok = false; break; }
+          if (!mbar_wait(&S.kfull[st], (J / kCkKStages) & 1u, ctx)) { ok = false; break; }
+          if (!mbar_wait(&S.sfree[sb], ((J >> 1) & 1u) ^ 1u, ctx)) { ok = false; break; }
           tc_fence_after();
-          const int valid = S.meta[st][1];
+          const int valid = S.meta[st];
           if (valid > 0) {
             const uint32_t k0 = smem_u32(S.k[st][0]);
             const uint32_t k1 = smem_u32(S.k[st][1]);
@@ -245,29 +293,24 @@ __global__ void __launch_bounds__(kCkThreads, 1)
             }
           }
           umma_commit(&S.sfull[sb]);
+          umma_commit(&S.kempty[st]);
           if (j == ntile - 1) umma_commit(&S.qempty[ps]);
-          if (have_prev && !issue_pv(prev_st, prev_valid, prev_J, prev_first, prev_last, prev_K)) {
-            ok = false;
-            break;
-          }
+          if (have_prev && !issue_pv(prev)) { ok = false; break; }
           have_prev = true;
-          prev_st = st;
-          prev_valid = valid;
-          prev_J = J;
-          prev_first = j == 0;
-          prev_last = j == ntile - 1;
-          prev_K = K;
+          prev = Pending{valid, J, K, j == 0, j == ntile - 1};
         }
         if (!ok) break;
         ++K;
       }
-      if (ok && have_prev) ok = issue_pv(prev_st, prev_valid, prev_J, prev_first, prev_last, prev_K);
+      if (ok && have_prev) ok = issue_pv(prev);
       umma_commit(&S.drain);
       mbar_drain(&S.drain, 0);
     }
     __syncwarp();
-  } else {
-    // ======================= softmax / epilogue (thread = query row) =======================
+  } else if (warp < 4) {
+    // ======================= softmax (thread = query row) =======================
+    // The four warps never meet at a named barrier (rows are independent), so a warp whose wait
+    // timed out may leave on its own.
     const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
     const int r = tid;
     uint32_t J = 0, K = 0;
@@ -280,34 +323,50 @@ __global__ void __launch_bounds__(kCkThreads, 1)
       const TileItem it = S.item[ps];
       __syncwarp();
       if (lane == 0) mbar_arrive(&S.qempty[ps]);
-      if (idx < 0) break;
+      const uint32_t ob = K & 1;
+      if (idx < 0) {
+        // tell the epilogue warps to stop
+        if (mbar_wait(&S.lfree[ob], ((K >> 1) & 1u) ^ 1u, ctx)) {
+          if (lane == 0) S.epi_stop[ob] = 1;
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&S.lready[ob]);
+        }
+        break;
+      }
       const bool row_ok = r < it.rows;
       const int limit = it.prefix + it.pos0 + r;  // last visible key of this row
       float m = -INFINITY, l = 0.f;
       for (int j = 0; j < ntile; ++j, ++J) {
-        const int st = J % kCkStages;
         const int sb = J & 1;
         if (!mbar_wait(&S.sfull[sb], (J >> 1) & 1u, ctx)) { ok = false; break; }
-        if (!mbar_wait(&S.kfull[st], (J / kCkStages) & 1u, ctx)) { ok = false; break; }
         tc_fence_after();
-        const int kt0 = S.meta[st][0];
-        const int valid = S.meta[st][1];
-        const uint32_t sp = tmem + lane_base + kColS0 + sb * 128;  // this tile's S, then its P
+        // this key tile, from the item descriptor (the K stage may already hold a later tile)
+        const int kt0 = it.k0 + j * kCkKeys;
+        const int valid = max(0, min(kCkKeys, it.k1 - kt0));
         // keys [0, nvis) of the tile are visible to this row: inside the split, at or before the
         // row's causal limit, and the row inside the chunk
         const int nvis = row_ok ? max(0, min(valid, limit - kt0 + 1)) : 0;
-        // pass 1: the row's maximum over the visible keys
+        const bool full = __all_sync(0xffffffffu, nvis == kCkKeys);
+        const uint32_t sp = tmem + lane_base + kColS0 + sb * 128;  // this tile's S, then its P
+        // pass 1: the row's maximum over its visible keys (scale > 0, so it is applied after)
         float tmax = -INFINITY;
         if (valid > 0) {
-#pragma unroll
-          for (int c = 0; c < kCkKeys; c += 32) {
-            uint32_t raw[32];
-            tmem_ld32(sp + c, raw);
+#pragma unroll 1
+          for (int h = 0; h < kCkKeys; h += 64) {
+            uint32_t raw[64];
+            tmem_ld32(sp + h, *reinterpret_cast<uint32_t(*)[32]>(raw));
+            tmem_ld32(sp + h + 32, *reinterpret_cast<uint32_t(*)[32]>(raw + 32));
             tmem_wait_ld();
+            if (full) {
 #pragma unroll
-            for (int i = 0; i < 32; ++i)
-              if (c + i < nvis) tmax = fmaxf(tmax, __uint_as_float(raw[i]) * p.scale_log2);
+              for (int i = 0; i < 64; ++i) tmax = fmaxf(tmax, __uint_as_float(raw[i]));
+            } else {
+#pragma unroll
+              for (int i = 0; i < 64; ++i)
+                if (h + i < nvis) tmax = fmaxf(tmax, __uint_as_float(raw[i]));
+            }
           }
+          tmax *= p.scale_log2;
         }
         const float mn = fmaxf(m, tmax);
         const bool move = mn > m + kRescaleThreshold || (m == -INFINITY && mn != -INFINITY);
@@ -317,79 +376,123 @@ __global__ void __launch_bounds__(kCkThreads, 1)
           // O changes only after the previous product has added into it
           if (!mbar_wait(&S.pfree, (J - 1) & 1u, ctx)) { ok = false; break; }
           tc_fence_after();
-#pragma unroll
+          const uint32_t oc = tmem + lane_base + kColO0 + ob * 128;
+#pragma unroll 1
           for (int c = 0; c < kCkD; c += 32) {
             uint32_t o[32];
-            tmem_ld32(tmem + lane_base + kColO + c, o);
+            tmem_ld32(oc + c, o);
             tmem_wait_ld();
 #pragma unroll
             for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-            tmem_st32(tmem + lane_base + kColO + c, o);
+            tmem_st32(oc + c, o);
           }
         }
+        // pass 2, 64 keys at a time: p = 2^(s - m), split into bf16 hi + lo, written over the
+        // tile's own S columns (a 32-key chunk's words cover only columns already read)
+        float rs = 0.f;
+#pragma unroll 1
+        for (int h = 0; h < kCkKeys; h += 64) {
+          uint32_t raw[64];
+          if (valid > 0) {
+            tmem_ld32(sp + h, *reinterpret_cast<uint32_t(*)[32]>(raw));
+            tmem_ld32(sp + h + 32, *reinterpret_cast<uint32_t(*)[32]>(raw + 32));
+            tmem_wait_ld();
+          }
+#pragma unroll
+          for (int c = 0; c < 64; c += 32) {
+            uint32_t w[32];
+#pragma unroll
+            for (int i = 0; i < 32; i += 2) {
+              const int k0 = h + c + i;
+              float x0 = __uint_as_float(raw[c + i]) * p.scale_log2;
+              float x1 = __uint_as_float(raw[c + i + 1]) * p.scale_log2;
+              if (!full) {
+                x0 = k0 < nvis ? x0 : -INFINITY;
+                x1 = k0 + 1 < nvis ? x1 : -INFINITY;
+              }
+              const float p0 = mref == -INFINITY ? 0.f : fast_exp2(x0 - mref);
+              const float p1 = mref == -INFINITY ? 0.f : fast_exp2(x1 - mref);
+              rs += p0 + p1;
+              const __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
+              const float2 hf = __bfloat1622float2(h2);
+              w[i / 2] = *reinterpret_cast<const uint32_t*>(&h2);
+              w[16 + i / 2] = pack_bf16x2(p0 - hf.x, p1 - hf.y);
+            }
+            tmem_st32(sp + h + c, w);
+          }
+        }
+        l = fmaf(l, alpha, rs);
+        m = mref;
         if ((valid & 15) != 0) {
           // zero V rows [valid, next multiple of 16): they may lie past the request's keys
-          if (!mbar_wait(&S.vfull[st], (J / kCkStages) & 1u, ctx)) { ok = false; break; }
+          const int vs = J % kCkVStages;
+          if (!mbar_wait(&S.vfull[vs], (J / kCkVStages) & 1u, ctx)) { ok = false; break; }
           const int r0 = valid, r1 = (valid + 15) & ~15;
-          for (int c = tid; c < (r1 - r0) * 16; c += kCkSoftmax) {
+          for (int c = tid; c < (r1 - r0) * 16; c += 128) {
             const int row = r0 + c / 16;
-            *reinterpret_cast<uint4*>(reinterpret_cast<unsigned char*>(S.v[st][(c / 8) & 1]) +
+            *reinterpret_cast<uint4*>(reinterpret_cast<unsigned char*>(S.v[vs][(c / 8) & 1]) +
                                       row * 128 + (c & 7) * 16) = make_uint4(0u, 0u, 0u, 0u);
           }
           fence_proxy_async_smem();
         }
-        // pass 2: p = 2^(s - m), split into bf16 hi + lo, written over the chunk's own columns
-        float rs = 0.f;
-#pragma unroll
-        for (int c = 0; c < kCkKeys; c += 32) {
-          uint32_t raw[32];
-          if (valid > 0) {
-            tmem_ld32(sp + c, raw);
-            tmem_wait_ld();
-          }
-          uint32_t w[32];
-#pragma unroll
-          for (int i = 0; i < 32; i += 2) {
-            const float x0 = c + i < nvis ? __uint_as_float(raw[i]) * p.scale_log2 : -INFINITY;
-            const float x1 = c + i + 1 < nvis ? __uint_as_float(raw[i + 1]) * p.scale_log2 : -INFINITY;
-            const float p0 = mref == -INFINITY ? 0.f : fast_exp2(x0 - mref);
-            const float p1 = mref == -INFINITY ? 0.f : fast_exp2(x1 - mref);
-            rs += p0 + p1;
-            const __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
-            const float2 hf = __bfloat1622float2(h2);
-            w[i / 2] = *reinterpret_cast<const uint32_t*>(&h2);
-            w[16 + i / 2] = pack_bf16x2(p0 - hf.x, p1 - hf.y);
-          }
-          tmem_st32(sp + c, w);
-        }
-        l = fmaf(l, alpha, rs);
-        m = mref;
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&S.pfull[sb]);
       }
       if (!ok) break;
-
-      // ---- epilogue: O / l and the LSE of every row of the tile ----
-      if (!mbar_wait(&S.ofin, K & 1u, ctx)) break;
+      // ---- hand the item to the epilogue warps ----
+      if (!mbar_wait(&S.lfree[ob], ((K >> 1) & 1u) ^ 1u, ctx)) break;
+      S.mfin[ob][r] = m;
+      S.lfin[ob][r] = l;
+      if (tid == 0) {
+        S.epi[ob] = it;
+        S.epi_stop[ob] = 0;
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&S.lready[ob]);
+      ++K;
+    }
+  } else {
+    // ======================= epilogue: O / l and the LSE of every row =======================
+    const int quad = warp & 3;
+    const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
+    const int r = quad * 32 + lane;
+    for (uint32_t K = 0;; ++K) {
+      const uint32_t ob = K & 1;
+      if (!mbar_wait(&S.lready[ob], (K >> 1) & 1u, ctx)) break;
+      if (S.epi_stop[ob]) break;
+      const TileItem it = S.epi[ob];
+      const float m = S.mfin[ob][r];
+      const float l = S.lfin[ob][r];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&S.lfree[ob]);
+      if (!mbar_wait(&S.ofin[ob], (K >> 1) & 1u, ctx)) break;
       tc_fence_after();
+      const bool row_ok = r < it.rows;
       const bool direct = it.nsplit == 1;
       const float inv = l > 0.f ? 1.f / l : 0.f;
       const float lse2 = l > 0.f ? m + log2f(l) : -INFINITY;
+      // a row that saw no key has O = 0 (its accumulator may never have been written)
+      const bool seen = l > 0.f;
       const int hkv = it.h / p.g, g = it.h - hkv * p.g;
       const int64_t row = static_cast<int64_t>(it.row0) + r;
       const int64_t slot = static_cast<int64_t>(it.slot0) +
                            (static_cast<int64_t>(r) * p.hkv + hkv) * it.nsplit + it.split;
-#pragma unroll
+      __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out) + row * p.o_sr +
+                           static_cast<int64_t>(it.h) * p.o_sh;
+      float* dst = p.part_o + (slot * p.g + g) * kCkD;
+#pragma unroll 1
       for (int c = 0; c < kCkD; c += 32) {
         uint32_t o[32];
-        tmem_ld32(tmem + lane_base + kColO + c, o);
+        tmem_ld32(tmem + lane_base + kColO0 + ob * 128 + c, o);
         tmem_wait_ld();
+        if (!seen) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) o[i] = 0u;
+        }
         if (row_ok) {
           if (direct) {
-            __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out) + row * p.o_sr +
-                                 static_cast<int64_t>(it.h) * p.o_sh + c;
 #pragma unroll
             for (int i = 0; i < 32; i += 8) {
               uint4 v;
@@ -397,26 +500,24 @@ __global__ void __launch_bounds__(kCkThreads, 1)
               v.y = pack_bf16x2(__uint_as_float(o[i + 2]) * inv, __uint_as_float(o[i + 3]) * inv);
               v.z = pack_bf16x2(__uint_as_float(o[i + 4]) * inv, __uint_as_float(o[i + 5]) * inv);
               v.w = pack_bf16x2(__uint_as_float(o[i + 6]) * inv, __uint_as_float(o[i + 7]) * inv);
-              *reinterpret_cast<uint4*>(out + i) = v;
+              *reinterpret_cast<uint4*>(out + c + i) = v;
             }
           } else {
-            float* dst = p.part_o + (slot * p.g + g) * kCkD + c;
 #pragma unroll
             for (int i = 0; i < 32; i += 4)
-              *reinterpret_cast<float4*>(dst + i) =
+              *reinterpret_cast<float4*>(dst + c + i) =
                   make_float4(__uint_as_float(o[i]) * inv, __uint_as_float(o[i + 1]) * inv,
                               __uint_as_float(o[i + 2]) * inv, __uint_as_float(o[i + 3]) * inv);
           }
         }
       }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&S.oempty[ob]);
       if (row_ok) {
         if (direct) p.lse[row * p.hq + it.h] = lse2 * kLn2;
         else p.part_lse[slot * p.g + g] = lse2;
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&S.oempty);
-      ++K;
     }
   }
 

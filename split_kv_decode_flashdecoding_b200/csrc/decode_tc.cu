@@ -35,7 +35,6 @@ constexpr int kTcD = 128;              // head dim = UMMA M of the Oᵀ product
 constexpr int kTcStages = 3;
 constexpr int kProducerWarp = 4;     // Q and K
 constexpr int kMmaWarp = 5;
-constexpr int kEpilogueWarp0 = 6;    // warps 6-9; warp w reads TMEM lanes 32 (w mod 4) + [0, 32)
 constexpr int kVProducerWarp = 10;
 constexpr int kTcThreads = 11 * 32;
 constexpr int kSoftmaxThreads = 128;
