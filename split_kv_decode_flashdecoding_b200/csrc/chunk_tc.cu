@@ -9,7 +9,8 @@
 //
 //   S[128 rows x 128 keys] = Q_tile · K_tileᵀ         UMMA M=128 N=128, both K-major (TMA SW128)
 //   one thread per row: mask, running max m (rescaled lazily), p = 2^(s·scale·log2e − m),
-//   running sum l, P split into bf16 hi + lo and stored into tensor memory
+//   running sum l, P split into bf16 hi + lo (truncated top bits and remainder) and stored
+//   into tensor memory
 //   O[128 x 128] += P_hi · V_tile + P_lo · V_tile      UMMA M=128 N=128, A from TMEM, V MN-major
 //
 // S is double-buffered in TMEM and P is written back over the S buffer it came from (per
@@ -387,8 +388,13 @@ __global__ void __launch_bounds__(kCkThreads, 1)
             tmem_st32(oc + c, o);
           }
         }
-        // pass 2, 64 keys at a time: p = 2^(s - m), split into bf16 hi + lo, written over the
-        // tile's own S columns (a 32-key chunk's words cover only columns already read)
+        // pass 2, 64 keys at a time: p = 2^(s·scale − m), split into bf16 hi + lo and written over
+        // the tile's own S columns (a 32-key chunk's words cover only columns already read). hi
+        // keeps the top 16 bits of p (bf16 truncation) and lo the exact fp32 remainder, truncated
+        // the same way, so p − hi − lo < 2^-15 p; both packings are byte permutes, which leaves
+        // the exponential pipe to the exponentials. mref = −inf only when no key is visible, and
+        // then every x below is −inf already.
+        const float negm = mref == -INFINITY ? 0.f : -mref;
         float rs = 0.f;
 #pragma unroll 1
         for (int h = 0; h < kCkKeys; h += 64) {
@@ -404,19 +410,19 @@ __global__ void __launch_bounds__(kCkThreads, 1)
 #pragma unroll
             for (int i = 0; i < 32; i += 2) {
               const int k0 = h + c + i;
-              float x0 = __uint_as_float(raw[c + i]) * p.scale_log2;
-              float x1 = __uint_as_float(raw[c + i + 1]) * p.scale_log2;
+              float x0 = fmaf(__uint_as_float(raw[c + i]), p.scale_log2, negm);
+              float x1 = fmaf(__uint_as_float(raw[c + i + 1]), p.scale_log2, negm);
               if (!full) {
                 x0 = k0 < nvis ? x0 : -INFINITY;
                 x1 = k0 + 1 < nvis ? x1 : -INFINITY;
               }
-              const float p0 = mref == -INFINITY ? 0.f : fast_exp2(x0 - mref);
-              const float p1 = mref == -INFINITY ? 0.f : fast_exp2(x1 - mref);
+              const float p0 = fast_exp2(x0), p1 = fast_exp2(x1);
               rs += p0 + p1;
-              const __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
-              const float2 hf = __bfloat1622float2(h2);
-              w[i / 2] = *reinterpret_cast<const uint32_t*>(&h2);
-              w[16 + i / 2] = pack_bf16x2(p0 - hf.x, p1 - hf.y);
+              const uint32_t b0 = __float_as_uint(p0), b1 = __float_as_uint(p1);
+              w[i / 2] = __byte_perm(b0, b1, 0x7632);
+              const float l0 = p0 - __uint_as_float(b0 & 0xffff0000u);
+              const float l1 = p1 - __uint_as_float(b1 & 0xffff0000u);
+              w[16 + i / 2] = __byte_perm(__float_as_uint(l0), __float_as_uint(l1), 0x7632);
             }
             tmem_st32(sp + h + c, w);
           }
