@@ -45,7 +45,8 @@ def parse_args():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["fd", "reference"], default="fd")
     ap.add_argument("--workload", type=int, default=3, choices=[1, 2, 3, 4, 5])
-    ap.add_argument("--batch", type=int, default=None, help="batch of the long-context workload")
+    ap.add_argument("--batch", type=int, default=None,
+                    help="batch of workload 4; for workloads 3 and 5, keep the first B requests")
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--profile-calls", type=int, default=200,
                     help="calls timed with per-kernel events after the timed region (0: skip)")
@@ -123,7 +124,7 @@ def traffic_from_profiles(kernel_file: str, workload: str):
     try:
         with open(path) as f:
             j = json.load(f)
-        e = j[workload]
+        e = j[f"{workload}:{kernel_file}"]
         if e.get("source_sha") == kernel_source_sha(kernel_file):
             return float(e["bytes_per_launch"])
     except Exception:

@@ -152,8 +152,10 @@ def workload(index: int, batch: Optional[int] = None, pad_fill: float = 0.0):
         dec = uniform_lens(lseed, 31, 512, 8192)
         prefix = [15872] + [n - 1 for n in dec]
         chunk = [512] + [1] * 31
-        return make_chunk_inputs(prefix, chunk, 32, 32, 128, 16384, torch.bfloat16, seed,
-                                 pad_fill=pad_fill, name=WORKLOADS[5])
+        b = 32 if batch is None else int(batch)   # a smaller batch keeps the first b requests
+        name = WORKLOADS[5] if b == 32 else f"{WORKLOADS[5]}_first{b}"
+        return make_chunk_inputs(prefix[:b], chunk[:b], 32, 32, 128, 16384, torch.bfloat16,
+                                 seed, pad_fill=pad_fill, name=name)
     raise ValueError(f"unknown workload {index}")
 
 
