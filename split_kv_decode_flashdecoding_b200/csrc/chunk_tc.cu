@@ -349,9 +349,13 @@ __global__ void __launch_bounds__(kCkThreads, 1)
         const int nvis = row_ok ? max(0, min(valid, limit - kt0 + 1)) : 0;
         const bool full = __all_sync(0xffffffffu, nvis == kCkKeys);
         const uint32_t sp = tmem + lane_base + kColS0 + sb * 128;  // this tile's S, then its P
-        // pass 1: the row's maximum over its visible keys (scale > 0, so it is applied after)
+        // pass 1: the row's maximum over its visible keys (scale > 0, so it is applied after);
+        // four independent maxima keep the dependency chains short
         float tmax = -INFINITY;
         if (valid > 0) {
+          float mx[4];
+#pragma unroll
+          for (int a = 0; a < 4; ++a) mx[a] = -INFINITY;
 #pragma unroll 1
           for (int h = 0; h < kCkKeys; h += 64) {
             uint32_t raw[64];
@@ -360,13 +364,14 @@ __global__ void __launch_bounds__(kCkThreads, 1)
             tmem_wait_ld();
             if (full) {
 #pragma unroll
-              for (int i = 0; i < 64; ++i) tmax = fmaxf(tmax, __uint_as_float(raw[i]));
+              for (int i = 0; i < 64; ++i) mx[i & 3] = fmaxf(mx[i & 3], __uint_as_float(raw[i]));
             } else {
 #pragma unroll
               for (int i = 0; i < 64; ++i)
-                if (h + i < nvis) tmax = fmaxf(tmax, __uint_as_float(raw[i]));
+                if (h + i < nvis) mx[i & 3] = fmaxf(mx[i & 3], __uint_as_float(raw[i]));
             }
           }
+          tmax = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
           tmax *= p.scale_log2;
         }
         const float mn = fmaxf(m, tmax);
@@ -395,7 +400,9 @@ __global__ void __launch_bounds__(kCkThreads, 1)
         // the exponential pipe to the exponentials. mref = −inf only when no key is visible, and
         // then every x below is −inf already.
         const float negm = mref == -INFINITY ? 0.f : -mref;
-        float rs = 0.f;
+        float rsum[4];  // four independent partial sums of p
+#pragma unroll
+        for (int a = 0; a < 4; ++a) rsum[a] = 0.f;
 #pragma unroll 1
         for (int h = 0; h < kCkKeys; h += 64) {
           uint32_t raw[64];
@@ -417,7 +424,7 @@ __global__ void __launch_bounds__(kCkThreads, 1)
                 x1 = k0 + 1 < nvis ? x1 : -INFINITY;
               }
               const float p0 = fast_exp2(x0), p1 = fast_exp2(x1);
-              rs += p0 + p1;
+              rsum[(i >> 1) & 3] += p0 + p1;
               const uint32_t b0 = __float_as_uint(p0), b1 = __float_as_uint(p1);
               w[i / 2] = __byte_perm(b0, b1, 0x7632);
               const float l0 = p0 - __uint_as_float(b0 & 0xffff0000u);
@@ -427,6 +434,7 @@ __global__ void __launch_bounds__(kCkThreads, 1)
             tmem_st32(sp + h + c, w);
           }
         }
+        const float rs = (rsum[0] + rsum[1]) + (rsum[2] + rsum[3]);
         l = fmaf(l, alpha, rs);
         m = mref;
         if ((valid & 15) != 0) {
