@@ -52,6 +52,8 @@ __all__ = [
     "decode_attention",
     "chunk_prefill_attention",
     "attention_rows",
+    "gather_pages",
+    "decode_attention_paged",
 ]
 
 
@@ -200,3 +202,41 @@ def chunk_prefill_attention(q_chunk: np.ndarray, k_cache: np.ndarray, v_cache: n
             out[p, h] = o[r]
             lse[p, h] = l[r]
     return out, lse
+
+
+def gather_pages(pages: np.ndarray, block_table: Sequence[Sequence[int]], lens: Sequence[int],
+                 capacity: int) -> np.ndarray:
+    """Contiguous cache [B, Hkv, capacity, D] from a paged one.
+
+    pages [num_pages, Hkv, page_size, D]; token t of sequence b lives in page
+    block_table[b][t // page_size] at row t % page_size. Rows at or past len_b are left zero (the
+    attention below never reads them). This is the meaning of a block table in the paged-cache
+    row of the hot path (the FlashDecoding page, "部署落地的工程细节", pairs FlashDecoding with a
+    paged KV cache); the gather is the whole definition.
+    """
+    npg, hkv, psz, d = pages.shape
+    B = len(lens)
+    out = np.zeros((B, hkv, capacity, d), dtype=pages.dtype)
+    for b in range(B):
+        n = max(0, min(int(lens[b]), capacity))
+        for t0 in range(0, n, psz):
+            pg = int(block_table[b][t0 // psz])
+            m = min(psz, n - t0)
+            out[b, :, t0:t0 + m] = pages[pg, :, :m]
+    return out
+
+
+def decode_attention_paged(q: np.ndarray, k_pages: np.ndarray, v_pages: np.ndarray,
+                           block_table: Sequence[Sequence[int]], cache_lens: Sequence[int],
+                           scale: Optional[float] = None,
+                           rows: Optional[Iterable[Tuple[int, int]]] = None
+                           ) -> Tuple[np.ndarray, np.ndarray]:
+    """Decode attention over a paged cache: the pages gathered into a contiguous cache, then
+    ``decode_attention`` (the plain definition) over it."""
+    psz = k_pages.shape[2]
+    # a sequence holds at most (entries of its block-table row) * page_size keys; longer lengths
+    # are clamped to that, as a contiguous cache clamps them to its capacity
+    cap = max(1, len(block_table[0]) if len(block_table) else 1) * psz
+    kc = gather_pages(k_pages, block_table, cache_lens, cap)
+    vc = gather_pages(v_pages, block_table, cache_lens, cap)
+    return decode_attention(q, kc, vc, cache_lens, scale=scale, rows=rows)

@@ -33,6 +33,12 @@ chunk_b = ceil(len_b / num_splits) tokens, split s = [min(s * chunk_b, len_b),
 min((s + 1) * chunk_b, len_b)) (the FlashDecoding page's chunk_size rule); trailing splits
 may be empty.
 
+Aligned plans (``align`` = A > 1, used for a paged cache so that no key tile of A keys crosses a
+page) put every split boundary on a multiple of A keys and change nothing else: with
+U_b = ceil(len_b / A) units, planner split s = [min(len_b, A floor(s U_b / n_b)),
+min(len_b, A floor((s + 1) U_b / n_b))), and a fixed count uses chunk_b rounded up to a multiple
+of A. With A = 1 both rules are the ones above.
+
 Chunked prefill (``chunk_plan``): a request with chunk_len = 1 is a decode row over
 prefix_len + 1 keys and is planned as above (over the decode requests only). A request with a
 longer chunk is cut into query tiles of 128 rows; tile t sees at most
@@ -82,22 +88,25 @@ class DecodePlan:
         return max(self.splits_per_seq) if self.splits_per_seq else 0
 
 
-def _split_bounds_equal(n_tok: int, n_split: int) -> List[Tuple[int, int]]:
-    return [((s * n_tok) // n_split, ((s + 1) * n_tok) // n_split) for s in range(n_split)]
+def _split_bounds_equal(n_tok: int, n_split: int, align: int = 1) -> List[Tuple[int, int]]:
+    units = _cdiv(n_tok, align)
+    return [(min(n_tok, align * ((s * units) // n_split)),
+             min(n_tok, align * (((s + 1) * units) // n_split))) for s in range(n_split)]
 
 
-def _split_bounds_fixed(n_tok: int, n_split: int) -> List[Tuple[int, int]]:
+def _split_bounds_fixed(n_tok: int, n_split: int, align: int = 1) -> List[Tuple[int, int]]:
     c = _cdiv(n_tok, n_split) if n_tok > 0 else 0
+    c = align * _cdiv(c, align)
     return [(min(s * c, n_tok), min((s + 1) * c, n_tok)) for s in range(n_split)]
 
 
 def decode_plan(cache_lens: Sequence[int], num_kv_heads: int, cache_capacity: int,
-                num_ctas: int, num_splits: int = 0) -> DecodePlan:
+                num_ctas: int, num_splits: int = 0, align: int = 1) -> DecodePlan:
     """Plan the split-KV work of one decode call (see the module docstring)."""
     lens = [max(0, min(int(x), int(cache_capacity))) for x in cache_lens]
     B = len(lens)
     if num_splits > 0:
-        bounds = [_split_bounds_fixed(n, num_splits) for n in lens]
+        bounds = [_split_bounds_fixed(n, num_splits, align) for n in lens]
         chunk = 0
         keys = [_cdiv(n, num_splits) for n in lens]
     else:
@@ -105,7 +114,7 @@ def decode_plan(cache_lens: Sequence[int], num_kv_heads: int, cache_capacity: in
         chunk = _cdiv(total * num_kv_heads, WAVES * max(1, num_ctas))
         chunk = max(MIN_CHUNK, min(MAX_CHUNK, chunk))
         counts = [max(1, _cdiv(n, chunk)) for n in lens]
-        bounds = [_split_bounds_equal(n, c) for n, c in zip(lens, counts)]
+        bounds = [_split_bounds_equal(n, c, align) for n, c in zip(lens, counts)]
         keys = [_cdiv(n, c) for n, c in zip(lens, counts)]
     order = sorted(range(B), key=lambda b: (-keys[b], b))
     items = []

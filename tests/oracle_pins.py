@@ -314,10 +314,65 @@ def pin_bf16_widening(att):
     assert np.array_equal(att.widen(sb), special.to(torch.float64).numpy()), "bf16 specials"
 
 
+def _paged_case(seed, B, Hkv, psz, lens, pages_per_seq, D=8, Hq=None):
+    """A contiguous cache and the same keys scattered over shuffled physical pages; unused page
+    slots hold NaN, and block-table entries past a sequence's pages hold -1."""
+    Hq = Hq or 2 * Hkv
+    rng = np.random.default_rng(seed)
+    cap = pages_per_seq * psz
+    q = _rand((B, Hq, D), seed + 1, 2.0)
+    k = _rand((B, Hkv, cap, D), seed + 2)
+    v = _rand((B, Hkv, cap, D), seed + 3)
+    npages = B * pages_per_seq + 3
+    phys = rng.permutation(npages)
+    kp = np.full((npages, Hkv, psz, D), np.nan)
+    vp = np.full((npages, Hkv, psz, D), np.nan)
+    table = [[-1] * pages_per_seq for _ in range(B)]
+    i = 0
+    for b in range(B):
+        used = -(-max(0, min(lens[b], cap)) // psz)
+        for j in range(used):
+            pg = int(phys[i])
+            i += 1
+            table[b][j] = pg
+            kp[pg] = k[b, :, j * psz:(j + 1) * psz]
+            vp[pg] = v[b, :, j * psz:(j + 1) * psz]
+    return q, k, v, kp, vp, table
+
+
+def pin_paged_equals_contiguous(att):
+    # the paged form is the contiguous definition over the gathered keys: any wrong page or row
+    # index reads another page (or a NaN slot) and changes the result
+    for seed, psz, lens in ((80, 1, [5, 0, 3]), (81, 3, [7, 9, 1]), (82, 16, [33, 16, 0, 47])):
+        B = len(lens)
+        pps = max(1, -(-max(lens) // psz))
+        q, k, v, kp, vp, table = _paged_case(seed, B, 2, psz, lens, pps)
+        o1, l1 = att.decode_attention(q, k, v, lens)
+        o2, l2 = att.decode_attention_paged(q, kp, vp, table, lens)
+        _close(o2, o1, 1e-12, f"paged psz {psz} O")
+        _close(l2, l1, 1e-12, f"paged psz {psz} LSE")
+
+
+def pin_paged_swapped_pages(att):
+    # page size 2, a 4-key sequence stored as [keys 2-3 | keys 0-1]; the first key dominates, so
+    # the output is v_0 exactly when (and only when) page 0 of the sequence is read as keys 0-1
+    D = 4
+    keys = np.zeros((4, D))
+    keys[0] = 40.0
+    vals = np.arange(4 * D, dtype=np.float64).reshape(4, D)
+    q = np.ones((1, 1, D))
+    kp = np.stack([keys[2:4], keys[0:2]])[:, None]   # [2 pages, 1 head, 2 rows, D]
+    vp = np.stack([vals[2:4], vals[0:2]])[:, None]
+    o, l = att.decode_attention_paged(q, kp, vp, [[1, 0]], [4])
+    _close(o[0, 0], vals[0], 1e-12, "dominant first key from the second physical page")
+    s0 = 40.0 * D / math.sqrt(D)
+    _close(l[0, 0], s0 + math.log1p(3 * math.exp(-s0)), 1e-12, "LSE of one dominant key")
+
+
 ALL_PINS = [
     pin_golden_decode, pin_golden_chunk, pin_zero_query_is_mean, pin_single_key,
     pin_two_keys_sigmoid, pin_one_hot, pin_equal_scores, pin_empty_and_clamp,
     pin_torch_softmax, pin_chunk_equals_full_causal, pin_chunk_batch_gqa,
     pin_split_invariance, pin_permutation_invariance, pin_page_formulations,
-    pin_bf16_widening,
+    pin_bf16_widening, pin_paged_equals_contiguous, pin_paged_swapped_pages,
 ]

@@ -35,6 +35,10 @@ MUTATIONS = {
     "bf16_widen_shift": ("<< np.uint32(16)", "<< np.uint32(15)"),
     "empty_lse_zero": ("lse = np.full((R,), -np.inf, dtype=np.float64)",
                        "lse = np.full((R,), 0.0, dtype=np.float64)"),
+    "page_index_mod": ("pg = int(block_table[b][t0 // psz])", "pg = int(block_table[b][t0 % psz])"),
+    "paged_k_from_v": ("kc = gather_pages(k_pages, block_table, cache_lens, cap)",
+                       "kc = gather_pages(v_pages, block_table, cache_lens, cap)"),
+    "page_physical_order": ("pg = int(block_table[b][t0 // psz])", "pg = t0 // psz + b"),
 }
 
 

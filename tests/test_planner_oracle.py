@@ -130,3 +130,40 @@ def test_chunk_plan_tiles_with_fewer_splits():
     assert cp.row_splits == [1] * 128 + [2] * 172
     assert [(t, s, k0, k1) for (b, t, h, s, k0, k1) in cp.tile_items] == [
         (0, 0, 0, 2028), (1, 0, 0, 2048), (2, 0, 0, 2048), (1, 1, 2048, 2156), (2, 1, 2048, 2200)]
+
+
+# ---- aligned plans (paged cache): split boundaries on multiples of the key tile ----------------
+
+def test_aligned_plan_hand_cases():
+    # planner mode: 300 keys, 2 splits of whole 128-key units: units = 3 -> [0, 128), [128, 300)
+    assert P._split_bounds_equal(300, 2, 128) == [(0, 128), (128, 300)]
+    # 1000 keys, 3 splits: units = 8 -> boundaries at units 0, 2, 5, 8
+    assert P._split_bounds_equal(1000, 3, 128) == [(0, 256), (256, 640), (640, 1000)]
+    # fixed mode: chunk ceil(300 / 2) = 150 rounded up to 256
+    assert P._split_bounds_fixed(300, 2, 128) == [(0, 256), (256, 300)]
+    assert P._split_bounds_fixed(100, 4, 16) == [(0, 32), (32, 64), (64, 96), (96, 100)]
+    # align 1 is the unaligned rule
+    assert P._split_bounds_equal(1000, 3, 1) == P._split_bounds_equal(1000, 3)
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_aligned_plan_properties(seed):
+    rng = random.Random(seed)
+    B = rng.randint(1, 39)
+    lens = [rng.randint(0, 19999) for _ in range(B)]
+    for fixed in (0, 3):
+        plan = P.decode_plan(lens, 4, 20000, 148, fixed, align=128)
+        ref = P.decode_plan(lens, 4, 20000, 148, fixed)
+        # same split counts and order, only the boundaries move
+        assert plan.splits_per_seq == ref.splits_per_seq
+        assert [it[:3] for it in plan.items] == [it[:3] for it in ref.items]
+        for b in range(B):
+            bounds = [(t0, t1) for (bb, h, s, t0, t1) in plan.items if bb == b and h == 0]
+            assert bounds[0][0] == 0 and bounds[-1][1] == lens[b]
+            for (a0, a1), (c0, c1) in zip(bounds, bounds[1:]):
+                assert a1 == c0
+            for t0, t1 in bounds:
+                # boundaries on the 128-key grid, except at the sequence end (trailing empty
+                # splits of a fixed count sit at [len, len))
+                assert t0 <= t1 and (t0 % 128 == 0 or t0 == lens[b])
+                assert t1 % 128 == 0 or t1 == lens[b]
