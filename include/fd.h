@@ -83,6 +83,7 @@ typedef struct {
 #define FD_FLAG_LEN_CLAMPED 0x1u  /* some cache/prefix/chunk length was outside [0, S_cap]     */
 #define FD_FLAG_WAIT_TIMEOUT 0x2u /* a kernel wait gave up; the call's results are invalid     */
 #define FD_FLAG_PLAN_OVERFLOW 0x4u /* the device plan exceeded the workspace bound (a bug)     */
+#define FD_FLAG_BAD_PAGE 0x8u      /* a block-table entry of a used page was outside the pool   */
 
 /*
  * fd_decode_attention — split-KV FlashDecoding decode attention (one query token per sequence).
@@ -114,6 +115,38 @@ fd_status fd_decode_attention(const fd_tensor* q, const fd_tensor* k_cache,
                               int32_t num_splits, fd_tensor* out, float* lse, void* stream);
 
 /*
+ * fd_decode_attention_paged — fd_decode_attention over a paged KV cache.
+ *
+ * The FlashDecoding page ("部署落地的工程细节") pairs split-KV decoding with a paged KV cache;
+ * the pages give no layout, so this one is read as the usual block-table form: the cache of
+ * sequence b is the sequence of pages block_table[b][0], block_table[b][1], ...; token t of
+ * sequence b is row t % page_size of page block_table[b][t / page_size]. The result is exactly
+ * fd_decode_attention's on the gathered contiguous cache. Splits are planned as in
+ * fd_split_plan with key_align = 128, so no key tile crosses a page.
+ *
+ *  q            [B, Hq, D]                      as in fd_decode_attention.
+ *  k_pages      [num_pages, Hkv, page_size, D]  the page pool (same dtype as q). page_size is
+ *  v_pages      [num_pages, Hkv, page_size, D]  8, 16, 32, 64 or a multiple of 128. The rows of
+ *                                               one (page, head) must be contiguous
+ *                                               (stride[2] == D); strides multiples of 16 bytes,
+ *                                               data 16-byte aligned; k and v share strides.
+ *  block_table  [B, pages_per_seq] int32 (device, contiguous rows): physical page of each
+ *               logical page. Entries past a sequence's last page are never dereferenced as
+ *               memory addresses (they may hold any value, e.g. -1).
+ *  pages_per_seq >= 1: the table's row length; a sequence holds at most pages_per_seq *
+ *               page_size keys, and longer cache_lens are clamped to that (status flag).
+ *  cache_lens, num_splits, out, lse, stream: as in fd_decode_attention.
+ * Table entries of pages a sequence uses must be valid page indices (0 <= id < num_pages). An
+ * out-of-range index there is never dereferenced: that page's keys are not read (their contents
+ * in the result are unspecified) and FD_FLAG_BAD_PAGE is raised.
+ */
+fd_status fd_decode_attention_paged(const fd_tensor* q, const fd_tensor* k_pages,
+                                    const fd_tensor* v_pages, const int32_t* block_table,
+                                    int32_t pages_per_seq, const int32_t* cache_lens,
+                                    int32_t num_splits, fd_tensor* out, float* lse,
+                                    void* stream);
+
+/*
  * fd_split_plan — the variable-length split planner, on the host (no CUDA call).
  *
  * FlashDecoding page, "Variable-Length序列动态切分策略" (allocator with min_chunk 128 and
@@ -123,11 +156,17 @@ fd_status fd_decode_attention(const fd_tensor* q, const fd_tensor* k_cache,
  * [floor(s*len_b/n_b), floor((s+1)*len_b/n_b)); items are ordered longest split first
  * (sequences by their longest split, descending, ties by index), then KV head, then split.
  * num_splits > 0 instead fixes n_b = num_splits with ceil(len_b/num_splits)-key splits.
- * This is the same plan fd_decode_attention builds on the device.
+ * key_align = A > 1 puts every split boundary on a multiple of A keys (the plan of a paged
+ * cache, A = 128, so that no key tile crosses a page): planner splits cut the ceil(len_b/A)
+ * units equally, [min(len_b, A*floor(s*U/n_b)), min(len_b, A*floor((s+1)*U/n_b))), and a fixed
+ * count rounds its split size up to a multiple of A; split counts and order do not change.
+ * key_align = 1 is the plan of a contiguous cache. This is the same plan fd_decode_attention
+ * (key_align 1) and fd_decode_attention_paged (key_align 128) build on the device.
  *
  *  cache_lens_host    [batch] int32 (host); clamped into [0, cache_capacity].
  *  num_ctas           persistent CTAs to plan for (>= 1); fd_decode_num_ctas() gives the count a
  *                     decode call on a device uses.
+ *  key_align          >= 1 (see above).
  *  splits_per_seq_host [batch] int32 (host, written) or NULL.
  *  items_host         [items_capacity][5] int32 (host, written) or NULL: per item
  *                     (b, kv_head, split, start, end) in execution order. Items beyond
@@ -136,7 +175,7 @@ fd_status fd_decode_attention(const fd_tensor* q, const fd_tensor* k_cache,
  */
 fd_status fd_split_plan(const int32_t* cache_lens_host, int32_t batch, int32_t num_kv_heads,
                         int32_t cache_capacity, int32_t num_splits, int32_t num_ctas,
-                        int32_t* splits_per_seq_host, int32_t* items_host,
+                        int32_t key_align, int32_t* splits_per_seq_host, int32_t* items_host,
                         int32_t items_capacity, fd_plan_info* info);
 
 /*
@@ -151,7 +190,7 @@ fd_status fd_split_plan(const int32_t* cache_lens_host, int32_t batch, int32_t n
  */
 fd_status fd_split_plan_device(const int32_t* cache_lens, int32_t batch, int32_t num_kv_heads,
                                int32_t cache_capacity, int32_t num_splits, int32_t num_ctas,
-                               int32_t* splits_per_seq_dev, int32_t* items_dev,
+                               int32_t key_align, int32_t* splits_per_seq_dev, int32_t* items_dev,
                                int32_t items_capacity, int32_t* total_items_dev, void* stream);
 
 /*

@@ -23,12 +23,14 @@ from typing import List, Optional, Sequence, Tuple
 import torch
 
 __all__ = [
-    "FdError", "LIB_PATH", "lib", "fd_decode_attention", "fd_decode_attention_static",
+    "FdError", "LIB_PATH", "lib", "fd_decode_attention", "fd_decode_attention_paged",
+    "fd_decode_attention_static",
     "fd_chunk_prefill_attention",
     "fd_split_plan", "fd_split_plan_device", "fd_decode_num_ctas", "fd_decode_workspace_bytes",
     "fd_chunk_workspace_bytes", "fd_reserve_workspace", "fd_poll_status", "fd_profile_begin",
     "fd_profile_end", "fd_shutdown", "fd_status_string", "FD_F32", "FD_BF16",
-    "FD_FLAG_LEN_CLAMPED", "FD_FLAG_WAIT_TIMEOUT", "FD_FLAG_PLAN_OVERFLOW", "ABI_FUNCTIONS",
+    "FD_FLAG_LEN_CLAMPED", "FD_FLAG_WAIT_TIMEOUT", "FD_FLAG_PLAN_OVERFLOW", "FD_FLAG_BAD_PAGE",
+    "ABI_FUNCTIONS",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libfd.so")
@@ -38,6 +40,7 @@ FD_F32, FD_BF16 = 0, 1
 FD_FLAG_LEN_CLAMPED = 0x1
 FD_FLAG_WAIT_TIMEOUT = 0x2
 FD_FLAG_PLAN_OVERFLOW = 0x4
+FD_FLAG_BAD_PAGE = 0x8
 
 c_i32, c_i64, c_size, c_vp, c_f32p = (ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t,
                                       ctypes.c_void_p, ctypes.POINTER(ctypes.c_float))
@@ -72,11 +75,13 @@ _TP = ctypes.POINTER(FdTensor)
 ABI_FUNCTIONS = {
     "fd_decode_attention": (c_i32, [_TP, _TP, _TP, c_i32p, c_i32, _TP, c_f32p, c_vp]),
     "fd_decode_attention_static": (c_i32, [_TP, _TP, _TP, c_i32p, c_i32, _TP, c_f32p, c_vp]),
-    "fd_split_plan": (c_i32, [c_i32p, c_i32, c_i32, c_i32, c_i32, c_i32, c_i32p, c_i32p, c_i32,
-                              ctypes.POINTER(FdPlanInfo)]),
-    "fd_split_plan_device": (c_i32, [c_i32p, c_i32, c_i32, c_i32, c_i32, c_i32, c_i32p, c_i32p,
-                                     c_i32, c_i32p, c_vp]),
+    "fd_split_plan": (c_i32, [c_i32p, c_i32, c_i32, c_i32, c_i32, c_i32, c_i32, c_i32p, c_i32p,
+                              c_i32, ctypes.POINTER(FdPlanInfo)]),
+    "fd_split_plan_device": (c_i32, [c_i32p, c_i32, c_i32, c_i32, c_i32, c_i32, c_i32, c_i32p,
+                                     c_i32p, c_i32, c_i32p, c_vp]),
     "fd_chunk_prefill_attention": (c_i32, [_TP, _TP, _TP, c_i32p, c_i32p, _TP, c_f32p, c_vp]),
+    "fd_decode_attention_paged": (c_i32, [_TP, _TP, _TP, c_i32p, c_i32, c_i32p, c_i32, _TP, c_f32p,
+                                          c_vp]),
     "fd_status_string": (ctypes.c_char_p, [c_i32]),
     "fd_last_error_message": (ctypes.c_char_p, []),
     "fd_decode_num_ctas": (c_i32, [c_i32, c_i32, c_i32, c_i32]),
@@ -153,6 +158,30 @@ def fd_decode_attention(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.T
     return out, lse
 
 
+def fd_decode_attention_paged(q: torch.Tensor, k_pages: torch.Tensor, v_pages: torch.Tensor,
+                              block_table: torch.Tensor, cache_lens: torch.Tensor,
+                              num_splits: int = 0, out: Optional[torch.Tensor] = None,
+                              lse: Optional[torch.Tensor] = None,
+                              stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Split-KV decode attention over a paged cache. k_pages / v_pages [num_pages, Hkv,
+    page_size, D]; block_table int32 [B, pages_per_seq] (contiguous rows); token t of sequence b
+    is row t % page_size of page block_table[b, t // page_size]."""
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty(q.shape[:2], dtype=torch.float32, device=q.device)
+    if block_table.dim() != 2 or block_table.stride(1) != 1 or block_table.stride(0) != block_table.shape[1]:
+        raise ValueError("block_table must be a contiguous [B, pages_per_seq] int32 tensor")
+    with torch.cuda.device(q.device):
+        st = lib.fd_decode_attention_paged(
+            ctypes.byref(_tensor(q)), ctypes.byref(_tensor(k_pages)),
+            ctypes.byref(_tensor(v_pages)), _ptr(block_table, c_i32), int(block_table.shape[1]),
+            _ptr(cache_lens, c_i32), int(num_splits), ctypes.byref(_tensor(out)),
+            _ptr(lse, ctypes.c_float), _stream(stream, q.device))
+    _check(st, "fd_decode_attention_paged")
+    return out, lse
+
+
 def fd_decode_attention_static(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
                                cache_lens: torch.Tensor, num_splits: int, out: torch.Tensor,
                                lse: torch.Tensor, stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
@@ -190,19 +219,20 @@ def fd_chunk_prefill_attention(q_chunk: torch.Tensor, k_cache: torch.Tensor,
 
 
 def fd_split_plan(cache_lens: Sequence[int], num_kv_heads: int, cache_capacity: int,
-                  num_splits: int = 0, num_ctas: int = 148, with_items: bool = True):
+                  num_splits: int = 0, num_ctas: int = 148, with_items: bool = True,
+                  key_align: int = 1):
     """Host planner. Returns (info dict, splits per sequence, items [(b,h,split,start,end)])."""
     B = len(cache_lens)
     lens = (c_i32 * max(1, B))(*[int(x) for x in cache_lens])
     splits = (c_i32 * max(1, B))()
     info = FdPlanInfo()
-    _check(lib.fd_split_plan(lens, B, num_kv_heads, cache_capacity, num_splits, num_ctas, splits,
-                             None, 0, ctypes.byref(info)), "fd_split_plan")
+    _check(lib.fd_split_plan(lens, B, num_kv_heads, cache_capacity, num_splits, num_ctas,
+                             key_align, splits, None, 0, ctypes.byref(info)), "fd_split_plan")
     items: List[Tuple[int, int, int, int, int]] = []
     if with_items and info.total_items > 0:
         buf = (c_i32 * (5 * info.total_items))()
         _check(lib.fd_split_plan(lens, B, num_kv_heads, cache_capacity, num_splits, num_ctas,
-                                 splits, buf, info.total_items, ctypes.byref(info)),
+                                 key_align, splits, buf, info.total_items, ctypes.byref(info)),
                "fd_split_plan")
         items = [tuple(buf[5 * i:5 * i + 5]) for i in range(info.total_items)]
     d = {f: getattr(info, f) for f, _ in FdPlanInfo._fields_}
@@ -211,7 +241,7 @@ def fd_split_plan(cache_lens: Sequence[int], num_kv_heads: int, cache_capacity: 
 
 def fd_split_plan_device(cache_lens: torch.Tensor, num_kv_heads: int, cache_capacity: int,
                          num_splits: int = 0, num_ctas: int = 148, items_capacity: int = 0,
-                         stream=None):
+                         stream=None, key_align: int = 1):
     """Run the device planner on device lengths. Returns (total_items, splits, items) tensors."""
     dev = cache_lens.device
     B = cache_lens.numel()
@@ -220,7 +250,7 @@ def fd_split_plan_device(cache_lens: torch.Tensor, num_kv_heads: int, cache_capa
     items = torch.zeros((max(1, items_capacity), 5), dtype=torch.int32, device=dev)
     with torch.cuda.device(dev):
         st = lib.fd_split_plan_device(_ptr(cache_lens, c_i32), B, num_kv_heads, cache_capacity,
-                                      num_splits, num_ctas, _ptr(splits, c_i32),
+                                      num_splits, num_ctas, key_align, _ptr(splits, c_i32),
                                       _ptr(items, c_i32) if items_capacity > 0 else None,
                                       items_capacity, _ptr(total, c_i32), _stream(stream, dev))
     _check(st, "fd_split_plan_device")

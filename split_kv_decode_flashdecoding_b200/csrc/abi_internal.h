@@ -25,6 +25,23 @@ struct DecodeShape {
 fd_status resolve_decode(const fd_tensor* q, const fd_tensor* k, const fd_tensor* v,
                          const fd_tensor* out, DecodeShape* sh);
 
+// A paged cache: K/V pages [num_pages, Hkv, page_size, D] read through a block table
+// [B, pages_per_seq]. page_size is filled in by resolve_paged.
+struct PagedCache {
+  const int32_t* block_table;
+  int32_t pages_per_seq;
+  int32_t page_size;
+};
+
+// Validate a paged decode call (S_cap becomes pages_per_seq * page_size).
+fd_status resolve_paged(const fd_tensor* q, const fd_tensor* k, const fd_tensor* v,
+                        PagedCache& pg, const fd_tensor* out, DecodeShape* sh);
+
+// The decode call of fd_decode_attention (pg == nullptr) and fd_decode_attention_paged.
+fd_status decode_call(const fd_tensor* q, const fd_tensor* k_cache, const fd_tensor* v_cache,
+                      const int32_t* cache_lens, int32_t num_splits, fd_tensor* out, float* lse,
+                      cudaStream_t stream, PagedCache* pg);
+
 // Persistent CTAs of the split kernel on device `dev`.
 int decode_ctas(int dev, bool use_tc);
 

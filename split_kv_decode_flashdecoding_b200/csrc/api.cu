@@ -244,6 +244,49 @@ fd_status resolve_decode(const fd_tensor* q, const fd_tensor* k, const fd_tensor
   return FD_OK;
 }
 
+fd_status resolve_paged(const fd_tensor* q, const fd_tensor* k, const fd_tensor* v,
+                        PagedCache& pg, const fd_tensor* out, DecodeShape* sh) {
+  fd_status s;
+  if ((s = check_q_out(q, out, "q")) != FD_OK) return s;
+  sh->B = static_cast<int>(q->shape[0]);
+  sh->hq = static_cast<int>(q->shape[1]);
+  sh->d = static_cast<int>(q->shape[2]);
+  sh->dtype = q->dtype;
+  if (sh->d != 64 && sh->d != 128) return fail(FD_ERR_UNSUPPORTED, "head_dim %d: only 64 and 128 are supported", sh->d);
+  if ((s = check_tensor(k, "k_pages", 4)) != FD_OK) return s;
+  if ((s = check_tensor(v, "v_pages", 4)) != FD_OK) return s;
+  if (k->dtype != sh->dtype || v->dtype != sh->dtype) return fail(FD_ERR_INVALID_ARGUMENT, "k_pages / v_pages dtype differs from q");
+  for (int i = 0; i < 4; ++i) {
+    if (k->shape[i] != v->shape[i]) return fail(FD_ERR_INVALID_ARGUMENT, "k_pages and v_pages shapes differ");
+    if (k->stride[i] != v->stride[i]) return fail(FD_ERR_UNSUPPORTED, "k_pages and v_pages must share strides");
+  }
+  if (k->shape[0] < 1) return fail(FD_ERR_INVALID_ARGUMENT, "the page pool needs at least one page");
+  if (k->shape[1] < 1) return fail(FD_ERR_INVALID_ARGUMENT, "k_pages needs at least one KV head");
+  if (k->shape[3] != sh->d) return fail(FD_ERR_INVALID_ARGUMENT, "k_pages head_dim %lld != q head_dim %d", (long long)k->shape[3], sh->d);
+  const int64_t psz = k->shape[2];
+  if (!(psz == 8 || psz == 16 || psz == 32 || psz == 64 || (psz >= 128 && psz % 128 == 0)))
+    return fail(FD_ERR_UNSUPPORTED, "page size %lld: must be 8, 16, 32, 64 or a multiple of 128", (long long)psz);
+  if (k->stride[2] != sh->d) return fail(FD_ERR_UNSUPPORTED, "token rows of a page must be contiguous (stride[2] == head_dim)");
+  if (sh->B > 0 && (!k->data || !v->data)) return fail(FD_ERR_INVALID_ARGUMENT, "k_pages / v_pages data is NULL");
+  if (!aligned16(k->data) || !aligned16(v->data) || !stride16(k->stride[0], sh->dtype) || !stride16(k->stride[1], sh->dtype))
+    return fail(FD_ERR_UNSUPPORTED, "page data and strides must be 16-byte aligned");
+  if (sh->B > 0 && !pg.block_table) return fail(FD_ERR_INVALID_ARGUMENT, "block_table is NULL");
+  if (pg.pages_per_seq < 1) return fail(FD_ERR_INVALID_ARGUMENT, "pages_per_seq must be >= 1");
+  if (static_cast<int64_t>(pg.pages_per_seq) * psz > INT32_MAX)
+    return fail(FD_ERR_UNSUPPORTED, "pages_per_seq * page_size exceeds 2^31 keys");
+  pg.page_size = static_cast<int32_t>(psz);
+  sh->hkv = static_cast<int>(k->shape[1]);
+  sh->cap = pg.pages_per_seq * pg.page_size;
+  if (sh->hq < 1 || sh->hq % sh->hkv != 0)
+    return fail(FD_ERR_INVALID_ARGUMENT, "q heads (%d) must be a positive multiple of KV heads (%d)", sh->hq, sh->hkv);
+  sh->g = sh->hq / sh->hkv;
+  if (sh->B > kMaxPlanBatch) return fail(FD_ERR_UNSUPPORTED, "batch %d exceeds %d", sh->B, kMaxPlanBatch);
+  sh->use_tc = sh->dtype == FD_BF16 && sh->d == 128 && sh->g >= 2 && sh->g <= 16;
+  if (!sh->use_tc && sh->g > 8)
+    return fail(FD_ERR_UNSUPPORTED, "group size %d needs bf16 with head_dim 128 (tensor-core kernel)", sh->g);
+  return FD_OK;
+}
+
 int decode_ctas(int dev, bool use_tc) {
   const int n = sm_count(dev);
   return use_tc ? n : n * simt_ctas_per_sm();
@@ -322,7 +365,7 @@ size_t fd_decode_workspace_bytes(int32_t batch, int32_t num_q_heads, int32_t num
 
 fd_status fd_split_plan(const int32_t* cache_lens_host, int32_t batch, int32_t num_kv_heads,
                         int32_t cache_capacity, int32_t num_splits, int32_t num_ctas,
-                        int32_t* splits_per_seq_host, int32_t* items_host,
+                        int32_t key_align, int32_t* splits_per_seq_host, int32_t* items_host,
                         int32_t items_capacity, fd_plan_info* info) {
   if (!info) return fail(FD_ERR_INVALID_ARGUMENT, "info is NULL");
   if (batch < 0) return fail(FD_ERR_INVALID_ARGUMENT, "batch must be >= 0");
@@ -331,6 +374,7 @@ fd_status fd_split_plan(const int32_t* cache_lens_host, int32_t batch, int32_t n
   if (cache_capacity < 0) return fail(FD_ERR_INVALID_ARGUMENT, "cache_capacity must be >= 0");
   if (num_splits < 0) return fail(FD_ERR_INVALID_ARGUMENT, "num_splits must be >= 0");
   if (num_ctas < 1) return fail(FD_ERR_INVALID_ARGUMENT, "num_ctas must be >= 1");
+  if (key_align < 1) return fail(FD_ERR_INVALID_ARGUMENT, "key_align must be >= 1");
   if (items_host && items_capacity < 0) return fail(FD_ERR_INVALID_ARGUMENT, "items_capacity must be >= 0");
   HostPlan hp;
   host_plan(cache_lens_host, batch, num_kv_heads, cache_capacity, num_splits, num_ctas, &hp);
@@ -348,7 +392,7 @@ fd_status fd_split_plan(const int32_t* cache_lens_host, int32_t batch, int32_t n
       for (int h = 0; h < num_kv_heads && i < items_capacity; ++h)
         for (int s = 0; s < n && i < items_capacity; ++s, ++i) {
           int32_t t0, t1;
-          plan_split_range(hp.lens[b], n, s, num_splits, &t0, &t1);
+          plan_split_range(hp.lens[b], n, s, num_splits, key_align, &t0, &t1);
           int32_t* o = items_host + 5 * i;
           o[0] = b; o[1] = h; o[2] = s; o[3] = t0; o[4] = t1;
         }
@@ -365,13 +409,13 @@ fd_status fd_split_plan(const int32_t* cache_lens_host, int32_t batch, int32_t n
 
 fd_status fd_split_plan_device(const int32_t* cache_lens, int32_t batch, int32_t num_kv_heads,
                                int32_t cache_capacity, int32_t num_splits, int32_t num_ctas,
-                               int32_t* splits_per_seq_dev, int32_t* items_dev,
+                               int32_t key_align, int32_t* splits_per_seq_dev, int32_t* items_dev,
                                int32_t items_capacity, int32_t* total_items_dev, void* stream_) {
   cudaStream_t stream = static_cast<cudaStream_t>(stream_);
   if (batch < 0 || batch > kMaxPlanBatch) return fail(FD_ERR_INVALID_ARGUMENT, "batch must be in [0, %d]", kMaxPlanBatch);
   if (batch > 0 && (!cache_lens || !splits_per_seq_dev)) return fail(FD_ERR_INVALID_ARGUMENT, "NULL device pointer");
   if (!total_items_dev) return fail(FD_ERR_INVALID_ARGUMENT, "total_items_dev is NULL");
-  if (num_kv_heads < 1 || cache_capacity < 0 || num_splits < 0 || num_ctas < 1)
+  if (num_kv_heads < 1 || cache_capacity < 0 || num_splits < 0 || num_ctas < 1 || key_align < 1)
     return fail(FD_ERR_INVALID_ARGUMENT, "bad plan arguments");
   if (items_dev && items_capacity < 0) return fail(FD_ERR_INVALID_ARGUMENT, "items_capacity must be >= 0");
   const int64_t items = decode_max_items(batch, num_kv_heads, cache_capacity, num_splits, num_ctas);
@@ -388,6 +432,7 @@ fd_status fd_split_plan_device(const int32_t* cache_lens, int32_t batch, int32_t
   pp.cap = cache_capacity;
   pp.fixed = num_splits;
   pp.nctas = num_ctas;
+  pp.align = key_align;
   pp.max_dec_items = items;
   pp.hdr = reinterpret_cast<WsHeader*>(base);
   pp.items = reinterpret_cast<DecodeItem*>(base + L.dec_items);
@@ -402,12 +447,17 @@ fd_status fd_split_plan_device(const int32_t* cache_lens, int32_t batch, int32_t
   return FD_OK;
 }
 
-fd_status fd_decode_attention(const fd_tensor* q, const fd_tensor* k_cache,
-                              const fd_tensor* v_cache, const int32_t* cache_lens,
-                              int32_t num_splits, fd_tensor* out, float* lse, void* stream_) {
-  cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+}  // extern "C"
+
+namespace fd_abi {
+
+// The decode call of both entry points: a contiguous cache (pg == nullptr) or a paged one.
+fd_status decode_call(const fd_tensor* q, const fd_tensor* k_cache, const fd_tensor* v_cache,
+                      const int32_t* cache_lens, int32_t num_splits, fd_tensor* out, float* lse,
+                      cudaStream_t stream, PagedCache* pg) {
   DecodeShape sh{};
-  fd_status s = resolve_decode(q, k_cache, v_cache, out, &sh);
+  fd_status s = pg ? resolve_paged(q, k_cache, v_cache, *pg, out, &sh)
+                   : resolve_decode(q, k_cache, v_cache, out, &sh);
   if (s != FD_OK) return s;
   if (num_splits < 0) return fail(FD_ERR_INVALID_ARGUMENT, "num_splits must be >= 0");
   if (num_splits > 65536) return fail(FD_ERR_UNSUPPORTED, "num_splits above 65536");
@@ -451,7 +501,16 @@ fd_status fd_decode_attention(const fd_tensor* q, const fd_tensor* k_cache,
   dp.d = sh.d;
   dp.cap = sh.cap;
   dp.q_box_rows = std::min(16, sh.hq);
-  dp.kv_box_rows = std::min(128, sh.cap);
+  dp.kv_box_rows = std::min(128, pg ? pg->page_size : sh.cap);
+  if (pg) {
+    dp.block_table = pg->block_table;
+    dp.pages_per_seq = pg->pages_per_seq;
+    dp.page_size = pg->page_size;
+    dp.num_pages = static_cast<int32_t>(std::min<int64_t>(k_cache->shape[0], INT32_MAX));
+    dp.align = kPagedKeyAlign;
+  } else {
+    dp.align = 1;
+  }
   dp.scale_log2 = static_cast<float>(1.0 / std::sqrt(static_cast<double>(sh.d)) * 1.4426950408889634);
   dp.hdr = hdr;
   dp.items = items;
@@ -466,7 +525,10 @@ fd_status fd_decode_attention(const fd_tensor* q, const fd_tensor* k_cache,
     const uint64_t qs[2] = {static_cast<uint64_t>(q->stride[1]) * 2, static_cast<uint64_t>(q->stride[0]) * 2};
     const uint32_t qb[3] = {64, static_cast<uint32_t>(dp.q_box_rows), 1};
     if ((s = make_tmap(&tq, q->data, 3, qd, qs, qb, "q")) != FD_OK) return s;
-    const uint64_t kd[4] = {static_cast<uint64_t>(sh.d), static_cast<uint64_t>(sh.cap), static_cast<uint64_t>(sh.hkv), static_cast<uint64_t>(sh.B)};
+    // contiguous: (D, S_cap, Hkv, B); paged: (D, page_size, Hkv, num_pages)
+    const uint64_t rows = pg ? static_cast<uint64_t>(pg->page_size) : static_cast<uint64_t>(sh.cap);
+    const uint64_t outer = static_cast<uint64_t>(k_cache->shape[0]);
+    const uint64_t kd[4] = {static_cast<uint64_t>(sh.d), rows, static_cast<uint64_t>(sh.hkv), outer};
     const uint64_t ks[3] = {static_cast<uint64_t>(k_cache->stride[2]) * 2, static_cast<uint64_t>(k_cache->stride[1]) * 2,
                             static_cast<uint64_t>(k_cache->stride[0]) * 2};
     const uint32_t kb[4] = {64, static_cast<uint32_t>(dp.kv_box_rows), 1, 1};
@@ -482,6 +544,7 @@ fd_status fd_decode_attention(const fd_tensor* q, const fd_tensor* k_cache,
   pp.cap = sh.cap;
   pp.fixed = num_splits;
   pp.nctas = nctas;
+  pp.align = dp.align;
   pp.max_dec_items = max_items;
   pp.hdr = hdr;
   pp.items = items;
@@ -536,6 +599,29 @@ fd_status fd_decode_attention(const fd_tensor* q, const fd_tensor* k_cache,
   if (sh.use_tc) FD_CUDA(launch_combine(cp, stream), "combine kernel launch");
   end_profile_events(ev, 4, stream);
   return FD_OK;
+}
+
+}  // namespace fd_abi
+
+extern "C" {
+
+fd_status fd_decode_attention(const fd_tensor* q, const fd_tensor* k_cache,
+                              const fd_tensor* v_cache, const int32_t* cache_lens,
+                              int32_t num_splits, fd_tensor* out, float* lse, void* stream) {
+  return decode_call(q, k_cache, v_cache, cache_lens, num_splits, out, lse,
+                     static_cast<cudaStream_t>(stream), nullptr);
+}
+
+fd_status fd_decode_attention_paged(const fd_tensor* q, const fd_tensor* k_pages,
+                                    const fd_tensor* v_pages, const int32_t* block_table,
+                                    int32_t pages_per_seq, const int32_t* cache_lens,
+                                    int32_t num_splits, fd_tensor* out, float* lse,
+                                    void* stream) {
+  PagedCache pg{};
+  pg.block_table = block_table;
+  pg.pages_per_seq = pages_per_seq;
+  return decode_call(q, k_pages, v_pages, cache_lens, num_splits, out, lse,
+                     static_cast<cudaStream_t>(stream), &pg);
 }
 
 fd_status fd_chunk_prefill_attention(const fd_tensor* q_chunk, const fd_tensor* k_cache,

@@ -59,6 +59,7 @@ struct __align__(128) SimtSmem {
   int abort_flag;
 };
 
+constexpr int kMaxPageSegs = 128 / 8;  // page segments of one tile (tile <= 128 keys, page >= 8)
 constexpr int kFirstTile = 1;
 constexpr int kLastTile = 2;
 
@@ -117,6 +118,7 @@ __global__ void __launch_bounds__(kSimtThreads) decode_simt_kernel(DecodeParams 
   if (warp == kSimtConsumerWarps) {
     // ---------------- producer: one thread streams K/V tiles ----------------
     if (lane != 0) return;
+    const bool paged = p.block_table != nullptr;
     const int n_items = *reinterpret_cast<volatile int32_t*>(&p.hdr->num_dec_items);
     const uint64_t pol = l2_evict_first_policy();
     uint32_t J = 0;
@@ -137,15 +139,43 @@ __global__ void __launch_bounds__(kSimtThreads) decode_simt_kernel(DecodeParams 
       for (int j = 0; j < ntile; ++j, ++J) {
         if (j == claim_j) nidx = atomicAdd(&p.hdr->dec_counter, 1);
         const int st = J % kSimtStages;
-        if (!mbar_wait(&S.empty[st], ((J / kSimtStages) & 1u) ^ 1u, ctx)) { ok = false; break; }
         const int t = it.t0 + j * C::kTile;
         const int valid = max(0, min(C::kTile, it.t1 - t));
+        // paged cache: the physical page of every page segment of the tile, loaded before the
+        // stage wait so that the loads overlap it (tiles start on multiples of kTile, which
+        // divides 128, and page sizes divide 128 or are multiples of it)
+        int32_t pid[kMaxPageSegs];
+        int nseg = 0, row0 = 0;
+        if (paged && valid > 0) {
+          const int P = p.page_size;
+          const int first = t / P;
+          row0 = t - first * P;
+          nseg = (row0 + valid + P - 1) / P;
+          const int32_t* trow = p.block_table + static_cast<int64_t>(it.b) * p.pages_per_seq;
+#pragma unroll
+          for (int i = 0; i < kMaxPageSegs; ++i) pid[i] = i < nseg ? trow[first + i] : -1;
+        }
+        if (!mbar_wait(&S.empty[st], ((J / kSimtStages) & 1u) ^ 1u, ctx)) { ok = false; break; }
         S.meta[st][0] = idx;
         S.meta[st][1] = t;
         S.meta[st][2] = valid;
         S.meta[st][3] = (j == 0 ? kFirstTile : 0) | (j == ntile - 1 ? kLastTile : 0);
         S.item[st] = it;
-        const uint32_t bytes = static_cast<uint32_t>(valid) * D * sizeof(T);
+        uint32_t bytes = static_cast<uint32_t>(valid) * D * sizeof(T);
+        if (paged && valid > 0) {
+          // a segment whose page index lies outside the pool is not read (FD_FLAG_BAD_PAGE)
+          bool bad = false;
+#pragma unroll
+          for (int i = 0; i < kMaxPageSegs; ++i) {
+            if (i < nseg && (pid[i] < 0 || pid[i] >= p.num_pages)) {
+              bad = true;
+              const int lo = i == 0 ? 0 : i * p.page_size - row0;
+              const int hi = min(valid, (i + 1) * p.page_size - row0);
+              bytes -= static_cast<uint32_t>(hi - lo) * D * sizeof(T);
+            }
+          }
+          if (bad) atomicOr(&p.hdr->status, FD_FLAG_BAD_PAGE);
+        }
         const uint32_t qbytes = j == 0 ? static_cast<uint32_t>(p.g) * D * sizeof(T) : 0u;
         if (bytes + qbytes > 0) {
           mbar_arrive_expect_tx(&S.full[st], 2u * bytes + qbytes);
@@ -155,7 +185,22 @@ __global__ void __launch_bounds__(kSimtThreads) decode_simt_kernel(DecodeParams 
               bulk_load(S.qs[st] + g * D, qrow + static_cast<int64_t>(it.h * p.g + g) * p.q_sh,
                         D * sizeof(T), &S.full[st]);
           }
-          if (bytes) {
+          if (paged) {
+            // segment i: tile rows [lo, hi) from rows [row0 + lo - i P, ...) of page pid[i]
+#pragma unroll
+            for (int i = 0; i < kMaxPageSegs; ++i) {
+              if (i < nseg && pid[i] >= 0 && pid[i] < p.num_pages) {
+                const int lo = i == 0 ? 0 : i * p.page_size - row0;
+                const int hi = min(valid, (i + 1) * p.page_size - row0);
+                const int64_t src = static_cast<int64_t>(pid[i]) * p.kv_sb +
+                                    static_cast<int64_t>(it.h) * p.kv_sh +
+                                    static_cast<int64_t>(row0 + lo - i * p.page_size) * D;
+                const uint32_t nb = static_cast<uint32_t>(hi - lo) * D * sizeof(T);
+                bulk_load(S.k[st] + lo * D, kbase + src, nb, &S.full[st]);
+                bulk_load(S.v[st] + lo * D, vbase + src, nb, &S.full[st]);
+              }
+            }
+          } else if (bytes) {
             bulk_load(S.k[st], kbase + off + static_cast<int64_t>(t) * D, bytes, &S.full[st]);
             bulk_load(S.v[st], vbase + off + static_cast<int64_t>(t) * D, bytes, &S.full[st]);
           }

@@ -77,6 +77,55 @@ struct __align__(1024) TcSmem {
   int abort_flag;
 };
 
+// Physical pages of the 128-key tile that starts at key t (a multiple of 128 in a paged plan)
+// and holds `valid` keys: with page_size >= 128 one box of the tile inside page t / page_size
+// from row t % page_size, else one box per page that holds some of the valid keys. Table
+// entries past the sequence's row are -1 (a TMA coordinate outside the pool, which reads zeros).
+constexpr int kMaxPageBoxes = 128 / 8;
+struct TilePages {
+  int32_t id[kMaxPageBoxes];
+  int n, row0;
+};
+
+__device__ __forceinline__ void tile_pages(const DecodeParams& p, int b, int t, int valid,
+                                           TilePages& tp) {
+  const int P = p.page_size;
+  const int first = t / P;
+  const int32_t* row = p.block_table + static_cast<int64_t>(b) * p.pages_per_seq;
+  tp.n = P >= kTcKeys ? 1 : (valid + P - 1) / P;
+  tp.row0 = P >= kTcKeys ? t - first * P : 0;
+#pragma unroll
+  for (int i = 0; i < kMaxPageBoxes; ++i)
+    tp.id[i] = (i < tp.n && first + i < p.pages_per_seq) ? row[first + i] : -1;
+}
+
+// Issue the K or V loads of one 128-key tile of a paged cache (both 64-column halves): the
+// tp.n boxes of paged_tile_bytes(). A page that holds some of the tile's `valid` keys but whose
+// index lies outside the pool raises FD_FLAG_BAD_PAGE; its copy still runs and reads zeros.
+__device__ __forceinline__ void load_tile_paged(__nv_bfloat16* dst0, __nv_bfloat16* dst1,
+                                                const CUtensorMap* map, uint64_t* bar,
+                                                const TilePages& tp, const DecodeParams& p,
+                                                int h, int valid, uint64_t pol) {
+  const int rows = p.page_size >= kTcKeys ? kTcKeys : p.page_size;
+  bool bad = false;
+#pragma unroll
+  for (int i = 0; i < kMaxPageBoxes; ++i) {
+    if (i < tp.n) {
+      const int32_t id = tp.id[i];
+      bad |= (i * rows < valid) && (id < 0 || id >= p.num_pages);
+      tma_load_4d_stream(dst0 + i * rows * 64, map, bar, 0, tp.row0, h, id, pol);
+      tma_load_4d_stream(dst1 + i * rows * 64, map, bar, 64, tp.row0, h, id, pol);
+    }
+  }
+  if (bad) atomicOr(&p.hdr->status, FD_FLAG_BAD_PAGE);
+}
+
+// Bytes the loads of load_tile_paged deliver (both halves).
+__device__ __forceinline__ uint32_t paged_tile_bytes(const TilePages& tp, const DecodeParams& p) {
+  const int rows = p.page_size >= kTcKeys ? kTcKeys : p.page_size;
+  return 2u * 128u * static_cast<uint32_t>(rows * tp.n);
+}
+
 // dynamic shared memory per CTA, plus the 1024 bytes of alignment slack the kernel may use
 static_assert(sizeof(TcSmem<8>) + 1024 <= 227 * 1024, "tensor-core decode smem (G <= 8)");
 static_assert(sizeof(TcSmem<16>) + 1024 <= 227 * 1024, "tensor-core decode smem (G <= 16)");
@@ -165,6 +214,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const uint32_t tmem = S.tmem_base;
   const WaitCtx ctx{&S.abort_flag, &p.hdr->status};
   const bool fused = p.items == nullptr;
+  const bool paged = p.block_table != nullptr;
   if (fused) {
     // ---- the split plan, computed by every CTA in shared memory (the planner's arithmetic):
     // clamped lengths and their sum, the chunk size, split counts, longest-first ranks, item
@@ -247,7 +297,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     it.b = b;
     it.h = h;
     it.split = s;
-    plan_split_range(S.plan_len[b], n, s, p.fixed, &it.t0, &it.t1);
+    plan_split_range(S.plan_len[b], n, s, p.fixed, p.align, &it.t0, &it.t1);
     it.nsplit = n;
     it.slot = S.plan_rbase[b] * p.hkv + h * n + s;
     return it;
@@ -289,14 +339,20 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           const uint32_t free_parity = ((J / kTcStages) & 1u) ^ 1u;
           const int t = it.t0 + j * kTcKeys;
           const int valid = max(0, min(kTcKeys, it.t1 - t));
-          const uint32_t tx = 2u * 128u * static_cast<uint32_t>(p.kv_box_rows);
+          TilePages tp;
+          if (paged && valid > 0) tile_pages(p, it.b, t, valid, tp);  // loads overlap the wait
           if (!mbar_wait(&S.kempty[st], free_parity, ctx)) { ok = false; break; }
           S.meta[st][0] = t;
           S.meta[st][1] = valid;
           if (valid > 0) {
-            mbar_arrive_expect_tx(&S.kfull[st], tx);
-            tma_load_4d_stream(S.k[st][0], &tmap_k, &S.kfull[st], 0, t, it.h, it.b, pol);
-            tma_load_4d_stream(S.k[st][1], &tmap_k, &S.kfull[st], 64, t, it.h, it.b, pol);
+            mbar_arrive_expect_tx(&S.kfull[st], paged ? paged_tile_bytes(tp, p)
+                                                      : 2u * 128u * static_cast<uint32_t>(p.kv_box_rows));
+            if (paged) {
+              load_tile_paged(S.k[st][0], S.k[st][1], &tmap_k, &S.kfull[st], tp, p, it.h, valid, pol);
+            } else {
+              tma_load_4d_stream(S.k[st][0], &tmap_k, &S.kfull[st], 0, t, it.h, it.b, pol);
+              tma_load_4d_stream(S.k[st][1], &tmap_k, &S.kfull[st], 64, t, it.h, it.b, pol);
+            }
           } else {
             mbar_arrive(&S.kfull[st]);
           }
@@ -344,11 +400,17 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           const int st = J % kTcStages;
           const int t = it.t0 + j * kTcKeys;
           const int valid = max(0, min(kTcKeys, it.t1 - t));
+          TilePages tp;
+          if (paged && valid > 0) tile_pages(p, it.b, t, valid, tp);  // loads overlap the wait
           if (!mbar_wait(&S.vempty[st], ((J / kTcStages) & 1u) ^ 1u, ctx)) { ok = false; break; }
           if (valid > 0) {
-            mbar_arrive_expect_tx(&S.vfull[st], tx);
-            tma_load_4d_stream(S.v[st][0], &tmap_v, &S.vfull[st], 0, t, it.h, it.b, pol);
-            tma_load_4d_stream(S.v[st][1], &tmap_v, &S.vfull[st], 64, t, it.h, it.b, pol);
+            mbar_arrive_expect_tx(&S.vfull[st], paged ? paged_tile_bytes(tp, p) : tx);
+            if (paged) {
+              load_tile_paged(S.v[st][0], S.v[st][1], &tmap_v, &S.vfull[st], tp, p, it.h, valid, pol);
+            } else {
+              tma_load_4d_stream(S.v[st][0], &tmap_v, &S.vfull[st], 0, t, it.h, it.b, pol);
+              tma_load_4d_stream(S.v[st][1], &tmap_v, &S.vfull[st], 64, t, it.h, it.b, pol);
+            }
           } else {
             mbar_arrive(&S.vfull[st]);
           }

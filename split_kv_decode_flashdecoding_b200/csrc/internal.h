@@ -15,6 +15,7 @@ struct PlanParams {
   const int32_t* lens;      // [B] cache lengths (decode) or prefix lengths (chunk mode)
   const int32_t* chunk_lens;  // chunk mode only: [B] chunk lengths; nullptr for decode
   int32_t B, hkv, hq, cap, fixed, nctas;
+  int32_t align;            // split boundaries on multiples of `align` keys (<= 1: unaligned)
   int64_t max_dec_items, max_tile_items, max_rows, max_slots;
   WsHeader* hdr;
   DecodeItem* items;
@@ -57,6 +58,13 @@ struct DecodeParams {
   int32_t B, fixed, plan_ctas, max_items;
   int32_t* row_nsplit_out;
   int32_t* row_base_out;
+  int32_t align;     // split boundaries on multiples of `align` keys (<= 1: unaligned)
+  // paged cache (block_table != nullptr): k and v are [num_pages, Hkv, page_size, D] with kv_sb
+  // the page stride; token t of sequence b is row t % page_size of page
+  // block_table[b * pages_per_seq + t / page_size]. page_size divides 128 or is a multiple of
+  // it, and split boundaries are 128-key aligned, so a key tile never crosses a page.
+  const int32_t* block_table;
+  int32_t pages_per_seq, page_size, num_pages;
 };
 
 __device__ __forceinline__ MergeTarget merge_target(const DecodeParams& p) {

@@ -30,6 +30,7 @@ constexpr int32_t kQTile = 128;           // chunked-prefill query rows per tile
 constexpr int32_t kChunkKvSplit = 2048;   // keys per split of a chunked-prefill query tile
 constexpr int32_t kMaxPlanBatch = 4096;   // largest batch the one-CTA device planner accepts
 constexpr int32_t kFusedPlanMaxBatch = 256;  // largest batch the tensor-core split kernel plans itself
+constexpr int32_t kPagedKeyAlign = 128;      // split boundaries of a paged cache: one key tile
 
 // One split of one (sequence, KV head): keys [t0, t1) of cache row b, output row `row`.
 struct DecodeItem {
@@ -95,12 +96,22 @@ FD_HD int32_t plan_num_splits(int32_t len, int32_t chunk, int32_t fixed) {
 
 // Key range of split s. Fixed mode: [min(s*c, len), min((s+1)*c, len)) with c = ceil(len/n)
 // (the FlashDecoding page's chunk_size rule); planner mode: equal splits
-// [floor(s*len/n), floor((s+1)*len/n)).
-FD_HD void plan_split_range(int32_t len, int32_t n, int32_t s, int32_t fixed, int32_t* t0,
-                            int32_t* t1) {
+// [floor(s*len/n), floor((s+1)*len/n)). With align = A > 1 (a paged cache, so that no key tile
+// crosses a page) every boundary sits on a multiple of A keys: planner mode cuts the
+// U = ceil(len/A) units equally, [min(len, A*floor(s*U/n)), min(len, A*floor((s+1)*U/n))), and
+// fixed mode rounds c up to a multiple of A.
+FD_HD void plan_split_range(int32_t len, int32_t n, int32_t s, int32_t fixed, int32_t align,
+                            int32_t* t0, int32_t* t1) {
   if (fixed > 0) {
     int64_t c = cdiv64(len, n);
+    if (align > 1) c = cdiv64(c, align) * align;
     int64_t a = s * c, e = (s + 1) * c;
+    *t0 = static_cast<int32_t>(a < len ? a : len);
+    *t1 = static_cast<int32_t>(e < len ? e : len);
+  } else if (align > 1) {
+    const int64_t units = cdiv64(len, align);
+    const int64_t a = (static_cast<int64_t>(s) * units / n) * align;
+    const int64_t e = (static_cast<int64_t>(s + 1) * units / n) * align;
     *t0 = static_cast<int32_t>(a < len ? a : len);
     *t1 = static_cast<int32_t>(e < len ? e : len);
   } else {

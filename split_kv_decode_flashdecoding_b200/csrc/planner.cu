@@ -146,7 +146,7 @@ __device__ void plan_decode_body(const PlanParams& p, const int32_t* len_src, in
     const int row = row_of ? row_of[b] : b;
     for (int32_t s = lane; s < n; s += 32) {
       int32_t t0, t1;
-      plan_split_range(L, n, s, p.fixed, &t0, &t1);
+      plan_split_range(L, n, s, p.fixed, p.align, &t0, &t1);
       for (int32_t h = 0; h < p.hkv; ++h) {
         const int32_t i = first + h * n + s;
         if (!overflow) {
@@ -302,7 +302,7 @@ __global__ void __launch_bounds__(kMaxPlanThreads, 1) plan_chunk_kernel(PlanPara
     const int32_t rbase = p.row_base[row];
     for (int32_t s = lane; s < n; s += 32) {
       int32_t t0, t1;
-      plan_split_range(L, n, s, 0, &t0, &t1);
+      plan_split_range(L, n, s, 0, 1, &t0, &t1);
       for (int32_t h = 0; h < p.hkv; ++h) {
         int4* dst = reinterpret_cast<int4*>(p.items + first + h * n + s);
         dst[0] = make_int4(row, b, h, s);

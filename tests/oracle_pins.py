@@ -37,7 +37,8 @@ def _close(a, b, tol=TOL, what=""):
     b = np.asarray(b, dtype=np.float64)
     assert a.shape == b.shape, f"{what}: shape {a.shape} vs {b.shape}"
     both_inf = np.isinf(a) & np.isinf(b) & (np.sign(a) == np.sign(b))
-    err = np.where(both_inf, 0.0, np.abs(a - b))
+    with np.errstate(invalid="ignore"):  # inf - inf where both sides are the same infinity
+        err = np.where(both_inf, 0.0, np.abs(a - b))
     assert np.all(np.isfinite(err)), f"{what}: non-finite mismatch"
     m = float(err.max()) if err.size else 0.0
     assert m <= tol * max(1.0, float(np.abs(np.where(both_inf, 0, b)).max() if b.size else 1.0)), \

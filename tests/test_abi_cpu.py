@@ -16,7 +16,8 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 
 def _declared():
-    src = open(os.path.join(ROOT, "include", "fd.h")).read()
+    with open(os.path.join(ROOT, "include", "fd.h")) as f:
+        src = f.read()
     src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
     return sorted(set(re.findall(r"\b(fd_[a-z_0-9]+)\s*\(", src)))
 
@@ -46,8 +47,9 @@ def test_host_plan_equals_oracle(seed):
     ctas = rng.choice([1, 7, 148, 296])
     fixed = rng.choice([0, 0, 0, 1, 4, 9])
     lens = [rng.choice([0, 1, cap - 1, cap, cap + 5, -2, rng.randint(0, cap)]) for _ in range(B)]
-    info, splits, items = fd.fd_split_plan(lens, hkv, cap, fixed, ctas)
-    ref = P.decode_plan(lens, hkv, cap, ctas, fixed)
+    align = rng.choice([1, 1, 128, 16])
+    info, splits, items = fd.fd_split_plan(lens, hkv, cap, fixed, ctas, key_align=align)
+    ref = P.decode_plan(lens, hkv, cap, ctas, fixed, align=align)
     assert info["chunk_tokens"] == ref.chunk_tokens
     assert splits == ref.splits_per_seq
     assert info["total_items"] == ref.total_items
@@ -68,12 +70,13 @@ def test_host_plan_workload_shapes():
 def test_plan_rejects_bad_arguments():
     info = fd.FdPlanInfo()
     lens = (ctypes.c_int32 * 2)(5, 6)
-    assert fd.lib.fd_split_plan(lens, -1, 1, 8, 0, 1, None, None, 0, ctypes.byref(info)) == 1
-    assert fd.lib.fd_split_plan(lens, 2, 0, 8, 0, 1, None, None, 0, ctypes.byref(info)) == 1
-    assert fd.lib.fd_split_plan(lens, 2, 1, 8, -1, 1, None, None, 0, ctypes.byref(info)) == 1
-    assert fd.lib.fd_split_plan(lens, 2, 1, 8, 0, 0, None, None, 0, ctypes.byref(info)) == 1
-    assert fd.lib.fd_split_plan(None, 2, 1, 8, 0, 1, None, None, 0, ctypes.byref(info)) == 1
-    assert fd.lib.fd_split_plan(lens, 2, 1, 8, 0, 1, None, None, 0, None) == 1
+    assert fd.lib.fd_split_plan(lens, -1, 1, 8, 0, 1, 1, None, None, 0, ctypes.byref(info)) == 1
+    assert fd.lib.fd_split_plan(lens, 2, 0, 8, 0, 1, 1, None, None, 0, ctypes.byref(info)) == 1
+    assert fd.lib.fd_split_plan(lens, 2, 1, 8, -1, 1, 1, None, None, 0, ctypes.byref(info)) == 1
+    assert fd.lib.fd_split_plan(lens, 2, 1, 8, 0, 0, 1, None, None, 0, ctypes.byref(info)) == 1
+    assert fd.lib.fd_split_plan(None, 2, 1, 8, 0, 1, 1, None, None, 0, ctypes.byref(info)) == 1
+    assert fd.lib.fd_split_plan(lens, 2, 1, 8, 0, 1, 0, None, None, 0, ctypes.byref(info)) == 1
+    assert fd.lib.fd_split_plan(lens, 2, 1, 8, 0, 1, 1, None, None, 0, None) == 1
     assert "info" in fd.lib.fd_last_error_message().decode()
 
 

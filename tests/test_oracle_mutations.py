@@ -14,7 +14,8 @@ import pytest
 from oracle_pins import ALL_PINS
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
-SRC = open(os.path.join(ROOT, "oracle", "attention.py")).read()
+with open(os.path.join(ROOT, "oracle", "attention.py")) as _f:
+    SRC = _f.read()
 
 MUTATIONS = {
     "scale_dropped_sqrt": ("scale = 1.0 / math.sqrt(D)", "scale = 1.0 / D"),

@@ -116,6 +116,40 @@ def make_chunk_inputs(prefix_lens: List[int], chunk_lens: List[int], q_heads: in
                        chunk_lens=torch.tensor(chunk_lens, dtype=torch.int32), name=name)
 
 
+@dataclass
+class PagedCache:
+    k_pages: torch.Tensor      # [num_pages, Hkv, page_size, D]
+    v_pages: torch.Tensor
+    block_table: torch.Tensor  # int32 [B, pages_per_seq]; -1 past each sequence's last page
+
+
+def make_paged(k_cache: torch.Tensor, v_cache: torch.Tensor, cache_lens: List[int],
+               page_size: int, seed: int, spare_pages: int = 3,
+               pad_fill: float = float("nan")) -> PagedCache:
+    """Scatter a contiguous cache [B, Hkv, S_cap, D] into pages at seeded, shuffled physical
+    positions. Every sequence gets ceil(S_cap / page_size) table entries; the pages holding its
+    first ceil(len / page_size) * page_size keys are copied, later entries are -1, and the
+    unused physical pages (plus `spare_pages` extra ones) hold `pad_fill`."""
+    B, hkv, cap, d = k_cache.shape
+    pps = max(1, -(-cap // page_size))
+    used = [-(-max(0, min(int(n), cap)) // page_size) for n in cache_lens]
+    npages = sum(used) + spare_pages
+    phys = np.random.default_rng(seed).permutation(max(1, npages))
+    kp = torch.full((max(1, npages), hkv, page_size, d), pad_fill, dtype=k_cache.dtype)
+    vp = torch.full((max(1, npages), hkv, page_size, d), pad_fill, dtype=v_cache.dtype)
+    table = torch.full((B, pps), -1, dtype=torch.int32)
+    i = 0
+    for b in range(B):
+        for j in range(used[b]):
+            pg = int(phys[i])
+            i += 1
+            table[b, j] = pg
+            rows = min(page_size, cap - j * page_size)
+            kp[pg, :, :rows] = k_cache[b, :, j * page_size:j * page_size + rows]
+            vp[pg, :, :rows] = v_cache[b, :, j * page_size:j * page_size + rows]
+    return PagedCache(k_pages=kp, v_pages=vp, block_table=table)
+
+
 # ---- the five named workloads --------------------------------------------------------------
 
 WORKLOADS = {
