@@ -47,6 +47,9 @@ def parse_args():
     ap.add_argument("--workload", type=int, default=3, choices=[1, 2, 3, 4, 5])
     ap.add_argument("--batch", type=int, default=None,
                     help="batch of workload 4; for workloads 3 and 5, keep the first B requests")
+    ap.add_argument("--page-size", type=int, default=0,
+                    help="decode workloads: read the cache through fd_decode_attention_paged, in "
+                         "pages of this many keys at shuffled physical positions (0: contiguous)")
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--profile-calls", type=int, default=200,
                     help="calls timed with per-kernel events after the timed region (0: skip)")
@@ -292,13 +295,24 @@ def run_fd(args, rank, world, local_rank):
     torch.cuda.set_device(dev)
     inp = load_workload(args)
     chunk = is_chunk(inp)
+    paged = args.page_size > 0 and not chunk
+    if paged:
+        from workloads import make_paged
+        pgc = make_paged(inp.k_cache, inp.v_cache, inp.cache_lens.tolist(), args.page_size,
+                         seed=7000 + args.workload, pad_fill=0.0)
+        inp.name = f"{inp.name}_paged{args.page_size}"
     alg = algorithmic_bytes(inp)
     R, hq, d = queries(inp).shape
     B, hkv = inp.k_cache.shape[:2]
     g = hq // hkv
     q = queries(inp).to(dev)
-    k = inp.k_cache.to(dev)
-    v = inp.v_cache.to(dev)
+    if paged:
+        k = pgc.k_pages.to(dev)
+        v = pgc.v_pages.to(dev)
+        table = pgc.block_table.to(dev)
+    else:
+        k = inp.k_cache.to(dev)
+        v = inp.v_cache.to(dev)
     if chunk:
         lens_h = [inp.prefix_lens, inp.chunk_lens]
     else:
@@ -322,8 +336,13 @@ def run_fd(args, rank, world, local_rank):
         # planner, split kernel and, after the tensor-core split kernel, the combine kernel
         launches_per_step = 3 if use_tc else 2
 
-        def step():
-            fd.fd_decode_attention(q, k, v, lens[0], ns, out=out, lse=lse, stream=stream)
+        if paged:
+            def step():
+                fd.fd_decode_attention_paged(q, k, v, table, lens[0], ns, out=out, lse=lse,
+                                             stream=stream)
+        else:
+            def step():
+                fd.fd_decode_attention(q, k, v, lens[0], ns, out=out, lse=lse, stream=stream)
 
     for _ in range(max(3, args.warmup)):
         step()
@@ -402,8 +421,8 @@ def run_fd(args, rank, world, local_rank):
     e2e = None
     if args.e2e_steps > 0:
         hq_ = queries(inp).pin_memory()
-        hk = inp.k_cache.pin_memory()
-        hv = inp.v_cache.pin_memory()
+        hk = (pgc.k_pages if paged else inp.k_cache).pin_memory()
+        hv = (pgc.v_pages if paged else inp.v_cache).pin_memory()
         hl = [t.pin_memory() for t in lens_h]
         ho = torch.empty_like(queries(inp)).pin_memory()
         hlse = torch.empty((R, hq), dtype=torch.float32).pin_memory()
@@ -446,12 +465,15 @@ def run_fd(args, rank, world, local_rank):
                "kind": "oracle", "sample": f"{desc}; {el:.1f}s"}
 
     if rank == 0:
-        config = {"workload": inp.name, "batch": B, "q_heads": hq, "kv_heads": hkv,
+        config = {"workload": inp.name, "batch": R if not chunk else B, "q_heads": hq, "kv_heads": hkv,
                   "head_dim": d, "cache_capacity": int(inp.k_cache.shape[2]),
                   "sum_key_len": int(sum(key_lens(inp))),
                   "num_splits": "planner" if ns == 0 else ns,
                   "algorithmic_bytes_per_call": alg, "input_bytes_resident": input_bytes,
                   "l2": l2_policy, "parallelism": f"replicas x{world}"}
+        if paged:
+            config["page_size"] = args.page_size
+            config["pages_in_pool"] = int(k.shape[0])
         if chunk:
             config["chunk_rows"] = int(R)
             config["chunk_tile_flops_per_call"] = chunk_tile_flops(inp)

@@ -126,6 +126,18 @@ __device__ __forceinline__ bool named_bar_or(uint32_t id, uint32_t nthreads, boo
 // ---- bulk and tensor copies (TMA) ---------------------------------------------------------------
 
 // Contiguous global -> shared copy completing on `bar` (addresses 16 B aligned, size % 16 == 0).
+// 4-byte asynchronous copy global -> shared (no register dependency on the loaded value).
+__device__ __forceinline__ void cp_async_4(void* dst, const void* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(dst)), "l"(src)
+               : "memory");
+}
+// Arrive on `bar` once every cp.async this thread issued so far has completed (the arrival is
+// the barrier's expected one: .noinc).
+__device__ __forceinline__ void cp_async_mbar_arrive(uint64_t* bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar))
+               : "memory");
+}
+
 __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes,
                                           uint64_t* bar) {
   asm volatile(

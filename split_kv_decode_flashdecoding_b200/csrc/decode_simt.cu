@@ -59,7 +59,6 @@ struct __align__(128) SimtSmem {
   int abort_flag;
 };
 
-constexpr int kMaxPageSegs = 128 / 8;  // page segments of one tile (tile <= 128 keys, page >= 8)
 constexpr int kFirstTile = 1;
 constexpr int kLastTile = 2;
 
@@ -141,19 +140,20 @@ __global__ void __launch_bounds__(kSimtThreads) decode_simt_kernel(DecodeParams 
         const int st = J % kSimtStages;
         const int t = it.t0 + j * C::kTile;
         const int valid = max(0, min(C::kTile, it.t1 - t));
-        // paged cache: the physical page of every page segment of the tile, loaded before the
-        // stage wait so that the loads overlap it (tiles start on multiples of kTile, which
-        // divides 128, and page sizes divide 128 or are multiples of it)
-        int32_t pid[kMaxPageSegs];
-        int nseg = 0, row0 = 0;
+        // paged cache: the tile's page segments (tiles start on multiples of kTile, which
+        // divides 128, and page sizes divide 128 or are multiples of it). The first segment's
+        // page is loaded before the stage wait, so that the load overlaps it; a tile that spans
+        // several (short) pages reads the others after the wait.
+        const int32_t* trow = nullptr;
+        int32_t pid0 = -1;
+        int nseg = 0, row0 = 0, first = 0;
         if (paged && valid > 0) {
           const int P = p.page_size;
-          const int first = t / P;
+          first = t / P;
           row0 = t - first * P;
           nseg = (row0 + valid + P - 1) / P;
-          const int32_t* trow = p.block_table + static_cast<int64_t>(it.b) * p.pages_per_seq;
-#pragma unroll
-          for (int i = 0; i < kMaxPageSegs; ++i) pid[i] = i < nseg ? trow[first + i] : -1;
+          trow = p.block_table + static_cast<int64_t>(it.b) * p.pages_per_seq + first;
+          pid0 = trow[0];
         }
         if (!mbar_wait(&S.empty[st], ((J / kSimtStages) & 1u) ^ 1u, ctx)) { ok = false; break; }
         S.meta[st][0] = idx;
@@ -165,9 +165,10 @@ __global__ void __launch_bounds__(kSimtThreads) decode_simt_kernel(DecodeParams 
         if (paged && valid > 0) {
           // a segment whose page index lies outside the pool is not read (FD_FLAG_BAD_PAGE)
           bool bad = false;
-#pragma unroll
-          for (int i = 0; i < kMaxPageSegs; ++i) {
-            if (i < nseg && (pid[i] < 0 || pid[i] >= p.num_pages)) {
+#pragma unroll 1  // kept rolled: the producer loop must stay small in the instruction cache
+          for (int i = 0; i < nseg; ++i) {
+            const int32_t id = i == 0 ? pid0 : trow[i];
+            if (id < 0 || id >= p.num_pages) {
               bad = true;
               const int lo = i == 0 ? 0 : i * p.page_size - row0;
               const int hi = min(valid, (i + 1) * p.page_size - row0);
@@ -187,12 +188,13 @@ __global__ void __launch_bounds__(kSimtThreads) decode_simt_kernel(DecodeParams 
           }
           if (paged) {
             // segment i: tile rows [lo, hi) from rows [row0 + lo - i P, ...) of page pid[i]
-#pragma unroll
-            for (int i = 0; i < kMaxPageSegs; ++i) {
-              if (i < nseg && pid[i] >= 0 && pid[i] < p.num_pages) {
+#pragma unroll 1  // kept rolled: the producer loop must stay small in the instruction cache
+            for (int i = 0; i < nseg; ++i) {
+              const int32_t id = i == 0 ? pid0 : trow[i];
+              if (id >= 0 && id < p.num_pages) {
                 const int lo = i == 0 ? 0 : i * p.page_size - row0;
                 const int hi = min(valid, (i + 1) * p.page_size - row0);
-                const int64_t src = static_cast<int64_t>(pid[i]) * p.kv_sb +
+                const int64_t src = static_cast<int64_t>(id) * p.kv_sb +
                                     static_cast<int64_t>(it.h) * p.kv_sh +
                                     static_cast<int64_t>(row0 + lo - i * p.page_size) * D;
                 const uint32_t nb = static_cast<uint32_t>(hi - lo) * D * sizeof(T);

@@ -41,6 +41,9 @@ constexpr int kSoftmaxThreads = 128;
 constexpr uint32_t kTmemCols = 128;
 constexpr uint32_t kHalfBytes = kTcKeys * 64 * 2;   // one 64-column half of a K or V tile
 
+constexpr int kMaxPageBoxes = 128 / 8;  // page boxes of one key tile (pages of >= 8 keys)
+constexpr int kPidSlots = 8;             // page-id ring of the paged producers
+
 template <int GPAD>
 struct __align__(1024) TcSmem {
   static constexpr int kNO = 2 * GPAD;           // Oᵀ columns: hi then lo
@@ -72,52 +75,80 @@ struct __align__(1024) TcSmem {
   uint64_t ofin[2];    // by item parity: the item's last P·V product has completed
   uint64_t oempty[2];  // by item parity: the epilogue has read that item's O accumulator
   uint64_t lready[2], lfree[2];  // by item parity: hand-off written / read
+  // paged cache: physical page ids of tile J in slot J mod kPidSlots, copied asynchronously by
+  // the Q/K producer two tiles ahead (pidfull) and released by the V producer (pidempty)
+  int32_t pid[kPidSlots][kMaxPageBoxes];
+  uint64_t pidfull[kPidSlots], pidempty[kPidSlots];
   uint64_t drain;
   uint32_t tmem_base;
   int abort_flag;
 };
 
-// Physical pages of the 128-key tile that starts at key t (a multiple of 128 in a paged plan)
-// and holds `valid` keys: with page_size >= 128 one box of the tile inside page t / page_size
-// from row t % page_size, else one box per page that holds some of the valid keys. Table
-// entries past the sequence's row are -1 (a TMA coordinate outside the pool, which reads zeros).
-constexpr int kMaxPageBoxes = 128 / 8;
+// Pages of the 128-key tile that starts at key t (a multiple of 128 in a paged plan) and holds
+// `valid` keys: with page_size >= 128 one box of the tile inside page t / page_size from row
+// t % page_size, else one box per page that holds some of the valid keys.
 struct TilePages {
-  int32_t id[kMaxPageBoxes];
-  int n, row0;
+  int first, n, row0;
 };
 
-__device__ __forceinline__ void tile_pages(const DecodeParams& p, int b, int t, int valid,
-                                           TilePages& tp) {
+__device__ __forceinline__ TilePages tile_pages(const DecodeParams& p, int t, int valid) {
+  TilePages tp;
   const int P = p.page_size;
-  const int first = t / P;
-  const int32_t* row = p.block_table + static_cast<int64_t>(b) * p.pages_per_seq;
-  tp.n = P >= kTcKeys ? 1 : (valid + P - 1) / P;
-  tp.row0 = P >= kTcKeys ? t - first * P : 0;
-#pragma unroll
-  for (int i = 0; i < kMaxPageBoxes; ++i)
-    tp.id[i] = (i < tp.n && first + i < p.pages_per_seq) ? row[first + i] : -1;
+  tp.first = t / P;
+  tp.n = valid <= 0 ? 0 : (P >= kTcKeys ? 1 : (valid + P - 1) / P);
+  tp.row0 = P >= kTcKeys ? t - tp.first * P : 0;
+  return tp;
 }
 
-// Issue the K or V loads of one 128-key tile of a paged cache (both 64-column halves): the
-// tp.n boxes of paged_tile_bytes(). A page that holds some of the tile's `valid` keys but whose
-// index lies outside the pool raises FD_FLAG_BAD_PAGE; its copy still runs and reads zeros.
+// Start the asynchronous copy of the tile's page ids from the block table into `dst` (entries
+// past the sequence's row are not copied; readers take them as -1).
+__device__ __forceinline__ void prefetch_tile_pages(int32_t* dst, const DecodeParams& p, int b,
+                                                    const TilePages& tp) {
+  const int32_t* row = p.block_table + static_cast<int64_t>(b) * p.pages_per_seq;
+#pragma unroll 1  // kept rolled: the producer loops must stay small in the instruction cache
+  for (int i = 0; i < kMaxPageBoxes; ++i)
+    if (i < tp.n && tp.first + i < p.pages_per_seq) cp_async_4(dst + i, row + tp.first + i);
+}
+
+// Page id of the tile starting at key t of sequence b when pages hold >= 128 keys (-1 past the
+// sequence's table row).
+__device__ __forceinline__ int32_t tile_page_id(const DecodeParams& p, int b, int t) {
+  const int first = t / p.page_size;
+  return first < p.pages_per_seq ? p.block_table[static_cast<int64_t>(b) * p.pages_per_seq + first]
+                                 : -1;
+}
+
+// Issue the K or V loads of one 128-key tile of a paged cache (both 64-column halves): the tp.n
+// boxes of paged_tile_bytes(), page ids from `ids` (a slot of the ring). A page that holds some
+// of the tile's `valid` keys but whose index lies outside the pool raises FD_FLAG_BAD_PAGE; its
+// copy still runs and reads zeros (a TMA coordinate outside the tensor).
 __device__ __forceinline__ void load_tile_paged(__nv_bfloat16* dst0, __nv_bfloat16* dst1,
                                                 const CUtensorMap* map, uint64_t* bar,
-                                                const TilePages& tp, const DecodeParams& p,
-                                                int h, int valid, uint64_t pol) {
+                                                const TilePages& tp, const int32_t* ids,
+                                                const DecodeParams& p, int h, int valid,
+                                                uint64_t pol) {
   const int rows = p.page_size >= kTcKeys ? kTcKeys : p.page_size;
   bool bad = false;
-#pragma unroll
+#pragma unroll 1  // kept rolled: the producer loops must stay small in the instruction cache
   for (int i = 0; i < kMaxPageBoxes; ++i) {
     if (i < tp.n) {
-      const int32_t id = tp.id[i];
+      const int32_t id = tp.first + i < p.pages_per_seq ? ids[i] : -1;
       bad |= (i * rows < valid) && (id < 0 || id >= p.num_pages);
       tma_load_4d_stream(dst0 + i * rows * 64, map, bar, 0, tp.row0, h, id, pol);
       tma_load_4d_stream(dst1 + i * rows * 64, map, bar, 64, tp.row0, h, id, pol);
     }
   }
   if (bad) atomicOr(&p.hdr->status, FD_FLAG_BAD_PAGE);
+}
+
+// The loads of one 128-key tile that lies inside one page of >= 128 keys, from row `row0`.
+__device__ __forceinline__ void load_tile_page1(__nv_bfloat16* dst0, __nv_bfloat16* dst1,
+                                                const CUtensorMap* map, uint64_t* bar, int32_t id,
+                                                int row0, const DecodeParams& p, int h,
+                                                uint64_t pol) {
+  if (id < 0 || id >= p.num_pages) atomicOr(&p.hdr->status, FD_FLAG_BAD_PAGE);
+  tma_load_4d_stream(dst0, map, bar, 0, row0, h, id, pol);
+  tma_load_4d_stream(dst1, map, bar, 64, row0, h, id, pol);
 }
 
 // Bytes the loads of load_tile_paged deliver (both halves).
@@ -160,7 +191,10 @@ __device__ __forceinline__ void warp_exclusive_scan(int n, F val, int32_t* out) 
 // without loss, so most tiles skip the exact cross-warp maximum and leave O untouched.
 constexpr float kRescaleThreshold = 8.f;
 
-template <int GPAD>
+// Cache layouts, one kernel instantiation each (the producers' loops stay small).
+enum PageMode : int { kContiguous = 0, kBigPages = 1, kSmallPages = 2 };
+
+template <int GPAD, int kMode>
 __global__ void __launch_bounds__(kTcThreads, 1)
     decode_tc_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmap_q,
                      const __grid_constant__ CUtensorMap tmap_k,
@@ -195,6 +229,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       mbar_init(&S.lready[i], 4);
       mbar_init(&S.lfree[i], 4);
     }
+    for (int i = 0; i < kPidSlots; ++i) {
+      mbar_init(&S.pidfull[i], 1);
+      mbar_init(&S.pidempty[i], 1);
+    }
     mbar_init(&S.drain, 1);
     S.abort_flag = 0;
     fence_mbar_init();
@@ -214,7 +252,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const uint32_t tmem = S.tmem_base;
   const WaitCtx ctx{&S.abort_flag, &p.hdr->status};
   const bool fused = p.items == nullptr;
-  const bool paged = p.block_table != nullptr;
+  constexpr bool paged = kMode != kContiguous;
+  constexpr bool big_pages = kMode == kBigPages;  // pages of >= 128 keys: one page per tile
   if (fused) {
     // ---- the split plan, computed by every CTA in shared memory (the planner's arithmetic):
     // clamped lengths and their sum, the chunk size, split counts, longest-first ranks, item
@@ -319,9 +358,16 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       int idx = atomicAdd(&p.hdr->dec_counter, 1);
       DecodeItem it{};
       if (idx < n_items) it = fused ? fused_item(idx) : p.items[idx];
+      // paged cache: the page ids of global tile pf are copied into the ring two tiles ahead
+      // (pages < 128 keys); with pages of >= 128 keys the one id of the next tile is loaded into
+      // a register one tile ahead and handed to the V producer through the ring
+      uint32_t pf = 0;
+      int32_t id_pre = -1;
+      bool have_pre = false;
       while (ok && idx < n_items) {
         int nidx = n_items;
         DecodeItem nit{};
+        bool have_next = false;
         const int len = it.t1 - it.t0;
         const int ntile = len > 0 ? (len + kTcKeys - 1) / kTcKeys : 1;
         const int ps = K & 1;
@@ -335,28 +381,92 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         const int claim_j = max(0, ntile - 3), read_j = max(0, ntile - 2);
         for (int j = 0; j < ntile; ++j, ++J) {
           if (j == claim_j) nidx = atomicAdd(&p.hdr->dec_counter, 1);
+          if constexpr (paged) {
+            // the page-id prefetch below needs the next item before this tile's copies
+            if (j == read_j && nidx < n_items) {
+              nit = fused ? fused_item(nidx) : p.items[nidx];
+              have_next = true;
+            }
+          }
           const int st = J % kTcStages;
           const uint32_t free_parity = ((J / kTcStages) & 1u) ^ 1u;
           const int t = it.t0 + j * kTcKeys;
           const int valid = max(0, min(kTcKeys, it.t1 - t));
-          TilePages tp;
-          if (paged && valid > 0) tile_pages(p, it.b, t, valid, tp);  // loads overlap the wait
+          TilePages tp{};
+          int32_t id_big = -1;
+          if constexpr (paged) {
+            if constexpr (big_pages) {
+              // this tile's page (loaded an iteration ago); start loading the next tile's
+              id_big = have_pre ? id_pre : tile_page_id(p, it.b, t);
+              have_pre = true;
+              if (j + 1 < ntile) id_pre = tile_page_id(p, it.b, t + kTcKeys);
+              else if (have_next) id_pre = tile_page_id(p, nit.b, nit.t0);
+              else have_pre = false;
+            }
+            // prefetch the page ids of the tiles up to J + 2 that are known (this item's and,
+            // once read, the next item's)
+            while (kMode == kSmallPages && ok && pf <= J + 2) {
+              const int ahead = j + static_cast<int>(pf - J);
+              const DecodeItem* x = nullptr;
+              int jj = 0;
+              if (ahead < ntile) {
+                x = &it;
+                jj = ahead;
+              } else if (have_next) {
+                const int nl = nit.t1 - nit.t0;
+                if (ahead - ntile < (nl > 0 ? (nl + kTcKeys - 1) / kTcKeys : 1)) {
+                  x = &nit;
+                  jj = ahead - ntile;
+                }
+              }
+              if (!x) break;
+              const int slot = pf % kPidSlots;
+              // the V producer has released the slot's previous tile
+              if (!mbar_wait(&S.pidempty[slot], ((pf / kPidSlots) & 1u) ^ 1u, ctx)) { ok = false; break; }
+              const int xt = x->t0 + jj * kTcKeys;
+              prefetch_tile_pages(S.pid[slot], p, x->b, tile_pages(p, xt, min(kTcKeys, x->t1 - xt)));
+              cp_async_mbar_arrive(&S.pidfull[slot]);
+              ++pf;
+            }
+            if (!ok) break;
+            tp = tile_pages(p, t, valid);
+          }
           if (!mbar_wait(&S.kempty[st], free_parity, ctx)) { ok = false; break; }
+          if constexpr (paged) {
+            if constexpr (big_pages) {
+              // hand the id to the V producer: the slot's previous tile has been released
+              const int slot = J % kPidSlots;
+              if (!mbar_wait(&S.pidempty[slot], ((J / kPidSlots) & 1u) ^ 1u, ctx)) { ok = false; break; }
+              S.pid[slot][0] = id_big;
+              mbar_arrive(&S.pidfull[slot]);
+            } else {
+              if (!mbar_wait(&S.pidfull[J % kPidSlots], (J / kPidSlots) & 1u, ctx)) { ok = false; break; }
+            }
+          }
           S.meta[st][0] = t;
           S.meta[st][1] = valid;
           if (valid > 0) {
-            mbar_arrive_expect_tx(&S.kfull[st], paged ? paged_tile_bytes(tp, p)
-                                                      : 2u * 128u * static_cast<uint32_t>(p.kv_box_rows));
-            if (paged) {
-              load_tile_paged(S.k[st][0], S.k[st][1], &tmap_k, &S.kfull[st], tp, p, it.h, valid, pol);
+            if constexpr (paged) {
+              if constexpr (big_pages) {
+                mbar_arrive_expect_tx(&S.kfull[st], 2u * 128u * kTcKeys);
+                load_tile_page1(S.k[st][0], S.k[st][1], &tmap_k, &S.kfull[st], id_big,
+                                t % p.page_size, p, it.h, pol);
+              } else {
+                mbar_arrive_expect_tx(&S.kfull[st], paged_tile_bytes(tp, p));
+                load_tile_paged(S.k[st][0], S.k[st][1], &tmap_k, &S.kfull[st], tp,
+                                S.pid[J % kPidSlots], p, it.h, valid, pol);
+              }
             } else {
+              mbar_arrive_expect_tx(&S.kfull[st], 2u * 128u * static_cast<uint32_t>(p.kv_box_rows));
               tma_load_4d_stream(S.k[st][0], &tmap_k, &S.kfull[st], 0, t, it.h, it.b, pol);
               tma_load_4d_stream(S.k[st][1], &tmap_k, &S.kfull[st], 64, t, it.h, it.b, pol);
             }
           } else {
             mbar_arrive(&S.kfull[st]);
           }
-          if (j == read_j && nidx < n_items) nit = fused ? fused_item(nidx) : p.items[nidx];
+          if constexpr (!paged) {
+            if (j == read_j && nidx < n_items) nit = fused ? fused_item(nidx) : p.items[nidx];
+          }
         }
         ++K;
         idx = nidx;
@@ -370,6 +480,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           mbar_arrive(&S.qfull[ps]);
         }
       }
+      if constexpr (paged) asm volatile("cp.async.wait_all;" ::: "memory");
       if (S.abort_flag) {
         // let copies already issued land before shared memory is released
         for (uint32_t back = 1; back <= kTcStages && back <= J; ++back) {
@@ -400,20 +511,29 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           const int st = J % kTcStages;
           const int t = it.t0 + j * kTcKeys;
           const int valid = max(0, min(kTcKeys, it.t1 - t));
-          TilePages tp;
-          if (paged && valid > 0) tile_pages(p, it.b, t, valid, tp);  // loads overlap the wait
           if (!mbar_wait(&S.vempty[st], ((J / kTcStages) & 1u) ^ 1u, ctx)) { ok = false; break; }
+          if constexpr (paged) {
+            if (!mbar_wait(&S.pidfull[J % kPidSlots], (J / kPidSlots) & 1u, ctx)) { ok = false; break; }
+          }
           if (valid > 0) {
-            mbar_arrive_expect_tx(&S.vfull[st], paged ? paged_tile_bytes(tp, p) : tx);
-            if (paged) {
-              load_tile_paged(S.v[st][0], S.v[st][1], &tmap_v, &S.vfull[st], tp, p, it.h, valid, pol);
+            if constexpr (big_pages) {
+              mbar_arrive_expect_tx(&S.vfull[st], 2u * 128u * kTcKeys);
+              load_tile_page1(S.v[st][0], S.v[st][1], &tmap_v, &S.vfull[st],
+                              S.pid[J % kPidSlots][0], t % p.page_size, p, it.h, pol);
+            } else if constexpr (paged) {
+              const TilePages tp = tile_pages(p, t, valid);
+              mbar_arrive_expect_tx(&S.vfull[st], paged_tile_bytes(tp, p));
+              load_tile_paged(S.v[st][0], S.v[st][1], &tmap_v, &S.vfull[st], tp,
+                              S.pid[J % kPidSlots], p, it.h, valid, pol);
             } else {
+              mbar_arrive_expect_tx(&S.vfull[st], tx);
               tma_load_4d_stream(S.v[st][0], &tmap_v, &S.vfull[st], 0, t, it.h, it.b, pol);
               tma_load_4d_stream(S.v[st][1], &tmap_v, &S.vfull[st], 64, t, it.h, it.b, pol);
             }
           } else {
             mbar_arrive(&S.vfull[st]);
           }
+          if constexpr (paged) mbar_arrive(&S.pidempty[J % kPidSlots]);  // ids read: slot free
         }
         ++K;
       }
@@ -731,11 +851,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   if (tid == 0) release_work_cursor(&p.hdr->dec_counter, &p.hdr->dec_exit);
 }
 
-template <int GPAD>
+template <int GPAD, int kMode>
 cudaError_t launch_tc_t(const DecodeParams& p, const CUtensorMap& tq, const CUtensorMap& tk,
                         const CUtensorMap& tv, int nctas, cudaStream_t stream) {
   const size_t smem = sizeof(TcSmem<GPAD>) + 1024;
-  cudaError_t e = cudaFuncSetAttribute(decode_tc_kernel<GPAD>,
+  cudaError_t e = cudaFuncSetAttribute(decode_tc_kernel<GPAD, kMode>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
@@ -749,7 +869,7 @@ cudaError_t launch_tc_t(const DecodeParams& p, const CUtensorMap& tq, const CUte
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, decode_tc_kernel<GPAD>, p, tq, tk, tv);
+  return cudaLaunchKernelEx(&cfg, decode_tc_kernel<GPAD, kMode>, p, tq, tk, tv);
 }
 
 }  // namespace
@@ -757,8 +877,16 @@ cudaError_t launch_tc_t(const DecodeParams& p, const CUtensorMap& tq, const CUte
 cudaError_t launch_decode_tc(const DecodeParams& p, const CUtensorMap& tmap_q,
                              const CUtensorMap& tmap_k, const CUtensorMap& tmap_v, int nctas,
                              cudaStream_t stream) {
-  if (p.g <= 8) return launch_tc_t<8>(p, tmap_q, tmap_k, tmap_v, nctas, stream);
-  return launch_tc_t<16>(p, tmap_q, tmap_k, tmap_v, nctas, stream);
+  const int mode = p.block_table == nullptr ? kContiguous
+                   : (p.page_size >= kTcKeys ? kBigPages : kSmallPages);
+  if (p.g <= 8) {
+    if (mode == kContiguous) return launch_tc_t<8, kContiguous>(p, tmap_q, tmap_k, tmap_v, nctas, stream);
+    if (mode == kBigPages) return launch_tc_t<8, kBigPages>(p, tmap_q, tmap_k, tmap_v, nctas, stream);
+    return launch_tc_t<8, kSmallPages>(p, tmap_q, tmap_k, tmap_v, nctas, stream);
+  }
+  if (mode == kContiguous) return launch_tc_t<16, kContiguous>(p, tmap_q, tmap_k, tmap_v, nctas, stream);
+  if (mode == kBigPages) return launch_tc_t<16, kBigPages>(p, tmap_q, tmap_k, tmap_v, nctas, stream);
+  return launch_tc_t<16, kSmallPages>(p, tmap_q, tmap_k, tmap_v, nctas, stream);
 }
 
 }  // namespace fd

@@ -125,16 +125,18 @@ class PagedCache:
 
 def make_paged(k_cache: torch.Tensor, v_cache: torch.Tensor, cache_lens: List[int],
                page_size: int, seed: int, spare_pages: int = 3,
-               pad_fill: float = float("nan")) -> PagedCache:
+               pad_fill: float = float("nan"), shuffle: bool = True) -> PagedCache:
     """Scatter a contiguous cache [B, Hkv, S_cap, D] into pages at seeded, shuffled physical
-    positions. Every sequence gets ceil(S_cap / page_size) table entries; the pages holding its
-    first ceil(len / page_size) * page_size keys are copied, later entries are -1, and the
-    unused physical pages (plus `spare_pages` extra ones) hold `pad_fill`."""
+    positions (`shuffle=False`: in order, sequence after sequence, as a fresh allocator hands them
+    out). Every sequence gets ceil(S_cap / page_size) table entries; the pages holding its first
+    ceil(len / page_size) * page_size keys are copied, later entries are -1, and the unused
+    physical pages (plus `spare_pages` extra ones) hold `pad_fill`."""
     B, hkv, cap, d = k_cache.shape
     pps = max(1, -(-cap // page_size))
     used = [-(-max(0, min(int(n), cap)) // page_size) for n in cache_lens]
     npages = sum(used) + spare_pages
-    phys = np.random.default_rng(seed).permutation(max(1, npages))
+    phys = (np.random.default_rng(seed).permutation(max(1, npages)) if shuffle
+            else np.arange(max(1, npages)))
     kp = torch.full((max(1, npages), hkv, page_size, d), pad_fill, dtype=k_cache.dtype)
     vp = torch.full((max(1, npages), hkv, page_size, d), pad_fill, dtype=v_cache.dtype)
     table = torch.full((B, pps), -1, dtype=torch.int32)
