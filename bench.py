@@ -7,6 +7,10 @@ one fd_decode_attention call (device planner + split kernel + LSE combine) over 
 Workload 5 (mixed chunked-prefill step) times one fd_chunk_prefill_attention call instead.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl fd|reference] [--workload 1-5]
+                    [--batch B] [--page-size P]
+
+--page-size P reads a decode workload's cache through fd_decode_attention_paged, in pages of P
+keys at shuffled physical positions.
 
 Prints one JSON line on rank 0. `value` is the whole-job GB/s: the algorithmic bytes every rank
 processed (K+V bytes of the valid keys plus the Q bytes) over the slowest rank's device time.
