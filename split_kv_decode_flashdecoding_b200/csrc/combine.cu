@@ -33,7 +33,7 @@ constexpr int kCombineWarps = 8;
 constexpr int kBatch = 8;  // splits whose loads one warp keeps in flight together
 // Above this many (row, query head) pairs every warp merges a pair of its own (eight pairs per
 // CTA); below, the eight warps of a CTA share one pair's splits.
-constexpr int64_t kWarpPerPairMin = 4096;
+constexpr int64_t kWarpPerPairMin = 1024;
 
 // Online merge of splits s = first, first + step, ... < n of one (row, query head) by one warp:
 // running max m, weight sum wsum, weighted sum acc (kVec elements of D per lane).
