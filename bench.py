@@ -195,6 +195,27 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
+def max_over_ranks(value: float, world: int, device) -> float:
+    """The largest of the ranks' values (all_reduce MAX); the value itself on one rank. Every
+    rank must call it, in the same order as every other collective."""
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    if world > 1:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_gbs(bytes_per_rank_step: int, steps: int, world: int, ms_max: float) -> float:
+    """Whole-job GB/s of `world` replicas, each processing bytes_per_rank_step per step, over the
+    slowest rank's time for `steps` steps."""
+    return world * bytes_per_rank_step * steps / (ms_max * 1e-3) / 1e9
+
+
+def emit(line: dict, rank: int) -> None:
+    """Rank 0 prints the one JSON line; the other ranks stay silent."""
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
 def cpu_threads() -> int:
     try:
         from threadpoolctl import threadpool_info
@@ -289,7 +310,7 @@ def run_reference(args, rank, world):
         "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
-    print(json.dumps(line), flush=True)
+    emit(line, rank)
     return 0
 
 
@@ -369,13 +390,9 @@ def run_fd(args, rank, world, local_rank):
     if world > 1:
         torch.distributed.barrier()
     clocks = sampler.stop() if sampler else None
-    ms_total = e0.elapsed_time(e1)
-    t = torch.tensor([ms_total], dtype=torch.float64, device=dev)
-    if world > 1:
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-    ms_max = float(t.item())
+    ms_max = max_over_ranks(e0.elapsed_time(e1), world, dev)
     ms_per_step = ms_max / args.steps
-    value = world * alg * args.steps / (ms_max * 1e-3) / 1e9
+    value = whole_job_gbs(alg, args.steps, world, ms_max)
 
     # ---- per-kernel durations (same calls, with events between the launches) ----
     nprof = min(args.steps, args.profile_calls)
@@ -454,10 +471,8 @@ def run_fd(args, rank, world, local_rank):
             e2e_step()
         a1.record(stream)
         torch.cuda.synchronize()
-        te = torch.tensor([a0.elapsed_time(a1)], dtype=torch.float64, device=dev)
-        if world > 1:
-            torch.distributed.all_reduce(te, op=torch.distributed.ReduceOp.MAX)
-        e2e = {"value": round(world * alg * args.e2e_steps / (float(te.item()) * 1e-3) / 1e9, 3),
+        te = max_over_ranks(a0.elapsed_time(a1), world, dev)
+        e2e = {"value": round(whole_job_gbs(alg, args.e2e_steps, world, te), 3),
                "unit": "GB/s", "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                "steps": args.e2e_steps,
                "note": "full cache tensors copied host->device every step"}
@@ -496,7 +511,7 @@ def run_fd(args, rank, world, local_rank):
         }
         if roofline_tiles is not None:
             line["roofline_secondary"] = roofline_tiles
-        print(json.dumps(line), flush=True)
+        emit(line, rank)
     return 0
 
 
