@@ -54,6 +54,11 @@ __all__ = [
     "attention_rows",
     "gather_pages",
     "decode_attention_paged",
+    "e4m3_value",
+    "dequant_e4m3",
+    "DequantView",
+    "decode_attention_fp8",
+    "decode_attention_paged_fp8",
 ]
 
 
@@ -240,3 +245,89 @@ def decode_attention_paged(q: np.ndarray, k_pages: np.ndarray, v_pages: np.ndarr
     kc = gather_pages(k_pages, block_table, cache_lens, cap)
     vc = gather_pages(v_pages, block_table, cache_lens, cap)
     return decode_attention(q, kc, vc, cache_lens, scale=scale, rows=rows)
+
+
+# ------------------------------------------------------------------------- FP8 KV cache ---
+#
+# The FlashDecoding page, section "与其他推理加速方案的组合使用" (combining FlashDecoding with
+# other speed-ups), item "Quantization + FlashDecoding", pairs the method with an INT8/FP8 KV
+# cache and has the scores computed on values dequantized to bf16. It names neither the FP8
+# format nor the scale granularity. The reading taken here: the cache holds OCP E4M3 codes
+# (4 exponent bits with bias 7, 3 mantissa bits, no infinities, S.1111.111 is NaN), with one
+# scale for all of K and one for all of V; the cached value of a code c is e4m3(c) * scale.
+# Every E4M3 value has at most 4 significant bits and an exponent inside bf16's range, so
+# "dequantize to bf16" loses nothing, and the definition below is the plain attention over the
+# exact values e4m3(c) * scale.
+
+
+def e4m3_value(code: int) -> float:
+    """Value of one E4M3 code (an integer 0..255), from the format's definition.
+
+    sign s = bit 7, exponent field e = bits 6..3, mantissa field m = bits 2..0:
+      e = 15 and m = 7   -> NaN
+      e = 0              -> (-1)^s * (m / 8) * 2^(1 - 7)      (subnormal)
+      otherwise          -> (-1)^s * (1 + m / 8) * 2^(e - 7)
+    """
+    code = int(code)
+    if not 0 <= code <= 255:
+        raise ValueError("oracle: an E4M3 code is one byte")
+    s = -1.0 if code & 0x80 else 1.0
+    e = (code >> 3) & 0xF
+    m = code & 0x7
+    if e == 15 and m == 7:
+        return math.nan
+    if e == 0:
+        return s * (m / 8.0) * 2.0 ** (1 - 7)
+    return s * (1.0 + m / 8.0) * 2.0 ** (e - 7)
+
+
+_E4M3_TABLE = np.array([e4m3_value(c) for c in range(256)], dtype=np.float64)
+
+
+def dequant_e4m3(codes: np.ndarray, scale: float) -> np.ndarray:
+    """float64 values e4m3(code) * scale of a uint8 array of E4M3 codes."""
+    codes = np.asarray(codes)
+    if codes.dtype != np.uint8:
+        raise TypeError(f"oracle: E4M3 codes must be uint8, got {codes.dtype}")
+    return _E4M3_TABLE[codes] * float(scale)
+
+
+class DequantView:
+    """Read-only view of an array of E4M3 codes as the float64 values e4m3(c) * scale. Indexing
+    it dequantizes only the selected elements, so the definition below reads a large cache one
+    (sequence, KV head) slab at a time, as it reads a bf16 one."""
+
+    def __init__(self, codes: np.ndarray, scale: float):
+        self.codes = np.asarray(codes)
+        if self.codes.dtype != np.uint8:
+            raise TypeError(f"oracle: E4M3 codes must be uint8, got {self.codes.dtype}")
+        self.scale = float(scale)
+        self.shape = self.codes.shape
+        self.dtype = np.dtype(np.float64)
+
+    def __getitem__(self, idx):
+        return dequant_e4m3(self.codes[idx], self.scale)
+
+
+def decode_attention_fp8(q: np.ndarray, k_codes: np.ndarray, v_codes: np.ndarray,
+                         k_scale: float, v_scale: float, cache_lens: Sequence[int],
+                         scale: Optional[float] = None,
+                         rows: Optional[Iterable[Tuple[int, int]]] = None
+                         ) -> Tuple[np.ndarray, np.ndarray]:
+    """Decode attention over an E4M3 cache: ``decode_attention`` (the plain definition) over the
+    dequantized values, K with k_scale and V with v_scale."""
+    kc = DequantView(k_codes, k_scale)
+    vc = DequantView(v_codes, v_scale)
+    return decode_attention(q, kc, vc, cache_lens, scale=scale, rows=rows)
+
+
+def decode_attention_paged_fp8(q: np.ndarray, k_pages: np.ndarray, v_pages: np.ndarray,
+                               k_scale: float, v_scale: float,
+                               block_table: Sequence[Sequence[int]], cache_lens: Sequence[int],
+                               scale: Optional[float] = None,
+                               rows: Optional[Iterable[Tuple[int, int]]] = None
+                               ) -> Tuple[np.ndarray, np.ndarray]:
+    """Paged E4M3 cache: ``decode_attention_paged`` over the dequantized pages."""
+    kp = DequantView(k_pages, k_scale)
+    vp = DequantView(v_pages, v_scale)
+    return decode_attention_paged(q, kp, vp, block_table, cache_lens, scale=scale, rows=rows)

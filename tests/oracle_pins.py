@@ -370,10 +370,118 @@ def pin_paged_swapped_pages(att):
     _close(l[0, 0], s0 + math.log1p(3 * math.exp(-s0)), 1e-12, "LSE of one dominant key")
 
 
+
+# ---- FP8 (E4M3) cache -----------------------------------------------------------------------
+
+def pin_e4m3_closed_forms(att):
+    # values fixed by the E4M3 definition: zeros, the subnormal step 2^-9, the smallest normal
+    # 2^-6, one, the largest finite 448, the NaN codes
+    cases = {0x00: 0.0, 0x80: -0.0, 0x01: 2.0 ** -9, 0x07: 7 * 2.0 ** -9, 0x08: 2.0 ** -6,
+             0x30: 0.5, 0x38: 1.0, 0x3F: 1.875, 0x40: 2.0, 0x7E: 448.0, 0xFE: -448.0,
+             0xB8: -1.0, 0x5A: 20.0}
+    for code, want in cases.items():
+        got = att.e4m3_value(code)
+        assert got == want and math.copysign(1, got) == math.copysign(1, want), (hex(code), got)
+    assert math.isnan(att.e4m3_value(0x7F)) and math.isnan(att.e4m3_value(0xFF))
+    vals = [att.e4m3_value(c) for c in range(0x7F)]
+    assert all(a < b for a, b in zip(vals, vals[1:])), "positive codes are ordered"
+
+
+def pin_e4m3_torch(att):
+    # every code against torch's float8_e4m3fn decoding (a library routine)
+    codes = np.arange(256, dtype=np.uint8)
+    ref = torch.from_numpy(codes).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    got = att.dequant_e4m3(codes, 1.0)
+    same = (got == ref) | (np.isnan(got) & np.isnan(ref))
+    assert same.all(), f"codes {np.nonzero(~same)[0][:8]}"
+    assert np.array_equal(att.dequant_e4m3(codes[:0x7F], 0.375), ref[:0x7F] * 0.375)
+
+
+def _fp8_codes(shape, seed, lo=0x00, hi=0x7E):
+    rng = np.random.default_rng(seed)
+    c = rng.integers(lo, hi + 1, size=shape).astype(np.uint8)
+    return c | (rng.integers(0, 2, size=shape).astype(np.uint8) << 7)   # random signs
+
+
+def pin_fp8_torch_softmax(att):
+    # the whole FP8 path against torch: codes decoded by torch, scores / softmax / logsumexp by
+    # torch in float64
+    B, Hq, Hkv, S, D = 2, 8, 2, 29, 16
+    q = _rand((B, Hq, D), 60)
+    kc = _fp8_codes((B, Hkv, S, D), 61, hi=0x50)
+    vc = _fp8_codes((B, Hkv, S, D), 62)
+    ks, vs = 0.0625, 0.75
+    lens = [29, 11]
+    out, lse = att.decode_attention_fp8(q, kc, vc, ks, vs, lens)
+    tk = torch.from_numpy(kc).view(torch.float8_e4m3fn).to(torch.float64).numpy() * ks
+    tv = torch.from_numpy(vc).view(torch.float8_e4m3fn).to(torch.float64).numpy() * vs
+    ro, rl = _torch_reference(q, tk, tv, lens, 1.0 / math.sqrt(D))
+    _close(out, ro, 1e-11, "fp8 torch O")
+    _close(lse, rl, 1e-11, "fp8 torch LSE")
+
+
+def pin_fp8_scale_laws(att):
+    # v_scale multiplies O and leaves LSE alone; k_scale acts exactly like scaling q
+    B, Hq, Hkv, S, D = 2, 4, 1, 17, 8
+    q = _rand((B, Hq, D), 63)
+    kc = _fp8_codes((B, Hkv, S, D), 64, hi=0x48)
+    vc = _fp8_codes((B, Hkv, S, D), 65)
+    lens = [17, 6]
+    o1, l1 = att.decode_attention_fp8(q, kc, vc, 0.5, 1.0, lens)
+    o2, l2 = att.decode_attention_fp8(q, kc, vc, 0.5, 4.0, lens)
+    _close(o2, 4.0 * o1, 1e-12, "v_scale scales O")
+    _close(l2, l1, 1e-12, "v_scale leaves LSE")
+    o3, l3 = att.decode_attention_fp8(q * 0.5, kc, vc, 1.0, 1.0, lens)
+    _close(o3, o1, 1e-12, "k_scale is a scale of the scores")
+    _close(l3, l1, 1e-12, "k_scale is a scale of the scores (LSE)")
+
+
+def pin_fp8_one_hot(att):
+    # key 3 holds code 0x7E (448) in every element, the others 0x00: with q = 1 it dominates
+    # and O is its V row, v_scale times the E4M3 values of that row's codes
+    S, D = 6, 4
+    kc = np.zeros((1, 1, S, D), dtype=np.uint8)
+    kc[0, 0, 3] = 0x7E
+    vc = np.zeros((1, 1, S, D), dtype=np.uint8)
+    vc[0, 0, 3] = [0x38, 0x40, 0xB8, 0x01]          # 1, 2, -1, 2^-9
+    vc[0, 0, 0] = 0x7E
+    q = np.ones((1, 1, D))
+    out, lse = att.decode_attention_fp8(q, kc, vc, 1.0, 3.0, [S])
+    _close(out[0, 0], 3.0 * np.array([1.0, 2.0, -1.0, 2.0 ** -9]), 1e-12, "fp8 one-hot O")
+    s3 = 448.0 * D / math.sqrt(D)
+    _close(lse[0, 0], s3 + math.log1p((S - 1) * math.exp(-s3)), 1e-12, "fp8 one-hot LSE")
+
+
+def pin_fp8_paged(att):
+    # the paged FP8 form is the contiguous FP8 form over the same codes
+    B, Hkv, psz, D = 2, 2, 4, 8
+    lens = [9, 4]
+    pps = 3
+    kc = _fp8_codes((B, Hkv, pps * psz, D), 66, hi=0x48)
+    vc = _fp8_codes((B, Hkv, pps * psz, D), 67)
+    q = _rand((B, 2 * Hkv, D), 68)
+    order = np.random.default_rng(69).permutation(B * pps)
+    kp = np.zeros((B * pps + 1, Hkv, psz, D), dtype=np.uint8)
+    vp = np.zeros_like(kp)
+    table = [[0] * pps for _ in range(B)]
+    for b in range(B):
+        for j in range(pps):
+            pg = int(order[b * pps + j])
+            table[b][j] = pg
+            kp[pg] = kc[b, :, j * psz:(j + 1) * psz]
+            vp[pg] = vc[b, :, j * psz:(j + 1) * psz]
+    o1, l1 = att.decode_attention_fp8(q, kc, vc, 0.25, 2.0, lens)
+    o2, l2 = att.decode_attention_paged_fp8(q, kp, vp, 0.25, 2.0, table, lens)
+    _close(o2, o1, 1e-12, "paged fp8 O")
+    _close(l2, l1, 1e-12, "paged fp8 LSE")
+
+
 ALL_PINS = [
     pin_golden_decode, pin_golden_chunk, pin_zero_query_is_mean, pin_single_key,
     pin_two_keys_sigmoid, pin_one_hot, pin_equal_scores, pin_empty_and_clamp,
     pin_torch_softmax, pin_chunk_equals_full_causal, pin_chunk_batch_gqa,
     pin_split_invariance, pin_permutation_invariance, pin_page_formulations,
     pin_bf16_widening, pin_paged_equals_contiguous, pin_paged_swapped_pages,
+    pin_e4m3_closed_forms, pin_e4m3_torch, pin_fp8_torch_softmax, pin_fp8_scale_laws,
+    pin_fp8_one_hot, pin_fp8_paged,
 ]

@@ -40,6 +40,19 @@ MUTATIONS = {
     "paged_k_from_v": ("kc = gather_pages(k_pages, block_table, cache_lens, cap)",
                        "kc = gather_pages(v_pages, block_table, cache_lens, cap)"),
     "page_physical_order": ("pg = int(block_table[b][t0 // psz])", "pg = t0 // psz + b"),
+    "e4m3_bias_8": ("return s * (1.0 + m / 8.0) * 2.0 ** (e - 7)",
+                    "return s * (1.0 + m / 8.0) * 2.0 ** (e - 8)"),
+    "e4m3_subnormal_as_normal": ("if e == 0:\n        return s * (m / 8.0) * 2.0 ** (1 - 7)",
+                                 "if e == 0:\n        return s * (1.0 + m / 8.0) * 2.0 ** (0 - 7)"),
+    "e4m3_mantissa_16ths": ("return s * (1.0 + m / 8.0) * 2.0 ** (e - 7)",
+                            "return s * (1.0 + m / 16.0) * 2.0 ** (e - 7)"),
+    "e4m3_sign_dropped": ("s = -1.0 if code & 0x80 else 1.0", "s = 1.0"),
+    "fp8_v_scale_dropped": ("vc = DequantView(v_codes, v_scale)", "vc = DequantView(v_codes, 1.0)"),
+    "fp8_scales_swapped": ("kc = DequantView(k_codes, k_scale)", "kc = DequantView(k_codes, v_scale)"),
+    "fp8_paged_v_scale_for_k": ("kp = DequantView(k_pages, k_scale)",
+                                "kp = DequantView(k_pages, v_scale)"),
+    "fp8_view_drops_scale": ("return dequant_e4m3(self.codes[idx], self.scale)",
+                             "return dequant_e4m3(self.codes[idx], 1.0)"),
 }
 
 

@@ -15,6 +15,9 @@ round-to-nearest-even):
   are drawn without replacement from numpy's default_rng(seed + 200) and those K rows are
   multiplied by ``peak_scale`` in float32 before the cast;
 * cache lengths drawn uniformly, both ends inclusive, with numpy default_rng(seed).
+* E4M3 caches (``make_fp8``) are the bf16 caches above quantized: one scale per tensor,
+  scale = (largest finite |value| over the tensor) / 448 rounded to float32, codes = torch's
+  round-to-nearest cast of value / scale to float8_e4m3fn (NaN padding stays NaN).
 
 The named workloads are the five benchmark shapes of this project (decode MHA fp32, decode
 MHA bf16 13B-like, decode GQA bf16 70B-like, long-context GQA, mixed chunked-prefill step);
@@ -31,7 +34,7 @@ import torch
 
 __all__ = [
     "DecodeInputs", "ChunkInputs", "uniform_lens", "make_decode_inputs", "make_chunk_inputs",
-    "WORKLOADS", "workload", "to_numpy_exact",
+    "WORKLOADS", "workload", "to_numpy_exact", "Fp8Cache", "quantize_e4m3", "make_fp8",
 ]
 
 
@@ -150,6 +153,43 @@ def make_paged(k_cache: torch.Tensor, v_cache: torch.Tensor, cache_lens: List[in
             kp[pg, :, :rows] = k_cache[b, :, j * page_size:j * page_size + rows]
             vp[pg, :, :rows] = v_cache[b, :, j * page_size:j * page_size + rows]
     return PagedCache(k_pages=kp, v_pages=vp, block_table=table)
+
+
+@dataclass
+class Fp8Cache:
+    k_codes: torch.Tensor      # uint8 E4M3 codes, the cache's shape
+    v_codes: torch.Tensor
+    k_scale: float             # the cached value of code c is e4m3(c) * scale
+    v_scale: float
+
+
+def _finite_amax(x: torch.Tensor) -> float:
+    m = 0.0
+    for i in range(x.shape[0]):   # one leading slice at a time (the caches are GBs)
+        xi = x[i].float()
+        xi = torch.where(torch.isfinite(xi), xi.abs(), torch.zeros((), dtype=torch.float32))
+        m = max(m, float(xi.max()) if xi.numel() else 0.0)
+    return m
+
+
+def quantize_e4m3(x: torch.Tensor, scale: float) -> torch.Tensor:
+    """uint8 E4M3 codes of x / scale: torch's round-to-nearest cast, after clamping to the
+    largest finite code (448); NaN stays NaN. Done one leading slice at a time."""
+    out = torch.empty(x.shape, dtype=torch.uint8)
+    for i in range(x.shape[0]):
+        y = torch.clamp(x[i].float() / scale, -448.0, 448.0)
+        out[i] = y.to(torch.float8_e4m3fn).view(torch.uint8)
+    return out
+
+
+def make_fp8(k_cache: torch.Tensor, v_cache: torch.Tensor,
+             k_scale: Optional[float] = None, v_scale: Optional[float] = None) -> Fp8Cache:
+    """E4M3 copy of a cache (or page pool) with one scale per tensor (default: amax / 448 as a
+    float32 number)."""
+    ks = k_scale if k_scale is not None else float(np.float32(max(_finite_amax(k_cache), 1e-30) / 448.0))
+    vs = v_scale if v_scale is not None else float(np.float32(max(_finite_amax(v_cache), 1e-30) / 448.0))
+    return Fp8Cache(k_codes=quantize_e4m3(k_cache, ks), v_codes=quantize_e4m3(v_cache, vs),
+                    k_scale=ks, v_scale=vs)
 
 
 # ---- the five named workloads --------------------------------------------------------------
