@@ -54,6 +54,9 @@ def parse_args():
     ap.add_argument("--page-size", type=int, default=0,
                     help="decode workloads: read the cache through fd_decode_attention_paged, in "
                          "pages of this many keys at shuffled physical positions (0: contiguous)")
+    ap.add_argument("--kv-dtype", choices=["native", "e4m3"], default="native",
+                    help="e4m3: the workload's cache quantized to FP8 E4M3 (one scale per tensor), "
+                         "timed through fd_decode_attention_fp8 / fd_decode_attention_paged_fp8")
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--profile-calls", type=int, default=200,
                     help="calls timed with per-kernel events after the timed region (0: skip)")
@@ -227,9 +230,10 @@ def cpu_threads() -> int:
     return os.cpu_count() or 1
 
 
-def oracle_sample(inp, seconds: float, seed: int = 0):
+def oracle_sample(inp, seconds: float, seed: int = 0, quant=None):
     """Time the oracle on whole (query row, KV head) groups of the workload, all G query heads
-    each, in a seeded order, until `seconds` of host time are spent.
+    each, in a seeded order, until `seconds` of host time are spent. `quant` = (k_scale, v_scale):
+    the cache holds E4M3 codes.
     Returns (bytes/s, description, groups, elapsed)."""
     from oracle import attention as oracle
     from workloads import to_numpy_exact
@@ -254,7 +258,10 @@ def oracle_sample(inp, seconds: float, seed: int = 0):
         vis = key_lens(inp)
 
         def run(rows):
-            oracle.decode_attention(q, k, v, lens, rows=rows)
+            if quant is not None:
+                oracle.decode_attention_fp8(q, k, v, quant[0], quant[1], lens, rows=rows)
+            else:
+                oracle.decode_attention(q, k, v, lens, rows=rows)
     order = np.random.default_rng(seed).permutation(R * hkv)
     done, nbytes = 0, 0
     t0 = time.perf_counter()
@@ -272,11 +279,21 @@ def oracle_sample(inp, seconds: float, seed: int = 0):
 
 
 def load_workload(args):
+    """The workload's inputs and, with --kv-dtype e4m3, its E4M3 cache (the codes replace the
+    bf16 cache tensors; the scales are returned beside them)."""
     from workloads import WORKLOADS, workload
     t0 = time.time()
     inp = workload(args.workload, batch=args.batch)
+    f8 = None
+    if args.kv_dtype == "e4m3":
+        if is_chunk(inp) or inp.k_cache.dtype != torch.bfloat16:
+            raise SystemExit("--kv-dtype e4m3 needs a bf16 decode workload (2, 3 or 4)")
+        from workloads import make_fp8
+        f8 = make_fp8(inp.k_cache, inp.v_cache)
+        inp.k_cache, inp.v_cache = f8.k_codes, f8.v_codes
+        inp.name = f"{inp.name}_e4m3"
     log(f"generated {inp.name} in {time.time() - t0:.1f}s")
-    return inp
+    return inp, f8
 
 
 # ------------------------------------------------------------------------------ arms ----------
@@ -284,15 +301,16 @@ def load_workload(args):
 def run_reference(args, rank, world):
     if rank != 0:
         return 0
-    inp = load_workload(args)
+    inp, f8 = load_workload(args)
+    quant = (f8.k_scale, f8.v_scale) if f8 else None
     per_step = max(0.2, min(5.0, 120.0 / max(1, args.steps + args.warmup)))
     for _ in range(args.warmup):
-        oracle_sample(inp, per_step / 4, seed=1)
+        oracle_sample(inp, per_step / 4, seed=1, quant=quant)
     rates = []
     t0 = time.perf_counter()
     total_bytes = 0
     for s in range(args.steps):
-        r, desc, groups, el = oracle_sample(inp, per_step, seed=100 + s)
+        r, desc, groups, el = oracle_sample(inp, per_step, seed=100 + s, quant=quant)
         rates.append(r)
         total_bytes += r * el
     el = time.perf_counter() - t0
@@ -318,9 +336,10 @@ def run_fd(args, rank, world, local_rank):
     import split_kv_decode_flashdecoding_b200 as fd
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
-    inp = load_workload(args)
+    inp, f8 = load_workload(args)
     chunk = is_chunk(inp)
     paged = args.page_size > 0 and not chunk
+    fp8 = f8 is not None
     if paged:
         from workloads import make_paged
         pgc = make_paged(inp.k_cache, inp.v_cache, inp.cache_lens.tolist(), args.page_size,
@@ -350,7 +369,8 @@ def run_fd(args, rank, world, local_rank):
     input_bytes = sum(t.numel() * t.element_size() for t in (q, k, v))
     l2_policy = ("inputs larger than L2 (valid K/V bytes per call exceed the 126 MB L2)"
                  if alg > 2 * L2_BYTES else "inputs smaller than L2: measured with warm L2")
-    use_tc = inp.k_cache.dtype == torch.bfloat16 and d == 128 and 2 <= g <= 16
+    use_tc = (inp.k_cache.dtype == torch.bfloat16 and d == 128 and 2 <= g <= 16) or \
+             (fp8 and d == 128 and g <= 8)
     if chunk:
         # planner, decode-row split kernel, chunk tile kernel, combine
         launches_per_step = 4
@@ -358,10 +378,20 @@ def run_fd(args, rank, world, local_rank):
         def step():
             fd.fd_chunk_prefill_attention(q, k, v, lens[0], lens[1], out=out, lse=lse, stream=stream)
     else:
-        # planner, split kernel and, after the tensor-core split kernel, the combine kernel
-        launches_per_step = 3 if use_tc else 2
+        # the tensor-core split kernel plans batches of up to 256 sequences itself and is
+        # followed by the combine kernel; the CUDA-core split kernel follows the planner kernel
+        # and merges its splits itself
+        launches_per_step = ((0 if B <= 256 else 1) + 2) if use_tc else 2
 
-        if paged:
+        if fp8 and paged:
+            def step():
+                fd.fd_decode_attention_paged_fp8(q, k, v, f8.k_scale, f8.v_scale, table, lens[0],
+                                                 ns, out=out, lse=lse, stream=stream)
+        elif fp8:
+            def step():
+                fd.fd_decode_attention_fp8(q, k, v, f8.k_scale, f8.v_scale, lens[0], ns, out=out,
+                                           lse=lse, stream=stream)
+        elif paged:
             def step():
                 fd.fd_decode_attention_paged(q, k, v, table, lens[0], ns, out=out, lse=lse,
                                              stream=stream)
@@ -479,7 +509,8 @@ def run_fd(args, rank, world, local_rank):
 
     cpu = None
     if rank == 0 and world == 1 and args.cpu_seconds > 0:
-        rate, desc, groups, el = oracle_sample(inp, args.cpu_seconds)
+        rate, desc, groups, el = oracle_sample(inp, args.cpu_seconds,
+                                               quant=(f8.k_scale, f8.v_scale) if fp8 else None)
         cpu = {"value": round(rate / 1e9, 4), "unit": "GB/s", "cores": cpu_threads(),
                "kind": "oracle", "sample": f"{desc}; {el:.1f}s"}
 
@@ -490,6 +521,8 @@ def run_fd(args, rank, world, local_rank):
                   "num_splits": "planner" if ns == 0 else ns,
                   "algorithmic_bytes_per_call": alg, "input_bytes_resident": input_bytes,
                   "l2": l2_policy, "parallelism": f"replicas x{world}"}
+        if fp8:
+            config["kv_cache"] = {"format": "E4M3", "k_scale": f8.k_scale, "v_scale": f8.v_scale}
         if paged:
             config["page_size"] = args.page_size
             config["pages_in_pool"] = int(k.shape[0])
@@ -500,8 +533,10 @@ def run_fd(args, rank, world, local_rank):
             "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
             "steps": args.steps, "warmup": max(3, args.warmup),
             "ms_per_step": round(ms_per_step, 5), "us_per_call": round(ms_per_step * 1e3, 2),
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16"
-            if inp.k_cache.dtype == torch.bfloat16 else "f32", "data": "synthetic",
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16" if inp.k_cache.dtype == torch.bfloat16 else
+                     ("bf16 (E4M3 cache expanded exactly to bf16)" if fp8 else "f32"),
+            "data": "synthetic",
             "config": config,
             "roofline": roofline,
             "clocks": clocks,

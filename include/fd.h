@@ -58,7 +58,9 @@ typedef enum {
   FD_ERR_WORKSPACE = 4         /* workspace allocation failed or is too small under capture  */
 } fd_status;
 
-typedef enum { FD_F32 = 0, FD_BF16 = 1 } fd_dtype;
+/* FD_E4M3: one-byte OCP FP8 E4M3 codes (4 exponent bits, bias 7, 3 mantissa bits, no
+ * infinities); a KV-cache dtype only, for the *_fp8 entry points. */
+typedef enum { FD_F32 = 0, FD_BF16 = 1, FD_E4M3 = 2 } fd_dtype;
 
 /* A strided device tensor. `stride` is in elements; the last dimension must be contiguous
  * (stride[ndim-1] == 1). Unused trailing shape/stride entries are ignored. */
@@ -145,6 +147,42 @@ fd_status fd_decode_attention_paged(const fd_tensor* q, const fd_tensor* k_pages
                                     int32_t pages_per_seq, const int32_t* cache_lens,
                                     int32_t num_splits, fd_tensor* out, float* lse,
                                     void* stream);
+
+/*
+ * fd_decode_attention_fp8 — fd_decode_attention over an FP8 (E4M3) KV cache.
+ *
+ * The FlashDecoding page, section "与其他推理加速方案的组合使用" (combining FlashDecoding with
+ * other speed-ups), item "Quantization + FlashDecoding", pairs split-KV decoding with an INT8/
+ * FP8 cache whose values are dequantized to bf16 for the score computation. Format and scale
+ * granularity are not given there; they are read as: E4M3 codes, one scale for all of K and one
+ * for all of V, the cached value of code c being e4m3(c) * scale. Every E4M3 value is exact in
+ * bf16, so the kernel expands the codes to bf16 without rounding, folds k_scale into the score
+ * scale and applies v_scale to the output: the result is the attention of fd_decode_attention
+ * over the exact values e4m3(c) * scale, up to fp32 rounding. The NaN codes (0x7F, 0xFF) are
+ * not given a special meaning by the kernel (a quantized cache holds none).
+ *
+ *  q          [B, Hq, D]          FD_BF16; D == 128; group size Hq / Hkv <= 8.
+ *  k_cache    [B, Hkv, S_cap, D]  FD_E4M3 (one byte per element); layout and alignment rules
+ *  v_cache    [B, Hkv, S_cap, D]  as in fd_decode_attention (strides in bytes, multiples of 16).
+ *  k_scale, v_scale               finite, > 0.
+ *  cache_lens, num_splits, out (FD_BF16), lse, stream: as in fd_decode_attention.
+ * Other dtypes, head sizes or group sizes return FD_ERR_UNSUPPORTED.
+ */
+fd_status fd_decode_attention_fp8(const fd_tensor* q, const fd_tensor* k_cache,
+                                  const fd_tensor* v_cache, float k_scale, float v_scale,
+                                  const int32_t* cache_lens, int32_t num_splits, fd_tensor* out,
+                                  float* lse, void* stream);
+
+/*
+ * fd_decode_attention_paged_fp8 — fd_decode_attention_paged over FP8 (E4M3) pages, with the
+ * scales of fd_decode_attention_fp8. k_pages / v_pages are FD_E4M3 [num_pages, Hkv, page_size,
+ * D]; every other argument is as in those two calls.
+ */
+fd_status fd_decode_attention_paged_fp8(const fd_tensor* q, const fd_tensor* k_pages,
+                                        const fd_tensor* v_pages, float k_scale, float v_scale,
+                                        const int32_t* block_table, int32_t pages_per_seq,
+                                        const int32_t* cache_lens, int32_t num_splits,
+                                        fd_tensor* out, float* lse, void* stream);
 
 /*
  * fd_split_plan — the variable-length split planner, on the host (no CUDA call).

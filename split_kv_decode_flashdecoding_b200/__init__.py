@@ -24,11 +24,11 @@ import torch
 
 __all__ = [
     "FdError", "LIB_PATH", "lib", "fd_decode_attention", "fd_decode_attention_paged",
-    "fd_decode_attention_static",
+    "fd_decode_attention_static", "fd_decode_attention_fp8", "fd_decode_attention_paged_fp8",
     "fd_chunk_prefill_attention",
     "fd_split_plan", "fd_split_plan_device", "fd_decode_num_ctas", "fd_decode_workspace_bytes",
     "fd_chunk_workspace_bytes", "fd_reserve_workspace", "fd_poll_status", "fd_profile_begin",
-    "fd_profile_end", "fd_shutdown", "fd_status_string", "FD_F32", "FD_BF16",
+    "fd_profile_end", "fd_shutdown", "fd_status_string", "FD_F32", "FD_BF16", "FD_E4M3",
     "FD_FLAG_LEN_CLAMPED", "FD_FLAG_WAIT_TIMEOUT", "FD_FLAG_PLAN_OVERFLOW", "FD_FLAG_BAD_PAGE",
     "ABI_FUNCTIONS",
 ]
@@ -36,7 +36,7 @@ __all__ = [
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libfd.so")
 
 FD_OK, FD_ERR_INVALID_ARGUMENT, FD_ERR_UNSUPPORTED, FD_ERR_CUDA, FD_ERR_WORKSPACE = range(5)
-FD_F32, FD_BF16 = 0, 1
+FD_F32, FD_BF16, FD_E4M3 = 0, 1, 2
 FD_FLAG_LEN_CLAMPED = 0x1
 FD_FLAG_WAIT_TIMEOUT = 0x2
 FD_FLAG_PLAN_OVERFLOW = 0x4
@@ -82,6 +82,10 @@ ABI_FUNCTIONS = {
     "fd_chunk_prefill_attention": (c_i32, [_TP, _TP, _TP, c_i32p, c_i32p, _TP, c_f32p, c_vp]),
     "fd_decode_attention_paged": (c_i32, [_TP, _TP, _TP, c_i32p, c_i32, c_i32p, c_i32, _TP, c_f32p,
                                           c_vp]),
+    "fd_decode_attention_fp8": (c_i32, [_TP, _TP, _TP, ctypes.c_float, ctypes.c_float, c_i32p,
+                                        c_i32, _TP, c_f32p, c_vp]),
+    "fd_decode_attention_paged_fp8": (c_i32, [_TP, _TP, _TP, ctypes.c_float, ctypes.c_float,
+                                              c_i32p, c_i32, c_i32p, c_i32, _TP, c_f32p, c_vp]),
     "fd_status_string": (ctypes.c_char_p, [c_i32]),
     "fd_last_error_message": (ctypes.c_char_p, []),
     "fd_decode_num_ctas": (c_i32, [c_i32, c_i32, c_i32, c_i32]),
@@ -109,7 +113,9 @@ def _check(status: int, what: str) -> None:
                               f"{lib.fd_last_error_message().decode()}")
 
 
-_DTYPES = {torch.float32: FD_F32, torch.bfloat16: FD_BF16}
+# an E4M3 cache may be passed as torch.float8_e4m3fn or as its uint8 codes
+_DTYPES = {torch.float32: FD_F32, torch.bfloat16: FD_BF16, torch.float8_e4m3fn: FD_E4M3,
+           torch.uint8: FD_E4M3}
 
 
 def _tensor(t: torch.Tensor) -> FdTensor:
@@ -179,6 +185,49 @@ def fd_decode_attention_paged(q: torch.Tensor, k_pages: torch.Tensor, v_pages: t
             _ptr(cache_lens, c_i32), int(num_splits), ctypes.byref(_tensor(out)),
             _ptr(lse, ctypes.c_float), _stream(stream, q.device))
     _check(st, "fd_decode_attention_paged")
+    return out, lse
+
+
+def fd_decode_attention_fp8(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
+                            k_scale: float, v_scale: float, cache_lens: torch.Tensor,
+                            num_splits: int = 0, out: Optional[torch.Tensor] = None,
+                            lse: Optional[torch.Tensor] = None,
+                            stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Decode attention over an E4M3 cache (torch.float8_e4m3fn or uint8 codes, [B,Hkv,S_cap,D]);
+    the cached value of code c is e4m3(c) * scale. q / out bf16."""
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty(q.shape[:2], dtype=torch.float32, device=q.device)
+    with torch.cuda.device(q.device):
+        st = lib.fd_decode_attention_fp8(
+            ctypes.byref(_tensor(q)), ctypes.byref(_tensor(k_cache)), ctypes.byref(_tensor(v_cache)),
+            float(k_scale), float(v_scale), _ptr(cache_lens, c_i32), int(num_splits),
+            ctypes.byref(_tensor(out)), _ptr(lse, ctypes.c_float), _stream(stream, q.device))
+    _check(st, "fd_decode_attention_fp8")
+    return out, lse
+
+
+def fd_decode_attention_paged_fp8(q: torch.Tensor, k_pages: torch.Tensor, v_pages: torch.Tensor,
+                                  k_scale: float, v_scale: float, block_table: torch.Tensor,
+                                  cache_lens: torch.Tensor, num_splits: int = 0,
+                                  out: Optional[torch.Tensor] = None,
+                                  lse: Optional[torch.Tensor] = None,
+                                  stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """fd_decode_attention_paged over E4M3 pages, with the scales of fd_decode_attention_fp8."""
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty(q.shape[:2], dtype=torch.float32, device=q.device)
+    if block_table.dim() != 2 or block_table.stride(1) != 1 or block_table.stride(0) != block_table.shape[1]:
+        raise ValueError("block_table must be a contiguous [B, pages_per_seq] int32 tensor")
+    with torch.cuda.device(q.device):
+        st = lib.fd_decode_attention_paged_fp8(
+            ctypes.byref(_tensor(q)), ctypes.byref(_tensor(k_pages)), ctypes.byref(_tensor(v_pages)),
+            float(k_scale), float(v_scale), _ptr(block_table, c_i32), int(block_table.shape[1]),
+            _ptr(cache_lens, c_i32), int(num_splits), ctypes.byref(_tensor(out)),
+            _ptr(lse, ctypes.c_float), _stream(stream, q.device))
+    _check(st, "fd_decode_attention_paged_fp8")
     return out, lse
 
 

@@ -1,6 +1,7 @@
 // C ABI of the library (include/fd.h): argument validation, the per-(device, stream) workspace,
 // tensor-map construction, kernel dispatch and optional per-launch timing.
 #include <algorithm>
+#include <cfloat>
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
@@ -130,7 +131,8 @@ EncodeTiledFn encode_fn() {
 
 // bf16 tensor map, 128-byte swizzle, 64-element inner box; dims/strides innermost first.
 fd_status make_tmap(CUtensorMap* map, const void* base, int rank, const uint64_t* dims,
-                    const uint64_t* strides_bytes, const uint32_t* box, const char* what) {
+                    const uint64_t* strides_bytes, const uint32_t* box, const char* what,
+                    CUtensorMapDataType dtype) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return fail(FD_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
   cuuint64_t d[5], s[4];
@@ -141,7 +143,7 @@ fd_status make_tmap(CUtensorMap* map, const void* base, int rank, const uint64_t
     es[i] = 1;
     if (i > 0) s[i - 1] = strides_bytes[i - 1];
   }
-  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(base), d, s, b,
+  CUresult r = fn(map, dtype, rank, const_cast<void*>(base), d, s, b,
                   es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(FD_ERR_CUDA, "cuTensorMapEncodeTiled(%s) failed: %d", what, (int)r);
@@ -169,13 +171,13 @@ cudaEvent_t* prof_next() {
 }
 
 // ---------------------------------------------------------------------------- validation -----
-size_t elem_size(int dtype) { return dtype == FD_F32 ? 4 : 2; }
+size_t elem_size(int dtype) { return dtype == FD_F32 ? 4 : (dtype == FD_E4M3 ? 1 : 2); }
 
 fd_status check_tensor(const fd_tensor* t, const char* name, int ndim) {
   if (!t) return fail(FD_ERR_INVALID_ARGUMENT, "%s is NULL", name);
   if (t->ndim != ndim) return fail(FD_ERR_INVALID_ARGUMENT, "%s must have %d dimensions, got %d", name, ndim, t->ndim);
-  if (t->dtype != FD_F32 && t->dtype != FD_BF16)
-    return fail(FD_ERR_UNSUPPORTED, "%s: dtype %d is not FD_F32 or FD_BF16", name, t->dtype);
+  if (t->dtype != FD_F32 && t->dtype != FD_BF16 && t->dtype != FD_E4M3)
+    return fail(FD_ERR_UNSUPPORTED, "%s: dtype %d is not FD_F32, FD_BF16 or FD_E4M3", name, t->dtype);
   for (int i = 0; i < ndim; ++i) {
     if (t->shape[i] < 0) return fail(FD_ERR_INVALID_ARGUMENT, "%s: negative shape[%d]", name, i);
     if (t->shape[i] > INT32_MAX) return fail(FD_ERR_UNSUPPORTED, "%s: shape[%d] exceeds int32", name, i);
@@ -193,7 +195,9 @@ fd_status check_kv(const fd_tensor* k, const fd_tensor* v, int dtype, int B, int
   fd_status s;
   if ((s = check_tensor(k, "k_cache", 4)) != FD_OK) return s;
   if ((s = check_tensor(v, "v_cache", 4)) != FD_OK) return s;
-  if (k->dtype != dtype || v->dtype != dtype) return fail(FD_ERR_INVALID_ARGUMENT, "k_cache / v_cache dtype differs from q");
+  if (k->dtype != dtype || v->dtype != dtype)
+    return fail(FD_ERR_INVALID_ARGUMENT, dtype == FD_E4M3 ? "k_cache / v_cache must be FD_E4M3"
+                                                           : "k_cache / v_cache dtype differs from q");
   for (int i = 0; i < 4; ++i) {
     if (k->shape[i] != v->shape[i]) return fail(FD_ERR_INVALID_ARGUMENT, "k_cache and v_cache shapes differ");
     if (k->stride[i] != v->stride[i]) return fail(FD_ERR_UNSUPPORTED, "k_cache and v_cache must share strides");
@@ -213,6 +217,7 @@ fd_status check_q_out(const fd_tensor* q, const fd_tensor* out, const char* qn) 
   fd_status s;
   if ((s = check_tensor(q, qn, 3)) != FD_OK) return s;
   if ((s = check_tensor(out, "out", 3)) != FD_OK) return s;
+  if (q->dtype == FD_E4M3) return fail(FD_ERR_UNSUPPORTED, "%s: FD_E4M3 is a cache dtype only", qn);
   if (out->dtype != q->dtype) return fail(FD_ERR_INVALID_ARGUMENT, "out dtype differs from %s", qn);
   for (int i = 0; i < 3; ++i)
     if (out->shape[i] != q->shape[i]) return fail(FD_ERR_INVALID_ARGUMENT, "out shape differs from %s", qn);
@@ -222,40 +227,70 @@ fd_status check_q_out(const fd_tensor* q, const fd_tensor* out, const char* qn) 
   return FD_OK;
 }
 
-fd_status resolve_decode(const fd_tensor* q, const fd_tensor* k, const fd_tensor* v,
-                         const fd_tensor* out, DecodeShape* sh) {
-  fd_status s;
-  if ((s = check_q_out(q, out, "q")) != FD_OK) return s;
-  sh->B = static_cast<int>(q->shape[0]);
-  sh->hq = static_cast<int>(q->shape[1]);
-  sh->d = static_cast<int>(q->shape[2]);
-  sh->dtype = q->dtype;
-  if (sh->d != 64 && sh->d != 128) return fail(FD_ERR_UNSUPPORTED, "head_dim %d: only 64 and 128 are supported", sh->d);
-  if ((s = check_kv(k, v, sh->dtype, sh->B, sh->d)) != FD_OK) return s;
-  sh->hkv = static_cast<int>(k->shape[1]);
-  sh->cap = static_cast<int>(k->shape[2]);
-  if (sh->hq < 1 || sh->hq % sh->hkv != 0)
-    return fail(FD_ERR_INVALID_ARGUMENT, "q heads (%d) must be a positive multiple of KV heads (%d)", sh->hq, sh->hkv);
-  sh->g = sh->hq / sh->hkv;
-  if (sh->B > kMaxPlanBatch) return fail(FD_ERR_UNSUPPORTED, "batch %d exceeds %d", sh->B, kMaxPlanBatch);
+// The split kernel of a call: tensor cores for bf16 groups of 2..16 with D 128 (and for every
+// group of <= 8 heads over an E4M3 cache), CUDA cores otherwise.
+fd_status choose_kernel(DecodeShape* sh) {
+  if (sh->kv_fp8) {
+    sh->use_tc = sh->d == 128 && sh->g <= 8;
+    if (!sh->use_tc)
+      return fail(FD_ERR_UNSUPPORTED, "an FP8 cache needs head_dim 128 and group size <= 8 (got %d, %d)",
+                  sh->d, sh->g);
+    return FD_OK;
+  }
   sh->use_tc = sh->dtype == FD_BF16 && sh->d == 128 && sh->g >= 2 && sh->g <= 16;
   if (!sh->use_tc && sh->g > 8)
     return fail(FD_ERR_UNSUPPORTED, "group size %d needs bf16 with head_dim 128 (tensor-core kernel)", sh->g);
   return FD_OK;
 }
 
-fd_status resolve_paged(const fd_tensor* q, const fd_tensor* k, const fd_tensor* v,
-                        PagedCache& pg, const fd_tensor* out, DecodeShape* sh) {
+fd_status check_quant(const fd_tensor* q, const KvQuant* quant) {
+  if (!quant) return FD_OK;
+  if (q->dtype != FD_BF16) return fail(FD_ERR_UNSUPPORTED, "an FP8 cache needs bf16 q and out");
+  const float ks = quant->k_scale, vs = quant->v_scale;
+  if (!(ks > 0.f && ks <= FLT_MAX) || !(vs > 0.f && vs <= FLT_MAX))
+    return fail(FD_ERR_INVALID_ARGUMENT, "k_scale and v_scale must be finite and > 0");
+  return FD_OK;
+}
+
+fd_status resolve_decode(const fd_tensor* q, const fd_tensor* k, const fd_tensor* v,
+                         const fd_tensor* out, DecodeShape* sh, const KvQuant* quant) {
   fd_status s;
   if ((s = check_q_out(q, out, "q")) != FD_OK) return s;
+  if ((s = check_quant(q, quant)) != FD_OK) return s;
   sh->B = static_cast<int>(q->shape[0]);
   sh->hq = static_cast<int>(q->shape[1]);
   sh->d = static_cast<int>(q->shape[2]);
   sh->dtype = q->dtype;
+  sh->kv_fp8 = quant != nullptr;
+  if (sh->d != 64 && sh->d != 128) return fail(FD_ERR_UNSUPPORTED, "head_dim %d: only 64 and 128 are supported", sh->d);
+  if ((s = check_kv(k, v, sh->kv_fp8 ? FD_E4M3 : sh->dtype, sh->B, sh->d)) != FD_OK) return s;
+  sh->hkv = static_cast<int>(k->shape[1]);
+  sh->cap = static_cast<int>(k->shape[2]);
+  if (sh->hq < 1 || sh->hq % sh->hkv != 0)
+    return fail(FD_ERR_INVALID_ARGUMENT, "q heads (%d) must be a positive multiple of KV heads (%d)", sh->hq, sh->hkv);
+  sh->g = sh->hq / sh->hkv;
+  if (sh->B > kMaxPlanBatch) return fail(FD_ERR_UNSUPPORTED, "batch %d exceeds %d", sh->B, kMaxPlanBatch);
+  return choose_kernel(sh);
+}
+
+fd_status resolve_paged(const fd_tensor* q, const fd_tensor* k, const fd_tensor* v,
+                        PagedCache& pg, const fd_tensor* out, DecodeShape* sh,
+                        const KvQuant* quant) {
+  fd_status s;
+  if ((s = check_q_out(q, out, "q")) != FD_OK) return s;
+  if ((s = check_quant(q, quant)) != FD_OK) return s;
+  sh->B = static_cast<int>(q->shape[0]);
+  sh->hq = static_cast<int>(q->shape[1]);
+  sh->d = static_cast<int>(q->shape[2]);
+  sh->dtype = q->dtype;
+  sh->kv_fp8 = quant != nullptr;
+  const int kvt = sh->kv_fp8 ? FD_E4M3 : sh->dtype;
   if (sh->d != 64 && sh->d != 128) return fail(FD_ERR_UNSUPPORTED, "head_dim %d: only 64 and 128 are supported", sh->d);
   if ((s = check_tensor(k, "k_pages", 4)) != FD_OK) return s;
   if ((s = check_tensor(v, "v_pages", 4)) != FD_OK) return s;
-  if (k->dtype != sh->dtype || v->dtype != sh->dtype) return fail(FD_ERR_INVALID_ARGUMENT, "k_pages / v_pages dtype differs from q");
+  if (k->dtype != kvt || v->dtype != kvt)
+    return fail(FD_ERR_INVALID_ARGUMENT, sh->kv_fp8 ? "k_pages / v_pages must be FD_E4M3"
+                                                    : "k_pages / v_pages dtype differs from q");
   for (int i = 0; i < 4; ++i) {
     if (k->shape[i] != v->shape[i]) return fail(FD_ERR_INVALID_ARGUMENT, "k_pages and v_pages shapes differ");
     if (k->stride[i] != v->stride[i]) return fail(FD_ERR_UNSUPPORTED, "k_pages and v_pages must share strides");
@@ -268,7 +303,7 @@ fd_status resolve_paged(const fd_tensor* q, const fd_tensor* k, const fd_tensor*
     return fail(FD_ERR_UNSUPPORTED, "page size %lld: must be 8, 16, 32, 64 or a multiple of 128", (long long)psz);
   if (k->stride[2] != sh->d) return fail(FD_ERR_UNSUPPORTED, "token rows of a page must be contiguous (stride[2] == head_dim)");
   if (sh->B > 0 && (!k->data || !v->data)) return fail(FD_ERR_INVALID_ARGUMENT, "k_pages / v_pages data is NULL");
-  if (!aligned16(k->data) || !aligned16(v->data) || !stride16(k->stride[0], sh->dtype) || !stride16(k->stride[1], sh->dtype))
+  if (!aligned16(k->data) || !aligned16(v->data) || !stride16(k->stride[0], kvt) || !stride16(k->stride[1], kvt))
     return fail(FD_ERR_UNSUPPORTED, "page data and strides must be 16-byte aligned");
   if (sh->B > 0 && !pg.block_table) return fail(FD_ERR_INVALID_ARGUMENT, "block_table is NULL");
   if (pg.pages_per_seq < 1) return fail(FD_ERR_INVALID_ARGUMENT, "pages_per_seq must be >= 1");
@@ -281,10 +316,7 @@ fd_status resolve_paged(const fd_tensor* q, const fd_tensor* k, const fd_tensor*
     return fail(FD_ERR_INVALID_ARGUMENT, "q heads (%d) must be a positive multiple of KV heads (%d)", sh->hq, sh->hkv);
   sh->g = sh->hq / sh->hkv;
   if (sh->B > kMaxPlanBatch) return fail(FD_ERR_UNSUPPORTED, "batch %d exceeds %d", sh->B, kMaxPlanBatch);
-  sh->use_tc = sh->dtype == FD_BF16 && sh->d == 128 && sh->g >= 2 && sh->g <= 16;
-  if (!sh->use_tc && sh->g > 8)
-    return fail(FD_ERR_UNSUPPORTED, "group size %d needs bf16 with head_dim 128 (tensor-core kernel)", sh->g);
-  return FD_OK;
+  return choose_kernel(sh);
 }
 
 int decode_ctas(int dev, bool use_tc) {
@@ -350,7 +382,8 @@ const char* fd_status_string(fd_status s) {
 const char* fd_last_error_message(void) { return g_last_error.c_str(); }
 
 int32_t fd_decode_num_ctas(int32_t device, int32_t dtype, int32_t group_size, int32_t head_dim) {
-  const bool tc = dtype == FD_BF16 && head_dim == 128 && group_size >= 2 && group_size <= 16;
+  const bool tc = (dtype == FD_BF16 && head_dim == 128 && group_size >= 2 && group_size <= 16) ||
+                  (dtype == FD_E4M3 && head_dim == 128 && group_size >= 1 && group_size <= 8);
   return decode_ctas(device, tc);
 }
 
@@ -454,10 +487,10 @@ namespace fd_abi {
 // The decode call of both entry points: a contiguous cache (pg == nullptr) or a paged one.
 fd_status decode_call(const fd_tensor* q, const fd_tensor* k_cache, const fd_tensor* v_cache,
                       const int32_t* cache_lens, int32_t num_splits, fd_tensor* out, float* lse,
-                      cudaStream_t stream, PagedCache* pg) {
+                      cudaStream_t stream, PagedCache* pg, const KvQuant* quant) {
   DecodeShape sh{};
-  fd_status s = pg ? resolve_paged(q, k_cache, v_cache, *pg, out, &sh)
-                   : resolve_decode(q, k_cache, v_cache, out, &sh);
+  fd_status s = pg ? resolve_paged(q, k_cache, v_cache, *pg, out, &sh, quant)
+                   : resolve_decode(q, k_cache, v_cache, out, &sh, quant);
   if (s != FD_OK) return s;
   if (num_splits < 0) return fail(FD_ERR_INVALID_ARGUMENT, "num_splits must be >= 0");
   if (num_splits > 65536) return fail(FD_ERR_UNSUPPORTED, "num_splits above 65536");
@@ -511,7 +544,11 @@ fd_status decode_call(const fd_tensor* q, const fd_tensor* k_cache, const fd_ten
   } else {
     dp.align = 1;
   }
-  dp.scale_log2 = static_cast<float>(1.0 / std::sqrt(static_cast<double>(sh.d)) * 1.4426950408889634);
+  // an E4M3 cache: k_scale multiplies every score, v_scale every output (both linear)
+  dp.scale_log2 = static_cast<float>(1.0 / std::sqrt(static_cast<double>(sh.d)) * 1.4426950408889634 *
+                                     (quant ? static_cast<double>(quant->k_scale) : 1.0));
+  dp.v_scale = quant ? quant->v_scale : 1.f;
+  dp.kv_fp8 = sh.kv_fp8 ? 1 : 0;
   dp.hdr = hdr;
   dp.items = items;
   dp.row_base = row_base;
@@ -528,12 +565,16 @@ fd_status decode_call(const fd_tensor* q, const fd_tensor* k_cache, const fd_ten
     // contiguous: (D, S_cap, Hkv, B); paged: (D, page_size, Hkv, num_pages)
     const uint64_t rows = pg ? static_cast<uint64_t>(pg->page_size) : static_cast<uint64_t>(sh.cap);
     const uint64_t outer = static_cast<uint64_t>(k_cache->shape[0]);
+    // bf16: boxes of 64 elements (one 128-byte swizzle row), two per tile row; E4M3: one box of
+    // 128 one-byte codes per tile row
+    const uint64_t es = sh.kv_fp8 ? 1 : 2;
     const uint64_t kd[4] = {static_cast<uint64_t>(sh.d), rows, static_cast<uint64_t>(sh.hkv), outer};
-    const uint64_t ks[3] = {static_cast<uint64_t>(k_cache->stride[2]) * 2, static_cast<uint64_t>(k_cache->stride[1]) * 2,
-                            static_cast<uint64_t>(k_cache->stride[0]) * 2};
-    const uint32_t kb[4] = {64, static_cast<uint32_t>(dp.kv_box_rows), 1, 1};
-    if ((s = make_tmap(&tk, k_cache->data, 4, kd, ks, kb, "k_cache")) != FD_OK) return s;
-    if ((s = make_tmap(&tv, v_cache->data, 4, kd, ks, kb, "v_cache")) != FD_OK) return s;
+    const uint64_t ks[3] = {static_cast<uint64_t>(k_cache->stride[2]) * es, static_cast<uint64_t>(k_cache->stride[1]) * es,
+                            static_cast<uint64_t>(k_cache->stride[0]) * es};
+    const uint32_t kb[4] = {sh.kv_fp8 ? 128u : 64u, static_cast<uint32_t>(dp.kv_box_rows), 1, 1};
+    const CUtensorMapDataType kt = sh.kv_fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    if ((s = make_tmap(&tk, k_cache->data, 4, kd, ks, kb, "k_cache", kt)) != FD_OK) return s;
+    if ((s = make_tmap(&tv, v_cache->data, 4, kd, ks, kb, "v_cache", kt)) != FD_OK) return s;
   }
 
   PlanParams pp{};
@@ -622,6 +663,28 @@ fd_status fd_decode_attention_paged(const fd_tensor* q, const fd_tensor* k_pages
   pg.pages_per_seq = pages_per_seq;
   return decode_call(q, k_pages, v_pages, cache_lens, num_splits, out, lse,
                      static_cast<cudaStream_t>(stream), &pg);
+}
+
+fd_status fd_decode_attention_fp8(const fd_tensor* q, const fd_tensor* k_cache,
+                                  const fd_tensor* v_cache, float k_scale, float v_scale,
+                                  const int32_t* cache_lens, int32_t num_splits, fd_tensor* out,
+                                  float* lse, void* stream) {
+  const KvQuant quant{k_scale, v_scale};
+  return decode_call(q, k_cache, v_cache, cache_lens, num_splits, out, lse,
+                     static_cast<cudaStream_t>(stream), nullptr, &quant);
+}
+
+fd_status fd_decode_attention_paged_fp8(const fd_tensor* q, const fd_tensor* k_pages,
+                                        const fd_tensor* v_pages, float k_scale, float v_scale,
+                                        const int32_t* block_table, int32_t pages_per_seq,
+                                        const int32_t* cache_lens, int32_t num_splits,
+                                        fd_tensor* out, float* lse, void* stream) {
+  const KvQuant quant{k_scale, v_scale};
+  PagedCache pg{};
+  pg.block_table = block_table;
+  pg.pages_per_seq = pages_per_seq;
+  return decode_call(q, k_pages, v_pages, cache_lens, num_splits, out, lse,
+                     static_cast<cudaStream_t>(stream), &pg, &quant);
 }
 
 fd_status fd_chunk_prefill_attention(const fd_tensor* q_chunk, const fd_tensor* k_cache,

@@ -23,6 +23,13 @@
 // and V halves are refilled independently; keys past the sequence end inside the last tile are
 // masked to p = 0 and their V rows are zeroed in shared memory before the P·V product, so stale
 // or poisoned cache rows never leak. The epilogue of an item overlaps the next item's tiles.
+//
+// E4M3 cache (FlashDecoding page, "与其他推理加速方案的组合使用", item "Quantization +
+// FlashDecoding": scores on values dequantized to bf16). The TMA brings a tile's one-byte codes
+// into a staging area and four more warps (11-14) expand them exactly to bf16: K straight into
+// tensor memory, where the Sᵀ product takes it as its A operand (so the expanded K never costs
+// shared-memory bandwidth), V in place into the bf16 layout of the stage. The key scale is folded
+// into the score scale and the value scale into the output; everything else is the bf16 kernel.
 #include "common.cuh"
 #include "internal.h"
 
@@ -37,6 +44,8 @@ constexpr int kProducerWarp = 4;     // Q and K
 constexpr int kMmaWarp = 5;
 constexpr int kVProducerWarp = 10;
 constexpr int kTcThreads = 11 * 32;
+constexpr int kConvWarp0 = 11;          // E4M3 cache: warps 11-14 expand the codes
+constexpr int kF8Threads = 15 * 32;
 constexpr int kSoftmaxThreads = 128;
 constexpr uint32_t kTmemCols = 128;
 constexpr uint32_t kHalfBytes = kTcKeys * 64 * 2;   // one 64-column half of a K or V tile
@@ -63,7 +72,7 @@ struct __align__(1024) TcSmem {
   int32_t plan_len[kFusedPlanMaxBatch], plan_n[kFusedPlanMaxBatch];
   int32_t plan_order[kFusedPlanMaxBatch], plan_rbase[kFusedPlanMaxBatch];
   int32_t plan_ioff[kFusedPlanMaxBatch + 1];
-  long long plan_red[kTcThreads / 32];
+  long long plan_red[kF8Threads / 32];
   int32_t plan_clamped;
   int32_t item_slot[2][2];                       // item index (-1: stop), tiles
   DecodeItem item[2];                            // the item's descriptor (by item parity)
@@ -75,6 +84,9 @@ struct __align__(1024) TcSmem {
   uint64_t ofin[2];    // by item parity: the item's last P·V product has completed
   uint64_t oempty[2];  // by item parity: the epilogue has read that item's O accumulator
   uint64_t lready[2], lfree[2];  // by item parity: hand-off written / read
+  // E4M3 cache: the TMA completes these (codes in the staging area); kfull / vfull then mean
+  // "expanded to bf16" and are completed by the four expanding warps
+  uint64_t kraw[kTcStages], vraw[kTcStages];
   // paged cache: physical page ids of tile J in slot J mod kPidSlots, copied asynchronously by
   // the Q/K producer two tiles ahead (pidfull) and released by the V producer (pidempty)
   int32_t pid[kPidSlots][kMaxPageBoxes];
@@ -122,6 +134,8 @@ __device__ __forceinline__ int32_t tile_page_id(const DecodeParams& p, int b, in
 // boxes of paged_tile_bytes(), page ids from `ids` (a slot of the ring). A page that holds some
 // of the tile's `valid` keys but whose index lies outside the pool raises FD_FLAG_BAD_PAGE; its
 // copy still runs and reads zeros (a TMA coordinate outside the tensor).
+// An E4M3 cache (kF8) has one 128-byte box per row, into the upper half (the staging area).
+template <bool kF8>
 __device__ __forceinline__ void load_tile_paged(__nv_bfloat16* dst0, __nv_bfloat16* dst1,
                                                 const CUtensorMap* map, uint64_t* bar,
                                                 const TilePages& tp, const int32_t* ids,
@@ -134,27 +148,93 @@ __device__ __forceinline__ void load_tile_paged(__nv_bfloat16* dst0, __nv_bfloat
     if (i < tp.n) {
       const int32_t id = tp.first + i < p.pages_per_seq ? ids[i] : -1;
       bad |= (i * rows < valid) && (id < 0 || id >= p.num_pages);
-      tma_load_4d_stream(dst0 + i * rows * 64, map, bar, 0, tp.row0, h, id, pol);
-      tma_load_4d_stream(dst1 + i * rows * 64, map, bar, 64, tp.row0, h, id, pol);
+      if constexpr (kF8) {
+        tma_load_4d_stream(reinterpret_cast<unsigned char*>(dst1) + i * rows * 128, map, bar, 0,
+                           tp.row0, h, id, pol);
+      } else {
+        tma_load_4d_stream(dst0 + i * rows * 64, map, bar, 0, tp.row0, h, id, pol);
+        tma_load_4d_stream(dst1 + i * rows * 64, map, bar, 64, tp.row0, h, id, pol);
+      }
     }
   }
   if (bad) atomicOr(&p.hdr->status, FD_FLAG_BAD_PAGE);
 }
 
 // The loads of one 128-key tile that lies inside one page of >= 128 keys, from row `row0`.
+template <bool kF8>
 __device__ __forceinline__ void load_tile_page1(__nv_bfloat16* dst0, __nv_bfloat16* dst1,
                                                 const CUtensorMap* map, uint64_t* bar, int32_t id,
                                                 int row0, const DecodeParams& p, int h,
                                                 uint64_t pol) {
   if (id < 0 || id >= p.num_pages) atomicOr(&p.hdr->status, FD_FLAG_BAD_PAGE);
-  tma_load_4d_stream(dst0, map, bar, 0, row0, h, id, pol);
-  tma_load_4d_stream(dst1, map, bar, 64, row0, h, id, pol);
+  if constexpr (kF8) {
+    tma_load_4d_stream(dst1, map, bar, 0, row0, h, id, pol);
+  } else {
+    tma_load_4d_stream(dst0, map, bar, 0, row0, h, id, pol);
+    tma_load_4d_stream(dst1, map, bar, 64, row0, h, id, pol);
+  }
 }
 
-// Bytes the loads of load_tile_paged deliver (both halves).
+// Bytes the loads of load_tile_paged deliver (both halves; E4M3: one byte per element).
+template <bool kF8>
 __device__ __forceinline__ uint32_t paged_tile_bytes(const TilePages& tp, const DecodeParams& p) {
   const int rows = p.page_size >= kTcKeys ? kTcKeys : p.page_size;
-  return 2u * 128u * static_cast<uint32_t>(rows * tp.n);
+  return (kF8 ? 1u : 2u) * 128u * static_cast<uint32_t>(rows * tp.n);
+}
+
+// Four E4M3 codes (the bytes of w, the first in the low byte) as two bf16 pairs, exactly. For a
+// code s.eeee.mmm the 16-bit pattern s.0000eeee.mmm0000 is a bf16 whose value is the code's
+// value times 2^-120 (a subnormal code, eeee = 0, lands on a bf16 subnormal the same way), and
+// one bf16 multiply by 2^120 restores it. The byte permute puts each code in the high byte of a
+// 16-bit lane with the code's sign replicated in the byte above the lower lane, so one
+// arithmetic shift and one mask place every bit. The NaN codes come out as +-480.
+__device__ __forceinline__ void e4m3x4_to_bf16(uint32_t w, uint32_t& lo, uint32_t& hi) {
+  uint32_t t0, t1;
+  asm("prmt.b32 %0, %1, %2, 0x1804;" : "=r"(t0) : "r"(w), "r"(0u));  // [0, c0, sign(c0), c1]
+  asm("prmt.b32 %0, %1, %2, 0x3A24;" : "=r"(t1) : "r"(w), "r"(0u));  // [0, c2, sign(c2), c3]
+  t0 = static_cast<uint32_t>(static_cast<int32_t>(t0) >> 4) & 0x87F087F0u;
+  t1 = static_cast<uint32_t>(static_cast<int32_t>(t1) >> 4) & 0x87F087F0u;
+  const uint32_t two120 = 0x7B807B80u;  // bf16 2^120 in both lanes
+  __nv_bfloat162 a, b, k;
+  memcpy(&a, &t0, 4);
+  memcpy(&b, &t1, 4);
+  memcpy(&k, &two120, 4);
+  a = __hmul2(a, k);
+  b = __hmul2(b, k);
+  memcpy(&lo, &a, 4);
+  memcpy(&hi, &b, 4);
+}
+
+// In-place expansion of one V tile of an E4M3 cache by 128 threads (ct = 0..127). The TMA put
+// the 128 rows of 128 codes (128-byte swizzle) into the upper 64-column half of the stage; the
+// bf16 rows go to both halves in the layout of a bf16 tile, rows >= valid as zeros. The upper
+// half of bf16 row r takes exactly the bytes of code row r, and the eight lanes that expand a
+// row load all of its codes in one instruction before the warp stores anything, so no code is
+// overwritten before it is read.
+__device__ __forceinline__ void expand_v_tile(__nv_bfloat16 (&buf)[2][kTcKeys * 64], int ct,
+                                              int valid) {
+  unsigned char* h0 = reinterpret_cast<unsigned char*>(buf[0]);
+  unsigned char* h1 = reinterpret_cast<unsigned char*>(buf[1]);
+#pragma unroll 2
+  for (int i = 0; i < kTcKeys * 8 / 128; ++i) {
+    const int id = i * 128 + ct;
+    const int r = id >> 3, c = id & 7, x = r & 7;
+    const uint4 w = *reinterpret_cast<const uint4*>(h1 + r * 128 + ((c ^ x) << 4));
+    __syncwarp();
+    uint4 a, b;  // bf16 of elements 16c .. 16c+7 and 16c+8 .. 16c+15
+    e4m3x4_to_bf16(w.x, a.x, a.y);
+    e4m3x4_to_bf16(w.y, a.z, a.w);
+    e4m3x4_to_bf16(w.z, b.x, b.y);
+    e4m3x4_to_bf16(w.w, b.z, b.w);
+    if (r >= valid) a = b = make_uint4(0u, 0u, 0u, 0u);
+    const bool upper = c >= 4;
+    const int ca = (2 * (c & 3)) ^ x;  // swizzled 16-byte slot of elements 16c .. 16c+7
+    unsigned char* row = (upper ? h1 : h0) + r * 128;
+    // lanes of the lower half store their even slot first, those of the upper half their odd
+    // one, so each store instruction covers 8 distinct bank groups of a row
+    *reinterpret_cast<uint4*>(row + ((upper ? ca ^ 1 : ca) << 4)) = upper ? b : a;
+    *reinterpret_cast<uint4*>(row + ((upper ? ca : ca ^ 1) << 4)) = upper ? a : b;
+  }
 }
 
 // dynamic shared memory per CTA, plus the 1024 bytes of alignment slack the kernel may use
@@ -194,14 +274,21 @@ constexpr float kRescaleThreshold = 8.f;
 // Cache layouts, one kernel instantiation each (the producers' loops stay small).
 enum PageMode : int { kContiguous = 0, kBigPages = 1, kSmallPages = 2 };
 
-template <int GPAD, int kMode>
-__global__ void __launch_bounds__(kTcThreads, 1)
+template <int GPAD, int kMode, bool kF8>
+__global__ void __launch_bounds__(kF8 ? kF8Threads : kTcThreads, 1)
     decode_tc_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmap_q,
                      const __grid_constant__ CUtensorMap tmap_k,
                      const __grid_constant__ CUtensorMap tmap_v) {
   using Smem = TcSmem<GPAD>;
   constexpr int kNO = Smem::kNO;
+  constexpr int kThreads = kF8 ? kF8Threads : kTcThreads;
   constexpr uint32_t kColO = 32;  // Sᵀ buffers at columns [0, 32), O accumulators after them
+  // E4M3 cache: the expanded K tile of each stage (128 key lanes x 64 columns of bf16 pairs)
+  constexpr uint32_t kColK = kColO + 2 * kNO;
+  constexpr uint32_t kCols = kF8 ? 256 : kTmemCols;
+  static_assert(!kF8 || kColK + kTcStages * 64 <= kCols, "tensor memory of the E4M3 kernel");
+  static_assert(!kF8 || GPAD == 8, "the E4M3 kernel serves groups of <= 8 heads");
+  constexpr uint32_t kRowBytes = kF8 ? 128u : 256u;  // bytes of one cached K or V row
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   // dynamic shared memory is only guaranteed 16-byte aligned: round up to 1024 for SW128
   Smem& S = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -211,10 +298,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 
   if (tid == 0) {
     for (int s = 0; s < kTcStages; ++s) {
-      mbar_init(&S.kfull[s], 1);
-      mbar_init(&S.vfull[s], 1);
+      mbar_init(&S.kfull[s], kF8 ? 4 : 1);
+      mbar_init(&S.vfull[s], kF8 ? 4 : 1);
       mbar_init(&S.kempty[s], 1);
       mbar_init(&S.vempty[s], 1);
+      mbar_init(&S.kraw[s], 1);
+      mbar_init(&S.vraw[s], 1);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&S.qfull[i], 1);
@@ -238,7 +327,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     fence_mbar_init();
   }
   if (warp == kMmaWarp) {
-    tmem_alloc(&S.tmem_base, kTmemCols);
+    tmem_alloc(&S.tmem_base, kCols);
     tmem_relinquish();
   }
   if (warp == kProducerWarp && lane == 0) {
@@ -262,7 +351,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const int B = p.B;
     long long local = 0;
     bool clamped = false;
-    for (int b = tid; b < B; b += kTcThreads) {
+    for (int b = tid; b < B; b += kThreads) {
       const int32_t raw = p.lens[b];
       const int32_t L = clamp_len(raw, p.cap);
       clamped |= L != raw;
@@ -278,16 +367,16 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     if (lane == 0 && clamped) S.plan_clamped = 1;
     long long total = 0;
 #pragma unroll
-    for (int w = 0; w < kTcThreads / 32; ++w) total += S.plan_red[w];
+    for (int w = 0; w < kThreads / 32; ++w) total += S.plan_red[w];
     const int32_t chunk = p.fixed > 0 ? 0 : plan_chunk_tokens(total, p.hkv, p.plan_ctas);
-    for (int b = tid; b < B; b += kTcThreads) {
+    for (int b = tid; b < B; b += kThreads) {
       const int32_t n = plan_num_splits(S.plan_len[b], chunk, p.fixed);
       S.plan_n[b] = n;
       S.plan_ioff[b] = plan_sort_key(S.plan_len[b], n);  // sort keys until the scan below
     }
     __syncthreads();
     // longest first: rank = sequences with a larger key, or an equal key and a smaller index
-    for (int b = tid; b < B; b += kTcThreads) {
+    for (int b = tid; b < B; b += kThreads) {
       const int32_t kb = S.plan_ioff[b];
       int r = 0;
       for (int j = 0; j < B; ++j) {
@@ -312,7 +401,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const bool fused_overflow = fused && fused_items > p.max_items;
   if (fused && blockIdx.x == 0) {
     // the combine kernel's row tables, and the status flags the planner would raise
-    for (int b = tid; b < p.B; b += kTcThreads) {
+    for (int b = tid; b < p.B; b += kThreads) {
       p.row_nsplit_out[b] = S.plan_n[b];
       p.row_base_out[b] = S.plan_rbase[b];
     }
@@ -445,24 +534,30 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           }
           S.meta[st][0] = t;
           S.meta[st][1] = valid;
+          // bf16: the copy completes kfull; E4M3: it completes kraw, the expanding warps kfull
+          uint64_t* kbar = kF8 ? &S.kraw[st] : &S.kfull[st];
           if (valid > 0) {
             if constexpr (paged) {
               if constexpr (big_pages) {
-                mbar_arrive_expect_tx(&S.kfull[st], 2u * 128u * kTcKeys);
-                load_tile_page1(S.k[st][0], S.k[st][1], &tmap_k, &S.kfull[st], id_big,
-                                t % p.page_size, p, it.h, pol);
+                mbar_arrive_expect_tx(kbar, kRowBytes * kTcKeys);
+                load_tile_page1<kF8>(S.k[st][0], S.k[st][1], &tmap_k, kbar, id_big,
+                                     t % p.page_size, p, it.h, pol);
               } else {
-                mbar_arrive_expect_tx(&S.kfull[st], paged_tile_bytes(tp, p));
-                load_tile_paged(S.k[st][0], S.k[st][1], &tmap_k, &S.kfull[st], tp,
-                                S.pid[J % kPidSlots], p, it.h, valid, pol);
+                mbar_arrive_expect_tx(kbar, paged_tile_bytes<kF8>(tp, p));
+                load_tile_paged<kF8>(S.k[st][0], S.k[st][1], &tmap_k, kbar, tp,
+                                     S.pid[J % kPidSlots], p, it.h, valid, pol);
               }
             } else {
-              mbar_arrive_expect_tx(&S.kfull[st], 2u * 128u * static_cast<uint32_t>(p.kv_box_rows));
-              tma_load_4d_stream(S.k[st][0], &tmap_k, &S.kfull[st], 0, t, it.h, it.b, pol);
-              tma_load_4d_stream(S.k[st][1], &tmap_k, &S.kfull[st], 64, t, it.h, it.b, pol);
+              mbar_arrive_expect_tx(kbar, kRowBytes * static_cast<uint32_t>(p.kv_box_rows));
+              if constexpr (kF8) {
+                tma_load_4d_stream(S.k[st][1], &tmap_k, kbar, 0, t, it.h, it.b, pol);
+              } else {
+                tma_load_4d_stream(S.k[st][0], &tmap_k, kbar, 0, t, it.h, it.b, pol);
+                tma_load_4d_stream(S.k[st][1], &tmap_k, kbar, 64, t, it.h, it.b, pol);
+              }
             }
           } else {
-            mbar_arrive(&S.kfull[st]);
+            mbar_arrive(kbar);
           }
           if constexpr (!paged) {
             if (j == read_j && nidx < n_items) nit = fused ? fused_item(nidx) : p.items[nidx];
@@ -479,13 +574,22 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           S.item_slot[ps][1] = 0;
           mbar_arrive(&S.qfull[ps]);
         }
+        if constexpr (kF8) {
+          // the expanding warps follow the stages, not the items: a stage without a tile (valid
+          // -1) stops them, once the stage's previous tile has been consumed
+          const int st = J % kTcStages;
+          if (mbar_wait(&S.kempty[st], ((J / kTcStages) & 1u) ^ 1u, ctx)) {
+            S.meta[st][1] = -1;
+            mbar_arrive(&S.kraw[st]);
+          }
+        }
       }
       if constexpr (paged) asm volatile("cp.async.wait_all;" ::: "memory");
       if (S.abort_flag) {
         // let copies already issued land before shared memory is released
         for (uint32_t back = 1; back <= kTcStages && back <= J; ++back) {
           const uint32_t jj = J - back;
-          mbar_drain(&S.kfull[jj % kTcStages], (jj / kTcStages) & 1u);
+          mbar_drain(kF8 ? &S.kraw[jj % kTcStages] : &S.kfull[jj % kTcStages], (jj / kTcStages) & 1u);
         }
       }
     }
@@ -496,7 +600,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     // of its previous tile has completed, independently of the K half.
     if (lane == 0) {
       const uint64_t pol = l2_evict_first_policy();
-      const uint32_t tx = 2u * 128u * static_cast<uint32_t>(p.kv_box_rows);
+      const uint32_t tx = kRowBytes * static_cast<uint32_t>(p.kv_box_rows);
       uint32_t J = 0, K = 0;
       bool ok = true;
       while (ok) {
@@ -515,23 +619,28 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           if constexpr (paged) {
             if (!mbar_wait(&S.pidfull[J % kPidSlots], (J / kPidSlots) & 1u, ctx)) { ok = false; break; }
           }
+          uint64_t* vbar = kF8 ? &S.vraw[st] : &S.vfull[st];
           if (valid > 0) {
             if constexpr (big_pages) {
-              mbar_arrive_expect_tx(&S.vfull[st], 2u * 128u * kTcKeys);
-              load_tile_page1(S.v[st][0], S.v[st][1], &tmap_v, &S.vfull[st],
-                              S.pid[J % kPidSlots][0], t % p.page_size, p, it.h, pol);
+              mbar_arrive_expect_tx(vbar, kRowBytes * kTcKeys);
+              load_tile_page1<kF8>(S.v[st][0], S.v[st][1], &tmap_v, vbar,
+                                   S.pid[J % kPidSlots][0], t % p.page_size, p, it.h, pol);
             } else if constexpr (paged) {
               const TilePages tp = tile_pages(p, t, valid);
-              mbar_arrive_expect_tx(&S.vfull[st], paged_tile_bytes(tp, p));
-              load_tile_paged(S.v[st][0], S.v[st][1], &tmap_v, &S.vfull[st], tp,
-                              S.pid[J % kPidSlots], p, it.h, valid, pol);
+              mbar_arrive_expect_tx(vbar, paged_tile_bytes<kF8>(tp, p));
+              load_tile_paged<kF8>(S.v[st][0], S.v[st][1], &tmap_v, vbar, tp,
+                                   S.pid[J % kPidSlots], p, it.h, valid, pol);
             } else {
-              mbar_arrive_expect_tx(&S.vfull[st], tx);
-              tma_load_4d_stream(S.v[st][0], &tmap_v, &S.vfull[st], 0, t, it.h, it.b, pol);
-              tma_load_4d_stream(S.v[st][1], &tmap_v, &S.vfull[st], 64, t, it.h, it.b, pol);
+              mbar_arrive_expect_tx(vbar, tx);
+              if constexpr (kF8) {
+                tma_load_4d_stream(S.v[st][1], &tmap_v, vbar, 0, t, it.h, it.b, pol);
+              } else {
+                tma_load_4d_stream(S.v[st][0], &tmap_v, vbar, 0, t, it.h, it.b, pol);
+                tma_load_4d_stream(S.v[st][1], &tmap_v, vbar, 64, t, it.h, it.b, pol);
+              }
             }
           } else {
-            mbar_arrive(&S.vfull[st]);
+            mbar_arrive(vbar);
           }
           if constexpr (paged) mbar_arrive(&S.pidempty[J % kPidSlots]);  // ids read: slot free
         }
@@ -540,7 +649,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       if (S.abort_flag) {
         for (uint32_t back = 1; back <= kTcStages && back <= J; ++back) {
           const uint32_t jj = J - back;
-          mbar_drain(&S.vfull[jj % kTcStages], (jj / kTcStages) & 1u);
+          mbar_drain(kF8 ? &S.vraw[jj % kTcStages] : &S.vfull[jj % kTcStages], (jj / kTcStages) & 1u);
         }
       }
     }
@@ -595,14 +704,24 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           tc_fence_after();
           const int valid = S.meta[st][1];
           if (valid > 0) {
-            const uint32_t k0 = smem_u32(S.k[st][0]);
-            const uint32_t k1 = smem_u32(S.k[st][1]);
+            if constexpr (kF8) {
+              // A = the expanded K tile in tensor memory: 16 d-columns are 8 columns of pairs
 #pragma unroll
-            for (int kk = 0; kk < kTcD / 16; ++kk) {
-              const uint32_t ka = (kk < 4 ? k0 : k1) + (kk & 3) * 32;
-              const uint32_t qa = (kk < 4 ? qaddr0 : qaddr1) + (kk & 3) * 32;
-              umma_bf16_ss(tmem + sb * 16, smem_desc(ka, 16, 1024, kLayoutSW128),
-                           smem_desc(qa, 16, 1024, kLayoutSW128), idesc_s, kk > 0 ? 1u : 0u);
+              for (int kk = 0; kk < kTcD / 16; ++kk) {
+                const uint32_t qa = (kk < 4 ? qaddr0 : qaddr1) + (kk & 3) * 32;
+                umma_bf16_ts(tmem + sb * 16, tmem + kColK + st * 64 + kk * 8,
+                             smem_desc(qa, 16, 1024, kLayoutSW128), idesc_s, kk > 0 ? 1u : 0u);
+              }
+            } else {
+              const uint32_t k0 = smem_u32(S.k[st][0]);
+              const uint32_t k1 = smem_u32(S.k[st][1]);
+#pragma unroll
+              for (int kk = 0; kk < kTcD / 16; ++kk) {
+                const uint32_t ka = (kk < 4 ? k0 : k1) + (kk & 3) * 32;
+                const uint32_t qa = (kk < 4 ? qaddr0 : qaddr1) + (kk & 3) * 32;
+                umma_bf16_ss(tmem + sb * 16, smem_desc(ka, 16, 1024, kLayoutSW128),
+                             smem_desc(qa, 16, 1024, kLayoutSW128), idesc_s, kk > 0 ? 1u : 0u);
+              }
             }
           }
           umma_commit(&S.sfull[sb]);
@@ -742,8 +861,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           lw[g / 2] = *reinterpret_cast<const uint32_t*>(&l2);
         }
         ok = ok && mbar_wait(&S.pempty[sb], ((J >> 1) & 1u) ^ 1u, ctx);
-        if ((valid & 15) != 0) {
-          // zero V rows [valid, next multiple of 16): they may lie past the sequence end
+        if (!kF8 && (valid & 15) != 0) {
+          // zero V rows [valid, next multiple of 16): they may lie past the sequence end (the
+          // expanding warps of an E4M3 cache write those rows as zeros themselves)
           ok = ok && mbar_wait(&S.vfull[st], (J / kTcStages) & 1u, ctx);
           const int r0 = valid, r1 = (valid + 15) & ~15;
           const int nchunks = (r1 - r0) * 2 * 8;
@@ -791,6 +911,47 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       if (lane == 0 && ok) mbar_arrive(&S.lready[ob]);
       ++K;
     }
+  } else if (warp >= kConvWarp0) {
+    if constexpr (kF8) {
+      // ======================= E4M3 -> bf16 expansion =======================
+      // Per stage, in tile order: K into the stage's tensor-memory tile (thread = key lane of its
+      // warp's lane quarter: one code row of 128 bytes -> 64 columns of bf16 pairs), then V in
+      // place in shared memory. A stage with valid < 0 is the producer's stop marker.
+      const int ct = tid - kConvWarp0 * 32;
+      const uint32_t quarter = static_cast<uint32_t>(warp & 3);
+      const int krow = static_cast<int>(quarter) * 32 + lane;
+      const uint32_t klane = (quarter * 32u) << 16;
+      for (uint32_t J = 0;; ++J) {
+        const int st = J % kTcStages;
+        const uint32_t par = (J / kTcStages) & 1u;
+        if (!mbar_wait(&S.kraw[st], par, ctx)) break;
+        const int valid = S.meta[st][1];
+        if (valid < 0) break;
+        const unsigned char* raw = reinterpret_cast<const unsigned char*>(S.k[st][1]) + krow * 128;
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+          uint32_t w[32];
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            const uint4 x = *reinterpret_cast<const uint4*>(raw + (((hh * 4 + c) ^ (krow & 7)) << 4));
+            e4m3x4_to_bf16(x.x, w[8 * c + 0], w[8 * c + 1]);
+            e4m3x4_to_bf16(x.y, w[8 * c + 2], w[8 * c + 3]);
+            e4m3x4_to_bf16(x.z, w[8 * c + 4], w[8 * c + 5]);
+            e4m3x4_to_bf16(x.w, w[8 * c + 6], w[8 * c + 7]);
+          }
+          tmem_st32(tmem + klane + kColK + st * 64 + hh * 32, w);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&S.kfull[st]);
+        if (!mbar_wait(&S.vraw[st], par, ctx)) break;
+        expand_v_tile(S.v[st], ct, valid);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&S.vfull[st]);
+      }
+    }
   } else {
     // ======================= epilogue: O = (O_hi + O_lo) / l =======================
     // Runs while the softmax warps already work on the next item; its O accumulator is the other
@@ -827,7 +988,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       for (int g = 0; g < GPAD; ++g) {
         if (g < p.g) {
           const float acc = __uint_as_float(o[g]) + __uint_as_float(o[GPAD + g]);
-          const float ov = l[g] > 0.f ? acc / l[g] : 0.f;
+          const float ov = l[g] > 0.f ? acc / l[g] * p.v_scale : 0.f;
           const float lse2 = l[g] > 0.f ? mf[g] + log2f(l[g]) : -INFINITY;
           const int hq = h * p.g + g;
           if (direct) {
@@ -847,21 +1008,21 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == kMmaWarp) tmem_dealloc(tmem, kTmemCols);
+  if (warp == kMmaWarp) tmem_dealloc(tmem, kCols);
   if (tid == 0) release_work_cursor(&p.hdr->dec_counter, &p.hdr->dec_exit);
 }
 
-template <int GPAD, int kMode>
+template <int GPAD, int kMode, bool kF8 = false>
 cudaError_t launch_tc_t(const DecodeParams& p, const CUtensorMap& tq, const CUtensorMap& tk,
                         const CUtensorMap& tv, int nctas, cudaStream_t stream) {
   const size_t smem = sizeof(TcSmem<GPAD>) + 1024;
-  cudaError_t e = cudaFuncSetAttribute(decode_tc_kernel<GPAD, kMode>,
+  cudaError_t e = cudaFuncSetAttribute(decode_tc_kernel<GPAD, kMode, kF8>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = dim3(nctas);
-  cfg.blockDim = dim3(kTcThreads);
+  cfg.blockDim = dim3(kF8 ? kF8Threads : kTcThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
@@ -869,7 +1030,7 @@ cudaError_t launch_tc_t(const DecodeParams& p, const CUtensorMap& tq, const CUte
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, decode_tc_kernel<GPAD, kMode>, p, tq, tk, tv);
+  return cudaLaunchKernelEx(&cfg, decode_tc_kernel<GPAD, kMode, kF8>, p, tq, tk, tv);
 }
 
 }  // namespace
@@ -879,6 +1040,12 @@ cudaError_t launch_decode_tc(const DecodeParams& p, const CUtensorMap& tmap_q,
                              cudaStream_t stream) {
   const int mode = p.block_table == nullptr ? kContiguous
                    : (p.page_size >= kTcKeys ? kBigPages : kSmallPages);
+  if (p.kv_fp8) {
+    if (p.g > 8) return cudaErrorInvalidValue;
+    if (mode == kContiguous) return launch_tc_t<8, kContiguous, true>(p, tmap_q, tmap_k, tmap_v, nctas, stream);
+    if (mode == kBigPages) return launch_tc_t<8, kBigPages, true>(p, tmap_q, tmap_k, tmap_v, nctas, stream);
+    return launch_tc_t<8, kSmallPages, true>(p, tmap_q, tmap_k, tmap_v, nctas, stream);
+  }
   if (p.g <= 8) {
     if (mode == kContiguous) return launch_tc_t<8, kContiguous>(p, tmap_q, tmap_k, tmap_v, nctas, stream);
     if (mode == kBigPages) return launch_tc_t<8, kBigPages>(p, tmap_q, tmap_k, tmap_v, nctas, stream);

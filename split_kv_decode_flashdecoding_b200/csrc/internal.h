@@ -65,6 +65,10 @@ struct DecodeParams {
   // it, and split boundaries are 128-key aligned, so a key tile never crosses a page.
   const int32_t* block_table;
   int32_t pages_per_seq, page_size, num_pages;
+  // E4M3 cache (kv_fp8 != 0, tensor-core kernel): k and v hold one-byte codes; the key scale is
+  // folded into scale_log2 and every output is multiplied by v_scale (1 for other caches)
+  float v_scale = 1.f;
+  int32_t kv_fp8 = 0;
 };
 
 __device__ __forceinline__ MergeTarget merge_target(const DecodeParams& p) {
@@ -119,7 +123,8 @@ cudaError_t launch_plan_chunk(const PlanParams& p, cudaStream_t stream);
 int simt_ctas_per_sm();
 cudaError_t launch_decode_simt(const DecodeParams& p, int dtype, int nctas, cudaStream_t stream);
 
-// tcgen05 split kernel: bf16, D == 128, 2 <= G <= 16.
+// tcgen05 split kernel: bf16 cache with D == 128, 2 <= G <= 16; or an E4M3 cache with D == 128,
+// 1 <= G <= 8 (p.kv_fp8).
 cudaError_t launch_decode_tc(const DecodeParams& p, const CUtensorMap& tmap_q,
                              const CUtensorMap& tmap_k, const CUtensorMap& tmap_v, int nctas,
                              cudaStream_t stream);

@@ -159,3 +159,38 @@ def test_workspace_bound_covers_plan():
             items_bound = (hkv * B * fixed if fixed else
                            hkv * B + max(P.WAVES * ctas, -(-hkv * B * cap // P.MAX_CHUNK)))
             assert ref.total_items <= items_bound
+
+
+def _decode_fp8(q, k, v, out, ks=1.0, vs=1.0, lens=0x200000, lse=0x300000, splits=0):
+    lp = ctypes.cast(ctypes.c_void_p(lens), ctypes.POINTER(ctypes.c_int32)) if lens else None
+    sp = ctypes.cast(ctypes.c_void_p(lse), ctypes.POINTER(ctypes.c_float)) if lse else None
+    return fd.lib.fd_decode_attention_fp8(ctypes.byref(q), ctypes.byref(k), ctypes.byref(v), ks, vs,
+                                          lp, splits, ctypes.byref(out), sp, None)
+
+
+def test_fp8_decode_rejects_bad_arguments_on_host():
+    B, Hq, Hkv, S, D = 2, 8, 1, 64, 128
+    q, o = _fake([B, Hq, D]), _fake([B, Hq, D])
+    k, v = _fake([B, Hkv, S, D], fd.FD_E4M3), _fake([B, Hkv, S, D], fd.FD_E4M3)
+    for ks, vs in ((0.0, 1.0), (1.0, -2.0), (float("inf"), 1.0), (1.0, float("nan"))):
+        assert _decode_fp8(q, k, v, o, ks, vs) == fd.FD_ERR_INVALID_ARGUMENT, (ks, vs)
+    # bf16 caches through the FP8 call, and E4M3 caches through the bf16 call
+    kb, vb = _fake([B, Hkv, S, D]), _fake([B, Hkv, S, D])
+    assert _decode_fp8(q, kb, vb, o) == fd.FD_ERR_INVALID_ARGUMENT
+    assert _decode(q, k, v, o) == fd.FD_ERR_INVALID_ARGUMENT
+    # E4M3 is a cache dtype only; fp32 q is not served with an FP8 cache
+    assert _decode_fp8(_fake([B, Hq, D], fd.FD_E4M3), k, v, _fake([B, Hq, D], fd.FD_E4M3)) == \
+        fd.FD_ERR_UNSUPPORTED
+    assert _decode_fp8(_fake([B, Hq, D], fd.FD_F32), k, v, _fake([B, Hq, D], fd.FD_F32)) == \
+        fd.FD_ERR_UNSUPPORTED
+    # head_dim 64 and groups above 8 are not served with an FP8 cache
+    assert _decode_fp8(_fake([B, Hq, 64]), _fake([B, Hkv, S, 64], fd.FD_E4M3),
+                       _fake([B, Hkv, S, 64], fd.FD_E4M3), _fake([B, Hq, 64])) == fd.FD_ERR_UNSUPPORTED
+    assert _decode_fp8(_fake([B, 16, D]), k, v, _fake([B, 16, D])) == fd.FD_ERR_UNSUPPORTED
+    # a row stride of the codes that is not a multiple of 16 bytes
+    kr = _fake([B, Hkv, S, D], fd.FD_E4M3, strides=[Hkv * S * D + 8, S * D, D, 1])
+    assert _decode_fp8(q, kr, kr, o) == fd.FD_ERR_UNSUPPORTED
+    # batch 0 is a no-op
+    q0, o0 = _fake([0, Hq, D]), _fake([0, Hq, D])
+    k0, v0 = _fake([0, Hkv, S, D], fd.FD_E4M3), _fake([0, Hkv, S, D], fd.FD_E4M3)
+    assert _decode_fp8(q0, k0, v0, o0) == fd.FD_OK
