@@ -17,18 +17,20 @@
 // cost: the tensor pipe is far from busy in this memory-bound loop, and N must be a multiple of
 // 16 anyway.
 //
-// Warp roles: 0-3 softmax (one thread per key lane); 4 TMA producer of Q and K; 5 MMA issuer and
-// TMEM owner; 6-9 epilogue (one thread per d lane: O / l, partial or final output); 10 TMA
-// producer of V. K/V tiles arrive by 4-D TMA with 128-byte swizzle into a 3-stage ring whose K
+// Warp roles: 0-3 softmax (one thread per key lane); 4 TMA producer of Q and K; 5 issuer of the
+// Sᵀ products and TMEM owner; 6-9 epilogue (one thread per d lane: O / l, partial or final
+// output); 10 TMA producer of V; 11 issuer of the P·V products. A product of these shapes (N of
+// 16) costs its issuing thread about as long as the tensor pipe needs for it, so the two chains
+// of 8 products per tile are issued by two threads side by side. K/V tiles arrive by 4-D TMA with 128-byte swizzle into a 3-stage ring whose K
 // and V halves are refilled independently; keys past the sequence end inside the last tile are
 // masked to p = 0 and their V rows are zeroed in shared memory before the P·V product, so stale
 // or poisoned cache rows never leak. The epilogue of an item overlaps the next item's tiles.
 //
 // E4M3 cache (FlashDecoding page, "与其他推理加速方案的组合使用", item "Quantization +
 // FlashDecoding": scores on values dequantized to bf16). The TMA brings a tile's one-byte codes
-// into a staging area and four more warps (11-14) expand them exactly to bf16: K straight into
-// tensor memory, where the Sᵀ product takes it as its A operand (so the expanded K never costs
-// shared-memory bandwidth), V in place into the bf16 layout of the stage. The key scale is folded
+// into a staging area and eight more warps expand them exactly to bf16, side by side: four K
+// straight into tensor memory, where the Sᵀ product takes it as its A operand (so the expanded K
+// never costs shared-memory bandwidth), four V in place into the bf16 layout of the stage. The key scale is folded
 // into the score scale and the value scale into the output; everything else is the bf16 kernel.
 #include "common.cuh"
 #include "internal.h"
@@ -43,9 +45,10 @@ constexpr int kTcStages = 3;
 constexpr int kProducerWarp = 4;     // Q and K
 constexpr int kMmaWarp = 5;
 constexpr int kVProducerWarp = 10;
-constexpr int kTcThreads = 11 * 32;
-constexpr int kConvWarp0 = 11;          // E4M3 cache: warps 11-14 expand the codes
-constexpr int kF8Threads = 15 * 32;
+constexpr int kPvWarp = 11;             // issues the P·V products (warp 5 the Sᵀ products)
+constexpr int kTcThreads = 12 * 32;
+constexpr int kConvWarp0 = 12;          // E4M3 cache: warps 12-15 expand K, 16-19 expand V
+constexpr int kF8Threads = 20 * 32;
 constexpr int kSoftmaxThreads = 128;
 constexpr uint32_t kTmemCols = 128;
 constexpr uint32_t kHalfBytes = kTcKeys * 64 * 2;   // one 64-column half of a K or V tile
@@ -53,12 +56,17 @@ constexpr uint32_t kHalfBytes = kTcKeys * 64 * 2;   // one 64-column half of a K
 constexpr int kMaxPageBoxes = 128 / 8;  // page boxes of one key tile (pages of >= 8 keys)
 constexpr int kPidSlots = 8;             // page-id ring of the paged producers
 
-template <int GPAD>
+// kF8 (E4M3 cache): a K stage holds only the tile's codes (128 rows of 128 bytes, the size of one
+// bf16 half), since the expanded K lives in tensor memory; a V stage holds the codes in its upper
+// half and is expanded in place.
+template <int GPAD, bool kF8 = false>
 struct __align__(1024) TcSmem {
   static constexpr int kNO = 2 * GPAD;           // Oᵀ columns: hi then lo
   static constexpr int kPGroups = kNO / 8;       // 8-column core-matrix groups of Pᵀ
-  __nv_bfloat16 k[kTcStages][2][kTcKeys * 64];   // [stage][d half][row*64 + col], SW128
-  __nv_bfloat16 v[kTcStages][2][kTcKeys * 64];
+  static constexpr int kStages = kTcStages;
+  static constexpr int kKSlabs = kF8 ? 1 : 2;
+  __nv_bfloat16 k[kStages][kKSlabs][kTcKeys * 64];  // [stage][d half][row*64 + col], SW128
+  __nv_bfloat16 v[kStages][2][kTcKeys * 64];
   __nv_bfloat16 q[2][2][16 * 64];                // [item parity][d half], SW128
   __nv_bfloat16 p[2][kPGroups * kTcKeys * 8];    // [tile parity], MN-major core matrices
   float wmax[2][4][GPAD];
@@ -66,7 +74,8 @@ struct __align__(1024) TcSmem {
   float lred[2][4][GPAD];                        // per softmax warp: sum of its key lanes' l
   float mfin[2][GPAD];                           // final running max
   int32_t epi[2][4];                             // row (-1: stop), KV head, splits, slot
-  int32_t meta[kTcStages][2];                    // per stage: tile start, valid keys (MMA warp)
+  int32_t meta[kStages][2];                      // per stage: tile start, valid keys (MMA warp)
+  int32_t vmeta[kStages];                        // E4M3: valid keys of the stage's V tile
   // in-kernel plan: lengths, split counts, rank order, partial-slot bases (row order) and item
   // offsets (rank order, B + 1 entries)
   int32_t plan_len[kFusedPlanMaxBatch], plan_n[kFusedPlanMaxBatch];
@@ -78,7 +87,7 @@ struct __align__(1024) TcSmem {
   DecodeItem item[2];                            // the item's descriptor (by item parity)
   // K and V of a stage are released separately: K once the Sᵀ product has read it, V once the
   // P·V product has, so the next K copy starts while the current tile is still in softmax.
-  uint64_t kfull[kTcStages], vfull[kTcStages], kempty[kTcStages], vempty[kTcStages];
+  uint64_t kfull[kStages], vfull[kStages], kempty[kStages], vempty[kStages];
   uint64_t qfull[2], qempty[2], sfull[2], sempty[2], pfull[2], pempty[2];
   uint64_t ofull[2];   // by tile parity: that tile's P·V product has completed
   uint64_t ofin[2];    // by item parity: the item's last P·V product has completed
@@ -86,12 +95,12 @@ struct __align__(1024) TcSmem {
   uint64_t lready[2], lfree[2];  // by item parity: hand-off written / read
   // E4M3 cache: the TMA completes these (codes in the staging area); kfull / vfull then mean
   // "expanded to bf16" and are completed by the four expanding warps
-  uint64_t kraw[kTcStages], vraw[kTcStages];
+  uint64_t kraw[kStages], vraw[kStages];
   // paged cache: physical page ids of tile J in slot J mod kPidSlots, copied asynchronously by
   // the Q/K producer two tiles ahead (pidfull) and released by the V producer (pidempty)
   int32_t pid[kPidSlots][kMaxPageBoxes];
   uint64_t pidfull[kPidSlots], pidempty[kPidSlots];
-  uint64_t drain;
+  uint64_t drain, drain_pv;
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -134,7 +143,7 @@ __device__ __forceinline__ int32_t tile_page_id(const DecodeParams& p, int b, in
 // boxes of paged_tile_bytes(), page ids from `ids` (a slot of the ring). A page that holds some
 // of the tile's `valid` keys but whose index lies outside the pool raises FD_FLAG_BAD_PAGE; its
 // copy still runs and reads zeros (a TMA coordinate outside the tensor).
-// An E4M3 cache (kF8) has one 128-byte box per row, into the upper half (the staging area).
+// An E4M3 cache (kF8) has one 128-byte box per row, into dst0 (the codes' staging area).
 template <bool kF8>
 __device__ __forceinline__ void load_tile_paged(__nv_bfloat16* dst0, __nv_bfloat16* dst1,
                                                 const CUtensorMap* map, uint64_t* bar,
@@ -149,7 +158,7 @@ __device__ __forceinline__ void load_tile_paged(__nv_bfloat16* dst0, __nv_bfloat
       const int32_t id = tp.first + i < p.pages_per_seq ? ids[i] : -1;
       bad |= (i * rows < valid) && (id < 0 || id >= p.num_pages);
       if constexpr (kF8) {
-        tma_load_4d_stream(reinterpret_cast<unsigned char*>(dst1) + i * rows * 128, map, bar, 0,
+        tma_load_4d_stream(reinterpret_cast<unsigned char*>(dst0) + i * rows * 128, map, bar, 0,
                            tp.row0, h, id, pol);
       } else {
         tma_load_4d_stream(dst0 + i * rows * 64, map, bar, 0, tp.row0, h, id, pol);
@@ -168,7 +177,7 @@ __device__ __forceinline__ void load_tile_page1(__nv_bfloat16* dst0, __nv_bfloat
                                                 uint64_t pol) {
   if (id < 0 || id >= p.num_pages) atomicOr(&p.hdr->status, FD_FLAG_BAD_PAGE);
   if constexpr (kF8) {
-    tma_load_4d_stream(dst1, map, bar, 0, row0, h, id, pol);
+    tma_load_4d_stream(dst0, map, bar, 0, row0, h, id, pol);
   } else {
     tma_load_4d_stream(dst0, map, bar, 0, row0, h, id, pol);
     tma_load_4d_stream(dst1, map, bar, 64, row0, h, id, pol);
@@ -207,39 +216,47 @@ __device__ __forceinline__ void e4m3x4_to_bf16(uint32_t w, uint32_t& lo, uint32_
 
 // In-place expansion of one V tile of an E4M3 cache by 128 threads (ct = 0..127). The TMA put
 // the 128 rows of 128 codes (128-byte swizzle) into the upper 64-column half of the stage; the
-// bf16 rows go to both halves in the layout of a bf16 tile, rows >= valid as zeros. The upper
-// half of bf16 row r takes exactly the bytes of code row r, and the eight lanes that expand a
-// row load all of its codes in one instruction before the warp stores anything, so no code is
+// bf16 rows go to both halves in the layout of a bf16 tile, rows >= valid as zeros. Thread ct
+// expands the 16-byte chunk c = ct % 8 of rows 16 i + ct / 8 (i = 0..7); the upper half of bf16
+// row r takes exactly the bytes of code row r, every row is expanded by the warp that loads it,
+// and a warp loads the codes of a group of rows before it stores any of them, so no code is
 // overwritten before it is read.
 __device__ __forceinline__ void expand_v_tile(__nv_bfloat16 (&buf)[2][kTcKeys * 64], int ct,
                                               int valid) {
   unsigned char* h0 = reinterpret_cast<unsigned char*>(buf[0]);
   unsigned char* h1 = reinterpret_cast<unsigned char*>(buf[1]);
-#pragma unroll 2
-  for (int i = 0; i < kTcKeys * 8 / 128; ++i) {
-    const int id = i * 128 + ct;
-    const int r = id >> 3, c = id & 7, x = r & 7;
-    const uint4 w = *reinterpret_cast<const uint4*>(h1 + r * 128 + ((c ^ x) << 4));
+  const int c = ct & 7, r0 = ct >> 3, x = r0 & 7;  // (16 i + r0) & 7 == x for every i
+  unsigned char* half = c >= 4 ? h1 : h0;
+  const int sa = ((2 * (c & 3)) ^ x) << 4;  // swizzled slot of elements 16c .. 16c+7
+  const int sb = sa ^ 16;                   // and of 16c+8 .. 16c+15
+  // two groups of four rows per thread; a group's stores touch only rows the warp loaded in it
+#pragma unroll 1
+  for (int g = 0; g < 2; ++g) {
+    uint4 w[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      w[i] = *reinterpret_cast<const uint4*>(h1 + (16 * (4 * g + i) + r0) * 128 + ((c ^ x) << 4));
     __syncwarp();
-    uint4 a, b;  // bf16 of elements 16c .. 16c+7 and 16c+8 .. 16c+15
-    e4m3x4_to_bf16(w.x, a.x, a.y);
-    e4m3x4_to_bf16(w.y, a.z, a.w);
-    e4m3x4_to_bf16(w.z, b.x, b.y);
-    e4m3x4_to_bf16(w.w, b.z, b.w);
-    if (r >= valid) a = b = make_uint4(0u, 0u, 0u, 0u);
-    const bool upper = c >= 4;
-    const int ca = (2 * (c & 3)) ^ x;  // swizzled 16-byte slot of elements 16c .. 16c+7
-    unsigned char* row = (upper ? h1 : h0) + r * 128;
-    // lanes of the lower half store their even slot first, those of the upper half their odd
-    // one, so each store instruction covers 8 distinct bank groups of a row
-    *reinterpret_cast<uint4*>(row + ((upper ? ca ^ 1 : ca) << 4)) = upper ? b : a;
-    *reinterpret_cast<uint4*>(row + ((upper ? ca : ca ^ 1) << 4)) = upper ? a : b;
+    const bool full = valid >= kTcKeys;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int r = 16 * (4 * g + i) + r0;
+      uint4 a, b;
+      e4m3x4_to_bf16(w[i].x, a.x, a.y);
+      e4m3x4_to_bf16(w[i].y, a.z, a.w);
+      e4m3x4_to_bf16(w[i].z, b.x, b.y);
+      e4m3x4_to_bf16(w[i].w, b.z, b.w);
+      if (!full && r >= valid) a = b = make_uint4(0u, 0u, 0u, 0u);
+      *reinterpret_cast<uint4*>(half + r * 128 + sa) = a;
+      *reinterpret_cast<uint4*>(half + r * 128 + sb) = b;
+    }
   }
 }
 
 // dynamic shared memory per CTA, plus the 1024 bytes of alignment slack the kernel may use
 static_assert(sizeof(TcSmem<8>) + 1024 <= 227 * 1024, "tensor-core decode smem (G <= 8)");
 static_assert(sizeof(TcSmem<16>) + 1024 <= 227 * 1024, "tensor-core decode smem (G <= 16)");
+static_assert(sizeof(TcSmem<8, true>) + 1024 <= 227 * 1024, "tensor-core decode smem (E4M3)");
 
 // Exclusive prefix sum over i < n (n <= 32 * 8 here) by one warp: out[i] = sum_{j<i} val(j),
 // out[n] = the total.
@@ -279,14 +296,15 @@ __global__ void __launch_bounds__(kF8 ? kF8Threads : kTcThreads, 1)
     decode_tc_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmap_q,
                      const __grid_constant__ CUtensorMap tmap_k,
                      const __grid_constant__ CUtensorMap tmap_v) {
-  using Smem = TcSmem<GPAD>;
+  using Smem = TcSmem<GPAD, kF8>;
   constexpr int kNO = Smem::kNO;
+  constexpr int kStages = Smem::kStages;
   constexpr int kThreads = kF8 ? kF8Threads : kTcThreads;
   constexpr uint32_t kColO = 32;  // Sᵀ buffers at columns [0, 32), O accumulators after them
   // E4M3 cache: the expanded K tile of each stage (128 key lanes x 64 columns of bf16 pairs)
   constexpr uint32_t kColK = kColO + 2 * kNO;
-  constexpr uint32_t kCols = kF8 ? 256 : kTmemCols;
-  static_assert(!kF8 || kColK + kTcStages * 64 <= kCols, "tensor memory of the E4M3 kernel");
+  constexpr uint32_t kCols = kF8 ? 512 : kTmemCols;
+  static_assert(!kF8 || kColK + kStages * 64 <= kCols, "tensor memory of the E4M3 kernel");
   static_assert(!kF8 || GPAD == 8, "the E4M3 kernel serves groups of <= 8 heads");
   constexpr uint32_t kRowBytes = kF8 ? 128u : 256u;  // bytes of one cached K or V row
   extern __shared__ __align__(1024) unsigned char smem_raw[];
@@ -297,7 +315,7 @@ __global__ void __launch_bounds__(kF8 ? kF8Threads : kTcThreads, 1)
   const int lane = tid & 31;
 
   if (tid == 0) {
-    for (int s = 0; s < kTcStages; ++s) {
+    for (int s = 0; s < kStages; ++s) {
       mbar_init(&S.kfull[s], kF8 ? 4 : 1);
       mbar_init(&S.vfull[s], kF8 ? 4 : 1);
       mbar_init(&S.kempty[s], 1);
@@ -307,7 +325,7 @@ __global__ void __launch_bounds__(kF8 ? kF8Threads : kTcThreads, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&S.qfull[i], 1);
-      mbar_init(&S.qempty[i], 1 + 4 + 1);  // MMA, softmax warps, V producer
+      mbar_init(&S.qempty[i], 1 + 4 + 1 + 1);  // Sᵀ issuer, softmax warps, V producer, P·V issuer
       mbar_init(&S.sfull[i], 1);
       mbar_init(&S.sempty[i], 4);
       mbar_init(&S.pfull[i], 4);
@@ -323,6 +341,7 @@ __global__ void __launch_bounds__(kF8 ? kF8Threads : kTcThreads, 1)
       mbar_init(&S.pidempty[i], 1);
     }
     mbar_init(&S.drain, 1);
+    mbar_init(&S.drain_pv, 1);
     S.abort_flag = 0;
     fence_mbar_init();
   }
@@ -477,8 +496,8 @@ __global__ void __launch_bounds__(kF8 ? kF8Threads : kTcThreads, 1)
               have_next = true;
             }
           }
-          const int st = J % kTcStages;
-          const uint32_t free_parity = ((J / kTcStages) & 1u) ^ 1u;
+          const int st = J % kStages;
+          const uint32_t free_parity = ((J / kStages) & 1u) ^ 1u;
           const int t = it.t0 + j * kTcKeys;
           const int valid = max(0, min(kTcKeys, it.t1 - t));
           TilePages tp{};
@@ -540,21 +559,18 @@ __global__ void __launch_bounds__(kF8 ? kF8Threads : kTcThreads, 1)
             if constexpr (paged) {
               if constexpr (big_pages) {
                 mbar_arrive_expect_tx(kbar, kRowBytes * kTcKeys);
-                load_tile_page1<kF8>(S.k[st][0], S.k[st][1], &tmap_k, kbar, id_big,
+                load_tile_page1<kF8>(S.k[st][0], S.k[st][Smem::kKSlabs - 1], &tmap_k, kbar, id_big,
                                      t % p.page_size, p, it.h, pol);
               } else {
                 mbar_arrive_expect_tx(kbar, paged_tile_bytes<kF8>(tp, p));
-                load_tile_paged<kF8>(S.k[st][0], S.k[st][1], &tmap_k, kbar, tp,
+                load_tile_paged<kF8>(S.k[st][0], S.k[st][Smem::kKSlabs - 1], &tmap_k, kbar, tp,
                                      S.pid[J % kPidSlots], p, it.h, valid, pol);
               }
             } else {
               mbar_arrive_expect_tx(kbar, kRowBytes * static_cast<uint32_t>(p.kv_box_rows));
-              if constexpr (kF8) {
-                tma_load_4d_stream(S.k[st][1], &tmap_k, kbar, 0, t, it.h, it.b, pol);
-              } else {
-                tma_load_4d_stream(S.k[st][0], &tmap_k, kbar, 0, t, it.h, it.b, pol);
-                tma_load_4d_stream(S.k[st][1], &tmap_k, kbar, 64, t, it.h, it.b, pol);
-              }
+              tma_load_4d_stream(S.k[st][0], &tmap_k, kbar, 0, t, it.h, it.b, pol);
+              if constexpr (!kF8)
+                tma_load_4d_stream(S.k[st][Smem::kKSlabs - 1], &tmap_k, kbar, 64, t, it.h, it.b, pol);
             }
           } else {
             mbar_arrive(kbar);
@@ -577,8 +593,8 @@ __global__ void __launch_bounds__(kF8 ? kF8Threads : kTcThreads, 1)
         if constexpr (kF8) {
           // the expanding warps follow the stages, not the items: a stage without a tile (valid
           // -1) stops them, once the stage's previous tile has been consumed
-          const int st = J % kTcStages;
-          if (mbar_wait(&S.kempty[st], ((J / kTcStages) & 1u) ^ 1u, ctx)) {
+          const int st = J % kStages;
+          if (mbar_wait(&S.kempty[st], ((J / kStages) & 1u) ^ 1u, ctx)) {
             S.meta[st][1] = -1;
             mbar_arrive(&S.kraw[st]);
           }
@@ -587,9 +603,9 @@ __global__ void __launch_bounds__(kF8 ? kF8Threads : kTcThreads, 1)
       if constexpr (paged) asm volatile("cp.async.wait_all;" ::: "memory");
       if (S.abort_flag) {
         // let copies already issued land before shared memory is released
-        for (uint32_t back = 1; back <= kTcStages && back <= J; ++back) {
+        for (uint32_t back = 1; back <= kStages && back <= J; ++back) {
           const uint32_t jj = J - back;
-          mbar_drain(kF8 ? &S.kraw[jj % kTcStages] : &S.kfull[jj % kTcStages], (jj / kTcStages) & 1u);
+          mbar_drain(kF8 ? &S.kraw[jj % kStages] : &S.kfull[jj % kStages], (jj / kStages) & 1u);
         }
       }
     }
@@ -612,23 +628,24 @@ __global__ void __launch_bounds__(kF8 ? kF8Threads : kTcThreads, 1)
         mbar_arrive(&S.qempty[ps]);
         if (idx < 0) break;
         for (int j = 0; j < ntile; ++j, ++J) {
-          const int st = J % kTcStages;
+          const int st = J % kStages;
           const int t = it.t0 + j * kTcKeys;
           const int valid = max(0, min(kTcKeys, it.t1 - t));
-          if (!mbar_wait(&S.vempty[st], ((J / kTcStages) & 1u) ^ 1u, ctx)) { ok = false; break; }
+          if (!mbar_wait(&S.vempty[st], ((J / kStages) & 1u) ^ 1u, ctx)) { ok = false; break; }
           if constexpr (paged) {
             if (!mbar_wait(&S.pidfull[J % kPidSlots], (J / kPidSlots) & 1u, ctx)) { ok = false; break; }
           }
           uint64_t* vbar = kF8 ? &S.vraw[st] : &S.vfull[st];
+          if constexpr (kF8) S.vmeta[st] = valid;
           if (valid > 0) {
             if constexpr (big_pages) {
               mbar_arrive_expect_tx(vbar, kRowBytes * kTcKeys);
-              load_tile_page1<kF8>(S.v[st][0], S.v[st][1], &tmap_v, vbar,
+              load_tile_page1<kF8>(S.v[st][kF8 ? 1 : 0], S.v[st][1], &tmap_v, vbar,
                                    S.pid[J % kPidSlots][0], t % p.page_size, p, it.h, pol);
             } else if constexpr (paged) {
               const TilePages tp = tile_pages(p, t, valid);
               mbar_arrive_expect_tx(vbar, paged_tile_bytes<kF8>(tp, p));
-              load_tile_paged<kF8>(S.v[st][0], S.v[st][1], &tmap_v, vbar, tp,
+              load_tile_paged<kF8>(S.v[st][kF8 ? 1 : 0], S.v[st][1], &tmap_v, vbar, tp,
                                    S.pid[J % kPidSlots], p, it.h, valid, pol);
             } else {
               mbar_arrive_expect_tx(vbar, tx);
@@ -646,48 +663,28 @@ __global__ void __launch_bounds__(kF8 ? kF8Threads : kTcThreads, 1)
         }
         ++K;
       }
+      if constexpr (kF8) {
+        // stop marker for the V expanding warps (a stage without a tile)
+        const int st = J % kStages;
+        if (ok && mbar_wait(&S.vempty[st], ((J / kStages) & 1u) ^ 1u, ctx)) {
+          S.vmeta[st] = -1;
+          mbar_arrive(&S.vraw[st]);
+        }
+      }
       if (S.abort_flag) {
-        for (uint32_t back = 1; back <= kTcStages && back <= J; ++back) {
+        for (uint32_t back = 1; back <= kStages && back <= J; ++back) {
           const uint32_t jj = J - back;
-          mbar_drain(kF8 ? &S.vraw[jj % kTcStages] : &S.vfull[jj % kTcStages], (jj / kTcStages) & 1u);
+          mbar_drain(kF8 ? &S.vraw[jj % kStages] : &S.vfull[jj % kStages], (jj / kStages) & 1u);
         }
       }
     }
     __syncwarp();
   } else if (warp == kMmaWarp) {
-    // ======================= MMA issuer =======================
+    // ======================= Sᵀ issuer =======================
     if (lane == 0) {
       const uint32_t idesc_s = idesc_bf16_f32(kTcKeys, 16, false, false);
-      const uint32_t idesc_o = idesc_bf16_f32(kTcD, kNO, true, true);
       uint32_t J = 0, K = 0;
       bool ok = true;
-      // the P·V product of a tile is issued after the Sᵀ product of the next one, so the tensor
-      // pipe computes Sᵀ(J + 1) while the softmax warps work on tile J
-      struct Pending { int st, valid; uint32_t jt, item; bool first, last; };
-      Pending prev{};
-      bool have_prev = false;
-      auto issue_pv = [&](const Pending& pv) -> bool {
-        const int pb = pv.jt & 1;
-        const int ob = pv.item & 1;
-        if (!mbar_wait(&S.vfull[pv.st], (pv.jt / kTcStages) & 1u, ctx)) return false;
-        if (!mbar_wait(&S.pfull[pb], (pv.jt >> 1) & 1u, ctx)) return false;
-        // the first product of an item overwrites the accumulator the item two back used
-        if (pv.first && !mbar_wait(&S.oempty[ob], ((pv.item >> 1) & 1u) ^ 1u, ctx)) return false;
-        tc_fence_after();
-        const int nk = (pv.valid + 15) / 16;
-        const uint32_t vaddr = smem_u32(S.v[pv.st][0]);
-        const uint32_t paddr = smem_u32(S.p[pb]);
-        for (int kk = 0; kk < nk; ++kk) {
-          const uint64_t ad = smem_desc(vaddr + kk * 2048, kHalfBytes, 1024, kLayoutSW128);
-          const uint64_t bd = smem_desc(paddr + kk * 256, 128, 2048, kLayoutNone);
-          umma_bf16_ss(tmem + kColO + ob * kNO, ad, bd, idesc_o, (pv.first && kk == 0) ? 0u : 1u);
-        }
-        umma_commit(&S.ofull[pb]);
-        if (pv.last) umma_commit(&S.ofin[ob]);
-        umma_commit(&S.pempty[pb]);
-        umma_commit(&S.vempty[pv.st]);
-        return true;
-      };
       while (ok) {
         const int ps = K & 1;
         if (!mbar_wait(&S.qfull[ps], (K >> 1) & 1u, ctx)) { ok = false; break; }
@@ -697,9 +694,9 @@ __global__ void __launch_bounds__(kF8 ? kF8Threads : kTcThreads, 1)
         const uint32_t qaddr0 = smem_u32(S.q[ps][0]);
         const uint32_t qaddr1 = smem_u32(S.q[ps][1]);
         for (int j = 0; j < ntile; ++j, ++J) {
-          const int st = J % kTcStages;
+          const int st = J % kStages;
           const int sb = J & 1;
-          if (!mbar_wait(&S.kfull[st], (J / kTcStages) & 1u, ctx)) { ok = false; break; }
+          if (!mbar_wait(&S.kfull[st], (J / kStages) & 1u, ctx)) { ok = false; break; }
           if (!mbar_wait(&S.sempty[sb], ((J >> 1) & 1u) ^ 1u, ctx)) { ok = false; break; }
           tc_fence_after();
           const int valid = S.meta[st][1];
@@ -714,7 +711,7 @@ __global__ void __launch_bounds__(kF8 ? kF8Threads : kTcThreads, 1)
               }
             } else {
               const uint32_t k0 = smem_u32(S.k[st][0]);
-              const uint32_t k1 = smem_u32(S.k[st][1]);
+              const uint32_t k1 = smem_u32(S.k[st][Smem::kKSlabs - 1]);
 #pragma unroll
               for (int kk = 0; kk < kTcD / 16; ++kk) {
                 const uint32_t ka = (kk < 4 ? k0 : k1) + (kk & 3) * 32;
@@ -727,17 +724,59 @@ __global__ void __launch_bounds__(kF8 ? kF8Threads : kTcThreads, 1)
           umma_commit(&S.sfull[sb]);
           umma_commit(&S.kempty[st]);
           if (j == ntile - 1) umma_commit(&S.qempty[ps]);
-          if (have_prev && !issue_pv(prev)) { ok = false; break; }
-          have_prev = true;
-          prev = Pending{st, valid, J, K, j == 0, j == ntile - 1};
         }
         if (!ok) break;
         ++K;
       }
-      if (ok && have_prev) ok = issue_pv(prev);
       // every MMA this thread issued has completed once `drain` flips
       umma_commit(&S.drain);
       mbar_drain(&S.drain, 0);
+    }
+    __syncwarp();
+  } else if (warp == kPvWarp) {
+    // ======================= P·V issuer =======================
+    // Follows the items the Q/K producer publishes. O of an item accumulates in the item
+    // parity's columns; its first product overwrites them once the epilogue has read the item
+    // two back.
+    if (lane == 0) {
+      const uint32_t idesc_o = idesc_bf16_f32(kTcD, kNO, true, true);
+      uint32_t J = 0, K = 0;
+      bool ok = true;
+      while (ok) {
+        const int ps = K & 1;
+        if (!mbar_wait(&S.qfull[ps], (K >> 1) & 1u, ctx)) { ok = false; break; }
+        const int idx = S.item_slot[ps][0];
+        const int ntile = S.item_slot[ps][1];
+        const DecodeItem it = S.item[ps];
+        mbar_arrive(&S.qempty[ps]);
+        if (idx < 0) break;
+        const int ob = K & 1;
+        for (int j = 0; j < ntile; ++j, ++J) {
+          const int st = J % kStages;
+          const int pb = J & 1;
+          const int valid = max(0, min(kTcKeys, it.t1 - (it.t0 + j * kTcKeys)));
+          if (!mbar_wait(&S.vfull[st], (J / kStages) & 1u, ctx)) { ok = false; break; }
+          if (!mbar_wait(&S.pfull[pb], (J >> 1) & 1u, ctx)) { ok = false; break; }
+          if (j == 0 && !mbar_wait(&S.oempty[ob], ((K >> 1) & 1u) ^ 1u, ctx)) { ok = false; break; }
+          tc_fence_after();
+          const int nk = (valid + 15) / 16;
+          const uint32_t vaddr = smem_u32(S.v[st][0]);
+          const uint32_t paddr = smem_u32(S.p[pb]);
+          for (int kk = 0; kk < nk; ++kk) {
+            const uint64_t ad = smem_desc(vaddr + kk * 2048, kHalfBytes, 1024, kLayoutSW128);
+            const uint64_t bd = smem_desc(paddr + kk * 256, 128, 2048, kLayoutNone);
+            umma_bf16_ss(tmem + kColO + ob * kNO, ad, bd, idesc_o, (j == 0 && kk == 0) ? 0u : 1u);
+          }
+          umma_commit(&S.ofull[pb]);
+          if (j == ntile - 1) umma_commit(&S.ofin[ob]);
+          umma_commit(&S.pempty[pb]);
+          umma_commit(&S.vempty[st]);
+        }
+        if (!ok) break;
+        ++K;
+      }
+      umma_commit(&S.drain_pv);
+      mbar_drain(&S.drain_pv, 0);
     }
     __syncwarp();
   } else if (warp < 4) {
@@ -780,7 +819,7 @@ __global__ void __launch_bounds__(kF8 ? kF8Threads : kTcThreads, 1)
       for (int g = 0; g < GPAD; ++g) { m[g] = -INFINITY; lp[g] = 0.f; }
       bool abort_item = false;
       for (int j = 0; j < ntile; ++j, ++J) {
-        const int st = J % kTcStages;
+        const int st = J % kStages;
         const int sb = J & 1;
         ok = ok && mbar_wait(&S.sfull[sb], (J >> 1) & 1u, ctx);
         tc_fence_after();
@@ -864,7 +903,7 @@ __global__ void __launch_bounds__(kF8 ? kF8Threads : kTcThreads, 1)
         if (!kF8 && (valid & 15) != 0) {
           // zero V rows [valid, next multiple of 16): they may lie past the sequence end (the
           // expanding warps of an E4M3 cache write those rows as zeros themselves)
-          ok = ok && mbar_wait(&S.vfull[st], (J / kTcStages) & 1u, ctx);
+          ok = ok && mbar_wait(&S.vfull[st], (J / kStages) & 1u, ctx);
           const int r0 = valid, r1 = (valid + 15) & ~15;
           const int nchunks = (r1 - r0) * 2 * 8;
           for (int c = tid; ok && c < nchunks; c += kSoftmaxThreads) {
@@ -914,42 +953,49 @@ __global__ void __launch_bounds__(kF8 ? kF8Threads : kTcThreads, 1)
   } else if (warp >= kConvWarp0) {
     if constexpr (kF8) {
       // ======================= E4M3 -> bf16 expansion =======================
-      // Per stage, in tile order: K into the stage's tensor-memory tile (thread = key lane of its
-      // warp's lane quarter: one code row of 128 bytes -> 64 columns of bf16 pairs), then V in
-      // place in shared memory. A stage with valid < 0 is the producer's stop marker.
-      const int ct = tid - kConvWarp0 * 32;
-      const uint32_t quarter = static_cast<uint32_t>(warp & 3);
-      const int krow = static_cast<int>(quarter) * 32 + lane;
-      const uint32_t klane = (quarter * 32u) << 16;
-      for (uint32_t J = 0;; ++J) {
-        const int st = J % kTcStages;
-        const uint32_t par = (J / kTcStages) & 1u;
-        if (!mbar_wait(&S.kraw[st], par, ctx)) break;
-        const int valid = S.meta[st][1];
-        if (valid < 0) break;
-        const unsigned char* raw = reinterpret_cast<const unsigned char*>(S.k[st][1]) + krow * 128;
+      // Warps 11-14: per stage, in tile order, K into the stage's tensor-memory tile (thread = key
+      // lane of its warp's lane quarter: one code row of 128 bytes -> 64 columns of bf16 pairs).
+      // Warps 15-18: V in place in shared memory. A stage whose valid count is < 0 is the
+      // producer's stop marker.
+      if (warp < kConvWarp0 + 4) {
+        const uint32_t quarter = static_cast<uint32_t>(warp & 3);
+        const int krow = static_cast<int>(quarter) * 32 + lane;
+        const uint32_t klane = (quarter * 32u) << 16;
+        for (uint32_t J = 0;; ++J) {
+          const int st = J % kStages;
+          if (!mbar_wait(&S.kraw[st], (J / kStages) & 1u, ctx)) break;
+          if (S.meta[st][1] < 0) break;
+          const unsigned char* raw = reinterpret_cast<const unsigned char*>(S.k[st][0]) + krow * 128;
+#pragma unroll 1
+          for (int hh = 0; hh < 2; ++hh) {
+            uint32_t w[32];
 #pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-          uint32_t w[32];
-#pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            const uint4 x = *reinterpret_cast<const uint4*>(raw + (((hh * 4 + c) ^ (krow & 7)) << 4));
-            e4m3x4_to_bf16(x.x, w[8 * c + 0], w[8 * c + 1]);
-            e4m3x4_to_bf16(x.y, w[8 * c + 2], w[8 * c + 3]);
-            e4m3x4_to_bf16(x.z, w[8 * c + 4], w[8 * c + 5]);
-            e4m3x4_to_bf16(x.w, w[8 * c + 6], w[8 * c + 7]);
+            for (int c = 0; c < 4; ++c) {
+              const uint4 x = *reinterpret_cast<const uint4*>(raw + (((hh * 4 + c) ^ (krow & 7)) << 4));
+              e4m3x4_to_bf16(x.x, w[8 * c + 0], w[8 * c + 1]);
+              e4m3x4_to_bf16(x.y, w[8 * c + 2], w[8 * c + 3]);
+              e4m3x4_to_bf16(x.z, w[8 * c + 4], w[8 * c + 5]);
+              e4m3x4_to_bf16(x.w, w[8 * c + 6], w[8 * c + 7]);
+            }
+            tmem_st32(tmem + klane + kColK + st * 64 + hh * 32, w);
           }
-          tmem_st32(tmem + klane + kColK + st * 64 + hh * 32, w);
+          tmem_wait_st();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&S.kfull[st]);
         }
-        tmem_wait_st();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&S.kfull[st]);
-        if (!mbar_wait(&S.vraw[st], par, ctx)) break;
-        expand_v_tile(S.v[st], ct, valid);
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&S.vfull[st]);
+      } else {
+        const int ct = tid - (kConvWarp0 + 4) * 32;
+        for (uint32_t J = 0;; ++J) {
+          const int st = J % kStages;
+          if (!mbar_wait(&S.vraw[st], (J / kStages) & 1u, ctx)) break;
+          const int valid = S.vmeta[st];
+          if (valid < 0) break;
+          expand_v_tile(S.v[st], ct, valid);
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&S.vfull[st]);
+        }
       }
     }
   } else {
@@ -1015,7 +1061,7 @@ __global__ void __launch_bounds__(kF8 ? kF8Threads : kTcThreads, 1)
 template <int GPAD, int kMode, bool kF8 = false>
 cudaError_t launch_tc_t(const DecodeParams& p, const CUtensorMap& tq, const CUtensorMap& tk,
                         const CUtensorMap& tv, int nctas, cudaStream_t stream) {
-  const size_t smem = sizeof(TcSmem<GPAD>) + 1024;
+  const size_t smem = sizeof(TcSmem<GPAD, kF8>) + 1024;
   cudaError_t e = cudaFuncSetAttribute(decode_tc_kernel<GPAD, kMode, kF8>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
