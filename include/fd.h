@@ -156,10 +156,11 @@ fd_status fd_decode_attention_paged(const fd_tensor* q, const fd_tensor* k_pages
  * FP8 cache whose values are dequantized to bf16 for the score computation. Format and scale
  * granularity are not given there; they are read as: E4M3 codes, one scale for all of K and one
  * for all of V, the cached value of code c being e4m3(c) * scale. Every E4M3 value is exact in
- * bf16, so the kernel expands the codes to bf16 without rounding, folds k_scale into the score
- * scale and applies v_scale to the output: the result is the attention of fd_decode_attention
- * over the exact values e4m3(c) * scale, up to fp32 rounding. The NaN codes (0x7F, 0xFF) are
- * not given a special meaning by the kernel (a quantized cache holds none).
+ * bf16 and in f16, so the kernel expands the codes without rounding (K to bf16, V to f16), folds
+ * k_scale into the score scale and applies v_scale to the output: the result is the attention of
+ * fd_decode_attention over the exact values e4m3(c) * scale, up to fp32 rounding. The NaN codes
+ * (0x7F, 0xFF) must not occur among a sequence's valid keys (a quantized cache holds none); the
+ * result is unspecified where they do.
  *
  *  q          [B, Hq, D]          FD_BF16; D == 128; group size Hq / Hkv <= 8.
  *  k_cache    [B, Hkv, S_cap, D]  FD_E4M3 (one byte per element); layout and alignment rules

@@ -28,10 +28,12 @@
 //
 // E4M3 cache (FlashDecoding page, "与其他推理加速方案的组合使用", item "Quantization +
 // FlashDecoding": scores on values dequantized to bf16). The TMA brings a tile's one-byte codes
-// into a staging area and eight more warps expand them exactly to bf16, side by side: four K
+// into a staging area and eight more warps expand them exactly, side by side: four K to bf16
 // straight into tensor memory, where the Sᵀ product takes it as its A operand (so the expanded K
-// never costs shared-memory bandwidth), four V in place into the bf16 layout of the stage. The key scale is folded
-// into the score scale and the value scale into the output; everything else is the bf16 kernel.
+// never costs shared-memory bandwidth), four V in place to f16 (one hardware conversion per pair
+// of codes; every E4M3 value is exact in f16 as in bf16). The P·V product of this instantiation
+// runs on f16 operands, P split into f16 hi + lo. The key scale is folded into the score scale
+// and the value scale into the output; everything else is the bf16 kernel.
 #include "common.cuh"
 #include "internal.h"
 
@@ -214,9 +216,20 @@ __device__ __forceinline__ void e4m3x4_to_bf16(uint32_t w, uint32_t& lo, uint32_
   memcpy(&hi, &b, 4);
 }
 
+// Four E4M3 codes (the bytes of w, the first in the low byte) as two f16 pairs, exactly, by the
+// hardware conversion of a pair of codes.
+__device__ __forceinline__ void e4m3x4_to_f16(uint32_t w, uint32_t& lo, uint32_t& hi) {
+  asm("{\n\t.reg .b16 a, b;\n\t"
+      "mov.b32 {a, b}, %2;\n\t"
+      "cvt.rn.f16x2.e4m3x2 %0, a;\n\t"
+      "cvt.rn.f16x2.e4m3x2 %1, b;\n\t}"
+      : "=r"(lo), "=r"(hi)
+      : "r"(w));
+}
+
 // In-place expansion of one V tile of an E4M3 cache by 128 threads (ct = 0..127). The TMA put
 // the 128 rows of 128 codes (128-byte swizzle) into the upper 64-column half of the stage; the
-// bf16 rows go to both halves in the layout of a bf16 tile, rows >= valid as zeros. Thread ct
+// f16 rows go to both halves in the layout of a 16-bit tile, rows >= valid as zeros. Thread ct
 // expands the 16-byte chunk c = ct % 8 of rows 16 i + ct / 8 (i = 0..7); the upper half of bf16
 // row r takes exactly the bytes of code row r, every row is expanded by the warp that loads it,
 // and a warp loads the codes of a group of rows before it stores any of them, so no code is
@@ -242,10 +255,10 @@ __device__ __forceinline__ void expand_v_tile(__nv_bfloat16 (&buf)[2][kTcKeys * 
     for (int i = 0; i < 4; ++i) {
       const int r = 16 * (4 * g + i) + r0;
       uint4 a, b;
-      e4m3x4_to_bf16(w[i].x, a.x, a.y);
-      e4m3x4_to_bf16(w[i].y, a.z, a.w);
-      e4m3x4_to_bf16(w[i].z, b.x, b.y);
-      e4m3x4_to_bf16(w[i].w, b.z, b.w);
+      e4m3x4_to_f16(w[i].x, a.x, a.y);
+      e4m3x4_to_f16(w[i].y, a.z, a.w);
+      e4m3x4_to_f16(w[i].z, b.x, b.y);
+      e4m3x4_to_f16(w[i].w, b.z, b.w);
       if (!full && r >= valid) a = b = make_uint4(0u, 0u, 0u, 0u);
       *reinterpret_cast<uint4*>(half + r * 128 + sa) = a;
       *reinterpret_cast<uint4*>(half + r * 128 + sb) = b;
@@ -739,7 +752,8 @@ __global__ void __launch_bounds__(kF8 ? kF8Threads : kTcThreads, 1)
     // parity's columns; its first product overwrites them once the epilogue has read the item
     // two back.
     if (lane == 0) {
-      const uint32_t idesc_o = idesc_bf16_f32(kTcD, kNO, true, true);
+      const uint32_t idesc_o = kF8 ? idesc_f16_f32(kTcD, kNO, true, true)
+                                   : idesc_bf16_f32(kTcD, kNO, true, true);
       uint32_t J = 0, K = 0;
       bool ok = true;
       while (ok) {
@@ -889,15 +903,23 @@ __global__ void __launch_bounds__(kF8 ? kF8Threads : kTcThreads, 1)
           pr[g] = (m[g] == -INFINITY) ? 0.f : fast_exp2(x[g] - m[g]);
           lp[g] += pr[g];
         }
-        // P_hi / P_lo for this key lane
+        // P_hi / P_lo for this key lane (f16 in the E4M3 instantiation, whose V is f16)
         uint32_t hw[GPAD / 2], lw[GPAD / 2];
 #pragma unroll
         for (int g = 0; g < GPAD; g += 2) {
-          const __nv_bfloat162 h2 = __floats2bfloat162_rn(pr[g], pr[g + 1]);
-          const float2 hf = __bfloat1622float2(h2);
-          const __nv_bfloat162 l2 = __floats2bfloat162_rn(pr[g] - hf.x, pr[g + 1] - hf.y);
-          hw[g / 2] = *reinterpret_cast<const uint32_t*>(&h2);
-          lw[g / 2] = *reinterpret_cast<const uint32_t*>(&l2);
+          if constexpr (kF8) {
+            const __half2 h2 = __floats2half2_rn(pr[g], pr[g + 1]);
+            const float2 hf = __half22float2(h2);
+            const __half2 l2 = __floats2half2_rn(pr[g] - hf.x, pr[g + 1] - hf.y);
+            hw[g / 2] = *reinterpret_cast<const uint32_t*>(&h2);
+            lw[g / 2] = *reinterpret_cast<const uint32_t*>(&l2);
+          } else {
+            const __nv_bfloat162 h2 = __floats2bfloat162_rn(pr[g], pr[g + 1]);
+            const float2 hf = __bfloat1622float2(h2);
+            const __nv_bfloat162 l2 = __floats2bfloat162_rn(pr[g] - hf.x, pr[g + 1] - hf.y);
+            hw[g / 2] = *reinterpret_cast<const uint32_t*>(&h2);
+            lw[g / 2] = *reinterpret_cast<const uint32_t*>(&l2);
+          }
         }
         ok = ok && mbar_wait(&S.pempty[sb], ((J >> 1) & 1u) ^ 1u, ctx);
         if (!kF8 && (valid & 15) != 0) {
