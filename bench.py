@@ -48,7 +48,7 @@ def parse_args():
     ap.add_argument("--steps", type=int, default=3000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["fd", "reference"], default="fd")
-    ap.add_argument("--workload", type=int, default=3, choices=[1, 2, 3, 4, 5])
+    ap.add_argument("--workload", type=int, default=3, choices=[1, 2, 3, 4, 5, 6])
     ap.add_argument("--batch", type=int, default=None,
                     help="batch of workload 4; for workloads 3 and 5, keep the first B requests")
     ap.add_argument("--page-size", type=int, default=0,
@@ -460,11 +460,27 @@ def run_fd(args, rank, world, local_rank):
         flops = chunk_tile_flops(inp)
         tpeak, tkind = measured_peak("bf16_tflops")
         ach = flops / (tile_ms * 1e-3) / 1e12
-        roofline_tiles = {"bound": "tensor", "kernel": "chunk_tc_kernel", "achieved": round(ach, 2),
-                          "peak": tpeak, "unit": "TFLOP/s", "frac": round(ach / tpeak, 4),
-                          "peak_kind": f"{tkind} dense bf16 (burst)",
-                          "algorithmic_flops_per_launch": flops,
-                          "traffic": traffic_from_profiles("chunk_tc.cu", inp.name)}
+        # the tile kernel's own K+V+Q bytes: requests of more than one row, keys read once per
+        # KV head (head-packed tiles) or once per query head from L2 (per-head tiles)
+        ck = inp.chunk_lens.tolist()
+        es = inp.k_cache.element_size()
+        tile_bytes = (2 * sum(n for n, c in zip(key_lens(inp), ck) if int(c) > 1) * hkv * d * es +
+                      sum(int(c) for c in ck if int(c) > 1) * hq * d * inp.q_chunk.element_size())
+        ridge = tpeak * 1e12 / (peak * 1e9)
+        tensor_view = {"bound": "tensor", "kernel": "chunk_tc_kernel", "achieved": round(ach, 2),
+                       "peak": tpeak, "unit": "TFLOP/s", "frac": round(ach / tpeak, 4),
+                       "peak_kind": f"{tkind} dense bf16 (burst)",
+                       "algorithmic_flops_per_launch": flops,
+                       "traffic": traffic_from_profiles("chunk_tc.cu", inp.name)}
+        hb = tile_bytes / (tile_ms * 1e-3) / 1e9
+        hbm_view = {"bound": "hbm", "kernel": "chunk_tc_kernel", "achieved": round(hb, 1),
+                    "peak": peak, "unit": "GB/s", "frac": round(hb / peak, 4),
+                    "peak_kind": f"{peak_kind} copy bandwidth",
+                    "algorithmic_bytes_per_launch": tile_bytes,
+                    "traffic": traffic_from_profiles("chunk_tc.cu", inp.name),
+                    "kernel_ms": roofline["kernel_ms"]}
+        # below the ridge point (flops per byte of the measured peaks) the tiles are memory-bound
+        roofline_tiles = hbm_view if flops / max(1, tile_bytes) < ridge else tensor_view
         if tile_ms > split_ms:
             roofline, roofline_tiles = roofline_tiles, roofline
 

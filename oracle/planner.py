@@ -47,7 +47,11 @@ CHUNK_KV_SPLIT keys: split s = [CHUNK_KV_SPLIT s, min(CHUNK_KV_SPLIT (s + 1), K_
 s < n_t = max(1, ceil(K_t / CHUNK_KV_SPLIT)). The grid is the same for every tile of a request, so
 the tiles of one head read the same K/V ranges. Every row of a tile owns n_t partial slots. Tile
 items run in the order (request, query head, split, tile): the tiles sharing a split's keys are
-adjacent, so they run at the same time and share those keys in L2.
+adjacent, so they run at the same time and share those keys in L2. A request with
+2 <= chunk_len <= 128 / G rows and G = Hq / Hkv >= 2 (a multi-token verification step, say) is
+served by head-packed tiles instead: one tile per (KV head, split) holds its rows for all G query
+heads (tile row r = chunk position r // G of query head h G + r mod G), so the head index of its
+items is a KV head; it has a single query tile (t = 0) and the same splits and slots.
 """
 
 from __future__ import annotations
@@ -129,9 +133,11 @@ def decode_plan(cache_lens: Sequence[int], num_kv_heads: int, cache_capacity: in
 class ChunkPlan:
     decode: DecodePlan                     # plan over the chunk_len == 1 requests (indexed by request)
     decode_requests: List[int]             # request index of each decode row, in request order
-    # (b, q_tile, q_head, split, key_start, key_end) in execution order
+    # (b, q_tile, q_head, split, key_start, key_end) in execution order; for a head-packed
+    # request the head is a KV head
     tile_items: List[Tuple[int, int, int, int, int, int]] = field(default_factory=list)
     row_splits: List[int] = field(default_factory=list)      # partial slots per packed row
+    head_packed: List[int] = field(default_factory=list)     # requests served by head-packed tiles
 
 
 def chunk_plan(prefix_lens: Sequence[int], chunk_lens: Sequence[int], num_q_heads: int,
@@ -145,6 +151,8 @@ def chunk_plan(prefix_lens: Sequence[int], chunk_lens: Sequence[int], num_q_head
     dec.items = [(dec_req[i], h, s, t0, t1) for (i, h, s, t0, t1) in dec.items]
     row_splits: List[int] = []
     tiles = []
+    packed: List[int] = []
+    G = num_q_heads // num_kv_heads
     for b in range(B):
         c = int(chunk_lens[b])
         if c == 1:
@@ -156,11 +164,15 @@ def chunk_plan(prefix_lens: Sequence[int], chunk_lens: Sequence[int], num_q_head
         n_t = [max(1, _cdiv(k, CHUNK_KV_SPLIT)) for k in k_t]
         for t in range(n_tiles):
             row_splits.extend([n_t[t]] * min(Q_TILE, c - Q_TILE * t))
-        for h in range(num_q_heads):
+        head_packed = G >= 2 and 2 <= c and c * G <= Q_TILE
+        if head_packed:
+            packed.append(b)
+        for h in range(num_kv_heads if head_packed else num_q_heads):
             for s in range(max(n_t)):
                 for t in range(n_tiles):
                     if s < n_t[t]:
                         k0 = min(CHUNK_KV_SPLIT * s, k_t[t])
                         k1 = min(CHUNK_KV_SPLIT * (s + 1), k_t[t])
                         tiles.append((b, t, h, s, k0, k1))
-    return ChunkPlan(decode=dec, decode_requests=dec_req, tile_items=tiles, row_splits=row_splits)
+    return ChunkPlan(decode=dec, decode_requests=dec_req, tile_items=tiles, row_splits=row_splits,
+                     head_packed=packed)

@@ -797,6 +797,8 @@ fd_status fd_chunk_prefill_attention(const fd_tensor* q_chunk, const fd_tensor* 
   tp.d = d;
   tp.cap = cap;
   tp.q_box_rows = std::min(128, T);
+  tp.qp_box_rows = std::min(kQTile / g, T);
+  tp.g_recip16 = (65536 + g - 1) / g;
   tp.kv_box_rows = std::min(128, cap);
   tp.scale_log2 = scale_log2;
   tp.hdr = hdr;
@@ -827,6 +829,11 @@ fd_status fd_chunk_prefill_attention(const fd_tensor* q_chunk, const fd_tensor* 
   const uint32_t qb_dec[3] = {64, static_cast<uint32_t>(dp.q_box_rows), 1};
   const uint32_t qb_tile[3] = {64, 1, static_cast<uint32_t>(tp.q_box_rows)};
   if ((s = make_tmap(&tq_tile, q_chunk->data, 3, qd, qs, qb_tile, "q_chunk")) != FD_OK) return s;
+  // head-packed tiles (groups >= 2): G heads x 128 / G rows per box
+  CUtensorMap tq_packed = tq_tile;
+  const uint32_t qb_packed[3] = {64, static_cast<uint32_t>(g), static_cast<uint32_t>(tp.qp_box_rows)};
+  if (g >= 2 && (s = make_tmap(&tq_packed, q_chunk->data, 3, qd, qs, qb_packed, "q_chunk (head-packed)")) != FD_OK)
+    return s;
   const uint64_t kd[4] = {static_cast<uint64_t>(d), static_cast<uint64_t>(cap), static_cast<uint64_t>(hkv), static_cast<uint64_t>(B)};
   const uint64_t ks[3] = {static_cast<uint64_t>(k_cache->stride[2]) * 2, static_cast<uint64_t>(k_cache->stride[1]) * 2,
                           static_cast<uint64_t>(k_cache->stride[0]) * 2};
@@ -845,7 +852,7 @@ fd_status fd_chunk_prefill_attention(const fd_tensor* q_chunk, const fd_tensor* 
     FD_CUDA(launch_decode_simt(dp, FD_BF16, dec_ctas, stream), "decode-row split kernel launch");
   }
   end_profile_events(ev, 2, stream);
-  FD_CUDA(launch_chunk_tc(tp, tq_tile, tk, tv, tile_ctas, stream), "chunk tile kernel launch");
+  FD_CUDA(launch_chunk_tc(tp, tq_tile, tq_packed, tk, tv, tile_ctas, stream), "chunk tile kernel launch");
   end_profile_events(ev, 3, stream);
   FD_CUDA(launch_combine(cp, stream), "combine kernel launch");
   end_profile_events(ev, 4, stream);

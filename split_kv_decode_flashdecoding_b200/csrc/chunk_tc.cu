@@ -22,10 +22,19 @@
 // LSE = m + log2 l: the final output when the tile has a single split, else a partial for the
 // combine kernel.
 //
+// Head-packed tiles (a request of 2 <= c <= 128 / G rows, G >= 2: a multi-token verification
+// step, "大模型推理加速FlashDecoding算法原理与多GPU并行解码实战", "与其他推理加速方案的组合使用",
+// item "Speculative Decoding + FlashDecoding"): one tile holds the c rows of all G query heads of
+// one KV head, tile row r being chunk position r / G of query head h G + r mod G, loaded by one
+// TMA box of G heads x 128 / G rows. Each key tile is then read and multiplied once per KV head,
+// not once per query head; the per-row causal limit and output address follow the mapping.
+//
 // Warp roles: 0-3 softmax (thread = TMEM lane = query row); 4 TMA producer of Q and K (2-stage
-// K ring, the next item's Q prefetched); 5 MMA issuer and TMEM owner; 6-9 epilogue (warp w reads
-// TMEM lanes 32 (w mod 4) + [0, 32)); 10 TMA producer of V (2-stage ring). K and V stages are
-// released separately: K once S has read it, V once P·V has.
+// K ring, the next item's Q prefetched); 5 issuer of the S products and TMEM owner; 6-9 epilogue
+// (warp w reads TMEM lanes 32 (w mod 4) + [0, 32)); 10 TMA producer of V (2-stage ring); 11
+// issuer of the P·V products. A tcgen05.mma holds its issuing thread for about as long as the
+// tensor pipe needs for it, so the two product chains of a tile are issued by two threads. K and
+// V stages are released separately: K once S has read it, V once P·V has.
 #include "common.cuh"
 #include "internal.h"
 
@@ -41,7 +50,8 @@ constexpr int kCkVStages = 2;
 constexpr int kCkProducer = 4;     // Q and K
 constexpr int kCkMma = 5;
 constexpr int kCkVProducer = 10;
-constexpr int kCkThreads = 11 * 32;
+constexpr int kCkPv = 11;          // issues the P·V products (warp 5 the S products)
+constexpr int kCkThreads = 12 * 32;
 constexpr uint32_t kCkTmemCols = 512;
 constexpr uint32_t kColS0 = 0, kColO0 = 256;   // S/P buffers at 0 and 128, O at 256 and 384
 constexpr uint32_t kCkHalf = kCkRows * 64 * 2;  // one 64-column half of a 128-row tile
@@ -66,7 +76,7 @@ struct __align__(1024) CkSmem {
   uint64_t pfull[2];
   uint64_t pfree;      // every P·V product (the softmax waits for the previous one to rescale O)
   uint64_t ofin[2], oempty[2], lready[2], lfree[2];  // by item parity
-  uint64_t drain;
+  uint64_t drain, drain_pv;
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -79,6 +89,7 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
 
 __global__ void __launch_bounds__(kCkThreads, 1)
     chunk_tc_kernel(const TileParams p, const __grid_constant__ CUtensorMap tmap_q,
+                    const __grid_constant__ CUtensorMap tmap_qp,
                     const __grid_constant__ CUtensorMap tmap_k,
                     const __grid_constant__ CUtensorMap tmap_v) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
@@ -98,7 +109,7 @@ __global__ void __launch_bounds__(kCkThreads, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&S.qfull[i], 1);
-      mbar_init(&S.qempty[i], 1 + 4 + 1);  // MMA, softmax warps, V producer
+      mbar_init(&S.qempty[i], 1 + 4 + 1 + 1);  // S issuer, softmax warps, V producer, P·V issuer
       mbar_init(&S.sfull[i], 1);
       mbar_init(&S.sfree[i], 1);
       mbar_init(&S.pfull[i], 4);
@@ -109,6 +120,7 @@ __global__ void __launch_bounds__(kCkThreads, 1)
     }
     mbar_init(&S.pfree, 1);
     mbar_init(&S.drain, 1);
+    mbar_init(&S.drain_pv, 1);
     S.abort_flag = 0;
     fence_mbar_init();
   }
@@ -118,6 +130,7 @@ __global__ void __launch_bounds__(kCkThreads, 1)
   }
   if (warp == kCkProducer && lane == 0) {
     prefetch_tensor_map(&tmap_q);
+    prefetch_tensor_map(&tmap_qp);
     prefetch_tensor_map(&tmap_k);
     prefetch_tensor_map(&tmap_v);
   }
@@ -151,10 +164,17 @@ __global__ void __launch_bounds__(kCkThreads, 1)
         S.item_slot[ps][0] = idx;
         S.item_slot[ps][1] = ntile;
         S.item[ps] = it;
-        mbar_arrive_expect_tx(&S.qfull[ps], 2u * 128u * static_cast<uint32_t>(p.q_box_rows));
-        tma_load_3d(S.q[ps][0], &tmap_q, &S.qfull[ps], 0, it.h, it.row0);
-        tma_load_3d(S.q[ps][1], &tmap_q, &S.qfull[ps], 64, it.h, it.row0);
-        const int hkv = it.h / p.g;
+        if (it.head_packed) {
+          // G heads x qp_box_rows chunk rows, rows ordered (chunk row, head)
+          mbar_arrive_expect_tx(&S.qfull[ps], 2u * 128u * static_cast<uint32_t>(p.g * p.qp_box_rows));
+          tma_load_3d(S.q[ps][0], &tmap_qp, &S.qfull[ps], 0, it.h * p.g, it.row0);
+          tma_load_3d(S.q[ps][1], &tmap_qp, &S.qfull[ps], 64, it.h * p.g, it.row0);
+        } else {
+          mbar_arrive_expect_tx(&S.qfull[ps], 2u * 128u * static_cast<uint32_t>(p.q_box_rows));
+          tma_load_3d(S.q[ps][0], &tmap_q, &S.qfull[ps], 0, it.h, it.row0);
+          tma_load_3d(S.q[ps][1], &tmap_q, &S.qfull[ps], 64, it.h, it.row0);
+        }
+        const int hkv = it.head_packed ? it.h : it.h / p.g;
         for (int j = 0; j < ntile; ++j, ++J) {
           if (j == claim_j) nidx = atomicAdd(&p.hdr->tile_counter, 1);
           const int st = J % kCkKStages;
@@ -205,7 +225,7 @@ __global__ void __launch_bounds__(kCkThreads, 1)
         const TileItem it = S.item[ps];
         mbar_arrive(&S.qempty[ps]);
         if (idx < 0) break;
-        const int hkv = it.h / p.g;
+        const int hkv = it.head_packed ? it.h : it.h / p.g;
         for (int j = 0; j < ntile; ++j, ++J) {
           const int st = J % kCkVStages;
           if (!mbar_wait(&S.vempty[st], ((J / kCkVStages) & 1u) ^ 1u, ctx)) { ok = false; break; }
@@ -230,43 +250,11 @@ __global__ void __launch_bounds__(kCkThreads, 1)
     }
     __syncwarp();
   } else if (warp == kCkMma) {
-    // ======================= MMA issuer =======================
+    // ======================= S issuer =======================
     if (lane == 0) {
       const uint32_t idesc_s = idesc_bf16_f32(kCkRows, kCkKeys, false, false);
-      const uint32_t idesc_o = idesc_bf16_f32(kCkRows, kCkD, false, true);
       uint32_t J = 0, K = 0;
       bool ok = true;
-      // the P·V product of a tile is issued after the S product of the next one
-      struct Pending { int valid; uint32_t jt, item; bool first, last; };
-      Pending prev{};
-      bool have_prev = false;
-      auto issue_pv = [&](const Pending& pv) -> bool {
-        const int vs = pv.jt % kCkVStages;
-        const int ob = pv.item & 1;
-        if (!mbar_wait(&S.vfull[vs], (pv.jt / kCkVStages) & 1u, ctx)) return false;
-        if (!mbar_wait(&S.pfull[pv.jt & 1], (pv.jt >> 1) & 1u, ctx)) return false;
-        // the item's first product overwrites the accumulator the item two back used
-        if (pv.first && !mbar_wait(&S.oempty[ob], ((pv.item >> 1) & 1u) ^ 1u, ctx)) return false;
-        tc_fence_after();
-        const int nk = (pv.valid + 15) / 16;
-        const uint32_t vaddr = smem_u32(S.v[vs][0]);
-        const uint32_t pcol = kColS0 + (pv.jt & 1) * 128;  // P of this tile, over its S buffer
-        const uint32_t ocol = kColO0 + ob * 128;
-        bool acc = !pv.first;
-        for (int part = 0; part < 2; ++part) {
-          for (int kk = 0; kk < nk; ++kk) {
-            const uint64_t bd = smem_desc(vaddr + kk * 2048, kCkHalf, 1024, kLayoutSW128);
-            const uint32_t acol = pcol + 32 * (kk >> 1) + 16 * part + 8 * (kk & 1);
-            umma_bf16_ts(tmem + ocol, tmem + acol, bd, idesc_o, acc ? 1u : 0u);
-            acc = true;
-          }
-        }
-        umma_commit(&S.pfree);
-        umma_commit(&S.sfree[pv.jt & 1]);
-        umma_commit(&S.vempty[vs]);
-        if (pv.last) umma_commit(&S.ofin[ob]);
-        return true;
-      };
       while (ok) {
         const int ps = K & 1;
         if (!mbar_wait(&S.qfull[ps], (K >> 1) & 1u, ctx)) { ok = false; break; }
@@ -279,6 +267,7 @@ __global__ void __launch_bounds__(kCkThreads, 1)
           const int st = J % kCkKStages;
           const int sb = J & 1;
           if (!mbar_wait(&S.kfull[st], (J / kCkKStages) & 1u, ctx)) { ok = false; break; }
+          // the S/P buffer is free once the P·V product of tile J - 2 has read its P
           if (!mbar_wait(&S.sfree[sb], ((J >> 1) & 1u) ^ 1u, ctx)) { ok = false; break; }
           tc_fence_after();
           const int valid = S.meta[st];
@@ -296,16 +285,61 @@ __global__ void __launch_bounds__(kCkThreads, 1)
           umma_commit(&S.sfull[sb]);
           umma_commit(&S.kempty[st]);
           if (j == ntile - 1) umma_commit(&S.qempty[ps]);
-          if (have_prev && !issue_pv(prev)) { ok = false; break; }
-          have_prev = true;
-          prev = Pending{valid, J, K, j == 0, j == ntile - 1};
         }
         if (!ok) break;
         ++K;
       }
-      if (ok && have_prev) ok = issue_pv(prev);
       umma_commit(&S.drain);
       mbar_drain(&S.drain, 0);
+    }
+    __syncwarp();
+  } else if (warp == kCkPv) {
+    // ======================= P·V issuer =======================
+    // Follows the items the Q/K producer publishes; each tile's keys come from the item.
+    if (lane == 0) {
+      const uint32_t idesc_o = idesc_bf16_f32(kCkRows, kCkD, false, true);
+      uint32_t J = 0, K = 0;
+      bool ok = true;
+      while (ok) {
+        const int ps = K & 1;
+        if (!mbar_wait(&S.qfull[ps], (K >> 1) & 1u, ctx)) { ok = false; break; }
+        const int idx = S.item_slot[ps][0];
+        const int ntile = S.item_slot[ps][1];
+        const TileItem it = S.item[ps];
+        mbar_arrive(&S.qempty[ps]);
+        if (idx < 0) break;
+        const int ob = K & 1;
+        for (int j = 0; j < ntile; ++j, ++J) {
+          const int vs = J % kCkVStages;
+          const int valid = max(0, min(kCkKeys, it.k1 - (it.k0 + j * kCkKeys)));
+          if (!mbar_wait(&S.vfull[vs], (J / kCkVStages) & 1u, ctx)) { ok = false; break; }
+          if (!mbar_wait(&S.pfull[J & 1], (J >> 1) & 1u, ctx)) { ok = false; break; }
+          // the item's first product overwrites the accumulator the item two back used
+          if (j == 0 && !mbar_wait(&S.oempty[ob], ((K >> 1) & 1u) ^ 1u, ctx)) { ok = false; break; }
+          tc_fence_after();
+          const int nk = (valid + 15) / 16;
+          const uint32_t vaddr = smem_u32(S.v[vs][0]);
+          const uint32_t pcol = kColS0 + (J & 1) * 128;  // P of this tile, over its S buffer
+          const uint32_t ocol = kColO0 + ob * 128;
+          bool acc = j > 0;
+          for (int part = 0; part < 2; ++part) {
+            for (int kk = 0; kk < nk; ++kk) {
+              const uint64_t bd = smem_desc(vaddr + kk * 2048, kCkHalf, 1024, kLayoutSW128);
+              const uint32_t acol = pcol + 32 * (kk >> 1) + 16 * part + 8 * (kk & 1);
+              umma_bf16_ts(tmem + ocol, tmem + acol, bd, idesc_o, acc ? 1u : 0u);
+              acc = true;
+            }
+          }
+          umma_commit(&S.pfree);
+          umma_commit(&S.sfree[J & 1]);
+          umma_commit(&S.vempty[vs]);
+          if (j == ntile - 1) umma_commit(&S.ofin[ob]);
+        }
+        if (!ok) break;
+        ++K;
+      }
+      umma_commit(&S.drain_pv);
+      mbar_drain(&S.drain_pv, 0);
     }
     __syncwarp();
   } else if (warp < 4) {
@@ -334,8 +368,18 @@ __global__ void __launch_bounds__(kCkThreads, 1)
         }
         break;
       }
-      const bool row_ok = r < it.rows;
-      const int limit = it.prefix + it.pos0 + r;  // last visible key of this row
+      // The item's descriptor goes to the epilogue warps now (their hand-off slot of this parity
+      // is free once they have read the item two back), so it need not stay in registers across
+      // the key tiles; the per-row max and sum follow at the end.
+      if (!mbar_wait(&S.lfree[ob], ((K >> 1) & 1u) ^ 1u, ctx)) break;
+      if (tid == 0) {
+        S.epi[ob] = it;
+        S.epi_stop[ob] = 0;
+      }
+      // chunk position of this tile row (head-packed: row r is position r / G of head r mod G)
+      // and the last key it sees (below every key when the row lies outside the chunk)
+      const int pos = it.head_packed ? (r * p.g_recip16) >> 16 : r;
+      const int limit = pos < it.rows ? it.prefix + it.pos0 + pos : -1;
       float m = -INFINITY, l = 0.f;
       for (int j = 0; j < ntile; ++j, ++J) {
         const int sb = J & 1;
@@ -346,7 +390,7 @@ __global__ void __launch_bounds__(kCkThreads, 1)
         const int valid = max(0, min(kCkKeys, it.k1 - kt0));
         // keys [0, nvis) of the tile are visible to this row: inside the split, at or before the
         // row's causal limit, and the row inside the chunk
-        const int nvis = row_ok ? max(0, min(valid, limit - kt0 + 1)) : 0;
+        const int nvis = max(0, min(valid, limit - kt0 + 1));
         const bool full = __all_sync(0xffffffffu, nvis == kCkKeys);
         const uint32_t sp = tmem + lane_base + kColS0 + sb * 128;  // this tile's S, then its P
         // pass 1: the row's maximum over its visible keys (scale > 0, so it is applied after);
@@ -455,14 +499,9 @@ __global__ void __launch_bounds__(kCkThreads, 1)
         if (lane == 0) mbar_arrive(&S.pfull[sb]);
       }
       if (!ok) break;
-      // ---- hand the item to the epilogue warps ----
-      if (!mbar_wait(&S.lfree[ob], ((K >> 1) & 1u) ^ 1u, ctx)) break;
+      // ---- hand the rows' running max and sum to the epilogue warps ----
       S.mfin[ob][r] = m;
       S.lfin[ob][r] = l;
-      if (tid == 0) {
-        S.epi[ob] = it;
-        S.epi_stop[ob] = 0;
-      }
       __syncwarp();
       if (lane == 0) mbar_arrive(&S.lready[ob]);
       ++K;
@@ -483,18 +522,20 @@ __global__ void __launch_bounds__(kCkThreads, 1)
       if (lane == 0) mbar_arrive(&S.lfree[ob]);
       if (!mbar_wait(&S.ofin[ob], (K >> 1) & 1u, ctx)) break;
       tc_fence_after();
-      const bool row_ok = r < it.rows;
+      const int pos = it.head_packed ? (r * p.g_recip16) >> 16 : r;  // chunk position of the row
+      const bool row_ok = pos < it.rows;
       const bool direct = it.nsplit == 1;
       const float inv = l > 0.f ? 1.f / l : 0.f;
       const float lse2 = l > 0.f ? m + log2f(l) : -INFINITY;
       // a row that saw no key has O = 0 (its accumulator may never have been written)
       const bool seen = l > 0.f;
-      const int hkv = it.h / p.g, g = it.h - hkv * p.g;
-      const int64_t row = static_cast<int64_t>(it.row0) + r;
+      const int head = it.head_packed ? it.h * p.g + (r - pos * p.g) : it.h;  // query head
+      const int hkv = head / p.g, g = head - hkv * p.g;
+      const int64_t row = static_cast<int64_t>(it.row0) + pos;
       const int64_t slot = static_cast<int64_t>(it.slot0) +
-                           (static_cast<int64_t>(r) * p.hkv + hkv) * it.nsplit + it.split;
+                           (static_cast<int64_t>(pos) * p.hkv + hkv) * it.nsplit + it.split;
       __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out) + row * p.o_sr +
-                           static_cast<int64_t>(it.h) * p.o_sh;
+                           static_cast<int64_t>(head) * p.o_sh;
       float* dst = p.part_o + (slot * p.g + g) * kCkD;
 #pragma unroll 1
       for (int c = 0; c < kCkD; c += 32) {
@@ -529,7 +570,7 @@ __global__ void __launch_bounds__(kCkThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&S.oempty[ob]);
       if (row_ok) {
-        if (direct) p.lse[row * p.hq + it.h] = lse2 * kLn2;
+        if (direct) p.lse[row * p.hq + head] = lse2 * kLn2;
         else p.part_lse[slot * p.g + g] = lse2;
       }
     }
@@ -543,8 +584,9 @@ __global__ void __launch_bounds__(kCkThreads, 1)
 
 }  // namespace
 
-cudaError_t launch_chunk_tc(const TileParams& p, const CUtensorMap& tq, const CUtensorMap& tk,
-                            const CUtensorMap& tv, int nctas, cudaStream_t stream) {
+cudaError_t launch_chunk_tc(const TileParams& p, const CUtensorMap& tq, const CUtensorMap& tqp,
+                            const CUtensorMap& tk, const CUtensorMap& tv, int nctas,
+                            cudaStream_t stream) {
   const size_t smem = sizeof(CkSmem) + 1024;
   cudaError_t e = cudaFuncSetAttribute(chunk_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
@@ -559,7 +601,7 @@ cudaError_t launch_chunk_tc(const TileParams& p, const CUtensorMap& tq, const CU
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, chunk_tc_kernel, p, tq, tk, tv);
+  return cudaLaunchKernelEx(&cfg, chunk_tc_kernel, p, tq, tqp, tk, tv);
 }
 
 }  // namespace fd

@@ -54,7 +54,9 @@ struct TileItem {
   int32_t rows;      // valid rows in the tile (<= kQTile)
   int32_t prefix;    // prefix length: row at chunk position i sees keys <= prefix + i
   int32_t slot0;     // partial slot of (row0, split 0); row r uses slot0 + r * nsplit + split
-  int32_t pad[5];
+  int32_t head_packed;  // 1: head-packed tile (h is a KV head; tile row r is chunk position r / G of
+                        // query head h * G + r % G); 0: one query head h, tile row = chunk position
+  int32_t pad[4];
 };
 static_assert(sizeof(TileItem) == 64, "TileItem is 64 bytes");
 
@@ -148,6 +150,11 @@ FD_HD int32_t chunk_tile_keys(int32_t prefix, int32_t c, int32_t t, int32_t cap)
   const int64_t k = static_cast<int64_t>(prefix) + (last < c ? last : c);
   return k < 0 ? 0 : (k > cap ? cap : static_cast<int32_t>(k));
 }
+// A request of 2 <= c <= kQTile / G chunk rows with G >= 2 query heads per KV head (a
+// multi-token verification step, say) is served by head-packed tiles: one 128-row tile holds its
+// c rows for all G heads of a KV head, so every key tile is read and multiplied once per KV head
+// rather than once per query head.
+FD_HD bool chunk_packed(int32_t c, int32_t g) { return g >= 2 && c >= 2 && c * g <= kQTile; }
 FD_HD int32_t chunk_tile_splits(int32_t keys) {
   const int32_t n = static_cast<int32_t>(cdiv64(keys, kChunkKvSplit));
   return n < 1 ? 1 : n;

@@ -251,7 +251,7 @@ __global__ void __launch_bounds__(kMaxPlanThreads, 1) plan_chunk_kernel(PlanPara
         const int32_t kt = chunk_tile_keys(s_p[b], c, t, p.cap);
         cnt += chunk_tile_splits(kt);
       }
-      s_tcnt[b] = cnt * p.hq;
+      s_tcnt[b] = cnt * (chunk_packed(c, p.hq / p.hkv) ? p.hkv : p.hq);
     }
   }
   __syncthreads();
@@ -310,15 +310,18 @@ __global__ void __launch_bounds__(kMaxPlanThreads, 1) plan_chunk_kernel(PlanPara
       }
     }
   }
-  // tile items: one warp per request, lanes over query heads, (split, tile) order per head
+  // tile items: one warp per request, lanes over query heads (KV heads for head-packed tiles),
+  // (split, tile) order per head
   for (int b = warp; b < B && !overflow; b += nthr / 32) {
     const int32_t c = s_c[b];
     if (c < 2) continue;
     const int32_t pp = s_p[b], r0 = s_roff[b];
     const int32_t ntiles = (c + kQTile - 1) / kQTile;
-    const int32_t per_head = s_tcnt[b] / p.hq;
+    const int32_t head_packed = chunk_packed(c, p.hq / p.hkv) ? 1 : 0;
+    const int32_t nheads = head_packed ? p.hkv : p.hq;
+    const int32_t per_head = s_tcnt[b] / nheads;
     const int32_t nmax = chunk_tile_splits(chunk_tile_keys(pp, c, ntiles - 1, p.cap));
-    for (int32_t h = lane; h < p.hq; h += 32) {
+    for (int32_t h = lane; h < nheads; h += 32) {
       int32_t i = s_tioff[b] + h * per_head;
       for (int32_t s = 0; s < nmax; ++s) {
         for (int32_t t = 0; t < ntiles; ++t) {
@@ -332,7 +335,7 @@ __global__ void __launch_bounds__(kMaxPlanThreads, 1) plan_chunk_kernel(PlanPara
           int4* dst = reinterpret_cast<int4*>(p.tiles + i);
           dst[0] = make_int4(b, h, s, nt);
           dst[1] = make_int4(k0, k1, row0, t * kQTile);
-          dst[2] = make_int4(rows, pp, slot0, 0);
+          dst[2] = make_int4(rows, pp, slot0, head_packed);
           dst[3] = make_int4(0, 0, 0, 0);
           ++i;
         }

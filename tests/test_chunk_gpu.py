@@ -102,3 +102,53 @@ def test_chunk_deterministic():
     o1, l1 = _run(inp)
     o2, l2 = _run(inp)
     assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
+# Multi-token verification steps: requests of 2 <= c <= 128 / G rows with G >= 2 heads per KV head
+# run as head-packed tiles (one tile holds the rows of all G heads of a KV head).
+VERIFY = [
+    # (prefix_lens, chunk_lens, Hq, Hkv, cap)
+    ([3000, 5, 0, 2047], [4, 4, 4, 4], 64, 8, 3072),        # G = 8, k = 4: 32 rows per tile
+    ([500, 9000], [16, 2], 64, 8, 9216),                     # k = 16 fills the tile; k = 2
+    ([700, 60], [32, 17], 16, 4, 1024),                      # G = 4, k = 32 (full) and 17
+    ([1000, 33, 2100], [8, 1, 3], 16, 2, 2304),              # G = 8 with a decode row
+    ([4100, 300, 90], [4, 17, 130], 32, 4, 4352),            # packed, per-head (17 > 16) and two tiles
+    ([257, 0], [3, 5], 6, 2, 320),                           # G = 3: rows r // 3 and r % 3
+]
+
+
+@pytest.mark.parametrize("case", range(len(VERIFY)))
+def test_verification_head_packed(case):
+    prefix, chunk, hq, hkv, cap = VERIFY[case]
+    inp = make_chunk_inputs(prefix, chunk, hq, hkv, 128, cap, torch.bfloat16, seed=700 + case,
+                            pad_fill=NAN)
+    out, lse = _run(inp)
+    ro, rl = _oracle(inp)
+    check_out(out, ro, "verification out")
+    check_lse(lse, rl, "verification lse")
+
+
+def test_verification_equals_decode_rows():
+    # k = 4 tokens of one request, G = 8: token i gives the decode result over prefix + i + 1 keys
+    import split_kv_decode_flashdecoding_b200 as fd
+    inp = make_chunk_inputs([1500], [4], 64, 8, 128, 2048, torch.bfloat16, seed=720)
+    out, lse = _run(inp)
+    dev = torch.device("cuda", 0)
+    for i in range(4):
+        q = inp.q_chunk[i:i + 1].to(dev)
+        lens = torch.tensor([1501 + i], dtype=torch.int32, device=dev)
+        o, l = fd.fd_decode_attention(q, inp.k_cache.to(dev), inp.v_cache.to(dev), lens)
+        torch.cuda.synchronize()
+        check_out(out[i:i + 1], o.float().cpu().numpy().astype(np.float64), f"token {i} vs decode")
+        check_lse(lse[i:i + 1], l.cpu().numpy().astype(np.float64), f"token {i} lse vs decode")
+
+
+def test_verification_workload_sampled():
+    # the 70B-like decode batch verifying 4 speculative tokens per sequence, at full size
+    inp = workload(6)
+    out, lse = _run(inp, guard=False)
+    T, hq = out.shape[0], out.shape[1]
+    rows = sample_rows(T, hq, 32, seed=11, must=[(0, 0), (T - 1, hq - 1), (3, 63)])
+    ro, rl = _oracle(inp, rows=rows)
+    check_out(out, ro, "verification workload out")
+    check_lse(lse, rl, "verification workload lse")

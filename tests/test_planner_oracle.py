@@ -167,3 +167,18 @@ def test_aligned_plan_properties(seed):
                 # splits of a fixed count sit at [len, len))
                 assert t0 <= t1 and (t0 % 128 == 0 or t0 == lens[b])
                 assert t1 % 128 == 0 or t1 == lens[b]
+
+
+def test_chunk_plan_head_packed_requests():
+    # G = 8: chunks of 2..16 rows are head-packed (one tile per KV head and split), longer ones
+    # and decode rows are not; G = 1 never packs
+    cp = P.chunk_plan([3000, 40, 100, 7], [4, 16, 17, 1], 64, 8, 8192, 148)
+    assert cp.head_packed == [0, 1]
+    heads0 = sorted({h for (b, t, h, s, k0, k1) in cp.tile_items if b == 0})
+    assert heads0 == list(range(8))
+    # request 0 sees 3004 keys: two splits per KV head, one query tile
+    assert sorted({(t, s, k0, k1) for (b, t, h, s, k0, k1) in cp.tile_items if b == 0}) == \
+        [(0, 0, 0, 2048), (0, 1, 2048, 3004)]
+    assert len([1 for it in cp.tile_items if it[0] == 2]) == 64      # per query head
+    assert cp.row_splits[:4] == [2, 2, 2, 2] and cp.row_splits[4:20] == [1] * 16
+    assert P.chunk_plan([10], [4], 8, 8, 1024, 148).head_packed == []

@@ -19,9 +19,10 @@ round-to-nearest-even):
   scale = (largest finite |value| over the tensor) / 448 rounded to float32, codes = torch's
   round-to-nearest cast of value / scale to float8_e4m3fn (NaN padding stays NaN).
 
-The named workloads are the five benchmark shapes of this project (decode MHA fp32, decode
-MHA bf16 13B-like, decode GQA bf16 70B-like, long-context GQA, mixed chunked-prefill step);
-tensor seed = 1000 + index, length seed = 1100 + index.
+The named workloads are the six benchmark shapes of this project (decode MHA fp32, decode
+MHA bf16 13B-like, decode GQA bf16 70B-like, long-context GQA, mixed chunked-prefill step, and
+the 70B-like batch verifying 4 speculative tokens per sequence); tensor seed = 1000 + index,
+length seed = 1100 + index (the verification step reuses the 70B-like lengths).
 """
 
 from __future__ import annotations
@@ -200,11 +201,12 @@ WORKLOADS = {
     3: "decode_gqa_bf16_b32_hq64_hkv8_d128_lenU1024-32768",
     4: "longctx_gqa_bf16_hq64_hkv8_d128_len32768_peaked",
     5: "mixed_chunk512_prefix15872_plus31decode_h32_d128",
+    6: "verify4_gqa_bf16_b32_hq64_hkv8_d128_lenU1024-32768",
 }
 
 
 def workload(index: int, batch: Optional[int] = None, pad_fill: float = 0.0):
-    """Build one of the five named workloads (index 1..5) at its full size."""
+    """Build one of the six named workloads (index 1..6) at its full size."""
     seed = 1000 + index
     lseed = 1100 + index
     if index == 1:
@@ -232,6 +234,14 @@ def workload(index: int, batch: Optional[int] = None, pad_fill: float = 0.0):
         name = WORKLOADS[5] if b == 32 else f"{WORKLOADS[5]}_first{b}"
         return make_chunk_inputs(prefix[:b], chunk[:b], 32, 32, 128, 16384, torch.bfloat16,
                                  seed, pad_fill=pad_fill, name=name)
+    if index == 6:
+        # multi-token verification: every sequence of the 70B-like decode batch checks 4
+        # speculative tokens, appended to its cache (prefix + 4 = a length of workload 3's draw)
+        lens = uniform_lens(1100 + 3, 32, 1024, 32768)
+        b = 32 if batch is None else int(batch)
+        name = WORKLOADS[6] if b == 32 else f"{WORKLOADS[6]}_first{b}"
+        return make_chunk_inputs([n - 4 for n in lens[:b]], [4] * b, 64, 8, 128, 32768,
+                                 torch.bfloat16, seed, pad_fill=pad_fill, name=name)
     raise ValueError(f"unknown workload {index}")
 
 
