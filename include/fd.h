@@ -241,7 +241,11 @@ fd_status fd_split_plan_device(const int32_t* cache_lens, int32_t batch, int32_t
  * cache. Reading: row i of request b sees keys j <= prefix_lens[b] + i (bottom-right aligned).
  * A request with chunk_len == 1 is a decode row and runs through the split-KV decode kernels;
  * longer chunks run through tensor-core tiles of 128 query rows, split along the keys; one
- * combine pass merges every row.
+ * combine pass merges every row. Multi-token verification (FlashDecoding page, "与其他推理加速
+ * 方案的组合使用", item "Speculative Decoding + FlashDecoding": k speculative tokens checked in
+ * one pass) is this call with chunk_lens[b] = k: a request of 2 <= k <= 128 / G rows (G = Hq /
+ * Hkv >= 2) runs as head-packed tiles, all G query heads of a KV head in one tile, so its keys
+ * are read once per KV head.
  *
  *  q_chunk     [T, Hq, D] with T = sum(chunk_lens), packed request by request; D == 128, bf16.
  *  k_cache,    [B, Hkv, S_cap, D] bf16, holding each request's keys/values at

@@ -252,7 +252,9 @@ def fd_chunk_prefill_attention(q_chunk: torch.Tensor, k_cache: torch.Tensor,
                                chunk_lens: torch.Tensor, out: Optional[torch.Tensor] = None,
                                lse: Optional[torch.Tensor] = None,
                                stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
-    """Causal attention of packed query chunks [T,Hq,D] against their cached prefix + self."""
+    """Causal attention of packed query chunks [T,Hq,D] against their cached prefix + self.
+    chunk_lens[b] = 1 is a decode row; chunk_lens[b] = k speculative tokens is a verification
+    step (head-packed tiles when 2 <= k <= 128 / (Hq / Hkv))."""
     if out is None:
         out = torch.empty_like(q_chunk)
     if lse is None:
