@@ -28,7 +28,7 @@ rounding, so the oracle is the definition itself with no splitting):
         O    = sum_j exp(s_j - M) v_j / sum_j exp(s_j - M)
         LSE  = M + ln sum_j exp(s_j - M)              (natural log of the scaled scores)
 
-Readings where the pages are silent (each is listed in the design doc):
+Readings where the pages are silent:
 
 * n = 0 gives O = 0 and LSE = -inf.
 * A cache length outside [0, S_cap] is clamped into that range (the CUDA side clamps too
