@@ -114,6 +114,8 @@ VERIFY = [
     ([1000, 33, 2100], [8, 1, 3], 16, 2, 2304),              # G = 8 with a decode row
     ([4100, 300, 90], [4, 17, 130], 32, 4, 4352),            # packed, per-head (17 > 16) and two tiles
     ([257, 0], [3, 5], 6, 2, 320),                           # G = 3: rows r // 3 and r % 3
+    ([900, 40], [8, 8], 16, 1, 1024),                        # G = 16, k = 8 fills the tile
+    ([2200, 10], [64, 33], 4, 2, 2304),                      # G = 2, k = 64 (full) and 33
 ]
 
 
@@ -152,3 +154,40 @@ def test_verification_workload_sampled():
     ro, rl = _oracle(inp, rows=rows)
     check_out(out, ro, "verification workload out")
     check_lse(lse, rl, "verification workload lse")
+
+
+def test_verification_cuda_graph_replay():
+    # a captured verification step replayed with new prefix lengths (same chunk lengths)
+    import split_kv_decode_flashdecoding_b200 as fd
+    from workloads import ChunkInputs
+    dev = torch.device("cuda", 0)
+    prefix, chunk = [3000, 500, 1000], [4, 4, 4]
+    base = make_chunk_inputs(prefix, chunk, 64, 8, 128, 4096, torch.bfloat16, seed=730)
+    q, k, v = base.q_chunk.to(dev), base.k_cache.to(dev), base.v_cache.to(dev)
+    pl, cl = base.prefix_lens.to(dev), base.chunk_lens.to(dev)
+    out = torch.empty_like(q)
+    lse = torch.empty(q.shape[:2], dtype=torch.float32, device=dev)
+    s = torch.cuda.Stream()
+    nct = fd.fd_decode_num_ctas(0, torch.bfloat16, 8, 128)
+    fd.fd_reserve_workspace(fd.fd_chunk_workspace_bytes(3, 12, 64, 8, 4096, 128, nct), stream=s)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        fd.fd_chunk_prefill_attention(q, k, v, pl, cl, out=out, lse=lse, stream=s)
+    for new in ([3000, 500, 1000], [10, 2500, 0]):
+        kk = base.k_cache.clone()
+        vv = base.v_cache.clone()
+        for b, p0 in enumerate(new):
+            kk[b, :, p0 + chunk[b]:] = NAN
+            vv[b, :, p0 + chunk[b]:] = NAN
+        k.copy_(kk)
+        v.copy_(vv)
+        pl.copy_(torch.tensor(new, dtype=torch.int32))
+        g.replay()
+        torch.cuda.synchronize()
+        ref_in = ChunkInputs(q_chunk=base.q_chunk, k_cache=kk, v_cache=vv,
+                             prefix_lens=torch.tensor(new, dtype=torch.int32),
+                             chunk_lens=base.chunk_lens)
+        ro, rl = _oracle(ref_in)
+        check_out(out, ro, "verification graph out")
+        check_lse(lse, rl, "verification graph lse")
+    del g

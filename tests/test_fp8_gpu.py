@@ -146,6 +146,7 @@ def test_fp8_accepts_float8_tensors():
 PAGED = [
     # (B, Hq, Hkv, page_size, lens, cap)
     (4, 64, 8, 16, [300, 1, 0, 129], 320),
+    (2, 64, 8, 8, [77, 200], 200),               # 8-key pages: 16 boxes per key tile
     (3, 64, 8, 128, [1000, 128, 257], 1024),
     (2, 32, 4, 256, [2000, 255], 2048),
     (2, 8, 8, 64, [513, 64], 576),
@@ -204,3 +205,52 @@ def test_fp8_workload_3_sampled():
                      rows=rows)
     check_out(out, ro, "fp8 w3 out")
     check_lse(lse, rl, "fp8 w3 lse")
+
+
+def test_fp8_planner_kernel_batch():
+    # above 256 sequences the planner kernel plans the call instead of the split kernel itself
+    rng = np.random.default_rng(660)
+    B = 300
+    lens = [int(x) for x in rng.integers(0, 400, size=B)]
+    inp = make_decode_inputs(B, 16, 2, 128, 400, lens, torch.bfloat16, seed=661, pad_fill=NAN)
+    f8 = make_fp8(inp.k_cache, inp.v_cache)
+    out, lse = _run(inp.q, f8.k_codes, f8.v_codes, f8.k_scale, f8.v_scale, inp.cache_lens)
+    rows = sample_rows(B, 16, 48, seed=5, must=[(0, 0), (B - 1, 15), (B // 2, 7)])
+    ro, rl = _oracle(inp.q, f8.k_codes, f8.v_codes, f8.k_scale, f8.v_scale, inp.cache_lens,
+                     rows=rows)
+    check_out(out, ro, "fp8 B 300 out")
+    check_lse(lse, rl, "fp8 B 300 lse")
+
+
+def test_fp8_cuda_graph_replay_new_lengths():
+    fd = _fd()
+    dev = _dev()
+    base = make_decode_inputs(3, 64, 8, 128, 2048, [2048] * 3, torch.bfloat16, seed=670)
+    f8 = make_fp8(base.k_cache, base.v_cache)
+    q, k, v = base.q.to(dev), f8.k_codes.to(dev), f8.v_codes.to(dev)
+    lens = base.cache_lens.to(dev)
+    out = torch.empty_like(q)
+    lse = torch.empty(q.shape[:2], dtype=torch.float32, device=dev)
+    s = torch.cuda.Stream()
+    nct = fd.fd_decode_num_ctas(0, torch.uint8, 8, 128)
+    fd.fd_reserve_workspace(fd.fd_decode_workspace_bytes(3, 64, 8, 2048, 128, 0, nct), stream=s)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        fd.fd_decode_attention_fp8(q, k, v, f8.k_scale, f8.v_scale, lens, 0, out=out, lse=lse,
+                                   stream=s)
+    for new in ([2048, 100, 1500], [7, 2000, 1]):
+        # codes past the new lengths must not be read: poison them with the NaN code
+        kk = f8.k_codes.clone()
+        vv = f8.v_codes.clone()
+        for b, n in enumerate(new):
+            kk[b, :, n:] = 0x7F
+            vv[b, :, n:] = 0x7F
+        k.copy_(kk)
+        v.copy_(vv)
+        lens.copy_(torch.tensor(new, dtype=torch.int32))
+        g.replay()
+        torch.cuda.synchronize()
+        ro, rl = _oracle(base.q, kk, vv, f8.k_scale, f8.v_scale, torch.tensor(new))
+        check_out(out, ro, "fp8 graph out")
+        check_lse(lse, rl, "fp8 graph lse")
+    del g
