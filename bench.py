@@ -230,6 +230,20 @@ def cpu_threads() -> int:
     return os.cpu_count() or 1
 
 
+def cpu_model() -> str:
+    """The host CPU's model name (first processor in /proc/cpuinfo) and its logical CPU count."""
+    name = "unknown"
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    name = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return f"{name}, {os.cpu_count() or 1} logical CPUs"
+
+
 def oracle_sample(inp, seconds: float, seed: int = 0, quant=None):
     """Time the oracle on whole (query row, KV head) groups of the workload, all G query heads
     each, in a seeded order, until `seconds` of host time are spent. `quant` = (k_scale, v_scale):
@@ -322,7 +336,7 @@ def run_reference(args, rank, world):
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": inp.name},
         "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": cpu_threads(),
-                         "kind": "oracle",
+                         "kind": "oracle", "cpu": cpu_model(),
                          "sample": f"per step: whole (query row, KV head) groups of the workload in a "
                                    f"seeded order until {per_step:.2f}s of host time (or all groups)"},
         "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
@@ -528,7 +542,7 @@ def run_fd(args, rank, world, local_rank):
         rate, desc, groups, el = oracle_sample(inp, args.cpu_seconds,
                                                quant=(f8.k_scale, f8.v_scale) if fp8 else None)
         cpu = {"value": round(rate / 1e9, 4), "unit": "GB/s", "cores": cpu_threads(),
-               "kind": "oracle", "sample": f"{desc}; {el:.1f}s"}
+               "kind": "oracle", "cpu": cpu_model(), "sample": f"{desc}; {el:.1f}s"}
 
     if rank == 0:
         config = {"workload": inp.name, "batch": R if not chunk else B, "q_heads": hq, "kv_heads": hkv,
