@@ -158,6 +158,8 @@ def chunk_plan(prefix_lens: Sequence[int], chunk_lens: Sequence[int], num_q_head
         if c == 1:
             row_splits.append(dec.splits_per_seq[dec_req.index(b)])
             continue
+        if c <= 0:
+            continue  # an empty chunk has no rows and no items
         p = int(prefix_lens[b])
         n_tiles = _cdiv(c, Q_TILE)
         k_t = [max(0, min(p + min(c, Q_TILE * (t + 1)), int(cache_capacity))) for t in range(n_tiles)]

@@ -182,3 +182,41 @@ def test_chunk_plan_head_packed_requests():
     assert len([1 for it in cp.tile_items if it[0] == 2]) == 64      # per query head
     assert cp.row_splits[:4] == [2, 2, 2, 2] and cp.row_splits[4:20] == [1] * 16
     assert P.chunk_plan([10], [4], 8, 8, 1024, 148).head_packed == []
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_chunk_plan_head_packed_coverage(seed):
+    # every chunk request is covered exactly once per (head, split, tile): KV heads for
+    # head-packed requests (2 <= c <= 128 / G, G >= 2), query heads otherwise
+    rng = random.Random(seed)
+    hkv = rng.choice([1, 2, 4, 8])
+    G = rng.choice([1, 2, 3, 4, 8, 16])
+    hq = hkv * G
+    cap = 8192
+    B = rng.randint(1, 10)
+    chunk = [rng.choice([0, 1, 2, 4, 8, 16, 17, 33, 64, 130, 300]) for _ in range(B)]
+    prefix = [rng.randint(0, cap - c) for c in chunk]
+    cp = P.chunk_plan(prefix, chunk, hq, hkv, cap, 148)
+    want_packed = [b for b in range(B) if G >= 2 and 2 <= chunk[b] and chunk[b] * G <= 128]
+    assert cp.head_packed == want_packed
+    for b in range(B):
+        c = chunk[b]
+        if c < 2:
+            assert not [it for it in cp.tile_items if it[0] == b]
+            continue
+        heads = hkv if b in want_packed else hq
+        n_tiles = -(-c // 128)
+        seen = {}
+        for (bb, t, h, s, k0, k1) in cp.tile_items:
+            if bb == b:
+                seen[(t, h, s)] = seen.get((t, h, s), 0) + 1
+                assert 0 <= h < heads and 0 <= t < n_tiles and k0 <= k1
+        assert set(seen.values()) == {1}
+        # each (tile, head) covers the tile's keys [0, K_t) exactly, split by split
+        for t in range(n_tiles):
+            kt = min(prefix[b] + min(c, 128 * (t + 1)), cap)
+            for h in range(heads):
+                spans = sorted((k0, k1) for (bb, tt, hh, s, k0, k1) in cp.tile_items
+                               if bb == b and tt == t and hh == h)
+                assert spans[0][0] == 0 and spans[-1][1] == kt
+                assert all(a[1] == b_[0] for a, b_ in zip(spans, spans[1:]))
