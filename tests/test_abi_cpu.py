@@ -194,3 +194,34 @@ def test_fp8_decode_rejects_bad_arguments_on_host():
     q0, o0 = _fake([0, Hq, D]), _fake([0, Hq, D])
     k0, v0 = _fake([0, Hkv, S, D], fd.FD_E4M3), _fake([0, Hkv, S, D], fd.FD_E4M3)
     assert _decode_fp8(q0, k0, v0, o0) == fd.FD_OK
+
+
+def _paged_fp8(q, kp, vp, ks=1.0, vs=1.0, table=0x400000, pps=4, lens=0x200000, lse=0x300000):
+    tp = ctypes.cast(ctypes.c_void_p(table), ctypes.POINTER(ctypes.c_int32)) if table else None
+    lp = ctypes.cast(ctypes.c_void_p(lens), ctypes.POINTER(ctypes.c_int32)) if lens else None
+    sp = ctypes.cast(ctypes.c_void_p(lse), ctypes.POINTER(ctypes.c_float)) if lse else None
+    out = _fake([q.shape[0], q.shape[1], q.shape[2]])
+    return fd.lib.fd_decode_attention_paged_fp8(ctypes.byref(q), ctypes.byref(kp), ctypes.byref(vp),
+                                                ks, vs, tp, pps, lp, 0, ctypes.byref(out), sp, None)
+
+
+def test_fp8_paged_rejects_bad_arguments_on_host():
+    B, Hq, Hkv, P, D = 2, 16, 2, 16, 128
+    q = _fake([B, Hq, D])
+    kp, vp = _fake([8, Hkv, P, D], fd.FD_E4M3), _fake([8, Hkv, P, D], fd.FD_E4M3)
+    assert _paged_fp8(q, kp, vp, ks=-1.0) == fd.FD_ERR_INVALID_ARGUMENT
+    assert _paged_fp8(q, kp, vp, table=0) == fd.FD_ERR_INVALID_ARGUMENT
+    assert _paged_fp8(q, kp, vp, pps=0) == fd.FD_ERR_INVALID_ARGUMENT
+    # bf16 pages through the FP8 call
+    assert _paged_fp8(q, _fake([8, Hkv, P, D]), _fake([8, Hkv, P, D])) == fd.FD_ERR_INVALID_ARGUMENT
+    # page size 48 is not a divisor or multiple of the 128-key tile
+    k48, v48 = _fake([8, Hkv, 48, D], fd.FD_E4M3), _fake([8, Hkv, 48, D], fd.FD_E4M3)
+    assert _paged_fp8(q, k48, v48) == fd.FD_ERR_UNSUPPORTED
+    # a page stride that is not a multiple of 16 bytes
+    kr = _fake([8, Hkv, P, D], fd.FD_E4M3, strides=[Hkv * P * D + 8, P * D, D, 1])
+    assert _paged_fp8(q, kr, kr) == fd.FD_ERR_UNSUPPORTED
+    # groups above 8 are not served with an FP8 cache
+    q16 = _fake([B, 16, D])
+    k1, v1 = _fake([8, 1, P, D], fd.FD_E4M3), _fake([8, 1, P, D], fd.FD_E4M3)
+    assert _paged_fp8(q16, k1, v1) == fd.FD_ERR_UNSUPPORTED
+    assert "group size" in fd.lib.fd_last_error_message().decode()
