@@ -297,7 +297,8 @@ const char* fd_status_string(fd_status s);
 const char* fd_last_error_message(void);
 
 /* Number of persistent CTAs a decode call with this dtype / group size uses on `device`
- * (the num_ctas its planner uses). Returns 0 on error. */
+ * (the num_ctas its planner uses). dtype is the cache's: FD_E4M3 for the *_fp8 calls. Returns
+ * 0 on error. */
 int32_t fd_decode_num_ctas(int32_t device, int32_t dtype, int32_t group_size, int32_t head_dim);
 
 /* Device workspace bytes a decode call of this shape needs (any cache_lens). */
