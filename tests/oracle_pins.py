@@ -476,6 +476,23 @@ def pin_fp8_paged(att):
     _close(l2, l1, 1e-12, "paged fp8 LSE")
 
 
+
+def pin_fp8_rows_match_full(att):
+    # the row-sampled form (used at full size, one (sequence, KV head) slab dequantized at a
+    # time) equals the full computation at those rows
+    B, Hq, Hkv, S, D = 3, 8, 2, 21, 16
+    q = _rand((B, Hq, D), 70)
+    kc = _fp8_codes((B, Hkv, S, D), 71, hi=0x48)
+    vc = _fp8_codes((B, Hkv, S, D), 72)
+    lens = [21, 0, 9]
+    o, l = att.decode_attention_fp8(q, kc, vc, 0.125, 3.0, lens)
+    rows = [(0, 5), (2, 0), (2, 7), (1, 3)]
+    o2, l2 = att.decode_attention_fp8(q, kc, vc, 0.125, 3.0, lens, rows=rows)
+    for b, h in rows:
+        _close(o2[b, h], o[b, h], 1e-12, f"fp8 row ({b}, {h}) O")
+        _close(l2[b, h], l[b, h], 1e-12, f"fp8 row ({b}, {h}) LSE")
+    assert np.isnan(o2[0, 0]).all(), "rows not asked for stay NaN"
+
 ALL_PINS = [
     pin_golden_decode, pin_golden_chunk, pin_zero_query_is_mean, pin_single_key,
     pin_two_keys_sigmoid, pin_one_hot, pin_equal_scores, pin_empty_and_clamp,
@@ -483,5 +500,5 @@ ALL_PINS = [
     pin_split_invariance, pin_permutation_invariance, pin_page_formulations,
     pin_bf16_widening, pin_paged_equals_contiguous, pin_paged_swapped_pages,
     pin_e4m3_closed_forms, pin_e4m3_torch, pin_fp8_torch_softmax, pin_fp8_scale_laws,
-    pin_fp8_one_hot, pin_fp8_paged,
+    pin_fp8_one_hot, pin_fp8_paged, pin_fp8_rows_match_full,
 ]
