@@ -974,10 +974,10 @@ __global__ void __launch_bounds__(kF8 ? kF8Threads : kTcThreads, 1)
     }
   } else if (warp >= kConvWarp0) {
     if constexpr (kF8) {
-      // ======================= E4M3 -> bf16 expansion =======================
-      // Warps 11-14: per stage, in tile order, K into the stage's tensor-memory tile (thread = key
+      // ================ E4M3 expansion (K to bf16, V to f16) ================
+      // Warps 12-15: per stage, in tile order, K into the stage's tensor-memory tile (thread = key
       // lane of its warp's lane quarter: one code row of 128 bytes -> 64 columns of bf16 pairs).
-      // Warps 15-18: V in place in shared memory. A stage whose valid count is < 0 is the
+      // Warps 16-19: V in place in shared memory. A stage whose valid count is < 0 is the
       // producer's stop marker.
       if (warp < kConvWarp0 + 4) {
         const uint32_t quarter = static_cast<uint32_t>(warp & 3);
