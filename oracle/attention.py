@@ -82,22 +82,29 @@ def attention_rows(q_rows: np.ndarray, keys: np.ndarray, values: np.ndarray,
     """Softmax attention of several query rows over a prefix of one key/value sequence.
 
     q_rows [R, D] float64, keys/values [N, D] float64, n_visible[r] = number of leading keys
-    row r may see. Returns (O [R, D], LSE [R]) in float64. This is the definition written out
-    once per row: scores, max, exponentials, normalised weighted sum, log-sum-exp.
+    row r may see. Returns (O [R, D], LSE [R]) in float64.
+
+    The definition in the matrix form of the ChunkedPrefill page §2.1 (scores = Q·Kᵀ/√d, then a
+    mask, a softmax per row and the product with V): the score matrix of all rows at once, each
+    row keeping its first n_visible[r] scores; then per row the max, the exponentials, the
+    normalised weighted sum of V rows and the log-sum-exp. A row with no visible key keeps
+    O = 0 and LSE = -inf.
     """
     R, D = q_rows.shape
     out = np.zeros((R, D), dtype=np.float64)
     lse = np.full((R,), -np.inf, dtype=np.float64)
-    for r in range(R):
-        n = int(n_visible[r])
-        if n <= 0:
-            continue  # no visible key: O = 0, LSE = -inf
-        s = (keys[:n] @ q_rows[r]) * scale          # s_j = q·k_j * scale
-        m = s.max()                                 # M = max_j s_j
-        e = np.exp(s - m)                           # exp(s_j - M)
-        z = e.sum()                                 # sum_j exp(s_j - M)
-        out[r] = (e @ values[:n]) / z               # sum_j exp(s_j - M) v_j / z
-        lse[r] = m + math.log(z)                    # M + ln z
+    n_vis = np.asarray(n_visible, dtype=np.int64).reshape(R)
+    N = int(n_vis.max()) if R else 0
+    if N <= 0:
+        return out, lse
+    s = (q_rows @ keys[:N].T) * scale                    # s[r, j] = q_r·k_j * scale
+    s[np.arange(N)[None, :] >= n_vis[:, None]] = -np.inf  # keys past row r's limit: excluded
+    has = n_vis > 0
+    m = s[has].max(axis=1)                               # M_r = max_j s[r, j]
+    e = np.exp(s[has] - m[:, None])                      # exp(s_j - M_r); 0 where excluded
+    z = e.sum(axis=1)                                    # sum_j exp(s_j - M_r)
+    out[has] = (e @ values[:N]) / z[:, None]             # sum_j exp(s_j - M_r) v_j / z_r
+    lse[has] = m + np.log(z)                             # M_r + ln z_r
     return out, lse
 
 

@@ -1,14 +1,15 @@
 """Second and third float64 formulations of decode attention, used only to pin the oracle.
 
-TEST INFRASTRUCTURE ONLY (see ``oracle/attention.py``). These follow the pages' own
-algorithms step by step, in float64, so that the plain definition in ``attention.py`` can be
-checked against independently written arithmetic:
+TEST INFRASTRUCTURE ONLY (see ``oracle/attention.py``). These restate the pages' own
+algorithms, in float64 and in code of this project's own, so that the plain definition in
+``attention.py`` can be checked against independently written arithmetic:
 
-* ``online_softmax_row``: the sequential block loop of the ChunkedPrefill page
+* ``online_softmax_row``: the block-wise online softmax of the ChunkedPrefill page
   ("大语言模型长序列推理优化：ChunkedPrefill与FlashDecoding技术解析", §3.1 "分块并行计算原理"):
-  a running maximum, the accumulated output and the running sum are both rescaled by
-  exp(old max - new max) whenever a block raises the maximum; the block's exp(s - new max)
-  weights are then added; the output is divided by the sum at the end.
+  the keys are visited one block at a time and only a running summary is kept (largest
+  score, sum of exponentials, weighted sum of V rows), corrected by exp(old max - new max)
+  when a block raises the maximum, and divided out at the end. Written here as a fold of
+  per-block summaries.
 * ``split_merge_row``: the split-then-merge form of the FlashDecoding page
   ("大模型推理加速FlashDecoding算法原理与多GPU并行解码实战", section
   "FlashDecoding算法原理与标准注意力机制对比" for the per-chunk pass with
@@ -29,31 +30,43 @@ import numpy as np
 __all__ = ["online_softmax_row", "split_merge_row", "merge_partials"]
 
 
+def _fold(a: Tuple[float, float, np.ndarray],
+          b: Tuple[float, float, np.ndarray]) -> Tuple[float, float, np.ndarray]:
+    """Combine two softmax states over disjoint key sets.
+
+    A state (m, l, acc) summarises a set of keys by its largest score m, l = sum exp(s - m) and
+    acc = sum exp(s - m) v. Both states are brought to the common reference max(m_a, m_b) and
+    added; an empty state (l = 0) contributes nothing, whatever its m.
+    """
+    m_a, l_a, acc_a = a
+    m_b, l_b, acc_b = b
+    ref = max(m_a, m_b)
+    c_a = math.exp(m_a - ref) if l_a > 0.0 else 0.0
+    c_b = math.exp(m_b - ref) if l_b > 0.0 else 0.0
+    return ref, c_a * l_a + c_b * l_b, c_a * acc_a + c_b * acc_b
+
+
 def online_softmax_row(q: np.ndarray, keys: np.ndarray, values: np.ndarray, n: int,
                        scale: float, block_size: int) -> Tuple[np.ndarray, float]:
-    """Sequential online softmax over blocks of ``block_size`` keys (float64 inputs)."""
+    """One query row over its first n keys, walked in blocks of ``block_size`` keys.
+
+    Each block is reduced on its own to a state (block max, its sum of exponentials, its
+    exponential-weighted sum of V rows); the running state absorbs it with ``_fold``, which
+    rescales whichever side has the smaller max. After the last block O = acc / l and
+    LSE = m + ln l. Float64 inputs.
+    """
     D = q.shape[0]
-    global_out = np.zeros(D, dtype=np.float64)
-    global_max = -math.inf
-    global_sum = 0.0
-    for start in range(0, n, block_size):
-        stop = min(start + block_size, n)
-        scores = (keys[start:stop] @ q) * scale
-        block_max = scores.max()
-        new_max = max(global_max, block_max)
-        # exp(-inf - finite) = 0 rescales the still-empty accumulators; the page's
-        # exp(global_max - new_max) would be exp(-inf - (-inf)) = NaN only if a block were
-        # empty, which the loop bounds exclude.
-        exp_diff = math.exp(global_max - new_max) if global_max != -math.inf else 0.0
-        global_out *= exp_diff
-        global_sum *= exp_diff
-        exp_scores = np.exp(scores - new_max)
-        global_out += exp_scores @ values[start:stop]
-        global_sum += exp_scores.sum()
-        global_max = new_max
-    if n <= 0:
+    state = (-math.inf, 0.0, np.zeros(D, dtype=np.float64))
+    for lo in range(0, max(n, 0), block_size):
+        hi = min(lo + block_size, n)
+        s = scale * (keys[lo:hi] @ q)
+        m_blk = float(s.max())
+        w = np.exp(s - m_blk)
+        state = _fold(state, (m_blk, float(w.sum()), w @ values[lo:hi]))
+    m, l, acc = state
+    if l == 0.0:
         return np.zeros(D, dtype=np.float64), -math.inf
-    return global_out / global_sum, global_max + math.log(global_sum)
+    return acc / l, m + math.log(l)
 
 
 def split_merge_row(q: np.ndarray, keys: np.ndarray, values: np.ndarray, n: int,

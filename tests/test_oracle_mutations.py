@@ -1,7 +1,8 @@
 """Plant plausible mistakes in a copy of the oracle (on the CPU) and check the pins catch each.
 
 Each mutation rewrites one expression of oracle/attention.py: a dropped term, a wrong sign,
-a wrong index or head mapping, a swapped operand, an off-by-one in the causal limit. The
+a wrong index or head mapping, a swapped operand, an off-by-one in a row's key limit or in
+the causal limit. The
 mutated source is executed as a throw-away module; at least one pin must then fail.
 """
 
@@ -19,16 +20,18 @@ with open(os.path.join(ROOT, "oracle", "attention.py")) as _f:
 
 MUTATIONS = {
     "scale_dropped_sqrt": ("scale = 1.0 / math.sqrt(D)", "scale = 1.0 / D"),
-    "lse_drops_max": ("lse[r] = m + math.log(z)", "lse[r] = math.log(z)"),
-    "lse_wrong_sign": ("lse[r] = m + math.log(z)", "lse[r] = m - math.log(z)"),
-    "no_normalisation": ("out[r] = (e @ values[:n]) / z", "out[r] = (e @ values[:n])"),
-    "exp_wrong_sign": ("e = np.exp(s - m)", "e = np.exp(m - s)"),
-    "k_v_swapped": ("s = (keys[:n] @ q_rows[r]) * scale", "s = (values[:n] @ q_rows[r]) * scale"),
+    "lse_drops_max": ("lse[has] = m + np.log(z)", "lse[has] = np.log(z)"),
+    "lse_wrong_sign": ("lse[has] = m + np.log(z)", "lse[has] = m - np.log(z)"),
+    "no_normalisation": ("out[has] = (e @ values[:N]) / z[:, None]", "out[has] = (e @ values[:N])"),
+    "exp_wrong_sign": ("e = np.exp(s[has] - m[:, None])", "e = np.exp(m[:, None] - s[has])"),
+    "k_v_swapped": ("s = (q_rows @ keys[:N].T) * scale", "s = (q_rows @ values[:N].T) * scale"),
     "gqa_mod_mapping": ("groups.setdefault((int(b), int(h) // G), []).append(int(h))",
                         "groups.setdefault((int(b), int(h) % Hkv), []).append(int(h))"),
     "ignores_cache_len": ("n = _clamp_len(cache_lens[b], S_cap)", "n = S_cap"),
     "len_off_by_one": ("n = _clamp_len(cache_lens[b], S_cap)",
                        "n = _clamp_len(cache_lens[b] - 1, S_cap)"),
+    "row_mask_off_by_one": ("s[np.arange(N)[None, :] >= n_vis[:, None]] = -np.inf",
+                            "s[np.arange(N)[None, :] > n_vis[:, None]] = -np.inf"),
     "causal_off_by_one": ("_clamp_len(int(prefix_lens[b]) + int(row_pos[p]) + 1, S_cap)",
                           "_clamp_len(int(prefix_lens[b]) + int(row_pos[p]), S_cap)"),
     "causal_top_left": ("_clamp_len(int(prefix_lens[b]) + int(row_pos[p]) + 1, S_cap)",
