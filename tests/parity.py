@@ -10,11 +10,16 @@ Tolerances:
   precision than any fp32-accumulating kernel has, so the magnitude used is
   max(|ref|, 2^-8 * max over the row of |ref|). The strict count (magnitude |ref| alone) is
   reported too, as is how many elements needed the floor.
+
+Every comparison prints one ``PARITY`` line with its counts (pytest shows it with ``-rP`` or
+``-s``); with FD_PARITY_LOG set to a file path the same record is appended there as JSON.
 """
 
 from __future__ import annotations
 
+import json
 import math
+import os
 
 import numpy as np
 import torch
@@ -36,6 +41,16 @@ def to_f64(t: torch.Tensor) -> np.ndarray:
     return t.detach().float().cpu().numpy().astype(np.float64)
 
 
+def record(what: str, stats: dict) -> None:
+    """Print one comparison's counts and append them to $FD_PARITY_LOG when it is set."""
+    rec = {"what": what, **stats}
+    print(f"PARITY {json.dumps(rec)}")
+    path = os.environ.get("FD_PARITY_LOG")
+    if path:
+        with open(path, "a") as f:
+            f.write(json.dumps(rec) + "\n")
+
+
 def check_out(gpu: torch.Tensor, ref: np.ndarray, what: str = "out") -> dict:
     """Compare outputs [..., D]. Rows of ref that are NaN (not computed) are skipped."""
     g = to_f64(gpu)
@@ -47,17 +62,20 @@ def check_out(gpu: torch.Tensor, ref: np.ndarray, what: str = "out") -> dict:
     err = np.abs(g - r)
     if gpu.dtype == torch.float32:
         m = float(err.max()) if err.size else 0.0
+        stats = {"dtype": "f32", "max_abs_err": m, "n": int(err.size)}
+        record(what, stats)
         assert m <= F32_TOL, f"{what}: max abs err {m:.3e} > {F32_TOL}"
-        return {"max_abs_err": m, "n": int(err.size)}
+        return stats
     rowmax = np.abs(r).max(axis=-1, keepdims=True)
     mag = np.maximum(np.abs(r), ROW_FLOOR * rowmax)
     tol = bf16_ulp(mag)
     bad = err > tol
     strict_bad = err > bf16_ulp(np.abs(r))
     floor_used = np.abs(r) < ROW_FLOOR * rowmax
-    stats = {"n": int(err.size), "fail": int(bad.sum()), "strict_fail": int(strict_bad.sum()),
-             "floor_used": int(floor_used.sum()),
+    stats = {"dtype": "bf16", "n": int(err.size), "fail": int(bad.sum()),
+             "strict_fail": int(strict_bad.sum()), "floor_used": int(floor_used.sum()),
              "max_err_in_ulps": float((err / np.where(tol > 0, tol, np.inf)).max()) if err.size else 0.0}
+    record(what, stats)
     if bad.any():
         i = np.argwhere(bad)[0]
         raise AssertionError(f"{what}: {stats['fail']} of {stats['n']} elements beyond 1 bf16 ulp; "
@@ -77,29 +95,7 @@ def check_lse(gpu: torch.Tensor, ref: np.ndarray, what: str = "lse") -> dict:
     fin = ~ninf
     assert np.isfinite(g[fin]).all(), f"{what}: non-finite GPU LSE"
     m = float(np.abs(g[fin] - r[fin]).max()) if fin.any() else 0.0
+    stats = {"dtype": "lse", "max_abs_err": m, "n": int(fin.sum()), "neg_inf": int(ninf.sum())}
+    record(what, stats)
     assert m <= LSE_TOL, f"{what}: max abs err {m:.3e} > {LSE_TOL}"
-    return {"max_abs_err": m, "n": int(fin.sum())}
-
-
-def sample_rows(B: int, H: int, n: int, seed: int, must=()):
-    rng = np.random.default_rng(seed)
-    rows = {(int(b), int(h)) for b, h in must}
-    while len(rows) < min(n, B * H):
-        rows.add((int(rng.integers(B)), int(rng.integers(H))))
-    return sorted(rows)
-
-
-def masked_ref(shape_rows, rows, full):
-    """Copy of `full` where only `rows` (pairs) are kept and everything else is NaN."""
-    out = np.full(full.shape, np.nan)
-    for r in rows:
-        out[r] = full[r]
-    return out
-
-
-def assert_finite(t: torch.Tensor, what: str):
-    assert bool(torch.isfinite(t.float()).all()), f"{what}: non-finite values"
-
-
-def nan_fill_value():
-    return math.nan
+    return stats

@@ -12,7 +12,7 @@ import torch
 
 from oracle import attention as oracle
 from oracle import planner as oplan
-from parity import check_lse, check_out, sample_rows
+from parity import check_lse, check_out
 from workloads import make_decode_inputs, to_numpy_exact, workload
 
 pytestmark = pytest.mark.gpu
@@ -115,22 +115,19 @@ def test_full_workload_1_fp32():
     inp = workload(1, pad_fill=NAN)
     out, lse = _run(inp)
     ro, rl = _oracle(inp)
-    check_out(out, ro)
-    check_lse(lse, rl)
+    check_out(out, ro, "workload 1 out")
+    check_lse(lse, rl, "workload 1 lse")
 
 
 @pytest.mark.parametrize("index,batch", [(2, None), (3, None), (4, 1), (4, 2)])
-def test_full_workloads_sampled(index, batch):
+def test_full_workloads(index, batch):
+    # the benchmark shapes at full size, in the launch configuration bench.py times: every
+    # output element against the oracle
     inp = workload(index, batch=batch)
     out, lse = _run(inp, guard=False)
-    assert bool(torch.isfinite(out.float()).all()) and bool(torch.isfinite(lse).all())
-    B, Hq, _ = inp.q.shape
-    lens = inp.cache_lens.tolist()
-    must = [(int(np.argmax(lens)), 0), (int(np.argmin(lens)), Hq - 1)]
-    rows = sample_rows(B, Hq, 48, seed=index, must=must)
-    ro, rl = _oracle(inp, rows=rows)
-    check_out(out, ro)
-    check_lse(lse, rl)
+    ro, rl = _oracle(inp)
+    check_out(out, ro, f"workload {index} (batch {batch or inp.q.shape[0]}) out")
+    check_lse(lse, rl, f"workload {index} (batch {batch or inp.q.shape[0]}) lse")
 
 
 def test_deterministic_and_stream():
@@ -229,10 +226,9 @@ def test_batch_around_in_kernel_plan_limit(B):
     inp = make_decode_inputs(B, 16, 2, 128, 320, lens, torch.bfloat16, seed=900 + B,
                              pad_fill=NAN)
     out, lse = _run(inp)
-    rows = sample_rows(B, 16, 48, seed=B, must=[(0, 0), (B - 1, 15), (B // 2, 7)])
-    ro, rl = _oracle(inp, rows=rows)
-    check_out(out, ro, "out")
-    check_lse(lse, rl, "lse")
+    ro, rl = _oracle(inp)
+    check_out(out, ro, f"B {B} out")
+    check_lse(lse, rl, f"B {B} lse")
 
 
 def test_paths_share_workspace_cursor():

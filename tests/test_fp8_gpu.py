@@ -13,7 +13,7 @@ import pytest
 import torch
 
 from oracle import attention as oracle
-from parity import check_lse, check_out, sample_rows
+from parity import check_lse, check_out
 from workloads import make_decode_inputs, make_fp8, make_paged, to_numpy_exact, workload
 
 pytestmark = pytest.mark.gpu
@@ -194,15 +194,14 @@ def test_fp8_rejections_on_device():
         fd.fd_decode_attention_fp8(q[:, :8], kc, kc, 0.0, 1.0, lens)
 
 
-def test_fp8_workload_3_sampled():
-    # the default decode workload quantized to E4M3, in the bench's launch configuration
+def test_fp8_workload_3():
+    # the default decode workload quantized to E4M3, in the bench's launch configuration: every
+    # output element against the oracle
     inp = workload(3)
     f8 = make_fp8(inp.k_cache, inp.v_cache)
     del inp.k_cache, inp.v_cache
     out, lse = _run(inp.q, f8.k_codes, f8.v_codes, f8.k_scale, f8.v_scale, inp.cache_lens)
-    rows = sample_rows(32, 64, 24, seed=9, must=[(0, 0), (31, 63)])
-    ro, rl = _oracle(inp.q, f8.k_codes, f8.v_codes, f8.k_scale, f8.v_scale, inp.cache_lens,
-                     rows=rows)
+    ro, rl = _oracle(inp.q, f8.k_codes, f8.v_codes, f8.k_scale, f8.v_scale, inp.cache_lens)
     check_out(out, ro, "fp8 w3 out")
     check_lse(lse, rl, "fp8 w3 lse")
 
@@ -215,9 +214,7 @@ def test_fp8_planner_kernel_batch():
     inp = make_decode_inputs(B, 16, 2, 128, 400, lens, torch.bfloat16, seed=661, pad_fill=NAN)
     f8 = make_fp8(inp.k_cache, inp.v_cache)
     out, lse = _run(inp.q, f8.k_codes, f8.v_codes, f8.k_scale, f8.v_scale, inp.cache_lens)
-    rows = sample_rows(B, 16, 48, seed=5, must=[(0, 0), (B - 1, 15), (B // 2, 7)])
-    ro, rl = _oracle(inp.q, f8.k_codes, f8.v_codes, f8.k_scale, f8.v_scale, inp.cache_lens,
-                     rows=rows)
+    ro, rl = _oracle(inp.q, f8.k_codes, f8.v_codes, f8.k_scale, f8.v_scale, inp.cache_lens)
     check_out(out, ro, "fp8 B 300 out")
     check_lse(lse, rl, "fp8 B 300 lse")
 

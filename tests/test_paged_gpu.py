@@ -12,7 +12,7 @@ import torch
 
 from oracle import attention as oracle
 from oracle import planner as oplan
-from parity import check_lse, check_out, sample_rows
+from parity import check_lse, check_out
 from workloads import make_decode_inputs, make_paged, to_numpy_exact, workload
 
 pytestmark = pytest.mark.gpu
@@ -82,8 +82,7 @@ def test_paged_planner_kernel_batch():
     inp = make_decode_inputs(B, 16, 2, 128, 400, lens, torch.bfloat16, seed=78, pad_fill=NAN)
     pg = make_paged(inp.k_cache, inp.v_cache, lens, 16, seed=79)
     out, lse = _run_paged(inp, pg)
-    rows = sample_rows(B, 16, 48, seed=3, must=[(0, 0), (B - 1, 15)])
-    ro, rl = _oracle(inp, rows=rows)
+    ro, rl = _oracle(inp)
     check_out(out, ro, "paged out")
     check_lse(lse, rl, "paged lse")
 
@@ -161,12 +160,11 @@ def test_paged_rejects_bad_layouts():
         fd.fd_decode_attention_paged(q, kp, kp, table, lens)
 
 
-def test_paged_workload_3_sampled():
-    # the default workload's keys in 128-key pages at shuffled positions
+def test_paged_workload_3():
+    # the default workload's keys in 128-key pages at shuffled positions: every output element
     inp = workload(3)
     pg = make_paged(inp.k_cache, inp.v_cache, inp.cache_lens.tolist(), 128, seed=1303)
     out, lse = _run_paged(inp, pg)
-    rows = sample_rows(32, 64, 24, seed=7, must=[(0, 0), (31, 63)])
-    ro, rl = _oracle(inp, rows=rows)
+    ro, rl = _oracle(inp)
     check_out(out, ro, "paged w3 out")
     check_lse(lse, rl, "paged w3 lse")
