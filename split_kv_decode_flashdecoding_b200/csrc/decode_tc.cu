@@ -79,9 +79,9 @@ struct __align__(1024) TcSmem {
   int32_t meta[kStages][2];                      // per stage: tile start, valid keys (MMA warp)
   int32_t vmeta[kStages];                        // E4M3: valid keys of the stage's V tile
   // in-kernel plan: lengths, split counts, rank order, partial-slot bases (row order) and item
-  // offsets (rank order, B + 1 entries)
+  // offsets (rank order); both scans also store their total after the last entry (B + 1)
   int32_t plan_len[kFusedPlanMaxBatch], plan_n[kFusedPlanMaxBatch];
-  int32_t plan_order[kFusedPlanMaxBatch], plan_rbase[kFusedPlanMaxBatch];
+  int32_t plan_order[kFusedPlanMaxBatch], plan_rbase[kFusedPlanMaxBatch + 1];
   int32_t plan_ioff[kFusedPlanMaxBatch + 1];
   long long plan_red[kF8Threads / 32];
   int32_t plan_clamped;
@@ -272,7 +272,7 @@ static_assert(sizeof(TcSmem<16>) + 1024 <= 227 * 1024, "tensor-core decode smem 
 static_assert(sizeof(TcSmem<8, true>) + 1024 <= 227 * 1024, "tensor-core decode smem (E4M3)");
 
 // Exclusive prefix sum over i < n (n <= 32 * 8 here) by one warp: out[i] = sum_{j<i} val(j),
-// out[n] = the total.
+// out[n] = the total (out holds n + 1 entries).
 template <typename F>
 __device__ __forceinline__ void warp_exclusive_scan(int n, F val, int32_t* out) {
   const int lane = threadIdx.x & 31;

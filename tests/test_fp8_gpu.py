@@ -206,17 +206,18 @@ def test_fp8_workload_3():
     check_lse(lse, rl, "fp8 w3 lse")
 
 
-def test_fp8_planner_kernel_batch():
-    # above 256 sequences the planner kernel plans the call instead of the split kernel itself
+@pytest.mark.parametrize("B", [256, 300])
+def test_fp8_planner_kernel_batch(B):
+    # 256 sequences: the largest batch the split kernel plans itself; above 256 the planner
+    # kernel plans the call instead
     rng = np.random.default_rng(660)
-    B = 300
     lens = [int(x) for x in rng.integers(0, 400, size=B)]
     inp = make_decode_inputs(B, 16, 2, 128, 400, lens, torch.bfloat16, seed=661, pad_fill=NAN)
     f8 = make_fp8(inp.k_cache, inp.v_cache)
     out, lse = _run(inp.q, f8.k_codes, f8.v_codes, f8.k_scale, f8.v_scale, inp.cache_lens)
     ro, rl = _oracle(inp.q, f8.k_codes, f8.v_codes, f8.k_scale, f8.v_scale, inp.cache_lens)
-    check_out(out, ro, "fp8 B 300 out")
-    check_lse(lse, rl, "fp8 B 300 lse")
+    check_out(out, ro, f"fp8 B {B} out")
+    check_lse(lse, rl, f"fp8 B {B} lse")
 
 
 def test_fp8_cuda_graph_replay_new_lengths():

@@ -74,17 +74,18 @@ def test_paged_small(case, num_splits):
     assert _fd().fd_poll_status() == 0
 
 
-def test_paged_planner_kernel_batch():
-    # above 256 sequences the planner kernel plans the call; aligned splits there too
+@pytest.mark.parametrize("B", [256, 300])
+def test_paged_planner_kernel_batch(B):
+    # 256 sequences: the largest batch the split kernel plans itself; above, the planner kernel
+    # plans the call; aligned splits in both
     rng = np.random.default_rng(77)
-    B = 300
     lens = [int(x) for x in rng.integers(0, 400, size=B)]
     inp = make_decode_inputs(B, 16, 2, 128, 400, lens, torch.bfloat16, seed=78, pad_fill=NAN)
     pg = make_paged(inp.k_cache, inp.v_cache, lens, 16, seed=79)
     out, lse = _run_paged(inp, pg)
     ro, rl = _oracle(inp)
-    check_out(out, ro, "paged out")
-    check_lse(lse, rl, "paged lse")
+    check_out(out, ro, f"paged B {B} out")
+    check_lse(lse, rl, f"paged B {B} lse")
 
 
 def test_paged_device_plan_is_aligned_oracle_plan():
