@@ -9,18 +9,22 @@
 //
 //   S[128 rows x 128 keys] = Q_tile · K_tileᵀ         UMMA M=128 N=128, both K-major (TMA SW128)
 //   one thread per row: mask, running max m (rescaled lazily), p = 2^(s·scale·log2e − m),
-//   running sum l, P split into bf16 hi + lo (truncated top bits and remainder) and stored
-//   into tensor memory
-//   O[128 x 128] += P_hi · V_tile + P_lo · V_tile      UMMA M=128 N=128, A from TMEM, V MN-major
+//   running sum l, P split into bf16 hi + lo (both rounded to nearest) and stored into tensor
+//   memory
+//   O_hi[128 x 128] += P_hi · V_tile, O_lo[128 x 128] += P_lo · V_tile
+//                                                        UMMA M=128 N=128, A from TMEM, V MN-major
 //
 // S is double-buffered in TMEM and P is written back over the S buffer it came from (per
-// 32-key chunk: 16 words of hi pairs, then 16 words of lo pairs), so P is double-buffered too; O
-// has one accumulator per item parity, so an item's epilogue overlaps the next item's tiles. The
-// reference maximum m moves only when a row's maximum grows by more than 2^8, so O is rescaled
-// rarely — only then does the softmax wait for the previous P·V product; p <= 2^8 is exact enough
-// in fp32 and in the hi/lo split. At the end of the split the epilogue writes O / l and
-// LSE = m + log2 l: the final output when the tile has a single split, else a partial for the
-// combine kernel.
+// 32-key chunk: 16 words of hi pairs, then 16 words of lo pairs), so P is double-buffered too.
+// The hi and lo products accumulate in two accumulators that the epilogue adds: the tensor
+// core's fp32 accumulation truncates, and the tiny lo terms added into the hi accumulator would
+// double the truncations the output carries. The two accumulators fill the rest of tensor
+// memory, so an item's first P·V product waits until the epilogue has read the previous item's
+// (the softmax of the new item runs meanwhile). The reference maximum m moves only when a row's
+// maximum grows by more than 2^8, so O is rescaled rarely — only then does the softmax wait for
+// the previous P·V product; p <= 2^8 is exact enough in fp32 and in the hi/lo split. At the end of
+// the split the epilogue writes O / l and LSE = m + log2 l: the final output when the tile has a
+// single split, else a partial for the combine kernel.
 //
 // Head-packed tiles (a request of 2 <= c <= 128 / G rows, G >= 2: a multi-token verification
 // step, "大模型推理加速FlashDecoding算法原理与多GPU并行解码实战", "与其他推理加速方案的组合使用",
@@ -53,7 +57,9 @@ constexpr int kCkVProducer = 10;
 constexpr int kCkPv = 11;          // issues the P·V products (warp 5 the S products)
 constexpr int kCkThreads = 12 * 32;
 constexpr uint32_t kCkTmemCols = 512;
-constexpr uint32_t kColS0 = 0, kColO0 = 256;   // S/P buffers at 0 and 128, O at 256 and 384
+constexpr uint32_t kColS0 = 0;     // S/P buffers at columns 0 and 128
+constexpr uint32_t kColOHi = 256;  // O accumulator of the P_hi products
+constexpr uint32_t kColOLo = 384;  // O accumulator of the P_lo products
 constexpr uint32_t kCkHalf = kCkRows * 64 * 2;  // one 64-column half of a 128-row tile
 constexpr float kRescaleThreshold = 8.0f;       // log2 units
 
@@ -75,7 +81,8 @@ struct __align__(1024) CkSmem {
   // tile J + 2, whose S needs P·V(J), which needs the whole phase of tile J
   uint64_t pfull[2];
   uint64_t pfree;      // every P·V product (the softmax waits for the previous one to rescale O)
-  uint64_t ofin[2], oempty[2], lready[2], lfree[2];  // by item parity
+  uint64_t ofin, oempty;            // per item: its last P·V product done / its O read
+  uint64_t lready[2], lfree[2];      // by item parity
   uint64_t drain, drain_pv;
   uint32_t tmem_base;
   int abort_flag;
@@ -113,12 +120,12 @@ __global__ void __launch_bounds__(kCkThreads, 1)
       mbar_init(&S.sfull[i], 1);
       mbar_init(&S.sfree[i], 1);
       mbar_init(&S.pfull[i], 4);
-      mbar_init(&S.ofin[i], 1);
-      mbar_init(&S.oempty[i], 4);
       mbar_init(&S.lready[i], 4);
       mbar_init(&S.lfree[i], 4);
     }
     mbar_init(&S.pfree, 1);
+    mbar_init(&S.ofin, 1);
+    mbar_init(&S.oempty, 4);
     mbar_init(&S.drain, 1);
     mbar_init(&S.drain_pv, 1);
     S.abort_flag = 0;
@@ -308,32 +315,29 @@ __global__ void __launch_bounds__(kCkThreads, 1)
         const TileItem it = S.item[ps];
         mbar_arrive(&S.qempty[ps]);
         if (idx < 0) break;
-        const int ob = K & 1;
         for (int j = 0; j < ntile; ++j, ++J) {
           const int vs = J % kCkVStages;
           const int valid = max(0, min(kCkKeys, it.k1 - (it.k0 + j * kCkKeys)));
           if (!mbar_wait(&S.vfull[vs], (J / kCkVStages) & 1u, ctx)) { ok = false; break; }
           if (!mbar_wait(&S.pfull[J & 1], (J >> 1) & 1u, ctx)) { ok = false; break; }
-          // the item's first product overwrites the accumulator the item two back used
-          if (j == 0 && !mbar_wait(&S.oempty[ob], ((K >> 1) & 1u) ^ 1u, ctx)) { ok = false; break; }
+          // the item's first products overwrite the accumulators the previous item used
+          if (j == 0 && !mbar_wait(&S.oempty, (K & 1u) ^ 1u, ctx)) { ok = false; break; }
           tc_fence_after();
           const int nk = (valid + 15) / 16;
           const uint32_t vaddr = smem_u32(S.v[vs][0]);
           const uint32_t pcol = kColS0 + (J & 1) * 128;  // P of this tile, over its S buffer
-          const uint32_t ocol = kColO0 + ob * 128;
-          bool acc = j > 0;
           for (int part = 0; part < 2; ++part) {
+            const uint32_t ocol = part ? kColOLo : kColOHi;
             for (int kk = 0; kk < nk; ++kk) {
               const uint64_t bd = smem_desc(vaddr + kk * 2048, kCkHalf, 1024, kLayoutSW128);
               const uint32_t acol = pcol + 32 * (kk >> 1) + 16 * part + 8 * (kk & 1);
-              umma_bf16_ts(tmem + ocol, tmem + acol, bd, idesc_o, acc ? 1u : 0u);
-              acc = true;
+              umma_bf16_ts(tmem + ocol, tmem + acol, bd, idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
             }
           }
           umma_commit(&S.pfree);
           umma_commit(&S.sfree[J & 1]);
           umma_commit(&S.vempty[vs]);
-          if (j == ntile - 1) umma_commit(&S.ofin[ob]);
+          if (j == ntile - 1) umma_commit(&S.ofin);
         }
         if (!ok) break;
         ++K;
@@ -426,9 +430,9 @@ __global__ void __launch_bounds__(kCkThreads, 1)
           // O changes only after the previous product has added into it
           if (!mbar_wait(&S.pfree, (J - 1) & 1u, ctx)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t oc = tmem + lane_base + kColO0 + ob * 128;
+          const uint32_t oc = tmem + lane_base + kColOHi;  // O_hi, then O_lo right after it
 #pragma unroll 1
-          for (int c = 0; c < kCkD; c += 32) {
+          for (int c = 0; c < 2 * kCkD; c += 32) {
             uint32_t o[32];
             tmem_ld32(oc + c, o);
             tmem_wait_ld();
@@ -438,11 +442,10 @@ __global__ void __launch_bounds__(kCkThreads, 1)
           }
         }
         // pass 2, 64 keys at a time: p = 2^(s·scale − m), split into bf16 hi + lo and written over
-        // the tile's own S columns (a 32-key chunk's words cover only columns already read). hi
-        // keeps the top 16 bits of p (bf16 truncation) and lo the exact fp32 remainder, truncated
-        // the same way, so p − hi − lo < 2^-15 p; both packings are byte permutes, which leaves
-        // the exponential pipe to the exponentials. mref = −inf only when no key is visible, and
-        // then every x below is −inf already.
+        // the tile's own S columns (a 32-key chunk's words cover only columns already read). hi is
+        // p rounded to the nearest bf16 and lo the exact fp32 remainder p − hi, rounded the same
+        // way, so |p − hi − lo| <= 2^-17 p, without bias. mref = −inf only when no key is visible,
+        // and then every x below is −inf already.
         const float negm = mref == -INFINITY ? 0.f : -mref;
         float rsum[4];  // four independent partial sums of p
 #pragma unroll
@@ -469,11 +472,10 @@ __global__ void __launch_bounds__(kCkThreads, 1)
               }
               const float p0 = fast_exp2(x0), p1 = fast_exp2(x1);
               rsum[(i >> 1) & 3] += p0 + p1;
-              const uint32_t b0 = __float_as_uint(p0), b1 = __float_as_uint(p1);
-              w[i / 2] = __byte_perm(b0, b1, 0x7632);
-              const float l0 = p0 - __uint_as_float(b0 & 0xffff0000u);
-              const float l1 = p1 - __uint_as_float(b1 & 0xffff0000u);
-              w[16 + i / 2] = __byte_perm(__float_as_uint(l0), __float_as_uint(l1), 0x7632);
+              const __nv_bfloat162 hi = __floats2bfloat162_rn(p0, p1);
+              const float2 hf = __bfloat1622float2(hi);
+              w[i / 2] = *reinterpret_cast<const uint32_t*>(&hi);
+              w[16 + i / 2] = pack_bf16x2(p0 - hf.x, p1 - hf.y);
             }
             tmem_st32(sp + h + c, w);
           }
@@ -520,7 +522,7 @@ __global__ void __launch_bounds__(kCkThreads, 1)
       const float l = S.lfin[ob][r];
       __syncwarp();
       if (lane == 0) mbar_arrive(&S.lfree[ob]);
-      if (!mbar_wait(&S.ofin[ob], (K >> 1) & 1u, ctx)) break;
+      if (!mbar_wait(&S.ofin, K & 1u, ctx)) break;
       tc_fence_after();
       const int pos = it.head_packed ? (r * p.g_recip16) >> 16 : r;  // chunk position of the row
       const bool row_ok = pos < it.rows;
@@ -537,15 +539,16 @@ __global__ void __launch_bounds__(kCkThreads, 1)
       __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out) + row * p.o_sr +
                            static_cast<int64_t>(head) * p.o_sh;
       float* dst = p.part_o + (slot * p.g + g) * kCkD;
+      // O = O_hi + O_lo, 32 columns at a time
 #pragma unroll 1
       for (int c = 0; c < kCkD; c += 32) {
-        uint32_t o[32];
-        tmem_ld32(tmem + lane_base + kColO0 + ob * 128 + c, o);
+        uint32_t o[32], lo[32];
+        tmem_ld32(tmem + lane_base + kColOHi + c, o);
+        tmem_ld32(tmem + lane_base + kColOLo + c, lo);
         tmem_wait_ld();
-        if (!seen) {
 #pragma unroll
-          for (int i = 0; i < 32; ++i) o[i] = 0u;
-        }
+        for (int i = 0; i < 32; ++i)
+          o[i] = seen ? __float_as_uint(__uint_as_float(o[i]) + __uint_as_float(lo[i])) : 0u;
         if (row_ok) {
           if (direct) {
 #pragma unroll
@@ -568,7 +571,7 @@ __global__ void __launch_bounds__(kCkThreads, 1)
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&S.oempty[ob]);
+      if (lane == 0) mbar_arrive(&S.oempty);  // both accumulators read: the next item may start
       if (row_ok) {
         if (direct) p.lse[row * p.hq + head] = lse2 * kLn2;
         else p.part_lse[slot * p.g + g] = lse2;
