@@ -277,13 +277,17 @@ fd_status fd_chunk_prefill_attention(const fd_tensor* q_chunk, const fd_tensor* 
  * allocates nothing; the caller still passes every input and output.
  *  - Every GPU that loads the library holds that array until the process exits.
  *  - The first call on a device looks up the array's device address (cudaGetSymbolAddress) with
- *    that device current; make that first call before any stream capture begins.
+ *    that device current; make that first call before any stream capture begins. The lookup is
+ *    repeated when the device's context has changed (after a device reset), so after a reset the
+ *    first call must again come before any capture.
  *  - All calls share the array and it keeps the last call's contents: calls that overlap on the GPU
  *    (different streams, or host threads without ordering between their calls) race on it and give
- *    wrong results. Each call clears, on its stream, the header that must start at zero.
+ *    wrong results. Each call clears, on its stream, the header fields that must start at zero
+ *    (work cursors), and keeps the status word.
  *  - A shape whose worst-case scratch (fd_decode_workspace_bytes) exceeds FD_STATIC_SCRATCH_BYTES
  *    returns FD_ERR_UNSUPPORTED before anything is enqueued.
- *  - Device status flags of these kernels are not reported by fd_poll_status.
+ *  - Device status flags these calls raise (FD_FLAG_*) collect in the array's status word until
+ *    fd_poll_status, called on the stream the calls used, returns and clears them.
  */
 fd_status fd_decode_attention_static(const fd_tensor* q, const fd_tensor* k_cache,
                                      const fd_tensor* v_cache, const int32_t* cache_lens,
@@ -316,7 +320,8 @@ size_t fd_chunk_workspace_bytes(int32_t batch, int32_t total_rows, int32_t num_q
 fd_status fd_reserve_workspace(size_t bytes, void* stream);
 
 /* Synchronise `stream`, return the device status word bits (FD_FLAG_*) raised since the last
- * poll on that stream's workspace, and clear them. */
+ * poll on that stream's workspace, together with those raised by fd_decode_attention_static calls
+ * on the current device since the last poll, and clear them. */
 fd_status fd_poll_status(void* stream, uint32_t* flags);
 
 /* Kernel timing for measurement. fd_profile_begin(n) makes the next n attention calls record a

@@ -45,11 +45,26 @@ fd_status resolve_paged(const fd_tensor* q, const fd_tensor* k, const fd_tensor*
                         PagedCache& pg, const fd_tensor* out, DecodeShape* sh,
                         const KvQuant* quant = nullptr);
 
+// Scratch memory a decode call uses instead of the library's per-stream workspace: `base` (256-byte
+// aligned device memory of `bytes` bytes) holds the same layout. A shape whose worst-case
+// scratch exceeds `bytes` is rejected with FD_ERR_UNSUPPORTED before anything is enqueued. The
+// call clears the header's cursors on its stream first and keeps its status word.
+struct PresetScratch {
+  void* base;
+  size_t bytes;
+  const char* name;  // for the error message
+};
+
 // The decode call of fd_decode_attention (pg == nullptr) and fd_decode_attention_paged, and of
-// their FP8 forms (quant != nullptr).
+// their FP8 forms (quant != nullptr); with `preset`, in that scratch.
 fd_status decode_call(const fd_tensor* q, const fd_tensor* k_cache, const fd_tensor* v_cache,
                       const int32_t* cache_lens, int32_t num_splits, fd_tensor* out, float* lse,
-                      cudaStream_t stream, PagedCache* pg, const KvQuant* quant = nullptr);
+                      cudaStream_t stream, PagedCache* pg, const KvQuant* quant = nullptr,
+                      const PresetScratch* preset = nullptr);
+
+// The status word of the allocation-free entry point's scratch on the current device, read and
+// cleared (0 when that scratch has not been set up on the device). The caller synchronises.
+fd_status static_scratch_take_status(uint32_t* flags);
 
 // Persistent CTAs of the split kernel on device `dev`.
 int decode_ctas(int dev, bool use_tc);

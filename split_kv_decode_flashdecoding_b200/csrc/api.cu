@@ -5,6 +5,7 @@
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
+#include <cstddef>
 #include <cstring>
 #include <map>
 #include <mutex>
@@ -487,7 +488,8 @@ namespace fd_abi {
 // The decode call of both entry points: a contiguous cache (pg == nullptr) or a paged one.
 fd_status decode_call(const fd_tensor* q, const fd_tensor* k_cache, const fd_tensor* v_cache,
                       const int32_t* cache_lens, int32_t num_splits, fd_tensor* out, float* lse,
-                      cudaStream_t stream, PagedCache* pg, const KvQuant* quant) {
+                      cudaStream_t stream, PagedCache* pg, const KvQuant* quant,
+                      const PresetScratch* preset) {
   DecodeShape sh{};
   fd_status s = pg ? resolve_paged(q, k_cache, v_cache, *pg, out, &sh, quant)
                    : resolve_decode(q, k_cache, v_cache, out, &sh, quant);
@@ -506,7 +508,16 @@ fd_status decode_call(const fd_tensor* q, const fd_tensor* k_cache, const fd_ten
   const int64_t max_slots = max_items;  // one partial slot (G heads) per split item
   const WsLayout L = ws_layout(max_items, 0, sh.B, max_slots, sh.hq, sh.d, sh.hkv);
   void* ws = nullptr;
-  if ((s = get_workspace(stream, L.total, &ws)) != FD_OK) return s;
+  if (preset) {
+    if (L.total > preset->bytes)
+      return fail(FD_ERR_UNSUPPORTED,
+                  "this decode shape needs up to %zu bytes of scratch, more than the %zu bytes of "
+                  "the %s; use fd_decode_attention",
+                  L.total, preset->bytes, preset->name);
+    ws = preset->base;
+  } else if ((s = get_workspace(stream, L.total, &ws)) != FD_OK) {
+    return s;
+  }
   char* base = static_cast<char*>(ws);
   WsHeader* hdr = reinterpret_cast<WsHeader*>(base);
   DecodeItem* items = reinterpret_cast<DecodeItem*>(base + L.dec_items);
@@ -622,6 +633,14 @@ fd_status decode_call(const fd_tensor* q, const fd_tensor* k_cache, const fd_ten
     dp.max_items = static_cast<int32_t>(std::min<int64_t>(max_items, INT32_MAX));
     dp.row_nsplit_out = row_nsplit;
     dp.row_base_out = row_base;
+  }
+
+  if (preset) {
+    // scratch shared with other calls: the cursors must start at zero whatever the last call
+    // left; the status word (offset 0) is kept until it is polled
+    static_assert(offsetof(WsHeader, status) == 0, "status word first");
+    FD_CUDA(cudaMemsetAsync(base + sizeof(uint32_t), 0, sizeof(WsHeader) - sizeof(uint32_t), stream),
+            "clear scratch header");
   }
 
   cudaEvent_t* ev = prof_next();
@@ -890,12 +909,17 @@ fd_status fd_poll_status(void* stream_, uint32_t* flags) {
     auto it = g_ws.find({dev, reinterpret_cast<uintptr_t>(stream)});
     if (it != g_ws.end()) ptr = it->second.ptr;
   }
-  if (!ptr) return FD_OK;
   uint32_t v = 0;
-  FD_CUDA(cudaMemcpy(&v, ptr, sizeof(v), cudaMemcpyDeviceToHost), "read status");
-  const uint32_t zero = 0;
-  FD_CUDA(cudaMemcpy(ptr, &zero, sizeof(zero), cudaMemcpyHostToDevice), "clear status");
-  *flags = v;
+  if (ptr) {
+    FD_CUDA(cudaMemcpy(&v, ptr, sizeof(v), cudaMemcpyDeviceToHost), "read status");
+    const uint32_t zero = 0;
+    FD_CUDA(cudaMemcpy(ptr, &zero, sizeof(zero), cudaMemcpyHostToDevice), "clear status");
+  }
+  // the status bits of fd_decode_attention_static calls on this device
+  uint32_t st = 0;
+  fd_status s = static_scratch_take_status(&st);
+  if (s != FD_OK) return s;
+  *flags = v | st;
   return FD_OK;
 }
 

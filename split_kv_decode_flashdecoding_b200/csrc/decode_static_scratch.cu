@@ -1,8 +1,9 @@
 // fd_decode_attention_static: the decode attention call for callers that cannot allocate device
-// memory. It runs the same planner, split and combine kernels as fd_decode_attention, but its
-// scratch (the split plan, the work items and the per-split partial results) lives in one
-// file-scope device array of FD_STATIC_SCRATCH_BYTES instead of the library's per-stream
-// workspace, so the call itself never allocates.
+// memory. It is fd_decode_attention itself (the same argument checks, split plan, kernels and
+// launch sequence, in fd_abi::decode_call), except that its scratch (the split plan, the work
+// items and the per-split partial results) lives in one file-scope device array of
+// FD_STATIC_SCRATCH_BYTES instead of the library's per-stream workspace, so the call itself never
+// allocates.
 //
 // Who needs this: serving engines that hand nearly all of a GPU's memory to their own KV-cache
 // pool (a late cudaMalloc would fail or fragment that pool), plugin hosts that only let a plugin
@@ -12,15 +13,17 @@
 // Rules for callers (also stated in include/fd.h):
 //  - Every GPU that loads this library holds the array until the process exits.
 //  - The first call on a device looks up the array's device address with cudaGetSymbolAddress,
-//    with that device current; make that first call before any stream capture begins.
+//    with that device current; make that first call before any stream capture begins. The
+//    lookup is repeated when the device's current context changes (after a device reset).
 //  - All calls share the one array, which keeps the previous call's contents: calls that overlap
 //    on the GPU (other streams, or other host threads without ordering between them) race on it.
-//    Each call clears the header it needs zeroed (status word and work cursor) on its stream.
+//    Each call clears, on its stream, the header fields that must start at zero.
 //  - A shape whose worst-case scratch exceeds FD_STATIC_SCRATCH_BYTES is rejected on the host with
 //    FD_ERR_UNSUPPORTED before anything is enqueued.
-//  - Device status flags raised by these kernels land in the array's header, which the next call
-//    clears; fd_poll_status does not report them.
-#include <cmath>
+//  - Device status flags raised by these kernels stay in the array's header until fd_poll_status
+//    reads and clears them.
+#include <cuda.h>
+
 #include <map>
 #include <mutex>
 
@@ -37,152 +40,110 @@ namespace {
 // address comes from cudaGetSymbolAddress below.
 static __device__ __align__(256) unsigned char g_fd_static_scratch[FD_STATIC_SCRATCH_BYTES];
 
+struct StaticAddr {
+  void* ptr;
+  CUcontext ctx;  // the context the address belongs to
+};
 std::mutex g_static_mu;
-std::map<int, void*> g_static_addr;  // device ordinal -> device address of g_fd_static_scratch
+std::map<int, StaticAddr> g_static_addr;  // device ordinal -> device address of the array
 
-// Device address of the scratch on device `dev` (the current device), looked up once.
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+
+// The driver's cuCtxGetCurrent (the runtime is linked statically; the driver entry point is
+// fetched at run time, like cuTensorMapEncodeTiled).
+CtxGetCurrentFn ctx_get_current_fn() {
+  static std::once_flag once;
+  static CtxGetCurrentFn fn = nullptr;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuCtxGetCurrent", &f, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<CtxGetCurrentFn>(f);
+  });
+  return fn;
+}
+
+// The context current on the calling thread (nullptr when it cannot be read).
+CUcontext current_context() {
+  CtxGetCurrentFn fn = ctx_get_current_fn();
+  CUcontext c = nullptr;
+  if (!fn || fn(&c) != CUDA_SUCCESS) return nullptr;
+  return c;
+}
+
+// True when `ctx` (the calling thread's current context, or nullptr if none is bound yet) may be
+// the context an address was taken in: only two known contexts that differ rule it out.
+bool same_context(CUcontext stored, CUcontext ctx) {
+  return stored == nullptr || ctx == nullptr || stored == ctx;
+}
+
+// Device address of the array on device `dev` (the current device): looked up once per device,
+// and again when the device's context is no longer the one the address was taken in (a device
+// reset destroys that context).
 fd_status static_scratch_address(int dev, void** out) {
+  const CUcontext ctx = current_context();
   std::lock_guard<std::mutex> lock(g_static_mu);
   auto it = g_static_addr.find(dev);
-  if (it != g_static_addr.end()) {
-    *out = it->second;
+  if (it != g_static_addr.end() && same_context(it->second.ctx, ctx)) {
+    *out = it->second.ptr;
     return FD_OK;
   }
   void* ptr = nullptr;
   cudaError_t e = cudaGetSymbolAddress(&ptr, g_fd_static_scratch);
   if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(static scratch)");
   if (!ptr) return fail(FD_ERR_CUDA, "cudaGetSymbolAddress returned a null static scratch address");
-  g_static_addr[dev] = ptr;
+  // the runtime call above has made the device's primary context current on this thread
+  g_static_addr[dev] = StaticAddr{ptr, current_context()};
   *out = ptr;
   return FD_OK;
 }
 
 }  // namespace
 
+namespace fd_abi {
+
+fd_status static_scratch_take_status(uint32_t* flags) {
+  *flags = 0;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  void* ptr = nullptr;
+  {
+    std::lock_guard<std::mutex> lock(g_static_mu);
+    auto it = g_static_addr.find(dev);
+    if (it == g_static_addr.end() || !same_context(it->second.ctx, current_context())) return FD_OK;
+    ptr = it->second.ptr;
+  }
+  uint32_t v = 0;
+  e = cudaMemcpy(&v, ptr, sizeof(v), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(e, "read static scratch status");
+  const uint32_t zero = 0;
+  e = cudaMemcpy(ptr, &zero, sizeof(zero), cudaMemcpyHostToDevice);
+  if (e != cudaSuccess) return cuda_fail(e, "clear static scratch status");
+  *flags = v;
+  return FD_OK;
+}
+
+}  // namespace fd_abi
+
 extern "C" fd_status fd_decode_attention_static(const fd_tensor* q, const fd_tensor* k_cache,
                                                 const fd_tensor* v_cache,
                                                 const int32_t* cache_lens, int32_t num_splits,
-                                                fd_tensor* out, float* lse, void* stream_) {
-  cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+                                                fd_tensor* out, float* lse, void* stream) {
+  // shapes that are rejected or need no launch never touch the array
   DecodeShape sh{};
   fd_status s = resolve_decode(q, k_cache, v_cache, out, &sh);
   if (s != FD_OK) return s;
-  if (num_splits < 0) return fail(FD_ERR_INVALID_ARGUMENT, "num_splits must be >= 0");
-  if (num_splits > 65536) return fail(FD_ERR_UNSUPPORTED, "num_splits above 65536");
-  if (sh.B == 0) return FD_OK;
-  if (!cache_lens) return fail(FD_ERR_INVALID_ARGUMENT, "cache_lens is NULL");
-  if (!lse) return fail(FD_ERR_INVALID_ARGUMENT, "lse is NULL");
-  int dev = 0;
-  cudaError_t ce = cudaGetDevice(&dev);
-  if (ce != cudaSuccess) return cuda_fail(ce, "cudaGetDevice");
-  const int nctas = decode_ctas(dev, sh.use_tc);
-  if (nctas < 1) return fail(FD_ERR_CUDA, "no multiprocessors reported for device %d", dev);
-
-  const int64_t max_items = decode_max_items(sh.B, sh.hkv, sh.cap, num_splits, nctas);
-  const int64_t max_slots = max_items;  // one partial slot (G heads) per split item
-  const WsLayout L = ws_layout(max_items, 0, sh.B, max_slots, sh.hq, sh.d, sh.hkv);
-  if (L.total > static_cast<size_t>(FD_STATIC_SCRATCH_BYTES))
-    return fail(FD_ERR_UNSUPPORTED,
-                "this decode shape needs up to %zu bytes of scratch, more than the %zu-byte static "
-                "scratch of fd_decode_attention_static; use fd_decode_attention",
-                L.total, static_cast<size_t>(FD_STATIC_SCRATCH_BYTES));
-
-  void* ws = nullptr;
-  if ((s = static_scratch_address(dev, &ws)) != FD_OK) return s;
-  char* base = static_cast<char*>(ws);
-  WsHeader* hdr = reinterpret_cast<WsHeader*>(base);
-  DecodeItem* items = reinterpret_cast<DecodeItem*>(base + L.dec_items);
-  int32_t* row_nsplit = reinterpret_cast<int32_t*>(base + L.row_nsplit);
-  int32_t* row_base = reinterpret_cast<int32_t*>(base + L.row_base);
-  float* part_o = reinterpret_cast<float*>(base + L.part_o);
-  float* part_lse = reinterpret_cast<float*>(base + L.part_lse);
-  int32_t* arrivals = reinterpret_cast<int32_t*>(base + L.arrivals);
-
-  DecodeParams dp{};
-  dp.q = q->data;
-  dp.q_sr = q->stride[0];
-  dp.q_sh = q->stride[1];
-  dp.k = k_cache->data;
-  dp.v = v_cache->data;
-  dp.kv_sb = k_cache->stride[0];
-  dp.kv_sh = k_cache->stride[1];
-  dp.out = out->data;
-  dp.o_sr = out->stride[0];
-  dp.o_sh = out->stride[1];
-  dp.lse = lse;
-  dp.hq = sh.hq;
-  dp.hkv = sh.hkv;
-  dp.g = sh.g;
-  dp.d = sh.d;
-  dp.cap = sh.cap;
-  dp.q_box_rows = sh.hq < 16 ? sh.hq : 16;
-  dp.kv_box_rows = sh.cap < 128 ? sh.cap : 128;
-  dp.scale_log2 = static_cast<float>(1.0 / std::sqrt(static_cast<double>(sh.d)) * 1.4426950408889634);
-  dp.hdr = hdr;
-  dp.items = items;
-  dp.row_base = row_base;
-  dp.part_o = part_o;
-  dp.part_lse = part_lse;
-  dp.arrivals = arrivals;
-
-  CUtensorMap tq, tk, tv;
-  if (sh.use_tc) {
-    const uint64_t qd[3] = {static_cast<uint64_t>(sh.d), static_cast<uint64_t>(sh.hq), static_cast<uint64_t>(sh.B)};
-    const uint64_t qs[2] = {static_cast<uint64_t>(q->stride[1]) * 2, static_cast<uint64_t>(q->stride[0]) * 2};
-    const uint32_t qb[3] = {64, static_cast<uint32_t>(dp.q_box_rows), 1};
-    if ((s = make_tmap(&tq, q->data, 3, qd, qs, qb, "q")) != FD_OK) return s;
-    const uint64_t kd[4] = {static_cast<uint64_t>(sh.d), static_cast<uint64_t>(sh.cap),
-                            static_cast<uint64_t>(sh.hkv), static_cast<uint64_t>(sh.B)};
-    const uint64_t ks[3] = {static_cast<uint64_t>(k_cache->stride[2]) * 2,
-                            static_cast<uint64_t>(k_cache->stride[1]) * 2,
-                            static_cast<uint64_t>(k_cache->stride[0]) * 2};
-    const uint32_t kb[4] = {64, static_cast<uint32_t>(dp.kv_box_rows), 1, 1};
-    if ((s = make_tmap(&tk, k_cache->data, 4, kd, ks, kb, "k_cache")) != FD_OK) return s;
-    if ((s = make_tmap(&tv, v_cache->data, 4, kd, ks, kb, "v_cache")) != FD_OK) return s;
+  PresetScratch scratch{nullptr, static_cast<size_t>(FD_STATIC_SCRATCH_BYTES),
+                        "static scratch of fd_decode_attention_static"};
+  if (sh.B > 0 && num_splits >= 0 && cache_lens && lse) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    if ((s = static_scratch_address(dev, &scratch.base)) != FD_OK) return s;
   }
-
-  PlanParams pp{};
-  pp.lens = cache_lens;
-  pp.B = sh.B;
-  pp.hkv = sh.hkv;
-  pp.hq = sh.hq;
-  pp.cap = sh.cap;
-  pp.fixed = num_splits;
-  pp.nctas = nctas;
-  pp.max_dec_items = max_items;
-  pp.hdr = hdr;
-  pp.items = items;
-  pp.row_nsplit = row_nsplit;
-  pp.row_base = row_base;
-  pp.arrivals = arrivals;
-
-  CombineParams cp{};
-  cp.row_nsplit = row_nsplit;
-  cp.row_base = row_base;
-  cp.part_o = part_o;
-  cp.part_lse = part_lse;
-  cp.out = out->data;
-  cp.o_sr = out->stride[0];
-  cp.o_sh = out->stride[1];
-  cp.lse = lse;
-  cp.rows = sh.B;
-  cp.hq = sh.hq;
-  cp.hkv = sh.hkv;
-  cp.g = sh.g;
-  cp.d = sh.d;
-  cp.dtype = sh.dtype;
-
-  // the status word and the work cursor must start at zero; the previous call left its own
-  ce = cudaMemsetAsync(hdr, 0, sizeof(WsHeader), stream);
-  if (ce != cudaSuccess) return cuda_fail(ce, "clear static scratch header");
-  ce = launch_plan_decode(pp, stream);
-  if (ce != cudaSuccess) return cuda_fail(ce, "plan kernel launch");
-  ce = sh.use_tc ? launch_decode_tc(dp, tq, tk, tv, nctas, stream)
-                 : launch_decode_simt(dp, sh.dtype, nctas, stream);
-  if (ce != cudaSuccess) return cuda_fail(ce, "split kernel launch");
-  if (sh.use_tc) {
-    ce = launch_combine(cp, stream);
-    if (ce != cudaSuccess) return cuda_fail(ce, "combine kernel launch");
-  }
-  return FD_OK;
+  return decode_call(q, k_cache, v_cache, cache_lens, num_splits, out, lse,
+                     static_cast<cudaStream_t>(stream), nullptr, nullptr, &scratch);
 }
