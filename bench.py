@@ -14,7 +14,8 @@ keys at shuffled physical positions.
 
 Prints one JSON line on rank 0. `value` is the whole-job GB/s: the algorithmic bytes every rank
 processed (K+V bytes of the valid keys plus the Q bytes) over the slowest rank's device time.
-With N > 1 (torchrun) every rank runs an independent replica: the path has no exchange step.
+With N > 1 every rank runs an independent replica: the path has no exchange step. Under torchrun
+--gpus must equal WORLD_SIZE; without it, --gpus N > 1 starts the N processes itself.
 `--impl reference` times the float64 CPU oracle on a bounded sample of the same workload.
 """
 
@@ -60,8 +61,9 @@ def parse_args():
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--profile-calls", type=int, default=200,
                     help="calls timed with per-kernel events after the timed region (0: skip)")
-    ap.add_argument("--cpu-seconds", type=float, default=15.0,
-                    help="host-time budget of the oracle CPU baseline sample")
+    ap.add_argument("--cpu-seconds", type=float, default=20.0,
+                    help="host-time budget of the oracle CPU baseline samples (half with every "
+                         "thread, half on one thread)")
     return ap.parse_args()
 
 
@@ -499,22 +501,36 @@ def run_fd(args, rank, world, local_rank):
             roofline, roofline_tiles = roofline_tiles, roofline
 
     # ---- end to end: host buffers, copies inside the timed region ----
+    # The step's inputs are q, the lengths and the cache rows that hold keys: each (sequence, KV
+    # head)'s first len rows of K and V (rows past the lengths are padding, not input), or the
+    # whole page pool and block table of a paged cache. They are copied from pinned host memory,
+    # one contiguous copy per (sequence, KV head) slab, and out / lse are read back every step.
     e2e = None
     if args.e2e_steps > 0:
         hq_ = queries(inp).pin_memory()
-        hk = (pgc.k_pages if paged else inp.k_cache).pin_memory()
-        hv = (pgc.v_pages if paged else inp.v_cache).pin_memory()
-        hl = [t.pin_memory() for t in lens_h]
+        hl = [t_.pin_memory() for t_ in lens_h]
         ho = torch.empty_like(queries(inp)).pin_memory()
         hlse = torch.empty((R, hq), dtype=torch.float32).pin_memory()
-        h2d = sum(x.numel() * x.element_size() for x in [hq_, hk, hv] + hl)
+        copies = [(q, hq_)] + list(zip(lens, hl))
+        if paged:
+            copies += [(k, pgc.k_pages.pin_memory()), (v, pgc.v_pages.pin_memory()),
+                       (table, pgc.block_table.pin_memory())]
+            what = "q, lengths, the whole page pool (all pages but 3 spares hold keys) and the block table"
+        else:
+            hk = inp.k_cache.pin_memory()
+            hv = inp.v_cache.pin_memory()
+            for b_, n_ in enumerate(key_lens(inp)):
+                if n_ > 0:
+                    for h_ in range(hkv):
+                        copies.append((k[b_, h_, :n_], hk[b_, h_, :n_]))
+                        copies.append((v[b_, h_, :n_], hv[b_, h_, :n_]))
+            what = ("q, lengths and the valid cache rows (the first len keys of every (sequence, KV "
+                    "head), one copy per slab); padding rows past the lengths are not copied")
+        h2d = sum(src.numel() * src.element_size() for _, src in copies)
         d2h = ho.numel() * ho.element_size() + hlse.numel() * 4
 
         def e2e_step():
-            q.copy_(hq_, non_blocking=True)
-            k.copy_(hk, non_blocking=True)
-            v.copy_(hv, non_blocking=True)
-            for dst, src in zip(lens, hl):
+            for dst, src in copies:
                 dst.copy_(src, non_blocking=True)
             step()
             ho.copy_(out, non_blocking=True)
@@ -534,15 +550,22 @@ def run_fd(args, rank, world, local_rank):
         te = max_over_ranks(a0.elapsed_time(a1), world, dev)
         e2e = {"value": round(whole_job_gbs(alg, args.e2e_steps, world, te), 3),
                "unit": "GB/s", "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
-               "steps": args.e2e_steps,
-               "note": "full cache tensors copied host->device every step"}
+               "steps": args.e2e_steps, "copies_per_step": len(copies) + 2,
+               "note": f"host->device every step: {what}; out and lse read back"}
 
     cpu = None
     if rank == 0 and world == 1 and args.cpu_seconds > 0:
-        rate, desc, groups, el = oracle_sample(inp, args.cpu_seconds,
-                                               quant=(f8.k_scale, f8.v_scale) if fp8 else None)
+        # the oracle as it stands on the host's cores: once with every thread its numpy uses,
+        # once limited to one thread, each on a bounded sample of the same workload
+        from threadpoolctl import threadpool_limits
+        quant = (f8.k_scale, f8.v_scale) if fp8 else None
+        rate, desc, groups, el = oracle_sample(inp, args.cpu_seconds / 2, quant=quant)
+        with threadpool_limits(limits=1):
+            rate1, desc1, groups1, el1 = oracle_sample(inp, args.cpu_seconds / 2, quant=quant)
         cpu = {"value": round(rate / 1e9, 4), "unit": "GB/s", "cores": cpu_threads(),
-               "kind": "oracle", "cpu": cpu_model(), "sample": f"{desc}; {el:.1f}s"}
+               "kind": "oracle", "cpu": cpu_model(), "sample": f"{desc}; {el:.1f}s",
+               "single_core": {"value": round(rate1 / 1e9, 4), "unit": "GB/s", "cores": 1,
+                               "sample": f"{desc1}; {el1:.1f}s"}}
 
     if rank == 0:
         config = {"workload": inp.name, "batch": R if not chunk else B, "q_heads": hq, "kv_heads": hkv,
@@ -580,11 +603,28 @@ def run_fd(args, rank, world, local_rank):
     return 0
 
 
+def free_port() -> int:
+    import socket
+    with socket.socket(socket.AF_INET, socket.SOCK_STREAM) as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
 def main():
     args = parse_args()
+    if "WORLD_SIZE" not in os.environ and args.gpus > 1:
+        # not under torchrun: start the N replicas (one process per GPU) here
+        cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1",
+               f"--nproc-per-node={args.gpus}", "--master-addr=127.0.0.1",
+               f"--master-port={free_port()}", os.path.abspath(__file__), *sys.argv[1:]]
+        return subprocess.call(cmd)
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        log(f"bench.py: --gpus {args.gpus} but WORLD_SIZE is {world}; launch one process per GPU "
+            f"(torchrun --nproc-per-node {args.gpus}) or pass --gpus {world}")
+        return 2
     if args.impl == "reference":
         return run_reference(args, rank, world)
     if world > 1:

@@ -44,3 +44,13 @@ def test_e4m3_option_rejects_a_chunk_workload():
            "--workload", "5", "--batch", "1", "--kv-dtype", "e4m3"]
     p = subprocess.run(cmd, cwd=ROOT, capture_output=True, text=True, timeout=600)
     assert p.returncode != 0 and "e4m3" in (p.stderr + p.stdout)
+
+
+def test_gpus_flag_must_match_the_launch():
+    # under a launcher that started a different number of processes, --gpus N is refused instead
+    # of silently measuring another count of GPUs
+    env = dict(os.environ, WORLD_SIZE="2", RANK="0", LOCAL_RANK="0")
+    cmd = [sys.executable, "bench.py", "--gpus", "1", "--steps", "1", "--warmup", "0"]
+    p = subprocess.run(cmd, cwd=ROOT, capture_output=True, text=True, timeout=600, env=env)
+    assert p.returncode == 2 and "WORLD_SIZE is 2" in p.stderr, p.stderr[-2000:]
+    assert p.stdout.strip() == ""
