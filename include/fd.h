@@ -189,9 +189,12 @@ fd_status fd_decode_attention_paged_fp8(const fd_tensor* q, const fd_tensor* k_p
  * fd_split_plan — the variable-length split planner, on the host (no CUDA call).
  *
  * FlashDecoding page, "Variable-Length序列动态切分策略" (allocator with min_chunk 128 and
- * max_chunk 1024), read for persistent CTAs on one GPU: chunk = clamp(ceil(sum(len) * Hkv /
- * (8 * num_ctas)), 256, 1024) tokens ("性能压测与瓶颈分析": pieces under ~256 tokens lose to
- * launch overhead); sequence b gets n_b = max(1, ceil(len_b / chunk)) equal splits
+ * max_chunk 1024), read for persistent CTAs on one GPU. For W = 8, 4, 2, 1 waves of items,
+ * chunk_W = clamp(ceil(sum(len) * Hkv / (W * num_ctas)), 256, 1024) tokens ("性能压测与瓶颈分析":
+ * pieces under ~256 tokens lose to launch overhead); the chunk is the chunk_W of least
+ * ceil(items_W / num_ctas) * (ceil(chunk_W / 128) + 2), items_W = Hkv * sum_b max(1,
+ * ceil(len_b / chunk_W)), ties to the larger W (a work item's fixed cost is taken as two 128-key
+ * tiles). Sequence b gets n_b = max(1, ceil(len_b / chunk)) equal splits
  * [floor(s*len_b/n_b), floor((s+1)*len_b/n_b)); items are ordered longest split first
  * (sequences by their longest split, descending, ties by index), then KV head, then split.
  * num_splits > 0 instead fixes n_b = num_splits with ceil(len_b/num_splits)-key splits.

@@ -17,7 +17,13 @@ Chunked-Prefills page ("Chunked-Prefillsåˆ†å—é¢„å¡«å……æœºåˆ¶ï¼šç ´è§£å¤§æ¨¡åž‹æ
 Reading used on one GPU (the workers are the persistent CTAs, one per SM):
 
 1. total = sum of the clamped cache lengths.
-2. chunk = clamp(ceil(total * Hkv / (WAVES * num_ctas)), 256, 1024) tokens.
+2. For each target of W = 8, 4, 2, 1 waves of items over the CTAs,
+   chunk_W = clamp(ceil(total * Hkv / (W * num_ctas)), 256, 1024) tokens and
+   items_W = Hkv * sum_b max(1, ceil(len_b / chunk_W)). The chunk is the chunk_W of least
+   estimated makespan ceil(items_W / num_ctas) * (ceil(chunk_W / 128) + 2), ties to the larger W
+   (2 = the fixed cost of a work item in 128-key tiles; the pages' allocator fills every worker
+   once, which W = 1 is, and its ~256-token floor keeps pieces from getting too small for their
+   overhead, which the cost term weighs).
 3. n_b = max(1, ceil(len_b / chunk)) splits for sequence b.
 4. Split s of sequence b is [floor(s * len_b / n_b), floor((s + 1) * len_b / n_b)): the offset
    restarts at 0 for every sequence and no token is dropped (the printed allocator never
@@ -61,13 +67,15 @@ from typing import List, Sequence, Tuple
 
 __all__ = [
     "MIN_CHUNK", "MAX_CHUNK", "WAVES", "Q_TILE", "CHUNK_KV_SPLIT",
-    "DecodePlan", "decode_plan", "ChunkPlan", "chunk_plan",
+    "DecodePlan", "decode_plan", "choose_chunk", "ChunkPlan", "chunk_plan",
 ]
 
 MIN_CHUNK = 256        # launch-overhead floor, FlashDecoding page "æ€§èƒ½åŽ‹æµ‹ä¸Žç“¶é¢ˆåˆ†æž"
 MAX_CHUNK = 1024       # max_chunk of the allocator / top of the 256-1024 tile range
 MIN_PIECE = 128        # min_chunk of the allocator
-WAVES = 8              # target items per persistent CTA
+WAVES = 8              # largest target of items per persistent CTA
+WAVE_CHOICES = (8, 4, 2, 1)
+ITEM_FIXED_TILES = 2   # fixed cost of a work item, in 128-key tiles
 Q_TILE = 128           # query rows per chunked-prefill tile
 CHUNK_KV_SPLIT = 2048  # keys per split for a chunked-prefill query tile
 
@@ -104,6 +112,20 @@ def _split_bounds_fixed(n_tok: int, n_split: int, align: int = 1) -> List[Tuple[
     return [(min(s * c, n_tok), min((s + 1) * c, n_tok)) for s in range(n_split)]
 
 
+def choose_chunk(lens: Sequence[int], num_kv_heads: int, num_ctas: int) -> int:
+    """Step 2 of the module docstring: the chunk of the least estimated makespan."""
+    total = sum(lens)
+    n = max(1, num_ctas)
+    best = None
+    for waves in WAVE_CHOICES:
+        chunk = max(MIN_CHUNK, min(MAX_CHUNK, _cdiv(total * num_kv_heads, waves * n)))
+        items = num_kv_heads * sum(max(1, _cdiv(x, chunk)) for x in lens)
+        cost = _cdiv(items, n) * (_cdiv(chunk, 128) + ITEM_FIXED_TILES)
+        if best is None or cost < best[0]:
+            best = (cost, chunk)
+    return best[1]
+
+
 def decode_plan(cache_lens: Sequence[int], num_kv_heads: int, cache_capacity: int,
                 num_ctas: int, num_splits: int = 0, align: int = 1) -> DecodePlan:
     """Plan the split-KV work of one decode call (see the module docstring)."""
@@ -114,9 +136,7 @@ def decode_plan(cache_lens: Sequence[int], num_kv_heads: int, cache_capacity: in
         chunk = 0
         keys = [_cdiv(n, num_splits) for n in lens]
     else:
-        total = sum(lens)
-        chunk = _cdiv(total * num_kv_heads, WAVES * max(1, num_ctas))
-        chunk = max(MIN_CHUNK, min(MAX_CHUNK, chunk))
+        chunk = choose_chunk(lens, num_kv_heads, num_ctas)
         counts = [max(1, _cdiv(n, chunk)) for n in lens]
         bounds = [_split_bounds_equal(n, c, align) for n, c in zip(lens, counts)]
         keys = [_cdiv(n, c) for n, c in zip(lens, counts)]

@@ -84,6 +84,7 @@ struct __align__(1024) TcSmem {
   int32_t plan_order[kFusedPlanMaxBatch], plan_rbase[kFusedPlanMaxBatch + 1];
   int32_t plan_ioff[kFusedPlanMaxBatch + 1];
   long long plan_red[kF8Threads / 32];
+  long long plan_red4[kF8Threads / 32][kPlanWaveChoices];  // split sums per wave choice
   int32_t plan_clamped;
   int32_t item_slot[2][2];                       // item index (-1: stop), tiles
   DecodeItem item[2];                            // the item's descriptor (by item parity)
@@ -400,7 +401,34 @@ __global__ void __launch_bounds__(kF8 ? kF8Threads : kTcThreads, 1)
     long long total = 0;
 #pragma unroll
     for (int w = 0; w < kThreads / 32; ++w) total += S.plan_red[w];
-    const int32_t chunk = p.fixed > 0 ? 0 : plan_chunk_tokens(total, p.hkv, p.plan_ctas);
+    int32_t chunk = 0;
+    if (p.fixed <= 0) {  // the same for every thread
+      int32_t chunks[kPlanWaveChoices];
+      long long cnt[kPlanWaveChoices];
+#pragma unroll
+      for (int i = 0; i < kPlanWaveChoices; ++i) {
+        chunks[i] = plan_chunk_for_waves(total, p.hkv, p.plan_ctas, plan_waves(i));
+        cnt[i] = 0;
+      }
+      for (int b = tid; b < B; b += kThreads)
+#pragma unroll
+        for (int i = 0; i < kPlanWaveChoices; ++i) cnt[i] += plan_num_splits(S.plan_len[b], chunks[i], 0);
+#pragma unroll
+      for (int i = 0; i < kPlanWaveChoices; ++i) {
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) cnt[i] += __shfl_xor_sync(0xffffffffu, cnt[i], o);
+        if (lane == 0) S.plan_red4[warp][i] = cnt[i];
+      }
+      __syncthreads();
+      int64_t sums[kPlanWaveChoices];
+#pragma unroll
+      for (int i = 0; i < kPlanWaveChoices; ++i) {
+        sums[i] = 0;
+#pragma unroll
+        for (int w = 0; w < kThreads / 32; ++w) sums[i] += S.plan_red4[w][i];
+      }
+      chunk = plan_pick_chunk(chunks, sums, p.hkv, p.plan_ctas);
+    }
     for (int b = tid; b < B; b += kThreads) {
       const int32_t n = plan_num_splits(S.plan_len[b], chunk, p.fixed);
       S.plan_n[b] = n;

@@ -70,7 +70,8 @@ struct WsHeader {
   int32_t tile_counter;
   int32_t dec_exit;         // CTAs of the tensor-core split kernel that have finished (zero
                             // between calls)
-  int32_t pad[58];
+  int32_t tile_ctas;        // chunked prefill: CTAs the tile kernel keeps (chunk_tile_ctas)
+  int32_t pad[57];
 };
 static_assert(sizeof(WsHeader) == 256, "WsHeader is 256 bytes");
 
@@ -81,12 +82,41 @@ FD_HD int32_t clamp_len(int64_t len, int32_t cap) {
   return len < 0 ? 0 : (len > cap ? cap : static_cast<int32_t>(len));
 }
 
-// chunk = clamp(ceil(total * Hkv / (kWaves * nctas)), kMinChunk, kMaxChunk)
-FD_HD int32_t plan_chunk_tokens(int64_t total, int32_t hkv, int32_t nctas) {
-  int64_t c = cdiv64(total * hkv, static_cast<int64_t>(kWaves) * (nctas > 0 ? nctas : 1));
+// The chunk (split size) comes from a target number of item waves W over the CTAs:
+//   chunk_W = clamp(ceil(total * Hkv / (W * nctas)), kMinChunk, kMaxChunk).
+// A small call (a few long sequences, say) under W = kWaves would be cut into items of one or two
+// key tiles, whose fixed cost (start, Q load, partial result, merge) then outweighs their keys;
+// so the planner weighs W = 8, 4, 2, 1 and keeps the chunk of least estimated makespan
+//   ceil(items_W / nctas) * (ceil(chunk_W / 128) + kItemFixedTiles),
+// items_W = Hkv * sum_b max(1, ceil(len_b / chunk_W)), ties to the larger W. Large calls, whose
+// chunk is kMaxChunk for every W, keep the plan of W = kWaves.
+constexpr int kPlanWaveChoices = 4;
+constexpr int32_t kItemFixedTiles = 2;  // fixed cost of a work item, in 128-key tiles
+FD_HD int32_t plan_waves(int i) { return kWaves >> i; }  // 8, 4, 2, 1
+
+FD_HD int32_t plan_chunk_for_waves(int64_t total, int32_t hkv, int32_t nctas, int32_t waves) {
+  int64_t c = cdiv64(total * hkv, static_cast<int64_t>(waves) * (nctas > 0 ? nctas : 1));
   if (c < kMinChunk) c = kMinChunk;
   if (c > kMaxChunk) c = kMaxChunk;
   return static_cast<int32_t>(c);
+}
+
+// The chunk of least estimated makespan among the candidates chunks[i] = plan_chunk_for_waves(...,
+// plan_waves(i)), given split_sums[i] = sum_b max(1, ceil(len_b / chunks[i])).
+FD_HD int32_t plan_pick_chunk(const int32_t* chunks, const int64_t* split_sums, int32_t hkv,
+                              int32_t nctas) {
+  const int64_t n = nctas > 0 ? nctas : 1;
+  int32_t best = chunks[0];
+  int64_t best_cost = 0;
+  for (int i = 0; i < kPlanWaveChoices; ++i) {
+    const int64_t waves = cdiv64(split_sums[i] * hkv, n);
+    const int64_t cost = waves * (cdiv64(chunks[i], 128) + kItemFixedTiles);
+    if (i == 0 || cost < best_cost) {
+      best = chunks[i];
+      best_cost = cost;
+    }
+  }
+  return best;
 }
 
 // Splits of a sequence: the fixed count, else max(1, ceil(len / chunk)).
@@ -158,6 +188,38 @@ FD_HD bool chunk_packed(int32_t c, int32_t g) { return g >= 2 && c >= 2 && c * g
 FD_HD int32_t chunk_tile_splits(int32_t keys) {
   const int32_t n = static_cast<int32_t>(cdiv64(keys, kChunkKvSplit));
   return n < 1 ? 1 : n;
+}
+
+// A chunked-prefill call runs its tile kernel and its decode-row split kernel side by side: the
+// tile kernel keeps N of the device's nsm multiprocessors (its other CTAs leave at once) and the
+// decode rows stream on the rest, taking over the tiles' multiprocessors when those finish.
+// Cost model (B200 measurements): a tile CTA spends kTileKeyTileUs per 128-key tile of a
+// 128-row query tile, whatever its valid rows; decode rows stream at most kDecodeSmGBs per
+// multiprocessor and kHbmGBs in all. While the tiles run (phase 1) the decode rows stream at
+// min(kHbmGBs, (nsm - N) kDecodeSmGBs); what is left then streams at kHbmGBs. N minimises the
+// total: the time of phase 1 plus that of the rest. `key_tiles` counts the 128-key tiles of all
+// tile items, `dec_bytes` the K/V bytes of the decode rows. No tiles: 0; no decode rows: nsm.
+constexpr float kTileKeyTileUs = 2.3f;  // 250 µs for workload 5's 16192 key tiles on 148 CTAs
+constexpr float kDecodeSmGBs = 51.f;    // CUDA-core decode rows beside 93 tile CTAs: 1.13 GB in 401 µs on 55 SMs
+constexpr float kHbmGBs = 6000.f;       // decode rows alone on the whole device
+FD_HD int32_t chunk_tile_ctas(int64_t key_tiles, int64_t dec_bytes, int32_t nsm) {
+  if (key_tiles <= 0) return 0;
+  if (dec_bytes <= 0 || nsm <= 1) return nsm;
+  const float dec = static_cast<float>(dec_bytes);
+  float best = 0.f;
+  int32_t best_n = nsm;
+  for (int32_t n = 1; n <= nsm; ++n) {
+    const float t1 = static_cast<float>(key_tiles) * kTileKeyTileUs / static_cast<float>(n);
+    const float sm_rate = static_cast<float>(nsm - n) * kDecodeSmGBs;
+    const float rate = (sm_rate < kHbmGBs ? sm_rate : kHbmGBs) * 1e3f;  // bytes per microsecond
+    const float left = dec - rate * t1;
+    const float t = t1 + (left > 0.f ? left / (kHbmGBs * 1e3f) : 0.f);
+    if (n == 1 || t < best) {
+      best = t;
+      best_n = n;
+    }
+  }
+  return best_n;
 }
 
 // Upper bounds for a chunked-prefill call of T packed rows over B requests (any lengths).

@@ -59,6 +59,35 @@ __device__ void block_exclusive_scan(const int32_t* in, int32_t* out, int n, int
   __syncthreads();
 }
 
+// The planner's chunk (plan.h, plan_pick_chunk) for the lengths len[0..B) whose sum is `total`;
+// entries < 0 are not sequences (chunk mode: requests that are not decode rows). All threads of
+// the CTA call it; `sums` holds kPlanWaveChoices zeroed 64-bit counters of shared memory.
+__device__ int32_t plan_pick_chunk_block(const int32_t* len, int B, int64_t total, int32_t hkv,
+                                         int32_t nctas, unsigned long long* sums) {
+  int32_t chunks[kPlanWaveChoices];
+  long long local[kPlanWaveChoices];
+#pragma unroll
+  for (int i = 0; i < kPlanWaveChoices; ++i) {
+    chunks[i] = plan_chunk_for_waves(total, hkv, nctas, plan_waves(i));
+    local[i] = 0;
+  }
+  for (int b = threadIdx.x; b < B; b += plan_threads()) {
+    if (len[b] < 0) continue;
+#pragma unroll
+    for (int i = 0; i < kPlanWaveChoices; ++i) local[i] += plan_num_splits(len[b], chunks[i], 0);
+  }
+#pragma unroll
+  for (int i = 0; i < kPlanWaveChoices; ++i) {
+    const long long s = warp_sum_i64(local[i]);
+    if (lane_id() == 0 && s != 0) atomicAdd(&sums[i], static_cast<unsigned long long>(s));
+  }
+  __syncthreads();
+  int64_t totals[kPlanWaveChoices];
+#pragma unroll
+  for (int i = 0; i < kPlanWaveChoices; ++i) totals[i] = static_cast<int64_t>(sums[i]);
+  return plan_pick_chunk(chunks, totals, hkv, nctas);
+}
+
 // Decode plan over sequences whose lengths are len[0..B): items in longest-first order.
 // `row_of` maps sequence index -> output row (identity for decode calls).
 __device__ void plan_decode_body(const PlanParams& p, const int32_t* len_src, int B,
@@ -75,9 +104,11 @@ __device__ void plan_decode_body(const PlanParams& p, const int32_t* len_src, in
   const int kPlanThreads = plan_threads();
   __shared__ int s_scan[33];
   __shared__ unsigned long long s_total;
+  __shared__ unsigned long long s_sums[kPlanWaveChoices];
   const int tid = threadIdx.x;
 
   if (tid == 0) s_total = 0ull;
+  if (tid < kPlanWaveChoices) s_sums[tid] = 0ull;
   __syncthreads();
   long long local = 0;
   uint32_t clamped = 0;
@@ -93,8 +124,9 @@ __device__ void plan_decode_body(const PlanParams& p, const int32_t* len_src, in
   if (clamped) atomicOr(s_flags, FD_FLAG_LEN_CLAMPED);
   __syncthreads();
 
-  const int32_t chunk =
-      p.fixed > 0 ? 0 : plan_chunk_tokens(static_cast<int64_t>(s_total), p.hkv, p.nctas);
+  const int32_t chunk = p.fixed > 0 ? 0
+                                    : plan_pick_chunk_block(s_len, B, static_cast<int64_t>(s_total),
+                                                            p.hkv, p.nctas, s_sums);
   for (int b = tid; b < B; b += kPlanThreads) {
     const int32_t n = plan_num_splits(s_len[b], chunk, p.fixed);
     s_n[b] = n;
@@ -210,9 +242,12 @@ __global__ void __launch_bounds__(kMaxPlanThreads, 1) plan_chunk_kernel(PlanPara
   int32_t* s_tioff = s_dioff + B + 1;  // B + 1: tile item offsets (request order)
   __shared__ int s_scan[33];
   __shared__ unsigned long long s_total;
+  __shared__ unsigned long long s_key_tiles;  // 128-key tiles of all tile items
+  __shared__ unsigned long long s_sums[kPlanWaveChoices];
   __shared__ uint32_t s_flags;
   __shared__ int s_ndec;
-  if (tid == 0) { s_total = 0ull; s_flags = 0u; s_ndec = 0; }
+  if (tid == 0) { s_total = 0ull; s_key_tiles = 0ull; s_flags = 0u; s_ndec = 0; }
+  if (tid < kPlanWaveChoices) s_sums[tid] = 0ull;
   __syncthreads();
 
   long long local = 0;
@@ -227,6 +262,7 @@ __global__ void __launch_bounds__(kMaxPlanThreads, 1) plan_chunk_kernel(PlanPara
     s_c[b] = c;
     s_p[b] = pp;
     s_dlen[b] = dlen;
+    s_key[b] = c == 1 ? dlen : -1;  // the decode rows' lengths, for the chunk choice below
     local += dlen;
     ndec += c == 1 ? 1 : 0;
   }
@@ -235,7 +271,9 @@ __global__ void __launch_bounds__(kMaxPlanThreads, 1) plan_chunk_kernel(PlanPara
   if (ndec) atomicAdd(&s_ndec, ndec);
   __syncthreads();
 
-  const int32_t chunk = plan_chunk_tokens(static_cast<int64_t>(s_total), p.hkv, p.nctas);
+  const int32_t chunk =
+      plan_pick_chunk_block(s_key, B, static_cast<int64_t>(s_total), p.hkv, p.nctas, s_sums);
+  __syncthreads();  // s_key is rewritten below
   for (int b = tid; b < B; b += nthr) {
     const int32_t c = s_c[b];
     if (c == 1) {
@@ -247,11 +285,15 @@ __global__ void __launch_bounds__(kMaxPlanThreads, 1) plan_chunk_kernel(PlanPara
       s_n[b] = 0;
       s_key[b] = -1;
       int32_t cnt = 0;
+      int64_t ktiles = 0;
       for (int32_t t = 0; t * kQTile < c; ++t) {
         const int32_t kt = chunk_tile_keys(s_p[b], c, t, p.cap);
         cnt += chunk_tile_splits(kt);
+        ktiles += cdiv64(kt, kQTile);  // the split grid is a multiple of the key tile
       }
-      s_tcnt[b] = cnt * (chunk_packed(c, p.hq / p.hkv) ? p.hkv : p.hq);
+      const int32_t nheads = chunk_packed(c, p.hq / p.hkv) ? p.hkv : p.hq;
+      s_tcnt[b] = cnt * nheads;
+      if (c > 1) atomicAdd(&s_key_tiles, static_cast<unsigned long long>(ktiles * nheads));
     }
   }
   __syncthreads();
@@ -354,6 +396,10 @@ __global__ void __launch_bounds__(kMaxPlanThreads, 1) plan_chunk_kernel(PlanPara
     p.hdr->num_tile_items = overflow ? 0 : n_tile_items;
     p.hdr->dec_counter = 0;
     p.hdr->tile_counter = 0;
+    p.hdr->tile_ctas = overflow ? 0
+                                : chunk_tile_ctas(static_cast<int64_t>(s_key_tiles),
+                                                  static_cast<int64_t>(s_total) * p.kv_key_bytes,
+                                                  p.tile_sms);
     uint32_t f = s_flags | (overflow ? FD_FLAG_PLAN_OVERFLOW : 0u);
     if (f) atomicOr(&p.hdr->status, f);
   }

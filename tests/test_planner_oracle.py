@@ -57,6 +57,26 @@ def test_auto_hand_worked_small():
                        (2, 0, 0, 0, 0)]
 
 
+def test_auto_hand_worked_long_context():
+    # one 32768-key sequence, 8 KV heads, 148 CTAs (U = 262144 token-heads):
+    #   W = 8: chunk max(256, ceil(U / 1184) = 222) = 256, 128 splits, 1024 items, 7 waves x (2 + 2) = 28
+    #   W = 4: chunk 443, 74 splits, 592 items, 4 waves x (4 + 2) = 24
+    #   W = 2: chunk 886, 37 splits, 296 items, 2 waves x (7 + 2) = 18   <- least
+    #   W = 1: chunk min(1772, 1024) = 1024, 32 splits, 256 items, 2 waves x (8 + 2) = 20
+    p = P.decode_plan([32768], 8, 32768, 148)
+    assert p.chunk_tokens == 886 and p.splits_per_seq == [37] and p.total_items == 296
+    # two such sequences: W = 4 (chunk 886, 592 items, 4 waves x 9 = 36) beats W = 2 / 1 (chunk
+    # 1024, 512 items, 4 waves x 10 = 40) and W = 8 (chunk 443, 1184 items, 8 waves x 6 = 48)
+    p = P.decode_plan([32768, 32768], 8, 32768, 148)
+    assert p.chunk_tokens == 886 and p.splits_per_seq == [37, 37]
+    # the 70B-like decode batch: chunk 1024 for every W, so the W = 8 plan
+    from workloads import uniform_lens
+    lens = uniform_lens(1103, 32, 1024, 32768)
+    p = P.decode_plan(lens, 8, 32768, 148)
+    assert p.chunk_tokens == 1024
+    assert p.splits_per_seq == [-(-n // 1024) for n in lens]
+
+
 def test_auto_clamps_lengths():
     p = P.decode_plan([-5, 10**9], 2, 3000, 148)
     assert p.splits_per_seq[0] == 1
