@@ -46,20 +46,27 @@ fd_status cuda_fail(cudaError_t e, const char* what) {
   } while (0)
 
 // ---------------------------------------------------------------------------- workspace ------
+// Per (device, stream): the grow-only device buffer, plus the side stream and the two events a
+// chunked-prefill call forks its decode rows onto and joins back with. They are created with the
+// first buffer, so a call under graph capture (which must find the buffer reserved) never
+// creates them.
 struct Workspace {
   void* ptr = nullptr;
   size_t bytes = 0;
+  cudaStream_t side = nullptr;
+  cudaEvent_t fork = nullptr, join = nullptr;
 };
 std::mutex g_mu;
 std::map<std::pair<int, uintptr_t>, Workspace> g_ws;
 
-fd_status get_workspace(cudaStream_t stream, size_t need, void** out) {
+fd_status get_workspace(cudaStream_t stream, size_t need, void** out, Workspace* view = nullptr) {
   int dev = 0;
   FD_CUDA(cudaGetDevice(&dev), "cudaGetDevice");
   std::lock_guard<std::mutex> lock(g_mu);
   Workspace& w = g_ws[{dev, reinterpret_cast<uintptr_t>(stream)}];
   if (w.ptr && w.bytes >= need) {
     *out = w.ptr;
+    if (view) *view = w;
     return FD_OK;
   }
   cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
@@ -93,7 +100,15 @@ fd_status get_workspace(cudaStream_t stream, size_t need, void** out) {
   FD_CUDA(cudaStreamSynchronize(stream), "cudaStreamSynchronize");
   w.ptr = p;
   w.bytes = nb;
+  if (!w.side) {
+    int prio_lo = 0, prio_hi = 0;
+    FD_CUDA(cudaDeviceGetStreamPriorityRange(&prio_lo, &prio_hi), "cudaDeviceGetStreamPriorityRange");
+    FD_CUDA(cudaStreamCreateWithPriority(&w.side, cudaStreamNonBlocking, prio_lo), "create side stream");
+    FD_CUDA(cudaEventCreateWithFlags(&w.fork, cudaEventDisableTiming), "create fork event");
+    FD_CUDA(cudaEventCreateWithFlags(&w.join, cudaEventDisableTiming), "create join event");
+  }
   *out = p;
+  if (view) *view = w;
   return FD_OK;
 }
 
@@ -152,10 +167,12 @@ fd_status make_tmap(CUtensorMap* map, const void* base, int rank, const uint64_t
 }
 
 // ---------------------------------------------------------------------------- profiling ------
-// Per profiled call: events around the planner, the decode split kernel, the chunk tile kernel
-// (nothing for a decode call) and the combine kernel.
+// Per profiled call: a start and an end event around each of the planner, the decode split
+// kernel, the chunk tile kernel and the combine kernel (both at the same point for a launch the
+// call does not make). A chunked-prefill call records its split kernel's pair on its side stream.
 constexpr int kProfSegments = 4;
-constexpr int kProfEvents = kProfSegments + 1;
+constexpr int kProfEvents = 2 * kProfSegments;
+enum ProfSeg { kSegPlan = 0, kSegSplit = 1, kSegTiles = 2, kSegCombine = 3 };
 struct Profiler {
   std::mutex mu;
   std::vector<cudaEvent_t> ev;  // kProfEvents per call
@@ -345,7 +362,17 @@ void host_plan(const int32_t* lens_in, int B, int hkv, int cap, int fixed, int n
     hp->lens[b] = clamp_len(lens_in[b], cap);
     total += hp->lens[b];
   }
-  hp->chunk = fixed > 0 ? 0 : plan_chunk_tokens(total, hkv, nctas);
+  hp->chunk = 0;
+  if (fixed <= 0) {
+    int32_t chunks[kPlanWaveChoices];
+    int64_t sums[kPlanWaveChoices];
+    for (int i = 0; i < kPlanWaveChoices; ++i) {
+      chunks[i] = plan_chunk_for_waves(total, hkv, nctas, plan_waves(i));
+      sums[i] = 0;
+      for (int b = 0; b < B; ++b) sums[i] += plan_num_splits(hp->lens[b], chunks[i], 0);
+    }
+    hp->chunk = plan_pick_chunk(chunks, sums, hkv, nctas);
+  }
   std::vector<int32_t> key(B);
   hp->total_items = 0;
   for (int b = 0; b < B; ++b) {
@@ -358,8 +385,16 @@ void host_plan(const int32_t* lens_in, int B, int hkv, int cap, int fixed, int n
   std::stable_sort(hp->order.begin(), hp->order.end(), [&](int a, int c) { return key[a] > key[c]; });
 }
 
-void end_profile_events(cudaEvent_t* ev, int slot, cudaStream_t stream) {
-  if (ev) cudaEventRecord(ev[slot], stream);
+void prof_start(cudaEvent_t* ev, int seg, cudaStream_t stream) {
+  if (ev) cudaEventRecord(ev[2 * seg], stream);
+}
+void prof_end(cudaEvent_t* ev, int seg, cudaStream_t stream) {
+  if (ev) cudaEventRecord(ev[2 * seg + 1], stream);
+}
+// a segment the call does not launch: both events at this point of the stream
+void prof_empty(cudaEvent_t* ev, int seg, cudaStream_t stream) {
+  prof_start(ev, seg, stream);
+  prof_end(ev, seg, stream);
 }
 
 }  // namespace fd_abi
@@ -644,20 +679,22 @@ fd_status decode_call(const fd_tensor* q, const fd_tensor* k_cache, const fd_ten
   }
 
   cudaEvent_t* ev = prof_next();
-  end_profile_events(ev, 0, stream);
+  prof_start(ev, kSegPlan, stream);
   if (!fused_plan) FD_CUDA(launch_plan_decode(pp, stream), "plan kernel launch");
-  end_profile_events(ev, 1, stream);
+  prof_end(ev, kSegPlan, stream);
+  prof_start(ev, kSegSplit, stream);
   if (sh.use_tc) {
     FD_CUDA(launch_decode_tc(dp, tq, tk, tv, nctas, stream), "tensor-core split kernel launch");
   } else {
     FD_CUDA(launch_decode_simt(dp, sh.dtype, nctas, stream), "split kernel launch");
   }
-  end_profile_events(ev, 2, stream);
-  end_profile_events(ev, 3, stream);  // no chunk tiles in a decode call
+  prof_end(ev, kSegSplit, stream);
+  prof_empty(ev, kSegTiles, stream);  // no chunk tiles in a decode call
   // the CUDA-core kernel merges each group's partials itself; the tensor-core kernel leaves them
   // to the combine kernel
+  prof_start(ev, kSegCombine, stream);
   if (sh.use_tc) FD_CUDA(launch_combine(cp, stream), "combine kernel launch");
-  end_profile_events(ev, 4, stream);
+  prof_end(ev, kSegCombine, stream);
   return FD_OK;
 }
 
@@ -717,7 +754,7 @@ fd_status fd_chunk_prefill_attention(const fd_tensor* q_chunk, const fd_tensor* 
   const int hq = static_cast<int>(q_chunk->shape[1]);
   const int d = static_cast<int>(q_chunk->shape[2]);
   if (q_chunk->dtype != FD_BF16) return fail(FD_ERR_UNSUPPORTED, "chunked prefill needs bf16 tensors");
-  if (d != 128) return fail(FD_ERR_UNSUPPORTED, "chunked prefill supports head_dim 128, got %d", d);
+  if (d != 64 && d != 128) return fail(FD_ERR_UNSUPPORTED, "chunked prefill supports head_dim 64 and 128, got %d", d);
   if (!k_cache) return fail(FD_ERR_INVALID_ARGUMENT, "k_cache is NULL");
   const int B = static_cast<int>(k_cache->shape[0]);
   if ((s = check_kv(k_cache, v_cache, FD_BF16, B, d)) != FD_OK) return s;
@@ -727,6 +764,8 @@ fd_status fd_chunk_prefill_attention(const fd_tensor* q_chunk, const fd_tensor* 
     return fail(FD_ERR_INVALID_ARGUMENT, "q heads (%d) must be a positive multiple of KV heads (%d)", hq, hkv);
   const int g = hq / hkv;
   if (g > 16) return fail(FD_ERR_UNSUPPORTED, "group size %d above 16", g);
+  if (d == 64 && g > 8)
+    return fail(FD_ERR_UNSUPPORTED, "group size %d above 8 needs head_dim 128 (its decode rows run on tensor cores)", g);
   if (B > kMaxPlanBatch) return fail(FD_ERR_UNSUPPORTED, "batch %d exceeds %d", B, kMaxPlanBatch);
   if (T == 0) return FD_OK;
   if (B == 0) return fail(FD_ERR_INVALID_ARGUMENT, "q_chunk has %d rows but the cache has no request", T);
@@ -734,7 +773,9 @@ fd_status fd_chunk_prefill_attention(const fd_tensor* q_chunk, const fd_tensor* 
   if (!lse) return fail(FD_ERR_INVALID_ARGUMENT, "lse is NULL");
   int dev = 0;
   FD_CUDA(cudaGetDevice(&dev), "cudaGetDevice");
-  const bool dec_tc = g >= 2;  // decode rows of a group >= 2 use the tensor-core decode kernel
+  // decode rows of a group >= 2 with head_dim 128 use the tensor-core decode kernel, the others
+  // the CUDA-core one
+  const bool dec_tc = g >= 2 && d == 128;
   const int dec_ctas = decode_ctas(dev, dec_tc);
   const int tile_ctas = sm_count(dev);
   if (dec_ctas < 1 || tile_ctas < 1) return fail(FD_ERR_CUDA, "no multiprocessors reported for device %d", dev);
@@ -744,7 +785,8 @@ fd_status fd_chunk_prefill_attention(const fd_tensor* q_chunk, const fd_tensor* 
   const int64_t max_slots = chunk_max_slots(B, T, hkv, cap, dec_ctas);
   const WsLayout L = ws_layout(max_dec, max_tiles, static_cast<int64_t>(T) + 1, max_slots, hq, d, hkv);
   void* ws = nullptr;
-  if ((s = get_workspace(stream, L.total, &ws)) != FD_OK) return s;
+  Workspace wv;
+  if ((s = get_workspace(stream, L.total, &ws, &wv)) != FD_OK) return s;
   char* base = static_cast<char*>(ws);
   WsHeader* hdr = reinterpret_cast<WsHeader*>(base);
   DecodeItem* items = reinterpret_cast<DecodeItem*>(base + L.dec_items);
@@ -774,6 +816,8 @@ fd_status fd_chunk_prefill_attention(const fd_tensor* q_chunk, const fd_tensor* 
   pp.arrivals = arrivals;
   pp.total_rows = T;
   pp.decode_merged_in_kernel = dec_tc ? 0 : 1;
+  pp.tile_sms = tile_ctas;
+  pp.kv_key_bytes = 2ll * hkv * d * 2;
 
   DecodeParams dp{};
   dp.q = q_chunk->data;
@@ -861,20 +905,33 @@ fd_status fd_chunk_prefill_attention(const fd_tensor* q_chunk, const fd_tensor* 
   if ((s = make_tmap(&tv, v_cache->data, 4, kd, ks, kb, "v_cache")) != FD_OK) return s;
   if (dec_tc && (s = make_tmap(&tq_dec, q_chunk->data, 3, qd, qs, qb_dec, "q_chunk (decode rows)")) != FD_OK) return s;
 
+  // The planner, then the tile kernel on this stream beside the decode-row split kernel on the
+  // side stream (forked after the planner, joined before the combine): the planner keeps
+  // hdr->tile_ctas of the tile kernel's CTAs (the rest leave at once) so that the decode rows,
+  // bound by HBM, stream on the other multiprocessors while the tiles, bound by the tensor
+  // cores, run ("大语言模型长序列推理优化：ChunkedPrefill与FlashDecoding技术解析" §2.2: chunks
+  // scheduled together with decode requests).
   cudaEvent_t* ev = prof_next();
-  end_profile_events(ev, 0, stream);
+  prof_start(ev, kSegPlan, stream);
   FD_CUDA(launch_plan_chunk(pp, stream), "chunk plan kernel launch");
-  end_profile_events(ev, 1, stream);
-  if (dec_tc) {
-    FD_CUDA(launch_decode_tc(dp, tq_dec, tk, tv, dec_ctas, stream), "decode-row split kernel launch");
-  } else {
-    FD_CUDA(launch_decode_simt(dp, FD_BF16, dec_ctas, stream), "decode-row split kernel launch");
-  }
-  end_profile_events(ev, 2, stream);
+  prof_end(ev, kSegPlan, stream);
+  FD_CUDA(cudaEventRecord(wv.fork, stream), "record fork event");
+  prof_start(ev, kSegTiles, stream);
   FD_CUDA(launch_chunk_tc(tp, tq_tile, tq_packed, tk, tv, tile_ctas, stream), "chunk tile kernel launch");
-  end_profile_events(ev, 3, stream);
+  prof_end(ev, kSegTiles, stream);
+  FD_CUDA(cudaStreamWaitEvent(wv.side, wv.fork, 0), "side stream waits for the planner");
+  prof_start(ev, kSegSplit, wv.side);
+  if (dec_tc) {
+    FD_CUDA(launch_decode_tc(dp, tq_dec, tk, tv, dec_ctas, wv.side), "decode-row split kernel launch");
+  } else {
+    FD_CUDA(launch_decode_simt(dp, FD_BF16, dec_ctas, wv.side), "decode-row split kernel launch");
+  }
+  prof_end(ev, kSegSplit, wv.side);
+  FD_CUDA(cudaEventRecord(wv.join, wv.side), "record join event");
+  FD_CUDA(cudaStreamWaitEvent(stream, wv.join, 0), "stream waits for the decode rows");
+  prof_start(ev, kSegCombine, stream);
   FD_CUDA(launch_combine(cp, stream), "combine kernel launch");
-  end_profile_events(ev, 4, stream);
+  prof_end(ev, kSegCombine, stream);
   return FD_OK;
 }
 
@@ -942,9 +999,10 @@ fd_status fd_profile_end(float* ms, int32_t max_calls, int32_t* n_calls) {
   const int n = std::min(g_prof.calls, max_calls);
   for (int i = 0; i < n; ++i) {
     cudaEvent_t* e = &g_prof.ev[kProfEvents * static_cast<size_t>(i)];
-    FD_CUDA(cudaEventSynchronize(e[kProfSegments]), "cudaEventSynchronize");
-    for (int j = 0; j < kProfSegments; ++j)
-      FD_CUDA(cudaEventElapsedTime(&ms[kProfSegments * i + j], e[j], e[j + 1]), "cudaEventElapsedTime");
+    for (int j = 0; j < kProfSegments; ++j) {
+      FD_CUDA(cudaEventSynchronize(e[2 * j + 1]), "cudaEventSynchronize");
+      FD_CUDA(cudaEventElapsedTime(&ms[kProfSegments * i + j], e[2 * j], e[2 * j + 1]), "cudaEventElapsedTime");
+    }
   }
   *n_calls = n;
   for (cudaEvent_t e : g_prof.ev) cudaEventDestroy(e);
@@ -958,14 +1016,15 @@ void fd_shutdown(void) {
   {
     std::lock_guard<std::mutex> lock(g_mu);
     for (auto& kv : g_ws) {
-      if (kv.second.ptr) {
-        int cur = 0;
-        cudaGetDevice(&cur);
-        cudaSetDevice(kv.first.first);
-        cudaDeviceSynchronize();
-        cudaFree(kv.second.ptr);
-        cudaSetDevice(cur);
-      }
+      int cur = 0;
+      cudaGetDevice(&cur);
+      cudaSetDevice(kv.first.first);
+      cudaDeviceSynchronize();
+      if (kv.second.ptr) cudaFree(kv.second.ptr);
+      if (kv.second.side) cudaStreamDestroy(kv.second.side);
+      if (kv.second.fork) cudaEventDestroy(kv.second.fork);
+      if (kv.second.join) cudaEventDestroy(kv.second.join);
+      cudaSetDevice(cur);
     }
     g_ws.clear();
   }

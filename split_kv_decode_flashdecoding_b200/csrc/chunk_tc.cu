@@ -7,12 +7,14 @@
 // §三.2). Row r of the tile is chunk position pos0 + r and sees keys j <= prefix + pos0 + r.
 // Per 128-key tile of the split:
 //
-//   S[128 rows x 128 keys] = Q_tile · K_tileᵀ         UMMA M=128 N=128, both K-major (TMA SW128)
+//   S[128 rows x 128 keys] = Q_tile · K_tileᵀ         UMMA M=128 N=128 K=D, both K-major (TMA SW128)
 //   one thread per row: mask, running max m (rescaled lazily), p = 2^(s·scale·log2e − m),
 //   running sum l, P split into bf16 hi + lo (both rounded to nearest) and stored into tensor
 //   memory
-//   O_hi[128 x 128] += P_hi · V_tile, O_lo[128 x 128] += P_lo · V_tile
-//                                                        UMMA M=128 N=128, A from TMEM, V MN-major
+//   O_hi[128 x D] += P_hi · V_tile, O_lo[128 x D] += P_lo · V_tile
+//                                                        UMMA M=128 N=D, A from TMEM, V MN-major
+//
+// with head_dim D = 64 or 128 (one instantiation each).
 //
 // S is double-buffered in TMEM and P is written back over the S buffer it came from (per
 // 32-key chunk: 16 words of hi pairs, then 16 words of lo pairs), so P is double-buffered too.
@@ -48,7 +50,6 @@ namespace {
 
 constexpr int kCkRows = 128;   // query rows per tile = UMMA M
 constexpr int kCkKeys = 128;   // keys per key tile = N of S, K of P·V
-constexpr int kCkD = 128;      // head dim = K of S, N of P·V
 constexpr int kCkKStages = 2;
 constexpr int kCkVStages = 2;
 constexpr int kCkProducer = 4;     // Q and K
@@ -58,15 +59,19 @@ constexpr int kCkPv = 11;          // issues the P·V products (warp 5 the S pro
 constexpr int kCkThreads = 12 * 32;
 constexpr uint32_t kCkTmemCols = 512;
 constexpr uint32_t kColS0 = 0;     // S/P buffers at columns 0 and 128
-constexpr uint32_t kColOHi = 256;  // O accumulator of the P_hi products
-constexpr uint32_t kColOLo = 384;  // O accumulator of the P_lo products
+constexpr uint32_t kColOHi = 256;  // O accumulator of the P_hi products (D columns); the
+                                   // P_lo accumulator follows at kColOHi + D
 constexpr uint32_t kCkHalf = kCkRows * 64 * 2;  // one 64-column half of a 128-row tile
 constexpr float kRescaleThreshold = 8.0f;       // log2 units
 
+// kD = head dim (64 or 128) = K of S, N of P·V; rows of Q, K and V are held in kD / 64
+// 64-column halves (one 128-byte swizzle row each).
+template <int kD>
 struct __align__(1024) CkSmem {
-  __nv_bfloat16 q[2][2][kCkRows * 64];           // [item parity][d half], SW128
-  __nv_bfloat16 k[kCkKStages][2][kCkKeys * 64];  // [stage][d half], SW128
-  __nv_bfloat16 v[kCkVStages][2][kCkKeys * 64];
+  static constexpr int kHalves = kD / 64;
+  __nv_bfloat16 q[2][kHalves][kCkRows * 64];           // [item parity][d half], SW128
+  __nv_bfloat16 k[kCkKStages][kHalves][kCkKeys * 64];  // [stage][d half], SW128
+  __nv_bfloat16 v[kCkVStages][kHalves][kCkKeys * 64];
   int32_t meta[kCkKStages];                      // valid keys of the K stage (MMA warp)
   int32_t item_slot[2][2];                       // item index (-1: stop), key tiles
   TileItem item[2];
@@ -87,23 +92,34 @@ struct __align__(1024) CkSmem {
   uint32_t tmem_base;
   int abort_flag;
 };
-static_assert(sizeof(CkSmem) + 1024 <= 227 * 1024, "chunk tile kernel shared memory");
+static_assert(sizeof(CkSmem<128>) + 1024 <= 227 * 1024, "chunk tile kernel shared memory");
+static_assert(kColOHi + 2 * 128 <= kCkTmemCols, "chunk tile kernel tensor memory");
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
   const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
   return *reinterpret_cast<const uint32_t*>(&h);
 }
 
+template <int kD>
 __global__ void __launch_bounds__(kCkThreads, 1)
     chunk_tc_kernel(const TileParams p, const __grid_constant__ CUtensorMap tmap_q,
                     const __grid_constant__ CUtensorMap tmap_qp,
                     const __grid_constant__ CUtensorMap tmap_k,
                     const __grid_constant__ CUtensorMap tmap_v) {
+  using Smem = CkSmem<kD>;
+  constexpr int kHalves = Smem::kHalves;
+  constexpr uint32_t kColOLo = kColOHi + kD;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
-  CkSmem& S = *reinterpret_cast<CkSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  Smem& S = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
   const int lane = tid & 31;
+
+  // The planner chose how many CTAs this kernel keeps: the decode rows of the same call run
+  // beside it on the other multiprocessors, so the rest leave before taking any resource.
+  pdl_wait_prerequisites();
+  pdl_launch_dependents();
+  if (static_cast<int>(blockIdx.x) >= *reinterpret_cast<volatile int32_t*>(&p.hdr->tile_ctas)) return;
 
   if (tid == 0) {
     for (int s = 0; s < kCkKStages; ++s) {
@@ -146,9 +162,7 @@ __global__ void __launch_bounds__(kCkThreads, 1)
   tc_fence_after();
   const uint32_t tmem = S.tmem_base;
   const WaitCtx ctx{&S.abort_flag, &p.hdr->status};
-  pdl_wait_prerequisites();
-  pdl_launch_dependents();
-  const uint32_t kv_tx = 2u * 128u * static_cast<uint32_t>(p.kv_box_rows);
+  const uint32_t kv_tx = kHalves * 128u * static_cast<uint32_t>(p.kv_box_rows);
 
   if (warp == kCkProducer) {
     // ======================= TMA producer of Q and K =======================
@@ -173,13 +187,15 @@ __global__ void __launch_bounds__(kCkThreads, 1)
         S.item[ps] = it;
         if (it.head_packed) {
           // G heads x qp_box_rows chunk rows, rows ordered (chunk row, head)
-          mbar_arrive_expect_tx(&S.qfull[ps], 2u * 128u * static_cast<uint32_t>(p.g * p.qp_box_rows));
-          tma_load_3d(S.q[ps][0], &tmap_qp, &S.qfull[ps], 0, it.h * p.g, it.row0);
-          tma_load_3d(S.q[ps][1], &tmap_qp, &S.qfull[ps], 64, it.h * p.g, it.row0);
+          mbar_arrive_expect_tx(&S.qfull[ps], kHalves * 128u * static_cast<uint32_t>(p.g * p.qp_box_rows));
+#pragma unroll
+          for (int hf = 0; hf < kHalves; ++hf)
+            tma_load_3d(S.q[ps][hf], &tmap_qp, &S.qfull[ps], 64 * hf, it.h * p.g, it.row0);
         } else {
-          mbar_arrive_expect_tx(&S.qfull[ps], 2u * 128u * static_cast<uint32_t>(p.q_box_rows));
-          tma_load_3d(S.q[ps][0], &tmap_q, &S.qfull[ps], 0, it.h, it.row0);
-          tma_load_3d(S.q[ps][1], &tmap_q, &S.qfull[ps], 64, it.h, it.row0);
+          mbar_arrive_expect_tx(&S.qfull[ps], kHalves * 128u * static_cast<uint32_t>(p.q_box_rows));
+#pragma unroll
+          for (int hf = 0; hf < kHalves; ++hf)
+            tma_load_3d(S.q[ps][hf], &tmap_q, &S.qfull[ps], 64 * hf, it.h, it.row0);
         }
         const int hkv = it.head_packed ? it.h : it.h / p.g;
         for (int j = 0; j < ntile; ++j, ++J) {
@@ -191,8 +207,9 @@ __global__ void __launch_bounds__(kCkThreads, 1)
           S.meta[st] = valid;
           if (valid > 0) {
             mbar_arrive_expect_tx(&S.kfull[st], kv_tx);
-            tma_load_4d_stream(S.k[st][0], &tmap_k, &S.kfull[st], 0, t, hkv, it.b, pol);
-            tma_load_4d_stream(S.k[st][1], &tmap_k, &S.kfull[st], 64, t, hkv, it.b, pol);
+#pragma unroll
+            for (int hf = 0; hf < kHalves; ++hf)
+              tma_load_4d_stream(S.k[st][hf], &tmap_k, &S.kfull[st], 64 * hf, t, hkv, it.b, pol);
           } else {
             mbar_arrive(&S.kfull[st]);
           }
@@ -240,8 +257,9 @@ __global__ void __launch_bounds__(kCkThreads, 1)
           const int valid = max(0, min(kCkKeys, it.k1 - t));
           if (valid > 0) {
             mbar_arrive_expect_tx(&S.vfull[st], kv_tx);
-            tma_load_4d_stream(S.v[st][0], &tmap_v, &S.vfull[st], 0, t, hkv, it.b, pol);
-            tma_load_4d_stream(S.v[st][1], &tmap_v, &S.vfull[st], 64, t, hkv, it.b, pol);
+#pragma unroll
+            for (int hf = 0; hf < kHalves; ++hf)
+              tma_load_4d_stream(S.v[st][hf], &tmap_v, &S.vfull[st], 64 * hf, t, hkv, it.b, pol);
           } else {
             mbar_arrive(&S.vfull[st]);
           }
@@ -269,7 +287,7 @@ __global__ void __launch_bounds__(kCkThreads, 1)
         const int ntile = S.item_slot[ps][1];
         if (idx < 0) break;
         const uint32_t q0 = smem_u32(S.q[ps][0]);
-        const uint32_t q1 = smem_u32(S.q[ps][1]);
+        const uint32_t q1 = smem_u32(S.q[ps][kHalves - 1]);
         for (int j = 0; j < ntile; ++j, ++J) {
           const int st = J % kCkKStages;
           const int sb = J & 1;
@@ -280,9 +298,9 @@ __global__ void __launch_bounds__(kCkThreads, 1)
           const int valid = S.meta[st];
           if (valid > 0) {
             const uint32_t k0 = smem_u32(S.k[st][0]);
-            const uint32_t k1 = smem_u32(S.k[st][1]);
+            const uint32_t k1 = smem_u32(S.k[st][kHalves - 1]);
 #pragma unroll
-            for (int kk = 0; kk < kCkD / 16; ++kk) {
+            for (int kk = 0; kk < kD / 16; ++kk) {
               const uint32_t qa = (kk < 4 ? q0 : q1) + (kk & 3) * 32;
               const uint32_t ka = (kk < 4 ? k0 : k1) + (kk & 3) * 32;
               umma_bf16_ss(tmem + kColS0 + sb * 128, smem_desc(qa, 16, 1024, kLayoutSW128),
@@ -304,7 +322,7 @@ __global__ void __launch_bounds__(kCkThreads, 1)
     // ======================= P·V issuer =======================
     // Follows the items the Q/K producer publishes; each tile's keys come from the item.
     if (lane == 0) {
-      const uint32_t idesc_o = idesc_bf16_f32(kCkRows, kCkD, false, true);
+      const uint32_t idesc_o = idesc_bf16_f32(kCkRows, kD, false, true);
       uint32_t J = 0, K = 0;
       bool ok = true;
       while (ok) {
@@ -432,7 +450,7 @@ __global__ void __launch_bounds__(kCkThreads, 1)
           tc_fence_after();
           const uint32_t oc = tmem + lane_base + kColOHi;  // O_hi, then O_lo right after it
 #pragma unroll 1
-          for (int c = 0; c < 2 * kCkD; c += 32) {
+          for (int c = 0; c < 2 * kD; c += 32) {
             uint32_t o[32];
             tmem_ld32(oc + c, o);
             tmem_wait_ld();
@@ -488,9 +506,9 @@ __global__ void __launch_bounds__(kCkThreads, 1)
           const int vs = J % kCkVStages;
           if (!mbar_wait(&S.vfull[vs], (J / kCkVStages) & 1u, ctx)) { ok = false; break; }
           const int r0 = valid, r1 = (valid + 15) & ~15;
-          for (int c = tid; c < (r1 - r0) * 16; c += 128) {
-            const int row = r0 + c / 16;
-            *reinterpret_cast<uint4*>(reinterpret_cast<unsigned char*>(S.v[vs][(c / 8) & 1]) +
+          for (int c = tid; c < (r1 - r0) * 8 * kHalves; c += 128) {
+            const int row = r0 + c / (8 * kHalves);
+            *reinterpret_cast<uint4*>(reinterpret_cast<unsigned char*>(S.v[vs][(c / 8) % kHalves]) +
                                       row * 128 + (c & 7) * 16) = make_uint4(0u, 0u, 0u, 0u);
           }
           fence_proxy_async_smem();
@@ -538,10 +556,10 @@ __global__ void __launch_bounds__(kCkThreads, 1)
                            (static_cast<int64_t>(pos) * p.hkv + hkv) * it.nsplit + it.split;
       __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out) + row * p.o_sr +
                            static_cast<int64_t>(head) * p.o_sh;
-      float* dst = p.part_o + (slot * p.g + g) * kCkD;
+      float* dst = p.part_o + (slot * p.g + g) * kD;
       // O = O_hi + O_lo, 32 columns at a time
 #pragma unroll 1
-      for (int c = 0; c < kCkD; c += 32) {
+      for (int c = 0; c < kD; c += 32) {
         uint32_t o[32], lo[32];
         tmem_ld32(tmem + lane_base + kColOHi + c, o);
         tmem_ld32(tmem + lane_base + kColOLo + c, lo);
@@ -585,13 +603,12 @@ __global__ void __launch_bounds__(kCkThreads, 1)
   if (warp == kCkMma) tmem_dealloc(tmem, kCkTmemCols);
 }
 
-}  // namespace
-
-cudaError_t launch_chunk_tc(const TileParams& p, const CUtensorMap& tq, const CUtensorMap& tqp,
-                            const CUtensorMap& tk, const CUtensorMap& tv, int nctas,
-                            cudaStream_t stream) {
-  const size_t smem = sizeof(CkSmem) + 1024;
-  cudaError_t e = cudaFuncSetAttribute(chunk_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+template <int kD>
+cudaError_t launch_chunk_tc_t(const TileParams& p, const CUtensorMap& tq, const CUtensorMap& tqp,
+                              const CUtensorMap& tk, const CUtensorMap& tv, int nctas,
+                              cudaStream_t stream) {
+  const size_t smem = sizeof(CkSmem<kD>) + 1024;
+  cudaError_t e = cudaFuncSetAttribute(chunk_tc_kernel<kD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg{};
@@ -604,7 +621,17 @@ cudaError_t launch_chunk_tc(const TileParams& p, const CUtensorMap& tq, const CU
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, chunk_tc_kernel, p, tq, tqp, tk, tv);
+  return cudaLaunchKernelEx(&cfg, chunk_tc_kernel<kD>, p, tq, tqp, tk, tv);
+}
+
+}  // namespace
+
+cudaError_t launch_chunk_tc(const TileParams& p, const CUtensorMap& tq, const CUtensorMap& tqp,
+                            const CUtensorMap& tk, const CUtensorMap& tv, int nctas,
+                            cudaStream_t stream) {
+  if (p.d == 128) return launch_chunk_tc_t<128>(p, tq, tqp, tk, tv, nctas, stream);
+  if (p.d == 64) return launch_chunk_tc_t<64>(p, tq, tqp, tk, tv, nctas, stream);
+  return cudaErrorInvalidValue;
 }
 
 }  // namespace fd

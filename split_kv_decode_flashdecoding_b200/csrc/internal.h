@@ -25,6 +25,8 @@ struct PlanParams {
   int32_t* arrivals;        // [rows * Hkv] split-completion counters of the in-kernel merge
   int32_t total_rows;       // chunk mode: packed query rows T (= sum of chunk lengths)
   int32_t decode_merged_in_kernel;  // chunk mode: decode rows merge inside their split kernel
+  int32_t tile_sms;         // chunk mode: multiprocessors the tile kernel is launched on
+  int64_t kv_key_bytes;     // chunk mode: K + V bytes of one key over all KV heads
   // optional export of the decode plan (fd_split_plan_device)
   int32_t* out_splits;
   int32_t* out_items;
@@ -131,7 +133,7 @@ cudaError_t launch_decode_tc(const DecodeParams& p, const CUtensorMap& tmap_q,
                              const CUtensorMap& tmap_k, const CUtensorMap& tmap_v, int nctas,
                              cudaStream_t stream);
 
-// tcgen05 chunked-prefill tile kernel: bf16, D == 128. tmap_qp loads head-packed Q tiles
+// tcgen05 chunked-prefill tile kernel: bf16, D == 64 or 128. tmap_qp loads head-packed Q tiles
 // (G heads x qp_box_rows rows); any Q map when no tile is head-packed.
 cudaError_t launch_chunk_tc(const TileParams& p, const CUtensorMap& tmap_q,
                             const CUtensorMap& tmap_qp, const CUtensorMap& tmap_k,

@@ -225,3 +225,25 @@ def test_fp8_paged_rejects_bad_arguments_on_host():
     k1, v1 = _fake([8, 1, P, D], fd.FD_E4M3), _fake([8, 1, P, D], fd.FD_E4M3)
     assert _paged_fp8(q16, k1, v1) == fd.FD_ERR_UNSUPPORTED
     assert "group size" in fd.lib.fd_last_error_message().decode()
+
+
+def _chunk(q, k, v, out, prefix=0x200000, chunk=0x200100, lse=0x300000):
+    ip = lambda a: ctypes.cast(ctypes.c_void_p(a), ctypes.POINTER(ctypes.c_int32)) if a else None
+    sp = ctypes.cast(ctypes.c_void_p(lse), ctypes.POINTER(ctypes.c_float)) if lse else None
+    return fd.lib.fd_chunk_prefill_attention(ctypes.byref(q), ctypes.byref(k), ctypes.byref(v),
+                                             ip(prefix), ip(chunk), ctypes.byref(out), sp, None)
+
+
+def test_chunk_rejects_bad_arguments_on_host():
+    B, T, S = 2, 5, 64
+    # head_dim 96 and fp32 are unsupported; head_dim 64 with a group above 8 too (its decode rows
+    # would need the CUDA-core kernel, which serves groups up to 8)
+    for D, hq, hkv, dt in [(96, 8, 2, fd.FD_BF16), (128, 8, 2, fd.FD_F32), (64, 32, 2, fd.FD_BF16)]:
+        q, o = _fake([T, hq, D], dt), _fake([T, hq, D], dt)
+        k, v = _fake([B, hkv, S, D], dt), _fake([B, hkv, S, D], dt)
+        assert _chunk(q, k, v, o) == fd.FD_ERR_UNSUPPORTED, (D, hq, hkv, dt)
+    # missing lengths or lse
+    q, o = _fake([T, 8, 64]), _fake([T, 8, 64])
+    k, v = _fake([B, 2, S, 64]), _fake([B, 2, S, 64])
+    assert _chunk(q, k, v, o, prefix=0) == fd.FD_ERR_INVALID_ARGUMENT
+    assert _chunk(q, k, v, o, lse=0) == fd.FD_ERR_INVALID_ARGUMENT

@@ -69,6 +69,27 @@ def test_small_chunks(case):
     check_lse(lse, rl, "chunk lse")
 
 
+# head_dim 64: the tile kernel's D = 64 instantiation; decode rows of any group run on CUDA cores
+CASES_D64 = [
+    # (prefix_lens, chunk_lens, Hq, Hkv, cap)
+    ([300], [130], 2, 2, 512),                     # two tiles, ragged second tile
+    ([1900, 10, 0], [300, 1, 1], 4, 4, 2304),      # two key splits per tile + decode rows
+    ([1000, 77, 4000], [129, 1, 1], 16, 2, 4200),  # GQA (G = 8)
+    ([3000, 5], [4, 4], 32, 8, 3072),              # verification, head-packed tiles (G = 4)
+]
+
+
+@pytest.mark.parametrize("case", range(len(CASES_D64)))
+def test_small_chunks_head_dim_64(case):
+    prefix, chunk, hq, hkv, cap = CASES_D64[case]
+    inp = make_chunk_inputs(prefix, chunk, hq, hkv, 64, cap, torch.bfloat16, seed=400 + case,
+                            pad_fill=NAN)
+    out, lse = _run(inp)
+    ro, rl = _oracle(inp)
+    check_out(out, ro, "chunk D 64 out")
+    check_lse(lse, rl, "chunk D 64 lse")
+
+
 def test_chunk_equals_decode_rows():
     # a chunk of 3 rows at prefix p gives, row by row, the decode results over p + i + 1 keys
     import split_kv_decode_flashdecoding_b200 as fd
