@@ -200,7 +200,7 @@ FD_HD int32_t chunk_tile_splits(int32_t keys) {
 // total: the time of phase 1 plus that of the rest. `key_tiles` counts the 128-key tiles of all
 // tile items, `dec_bytes` the K/V bytes of the decode rows. No tiles: 0; no decode rows: nsm.
 constexpr float kTileKeyTileUs = 2.3f;  // 250 µs for workload 5's 16192 key tiles on 148 CTAs
-constexpr float kDecodeSmGBs = 51.f;    // CUDA-core decode rows beside 93 tile CTAs: 1.13 GB in 401 µs on 55 SMs
+constexpr float kDecodeSmGBs = 45.f;    // tensor-core decode rows beside 80 tile CTAs: ~1.4 GB in 465 µs on 68 SMs
 constexpr float kHbmGBs = 6000.f;       // decode rows alone on the whole device
 FD_HD int32_t chunk_tile_ctas(int64_t key_tiles, int64_t dec_bytes, int32_t nsm) {
   if (key_tiles <= 0) return 0;

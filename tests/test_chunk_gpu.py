@@ -133,6 +133,9 @@ VERIFY = [
     ([257, 0], [3, 5], 6, 2, 320),                           # G = 3: rows r // 3 and r % 3
     ([900, 40], [8, 8], 16, 1, 1024),                        # G = 16, k = 8 fills the tile
     ([2200, 10], [64, 33], 4, 2, 2304),                      # G = 2, k = 64 (full) and 33
+    ([6000, 17], [2, 2], 32, 2, 6144),                       # G = 16, k = 2 (32 rows), many splits
+    ([1500, 3000], [16, 9], 4, 2, 3072),                     # G = 2, k = 16 and 9
+    ([100, 2500, 40], [8, 5, 1], 32, 8, 2560),               # G = 4 with a decode row
 ]
 
 

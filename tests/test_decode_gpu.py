@@ -268,3 +268,20 @@ def test_paths_share_workspace_cursor():
                  lambda: decode_call(gqa), lambda: decode_call(mha), lambda: decode_call(gqa)):
         step()
     assert fd.fd_poll_status(stream=s) & (fd.FD_FLAG_WAIT_TIMEOUT | fd.FD_FLAG_PLAN_OVERFLOW) == 0
+
+
+def test_many_kv_heads_then_small_calls():
+    # 256 sequences x 257 KV heads (G = 2, 65792 groups, the in-kernel plan's largest batch)
+    # between two small calls on the same stream: all three match the oracle
+    rng = np.random.default_rng(4242)
+    B, hkv = 256, 257
+    lens = [int(x) for x in rng.integers(0, 33, size=B)]
+    big = make_decode_inputs(B, 2 * hkv, hkv, 128, 32, lens, torch.bfloat16, seed=4243,
+                             pad_fill=NAN)
+    small = make_decode_inputs(3, 64, 8, 128, 700, [700, 5, 300], torch.bfloat16, seed=4244,
+                               pad_fill=NAN)
+    for inp, ns in ((small, 4), (big, 2), (small, 0)):
+        out, lse = _run(inp, ns)
+        ro, rl = _oracle(inp)
+        check_out(out, ro, f"B {inp.q.shape[0]} x {inp.k_cache.shape[1]} KV heads out")
+        check_lse(lse, rl, f"B {inp.q.shape[0]} x {inp.k_cache.shape[1]} KV heads lse")
