@@ -385,7 +385,9 @@ def run_fd(args, rank, world, local_rank):
     input_bytes = sum(t.numel() * t.element_size() for t in (q, k, v))
     l2_policy = ("inputs larger than L2 (valid K/V bytes per call exceed the 126 MB L2)"
                  if alg > 2 * L2_BYTES else "inputs smaller than L2: measured with warm L2")
-    use_tc = (inp.k_cache.dtype == torch.bfloat16 and d == 128 and 2 <= g <= 16) or \
+    # the tensor-core split kernel: decode calls of bf16 groups of 2..16 (or any E4M3 group of
+    # <= 8) with head_dim 128, and the decode rows of every chunked call with head_dim 128
+    use_tc = (inp.k_cache.dtype == torch.bfloat16 and d == 128 and (chunk or 2 <= g <= 16)) or \
              (fp8 and d == 128 and g <= 8)
     if chunk:
         # planner, decode-row split kernel, chunk tile kernel, combine
@@ -487,7 +489,8 @@ def run_fd(args, rank, world, local_rank):
                        "peak": tpeak, "unit": "TFLOP/s", "frac": round(ach / tpeak, 4),
                        "peak_kind": f"{tkind} dense bf16 (burst)",
                        "algorithmic_flops_per_launch": flops,
-                       "traffic": traffic_from_profiles("chunk_tc.cu", inp.name)}
+                       "traffic": traffic_from_profiles("chunk_tc.cu", inp.name),
+                       "kernel_ms": roofline["kernel_ms"]}
         hb = tile_bytes / (tile_ms * 1e-3) / 1e9
         hbm_view = {"bound": "hbm", "kernel": "chunk_tc_kernel", "achieved": round(hb, 1),
                     "peak": peak, "unit": "GB/s", "frac": round(hb / peak, 4),
@@ -599,6 +602,10 @@ def run_fd(args, rank, world, local_rank):
         }
         if roofline_tiles is not None:
             line["roofline_secondary"] = roofline_tiles
+        if chunk:
+            line["note"] = ("the tile kernel and the decode-row split kernel run side by side (the "
+                            "planner splits the multiprocessors between them); each kernel's "
+                            "duration is measured while they share the device")
         emit(line, rank)
     return 0
 

@@ -27,13 +27,17 @@
 // or poisoned cache rows never leak. The epilogue of an item overlaps the next item's tiles.
 //
 // E4M3 cache (FlashDecoding page, "与其他推理加速方案的组合使用", item "Quantization +
-// FlashDecoding": scores on values dequantized to bf16). The TMA brings a tile's one-byte codes
-// into a staging area and eight more warps expand them exactly, side by side: four K to bf16
-// straight into tensor memory, where the Sᵀ product takes it as its A operand (so the expanded K
-// never costs shared-memory bandwidth), four V in place to f16 (one hardware conversion per pair
-// of codes; every E4M3 value is exact in f16 as in bf16). The P·V product of this instantiation
-// runs on f16 operands, P split into f16 hi + lo. The key scale is folded into the score scale
-// and the value scale into the output; everything else is the bf16 kernel.
+// FlashDecoding": scores on dequantized values). The Sᵀ product runs on the codes themselves
+// (tcgen05 kind::f8f6f4, K-step 32): the TMA brings a tile's K codes into shared memory with the
+// 128-byte swizzle and they are the product's A operand as they are. Q goes in as two E4M3 terms
+// per head, q = 2^e (c1 + c2): c1 = E4M3(q / 2^e), c2 = E4M3(q / 2^e - c1), e chosen so the head's
+// largest |q| / 2^e lies in [128, 256); a bf16 value's 8 significant bits fit in the two 4-bit
+// terms, so the split is exact but for values under 2^-9 of the head's scale. Columns 0-7 of Sᵀ
+// are K·c1ᵀ, columns 8-15 K·c2ᵀ; the softmax adds them and applies 2^e. Four warps make the Q
+// terms per item, four more expand V in place to f16 (one hardware conversion per pair of codes;
+// every E4M3 value is exact in f16), and the P·V product runs on f16 operands, P split into f16
+// hi + lo. The key scale is folded into the score scale and the value scale into the output;
+// everything else is the bf16 kernel.
 #include "common.cuh"
 #include "internal.h"
 
@@ -49,7 +53,7 @@ constexpr int kMmaWarp = 5;
 constexpr int kVProducerWarp = 10;
 constexpr int kPvWarp = 11;             // issues the P·V products (warp 5 the Sᵀ products)
 constexpr int kTcThreads = 12 * 32;
-constexpr int kConvWarp0 = 12;          // E4M3 cache: warps 12-15 expand K, 16-19 expand V
+constexpr int kConvWarp0 = 12;          // E4M3 cache: warps 12-15 split Q, 16-19 expand V
 constexpr int kF8Threads = 20 * 32;
 constexpr int kSoftmaxThreads = 128;
 constexpr uint32_t kTmemCols = 128;
@@ -70,6 +74,10 @@ struct __align__(1024) TcSmem {
   __nv_bfloat16 k[kStages][kKSlabs][kTcKeys * 64];  // [stage][d half][row*64 + col], SW128
   __nv_bfloat16 v[kStages][2][kTcKeys * 64];
   __nv_bfloat16 q[2][2][16 * 64];                // [item parity][d half], SW128
+  // E4M3 cache: Q as two E4M3 terms per head (rows 0-7 c1, rows 8-15 c2; 128 codes per row,
+  // SW128), by item parity, and each head's scale 2^e
+  unsigned char q8[kF8 ? 2 : 1][kF8 ? 16 * 128 : 16];
+  float qscale[2][GPAD];
   __nv_bfloat16 p[2][kPGroups * kTcKeys * 8];    // [tile parity], MN-major core matrices
   float wmax[2][4][GPAD];
   // hand-off to the epilogue warps, by item parity
@@ -96,9 +104,11 @@ struct __align__(1024) TcSmem {
   uint64_t ofin[2];    // by item parity: the item's last P·V product has completed
   uint64_t oempty[2];  // by item parity: the epilogue has read that item's O accumulator
   uint64_t lready[2], lfree[2];  // by item parity: hand-off written / read
-  // E4M3 cache: the TMA completes these (codes in the staging area); kfull / vfull then mean
-  // "expanded to bf16" and are completed by the four expanding warps
-  uint64_t kraw[kStages], vraw[kStages];
+  // E4M3 cache: the TMA completes vraw (V codes in the upper half of the stage); vfull then
+  // means "expanded to f16" and is completed by the four expanding warps. q8full: the item's Q
+  // terms are ready (the four Q warps).
+  uint64_t vraw[kStages];
+  uint64_t q8full[2];
   // paged cache: physical page ids of tile J in slot J mod kPidSlots, copied asynchronously by
   // the Q/K producer two tiles ahead (pidfull) and released by the V producer (pidempty)
   int32_t pid[kPidSlots][kMaxPageBoxes];
@@ -192,29 +202,6 @@ template <bool kF8>
 __device__ __forceinline__ uint32_t paged_tile_bytes(const TilePages& tp, const DecodeParams& p) {
   const int rows = p.page_size >= kTcKeys ? kTcKeys : p.page_size;
   return (kF8 ? 1u : 2u) * 128u * static_cast<uint32_t>(rows * tp.n);
-}
-
-// Four E4M3 codes (the bytes of w, the first in the low byte) as two bf16 pairs, exactly. For a
-// code s.eeee.mmm the 16-bit pattern s.0000eeee.mmm0000 is a bf16 whose value is the code's
-// value times 2^-120 (a subnormal code, eeee = 0, lands on a bf16 subnormal the same way), and
-// one bf16 multiply by 2^120 restores it. The byte permute puts each code in the high byte of a
-// 16-bit lane with the code's sign replicated in the byte above the lower lane, so one
-// arithmetic shift and one mask place every bit. The NaN codes come out as +-480.
-__device__ __forceinline__ void e4m3x4_to_bf16(uint32_t w, uint32_t& lo, uint32_t& hi) {
-  uint32_t t0, t1;
-  asm("prmt.b32 %0, %1, %2, 0x1804;" : "=r"(t0) : "r"(w), "r"(0u));  // [0, c0, sign(c0), c1]
-  asm("prmt.b32 %0, %1, %2, 0x3A24;" : "=r"(t1) : "r"(w), "r"(0u));  // [0, c2, sign(c2), c3]
-  t0 = static_cast<uint32_t>(static_cast<int32_t>(t0) >> 4) & 0x87F087F0u;
-  t1 = static_cast<uint32_t>(static_cast<int32_t>(t1) >> 4) & 0x87F087F0u;
-  const uint32_t two120 = 0x7B807B80u;  // bf16 2^120 in both lanes
-  __nv_bfloat162 a, b, k;
-  memcpy(&a, &t0, 4);
-  memcpy(&b, &t1, 4);
-  memcpy(&k, &two120, 4);
-  a = __hmul2(a, k);
-  b = __hmul2(b, k);
-  memcpy(&lo, &a, 4);
-  memcpy(&hi, &b, 4);
 }
 
 // Four E4M3 codes (the bytes of w, the first in the low byte) as two f16 pairs, exactly, by the
@@ -315,10 +302,8 @@ __global__ void __launch_bounds__(kF8 ? kF8Threads : kTcThreads, 1)
   constexpr int kStages = Smem::kStages;
   constexpr int kThreads = kF8 ? kF8Threads : kTcThreads;
   constexpr uint32_t kColO = 32;  // Sᵀ buffers at columns [0, 32), O accumulators after them
-  // E4M3 cache: the expanded K tile of each stage (128 key lanes x 64 columns of bf16 pairs)
-  constexpr uint32_t kColK = kColO + 2 * kNO;
-  constexpr uint32_t kCols = kF8 ? 512 : kTmemCols;
-  static_assert(!kF8 || kColK + kStages * 64 <= kCols, "tensor memory of the E4M3 kernel");
+  constexpr uint32_t kCols = kTmemCols;
+  static_assert(kColO + 2 * kNO <= kCols, "tensor memory of the decode kernel");
   static_assert(!kF8 || GPAD == 8, "the E4M3 kernel serves groups of <= 8 heads");
   constexpr uint32_t kRowBytes = kF8 ? 128u : 256u;  // bytes of one cached K or V row
   extern __shared__ __align__(1024) unsigned char smem_raw[];
@@ -330,16 +315,17 @@ __global__ void __launch_bounds__(kF8 ? kF8Threads : kTcThreads, 1)
 
   if (tid == 0) {
     for (int s = 0; s < kStages; ++s) {
-      mbar_init(&S.kfull[s], kF8 ? 4 : 1);
+      mbar_init(&S.kfull[s], 1);
       mbar_init(&S.vfull[s], kF8 ? 4 : 1);
       mbar_init(&S.kempty[s], 1);
       mbar_init(&S.vempty[s], 1);
-      mbar_init(&S.kraw[s], 1);
       mbar_init(&S.vraw[s], 1);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&S.qfull[i], 1);
-      mbar_init(&S.qempty[i], 1 + 4 + 1 + 1);  // Sᵀ issuer, softmax warps, V producer, P·V issuer
+      // Sᵀ issuer, softmax warps, V producer, P·V issuer (and the four Q warps of an E4M3 cache)
+      mbar_init(&S.qempty[i], kF8 ? 1 + 4 + 1 + 1 + 4 : 1 + 4 + 1 + 1);
+      mbar_init(&S.q8full[i], 4);
       mbar_init(&S.sfull[i], 1);
       mbar_init(&S.sempty[i], 4);
       mbar_init(&S.pfull[i], 4);
@@ -594,8 +580,7 @@ __global__ void __launch_bounds__(kF8 ? kF8Threads : kTcThreads, 1)
           }
           S.meta[st][0] = t;
           S.meta[st][1] = valid;
-          // bf16: the copy completes kfull; E4M3: it completes kraw, the expanding warps kfull
-          uint64_t* kbar = kF8 ? &S.kraw[st] : &S.kfull[st];
+          uint64_t* kbar = &S.kfull[st];  // the copy completes kfull (E4M3: the codes as they are)
           if (valid > 0) {
             if constexpr (paged) {
               if constexpr (big_pages) {
@@ -631,22 +616,13 @@ __global__ void __launch_bounds__(kF8 ? kF8Threads : kTcThreads, 1)
           S.item_slot[ps][1] = 0;
           mbar_arrive(&S.qfull[ps]);
         }
-        if constexpr (kF8) {
-          // the expanding warps follow the stages, not the items: a stage without a tile (valid
-          // -1) stops them, once the stage's previous tile has been consumed
-          const int st = J % kStages;
-          if (mbar_wait(&S.kempty[st], ((J / kStages) & 1u) ^ 1u, ctx)) {
-            S.meta[st][1] = -1;
-            mbar_arrive(&S.kraw[st]);
-          }
-        }
       }
       if constexpr (paged) asm volatile("cp.async.wait_all;" ::: "memory");
       if (S.abort_flag) {
         // let copies already issued land before shared memory is released
         for (uint32_t back = 1; back <= kStages && back <= J; ++back) {
           const uint32_t jj = J - back;
-          mbar_drain(kF8 ? &S.kraw[jj % kStages] : &S.kfull[jj % kStages], (jj / kStages) & 1u);
+          mbar_drain(&S.kfull[jj % kStages], (jj / kStages) & 1u);
         }
       }
     }
@@ -723,7 +699,7 @@ __global__ void __launch_bounds__(kF8 ? kF8Threads : kTcThreads, 1)
   } else if (warp == kMmaWarp) {
     // ======================= Sᵀ issuer =======================
     if (lane == 0) {
-      const uint32_t idesc_s = idesc_bf16_f32(kTcKeys, 16, false, false);
+      const uint32_t idesc_s = kF8 ? idesc_e4m3_f32(kTcKeys, 16) : idesc_bf16_f32(kTcKeys, 16, false, false);
       uint32_t J = 0, K = 0;
       bool ok = true;
       while (ok) {
@@ -734,6 +710,8 @@ __global__ void __launch_bounds__(kF8 ? kF8Threads : kTcThreads, 1)
         if (idx < 0) break;
         const uint32_t qaddr0 = smem_u32(S.q[ps][0]);
         const uint32_t qaddr1 = smem_u32(S.q[ps][1]);
+        // E4M3 cache: the item's Q terms, from the Q warps
+        if (kF8 && !mbar_wait(&S.q8full[ps], (K >> 1) & 1u, ctx)) { ok = false; break; }
         for (int j = 0; j < ntile; ++j, ++J) {
           const int st = J % kStages;
           const int sb = J & 1;
@@ -743,13 +721,13 @@ __global__ void __launch_bounds__(kF8 ? kF8Threads : kTcThreads, 1)
           const int valid = S.meta[st][1];
           if (valid > 0) {
             if constexpr (kF8) {
-              // A = the expanded K tile in tensor memory: 16 d-columns are 8 columns of pairs
+              // A = the tile's K codes, B = the Q terms: 32 codes (32 bytes) of D per product
+              const uint32_t ka = smem_u32(S.k[st][0]);
+              const uint32_t qa = smem_u32(S.q8[ps]);
 #pragma unroll
-              for (int kk = 0; kk < kTcD / 16; ++kk) {
-                const uint32_t qa = (kk < 4 ? qaddr0 : qaddr1) + (kk & 3) * 32;
-                umma_bf16_ts(tmem + sb * 16, tmem + kColK + st * 64 + kk * 8,
-                             smem_desc(qa, 16, 1024, kLayoutSW128), idesc_s, kk > 0 ? 1u : 0u);
-              }
+              for (int kk = 0; kk < kTcD / 32; ++kk)
+                umma_f8_ss(tmem + sb * 16, smem_desc(ka + kk * 32, 16, 1024, kLayoutSW128),
+                           smem_desc(qa + kk * 32, 16, 1024, kLayoutSW128), idesc_s, kk > 0 ? 1u : 0u);
             } else {
               const uint32_t k0 = smem_u32(S.k[st][0]);
               const uint32_t k1 = smem_u32(S.k[st][Smem::kKSlabs - 1]);
@@ -845,6 +823,14 @@ __global__ void __launch_bounds__(kF8 ? kF8Threads : kTcThreads, 1)
       const int idx = S.item_slot[ps][0];
       const int ntile = S.item_slot[ps][1];
       const DecodeItem it = S.item[ps];
+      // E4M3 cache: each head's score factor 2^e * scale (read before the Q slot is released)
+      float qs[GPAD];
+      if constexpr (kF8) {
+        if (idx >= 0) ok = ok && mbar_wait(&S.q8full[ps], (K >> 1) & 1u, ctx);
+        if (named_bar_or(1, kSoftmaxThreads, !ok)) break;
+#pragma unroll
+        for (int g = 0; g < GPAD; ++g) qs[g] = S.qscale[ps][g] * p.scale_log2;
+      }
       __syncwarp();
       if (lane == 0) mbar_arrive(&S.qempty[ps]);
       const uint32_t ob = K & 1;
@@ -882,7 +868,10 @@ __global__ void __launch_bounds__(kF8 ? kF8Threads : kTcThreads, 1)
         bool grow = false;
 #pragma unroll
         for (int g = 0; g < GPAD; ++g) {
-          x[g] = (in && g < p.g) ? __uint_as_float(sr[g]) * p.scale_log2 : -INFINITY;
+          if constexpr (kF8)  // the two Q terms' columns, then the head's factor
+            x[g] = (in && g < p.g) ? (__uint_as_float(sr[g]) + __uint_as_float(sr[8 + g])) * qs[g] : -INFINITY;
+          else
+            x[g] = (in && g < p.g) ? __uint_as_float(sr[g]) * p.scale_log2 : -INFINITY;
           grow |= x[g] > m[g] + kRescaleThreshold;
         }
         // One barrier per tile, which also tells every thread whether any key of the tile lies
@@ -1002,37 +991,79 @@ __global__ void __launch_bounds__(kF8 ? kF8Threads : kTcThreads, 1)
     }
   } else if (warp >= kConvWarp0) {
     if constexpr (kF8) {
-      // ================ E4M3 expansion (K to bf16, V to f16) ================
-      // Warps 12-15: per stage, in tile order, K into the stage's tensor-memory tile (thread = key
-      // lane of its warp's lane quarter: one code row of 128 bytes -> 64 columns of bf16 pairs).
-      // Warps 16-19: V in place in shared memory. A stage whose valid count is < 0 is the
-      // producer's stop marker.
+      // ================ E4M3 cache: Q terms (warps 12-15), V expansion (16-19) ================
       if (warp < kConvWarp0 + 4) {
-        const uint32_t quarter = static_cast<uint32_t>(warp & 3);
-        const int krow = static_cast<int>(quarter) * 32 + lane;
-        const uint32_t klane = (quarter * 32u) << 16;
-        for (uint32_t J = 0;; ++J) {
-          const int st = J % kStages;
-          if (!mbar_wait(&S.kraw[st], (J / kStages) & 1u, ctx)) break;
-          if (S.meta[st][1] < 0) break;
-          const unsigned char* raw = reinterpret_cast<const unsigned char*>(S.k[st][0]) + krow * 128;
-#pragma unroll 1
-          for (int hh = 0; hh < 2; ++hh) {
-            uint32_t w[32];
-#pragma unroll
-            for (int c = 0; c < 4; ++c) {
-              const uint4 x = *reinterpret_cast<const uint4*>(raw + (((hh * 4 + c) ^ (krow & 7)) << 4));
-              e4m3x4_to_bf16(x.x, w[8 * c + 0], w[8 * c + 1]);
-              e4m3x4_to_bf16(x.y, w[8 * c + 2], w[8 * c + 3]);
-              e4m3x4_to_bf16(x.z, w[8 * c + 4], w[8 * c + 5]);
-              e4m3x4_to_bf16(x.w, w[8 * c + 6], w[8 * c + 7]);
-            }
-            tmem_st32(tmem + klane + kColK + st * 64 + hh * 32, w);
+        // Per item, Q (bf16, SW128, 16 head rows) becomes two E4M3 terms per head for the Sᵀ
+        // product: thread ct handles 8 consecutive d of head ct / 16. Rows 0-7 of q8 take c1, rows
+        // 8-15 c2, in the 128-byte swizzle of a K-major operand of one-byte elements.
+        const int ct = tid - kConvWarp0 * 32;
+        const int hd = ct >> 4;
+        const int d0 = (ct & 15) * 8;
+        for (uint32_t K = 0;; ++K) {
+          const int ps = K & 1;
+          if (!mbar_wait(&S.qfull[ps], (K >> 1) & 1u, ctx)) break;
+          const int idx = S.item_slot[ps][0];
+          if (idx < 0) {
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&S.qempty[ps]);
+            break;
           }
-          tmem_wait_st();
-          tc_fence_before();
+          const unsigned char* qrow = reinterpret_cast<const unsigned char*>(S.q[ps][d0 >> 6]) + hd * 128;
+          const uint4 raw = *reinterpret_cast<const uint4*>(qrow + ((((d0 & 63) >> 3) ^ (hd & 7)) << 4));
+          float x[8];
+          {
+            const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              x[2 * i] = __uint_as_float(w[i] << 16);
+              x[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+            }
+          }
+          float mx = 0.f;
+#pragma unroll
+          for (int i = 0; i < 8; ++i) mx = fmaxf(mx, fabsf(x[i]));
+#pragma unroll
+          for (int o = 8; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+          // e with the head's largest |q| / 2^e in [128, 256) (a power of two: the scaling is
+          // exact); an all-zero head (or one below 2^-100) gets e = 0 and zero terms
+          int e = 0;
+          if (mx >= 0x1p-100f) e = static_cast<int>((__float_as_uint(mx) >> 23) & 0xffu) - 127 - 7;
+          const float inv = __uint_as_float(static_cast<uint32_t>(127 - e) << 23);  // 2^-e
+          uint32_t c1w[2], c2w[2];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const float a = x[2 * i] * inv, b = x[2 * i + 1] * inv;
+            uint16_t c1, c2;
+            uint32_t h1;
+            // c1 = E4M3(a, b) (a in the low byte), back to f16 pairs, residual, c2 = E4M3(residual)
+            asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(c1) : "f"(b), "f"(a));
+            asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h1) : "h"(c1));
+            __half2 h2;
+            memcpy(&h2, &h1, 4);
+            const float2 f = __half22float2(h2);
+            asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(c2) : "f"(b - f.y), "f"(a - f.x));
+            const uint32_t sh = (i & 1) * 16;
+            if ((i & 1) == 0) {
+              c1w[i >> 1] = 0u;
+              c2w[i >> 1] = 0u;
+            }
+            c1w[i >> 1] |= static_cast<uint32_t>(c1) << sh;
+            c2w[i >> 1] |= static_cast<uint32_t>(c2) << sh;
+          }
+          // 8 codes at d0 of rows hd (c1) and 8 + hd (c2): half of the 16-byte chunk d0 / 16
+          const int r1 = hd, r2 = 8 + hd;
+          unsigned char* q8 = S.q8[ps];
+          *reinterpret_cast<uint2*>(q8 + r1 * 128 + ((((d0 >> 4) ^ (r1 & 7)) << 4) | (d0 & 15))) =
+              make_uint2(c1w[0], c1w[1]);
+          *reinterpret_cast<uint2*>(q8 + r2 * 128 + ((((d0 >> 4) ^ (r2 & 7)) << 4) | (d0 & 15))) =
+              make_uint2(c2w[0], c2w[1]);
+          if ((ct & 15) == 0) S.qscale[ps][hd] = __uint_as_float(static_cast<uint32_t>(127 + e) << 23);
+          fence_proxy_async_smem();
           __syncwarp();
-          if (lane == 0) mbar_arrive(&S.kfull[st]);
+          if (lane == 0) {
+            mbar_arrive(&S.q8full[ps]);
+            mbar_arrive(&S.qempty[ps]);
+          }
         }
       } else {
         const int ct = tid - (kConvWarp0 + 4) * 32;
