@@ -59,8 +59,9 @@ constexpr int kSoftmaxThreads = 128;
 constexpr uint32_t kTmemCols = 128;
 constexpr uint32_t kHalfBytes = kTcKeys * 64 * 2;   // one 64-column half of a K or V tile
 
-constexpr int kMaxPageBoxes = 128 / 8;  // page boxes of one key tile (pages of >= 8 keys)
+constexpr int kMaxPageBoxes = 128 / 8;  // pages of one key tile (pages of >= 8 keys)
 constexpr int kPidSlots = 8;             // page-id ring of the paged producers
+constexpr int kPidAhead = 4;             // pages < 128 keys: ids copied this many tiles ahead
 
 // kF8 (E4M3 cache): a K stage holds only the tile's codes (128 rows of 128 bytes, the size of one
 // bf16 half), since the expanded K lives in tensor memory; a V stage holds the codes in its upper
@@ -109,8 +110,9 @@ struct __align__(1024) TcSmem {
   // terms are ready (the four Q warps).
   uint64_t vraw[kStages];
   uint64_t q8full[2];
-  // paged cache: physical page ids of tile J in slot J mod kPidSlots, copied asynchronously by
-  // the Q/K producer two tiles ahead (pidfull) and released by the V producer (pidempty)
+  // paged cache: physical page ids of tile J in slot J mod kPidSlots, written by the Q/K producer
+  // (pages < 128 keys: copied asynchronously kPidAhead tiles ahead by its 32 lanes) and released
+  // by the V producer (pidempty)
   int32_t pid[kPidSlots][kMaxPageBoxes];
   uint64_t pidfull[kPidSlots], pidempty[kPidSlots];
   uint64_t drain, drain_pv;
@@ -118,30 +120,28 @@ struct __align__(1024) TcSmem {
   int abort_flag;
 };
 
-// Pages of the 128-key tile that starts at key t (a multiple of 128 in a paged plan) and holds
-// `valid` keys: with page_size >= 128 one box of the tile inside page t / page_size from row
-// t % page_size, else one box per page that holds some of the valid keys.
-struct TilePages {
-  int first, n, row0;
+// Pages of < 128 keys (8, 16, 32 or 64): the 128-key tile that starts at key t (a multiple of
+// 128 in a paged plan) and holds `valid` keys spans the n pages first .. first + n - 1 of the
+// sequence's block-table row that hold some of its valid keys.
+struct SmallPages {
+  int first, n;
 };
-
-__device__ __forceinline__ TilePages tile_pages(const DecodeParams& p, int t, int valid) {
-  TilePages tp;
-  const int P = p.page_size;
-  tp.first = t / P;
-  tp.n = valid <= 0 ? 0 : (P >= kTcKeys ? 1 : (valid + P - 1) / P);
-  tp.row0 = P >= kTcKeys ? t - tp.first * P : 0;
-  return tp;
+__device__ __forceinline__ SmallPages small_pages(int t, int valid, int page_shift) {
+  SmallPages sp;
+  sp.first = t >> page_shift;
+  sp.n = valid <= 0 ? 0 : ((valid - 1) >> page_shift) + 1;
+  return sp;
 }
 
-// Start the asynchronous copy of the tile's page ids from the block table into `dst` (entries
-// past the sequence's row are not copied; readers take them as -1).
-__device__ __forceinline__ void prefetch_tile_pages(int32_t* dst, const DecodeParams& p, int b,
-                                                    const TilePages& tp) {
-  const int32_t* row = p.block_table + static_cast<int64_t>(b) * p.pages_per_seq;
-#pragma unroll 1  // kept rolled: the producer loops must stay small in the instruction cache
-  for (int i = 0; i < kMaxPageBoxes; ++i)
-    if (i < tp.n && tp.first + i < p.pages_per_seq) cp_async_4(dst + i, row + tp.first + i);
+// Whole warp: start the asynchronous copy of a tile's page ids from the block table into `dst`,
+// lane i copying entry i (entries past the sequence's row are not copied; readers take them as
+// -1), then let `bar` count this lane's copies (every lane arrives: the barrier expects 32).
+__device__ __forceinline__ void prefetch_small_pages(int32_t* dst, uint64_t* bar,
+                                                     const DecodeParams& p, int b,
+                                                     const SmallPages& sp, int lane) {
+  if (lane < sp.n && sp.first + lane < p.pages_per_seq)
+    cp_async_4(dst + lane, p.block_table + static_cast<int64_t>(b) * p.pages_per_seq + sp.first + lane);
+  cp_async_mbar_arrive(bar);
 }
 
 // Page id of the tile starting at key t of sequence b when pages hold >= 128 keys (-1 past the
@@ -152,34 +152,47 @@ __device__ __forceinline__ int32_t tile_page_id(const DecodeParams& p, int b, in
                                  : -1;
 }
 
-// Issue the K or V loads of one 128-key tile of a paged cache (both 64-column halves): the tp.n
-// boxes of paged_tile_bytes(), page ids from `ids` (a slot of the ring). A page that holds some
-// of the tile's `valid` keys but whose index lies outside the pool raises FD_FLAG_BAD_PAGE; its
-// copy still runs and reads zeros (a TMA coordinate outside the tensor).
-// An E4M3 cache (kF8) has one 128-byte box per row, into dst0 (the codes' staging area).
+// Whole warp: issue the K or V loads of one 128-key tile over pages of < 128 keys, one box per
+// lane: lane i < n copies page i's first 64-column half (an E4M3 cache: its whole 128-byte
+// rows) and lane n + i its second half, page ids from `ids` (a slot of the ring). A page that
+// holds some of the tile's `valid` keys but whose index lies outside the pool raises
+// FD_FLAG_BAD_PAGE; its copy still runs and reads zeros (a TMA coordinate outside the tensor).
+// The caller has announced small_pages_bytes() on `bar`.
 template <bool kF8>
-__device__ __forceinline__ void load_tile_paged(__nv_bfloat16* dst0, __nv_bfloat16* dst1,
-                                                const CUtensorMap* map, uint64_t* bar,
-                                                const TilePages& tp, const int32_t* ids,
-                                                const DecodeParams& p, int h, int valid,
-                                                uint64_t pol) {
-  const int rows = p.page_size >= kTcKeys ? kTcKeys : p.page_size;
+__device__ __forceinline__ void load_small_pages(__nv_bfloat16* dst0, __nv_bfloat16* dst1,
+                                                 const CUtensorMap* map, uint64_t* bar,
+                                                 const SmallPages& sp, const int32_t* ids,
+                                                 const DecodeParams& p, int h, int valid,
+                                                 uint64_t pol, int lane) {
+  const int rows = p.page_size;
+  const int boxes = kF8 ? sp.n : 2 * sp.n;
   bool bad = false;
-#pragma unroll 1  // kept rolled: the producer loops must stay small in the instruction cache
-  for (int i = 0; i < kMaxPageBoxes; ++i) {
-    if (i < tp.n) {
-      const int32_t id = tp.first + i < p.pages_per_seq ? ids[i] : -1;
-      bad |= (i * rows < valid) && (id < 0 || id >= p.num_pages);
-      if constexpr (kF8) {
-        tma_load_4d_stream(reinterpret_cast<unsigned char*>(dst0) + i * rows * 128, map, bar, 0,
-                           tp.row0, h, id, pol);
-      } else {
-        tma_load_4d_stream(dst0 + i * rows * 64, map, bar, 0, tp.row0, h, id, pol);
-        tma_load_4d_stream(dst1 + i * rows * 64, map, bar, 64, tp.row0, h, id, pol);
-      }
+  if (lane < boxes) {
+    const int half = kF8 ? 0 : (lane >= sp.n ? 1 : 0);
+    const int i = lane - half * sp.n;
+    const int32_t id = sp.first + i < p.pages_per_seq ? ids[i] : -1;
+    bad = i * rows < valid && (id < 0 || id >= p.num_pages);
+    if constexpr (kF8) {
+      tma_load_4d_stream(reinterpret_cast<unsigned char*>(dst0) + i * rows * 128, map, bar, 0, 0,
+                         h, id, pol);
+    } else {
+      tma_load_4d_stream((half ? dst1 : dst0) + i * rows * 64, map, bar, half * 64, 0, h, id, pol);
     }
   }
-  if (bad) atomicOr(&p.hdr->status, FD_FLAG_BAD_PAGE);
+  if (__any_sync(0xffffffffu, bad) && lane == 0) atomicOr(&p.hdr->status, FD_FLAG_BAD_PAGE);
+}
+
+// Bytes load_small_pages delivers (both halves; E4M3: one byte per element).
+template <bool kF8>
+__device__ __forceinline__ uint32_t small_pages_bytes(const SmallPages& sp, const DecodeParams& p) {
+  return (kF8 ? 1u : 2u) * 128u * static_cast<uint32_t>(p.page_size * sp.n);
+}
+
+// Whole warp: every lane waits for the phase itself (so each lane sees what the phase guards);
+// true only if every lane's wait succeeded.
+__device__ __forceinline__ bool warp_mbar_wait(uint64_t* bar, uint32_t parity, const WaitCtx& ctx) {
+  const bool ok = mbar_wait(bar, parity, ctx);
+  return __all_sync(0xffffffffu, ok);
 }
 
 // The loads of one 128-key tile that lies inside one page of >= 128 keys, from row `row0`.
@@ -195,13 +208,6 @@ __device__ __forceinline__ void load_tile_page1(__nv_bfloat16* dst0, __nv_bfloat
     tma_load_4d_stream(dst0, map, bar, 0, row0, h, id, pol);
     tma_load_4d_stream(dst1, map, bar, 64, row0, h, id, pol);
   }
-}
-
-// Bytes the loads of load_tile_paged deliver (both halves; E4M3: one byte per element).
-template <bool kF8>
-__device__ __forceinline__ uint32_t paged_tile_bytes(const TilePages& tp, const DecodeParams& p) {
-  const int rows = p.page_size >= kTcKeys ? kTcKeys : p.page_size;
-  return (kF8 ? 1u : 2u) * 128u * static_cast<uint32_t>(rows * tp.n);
 }
 
 // Four E4M3 codes (the bytes of w, the first in the low byte) as two f16 pairs, exactly, by the
@@ -337,7 +343,7 @@ __global__ void __launch_bounds__(kF8 ? kF8Threads : kTcThreads, 1)
       mbar_init(&S.lfree[i], 4);
     }
     for (int i = 0; i < kPidSlots; ++i) {
-      mbar_init(&S.pidfull[i], 1);
+      mbar_init(&S.pidfull[i], kMode == kSmallPages ? 32 : 1);
       mbar_init(&S.pidempty[i], 1);
     }
     mbar_init(&S.drain, 1);
@@ -361,7 +367,6 @@ __global__ void __launch_bounds__(kF8 ? kF8Threads : kTcThreads, 1)
   const WaitCtx ctx{&S.abort_flag, &p.hdr->status};
   const bool fused = p.items == nullptr;
   constexpr bool paged = kMode != kContiguous;
-  constexpr bool big_pages = kMode == kBigPages;  // pages of >= 128 keys: one page per tile
   if (fused) {
     // ---- the split plan, computed by every CTA in shared memory (the planner's arithmetic):
     // clamped lengths and their sum, the chunk size, split counts, longest-first ranks, item
@@ -477,8 +482,110 @@ __global__ void __launch_bounds__(kF8 ? kF8Threads : kTcThreads, 1)
     return it;
   };
 
-  if (warp == kProducerWarp) {
-    // ======================= TMA producer =======================
+  if (warp == kProducerWarp && kMode == kSmallPages) {
+    // ============ TMA producer of Q and K, pages of < 128 keys (whole warp) ============
+    // A tile spans up to 16 pages here, so its page ids and page copies go one per lane: the
+    // warp spends a few instructions per tile whatever the page count, where one thread would
+    // spend one short dependent sequence per page. The item schedule is the one below.
+    const int pshift = __ffs(p.page_size) - 1;  // page sizes 8, 16, 32, 64
+    const int n_items = fused ? (fused_overflow ? 0 : fused_items)
+                              : *reinterpret_cast<volatile int32_t*>(&p.hdr->num_dec_items);
+    const uint64_t pol = l2_evict_first_policy();
+    auto claim = [&]() {
+      int v = 0;
+      if (lane == 0) v = atomicAdd(&p.hdr->dec_counter, 1);
+      return __shfl_sync(0xffffffffu, v, 0);
+    };
+    uint32_t J = 0, K = 0, pf = 0;
+    bool ok = true;
+    int idx = claim();
+    DecodeItem it{};
+    if (idx < n_items) it = fused ? fused_item(idx) : p.items[idx];
+    while (ok && idx < n_items) {
+      int nidx = n_items;
+      DecodeItem nit{};
+      bool have_next = false;
+      const int len = it.t1 - it.t0;
+      const int ntile = len > 0 ? (len + kTcKeys - 1) / kTcKeys : 1;
+      const int ps = K & 1;
+      if (!warp_mbar_wait(&S.qempty[ps], ((K >> 1) & 1u) ^ 1u, ctx)) { ok = false; break; }
+      if (lane == 0) {
+        S.item_slot[ps][0] = idx;
+        S.item_slot[ps][1] = ntile;
+        S.item[ps] = it;
+        mbar_arrive_expect_tx(&S.qfull[ps], 2u * 128u * static_cast<uint32_t>(p.q_box_rows));
+        tma_load_3d(S.q[ps][0], &tmap_q, &S.qfull[ps], 0, it.h * p.g, it.row);
+        tma_load_3d(S.q[ps][1], &tmap_q, &S.qfull[ps], 64, it.h * p.g, it.row);
+      }
+      const int claim_j = max(0, ntile - 3), read_j = max(0, ntile - 2);
+      for (int j = 0; j < ntile; ++j, ++J) {
+        if (j == claim_j) nidx = claim();
+        if (j == read_j && nidx < n_items) {
+          nit = fused ? fused_item(nidx) : p.items[nidx];
+          have_next = true;
+        }
+        // page ids of the tiles up to J + kPidAhead that are known (this item's and, once read,
+        // the next item's)
+        while (pf <= J + kPidAhead) {
+          const int ahead = j + static_cast<int>(pf - J);
+          int xb, xt, xend;  // sequence, first key and key end of tile pf
+          if (ahead < ntile) {
+            xb = it.b;
+            xt = it.t0 + ahead * kTcKeys;
+            xend = it.t1;
+          } else {
+            const int nl = nit.t1 - nit.t0;
+            if (!have_next || ahead - ntile >= (nl > 0 ? (nl + kTcKeys - 1) / kTcKeys : 1)) break;
+            xb = nit.b;
+            xt = nit.t0 + (ahead - ntile) * kTcKeys;
+            xend = nit.t1;
+          }
+          const int slot = pf % kPidSlots;
+          // the V producer has released the slot's previous tile
+          if (!warp_mbar_wait(&S.pidempty[slot], ((pf / kPidSlots) & 1u) ^ 1u, ctx)) { ok = false; break; }
+          prefetch_small_pages(S.pid[slot], &S.pidfull[slot], p, xb,
+                               small_pages(xt, min(kTcKeys, xend - xt), pshift), lane);
+          ++pf;
+        }
+        if (!ok) break;
+        const int st = J % kStages;
+        const int t = it.t0 + j * kTcKeys;
+        const int valid = max(0, min(kTcKeys, it.t1 - t));
+        if (!warp_mbar_wait(&S.kempty[st], ((J / kStages) & 1u) ^ 1u, ctx)) { ok = false; break; }
+        if (!warp_mbar_wait(&S.pidfull[J % kPidSlots], (J / kPidSlots) & 1u, ctx)) { ok = false; break; }
+        const SmallPages sp = small_pages(t, valid, pshift);
+        uint64_t* kbar = &S.kfull[st];  // the copy completes kfull (E4M3: the codes as they are)
+        if (lane == 0) {
+          S.meta[st][0] = t;
+          S.meta[st][1] = valid;
+          if (valid > 0) mbar_arrive_expect_tx(kbar, small_pages_bytes<kF8>(sp, p));
+          else mbar_arrive(kbar);
+        }
+        __syncwarp();
+        if (valid > 0)
+          load_small_pages<kF8>(S.k[st][0], S.k[st][Smem::kKSlabs - 1], &tmap_k, kbar, sp,
+                                S.pid[J % kPidSlots], p, it.h, valid, pol, lane);
+      }
+      ++K;
+      idx = nidx;
+      it = nit;
+    }
+    if (ok && warp_mbar_wait(&S.qempty[K & 1], ((K >> 1) & 1u) ^ 1u, ctx) && lane == 0) {
+      S.item_slot[K & 1][0] = -1;
+      S.item_slot[K & 1][1] = 0;
+      mbar_arrive(&S.qfull[K & 1]);
+    }
+    asm volatile("cp.async.wait_all;" ::: "memory");
+    if (S.abort_flag && lane == 0) {
+      // let copies already issued land before shared memory is released
+      for (uint32_t back = 1; back <= kStages && back <= J; ++back) {
+        const uint32_t jj = J - back;
+        mbar_drain(&S.kfull[jj % kStages], (jj / kStages) & 1u);
+      }
+    }
+    __syncwarp();
+  } else if (kMode != kSmallPages && warp == kProducerWarp) {
+    // ============ TMA producer of Q and K (contiguous cache, or pages of >= 128 keys) ============
     if (lane == 0) {
       const int n_items = fused ? (fused_overflow ? 0 : fused_items)
                                 : *reinterpret_cast<volatile int32_t*>(&p.hdr->num_dec_items);
@@ -493,10 +600,8 @@ __global__ void __launch_bounds__(kF8 ? kF8Threads : kTcThreads, 1)
       int idx = atomicAdd(&p.hdr->dec_counter, 1);
       DecodeItem it{};
       if (idx < n_items) it = fused ? fused_item(idx) : p.items[idx];
-      // paged cache: the page ids of global tile pf are copied into the ring two tiles ahead
-      // (pages < 128 keys); with pages of >= 128 keys the one id of the next tile is loaded into
-      // a register one tile ahead and handed to the V producer through the ring
-      uint32_t pf = 0;
+      // pages of >= 128 keys: the one id of the next tile is loaded into a register one tile
+      // ahead and handed to the V producer through the ring
       int32_t id_pre = -1;
       bool have_pre = false;
       while (ok && idx < n_items) {
@@ -517,7 +622,7 @@ __global__ void __launch_bounds__(kF8 ? kF8Threads : kTcThreads, 1)
         for (int j = 0; j < ntile; ++j, ++J) {
           if (j == claim_j) nidx = atomicAdd(&p.hdr->dec_counter, 1);
           if constexpr (paged) {
-            // the page-id prefetch below needs the next item before this tile's copies
+            // the page-id load below needs the next item before this tile's copies
             if (j == read_j && nidx < n_items) {
               nit = fused ? fused_item(nidx) : p.items[nidx];
               have_next = true;
@@ -527,71 +632,31 @@ __global__ void __launch_bounds__(kF8 ? kF8Threads : kTcThreads, 1)
           const uint32_t free_parity = ((J / kStages) & 1u) ^ 1u;
           const int t = it.t0 + j * kTcKeys;
           const int valid = max(0, min(kTcKeys, it.t1 - t));
-          TilePages tp{};
           int32_t id_big = -1;
           if constexpr (paged) {
-            if constexpr (big_pages) {
-              // this tile's page (loaded an iteration ago); start loading the next tile's
-              id_big = have_pre ? id_pre : tile_page_id(p, it.b, t);
-              have_pre = true;
-              if (j + 1 < ntile) id_pre = tile_page_id(p, it.b, t + kTcKeys);
-              else if (have_next) id_pre = tile_page_id(p, nit.b, nit.t0);
-              else have_pre = false;
-            }
-            // prefetch the page ids of the tiles up to J + 2 that are known (this item's and,
-            // once read, the next item's)
-            while (kMode == kSmallPages && ok && pf <= J + 2) {
-              const int ahead = j + static_cast<int>(pf - J);
-              const DecodeItem* x = nullptr;
-              int jj = 0;
-              if (ahead < ntile) {
-                x = &it;
-                jj = ahead;
-              } else if (have_next) {
-                const int nl = nit.t1 - nit.t0;
-                if (ahead - ntile < (nl > 0 ? (nl + kTcKeys - 1) / kTcKeys : 1)) {
-                  x = &nit;
-                  jj = ahead - ntile;
-                }
-              }
-              if (!x) break;
-              const int slot = pf % kPidSlots;
-              // the V producer has released the slot's previous tile
-              if (!mbar_wait(&S.pidempty[slot], ((pf / kPidSlots) & 1u) ^ 1u, ctx)) { ok = false; break; }
-              const int xt = x->t0 + jj * kTcKeys;
-              prefetch_tile_pages(S.pid[slot], p, x->b, tile_pages(p, xt, min(kTcKeys, x->t1 - xt)));
-              cp_async_mbar_arrive(&S.pidfull[slot]);
-              ++pf;
-            }
-            if (!ok) break;
-            tp = tile_pages(p, t, valid);
+            // this tile's page (loaded an iteration ago); start loading the next tile's
+            id_big = have_pre ? id_pre : tile_page_id(p, it.b, t);
+            have_pre = true;
+            if (j + 1 < ntile) id_pre = tile_page_id(p, it.b, t + kTcKeys);
+            else if (have_next) id_pre = tile_page_id(p, nit.b, nit.t0);
+            else have_pre = false;
           }
           if (!mbar_wait(&S.kempty[st], free_parity, ctx)) { ok = false; break; }
           if constexpr (paged) {
-            if constexpr (big_pages) {
-              // hand the id to the V producer: the slot's previous tile has been released
-              const int slot = J % kPidSlots;
-              if (!mbar_wait(&S.pidempty[slot], ((J / kPidSlots) & 1u) ^ 1u, ctx)) { ok = false; break; }
-              S.pid[slot][0] = id_big;
-              mbar_arrive(&S.pidfull[slot]);
-            } else {
-              if (!mbar_wait(&S.pidfull[J % kPidSlots], (J / kPidSlots) & 1u, ctx)) { ok = false; break; }
-            }
+            // hand the id to the V producer: the slot's previous tile has been released
+            const int slot = J % kPidSlots;
+            if (!mbar_wait(&S.pidempty[slot], ((J / kPidSlots) & 1u) ^ 1u, ctx)) { ok = false; break; }
+            S.pid[slot][0] = id_big;
+            mbar_arrive(&S.pidfull[slot]);
           }
           S.meta[st][0] = t;
           S.meta[st][1] = valid;
           uint64_t* kbar = &S.kfull[st];  // the copy completes kfull (E4M3: the codes as they are)
           if (valid > 0) {
             if constexpr (paged) {
-              if constexpr (big_pages) {
-                mbar_arrive_expect_tx(kbar, kRowBytes * kTcKeys);
-                load_tile_page1<kF8>(S.k[st][0], S.k[st][Smem::kKSlabs - 1], &tmap_k, kbar, id_big,
-                                     t % p.page_size, p, it.h, pol);
-              } else {
-                mbar_arrive_expect_tx(kbar, paged_tile_bytes<kF8>(tp, p));
-                load_tile_paged<kF8>(S.k[st][0], S.k[st][Smem::kKSlabs - 1], &tmap_k, kbar, tp,
-                                     S.pid[J % kPidSlots], p, it.h, valid, pol);
-              }
+              mbar_arrive_expect_tx(kbar, kRowBytes * kTcKeys);
+              load_tile_page1<kF8>(S.k[st][0], S.k[st][Smem::kKSlabs - 1], &tmap_k, kbar, id_big,
+                                   t % p.page_size, p, it.h, pol);
             } else {
               mbar_arrive_expect_tx(kbar, kRowBytes * static_cast<uint32_t>(p.kv_box_rows));
               tma_load_4d_stream(S.k[st][0], &tmap_k, kbar, 0, t, it.h, it.b, pol);
@@ -617,7 +682,6 @@ __global__ void __launch_bounds__(kF8 ? kF8Threads : kTcThreads, 1)
           mbar_arrive(&S.qfull[ps]);
         }
       }
-      if constexpr (paged) asm volatile("cp.async.wait_all;" ::: "memory");
       if (S.abort_flag) {
         // let copies already issued land before shared memory is released
         for (uint32_t back = 1; back <= kStages && back <= J; ++back) {
@@ -627,7 +691,61 @@ __global__ void __launch_bounds__(kF8 ? kF8Threads : kTcThreads, 1)
       }
     }
     __syncwarp();
-  } else if (warp == kVProducerWarp) {
+  } else if (warp == kVProducerWarp && kMode == kSmallPages) {
+    // ============ TMA producer of V, pages of < 128 keys (whole warp, as the K producer) ============
+    const int pshift = __ffs(p.page_size) - 1;
+    const uint64_t pol = l2_evict_first_policy();
+    uint32_t J = 0, K = 0;
+    bool ok = true;
+    while (ok) {
+      const int ps = K & 1;
+      if (!warp_mbar_wait(&S.qfull[ps], (K >> 1) & 1u, ctx)) { ok = false; break; }
+      const int idx = S.item_slot[ps][0];
+      const int ntile = S.item_slot[ps][1];
+      const DecodeItem it = S.item[ps];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&S.qempty[ps]);
+      if (idx < 0) break;
+      for (int j = 0; j < ntile; ++j, ++J) {
+        const int st = J % kStages;
+        const int t = it.t0 + j * kTcKeys;
+        const int valid = max(0, min(kTcKeys, it.t1 - t));
+        if (!warp_mbar_wait(&S.vempty[st], ((J / kStages) & 1u) ^ 1u, ctx)) { ok = false; break; }
+        if (!warp_mbar_wait(&S.pidfull[J % kPidSlots], (J / kPidSlots) & 1u, ctx)) { ok = false; break; }
+        const SmallPages sp = small_pages(t, valid, pshift);
+        uint64_t* vbar = kF8 ? &S.vraw[st] : &S.vfull[st];
+        if (lane == 0) {
+          if constexpr (kF8) S.vmeta[st] = valid;
+          if (valid > 0) mbar_arrive_expect_tx(vbar, small_pages_bytes<kF8>(sp, p));
+          else mbar_arrive(vbar);
+        }
+        __syncwarp();
+        if (valid > 0)
+          load_small_pages<kF8>(S.v[st][kF8 ? 1 : 0], S.v[st][1], &tmap_v, vbar, sp,
+                                S.pid[J % kPidSlots], p, it.h, valid, pol, lane);
+        __syncwarp();  // every lane has read its page id: the slot is free
+        if (lane == 0) mbar_arrive(&S.pidempty[J % kPidSlots]);
+      }
+      ++K;
+    }
+    if (lane == 0) {
+      if constexpr (kF8) {
+        // stop marker for the V expanding warps (a stage without a tile)
+        const int st = J % kStages;
+        if (ok && mbar_wait(&S.vempty[st], ((J / kStages) & 1u) ^ 1u, ctx)) {
+          S.vmeta[st] = -1;
+          mbar_arrive(&S.vraw[st]);
+        }
+      }
+      if (S.abort_flag) {
+        for (uint32_t back = 1; back <= kStages && back <= J; ++back) {
+          const uint32_t jj = J - back;
+          mbar_drain(kF8 ? &S.vraw[jj % kStages] : &S.vfull[jj % kStages], (jj / kStages) & 1u);
+        }
+      }
+    }
+    __syncwarp();
+  } else if (kMode != kSmallPages && warp == kVProducerWarp) {
     // ======================= TMA producer of V =======================
     // Follows the items the Q/K producer publishes; a V stage is refilled once the P·V product
     // of its previous tile has completed, independently of the K half.
@@ -655,15 +773,10 @@ __global__ void __launch_bounds__(kF8 ? kF8Threads : kTcThreads, 1)
           uint64_t* vbar = kF8 ? &S.vraw[st] : &S.vfull[st];
           if constexpr (kF8) S.vmeta[st] = valid;
           if (valid > 0) {
-            if constexpr (big_pages) {
+            if constexpr (paged) {
               mbar_arrive_expect_tx(vbar, kRowBytes * kTcKeys);
               load_tile_page1<kF8>(S.v[st][kF8 ? 1 : 0], S.v[st][1], &tmap_v, vbar,
                                    S.pid[J % kPidSlots][0], t % p.page_size, p, it.h, pol);
-            } else if constexpr (paged) {
-              const TilePages tp = tile_pages(p, t, valid);
-              mbar_arrive_expect_tx(vbar, paged_tile_bytes<kF8>(tp, p));
-              load_tile_paged<kF8>(S.v[st][kF8 ? 1 : 0], S.v[st][1], &tmap_v, vbar, tp,
-                                   S.pid[J % kPidSlots], p, it.h, valid, pol);
             } else {
               mbar_arrive_expect_tx(vbar, tx);
               if constexpr (kF8) {

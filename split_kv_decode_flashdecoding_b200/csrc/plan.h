@@ -70,7 +70,7 @@ struct WsHeader {
   int32_t tile_counter;
   int32_t dec_exit;         // CTAs of the tensor-core split kernel that have finished (zero
                             // between calls)
-  int32_t tile_ctas;        // chunked prefill: CTAs the tile kernel keeps (chunk_tile_ctas)
+  int32_t tile_ctas;        // chunked prefill: CTAs the tile kernel keeps (least chunk_tile_cost)
   int32_t pad[57];
 };
 static_assert(sizeof(WsHeader) == 256, "WsHeader is 256 bytes");
@@ -202,24 +202,15 @@ FD_HD int32_t chunk_tile_splits(int32_t keys) {
 constexpr float kTileKeyTileUs = 2.3f;  // 250 µs for workload 5's 16192 key tiles on 148 CTAs
 constexpr float kDecodeSmGBs = 45.f;    // tensor-core decode rows beside 80 tile CTAs: ~1.4 GB in 465 µs on 68 SMs
 constexpr float kHbmGBs = 6000.f;       // decode rows alone on the whole device
-FD_HD int32_t chunk_tile_ctas(int64_t key_tiles, int64_t dec_bytes, int32_t nsm) {
-  if (key_tiles <= 0) return 0;
-  if (dec_bytes <= 0 || nsm <= 1) return nsm;
-  const float dec = static_cast<float>(dec_bytes);
-  float best = 0.f;
-  int32_t best_n = nsm;
-  for (int32_t n = 1; n <= nsm; ++n) {
-    const float t1 = static_cast<float>(key_tiles) * kTileKeyTileUs / static_cast<float>(n);
-    const float sm_rate = static_cast<float>(nsm - n) * kDecodeSmGBs;
-    const float rate = (sm_rate < kHbmGBs ? sm_rate : kHbmGBs) * 1e3f;  // bytes per microsecond
-    const float left = dec - rate * t1;
-    const float t = t1 + (left > 0.f ? left / (kHbmGBs * 1e3f) : 0.f);
-    if (n == 1 || t < best) {
-      best = t;
-      best_n = n;
-    }
-  }
-  return best_n;
+// Estimated time (µs) of the call when the tile kernel keeps n of the nsm multiprocessors. The
+// planner keeps the n of least cost (the smallest such n on ties); with no tile items it keeps
+// 0, with no decode rows all nsm.
+FD_HD float chunk_tile_cost(int64_t key_tiles, float dec_bytes, int32_t nsm, int32_t n) {
+  const float t1 = static_cast<float>(key_tiles) * kTileKeyTileUs / static_cast<float>(n);
+  const float sm_rate = static_cast<float>(nsm - n) * kDecodeSmGBs;
+  const float rate = (sm_rate < kHbmGBs ? sm_rate : kHbmGBs) * 1e3f;  // bytes per microsecond
+  const float left = dec_bytes - rate * t1;
+  return t1 + (left > 0.f ? left / (kHbmGBs * 1e3f) : 0.f);
 }
 
 // Upper bounds for a chunked-prefill call of T packed rows over B requests (any lengths).

@@ -363,17 +363,24 @@ __global__ void __launch_bounds__(kMaxPlanThreads, 1) plan_chunk_kernel(PlanPara
     const int32_t nheads = head_packed ? p.hkv : p.hq;
     const int32_t per_head = s_tcnt[b] / nheads;
     const int32_t nmax = chunk_tile_splits(chunk_tile_keys(pp, c, ntiles - 1, p.cap));
+    // partial-slot base of the request's first row, read once: the bases of its later tiles
+    // follow from the split counts (every row of tile t has nt(t) slots and the tiles before the
+    // last are full), so the loop below makes no dependent global load per item
+    const int32_t rb0 = p.row_base[r0];
     for (int32_t h = lane; h < nheads; h += 32) {
       int32_t i = s_tioff[b] + h * per_head;
       for (int32_t s = 0; s < nmax; ++s) {
+        int32_t next_base = rb0;
         for (int32_t t = 0; t < ntiles; ++t) {
           const int32_t kt = chunk_tile_keys(pp, c, t, p.cap);
           const int32_t nt = chunk_tile_splits(kt);
+          const int32_t tbase = next_base;  // row_base of tile t's first row
+          next_base += kQTile * nt;
           if (s >= nt) continue;
           const int32_t row0 = r0 + t * kQTile;
           const int32_t rows = min(kQTile, c - t * kQTile);
           const int32_t k0 = min(s * kChunkKvSplit, kt), k1 = min((s + 1) * kChunkKvSplit, kt);
-          const int32_t slot0 = p.row_base[row0] * p.hkv;
+          const int32_t slot0 = tbase * p.hkv;
           int4* dst = reinterpret_cast<int4*>(p.tiles + i);
           dst[0] = make_int4(b, h, s, nt);
           dst[1] = make_int4(k0, k1, row0, t * kQTile);
@@ -391,15 +398,40 @@ __global__ void __launch_bounds__(kMaxPlanThreads, 1) plan_chunk_kernel(PlanPara
     if (p.decode_merged_in_kernel) p.row_nsplit[row] = 1;
     for (int32_t h = 0; h < p.hkv; ++h) p.arrivals[row * p.hkv + h] = 0;
   }
+  if (warp == 0) {
+    // the tile kernel's CTAs: the n of least chunk_tile_cost, smallest on ties; lane l weighs
+    // n = l + 1, l + 33, ... and the warp keeps the lexicographic minimum of (cost, n)
+    const int64_t key_tiles = static_cast<int64_t>(s_key_tiles);
+    const int64_t dec_bytes = static_cast<int64_t>(s_total) * p.kv_key_bytes;
+    const int32_t nsm = p.tile_sms;
+    int32_t n_best;
+    if (overflow || key_tiles <= 0) {
+      n_best = 0;
+    } else if (dec_bytes <= 0 || nsm <= 1) {
+      n_best = nsm;
+    } else {
+      const float dec = static_cast<float>(dec_bytes);
+      float t_best = 0.f;
+      n_best = 0;
+      for (int32_t n = lane + 1; n <= nsm; n += 32) {
+        const float t = chunk_tile_cost(key_tiles, dec, nsm, n);
+        if (n_best == 0 || t < t_best) { t_best = t; n_best = n; }
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        const float t2 = __shfl_xor_sync(0xffffffffu, t_best, o);
+        const int32_t n2 = __shfl_xor_sync(0xffffffffu, n_best, o);
+        const bool take = n2 != 0 && (n_best == 0 || t2 < t_best || (t2 == t_best && n2 < n_best));
+        if (take) { t_best = t2; n_best = n2; }
+      }
+    }
+    if (lane == 0) p.hdr->tile_ctas = n_best;
+  }
   if (tid == 0) {
     p.hdr->num_dec_items = overflow ? 0 : n_dec_items;
     p.hdr->num_tile_items = overflow ? 0 : n_tile_items;
     p.hdr->dec_counter = 0;
     p.hdr->tile_counter = 0;
-    p.hdr->tile_ctas = overflow ? 0
-                                : chunk_tile_ctas(static_cast<int64_t>(s_key_tiles),
-                                                  static_cast<int64_t>(s_total) * p.kv_key_bytes,
-                                                  p.tile_sms);
     uint32_t f = s_flags | (overflow ? FD_FLAG_PLAN_OVERFLOW : 0u);
     if (f) atomicOr(&p.hdr->status, f);
   }
