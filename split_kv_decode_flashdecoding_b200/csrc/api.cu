@@ -862,6 +862,8 @@ fd_status fd_chunk_prefill_attention(const fd_tensor* q_chunk, const fd_tensor* 
   tp.cap = cap;
   tp.q_box_rows = std::min(128, T);
   tp.qp_box_rows = std::min(kQTile / g, T);
+  tp.quad_rows = g >= 2 ? 32 / g : 0;
+  tp.qq_box_rows = std::min(std::max(tp.quad_rows, 1), T);
   tp.g_recip16 = (65536 + g - 1) / g;
   tp.kv_box_rows = std::min(128, cap);
   tp.scale_log2 = scale_log2;
@@ -898,6 +900,12 @@ fd_status fd_chunk_prefill_attention(const fd_tensor* q_chunk, const fd_tensor* 
   const uint32_t qb_packed[3] = {64, static_cast<uint32_t>(g), static_cast<uint32_t>(tp.qp_box_rows)};
   if (g >= 2 && (s = make_tmap(&tq_packed, q_chunk->data, 3, qd, qs, qb_packed, "q_chunk (head-packed)")) != FD_OK)
     return s;
+  // quarter items (head-packed requests of <= 32 / G rows): G heads x 32 / G rows per box
+  CUtensorMap tq_quarter = tq_tile;
+  const uint32_t qb_quarter[3] = {64, static_cast<uint32_t>(g), static_cast<uint32_t>(tp.qq_box_rows)};
+  if (tp.quad_rows > 0 &&
+      (s = make_tmap(&tq_quarter, q_chunk->data, 3, qd, qs, qb_quarter, "q_chunk (quarter items)")) != FD_OK)
+    return s;
   const uint64_t kd[4] = {static_cast<uint64_t>(d), static_cast<uint64_t>(cap), static_cast<uint64_t>(hkv), static_cast<uint64_t>(B)};
   const uint64_t ks[3] = {static_cast<uint64_t>(k_cache->stride[2]) * 2, static_cast<uint64_t>(k_cache->stride[1]) * 2,
                           static_cast<uint64_t>(k_cache->stride[0]) * 2};
@@ -918,7 +926,8 @@ fd_status fd_chunk_prefill_attention(const fd_tensor* q_chunk, const fd_tensor* 
   prof_end(ev, kSegPlan, stream);
   FD_CUDA(cudaEventRecord(wv.fork, stream), "record fork event");
   prof_start(ev, kSegTiles, stream);
-  FD_CUDA(launch_chunk_tc(tp, tq_tile, tq_packed, tk, tv, tile_ctas, stream), "chunk tile kernel launch");
+  FD_CUDA(launch_chunk_tc(tp, tq_tile, tq_packed, tq_quarter, tk, tv, tile_ctas, stream),
+          "chunk tile kernel launch");
   prof_end(ev, kSegTiles, stream);
   FD_CUDA(cudaStreamWaitEvent(wv.side, wv.fork, 0), "side stream waits for the planner");
   prof_start(ev, kSegSplit, wv.side);

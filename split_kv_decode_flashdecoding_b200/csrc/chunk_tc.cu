@@ -8,9 +8,9 @@
 // Per 128-key tile of the split:
 //
 //   S[128 rows x 128 keys] = Q_tile · K_tileᵀ         UMMA M=128 N=128 K=D, both K-major (TMA SW128)
-//   one thread per row: mask, running max m (rescaled lazily), p = 2^(s·scale·log2e − m),
-//   running sum l, P split into bf16 hi + lo (both rounded to nearest) and stored into tensor
-//   memory
+//   two threads per row, 64 keys each: mask, running max m (rescaled lazily; the pair swaps
+//   its tile maxima), p = 2^(s·scale·log2e − m), running sums of p, P split into bf16 hi + lo
+//   (both rounded to nearest) and stored into tensor memory
 //   O_hi[128 x D] += P_hi · V_tile, O_lo[128 x D] += P_lo · V_tile
 //                                                        UMMA M=128 N=D, A from TMEM, V MN-major
 //
@@ -34,13 +34,20 @@
 // one KV head, tile row r being chunk position r / G of query head h G + r mod G, loaded by one
 // TMA box of G heads x 128 / G rows. Each key tile is then read and multiplied once per KV head,
 // not once per query head; the per-row causal limit and output address follow the mapping.
+// A request of c <= 32 / G rows (a few speculative tokens) is a quarter item: its c G rows are
+// loaded once into each 32-lane quarter of the tile, every copy's softmax takes a quarter of the
+// keys (the other quarters' P words are zero), and the epilogue adds the four partial products.
+// The softmax of a tile then runs on all four schedulers instead of one quarter's.
 //
-// Warp roles: 0-3 softmax (thread = TMEM lane = query row); 4 TMA producer of Q and K (2-stage
-// K ring, the next item's Q prefetched); 5 issuer of the S products and TMEM owner; 6-9 epilogue
-// (warp w reads TMEM lanes 32 (w mod 4) + [0, 32)); 10 TMA producer of V (2-stage ring); 11
-// issuer of the P·V products. A tcgen05.mma holds its issuing thread for about as long as the
-// tensor pipe needs for it, so the two product chains of a tile are issued by two threads. K and
-// V stages are released separately: K once S has read it, V once P·V has.
+// Warp roles: 0-3 and 12-15 softmax (warps w and w + 12 share TMEM lanes 32 w + [0, 32), one
+// query row per lane, and take keys [0, 64) and [64, 128) of each tile); 4 TMA producer of Q and
+// K (2-stage K ring, the next item's Q prefetched); 5 issuer of the S products and TMEM owner;
+// 6-9 epilogue (warp w reads TMEM lanes 32 (w mod 4) + [0, 32)); 10 TMA producer of V (2-stage
+// ring); 11 issuer of the P·V products. The softmax is the longest step of a tile (an exp2, two
+// roundings and a subtraction per key on one thread), so two warps per lane quarter halve it.
+// A tcgen05.mma holds its issuing thread for about as long as the tensor pipe needs for it, so
+// the two product chains of a tile are issued by two threads. K and V stages are released
+// separately: K once S has read it, V once P·V has.
 #include "common.cuh"
 #include "internal.h"
 
@@ -56,7 +63,8 @@ constexpr int kCkProducer = 4;     // Q and K
 constexpr int kCkMma = 5;
 constexpr int kCkVProducer = 10;
 constexpr int kCkPv = 11;          // issues the P·V products (warp 5 the S products)
-constexpr int kCkThreads = 12 * 32;
+constexpr int kCkSoft2 = 12;       // warps 12-15: the second key half of the softmax
+constexpr int kCkThreads = 16 * 32;
 constexpr uint32_t kCkTmemCols = 512;
 constexpr uint32_t kColS0 = 0;     // S/P buffers at columns 0 and 128
 constexpr uint32_t kColOHi = 256;  // O accumulator of the P_hi products (D columns); the
@@ -75,8 +83,19 @@ struct __align__(1024) CkSmem {
   int32_t meta[kCkKStages];                      // valid keys of the K stage (MMA warp)
   int32_t item_slot[2][2];                       // item index (-1: stop), key tiles
   TileItem item[2];
-  // hand-off to the epilogue warps, by item parity: per-row running max and sum, the item
-  float mfin[2][kCkRows], lfin[2][kCkRows];
+  // each softmax warp's scaled tile maxima, [parity][2 quarter + half][lane]: per-head and
+  // larger head-packed tiles swap them within a lane quarter (xpair[parity][quarter], two
+  // arrivals), quarter items among all eight warps (xall[parity], eight arrivals); each kind
+  // counts its own tiles for the parity
+  float tmx_pair[2][8][32], tmx_all[2][8][32];
+  uint64_t xpair[2][4], xall[2];
+  // quarter items: the four lane quarters' partial O (32 columns at a time) meet here, and
+  // lane quarter 0 adds them (redfull: the four partials written; redfree: added)
+  float red[4][32][33];
+  uint64_t redfull, redfree;
+  // hand-off to the epilogue warps, by item parity: per-row running max, each key half's running
+  // sum, the item
+  float mfin[2][kCkRows], lfin[2][2][kCkRows];
   TileItem epi[2];
   int32_t epi_stop[2];
   uint64_t kfull[kCkKStages], kempty[kCkKStages], vfull[kCkVStages], vempty[kCkVStages];
@@ -100,10 +119,57 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
   return *reinterpret_cast<const uint32_t*>(&h);
 }
 
+// Maximum of the visible keys among W consecutive S values of a row (key kbeg + i is visible
+// when < nvis; full: all are); four independent maxima keep the dependency chains short.
+template <int W>
+__device__ __forceinline__ float masked_max(const uint32_t* raw, bool full, int kbeg, int nvis) {
+  float mx[4];
+#pragma unroll
+  for (int a = 0; a < 4; ++a) mx[a] = -INFINITY;
+  if (full) {
+#pragma unroll
+    for (int i = 0; i < W; ++i) mx[i & 3] = fmaxf(mx[i & 3], __uint_as_float(raw[i]));
+  } else {
+#pragma unroll
+    for (int i = 0; i < W; ++i)
+      if (kbeg + i < nvis) mx[i & 3] = fmaxf(mx[i & 3], __uint_as_float(raw[i]));
+  }
+  return fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
+}
+
+// p = 2^(s·scale − m) for W consecutive S values of a row (invisible keys give 0), as bf16 pairs:
+// whi[i] holds the nearest bf16 of keys 2i and 2i + 1, wlo[i] that of their fp32 remainders.
+// Returns the fp32 sum of the p.
+template <int W>
+__device__ __forceinline__ float exp_split(const uint32_t* raw, bool full, int kbeg, int nvis,
+                                           float scale, float negm, uint32_t (&whi)[W / 2],
+                                           uint32_t (&wlo)[W / 2]) {
+  float rsum[4];  // four independent partial sums of p
+#pragma unroll
+  for (int a = 0; a < 4; ++a) rsum[a] = 0.f;
+#pragma unroll
+  for (int i = 0; i < W; i += 2) {
+    float x0 = fmaf(__uint_as_float(raw[i]), scale, negm);
+    float x1 = fmaf(__uint_as_float(raw[i + 1]), scale, negm);
+    if (!full) {
+      x0 = kbeg + i < nvis ? x0 : -INFINITY;
+      x1 = kbeg + i + 1 < nvis ? x1 : -INFINITY;
+    }
+    const float p0 = fast_exp2(x0), p1 = fast_exp2(x1);
+    rsum[(i >> 1) & 3] += p0 + p1;
+    const __nv_bfloat162 hi = __floats2bfloat162_rn(p0, p1);
+    const float2 hf = __bfloat1622float2(hi);
+    whi[i / 2] = *reinterpret_cast<const uint32_t*>(&hi);
+    wlo[i / 2] = pack_bf16x2(p0 - hf.x, p1 - hf.y);
+  }
+  return (rsum[0] + rsum[1]) + (rsum[2] + rsum[3]);
+}
+
 template <int kD>
 __global__ void __launch_bounds__(kCkThreads, 1)
     chunk_tc_kernel(const TileParams p, const __grid_constant__ CUtensorMap tmap_q,
                     const __grid_constant__ CUtensorMap tmap_qp,
+                    const __grid_constant__ CUtensorMap tmap_qq,
                     const __grid_constant__ CUtensorMap tmap_k,
                     const __grid_constant__ CUtensorMap tmap_v) {
   using Smem = CkSmem<kD>;
@@ -132,16 +198,20 @@ __global__ void __launch_bounds__(kCkThreads, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&S.qfull[i], 1);
-      mbar_init(&S.qempty[i], 1 + 4 + 1 + 1);  // S issuer, softmax warps, V producer, P·V issuer
+      mbar_init(&S.qempty[i], 1 + 8 + 1 + 1);  // S issuer, softmax warps, V producer, P·V issuer
       mbar_init(&S.sfull[i], 1);
       mbar_init(&S.sfree[i], 1);
-      mbar_init(&S.pfull[i], 4);
-      mbar_init(&S.lready[i], 4);
+      mbar_init(&S.pfull[i], 8);
+      mbar_init(&S.lready[i], 8);
       mbar_init(&S.lfree[i], 4);
+      for (int q = 0; q < 4; ++q) mbar_init(&S.xpair[i][q], 2);
+      mbar_init(&S.xall[i], 8);
     }
     mbar_init(&S.pfree, 1);
     mbar_init(&S.ofin, 1);
     mbar_init(&S.oempty, 4);
+    mbar_init(&S.redfull, 4);
+    mbar_init(&S.redfree, 1);
     mbar_init(&S.drain, 1);
     mbar_init(&S.drain_pv, 1);
     S.abort_flag = 0;
@@ -154,6 +224,7 @@ __global__ void __launch_bounds__(kCkThreads, 1)
   if (warp == kCkProducer && lane == 0) {
     prefetch_tensor_map(&tmap_q);
     prefetch_tensor_map(&tmap_qp);
+    prefetch_tensor_map(&tmap_qq);
     prefetch_tensor_map(&tmap_k);
     prefetch_tensor_map(&tmap_v);
   }
@@ -185,7 +256,16 @@ __global__ void __launch_bounds__(kCkThreads, 1)
         S.item_slot[ps][0] = idx;
         S.item_slot[ps][1] = ntile;
         S.item[ps] = it;
-        if (it.head_packed) {
+        if (it.head_packed && it.rows <= p.quad_rows) {
+          // a quarter item: the request's rows of G heads (at most 32 tile rows, ordered (chunk
+          // row, head)) once in each lane quarter
+          mbar_arrive_expect_tx(&S.qfull[ps], 4u * kHalves * 128u * static_cast<uint32_t>(p.g * p.qq_box_rows));
+#pragma unroll
+          for (int hf = 0; hf < kHalves; ++hf)
+#pragma unroll
+            for (int q4 = 0; q4 < 4; ++q4)
+              tma_load_3d(S.q[ps][hf] + q4 * 32 * 64, &tmap_qq, &S.qfull[ps], 64 * hf, it.h * p.g, it.row0);
+        } else if (it.head_packed) {
           // G heads x qp_box_rows chunk rows, rows ordered (chunk row, head)
           mbar_arrive_expect_tx(&S.qfull[ps], kHalves * 128u * static_cast<uint32_t>(p.g * p.qp_box_rows));
 #pragma unroll
@@ -364,13 +444,19 @@ __global__ void __launch_bounds__(kCkThreads, 1)
       mbar_drain(&S.drain_pv, 0);
     }
     __syncwarp();
-  } else if (warp < 4) {
-    // ======================= softmax (thread = query row) =======================
-    // The four warps never meet at a named barrier (rows are independent), so a warp whose wait
-    // timed out may leave on its own.
-    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
-    const int r = tid;
+  } else if (warp < 4 || warp >= kCkSoft2) {
+    // ======================= softmax (thread = TMEM lane, warp = keys of the tile) =======================
+    // Warps meet only at a bounded mbarrier wait (the tile-maximum exchange), never at a named
+    // barrier, so a warp whose wait timed out may leave on its own: the others' next waits time
+    // out too.
+    const int quad = warp & 3;
+    const int half = warp >= kCkSoft2 ? 1 : 0;
+    const int wslot = 2 * quad + half;
+    const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
+    const int r = quad * 32 + lane;     // TMEM lane = tile row
+    const int stid = half * 128 + r;    // 0..255 over the eight softmax warps
     uint32_t J = 0, K = 0;
+    uint32_t Jp = 0, Ja = 0;  // tiles of each exchange kind so far
     bool ok = true;
     while (ok) {
       const int ps = K & 1;
@@ -392,17 +478,29 @@ __global__ void __launch_bounds__(kCkThreads, 1)
       }
       // The item's descriptor goes to the epilogue warps now (their hand-off slot of this parity
       // is free once they have read the item two back), so it need not stay in registers across
-      // the key tiles; the per-row max and sum follow at the end.
+      // the key tiles; the per-row max and sums follow at the end.
       if (!mbar_wait(&S.lfree[ob], ((K >> 1) & 1u) ^ 1u, ctx)) break;
       if (tid == 0) {
         S.epi[ob] = it;
         S.epi_stop[ob] = 0;
       }
-      // chunk position of this tile row (head-packed: row r is position r / G of head r mod G)
-      // and the last key it sees (below every key when the row lies outside the chunk)
-      const int pos = it.head_packed ? (r * p.g_recip16) >> 16 : r;
+      // Tile rows. A quarter item (a head-packed request of c <= 32 / G rows) holds its c G rows
+      // in every lane quarter (row r is slot r mod 32: chunk position slot / G of head
+      // slot mod G), and each of the eight warps takes 16 keys of a tile: quarter q and half h
+      // take keys 32 q + 16 h + [0, 16), so a row's 128 keys are spread over eight warps on four
+      // schedulers. Other head-packed tiles hold position r / G of head r mod G, per-head tiles
+      // position r; there each half takes 64 keys.
+      const bool quarter_item = it.head_packed && it.rows <= p.quad_rows;
+      const int prow = quarter_item ? lane : r;
+      const int pos = it.head_packed ? (prow * p.g_recip16) >> 16 : r;
       const int limit = pos < it.rows ? it.prefix + it.pos0 + pos : -1;
-      float m = -INFINITY, l = 0.f;
+      // A warp whose 32 rows all lie outside the chunk (the last lane quarter of a head-packed
+      // tile of 9 rows x 8 heads, say) has no output: it leaves its rows' P as the S bits it
+      // finds, so those rows of O hold garbage that the epilogue never stores, and the next
+      // item's first products overwrite.
+      const bool dead = __all_sync(0xffffffffu, pos >= it.rows);
+      const int kbeg = quarter_item ? 32 * quad + 16 * half : 64 * half;
+      float m = -INFINITY, l = 0.f;  // l: the sum over this warp's keys
       for (int j = 0; j < ntile; ++j, ++J) {
         const int sb = J & 1;
         if (!mbar_wait(&S.sfull[sb], (J >> 1) & 1u, ctx)) { ok = false; break; }
@@ -415,42 +513,62 @@ __global__ void __launch_bounds__(kCkThreads, 1)
         const int nvis = max(0, min(valid, limit - kt0 + 1));
         const bool full = __all_sync(0xffffffffu, nvis == kCkKeys);
         const uint32_t sp = tmem + lane_base + kColS0 + sb * 128;  // this tile's S, then its P
-        // pass 1: the row's maximum over its visible keys (scale > 0, so it is applied after);
-        // four independent maxima keep the dependency chains short
-        float tmax = -INFINITY;
-        if (valid > 0) {
-          float mx[4];
-#pragma unroll
-          for (int a = 0; a < 4; ++a) mx[a] = -INFINITY;
-#pragma unroll 1
-          for (int h = 0; h < kCkKeys; h += 64) {
-            uint32_t raw[64];
-            tmem_ld32(sp + h, *reinterpret_cast<uint32_t(*)[32]>(raw));
-            tmem_ld32(sp + h + 32, *reinterpret_cast<uint32_t(*)[32]>(raw + 32));
+        // pass 1: the maximum over this warp's visible keys (scale > 0, so it is applied after);
+        // a quarter item keeps its 16 values for pass 2, the 64-key halves go 32 keys at a time
+        // in rolled loops (the eight roles' code shares the instruction cache)
+        uint32_t raw16[16];
+        float hmax = -INFINITY;
+        if (valid > 0 && !dead) {
+          if (quarter_item) {
+            tmem_ld16(sp + kbeg, raw16);
             tmem_wait_ld();
-            if (full) {
-#pragma unroll
-              for (int i = 0; i < 64; ++i) mx[i & 3] = fmaxf(mx[i & 3], __uint_as_float(raw[i]));
-            } else {
-#pragma unroll
-              for (int i = 0; i < 64; ++i)
-                if (h + i < nvis) mx[i & 3] = fmaxf(mx[i & 3], __uint_as_float(raw[i]));
+            hmax = masked_max<16>(raw16, full, kbeg, nvis);
+          } else {
+#pragma unroll 1
+            for (int c = 0; c < 64; c += 32) {
+              uint32_t raw[32];
+              tmem_ld32(sp + kbeg + c, raw);
+              tmem_wait_ld();
+              hmax = fmaxf(hmax, masked_max<32>(raw, full, kbeg + c, nvis));
             }
           }
-          tmax = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
-          tmax *= p.scale_log2;
+          hmax *= p.scale_log2;
         }
+        // the row's tile maximum: every warp posts its own, then reads those of the warps that
+        // share its row (the other half of its quarter; in a quarter item all eight)
+        float tmax;
+        if (quarter_item) {
+          float (&x)[8][32] = S.tmx_all[Ja & 1];
+          x[wslot][lane] = hmax;
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&S.xall[Ja & 1]);
+          if (!mbar_wait(&S.xall[Ja & 1], (Ja >> 1) & 1u, ctx)) { ok = false; break; }
+          tmax = x[0][lane];
+#pragma unroll
+          for (int w = 1; w < 8; ++w) tmax = fmaxf(tmax, x[w][lane]);
+          ++Ja;
+        } else {
+          float (&x)[8][32] = S.tmx_pair[Jp & 1];
+          x[wslot][lane] = hmax;
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&S.xpair[Jp & 1][quad]);
+          if (!mbar_wait(&S.xpair[Jp & 1][quad], (Jp >> 1) & 1u, ctx)) { ok = false; break; }
+          tmax = fmaxf(x[2 * quad][lane], x[2 * quad + 1][lane]);
+          ++Jp;
+        }
+        // every warp of a row reaches the same decisions from the same numbers
         const float mn = fmaxf(m, tmax);
         const bool move = mn > m + kRescaleThreshold || (m == -INFINITY && mn != -INFINITY);
         const float mref = move ? mn : m;
         const float alpha = move ? (m == -INFINITY ? 0.f : fast_exp2(m - mn)) : 1.f;
         if (j > 0 && __any_sync(0xffffffffu, move)) {
-          // O changes only after the previous product has added into it
+          // O changes only after the previous product has added into it; half 0 rescales O_hi,
+          // half 1 O_lo (each lane quarter its own rows, or its own copy of them)
           if (!mbar_wait(&S.pfree, (J - 1) & 1u, ctx)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t oc = tmem + lane_base + kColOHi;  // O_hi, then O_lo right after it
+          const uint32_t oc = tmem + lane_base + kColOHi + half * kD;
 #pragma unroll 1
-          for (int c = 0; c < 2 * kD; c += 32) {
+          for (int c = 0; c < kD; c += 32) {
             uint32_t o[32];
             tmem_ld32(oc + c, o);
             tmem_wait_ld();
@@ -459,46 +577,46 @@ __global__ void __launch_bounds__(kCkThreads, 1)
             tmem_st32(oc + c, o);
           }
         }
-        // pass 2, 64 keys at a time: p = 2^(s·scale − m), split into bf16 hi + lo and written over
-        // the tile's own S columns (a 32-key chunk's words cover only columns already read). hi is
-        // p rounded to the nearest bf16 and lo the exact fp32 remainder p − hi, rounded the same
-        // way, so |p − hi − lo| <= 2^-17 p, without bias. mref = −inf only when no key is visible,
-        // and then every x below is −inf already.
+        // pass 2: p = 2^(s·scale − m) over this warp's keys, split into bf16 hi + lo and written
+        // over the tile's own S columns (each 32-key chunk: 16 words of hi pairs, then 16 of lo
+        // pairs; a warp writes only columns it or its half-partner has read). hi is p rounded to
+        // the nearest bf16 and lo the exact fp32 remainder p − hi, rounded the same way, so
+        // |p − hi − lo| <= 2^-17 p, without bias. mref = −inf only when no key is visible, and
+        // then every x is −inf already. A quarter item's row copy also zeroes the P words of the
+        // keys other quarters take, so the four copies' products are partial sums.
         const float negm = mref == -INFINITY ? 0.f : -mref;
-        float rsum[4];  // four independent partial sums of p
+        float rs = 0.f;
+        if (!dead) {
+          if (quarter_item) {
+            uint32_t whi[8], wlo[8];
+            rs = exp_split<16>(raw16, full, kbeg, nvis, p.scale_log2, negm, whi, wlo);
+            const uint32_t chunk = sp + 32 * quad;
+            tmem_st8(chunk + 8 * half, whi);
+            tmem_st8(chunk + 16 + 8 * half, wlo);
+            uint32_t z[32];
 #pragma unroll
-        for (int a = 0; a < 4; ++a) rsum[a] = 0.f;
-#pragma unroll 1
-        for (int h = 0; h < kCkKeys; h += 64) {
-          uint32_t raw[64];
-          if (valid > 0) {
-            tmem_ld32(sp + h, *reinterpret_cast<uint32_t(*)[32]>(raw));
-            tmem_ld32(sp + h + 32, *reinterpret_cast<uint32_t(*)[32]>(raw + 32));
-            tmem_wait_ld();
-          }
-#pragma unroll
-          for (int c = 0; c < 64; c += 32) {
-            uint32_t w[32];
-#pragma unroll
-            for (int i = 0; i < 32; i += 2) {
-              const int k0 = h + c + i;
-              float x0 = fmaf(__uint_as_float(raw[c + i]), p.scale_log2, negm);
-              float x1 = fmaf(__uint_as_float(raw[c + i + 1]), p.scale_log2, negm);
-              if (!full) {
-                x0 = k0 < nvis ? x0 : -INFINITY;
-                x1 = k0 + 1 < nvis ? x1 : -INFINITY;
-              }
-              const float p0 = fast_exp2(x0), p1 = fast_exp2(x1);
-              rsum[(i >> 1) & 3] += p0 + p1;
-              const __nv_bfloat162 hi = __floats2bfloat162_rn(p0, p1);
-              const float2 hf = __bfloat1622float2(hi);
-              w[i / 2] = *reinterpret_cast<const uint32_t*>(&hi);
-              w[16 + i / 2] = pack_bf16x2(p0 - hf.x, p1 - hf.y);
+            for (int i = 0; i < 32; ++i) z[i] = 0u;
+            if (half == 0) {
+              tmem_st32(sp + 32 * ((quad + 1) & 3), z);
+              tmem_st32(sp + 32 * ((quad + 2) & 3), z);
+            } else {
+              tmem_st32(sp + 32 * ((quad + 3) & 3), z);
             }
-            tmem_st32(sp + h + c, w);
+          } else {
+#pragma unroll 1
+            for (int c = 0; c < 64; c += 32) {
+              uint32_t raw[32], w[32];
+              if (valid > 0) {
+                tmem_ld32(sp + kbeg + c, raw);
+                tmem_wait_ld();
+              }
+              rs += exp_split<32>(raw, full, kbeg + c, nvis, p.scale_log2, negm,
+                                  *reinterpret_cast<uint32_t(*)[16]>(w),
+                                  *reinterpret_cast<uint32_t(*)[16]>(w + 16));
+              tmem_st32(sp + kbeg + c, w);
+            }
           }
         }
-        const float rs = (rsum[0] + rsum[1]) + (rsum[2] + rsum[3]);
         l = fmaf(l, alpha, rs);
         m = mref;
         if ((valid & 15) != 0) {
@@ -506,7 +624,7 @@ __global__ void __launch_bounds__(kCkThreads, 1)
           const int vs = J % kCkVStages;
           if (!mbar_wait(&S.vfull[vs], (J / kCkVStages) & 1u, ctx)) { ok = false; break; }
           const int r0 = valid, r1 = (valid + 15) & ~15;
-          for (int c = tid; c < (r1 - r0) * 8 * kHalves; c += 128) {
+          for (int c = stid; c < (r1 - r0) * 8 * kHalves; c += 256) {
             const int row = r0 + c / (8 * kHalves);
             *reinterpret_cast<uint4*>(reinterpret_cast<unsigned char*>(S.v[vs][(c / 8) % kHalves]) +
                                       row * 128 + (c & 7) * 16) = make_uint4(0u, 0u, 0u, 0u);
@@ -519,9 +637,9 @@ __global__ void __launch_bounds__(kCkThreads, 1)
         if (lane == 0) mbar_arrive(&S.pfull[sb]);
       }
       if (!ok) break;
-      // ---- hand the rows' running max and sum to the epilogue warps ----
-      S.mfin[ob][r] = m;
-      S.lfin[ob][r] = l;
+      // ---- hand the rows' running max and this warp's sum to the epilogue warps ----
+      if (half == 0) S.mfin[ob][r] = m;
+      S.lfin[ob][half][r] = l;
       __syncwarp();
       if (lane == 0) mbar_arrive(&S.lready[ob]);
       ++K;
@@ -531,25 +649,36 @@ __global__ void __launch_bounds__(kCkThreads, 1)
     const int quad = warp & 3;
     const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
     const int r = quad * 32 + lane;
-    for (uint32_t K = 0;; ++K) {
+    uint32_t E = 0;  // reduction steps of quarter items so far (the same count in all four warps)
+    bool ok = true;
+    for (uint32_t K = 0; ok; ++K) {
       const uint32_t ob = K & 1;
       if (!mbar_wait(&S.lready[ob], (K >> 1) & 1u, ctx)) break;
       if (S.epi_stop[ob]) break;
       const TileItem it = S.epi[ob];
+      const bool quarter_item = it.head_packed && it.rows <= p.quad_rows;
+      // a quarter item's row (slot = lane) has a running sum in each of the eight softmax warps
       const float m = S.mfin[ob][r];
-      const float l = S.lfin[ob][r];
+      float l = S.lfin[ob][0][r] + S.lfin[ob][1][r];
+      if (quarter_item)
+#pragma unroll
+        for (int q = 1; q < 4; ++q)
+          l += S.lfin[ob][0][((quad + q) & 3) * 32 + lane] + S.lfin[ob][1][((quad + q) & 3) * 32 + lane];
       __syncwarp();
       if (lane == 0) mbar_arrive(&S.lfree[ob]);
       if (!mbar_wait(&S.ofin, K & 1u, ctx)) break;
       tc_fence_after();
-      const int pos = it.head_packed ? (r * p.g_recip16) >> 16 : r;  // chunk position of the row
-      const bool row_ok = pos < it.rows;
+      // chunk position and query head of the row (the tile-row layouts of the softmax warps);
+      // a quarter item's output is written by lane quarter 0, from the sum of the four copies
+      const int prow = quarter_item ? lane : r;
+      const int pos = it.head_packed ? (prow * p.g_recip16) >> 16 : r;
+      const bool row_ok = pos < it.rows && (!quarter_item || quad == 0);
       const bool direct = it.nsplit == 1;
       const float inv = l > 0.f ? 1.f / l : 0.f;
       const float lse2 = l > 0.f ? m + log2f(l) : -INFINITY;
       // a row that saw no key has O = 0 (its accumulator may never have been written)
       const bool seen = l > 0.f;
-      const int head = it.head_packed ? it.h * p.g + (r - pos * p.g) : it.h;  // query head
+      const int head = it.head_packed ? it.h * p.g + (prow - pos * p.g) : it.h;  // query head
       const int hkv = head / p.g, g = head - hkv * p.g;
       const int64_t row = static_cast<int64_t>(it.row0) + pos;
       const int64_t slot = static_cast<int64_t>(it.slot0) +
@@ -565,9 +694,30 @@ __global__ void __launch_bounds__(kCkThreads, 1)
         tmem_ld32(tmem + lane_base + kColOLo + c, lo);
         tmem_wait_ld();
 #pragma unroll
-        for (int i = 0; i < 32; ++i)
-          o[i] = seen ? __float_as_uint(__uint_as_float(o[i]) + __uint_as_float(lo[i])) : 0u;
+        for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) + __uint_as_float(lo[i]));
+        if (quarter_item) {
+          // the four lane quarters' partial sums meet in shared memory (the buffer is free once
+          // quarter 0 has added the previous step's)
+          if (!mbar_wait(&S.redfree, (E & 1u) ^ 1u, ctx)) { ok = false; break; }
+#pragma unroll
+          for (int i = 0; i < 32; ++i) S.red[quad][lane][i] = __uint_as_float(o[i]);
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&S.redfull);
+          if (quad == 0) {
+            if (!mbar_wait(&S.redfull, E & 1u, ctx)) { ok = false; break; }
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+              o[i] = __float_as_uint((S.red[0][lane][i] + S.red[1][lane][i]) +
+                                     (S.red[2][lane][i] + S.red[3][lane][i]));
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&S.redfree);
+          }
+          ++E;
+        }
         if (row_ok) {
+          if (!seen)
+#pragma unroll
+            for (int i = 0; i < 32; ++i) o[i] = 0u;
           if (direct) {
 #pragma unroll
             for (int i = 0; i < 32; i += 8) {
@@ -587,6 +737,7 @@ __global__ void __launch_bounds__(kCkThreads, 1)
           }
         }
       }
+      if (!ok) break;
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&S.oempty);  // both accumulators read: the next item may start
@@ -605,8 +756,8 @@ __global__ void __launch_bounds__(kCkThreads, 1)
 
 template <int kD>
 cudaError_t launch_chunk_tc_t(const TileParams& p, const CUtensorMap& tq, const CUtensorMap& tqp,
-                              const CUtensorMap& tk, const CUtensorMap& tv, int nctas,
-                              cudaStream_t stream) {
+                              const CUtensorMap& tqq, const CUtensorMap& tk, const CUtensorMap& tv,
+                              int nctas, cudaStream_t stream) {
   const size_t smem = sizeof(CkSmem<kD>) + 1024;
   cudaError_t e = cudaFuncSetAttribute(chunk_tc_kernel<kD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
@@ -621,16 +772,16 @@ cudaError_t launch_chunk_tc_t(const TileParams& p, const CUtensorMap& tq, const 
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, chunk_tc_kernel<kD>, p, tq, tqp, tk, tv);
+  return cudaLaunchKernelEx(&cfg, chunk_tc_kernel<kD>, p, tq, tqp, tqq, tk, tv);
 }
 
 }  // namespace
 
 cudaError_t launch_chunk_tc(const TileParams& p, const CUtensorMap& tq, const CUtensorMap& tqp,
-                            const CUtensorMap& tk, const CUtensorMap& tv, int nctas,
-                            cudaStream_t stream) {
-  if (p.d == 128) return launch_chunk_tc_t<128>(p, tq, tqp, tk, tv, nctas, stream);
-  if (p.d == 64) return launch_chunk_tc_t<64>(p, tq, tqp, tk, tv, nctas, stream);
+                            const CUtensorMap& tqq, const CUtensorMap& tk, const CUtensorMap& tv,
+                            int nctas, cudaStream_t stream) {
+  if (p.d == 128) return launch_chunk_tc_t<128>(p, tq, tqp, tqq, tk, tv, nctas, stream);
+  if (p.d == 64) return launch_chunk_tc_t<64>(p, tq, tqp, tqq, tk, tv, nctas, stream);
   return cudaErrorInvalidValue;
 }
 

@@ -99,6 +99,8 @@ struct TileParams {
   int32_t hq, hkv, g, d, cap;
   int32_t q_box_rows;   // rows of one Q tensor-map box: min(128, T)
   int32_t qp_box_rows;  // chunk rows of one head-packed Q box (G heads each): min(128 / G, T)
+  int32_t quad_rows;    // head-packed requests of <= 32 / G rows are quarter items (0: none)
+  int32_t qq_box_rows;  // chunk rows of one quarter-item Q box (G heads each): min(32 / G, T)
   int32_t g_recip16;    // ceil(2^16 / G): (r * g_recip16) >> 16 == r / G for 0 <= r < 128
   int32_t kv_box_rows;  // rows of one K/V tensor-map box: min(128, S_cap)
   float scale_log2;
@@ -136,8 +138,9 @@ cudaError_t launch_decode_tc(const DecodeParams& p, const CUtensorMap& tmap_q,
 // tcgen05 chunked-prefill tile kernel: bf16, D == 64 or 128. tmap_qp loads head-packed Q tiles
 // (G heads x qp_box_rows rows); any Q map when no tile is head-packed.
 cudaError_t launch_chunk_tc(const TileParams& p, const CUtensorMap& tmap_q,
-                            const CUtensorMap& tmap_qp, const CUtensorMap& tmap_k,
-                            const CUtensorMap& tmap_v, int nctas, cudaStream_t stream);
+                            const CUtensorMap& tmap_qp, const CUtensorMap& tmap_qq,
+                            const CUtensorMap& tmap_k, const CUtensorMap& tmap_v, int nctas,
+                            cudaStream_t stream);
 
 // Launched with programmatic dependent launch after a split kernel (tensor-core decode path; the
 // CUDA-core kernel merges its own groups in-kernel).

@@ -240,6 +240,8 @@ __global__ void __launch_bounds__(kMaxPlanThreads, 1) plan_chunk_kernel(PlanPara
   int32_t* s_roff = s_tmp + B;         // B + 1: first packed row of each request
   int32_t* s_dioff = s_roff + B + 1;   // B + 1: decode item offsets (rank order)
   int32_t* s_tioff = s_dioff + B + 1;  // B + 1: tile item offsets (request order)
+  int32_t* s_nmax = s_tioff + B + 1;   // key splits of a request's last query tile (0: no tiles)
+  int32_t* s_soff = s_nmax + B;        // B + 1: first (request, split) pair of each request
   __shared__ int s_scan[33];
   __shared__ unsigned long long s_total;
   __shared__ unsigned long long s_key_tiles;  // 128-key tiles of all tile items
@@ -281,6 +283,7 @@ __global__ void __launch_bounds__(kMaxPlanThreads, 1) plan_chunk_kernel(PlanPara
       s_n[b] = n;
       s_key[b] = plan_sort_key(s_dlen[b], n);
       s_tcnt[b] = 0;
+      s_nmax[b] = 0;
     } else {
       s_n[b] = 0;
       s_key[b] = -1;
@@ -293,6 +296,7 @@ __global__ void __launch_bounds__(kMaxPlanThreads, 1) plan_chunk_kernel(PlanPara
       }
       const int32_t nheads = chunk_packed(c, p.hq / p.hkv) ? p.hkv : p.hq;
       s_tcnt[b] = cnt * nheads;
+      s_nmax[b] = c > 1 ? chunk_tile_splits(chunk_tile_keys(s_p[b], c, (c - 1) / kQTile, p.cap)) : 0;
       if (c > 1) atomicAdd(&s_key_tiles, static_cast<unsigned long long>(ktiles * nheads));
     }
   }
@@ -315,6 +319,7 @@ __global__ void __launch_bounds__(kMaxPlanThreads, 1) plan_chunk_kernel(PlanPara
   __syncthreads();
   block_exclusive_scan(s_tmp, s_dioff, nd, s_scan);
   block_exclusive_scan(s_tcnt, s_tioff, B, s_scan);
+  block_exclusive_scan(s_nmax, s_soff, B, s_scan);
   // chunk lengths that do not add up to the packed rows of q_chunk: nothing is computed (the
   // outputs are left as they were) and the status word says why
   const bool inconsistent = s_roff[B] != T;
@@ -331,72 +336,83 @@ __global__ void __launch_bounds__(kMaxPlanThreads, 1) plan_chunk_kernel(PlanPara
     for (int32_t row = tid; row < T; row += nthr) p.row_nsplit[row] = 0;
   __syncthreads();
   block_exclusive_scan(p.row_nsplit, p.row_base, T, s_scan);
+  // partial-slot base of each request's first row, for the item loops below (s_tmp is free
+  // again: the decode ranks' scan has consumed it)
+  int32_t* s_rb = s_tmp;
+  for (int b = tid; b < B && !inconsistent; b += nthr) s_rb[b] = s_c[b] > 0 ? p.row_base[s_roff[b]] : 0;
+  __syncthreads();
 
   const int32_t n_dec_items = s_dioff[nd];
   const int32_t n_tile_items = s_tioff[B];
   const bool overflow =
       inconsistent || n_dec_items > p.max_dec_items || n_tile_items > p.max_tile_items;
-  // decode items: one warp per decode request, lanes over splits
+  // decode items: one warp per decode request, lanes over its (KV head, split) items
   for (int r = warp; r < nd && !overflow; r += nthr / 32) {
     const int b = s_order[r];
     const int32_t row = s_roff[b];
     const int32_t n = s_n[b], L = s_dlen[b], first = s_dioff[r];
-    const int32_t rbase = p.row_base[row];
-    for (int32_t s = lane; s < n; s += 32) {
+    const int32_t rbase = s_rb[b];
+    for (int32_t e = lane; e < n * p.hkv; e += 32) {
+      const int32_t h = e / n, s = e - h * n;
       int32_t t0, t1;
       plan_split_range(L, n, s, 0, 1, &t0, &t1);
-      for (int32_t h = 0; h < p.hkv; ++h) {
-        int4* dst = reinterpret_cast<int4*>(p.items + first + h * n + s);
-        dst[0] = make_int4(row, b, h, s);
-        dst[1] = make_int4(t0, t1, n, rbase * p.hkv + h * n + s);
-      }
+      int4* dst = reinterpret_cast<int4*>(p.items + first + e);
+      dst[0] = make_int4(row, b, h, s);
+      dst[1] = make_int4(t0, t1, n, rbase * p.hkv + h * n + s);
     }
   }
-  // tile items: one warp per request, lanes over query heads (KV heads for head-packed tiles),
-  // (split, tile) order per head
-  for (int b = warp; b < B && !overflow; b += nthr / 32) {
-    const int32_t c = s_c[b];
-    if (c < 2) continue;
-    const int32_t pp = s_p[b], r0 = s_roff[b];
+  // tile items: one warp per (request, split) pair, lanes over query heads (KV heads for
+  // head-packed tiles). Per head the items run split by split and, within a split, tile by tile
+  // over the query tiles that see that split's keys.
+  const int32_t n_pairs = s_soff[B];
+  for (int k = warp; k < n_pairs && !overflow; k += nthr / 32) {
+    int lo = 0, hi = B;  // the request of pair k: s_soff[lo] <= k < s_soff[lo + 1]
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (s_soff[mid] <= k) lo = mid; else hi = mid;
+    }
+    const int b = lo;
+    const int32_t s = k - s_soff[b];
+    const int32_t c = s_c[b], pp = s_p[b], r0 = s_roff[b];
     const int32_t ntiles = (c + kQTile - 1) / kQTile;
     const int32_t head_packed = chunk_packed(c, p.hq / p.hkv) ? 1 : 0;
     const int32_t nheads = head_packed ? p.hkv : p.hq;
     const int32_t per_head = s_tcnt[b] / nheads;
-    const int32_t nmax = chunk_tile_splits(chunk_tile_keys(pp, c, ntiles - 1, p.cap));
-    // partial-slot base of the request's first row, read once: the bases of its later tiles
-    // follow from the split counts (every row of tile t has nt(t) slots and the tiles before the
-    // last are full), so the loop below makes no dependent global load per item
-    const int32_t rb0 = p.row_base[r0];
+    // items of the earlier splits in each head's run: query tile t has min(nt(t), s) of them
+    int32_t before = 0;
+    for (int32_t t = 0; t < ntiles; ++t)
+      before += min(chunk_tile_splits(chunk_tile_keys(pp, c, t, p.cap)), s);
+    // the bases of the request's later tiles follow from its first row's: every row of tile t
+    // has nt(t) slots and the tiles before the last are full
+    const int32_t rb0 = s_rb[b];
     for (int32_t h = lane; h < nheads; h += 32) {
-      int32_t i = s_tioff[b] + h * per_head;
-      for (int32_t s = 0; s < nmax; ++s) {
-        int32_t next_base = rb0;
-        for (int32_t t = 0; t < ntiles; ++t) {
-          const int32_t kt = chunk_tile_keys(pp, c, t, p.cap);
-          const int32_t nt = chunk_tile_splits(kt);
-          const int32_t tbase = next_base;  // row_base of tile t's first row
-          next_base += kQTile * nt;
-          if (s >= nt) continue;
-          const int32_t row0 = r0 + t * kQTile;
-          const int32_t rows = min(kQTile, c - t * kQTile);
-          const int32_t k0 = min(s * kChunkKvSplit, kt), k1 = min((s + 1) * kChunkKvSplit, kt);
-          const int32_t slot0 = tbase * p.hkv;
-          int4* dst = reinterpret_cast<int4*>(p.tiles + i);
-          dst[0] = make_int4(b, h, s, nt);
-          dst[1] = make_int4(k0, k1, row0, t * kQTile);
-          dst[2] = make_int4(rows, pp, slot0, head_packed);
-          dst[3] = make_int4(0, 0, 0, 0);
-          ++i;
-        }
+      int32_t i = s_tioff[b] + h * per_head + before;
+      int32_t next_base = rb0;
+      for (int32_t t = 0; t < ntiles; ++t) {
+        const int32_t kt = chunk_tile_keys(pp, c, t, p.cap);
+        const int32_t nt = chunk_tile_splits(kt);
+        const int32_t tbase = next_base;  // row_base of tile t's first row
+        next_base += kQTile * nt;
+        if (s >= nt) continue;
+        const int32_t row0 = r0 + t * kQTile;
+        const int32_t rows = min(kQTile, c - t * kQTile);
+        const int32_t k0 = min(s * kChunkKvSplit, kt), k1 = min((s + 1) * kChunkKvSplit, kt);
+        int4* dst = reinterpret_cast<int4*>(p.tiles + i);
+        dst[0] = make_int4(b, h, s, nt);
+        dst[1] = make_int4(k0, k1, row0, t * kQTile);
+        dst[2] = make_int4(rows, pp, tbase * p.hkv, head_packed);
+        dst[3] = make_int4(0, 0, 0, 0);
+        ++i;
       }
     }
   }
   __syncthreads();
   // decode rows merged inside their split kernel: the combine skips them; their counters reset
-  for (int r = tid; r < nd && !inconsistent; r += nthr) {
+  for (int e = tid; e < nd * p.hkv && !inconsistent; e += nthr) {
+    const int r = e / p.hkv, h = e - r * p.hkv;
     const int32_t row = s_roff[s_order[r]];
-    if (p.decode_merged_in_kernel) p.row_nsplit[row] = 1;
-    for (int32_t h = 0; h < p.hkv; ++h) p.arrivals[row * p.hkv + h] = 0;
+    if (p.decode_merged_in_kernel && h == 0) p.row_nsplit[row] = 1;
+    p.arrivals[row * p.hkv + h] = 0;
   }
   if (warp == 0) {
     // the tile kernel's CTAs: the n of least chunk_tile_cost, smallest on ties; lane l weighs
@@ -440,7 +456,7 @@ __global__ void __launch_bounds__(kMaxPlanThreads, 1) plan_chunk_kernel(PlanPara
 }  // namespace
 
 cudaError_t launch_plan_chunk(const PlanParams& p, cudaStream_t stream) {
-  const size_t smem = sizeof(int32_t) * (11 * static_cast<size_t>(p.B) + 3);
+  const size_t smem = sizeof(int32_t) * (13 * static_cast<size_t>(p.B) + 4);
   if (smem > 48 * 1024) {
     cudaError_t e = cudaFuncSetAttribute(plan_chunk_kernel,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
