@@ -70,10 +70,13 @@ template <int GPAD, bool kF8 = false>
 struct __align__(1024) TcSmem {
   static constexpr int kNO = 2 * GPAD;           // Oᵀ columns: hi then lo
   static constexpr int kPGroups = kNO / 8;       // 8-column core-matrix groups of Pᵀ
-  static constexpr int kStages = kTcStages;
+  static constexpr int kStages = kTcStages;  // K stages
+  // V stages: an E4M3 tile's V path is longer (copy, expansion to f16, then P·V) and its stages
+  // are refilled only once that product has completed, so it keeps one stage more
+  static constexpr int kVStages = kF8 ? kTcStages + 1 : kTcStages;
   static constexpr int kKSlabs = kF8 ? 1 : 2;
   __nv_bfloat16 k[kStages][kKSlabs][kTcKeys * 64];  // [stage][d half][row*64 + col], SW128
-  __nv_bfloat16 v[kStages][2][kTcKeys * 64];
+  __nv_bfloat16 v[kVStages][2][kTcKeys * 64];
   __nv_bfloat16 q[2][2][16 * 64];                // [item parity][d half], SW128
   // E4M3 cache: Q as two E4M3 terms per head (rows 0-7 c1, rows 8-15 c2; 128 codes per row,
   // SW128), by item parity, and each head's scale 2^e
@@ -86,7 +89,7 @@ struct __align__(1024) TcSmem {
   float mfin[2][GPAD];                           // final running max
   int32_t epi[2][4];                             // row (-1: stop), KV head, splits, slot
   int32_t meta[kStages][2];                      // per stage: tile start, valid keys (MMA warp)
-  int32_t vmeta[kStages];                        // E4M3: valid keys of the stage's V tile
+  int32_t vmeta[kVStages];                        // E4M3: valid keys of the stage's V tile
   // in-kernel plan: lengths, split counts, rank order, partial-slot bases (row order) and item
   // offsets (rank order); both scans also store their total after the last entry (B + 1)
   int32_t plan_len[kFusedPlanMaxBatch], plan_n[kFusedPlanMaxBatch];
@@ -99,7 +102,7 @@ struct __align__(1024) TcSmem {
   DecodeItem item[2];                            // the item's descriptor (by item parity)
   // K and V of a stage are released separately: K once the Sᵀ product has read it, V once the
   // P·V product has, so the next K copy starts while the current tile is still in softmax.
-  uint64_t kfull[kStages], vfull[kStages], kempty[kStages], vempty[kStages];
+  uint64_t kfull[kStages], vfull[kVStages], kempty[kStages], vempty[kVStages];
   uint64_t qfull[2], qempty[2], sfull[2], sempty[2], pfull[2], pempty[2];
   uint64_t ofull[2];   // by tile parity: that tile's P·V product has completed
   uint64_t ofin[2];    // by item parity: the item's last P·V product has completed
@@ -108,7 +111,7 @@ struct __align__(1024) TcSmem {
   // E4M3 cache: the TMA completes vraw (V codes in the upper half of the stage); vfull then
   // means "expanded to f16" and is completed by the four expanding warps. q8full: the item's Q
   // terms are ready (the four Q warps).
-  uint64_t vraw[kStages];
+  uint64_t vraw[kVStages];
   uint64_t q8full[2];
   // paged cache: physical page ids of tile J in slot J mod kPidSlots, written by the Q/K producer
   // (pages < 128 keys: copied asynchronously kPidAhead tiles ahead by its 32 lanes) and released
@@ -306,6 +309,7 @@ __global__ void __launch_bounds__(kF8 ? kF8Threads : kTcThreads, 1)
   using Smem = TcSmem<GPAD, kF8>;
   constexpr int kNO = Smem::kNO;
   constexpr int kStages = Smem::kStages;
+  constexpr int kVStages = Smem::kVStages;
   constexpr int kThreads = kF8 ? kF8Threads : kTcThreads;
   constexpr uint32_t kColO = 32;  // Sᵀ buffers at columns [0, 32), O accumulators after them
   constexpr uint32_t kCols = kTmemCols;
@@ -322,8 +326,10 @@ __global__ void __launch_bounds__(kF8 ? kF8Threads : kTcThreads, 1)
   if (tid == 0) {
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&S.kfull[s], 1);
-      mbar_init(&S.vfull[s], kF8 ? 4 : 1);
       mbar_init(&S.kempty[s], 1);
+    }
+    for (int s = 0; s < kVStages; ++s) {
+      mbar_init(&S.vfull[s], kF8 ? 4 : 1);
       mbar_init(&S.vempty[s], 1);
       mbar_init(&S.vraw[s], 1);
     }
@@ -707,10 +713,10 @@ __global__ void __launch_bounds__(kF8 ? kF8Threads : kTcThreads, 1)
       if (lane == 0) mbar_arrive(&S.qempty[ps]);
       if (idx < 0) break;
       for (int j = 0; j < ntile; ++j, ++J) {
-        const int st = J % kStages;
+        const int st = J % kVStages;
         const int t = it.t0 + j * kTcKeys;
         const int valid = max(0, min(kTcKeys, it.t1 - t));
-        if (!warp_mbar_wait(&S.vempty[st], ((J / kStages) & 1u) ^ 1u, ctx)) { ok = false; break; }
+        if (!warp_mbar_wait(&S.vempty[st], ((J / kVStages) & 1u) ^ 1u, ctx)) { ok = false; break; }
         if (!warp_mbar_wait(&S.pidfull[J % kPidSlots], (J / kPidSlots) & 1u, ctx)) { ok = false; break; }
         const SmallPages sp = small_pages(t, valid, pshift);
         uint64_t* vbar = kF8 ? &S.vraw[st] : &S.vfull[st];
@@ -731,16 +737,16 @@ __global__ void __launch_bounds__(kF8 ? kF8Threads : kTcThreads, 1)
     if (lane == 0) {
       if constexpr (kF8) {
         // stop marker for the V expanding warps (a stage without a tile)
-        const int st = J % kStages;
-        if (ok && mbar_wait(&S.vempty[st], ((J / kStages) & 1u) ^ 1u, ctx)) {
+        const int st = J % kVStages;
+        if (ok && mbar_wait(&S.vempty[st], ((J / kVStages) & 1u) ^ 1u, ctx)) {
           S.vmeta[st] = -1;
           mbar_arrive(&S.vraw[st]);
         }
       }
       if (S.abort_flag) {
-        for (uint32_t back = 1; back <= kStages && back <= J; ++back) {
+        for (uint32_t back = 1; back <= kVStages && back <= J; ++back) {
           const uint32_t jj = J - back;
-          mbar_drain(kF8 ? &S.vraw[jj % kStages] : &S.vfull[jj % kStages], (jj / kStages) & 1u);
+          mbar_drain(kF8 ? &S.vraw[jj % kVStages] : &S.vfull[jj % kVStages], (jj / kVStages) & 1u);
         }
       }
     }
@@ -763,10 +769,10 @@ __global__ void __launch_bounds__(kF8 ? kF8Threads : kTcThreads, 1)
         mbar_arrive(&S.qempty[ps]);
         if (idx < 0) break;
         for (int j = 0; j < ntile; ++j, ++J) {
-          const int st = J % kStages;
+          const int st = J % kVStages;
           const int t = it.t0 + j * kTcKeys;
           const int valid = max(0, min(kTcKeys, it.t1 - t));
-          if (!mbar_wait(&S.vempty[st], ((J / kStages) & 1u) ^ 1u, ctx)) { ok = false; break; }
+          if (!mbar_wait(&S.vempty[st], ((J / kVStages) & 1u) ^ 1u, ctx)) { ok = false; break; }
           if constexpr (paged) {
             if (!mbar_wait(&S.pidfull[J % kPidSlots], (J / kPidSlots) & 1u, ctx)) { ok = false; break; }
           }
@@ -795,16 +801,16 @@ __global__ void __launch_bounds__(kF8 ? kF8Threads : kTcThreads, 1)
       }
       if constexpr (kF8) {
         // stop marker for the V expanding warps (a stage without a tile)
-        const int st = J % kStages;
-        if (ok && mbar_wait(&S.vempty[st], ((J / kStages) & 1u) ^ 1u, ctx)) {
+        const int st = J % kVStages;
+        if (ok && mbar_wait(&S.vempty[st], ((J / kVStages) & 1u) ^ 1u, ctx)) {
           S.vmeta[st] = -1;
           mbar_arrive(&S.vraw[st]);
         }
       }
       if (S.abort_flag) {
-        for (uint32_t back = 1; back <= kStages && back <= J; ++back) {
+        for (uint32_t back = 1; back <= kVStages && back <= J; ++back) {
           const uint32_t jj = J - back;
-          mbar_drain(kF8 ? &S.vraw[jj % kStages] : &S.vfull[jj % kStages], (jj / kStages) & 1u);
+          mbar_drain(kF8 ? &S.vraw[jj % kVStages] : &S.vfull[jj % kVStages], (jj / kVStages) & 1u);
         }
       }
     }
@@ -885,10 +891,10 @@ __global__ void __launch_bounds__(kF8 ? kF8Threads : kTcThreads, 1)
         if (idx < 0) break;
         const int ob = K & 1;
         for (int j = 0; j < ntile; ++j, ++J) {
-          const int st = J % kStages;
+          const int st = J % kVStages;
           const int pb = J & 1;
           const int valid = max(0, min(kTcKeys, it.t1 - (it.t0 + j * kTcKeys)));
-          if (!mbar_wait(&S.vfull[st], (J / kStages) & 1u, ctx)) { ok = false; break; }
+          if (!mbar_wait(&S.vfull[st], (J / kVStages) & 1u, ctx)) { ok = false; break; }
           if (!mbar_wait(&S.pfull[pb], (J >> 1) & 1u, ctx)) { ok = false; break; }
           if (j == 0 && !mbar_wait(&S.oempty[ob], ((K >> 1) & 1u) ^ 1u, ctx)) { ok = false; break; }
           tc_fence_after();
@@ -960,7 +966,7 @@ __global__ void __launch_bounds__(kF8 ? kF8Threads : kTcThreads, 1)
       for (int g = 0; g < GPAD; ++g) { m[g] = -INFINITY; lp[g] = 0.f; }
       bool abort_item = false;
       for (int j = 0; j < ntile; ++j, ++J) {
-        const int st = J % kStages;
+        const int st = J % kVStages;
         const int sb = J & 1;
         ok = ok && mbar_wait(&S.sfull[sb], (J >> 1) & 1u, ctx);
         tc_fence_after();
@@ -1055,7 +1061,7 @@ __global__ void __launch_bounds__(kF8 ? kF8Threads : kTcThreads, 1)
         if (!kF8 && (valid & 15) != 0) {
           // zero V rows [valid, next multiple of 16): they may lie past the sequence end (the
           // expanding warps of an E4M3 cache write those rows as zeros themselves)
-          ok = ok && mbar_wait(&S.vfull[st], (J / kStages) & 1u, ctx);
+          ok = ok && mbar_wait(&S.vfull[st], (J / kVStages) & 1u, ctx);
           const int r0 = valid, r1 = (valid + 15) & ~15;
           const int nchunks = (r1 - r0) * 2 * 8;
           for (int c = tid; ok && c < nchunks; c += kSoftmaxThreads) {
@@ -1181,8 +1187,8 @@ __global__ void __launch_bounds__(kF8 ? kF8Threads : kTcThreads, 1)
       } else {
         const int ct = tid - (kConvWarp0 + 4) * 32;
         for (uint32_t J = 0;; ++J) {
-          const int st = J % kStages;
-          if (!mbar_wait(&S.vraw[st], (J / kStages) & 1u, ctx)) break;
+          const int st = J % kVStages;
+          if (!mbar_wait(&S.vraw[st], (J / kVStages) & 1u, ctx)) break;
           const int valid = S.vmeta[st];
           if (valid < 0) break;
           expand_v_tile(S.v[st], ct, valid);
