@@ -64,11 +64,18 @@ __device__ void block_exclusive_scan(const int32_t* in, int32_t* out, int n, int
 // the CTA call it; `sums` holds kPlanWaveChoices zeroed 64-bit counters of shared memory.
 __device__ int32_t plan_pick_chunk_block(const int32_t* len, int B, int64_t total, int32_t hkv,
                                          int32_t nctas, unsigned long long* sums) {
+  // the candidate chunks and the pick are the same for every thread: computed once (64-bit
+  // divisions) and shared
+  __shared__ int32_t s_chunks[kPlanWaveChoices];
+  __shared__ int32_t s_pick;
+  if (threadIdx.x < kPlanWaveChoices)
+    s_chunks[threadIdx.x] = plan_chunk_for_waves(total, hkv, nctas, plan_waves(threadIdx.x));
+  __syncthreads();
   int32_t chunks[kPlanWaveChoices];
   long long local[kPlanWaveChoices];
 #pragma unroll
   for (int i = 0; i < kPlanWaveChoices; ++i) {
-    chunks[i] = plan_chunk_for_waves(total, hkv, nctas, plan_waves(i));
+    chunks[i] = s_chunks[i];
     local[i] = 0;
   }
   for (int b = threadIdx.x; b < B; b += plan_threads()) {
@@ -82,10 +89,14 @@ __device__ int32_t plan_pick_chunk_block(const int32_t* len, int B, int64_t tota
     if (lane_id() == 0 && s != 0) atomicAdd(&sums[i], static_cast<unsigned long long>(s));
   }
   __syncthreads();
-  int64_t totals[kPlanWaveChoices];
+  if (threadIdx.x == 0) {
+    int64_t totals[kPlanWaveChoices];
 #pragma unroll
-  for (int i = 0; i < kPlanWaveChoices; ++i) totals[i] = static_cast<int64_t>(sums[i]);
-  return plan_pick_chunk(chunks, totals, hkv, nctas);
+    for (int i = 0; i < kPlanWaveChoices; ++i) totals[i] = static_cast<int64_t>(sums[i]);
+    s_pick = plan_pick_chunk(chunks, totals, hkv, nctas);
+  }
+  __syncthreads();
+  return s_pick;
 }
 
 // Decode plan over sequences whose lengths are len[0..B): items in longest-first order.
@@ -240,7 +251,7 @@ __global__ void __launch_bounds__(kMaxPlanThreads, 1) plan_chunk_kernel(PlanPara
   int32_t* s_roff = s_tmp + B;         // B + 1: first packed row of each request
   int32_t* s_dioff = s_roff + B + 1;   // B + 1: decode item offsets (rank order)
   int32_t* s_tioff = s_dioff + B + 1;  // B + 1: tile item offsets (request order)
-  int32_t* s_nmax = s_tioff + B + 1;   // key splits of a request's last query tile (0: no tiles)
+  int32_t* s_nmax = s_tioff + B + 1;   // key splits of a multi-tile request's last query tile
   int32_t* s_soff = s_nmax + B;        // B + 1: first (request, split) pair of each request
   __shared__ int s_scan[33];
   __shared__ unsigned long long s_total;
@@ -296,7 +307,9 @@ __global__ void __launch_bounds__(kMaxPlanThreads, 1) plan_chunk_kernel(PlanPara
       }
       const int32_t nheads = chunk_packed(c, p.hq / p.hkv) ? p.hkv : p.hq;
       s_tcnt[b] = cnt * nheads;
-      s_nmax[b] = c > 1 ? chunk_tile_splits(chunk_tile_keys(s_p[b], c, (c - 1) / kQTile, p.cap)) : 0;
+      // (request, split) pairs of the requests of more than one query tile; single-tile requests
+      // have their items written one per thread
+      s_nmax[b] = c > kQTile ? chunk_tile_splits(chunk_tile_keys(s_p[b], c, (c - 1) / kQTile, p.cap)) : 0;
       if (c > 1) atomicAdd(&s_key_tiles, static_cast<unsigned long long>(ktiles * nheads));
     }
   }
@@ -361,9 +374,32 @@ __global__ void __launch_bounds__(kMaxPlanThreads, 1) plan_chunk_kernel(PlanPara
       dst[1] = make_int4(t0, t1, n, rbase * p.hkv + h * n + s);
     }
   }
-  // tile items: one warp per (request, split) pair, lanes over query heads (KV heads for
-  // head-packed tiles). Per head the items run split by split and, within a split, tile by tile
-  // over the query tiles that see that split's keys.
+  // tile items of single-tile requests (2 <= c <= 128 rows: verification steps, short chunks):
+  // one thread per item. Item e of the request is head e / n, split e mod n (n splits).
+  for (int i = tid; i < (overflow ? 0 : s_tioff[B]); i += nthr) {
+    int lo = 0, hi = B;  // the request of item i: s_tioff[lo] <= i < s_tioff[lo + 1]
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (s_tioff[mid] <= i) lo = mid; else hi = mid;
+    }
+    const int b = lo;
+    const int32_t c = s_c[b];
+    if (c > kQTile) continue;  // written below, per (request, split) pair
+    const int32_t pp = s_p[b];
+    const int32_t kt = chunk_tile_keys(pp, c, 0, p.cap);
+    const int32_t nt = chunk_tile_splits(kt);
+    const int32_t e = i - s_tioff[b];
+    const int32_t h = e / nt, s = e - h * nt;
+    const int32_t k0 = min(s * kChunkKvSplit, kt), k1 = min((s + 1) * kChunkKvSplit, kt);
+    int4* dst = reinterpret_cast<int4*>(p.tiles + i);
+    dst[0] = make_int4(b, h, s, nt);
+    dst[1] = make_int4(k0, k1, s_roff[b], 0);
+    dst[2] = make_int4(c, pp, s_rb[b] * p.hkv, chunk_packed(c, p.hq / p.hkv) ? 1 : 0);
+    dst[3] = make_int4(0, 0, 0, 0);
+  }
+  // tile items of longer requests: one warp per (request, split) pair, lanes over query heads
+  // (KV heads for head-packed tiles). Per head the items run split by split and, within a
+  // split, tile by tile over the query tiles that see that split's keys.
   const int32_t n_pairs = s_soff[B];
   for (int k = warp; k < n_pairs && !overflow; k += nthr / 32) {
     int lo = 0, hi = B;  // the request of pair k: s_soff[lo] <= k < s_soff[lo + 1]
