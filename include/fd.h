@@ -198,12 +198,13 @@ fd_status fd_decode_attention_paged_fp8(const fd_tensor* q, const fd_tensor* k_p
  * [floor(s*len_b/n_b), floor((s+1)*len_b/n_b)); items are ordered longest split first
  * (sequences by their longest split, descending, ties by index), then KV head, then split.
  * num_splits > 0 instead fixes n_b = num_splits with ceil(len_b/num_splits)-key splits.
- * key_align = A > 1 puts every split boundary on a multiple of A keys (the plan of a paged
- * cache, A = 128, so that no key tile crosses a page): planner splits cut the ceil(len_b/A)
- * units equally, [min(len_b, A*floor(s*U/n_b)), min(len_b, A*floor((s+1)*U/n_b))), and a fixed
- * count rounds its split size up to a multiple of A; split counts and order do not change.
- * key_align = 1 is the plan of a contiguous cache. This is the same plan fd_decode_attention
- * (key_align 1) and fd_decode_attention_paged (key_align 128) build on the device.
+ * key_align = A > 1 puts every split boundary on a multiple of A keys: planner splits cut the
+ * ceil(len_b/A) units equally, [min(len_b, A*floor(s*U/n_b)), min(len_b, A*floor((s+1)*U/n_b))),
+ * and a fixed count rounds its split size up to a multiple of A; split counts and order do not
+ * change. The decode calls build this plan on the device with A = 128 for a paged cache (no key
+ * tile crosses a page) and for a contiguous bf16 cache on the tensor-core kernel (groups of
+ * 2..16 query heads per KV head: a split then ends on a key-tile boundary), and with A = 1 for a
+ * contiguous E4M3 cache and on the CUDA-core kernel (MHA, fp32).
  *
  *  cache_lens_host    [batch] int32 (host); clamped into [0, cache_capacity].
  *  num_ctas           persistent CTAs to plan for (>= 1); fd_decode_num_ctas() gives the count a

@@ -588,7 +588,11 @@ fd_status decode_call(const fd_tensor* q, const fd_tensor* k_cache, const fd_ten
     dp.num_pages = static_cast<int32_t>(std::min<int64_t>(k_cache->shape[0], INT32_MAX));
     dp.align = kPagedKeyAlign;
   } else {
-    dp.align = 1;
+    // the tensor-core kernel reads whole 128-key tiles: with a bf16 cache, splits that end on a
+    // tile boundary (no partly used tile in the middle of a sequence) run ~2% faster at the
+    // 70B-like shape; an E4M3 cache ran 20% slower that way (measured A/B), so it keeps
+    // unaligned splits
+    dp.align = (sh.use_tc && !sh.kv_fp8) ? kTcKeyAlign : 1;
   }
   // an E4M3 cache: k_scale multiplies every score, v_scale every output (both linear)
   dp.scale_log2 = static_cast<float>(1.0 / std::sqrt(static_cast<double>(sh.d)) * 1.4426950408889634 *
@@ -817,6 +821,7 @@ fd_status fd_chunk_prefill_attention(const fd_tensor* q_chunk, const fd_tensor* 
   pp.arrivals = arrivals;
   pp.total_rows = T;
   pp.decode_merged_in_kernel = dec_tc ? 0 : 1;
+  pp.align = dec_tc ? kTcKeyAlign : 1;  // decode rows' split boundaries
   pp.tile_sms = tile_ctas;
   pp.kv_key_bytes = 2ll * hkv * d * 2;
 

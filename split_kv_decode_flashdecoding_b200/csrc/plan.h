@@ -31,6 +31,7 @@ constexpr int32_t kChunkKvSplit = 2048;   // keys per split of a chunked-prefill
 constexpr int32_t kMaxPlanBatch = 4096;   // largest batch the one-CTA device planner accepts
 constexpr int32_t kFusedPlanMaxBatch = 256;  // largest batch the tensor-core split kernel plans itself
 constexpr int32_t kPagedKeyAlign = 128;      // split boundaries of a paged cache: one key tile
+constexpr int32_t kTcKeyAlign = 128;         // split boundaries on the tensor-core decode path
 
 // One split of one (sequence, KV head): keys [t0, t1) of cache row b, output row `row`.
 struct DecodeItem {

@@ -368,7 +368,7 @@ __global__ void __launch_bounds__(kMaxPlanThreads, 1) plan_chunk_kernel(PlanPara
     for (int32_t e = lane; e < n * p.hkv; e += 32) {
       const int32_t h = e / n, s = e - h * n;
       int32_t t0, t1;
-      plan_split_range(L, n, s, 0, 1, &t0, &t1);
+      plan_split_range(L, n, s, 0, p.align, &t0, &t1);
       int4* dst = reinterpret_cast<int4*>(p.items + first + e);
       dst[0] = make_int4(row, b, h, s);
       dst[1] = make_int4(t0, t1, n, rbase * p.hkv + h * n + s);
