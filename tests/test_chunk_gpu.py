@@ -136,6 +136,8 @@ VERIFY = [
     ([6000, 17], [2, 2], 32, 2, 6144),                       # G = 16, k = 2 (32 rows), many splits
     ([1500, 3000], [16, 9], 4, 2, 3072),                     # G = 2, k = 16 and 9
     ([100, 2500, 40], [8, 5, 1], 32, 8, 2560),               # G = 4 with a decode row
+    ([800, 50], [5, 4], 12, 2, 1024),                        # G = 6: quarter items of 30 and 24 rows
+    ([1300, 2], [4, 3], 7, 1, 1536),                         # G = 7: 28 and 21 rows
 ]
 
 
