@@ -119,15 +119,12 @@ _DTYPES = {torch.float32: FD_F32, torch.bfloat16: FD_BF16, torch.float8_e4m3fn: 
 
 
 def _tensor(t: torch.Tensor) -> FdTensor:
-    if t.dim() > 4:
+    n = t.dim()
+    if n > 4:
         raise ValueError("at most 4 dimensions")
-    ft = FdTensor()
-    ft.data = t.data_ptr() if t.numel() > 0 else None
-    ft.dtype = _DTYPES.get(t.dtype, -1)
-    ft.ndim = t.dim()
-    for i in range(t.dim()):
-        ft.shape[i] = t.shape[i]
-        ft.stride[i] = t.stride(i)
+    ft = FdTensor(t.data_ptr() if t.numel() > 0 else None, _DTYPES.get(t.dtype, -1), n)
+    ft.shape[:n] = t.shape
+    ft.stride[:n] = t.stride()
     return ft
 
 
