@@ -377,15 +377,15 @@ __global__ void __launch_bounds__(kCkThreads, 1)
           tc_fence_after();
           const int valid = S.meta[st];
           if (valid > 0) {
-            const uint32_t k0 = smem_u32(S.k[st][0]);
-            const uint32_t k1 = smem_u32(S.k[st][kHalves - 1]);
+            // descriptors of the two 64-column halves; a 16-column step is 32 bytes, i.e. 2 in the
+            // start-address field
+            const uint64_t qd[2] = {smem_desc(q0, 16, 1024, kLayoutSW128), smem_desc(q1, 16, 1024, kLayoutSW128)};
+            const uint64_t kd[2] = {smem_desc(smem_u32(S.k[st][0]), 16, 1024, kLayoutSW128),
+                                    smem_desc(smem_u32(S.k[st][kHalves - 1]), 16, 1024, kLayoutSW128)};
 #pragma unroll
-            for (int kk = 0; kk < kD / 16; ++kk) {
-              const uint32_t qa = (kk < 4 ? q0 : q1) + (kk & 3) * 32;
-              const uint32_t ka = (kk < 4 ? k0 : k1) + (kk & 3) * 32;
-              umma_bf16_ss(tmem + kColS0 + sb * 128, smem_desc(qa, 16, 1024, kLayoutSW128),
-                           smem_desc(ka, 16, 1024, kLayoutSW128), idesc_s, kk > 0 ? 1u : 0u);
-            }
+            for (int kk = 0; kk < kD / 16; ++kk)
+              umma_bf16_ss(tmem + kColS0 + sb * 128, qd[kk >> 2] + static_cast<uint64_t>((kk & 3) * 2),
+                           kd[kk >> 2] + static_cast<uint64_t>((kk & 3) * 2), idesc_s, kk > 0 ? 1u : 0u);
           }
           umma_commit(&S.sfull[sb]);
           umma_commit(&S.kempty[st]);
@@ -422,14 +422,27 @@ __global__ void __launch_bounds__(kCkThreads, 1)
           if (j == 0 && !mbar_wait(&S.oempty, (K & 1u) ^ 1u, ctx)) { ok = false; break; }
           tc_fence_after();
           const int nk = (valid + 15) / 16;
-          const uint32_t vaddr = smem_u32(S.v[vs][0]);
-          const uint32_t pcol = kColS0 + (J & 1) * 128;  // P of this tile, over its S buffer
-          for (int part = 0; part < 2; ++part) {
-            const uint32_t ocol = part ? kColOLo : kColOHi;
-            for (int kk = 0; kk < nk; ++kk) {
-              const uint64_t bd = smem_desc(vaddr + kk * 2048, kCkHalf, 1024, kLayoutSW128);
-              const uint32_t acol = pcol + 32 * (kk >> 1) + 16 * part + 8 * (kk & 1);
-              umma_bf16_ts(tmem + ocol, tmem + acol, bd, idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
+          // V's descriptor for the first 16 keys; key step kk starts 2048 bytes further, i.e.
+          // kk * 128 in the descriptor's start-address field (shared addresses stay below
+          // 2^18 bytes, so the 14-bit field never carries)
+          const uint64_t bd0 = smem_desc(smem_u32(S.v[vs][0]), kCkHalf, 1024, kLayoutSW128);
+          const uint32_t pa = tmem + kColS0 + (J & 1) * 128;  // P of this tile, over its S buffer
+          const uint32_t acc = j > 0 ? 1u : 0u;
+          if (nk == kCkKeys / 16) {
+            // a full tile: every address is a constant offset, so the thread issues little but
+            // the products themselves
+#pragma unroll
+            for (int part = 0; part < 2; ++part)
+#pragma unroll
+              for (int kk = 0; kk < kCkKeys / 16; ++kk)
+                umma_bf16_ts(tmem + (part ? kColOLo : kColOHi), pa + 32 * (kk >> 1) + 16 * part + 8 * (kk & 1),
+                             bd0 + static_cast<uint64_t>(kk * 128), idesc_o, kk > 0 ? 1u : acc);
+          } else {
+            for (int part = 0; part < 2; ++part) {
+              const uint32_t ocol = part ? kColOLo : kColOHi;
+              for (int kk = 0; kk < nk; ++kk)
+                umma_bf16_ts(tmem + ocol, pa + 32 * (kk >> 1) + 16 * part + 8 * (kk & 1),
+                             bd0 + static_cast<uint64_t>(kk * 128), idesc_o, kk > 0 ? 1u : acc);
             }
           }
           umma_commit(&S.pfree);
