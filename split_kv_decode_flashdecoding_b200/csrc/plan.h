@@ -206,9 +206,11 @@ FD_HD int32_t chunk_tile_splits(int32_t keys) {
 // min(kHbmGBs, (nsm - N) kDecodeSmGBs); what is left then streams at kHbmGBs. N minimises the
 // total: the time of phase 1 plus that of the rest. `key_tiles` counts the 128-key tiles of all
 // tile items, `dec_bytes` the K/V bytes of the decode rows. No tiles: 0; no decode rows: nsm.
-constexpr float kTileKeyTileUs = 2.3f;  // 250 µs for workload 5's 16192 key tiles on 148 CTAs
-constexpr float kDecodeSmGBs = 45.f;    // tensor-core decode rows beside 80 tile CTAs: ~1.4 GB in 465 µs on 68 SMs
-constexpr float kHbmGBs = 6000.f;       // decode rows alone on the whole device
+// The three constants were fitted to one B200 sweep of N = 50..95 on the mixed workload (16192 key
+// tiles, 2.19 GB of decode rows), which they reproduce within 2 % for N >= 70.
+constexpr float kTileKeyTileUs = 2.3f;  // µs per key tile of a 128-row query tile, per CTA
+constexpr float kDecodeSmGBs = 60.f;    // tensor-core decode rows per multiprocessor, beside the tiles
+constexpr float kHbmGBs = 6500.f;       // decode rows on the whole device
 // Estimated time (µs) of the call when the tile kernel keeps n of the nsm multiprocessors. The
 // planner keeps the n of least cost (the smallest such n on ties); with no tile items it keeps
 // 0, with no decode rows all nsm.
