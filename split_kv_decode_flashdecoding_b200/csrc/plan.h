@@ -110,14 +110,18 @@ FD_HD int32_t plan_chunk_for_waves(int64_t total, int32_t hkv, int32_t nctas, in
 
 // The chunk of least estimated makespan among the candidates chunks[i] = plan_chunk_for_waves(...,
 // plan_waves(i)), given split_sums[i] = sum_b max(1, ceil(len_b / chunks[i])).
+// Estimated makespan of one candidate: ceil(items / nctas) * (ceil(chunk / 128) + kItemFixedTiles).
+FD_HD int64_t plan_chunk_cost(int64_t split_sum, int32_t chunk, int32_t hkv, int32_t nctas) {
+  const int64_t n = nctas > 0 ? nctas : 1;
+  return cdiv64(split_sum * hkv, n) * (cdiv64(chunk, 128) + kItemFixedTiles);
+}
+
 FD_HD int32_t plan_pick_chunk(const int32_t* chunks, const int64_t* split_sums, int32_t hkv,
                               int32_t nctas) {
-  const int64_t n = nctas > 0 ? nctas : 1;
   int32_t best = chunks[0];
   int64_t best_cost = 0;
   for (int i = 0; i < kPlanWaveChoices; ++i) {
-    const int64_t waves = cdiv64(split_sums[i] * hkv, n);
-    const int64_t cost = waves * (cdiv64(chunks[i], 128) + kItemFixedTiles);
+    const int64_t cost = plan_chunk_cost(split_sums[i], chunks[i], hkv, nctas);
     if (i == 0 || cost < best_cost) {
       best = chunks[i];
       best_cost = cost;

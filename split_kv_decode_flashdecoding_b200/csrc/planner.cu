@@ -89,11 +89,18 @@ __device__ int32_t plan_pick_chunk_block(const int32_t* len, int B, int64_t tota
     if (lane_id() == 0 && s != 0) atomicAdd(&sums[i], static_cast<unsigned long long>(s));
   }
   __syncthreads();
+  // the candidates' costs in parallel, then plan_pick_chunk's choice (the first least cost)
+  __shared__ long long s_cost[kPlanWaveChoices];
+  if (threadIdx.x < kPlanWaveChoices)
+    s_cost[threadIdx.x] = plan_chunk_cost(static_cast<int64_t>(sums[threadIdx.x]),
+                                          s_chunks[threadIdx.x], hkv, nctas);
+  __syncthreads();
   if (threadIdx.x == 0) {
-    int64_t totals[kPlanWaveChoices];
+    int best = 0;
 #pragma unroll
-    for (int i = 0; i < kPlanWaveChoices; ++i) totals[i] = static_cast<int64_t>(sums[i]);
-    s_pick = plan_pick_chunk(chunks, totals, hkv, nctas);
+    for (int i = 1; i < kPlanWaveChoices; ++i)
+      if (s_cost[i] < s_cost[best]) best = i;
+    s_pick = s_chunks[best];
   }
   __syncthreads();
   return s_pick;
@@ -359,19 +366,26 @@ __global__ void __launch_bounds__(kMaxPlanThreads, 1) plan_chunk_kernel(PlanPara
   const int32_t n_tile_items = s_tioff[B];
   const bool overflow =
       inconsistent || n_dec_items > p.max_dec_items || n_tile_items > p.max_tile_items;
-  // decode items: one warp per decode request, lanes over its (KV head, split) items
+  // decode items: one warp per decode request. With n <= 32 splits, lane L takes split L mod n of
+  // heads L / n, L / n + 32 / n, ... (its key range computed once); with more, lanes take splits
+  // and loop over the heads. Item (h, s) sits at first + h n + s.
   for (int r = warp; r < nd && !overflow; r += nthr / 32) {
     const int b = s_order[r];
     const int32_t row = s_roff[b];
     const int32_t n = s_n[b], L = s_dlen[b], first = s_dioff[r];
     const int32_t rbase = s_rb[b];
-    for (int32_t e = lane; e < n * p.hkv; e += 32) {
-      const int32_t h = e / n, s = e - h * n;
+    const int32_t per = n <= 32 ? 32 / n : 1;  // heads a pass covers
+    const int32_t s0 = n <= 32 ? lane % n : lane;
+    const int32_t h0 = n <= 32 ? lane / n : 0;
+    if (h0 >= per) continue;  // lanes past the last whole group of n
+    for (int32_t s = s0; s < n; s += 32) {
       int32_t t0, t1;
       plan_split_range(L, n, s, 0, p.align, &t0, &t1);
-      int4* dst = reinterpret_cast<int4*>(p.items + first + e);
-      dst[0] = make_int4(row, b, h, s);
-      dst[1] = make_int4(t0, t1, n, rbase * p.hkv + h * n + s);
+      for (int32_t h = h0; h < p.hkv; h += per) {
+        int4* dst = reinterpret_cast<int4*>(p.items + first + h * n + s);
+        dst[0] = make_int4(row, b, h, s);
+        dst[1] = make_int4(t0, t1, n, rbase * p.hkv + h * n + s);
+      }
     }
   }
   // tile items of single-tile requests (2 <= c <= 128 rows: verification steps, short chunks):
