@@ -145,12 +145,12 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// bf16 tensor map, 128-byte swizzle, 64-element inner box; dims/strides innermost first.
-fd_status make_tmap(CUtensorMap* map, const void* base, int rank, const uint64_t* dims,
-                    const uint64_t* strides_bytes, const uint32_t* box, const char* what,
-                    CUtensorMapDataType dtype) {
+// Tensor map with 128-byte swizzle (rank <= 5); dims/strides innermost first. Returns the
+// driver's result (CUDA_ERROR_NOT_SUPPORTED when the encoder is missing).
+CUresult encode_tmap(CUtensorMap* map, const void* base, int rank, const uint64_t* dims,
+                     const uint64_t* strides_bytes, const uint32_t* box, CUtensorMapDataType dtype) {
   EncodeTiledFn fn = encode_fn();
-  if (!fn) return fail(FD_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  if (!fn) return CUDA_ERROR_NOT_SUPPORTED;
   cuuint64_t d[5], s[4];
   cuuint32_t b[5], es[5];
   for (int i = 0; i < rank; ++i) {
@@ -159,9 +159,17 @@ fd_status make_tmap(CUtensorMap* map, const void* base, int rank, const uint64_t
     es[i] = 1;
     if (i > 0) s[i - 1] = strides_bytes[i - 1];
   }
-  CUresult r = fn(map, dtype, rank, const_cast<void*>(base), d, s, b,
-                  es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return fn(map, dtype, rank, const_cast<void*>(base), d, s, b,
+            es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+}
+
+// The same, failing the call with a message.
+fd_status make_tmap(CUtensorMap* map, const void* base, int rank, const uint64_t* dims,
+                    const uint64_t* strides_bytes, const uint32_t* box, const char* what,
+                    CUtensorMapDataType dtype) {
+  if (!encode_fn()) return fail(FD_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  const CUresult r = encode_tmap(map, base, rank, dims, strides_bytes, box, dtype);
   if (r != CUDA_SUCCESS) return fail(FD_ERR_CUDA, "cuTensorMapEncodeTiled(%s) failed: %d", what, (int)r);
   return FD_OK;
 }
@@ -623,8 +631,25 @@ fd_status decode_call(const fd_tensor* q, const fd_tensor* k_cache, const fd_ten
                             static_cast<uint64_t>(k_cache->stride[0]) * es};
     const uint32_t kb[4] = {sh.kv_fp8 ? 128u : 64u, static_cast<uint32_t>(dp.kv_box_rows), 1, 1};
     const CUtensorMapDataType kt = sh.kv_fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
-    if ((s = make_tmap(&tk, k_cache->data, 4, kd, ks, kb, "k_cache", kt)) != FD_OK) return s;
-    if ((s = make_tmap(&tv, v_cache->data, 4, kd, ks, kb, "v_cache", kt)) != FD_OK) return s;
+    // bf16 pages of < 128 keys with their KV heads one after another: 5-D maps (64 columns,
+    // 8 rows 256 bytes apart, 2 halves 128 bytes apart, Hkv * page_size / 8 row groups 2048
+    // bytes apart, pages) whose box is a whole page, laid out as the tensor-core kernel's
+    // interleaved tile (one copy per page instead of two). Where the driver rejects a map of
+    // such strides, the 4-D maps below serve.
+    if (pg && !sh.kv_fp8 && pg->page_size < 128 &&
+        k_cache->stride[1] == static_cast<int64_t>(pg->page_size) * sh.d) {
+      const uint64_t groups = static_cast<uint64_t>(pg->page_size / 8) * static_cast<uint64_t>(sh.hkv);
+      const uint64_t id[5] = {64, 8, 2, groups, outer};
+      const uint64_t is[4] = {256, 128, 2048, static_cast<uint64_t>(k_cache->stride[0]) * 2};
+      const uint32_t ib[5] = {64, 8, 2, static_cast<uint32_t>(pg->page_size / 8), 1};
+      if (encode_tmap(&tk, k_cache->data, 5, id, is, ib, kt) == CUDA_SUCCESS &&
+          encode_tmap(&tv, v_cache->data, 5, id, is, ib, kt) == CUDA_SUCCESS)
+        dp.pg_interleave = 1;
+    }
+    if (!dp.pg_interleave) {
+      if ((s = make_tmap(&tk, k_cache->data, 4, kd, ks, kb, "k_cache", kt)) != FD_OK) return s;
+      if ((s = make_tmap(&tv, v_cache->data, 4, kd, ks, kb, "v_cache", kt)) != FD_OK) return s;
+    }
   }
 
   PlanParams pp{};

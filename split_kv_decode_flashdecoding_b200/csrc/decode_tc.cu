@@ -155,12 +155,32 @@ __device__ __forceinline__ int32_t tile_page_id(const DecodeParams& p, int b, in
                                  : -1;
 }
 
-// Whole warp: issue the K or V loads of one 128-key tile over pages of < 128 keys, one box per
-// lane: lane i < n copies page i's first 64-column half (an E4M3 cache: its whole 128-byte
-// rows) and lane n + i its second half, page ids from `ids` (a slot of the ring). A page that
-// holds some of the tile's `valid` keys but whose index lies outside the pool raises
-// FD_FLAG_BAD_PAGE; its copy still runs and reads zeros (a TMA coordinate outside the tensor).
-// The caller has announced small_pages_bytes() on `bar`.
+// tma_load_4d_stream over a 5-D map (one page of a paged cache in the interleaved layout of
+// load_small_pages).
+__device__ __forceinline__ void tma_load_5d_stream(void* dst, const CUtensorMap* map,
+                                                   uint64_t* bar, int32_t c0, int32_t c1,
+                                                   int32_t c2, int32_t c3, int32_t c4,
+                                                   uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.5d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      ".L2::cache_hint [%0], [%1, {%3, %4, %5, %6, %7}], [%2], %8;" ::"r"(smem_u32(dst)),
+      "l"(map), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(c4), "l"(policy)
+      : "memory");
+}
+
+// Whole warp: issue the K or V loads of one 128-key tile over pages of < 128 keys, page ids
+// from `ids` (a slot of the ring), one box per lane:
+// - an E4M3 cache: lane i < n copies page i's whole 128-byte rows;
+// - bf16 with p.pg_interleave: lane i < n copies page i whole through the 5-D map, into the
+//   interleaved tile layout (8-row group r of the tile at r * 2048 bytes, its first 64-column
+//   half there and its second 1024 bytes further: both halves are 1024-byte swizzle atoms, so
+//   the products read them with a group stride of 2048);
+// - bf16 otherwise: lane i < n copies page i's first 64-column half into dst0 (the two-slab
+//   layout, each half's rows 128 bytes apart) and lane n + i its second half into dst1.
+// A box costs the copy engine about the same whatever its size, so one box per page halves the
+// issue work of 16-key pages. A page that holds some of the tile's `valid` keys but whose index
+// lies outside the pool raises FD_FLAG_BAD_PAGE; its copy still runs and reads zeros (a TMA
+// coordinate outside the tensor). The caller has announced small_pages_bytes() on `bar`.
 template <bool kF8>
 __device__ __forceinline__ void load_small_pages(__nv_bfloat16* dst0, __nv_bfloat16* dst1,
                                                  const CUtensorMap* map, uint64_t* bar,
@@ -168,10 +188,11 @@ __device__ __forceinline__ void load_small_pages(__nv_bfloat16* dst0, __nv_bfloa
                                                  const DecodeParams& p, int h, int valid,
                                                  uint64_t pol, int lane) {
   const int rows = p.page_size;
-  const int boxes = kF8 ? sp.n : 2 * sp.n;
+  const bool whole = kF8 || p.pg_interleave != 0;  // one box per page
+  const int boxes = whole ? sp.n : 2 * sp.n;
   bool bad = false;
   if (lane < boxes) {
-    const int half = kF8 ? 0 : (lane >= sp.n ? 1 : 0);
+    const int half = whole ? 0 : (lane >= sp.n ? 1 : 0);
     const int i = lane - half * sp.n;
     const int32_t id = sp.first + i < p.pages_per_seq ? ids[i] : -1;
     bad = i * rows < valid && (id < 0 || id >= p.num_pages);
@@ -179,7 +200,10 @@ __device__ __forceinline__ void load_small_pages(__nv_bfloat16* dst0, __nv_bfloa
       tma_load_4d_stream(reinterpret_cast<unsigned char*>(dst0) + i * rows * 128, map, bar, 0, 0,
                          h, id, pol);
     } else {
-      tma_load_4d_stream((half ? dst1 : dst0) + i * rows * 64, map, bar, half * 64, 0, h, id, pol);
+      if (whole)  // page i = 8-row groups i * rows / 8 ..: 256 bytes (128 elements) per row
+        tma_load_5d_stream(dst0 + i * rows * 128, map, bar, 0, 0, 0, h * (rows >> 3), id, pol);
+      else
+        tma_load_4d_stream((half ? dst1 : dst0) + i * rows * 64, map, bar, half * 64, 0, h, id, pol);
     }
   }
   if (__any_sync(0xffffffffu, bad) && lane == 0) atomicOr(&p.hdr->status, FD_FLAG_BAD_PAGE);
@@ -857,9 +881,13 @@ __global__ void __launch_bounds__(kF8 ? kF8Threads : kTcThreads, 1)
                 umma_f8_ss(tmem + sb * 16, smem_desc(ka + kk * 32, 16, 1024, kLayoutSW128),
                            smem_desc(qa + kk * 32, 16, 1024, kLayoutSW128), idesc_s, kk > 0 ? 1u : 0u);
             } else if constexpr (kMode == kSmallPages) {
-              // descriptors built once per tile, as above
-              const uint64_t kd[2] = {smem_desc(smem_u32(S.k[st][0]), 16, 1024, kLayoutSW128),
-                                      smem_desc(smem_u32(S.k[st][Smem::kKSlabs - 1]), 16, 1024, kLayoutSW128)};
+              // descriptors built once per tile, as above; the interleaved layout has the second
+              // half 1024 bytes after the first and 8-row groups 2048 bytes apart
+              const uint32_t kil = p.pg_interleave ? 1u : 0u;
+              const uint32_t kbase = smem_u32(S.k[st][0]);
+              const uint64_t kd[2] = {smem_desc(kbase, 16, 1024u << kil, kLayoutSW128),
+                                      smem_desc(kil ? kbase + 1024u : smem_u32(S.k[st][Smem::kKSlabs - 1]), 16,
+                                                1024u << kil, kLayoutSW128)};
               const uint64_t qd[2] = {smem_desc(qaddr0, 16, 1024, kLayoutSW128),
                                       smem_desc(qaddr1, 16, 1024, kLayoutSW128)};
 #pragma unroll
@@ -926,10 +954,14 @@ __global__ void __launch_bounds__(kF8 ? kF8Threads : kTcThreads, 1)
             // tile's products unrolled. Measured A/B at the 70B-like shape: E4M3 268 -> 258 us,
             // 16-key pages 411 -> 399 us; the contiguous bf16 kernel did not change and the
             // 128-key-page E4M3 kernel slowed (363 -> 389 us), so those keep the plain loop.
-            const uint64_t ad0 = smem_desc(vaddr, kHalfBytes, 1024, kLayoutSW128);
+            // V of 16-key pages in the interleaved layout: halves 1024 bytes apart (LBO), 8-key
+            // groups 2048 (SBO), so 16 keys a step are 4096 bytes (256 in the field)
+            const uint32_t vil = (kMode == kSmallPages && p.pg_interleave) ? 1u : 0u;
+            const uint64_t ad0 = smem_desc(vaddr, vil ? 1024u : kHalfBytes, 1024u << vil, kLayoutSW128);
             const uint64_t bd0 = smem_desc(paddr, 128, 2048, kLayoutNone);
             const uint32_t dcol = tmem + kColO + ob * kNO;
             const uint32_t acc = j > 0 ? 1u : 0u;
+            const uint32_t vstep = 128u << vil;
             if (kF8 && kMode == kContiguous && nk == kTcKeys / 16) {
 #pragma unroll
               for (int kk = 0; kk < kTcKeys / 16; ++kk)
@@ -937,7 +969,7 @@ __global__ void __launch_bounds__(kF8 ? kF8Threads : kTcThreads, 1)
                              idesc_o, kk > 0 ? 1u : acc);
             } else {
               for (int kk = 0; kk < nk; ++kk)
-                umma_bf16_ss(dcol, ad0 + static_cast<uint64_t>(kk * 128), bd0 + static_cast<uint64_t>(kk * 16),
+                umma_bf16_ss(dcol, ad0 + static_cast<uint64_t>(kk * vstep), bd0 + static_cast<uint64_t>(kk * 16),
                              idesc_o, kk > 0 ? 1u : acc);
             }
           } else {
@@ -1105,11 +1137,15 @@ __global__ void __launch_bounds__(kF8 ? kF8Threads : kTcThreads, 1)
           ok = ok && mbar_wait(&S.vfull[st], (J / kVStages) & 1u, ctx);
           const int r0 = valid, r1 = (valid + 15) & ~15;
           const int nchunks = (r1 - r0) * 2 * 8;
+          const bool vil = kMode == kSmallPages && p.pg_interleave;
           for (int c = tid; ok && c < nchunks; c += kSoftmaxThreads) {
             const int row = r0 + c / 16;
             const int half = (c / 8) & 1;
             const int ch = c & 7;
-            *reinterpret_cast<uint4*>(reinterpret_cast<unsigned char*>(S.v[st][half]) + row * 128 + ch * 16) =
+            // byte offset of the row's half from the stage start (interleaved: see load_small_pages)
+            const int off = vil ? (row >> 3) * 2048 + half * 1024 + (row & 7) * 128
+                                : half * static_cast<int>(kHalfBytes) + row * 128;
+            *reinterpret_cast<uint4*>(reinterpret_cast<unsigned char*>(S.v[st][0]) + off + ch * 16) =
                 make_uint4(0u, 0u, 0u, 0u);
           }
         }

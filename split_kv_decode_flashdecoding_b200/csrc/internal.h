@@ -67,6 +67,10 @@ struct DecodeParams {
   // it, and split boundaries are 128-key aligned, so a key tile never crosses a page.
   const int32_t* block_table;
   int32_t pages_per_seq, page_size, num_pages;
+  // bf16 pages of < 128 keys whose KV heads are consecutive (head stride = page_size rows):
+  // the K/V maps are 5-D and copy a whole page per box, each 8-row group's two 64-column halves
+  // side by side (see load_small_pages); 0: the 4-D maps, one box per page and half
+  int32_t pg_interleave = 0;
   // E4M3 cache (kv_fp8 != 0, tensor-core kernel): k and v hold one-byte codes; the key scale is
   // folded into scale_log2 and every output is multiplied by v_scale (1 for other caches)
   float v_scale = 1.f;

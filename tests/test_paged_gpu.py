@@ -161,11 +161,46 @@ def test_paged_rejects_bad_layouts():
         fd.fd_decode_attention_paged(q, kp, kp, table, lens)
 
 
-def test_paged_workload_3():
-    # the default workload's keys in 128-key pages at shuffled positions: every output element
+@pytest.mark.parametrize("layout", ["head_major", "kv_pool"])
+@pytest.mark.parametrize("psz", [8, 16, 64])
+def test_paged_pool_layouts(layout, psz):
+    # pools that are not [pages, Hkv, page_size, D] contiguous:
+    # - head_major: stored [Hkv, pages, page_size, D] (a page's KV heads are not consecutive, so
+    #   the tensor-core kernel copies each half of a page separately);
+    # - kv_pool: K and V of a page side by side in one [pages, 2, Hkv, page_size, D] pool (a page
+    #   stride twice the page's bytes; the heads are consecutive, so a page is one copy).
+    fd = _fd()
+    dev = torch.device("cuda", 0)
+    lens = [700, 1, 129, 0, 383]
+    inp = make_decode_inputs(5, 64, 8, 128, 768, lens, torch.bfloat16, seed=610 + psz, pad_fill=NAN)
+    pg = make_paged(inp.k_cache, inp.v_cache, lens, psz, seed=620 + psz)
+    if layout == "head_major":
+        kp = pg.k_pages.permute(1, 0, 2, 3).contiguous().to(dev).permute(1, 0, 2, 3)
+        vp = pg.v_pages.permute(1, 0, 2, 3).contiguous().to(dev).permute(1, 0, 2, 3)
+        assert kp.stride(1) != psz * 128
+    else:
+        pool = torch.stack([pg.k_pages, pg.v_pages], dim=1).to(dev)
+        kp, vp = pool[:, 0], pool[:, 1]
+        assert kp.stride(0) == 2 * kp.shape[1] * psz * 128 and kp.stride(1) == psz * 128
+    q = inp.q.to(dev)
+    out = torch.empty_like(q)
+    lse = torch.empty((5, 64), dtype=torch.float32, device=dev)
+    fd.fd_decode_attention_paged(q, kp, vp, pg.block_table.to(dev), inp.cache_lens.to(dev),
+                                 out=out, lse=lse)
+    torch.cuda.synchronize()
+    ro, rl = _oracle(inp)
+    check_out(out, ro, f"paged {layout} {psz} out")
+    check_lse(lse, rl, f"paged {layout} {psz} lse")
+    assert fd.fd_poll_status() == 0
+
+
+@pytest.mark.parametrize("psz", [128, 16])
+def test_paged_workload_3(psz):
+    # the default workload's keys in 128- or 16-key pages at shuffled positions: every output
+    # element
     inp = workload(3)
-    pg = make_paged(inp.k_cache, inp.v_cache, inp.cache_lens.tolist(), 128, seed=1303)
+    pg = make_paged(inp.k_cache, inp.v_cache, inp.cache_lens.tolist(), psz, seed=1303)
     out, lse = _run_paged(inp, pg)
     ro, rl = _oracle(inp)
-    check_out(out, ro, "paged w3 out")
-    check_lse(lse, rl, "paged w3 lse")
+    check_out(out, ro, f"paged w3 (pages of {psz}) out")
+    check_lse(lse, rl, f"paged w3 (pages of {psz}) lse")
