@@ -77,7 +77,7 @@ WAVES = 8              # largest target of items per persistent CTA
 WAVE_CHOICES = (8, 4, 2, 1)
 ITEM_FIXED_TILES = 2   # fixed cost of a work item, in 128-key tiles
 Q_TILE = 128           # query rows per chunked-prefill tile
-CHUNK_KV_SPLIT = 2048  # keys per split for a chunked-prefill query tile
+CHUNK_KV_SPLIT = 4096  # keys per split for a chunked-prefill query tile
 
 
 def _cdiv(a: int, b: int) -> int:

@@ -9,6 +9,7 @@ namespace fd {
 namespace {
 
 constexpr int kMaxPlanThreads = 1024;
+constexpr int kPlanChunkCtas = 16;  // CTAs of the chunked-prefill planner (see plan_chunk_kernel)
 
 __device__ __forceinline__ int plan_threads() { return static_cast<int>(blockDim.x); }
 
@@ -233,11 +234,72 @@ __global__ void __launch_bounds__(kMaxPlanThreads, 1) plan_decode_kernel(PlanPar
   if (threadIdx.x == 0 && s_flags) atomicOr(&p.hdr->status, s_flags);
 }
 
-// Chunked-prefill plan (one CTA): requests with chunk_len == 1 are decode rows over
-// prefix + 1 keys, planned like a decode call over those requests; longer chunks become query
-// tiles of kQTile rows whose keys are cut on a fixed kChunkKvSplit grid, items ordered
-// (request, query head, split, tile). One exclusive scan over all packed rows gives every row
-// its partial slots, so the same combine merges decode rows and tile rows.
+// Exclusive prefix sums of K arrays of n ints at once (out[k][n] = the total of in[k]), with
+// the three barriers of one scan. All threads of the CTA call it; `scratch` holds 33 * K ints.
+template <int K>
+__device__ void block_exclusive_scan_k(const int32_t* const* in, int32_t* const* out, int n,
+                                       int* scratch) {
+  const int tid = threadIdx.x;
+  const int nthr = plan_threads();
+  const int per = (n + nthr - 1) / nthr;
+  const int lo = tid * per;
+  const int warp = tid >> 5;
+  int local[K], incl[K];
+#pragma unroll
+  for (int k = 0; k < K; ++k) {
+    local[k] = 0;
+    for (int i = 0; i < per; ++i)
+      if (lo + i < n) local[k] += in[k][lo + i];
+    incl[k] = warp_incl_scan(local[k]);
+    if (lane_id() == 31) scratch[k * 33 + warp] = incl[k];
+  }
+  __syncthreads();
+  if (warp == 0) {
+#pragma unroll
+    for (int k = 0; k < K; ++k) {
+      const int w = (lane_id() < static_cast<uint32_t>(nthr / 32)) ? scratch[k * 33 + lane_id()] : 0;
+      const int wi = warp_incl_scan(w);
+      scratch[k * 33 + lane_id()] = wi - w;  // exclusive warp offsets
+      if (lane_id() == 31) scratch[k * 33 + 32] = wi;
+    }
+  }
+  __syncthreads();
+#pragma unroll
+  for (int k = 0; k < K; ++k) {
+    int run = scratch[k * 33 + warp] + incl[k] - local[k];
+    for (int i = 0; i < per; ++i) {
+      if (lo + i < n) {
+        out[k][lo + i] = run;
+        run += in[k][lo + i];
+      }
+    }
+    if (tid == 0) out[k][n] = scratch[k * 33 + 32];
+  }
+  __syncthreads();
+}
+
+// The largest i in [0, n) with off[i] <= x (off non-decreasing, off[0] <= x): the request (or
+// rank) whose range [off[i], off[i + 1]) holds x, skipping empty ranges before it.
+__device__ __forceinline__ int owner_of(const int32_t* off, int n, int32_t x) {
+  int lo = 0, hi = n;
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (off[mid] <= x) lo = mid; else hi = mid;
+  }
+  return lo;
+}
+
+// Chunked-prefill plan: requests with chunk_len == 1 are decode rows over prefix + 1 keys,
+// planned like a decode call over those requests; longer chunks become query tiles of kQTile
+// rows whose keys are cut on a fixed kChunkKvSplit grid, items ordered (request, query head,
+// split, tile). Every packed row gets its partial slots (its split count and the base of its
+// slots, the exclusive sum of the split counts of the rows before it), so the same combine
+// merges decode rows and tile rows.
+//
+// Launched on kPlanChunkCtas CTAs: each CTA derives the whole per-request plan (a few scans over
+// the B requests, latency-bound) in its own shared memory, identically, then writes its share
+// of the items and row tables, so the item stores, which one multiprocessor would serialise,
+// spread over the CTAs. CTA 0 alone writes the header.
 __global__ void __launch_bounds__(kMaxPlanThreads, 1) plan_chunk_kernel(PlanParams p) {
   pdl_launch_dependents();
   extern __shared__ int32_t smem[];
@@ -247,20 +309,29 @@ __global__ void __launch_bounds__(kMaxPlanThreads, 1) plan_chunk_kernel(PlanPara
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
   const int lane = static_cast<int>(lane_id());
+  const int g = p.hq / p.hkv;
+  // this CTA's share: threads take indices blockIdx.x * nthr + tid, ... (stride gt_step); warps
+  // take warp * gridDim.x + blockIdx.x, ... (stride gw_step), so a short warp loop spreads too
+  const int gt0 = static_cast<int>(blockIdx.x) * nthr + tid;
+  const int gt_step = static_cast<int>(gridDim.x) * nthr;
+  const int gw0 = warp * static_cast<int>(gridDim.x) + static_cast<int>(blockIdx.x);
+  const int gw_step = static_cast<int>(gridDim.x) * (nthr / 32);
+  const bool lead = blockIdx.x == 0;
   int32_t* s_c = smem;                 // chunk rows (>= 0)
   int32_t* s_p = s_c + B;              // prefix, clamped to [0, S_cap]
   int32_t* s_dlen = s_p + B;           // decode length (0 for tile requests)
   int32_t* s_n = s_dlen + B;           // decode splits
-  int32_t* s_key = s_n + B;            // decode ordering key
+  int32_t* s_key = s_n + B;            // decode ordering key; then the rank-ordered item counts
   int32_t* s_order = s_key + B;        // decode requests, longest first
   int32_t* s_tcnt = s_order + B;       // tile items per request
-  int32_t* s_tmp = s_tcnt + B;
-  int32_t* s_roff = s_tmp + B;         // B + 1: first packed row of each request
+  int32_t* s_nmax = s_tcnt + B;        // key splits of a multi-tile request's last query tile
+  int32_t* s_slots = s_nmax + B;       // partial slots of the request's rows
+  int32_t* s_roff = s_slots + B;       // B + 1: first packed row of each request
   int32_t* s_dioff = s_roff + B + 1;   // B + 1: decode item offsets (rank order)
   int32_t* s_tioff = s_dioff + B + 1;  // B + 1: tile item offsets (request order)
-  int32_t* s_nmax = s_tioff + B + 1;   // key splits of a multi-tile request's last query tile
-  int32_t* s_soff = s_nmax + B;        // B + 1: first (request, split) pair of each request
-  __shared__ int s_scan[33];
+  int32_t* s_soff = s_tioff + B + 1;   // B + 1: first (request, split) pair of each request
+  int32_t* s_rb = s_soff + B + 1;      // B + 1: partial-slot base of each request's first row
+  __shared__ int s_scan[3 * 33];
   __shared__ unsigned long long s_total;
   __shared__ unsigned long long s_key_tiles;  // 128-key tiles of all tile items
   __shared__ unsigned long long s_sums[kPlanWaveChoices];
@@ -270,6 +341,7 @@ __global__ void __launch_bounds__(kMaxPlanThreads, 1) plan_chunk_kernel(PlanPara
   if (tid < kPlanWaveChoices) s_sums[tid] = 0ull;
   __syncthreads();
 
+  // per request: what does not depend on the decode rows' chunk
   long long local = 0;
   int ndec = 0;
   for (int b = tid; b < B; b += nthr) {
@@ -283,45 +355,52 @@ __global__ void __launch_bounds__(kMaxPlanThreads, 1) plan_chunk_kernel(PlanPara
     s_p[b] = pp;
     s_dlen[b] = dlen;
     s_key[b] = c == 1 ? dlen : -1;  // the decode rows' lengths, for the chunk choice below
+    int32_t cnt = 0, slots = 0;
+    int64_t ktiles = 0;
+    if (c > 1) {
+      for (int32_t t = 0; t * kQTile < c; ++t) {
+        const int32_t kt = chunk_tile_keys(pp, c, t, p.cap);
+        const int32_t nt = chunk_tile_splits(kt);
+        cnt += nt;
+        slots += min(kQTile, c - t * kQTile) * nt;
+        ktiles += cdiv64(kt, kQTile);  // the split grid is a multiple of the key tile
+      }
+      const int32_t nheads = chunk_packed(c, g) ? p.hkv : p.hq;
+      atomicAdd(&s_key_tiles, static_cast<unsigned long long>(ktiles * nheads));
+      cnt *= nheads;
+    }
+    s_tcnt[b] = cnt;
+    s_slots[b] = slots;  // decode rows: their split count, once the chunk is known
+    // (request, split) pairs of the requests of more than one query tile; single-tile requests
+    // have their items written one per thread
+    s_nmax[b] = c > kQTile ? chunk_tile_splits(chunk_tile_keys(pp, c, (c - 1) / kQTile, p.cap)) : 0;
     local += dlen;
     ndec += c == 1 ? 1 : 0;
   }
   local = warp_sum_i64(local);
-  if (lane_id() == 0 && local != 0) atomicAdd(&s_total, static_cast<unsigned long long>(local));
+  if (lane == 0 && local != 0) atomicAdd(&s_total, static_cast<unsigned long long>(local));
   if (ndec) atomicAdd(&s_ndec, ndec);
   __syncthreads();
+  {
+    const int32_t* in[3] = {s_c, s_tcnt, s_nmax};
+    int32_t* out[3] = {s_roff, s_tioff, s_soff};
+    block_exclusive_scan_k<3>(in, out, B, s_scan);
+  }
 
   const int32_t chunk =
       plan_pick_chunk_block(s_key, B, static_cast<int64_t>(s_total), p.hkv, p.nctas, s_sums);
-  __syncthreads();  // s_key is rewritten below
   for (int b = tid; b < B; b += nthr) {
-    const int32_t c = s_c[b];
-    if (c == 1) {
+    if (s_c[b] == 1) {
       const int32_t n = plan_num_splits(s_dlen[b], chunk, 0);
       s_n[b] = n;
       s_key[b] = plan_sort_key(s_dlen[b], n);
-      s_tcnt[b] = 0;
-      s_nmax[b] = 0;
+      s_slots[b] = n;
     } else {
       s_n[b] = 0;
       s_key[b] = -1;
-      int32_t cnt = 0;
-      int64_t ktiles = 0;
-      for (int32_t t = 0; t * kQTile < c; ++t) {
-        const int32_t kt = chunk_tile_keys(s_p[b], c, t, p.cap);
-        cnt += chunk_tile_splits(kt);
-        ktiles += cdiv64(kt, kQTile);  // the split grid is a multiple of the key tile
-      }
-      const int32_t nheads = chunk_packed(c, p.hq / p.hkv) ? p.hkv : p.hq;
-      s_tcnt[b] = cnt * nheads;
-      // (request, split) pairs of the requests of more than one query tile; single-tile requests
-      // have their items written one per thread
-      s_nmax[b] = c > kQTile ? chunk_tile_splits(chunk_tile_keys(s_p[b], c, (c - 1) / kQTile, p.cap)) : 0;
-      if (c > 1) atomicAdd(&s_key_tiles, static_cast<unsigned long long>(ktiles * nheads));
     }
   }
   __syncthreads();
-  block_exclusive_scan(s_c, s_roff, B, s_scan);
   // decode requests longest first (stable counting rank among decode requests)
   for (int b = tid; b < B; b += nthr) {
     if (s_c[b] != 1) continue;
@@ -335,68 +414,62 @@ __global__ void __launch_bounds__(kMaxPlanThreads, 1) plan_chunk_kernel(PlanPara
   }
   __syncthreads();
   const int nd = s_ndec;
-  for (int r = tid; r < nd; r += nthr) s_tmp[r] = s_n[s_order[r]] * p.hkv;
+  // the keys are consumed: s_key now holds the item counts in rank order (zero past the last)
+  for (int r = tid; r < B; r += nthr) s_key[r] = r < nd ? s_n[s_order[r]] * p.hkv : 0;
   __syncthreads();
-  block_exclusive_scan(s_tmp, s_dioff, nd, s_scan);
-  block_exclusive_scan(s_tcnt, s_tioff, B, s_scan);
-  block_exclusive_scan(s_nmax, s_soff, B, s_scan);
+  {
+    const int32_t* in[2] = {s_key, s_slots};
+    int32_t* out[2] = {s_dioff, s_rb};
+    block_exclusive_scan_k<2>(in, out, B, s_scan);
+  }
   // chunk lengths that do not add up to the packed rows of q_chunk: nothing is computed (the
   // outputs are left as they were) and the status word says why
   const bool inconsistent = s_roff[B] != T;
-  if (tid == 0 && inconsistent) atomicOr(&s_flags, FD_FLAG_LEN_CLAMPED);
-
-  // partial slots per packed row, then their exclusive scan (global memory)
-  for (int b = warp; b < B && !inconsistent; b += nthr / 32) {
-    const int32_t c = s_c[b];
-    const int32_t r0 = s_roff[b];
-    for (int32_t r = lane; r < c; r += 32)
-      p.row_nsplit[r0 + r] = c == 1 ? s_n[b] : chunk_tile_splits(chunk_tile_keys(s_p[b], c, r / kQTile, p.cap));
-  }
-  if (inconsistent)
-    for (int32_t row = tid; row < T; row += nthr) p.row_nsplit[row] = 0;
-  __syncthreads();
-  block_exclusive_scan(p.row_nsplit, p.row_base, T, s_scan);
-  // partial-slot base of each request's first row, for the item loops below (s_tmp is free
-  // again: the decode ranks' scan has consumed it)
-  int32_t* s_rb = s_tmp;
-  for (int b = tid; b < B && !inconsistent; b += nthr) s_rb[b] = s_c[b] > 0 ? p.row_base[s_roff[b]] : 0;
-  __syncthreads();
-
-  const int32_t n_dec_items = s_dioff[nd];
+  const int32_t n_dec_items = s_dioff[B];
   const int32_t n_tile_items = s_tioff[B];
   const bool overflow =
       inconsistent || n_dec_items > p.max_dec_items || n_tile_items > p.max_tile_items;
-  // decode items: one warp per decode request. With n <= 32 splits, lane L takes split L mod n of
-  // heads L / n, L / n + 32 / n, ... (its key range computed once); with more, lanes take splits
-  // and loop over the heads. Item (h, s) sits at first + h n + s.
-  for (int r = warp; r < nd && !overflow; r += nthr / 32) {
-    const int b = s_order[r];
-    const int32_t row = s_roff[b];
-    const int32_t n = s_n[b], L = s_dlen[b], first = s_dioff[r];
-    const int32_t rbase = s_rb[b];
-    const int32_t per = n <= 32 ? 32 / n : 1;  // heads a pass covers
-    const int32_t s0 = n <= 32 ? lane % n : lane;
-    const int32_t h0 = n <= 32 ? lane / n : 0;
-    if (h0 >= per) continue;  // lanes past the last whole group of n
-    for (int32_t s = s0; s < n; s += 32) {
-      int32_t t0, t1;
-      plan_split_range(L, n, s, 0, p.align, &t0, &t1);
-      for (int32_t h = h0; h < p.hkv; h += per) {
-        int4* dst = reinterpret_cast<int4*>(p.items + first + h * n + s);
-        dst[0] = make_int4(row, b, h, s);
-        dst[1] = make_int4(t0, t1, n, rbase * p.hkv + h * n + s);
-      }
+
+  // split count and partial-slot base of every packed row: a decode row has its request's n
+  // slots (1 when it merges inside its split kernel: the combine skips it); row j of a tile
+  // request sits in query tile t = j / kQTile, after the full tiles before it, with nt(t) slots
+  for (int r = gt0; r < T; r += gt_step) {
+    if (inconsistent) {
+      p.row_nsplit[r] = 0;
+      p.row_base[r] = 0;
+      continue;
     }
+    const int b = owner_of(s_roff, B, r);
+    const int32_t c = s_c[b], j = r - s_roff[b];
+    int32_t nsplit, base = s_rb[b];
+    if (c == 1) {
+      nsplit = p.decode_merged_in_kernel ? 1 : s_n[b];
+    } else {
+      const int32_t t = j / kQTile;
+      for (int32_t u = 0; u < t; ++u) base += kQTile * chunk_tile_splits(chunk_tile_keys(s_p[b], c, u, p.cap));
+      nsplit = chunk_tile_splits(chunk_tile_keys(s_p[b], c, t, p.cap));
+      base += (j - t * kQTile) * nsplit;
+    }
+    p.row_nsplit[r] = nsplit;
+    p.row_base[r] = base;
+  }
+  // decode items, one per thread: item i of rank r's request is (head e / n, split e mod n),
+  // e = i - first, so item (h, s) sits at first + h n + s
+  for (int i = gt0; i < (overflow ? 0 : n_dec_items); i += gt_step) {
+    const int r = owner_of(s_dioff, nd, i);
+    const int b = s_order[r];
+    const int32_t n = s_n[b], e = i - s_dioff[r];
+    const int32_t h = e / n, s = e - h * n;
+    int32_t t0, t1;
+    plan_split_range(s_dlen[b], n, s, 0, p.align, &t0, &t1);
+    int4* dst = reinterpret_cast<int4*>(p.items + i);
+    dst[0] = make_int4(s_roff[b], b, h, s);
+    dst[1] = make_int4(t0, t1, n, s_rb[b] * p.hkv + h * n + s);
   }
   // tile items of single-tile requests (2 <= c <= 128 rows: verification steps, short chunks):
   // one thread per item. Item e of the request is head e / n, split e mod n (n splits).
-  for (int i = tid; i < (overflow ? 0 : s_tioff[B]); i += nthr) {
-    int lo = 0, hi = B;  // the request of item i: s_tioff[lo] <= i < s_tioff[lo + 1]
-    while (hi - lo > 1) {
-      const int mid = (lo + hi) >> 1;
-      if (s_tioff[mid] <= i) lo = mid; else hi = mid;
-    }
-    const int b = lo;
+  for (int i = gt0; i < (overflow ? 0 : n_tile_items); i += gt_step) {
+    const int b = owner_of(s_tioff, B, i);
     const int32_t c = s_c[b];
     if (c > kQTile) continue;  // written below, per (request, split) pair
     const int32_t pp = s_p[b];
@@ -408,24 +481,19 @@ __global__ void __launch_bounds__(kMaxPlanThreads, 1) plan_chunk_kernel(PlanPara
     int4* dst = reinterpret_cast<int4*>(p.tiles + i);
     dst[0] = make_int4(b, h, s, nt);
     dst[1] = make_int4(k0, k1, s_roff[b], 0);
-    dst[2] = make_int4(c, pp, s_rb[b] * p.hkv, chunk_packed(c, p.hq / p.hkv) ? 1 : 0);
+    dst[2] = make_int4(c, pp, s_rb[b] * p.hkv, chunk_packed(c, g) ? 1 : 0);
     dst[3] = make_int4(0, 0, 0, 0);
   }
   // tile items of longer requests: one warp per (request, split) pair, lanes over query heads
   // (KV heads for head-packed tiles). Per head the items run split by split and, within a
   // split, tile by tile over the query tiles that see that split's keys.
   const int32_t n_pairs = s_soff[B];
-  for (int k = warp; k < n_pairs && !overflow; k += nthr / 32) {
-    int lo = 0, hi = B;  // the request of pair k: s_soff[lo] <= k < s_soff[lo + 1]
-    while (hi - lo > 1) {
-      const int mid = (lo + hi) >> 1;
-      if (s_soff[mid] <= k) lo = mid; else hi = mid;
-    }
-    const int b = lo;
+  for (int k = gw0; k < (overflow ? 0 : n_pairs); k += gw_step) {
+    const int b = owner_of(s_soff, B, k);
     const int32_t s = k - s_soff[b];
     const int32_t c = s_c[b], pp = s_p[b], r0 = s_roff[b];
     const int32_t ntiles = (c + kQTile - 1) / kQTile;
-    const int32_t head_packed = chunk_packed(c, p.hq / p.hkv) ? 1 : 0;
+    const int32_t head_packed = chunk_packed(c, g) ? 1 : 0;
     const int32_t nheads = head_packed ? p.hkv : p.hq;
     const int32_t per_head = s_tcnt[b] / nheads;
     // items of the earlier splits in each head's run: query tile t has min(nt(t), s) of them
@@ -456,14 +524,12 @@ __global__ void __launch_bounds__(kMaxPlanThreads, 1) plan_chunk_kernel(PlanPara
       }
     }
   }
-  __syncthreads();
-  // decode rows merged inside their split kernel: the combine skips them; their counters reset
-  for (int e = tid; e < nd * p.hkv && !inconsistent; e += nthr) {
+  // the split kernels' completion counters of the decode rows
+  for (int e = gt0; e < (inconsistent ? 0 : nd * p.hkv); e += gt_step) {
     const int r = e / p.hkv, h = e - r * p.hkv;
-    const int32_t row = s_roff[s_order[r]];
-    if (p.decode_merged_in_kernel && h == 0) p.row_nsplit[row] = 1;
-    p.arrivals[row * p.hkv + h] = 0;
+    p.arrivals[s_roff[s_order[r]] * p.hkv + h] = 0;
   }
+  if (!lead) return;
   if (warp == 0) {
     // the tile kernel's CTAs: the n of least chunk_tile_cost, smallest on ties; lane l weighs
     // n = l + 1, l + 33, ... and the warp keeps the lexicographic minimum of (cost, n)
@@ -494,11 +560,12 @@ __global__ void __launch_bounds__(kMaxPlanThreads, 1) plan_chunk_kernel(PlanPara
     if (lane == 0) p.hdr->tile_ctas = n_best;
   }
   if (tid == 0) {
+    p.row_base[T] = inconsistent ? 0 : s_rb[B];
     p.hdr->num_dec_items = overflow ? 0 : n_dec_items;
     p.hdr->num_tile_items = overflow ? 0 : n_tile_items;
     p.hdr->dec_counter = 0;
     p.hdr->tile_counter = 0;
-    uint32_t f = s_flags | (overflow ? FD_FLAG_PLAN_OVERFLOW : 0u);
+    uint32_t f = s_flags | (inconsistent ? FD_FLAG_LEN_CLAMPED : 0u) | (overflow ? FD_FLAG_PLAN_OVERFLOW : 0u);
     if (f) atomicOr(&p.hdr->status, f);
   }
 }
@@ -506,14 +573,14 @@ __global__ void __launch_bounds__(kMaxPlanThreads, 1) plan_chunk_kernel(PlanPara
 }  // namespace
 
 cudaError_t launch_plan_chunk(const PlanParams& p, cudaStream_t stream) {
-  const size_t smem = sizeof(int32_t) * (13 * static_cast<size_t>(p.B) + 4);
+  const size_t smem = sizeof(int32_t) * (14 * static_cast<size_t>(p.B) + 5);
   if (smem > 48 * 1024) {
     cudaError_t e = cudaFuncSetAttribute(plan_chunk_kernel,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
     if (e != cudaSuccess) return e;
   }
-  plan_chunk_kernel<<<1, kMaxPlanThreads, smem, stream>>>(p);
+  plan_chunk_kernel<<<kPlanChunkCtas, kMaxPlanThreads, smem, stream>>>(p);
   return cudaGetLastError();
 }
 

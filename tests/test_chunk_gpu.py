@@ -51,7 +51,7 @@ CASES = [
     # (prefix_lens, chunk_lens, Hq, Hkv, cap)
     ([0], [5], 2, 2, 64),                          # tiny chunk, no prefix
     ([300], [130], 2, 2, 512),                     # two tiles, ragged second tile
-    ([1900], [300], 2, 2, 4096),                   # tile 0 one split, tiles 1-2 two splits
+    ([3900], [300], 2, 2, 8192),                   # tile 0 one split, tiles 1-2 two splits
     ([2500, 10, 0, 700, 33], [200, 1, 1, 1, 0], 4, 4, 4096),  # chunk + decode rows + empty
     ([1000, 77, 4000], [129, 1, 1], 16, 2, 4200),  # GQA (G = 8): decode rows on tensor cores
     ([64], [64], 4, 1, 128),                       # GQA G = 4, capacity = prefix + chunk
@@ -112,6 +112,40 @@ def test_full_mixed_workload():
     ro, rl = _oracle(inp)
     check_out(out, ro, "workload 5 out")
     check_lse(lse, rl, "workload 5 lse")
+
+
+def test_many_requests_of_every_kind():
+    # 70 requests in one call: empty ones, decode rows, head-packed verification steps (G = 4),
+    # single-tile and multi-tile chunks, in an irregular order, so the planner's CTAs each write
+    # a share of every item kind and of the row tables
+    rng = np.random.default_rng(81)
+    kinds = [0, 1, 4, 1, 200, 0, 1, 17, 3, 130, 1, 1, 32, 33, 2, 0, 1, 260, 1, 5]
+    chunk = [kinds[i % len(kinds)] if i % 7 else int(rng.integers(0, 40)) for i in range(70)]
+    cap = 1536
+    prefix = [int(rng.integers(0, cap - c + 1)) for c in chunk]
+    inp = make_chunk_inputs(prefix, chunk, 16, 4, 128, cap, torch.bfloat16, seed=82, pad_fill=NAN)
+    out, lse = _run(inp)
+    ro, rl = _oracle(inp)
+    check_out(out, ro, "70 requests out")
+    check_lse(lse, rl, "70 requests lse")
+
+
+def test_chunk_lengths_not_matching_rows():
+    # chunk lengths that do not add up to q_chunk's rows: nothing is written, the flag is raised
+    import split_kv_decode_flashdecoding_b200 as fd
+    dev = torch.device("cuda", 0)
+    inp = make_chunk_inputs([300, 40], [20, 1], 8, 2, 128, 512, torch.bfloat16, seed=83)
+    q = inp.q_chunk.to(dev)
+    out = torch.full_like(q, 7.0)
+    lse = torch.full(q.shape[:2], 9.0, dtype=torch.float32, device=dev)
+    fd.fd_poll_status()
+    fd.fd_chunk_prefill_attention(q, inp.k_cache.to(dev), inp.v_cache.to(dev),
+                                  inp.prefix_lens.to(dev),
+                                  torch.tensor([20, 2], dtype=torch.int32, device=dev),
+                                  out=out, lse=lse)
+    torch.cuda.synchronize()
+    assert fd.fd_poll_status() & fd.FD_FLAG_LEN_CLAMPED
+    assert bool((out == 7.0).all()) and bool((lse == 9.0).all())
 
 
 def test_chunk_deterministic():

@@ -134,22 +134,22 @@ def test_chunk_plan_hand_worked():
     cp = P.chunk_plan([5000, 69], [300, 1], 2, 2, 8192, 148)
     assert cp.decode_requests == [1]
     assert cp.decode.splits_per_seq == [1]
-    # tiles see <= 5128, 5256, 5300 keys -> 3 splits each on the 2048-key grid
-    assert cp.row_splits == [3] * 300 + [1]
+    # tiles see <= 5128, 5256, 5300 keys -> 2 splits each on the 4096-key grid
+    assert cp.row_splits == [2] * 300 + [1]
     spans = sorted({(t, s, k0, k1) for (b, t, h, s, k0, k1) in cp.tile_items if t == 0})
-    assert spans == [(0, 0, 0, 2048), (0, 1, 2048, 4096), (0, 2, 4096, 5128)]
-    assert len(cp.tile_items) == 3 * 2 * 3
+    assert spans == [(0, 0, 0, 4096), (0, 1, 4096, 5128)]
+    assert len(cp.tile_items) == 3 * 2 * 2
     # order: head, split, tile
     assert [(h, s, t) for (b, t, h, s, k0, k1) in cp.tile_items[:4]] == [
         (0, 0, 0), (0, 0, 1), (0, 0, 2), (0, 1, 0)]
 
 
 def test_chunk_plan_tiles_with_fewer_splits():
-    # a 300-row chunk at prefix 1900: tile 0 sees <= 2028 keys (1 split), tiles 1-2 see more (2)
-    cp = P.chunk_plan([1900], [300], 1, 1, 4096, 148)
+    # a 300-row chunk at prefix 3900: tile 0 sees <= 4028 keys (1 split), tiles 1-2 see more (2)
+    cp = P.chunk_plan([3900], [300], 1, 1, 8192, 148)
     assert cp.row_splits == [1] * 128 + [2] * 172
     assert [(t, s, k0, k1) for (b, t, h, s, k0, k1) in cp.tile_items] == [
-        (0, 0, 0, 2028), (1, 0, 0, 2048), (2, 0, 0, 2048), (1, 1, 2048, 2156), (2, 1, 2048, 2200)]
+        (0, 0, 0, 4028), (1, 0, 0, 4096), (2, 0, 0, 4096), (1, 1, 4096, 4156), (2, 1, 4096, 4200)]
 
 
 # ---- aligned plans (paged cache): split boundaries on multiples of the key tile ----------------
@@ -192,13 +192,13 @@ def test_aligned_plan_properties(seed):
 def test_chunk_plan_head_packed_requests():
     # G = 8: chunks of 2..16 rows are head-packed (one tile per KV head and split), longer ones
     # and decode rows are not; G = 1 never packs
-    cp = P.chunk_plan([3000, 40, 100, 7], [4, 16, 17, 1], 64, 8, 8192, 148)
+    cp = P.chunk_plan([5000, 40, 100, 7], [4, 16, 17, 1], 64, 8, 8192, 148)
     assert cp.head_packed == [0, 1]
     heads0 = sorted({h for (b, t, h, s, k0, k1) in cp.tile_items if b == 0})
     assert heads0 == list(range(8))
-    # request 0 sees 3004 keys: two splits per KV head, one query tile
+    # request 0 sees 5004 keys: two splits per KV head, one query tile
     assert sorted({(t, s, k0, k1) for (b, t, h, s, k0, k1) in cp.tile_items if b == 0}) == \
-        [(0, 0, 0, 2048), (0, 1, 2048, 3004)]
+        [(0, 0, 0, 4096), (0, 1, 4096, 5004)]
     assert len([1 for it in cp.tile_items if it[0] == 2]) == 64      # per query head
     assert cp.row_splits[:4] == [2, 2, 2, 2] and cp.row_splits[4:20] == [1] * 16
     assert P.chunk_plan([10], [4], 8, 8, 1024, 148).head_packed == []
