@@ -341,87 +341,182 @@ __global__ void __launch_bounds__(kMaxPlanThreads, 1) plan_chunk_kernel(PlanPara
   if (tid < kPlanWaveChoices) s_sums[tid] = 0ull;
   __syncthreads();
 
-  // per request: what does not depend on the decode rows' chunk
-  long long local = 0;
-  int ndec = 0;
-  for (int b = tid; b < B; b += nthr) {
-    const int32_t raw_p = p.lens[b], raw_c = p.chunk_lens[b];
-    const int32_t c = raw_c < 0 ? 0 : raw_c;
-    const int32_t pp = clamp_len(raw_p, p.cap);
-    if (raw_c < 0 || pp != raw_p || static_cast<int64_t>(pp) + c > p.cap)
-      atomicOr(&s_flags, FD_FLAG_LEN_CLAMPED);
-    const int32_t dlen = c == 1 ? clamp_len(static_cast<int64_t>(pp) + 1, p.cap) : 0;
-    s_c[b] = c;
-    s_p[b] = pp;
-    s_dlen[b] = dlen;
-    s_key[b] = c == 1 ? dlen : -1;  // the decode rows' lengths, for the chunk choice below
-    int32_t cnt = 0, slots = 0;
-    int64_t ktiles = 0;
-    if (c > 1) {
-      for (int32_t t = 0; t * kQTile < c; ++t) {
-        const int32_t kt = chunk_tile_keys(pp, c, t, p.cap);
-        const int32_t nt = chunk_tile_splits(kt);
-        cnt += nt;
-        slots += min(kQTile, c - t * kQTile) * nt;
-        ktiles += cdiv64(kt, kQTile);  // the split grid is a multiple of the key tile
+  if (B <= 32) {
+    // Up to 32 requests: one warp derives the same per-request plan as the block path below, a
+    // request per lane, with shuffles in place of barrier-separated phases (each ~2 µs of
+    // latency there: loads, block scans, the chunk choice, the ranking).
+    if (warp == 0) {
+      const bool has = lane < B;
+      const int32_t raw_p = has ? p.lens[lane] : 0, raw_c = has ? p.chunk_lens[lane] : 0;
+      const int32_t c = raw_c < 0 ? 0 : raw_c;
+      const int32_t pp = clamp_len(raw_p, p.cap);
+      const bool clamped =
+          has && (raw_c < 0 || pp != raw_p || static_cast<int64_t>(pp) + c > p.cap);
+      const bool dec = has && c == 1;
+      const int32_t dlen = dec ? clamp_len(static_cast<int64_t>(pp) + 1, p.cap) : 0;
+      int32_t cnt = 0, slots = 0;
+      long long ktiles = 0;
+      if (has && c > 1) {
+        for (int32_t t = 0; t * kQTile < c; ++t) {
+          const int32_t kt = chunk_tile_keys(pp, c, t, p.cap);
+          const int32_t nt = chunk_tile_splits(kt);
+          cnt += nt;
+          slots += min(kQTile, c - t * kQTile) * nt;
+          ktiles += cdiv64(kt, kQTile);
+        }
+        const int32_t nheads = chunk_packed(c, g) ? p.hkv : p.hq;
+        cnt *= nheads;
+        ktiles *= nheads;
       }
-      const int32_t nheads = chunk_packed(c, g) ? p.hkv : p.hq;
-      atomicAdd(&s_key_tiles, static_cast<unsigned long long>(ktiles * nheads));
-      cnt *= nheads;
+      const int32_t nmax =
+          (has && c > kQTile) ? chunk_tile_splits(chunk_tile_keys(pp, c, (c - 1) / kQTile, p.cap)) : 0;
+      const long long total = warp_sum_i64(dlen);
+      const long long key_tiles = warp_sum_i64(ktiles);
+      const uint32_t dmask = __ballot_sync(0xffffffffu, dec);
+      const int nd = __popc(dmask);
+      // the decode rows' chunk (plan_pick_chunk over their lengths)
+      int32_t chunks[kPlanWaveChoices];
+      int64_t sums[kPlanWaveChoices];
+#pragma unroll
+      for (int i = 0; i < kPlanWaveChoices; ++i) {
+        chunks[i] = plan_chunk_for_waves(total, p.hkv, p.nctas, plan_waves(i));
+        sums[i] = warp_sum_i64(dec ? plan_num_splits(dlen, chunks[i], 0) : 0);
+      }
+      const int32_t chunk = plan_pick_chunk(chunks, sums, p.hkv, p.nctas);
+      const int32_t n = dec ? plan_num_splits(dlen, chunk, 0) : 0;
+      const int32_t key = dec ? plan_sort_key(dlen, n) : -1;
+      if (dec) slots = n;
+      // longest-first rank among the decode requests (stable) and the first decode item of the
+      // request in rank order
+      int r = 0, ioff = 0;
+      for (int j = 0; j < 32; ++j) {
+        const int32_t kj = __shfl_sync(0xffffffffu, key, j);
+        const int32_t nj = __shfl_sync(0xffffffffu, n, j);
+        const bool before = ((dmask >> j) & 1u) && (kj > key || (kj == key && j < lane));
+        r += before ? 1 : 0;
+        ioff += before ? nj * p.hkv : 0;
+      }
+      const int dec_items = static_cast<int>(warp_sum_i64(n * p.hkv));
+      // exclusive scans over the requests: rows, tile items, (request, split) pairs, slots
+      const int i_c = warp_incl_scan(c), i_t = warp_incl_scan(cnt), i_s = warp_incl_scan(nmax);
+      const int i_r = warp_incl_scan(slots);
+      if (has) {
+        s_c[lane] = c;
+        s_p[lane] = pp;
+        s_dlen[lane] = dlen;
+        s_n[lane] = n;
+        s_tcnt[lane] = cnt;
+        s_nmax[lane] = nmax;
+        s_slots[lane] = slots;
+        s_roff[lane] = i_c - c;
+        s_tioff[lane] = i_t - cnt;
+        s_soff[lane] = i_s - nmax;
+        s_rb[lane] = i_r - slots;
+        if (dec) {
+          s_order[r] = lane;
+          s_dioff[r] = ioff;
+        }
+      }
+      for (int j = nd + lane; j <= B; j += 32) s_dioff[j] = dec_items;
+      const bool any_clamped = __any_sync(0xffffffffu, clamped);
+      if (lane == B - 1) {
+        s_roff[B] = i_c;
+        s_tioff[B] = i_t;
+        s_soff[B] = i_s;
+        s_rb[B] = i_r;
+      }
+      if (lane == 0) {
+        s_total = static_cast<unsigned long long>(total);
+        s_key_tiles = static_cast<unsigned long long>(key_tiles);
+        s_ndec = nd;
+        if (any_clamped) s_flags = FD_FLAG_LEN_CLAMPED;
+      }
     }
-    s_tcnt[b] = cnt;
-    s_slots[b] = slots;  // decode rows: their split count, once the chunk is known
-    // (request, split) pairs of the requests of more than one query tile; single-tile requests
-    // have their items written one per thread
-    s_nmax[b] = c > kQTile ? chunk_tile_splits(chunk_tile_keys(pp, c, (c - 1) / kQTile, p.cap)) : 0;
-    local += dlen;
-    ndec += c == 1 ? 1 : 0;
-  }
-  local = warp_sum_i64(local);
-  if (lane == 0 && local != 0) atomicAdd(&s_total, static_cast<unsigned long long>(local));
-  if (ndec) atomicAdd(&s_ndec, ndec);
-  __syncthreads();
-  {
-    const int32_t* in[3] = {s_c, s_tcnt, s_nmax};
-    int32_t* out[3] = {s_roff, s_tioff, s_soff};
-    block_exclusive_scan_k<3>(in, out, B, s_scan);
-  }
+    __syncthreads();
+  } else {
+    // per request: what does not depend on the decode rows' chunk
+    long long local = 0;
+    int ndec = 0;
+    for (int b = tid; b < B; b += nthr) {
+      const int32_t raw_p = p.lens[b], raw_c = p.chunk_lens[b];
+      const int32_t c = raw_c < 0 ? 0 : raw_c;
+      const int32_t pp = clamp_len(raw_p, p.cap);
+      if (raw_c < 0 || pp != raw_p || static_cast<int64_t>(pp) + c > p.cap)
+        atomicOr(&s_flags, FD_FLAG_LEN_CLAMPED);
+      const int32_t dlen = c == 1 ? clamp_len(static_cast<int64_t>(pp) + 1, p.cap) : 0;
+      s_c[b] = c;
+      s_p[b] = pp;
+      s_dlen[b] = dlen;
+      s_key[b] = c == 1 ? dlen : -1;  // the decode rows' lengths, for the chunk choice below
+      int32_t cnt = 0, slots = 0;
+      int64_t ktiles = 0;
+      if (c > 1) {
+        for (int32_t t = 0; t * kQTile < c; ++t) {
+          const int32_t kt = chunk_tile_keys(pp, c, t, p.cap);
+          const int32_t nt = chunk_tile_splits(kt);
+          cnt += nt;
+          slots += min(kQTile, c - t * kQTile) * nt;
+          ktiles += cdiv64(kt, kQTile);  // the split grid is a multiple of the key tile
+        }
+        const int32_t nheads = chunk_packed(c, g) ? p.hkv : p.hq;
+        atomicAdd(&s_key_tiles, static_cast<unsigned long long>(ktiles * nheads));
+        cnt *= nheads;
+      }
+      s_tcnt[b] = cnt;
+      s_slots[b] = slots;  // decode rows: their split count, once the chunk is known
+      // (request, split) pairs of the requests of more than one query tile; single-tile requests
+      // have their items written one per thread
+      s_nmax[b] = c > kQTile ? chunk_tile_splits(chunk_tile_keys(pp, c, (c - 1) / kQTile, p.cap)) : 0;
+      local += dlen;
+      ndec += c == 1 ? 1 : 0;
+    }
+    local = warp_sum_i64(local);
+    if (lane == 0 && local != 0) atomicAdd(&s_total, static_cast<unsigned long long>(local));
+    if (ndec) atomicAdd(&s_ndec, ndec);
+    __syncthreads();
+    {
+      const int32_t* in[3] = {s_c, s_tcnt, s_nmax};
+      int32_t* out[3] = {s_roff, s_tioff, s_soff};
+      block_exclusive_scan_k<3>(in, out, B, s_scan);
+    }
 
-  const int32_t chunk =
-      plan_pick_chunk_block(s_key, B, static_cast<int64_t>(s_total), p.hkv, p.nctas, s_sums);
-  for (int b = tid; b < B; b += nthr) {
-    if (s_c[b] == 1) {
-      const int32_t n = plan_num_splits(s_dlen[b], chunk, 0);
-      s_n[b] = n;
-      s_key[b] = plan_sort_key(s_dlen[b], n);
-      s_slots[b] = n;
-    } else {
-      s_n[b] = 0;
-      s_key[b] = -1;
+    const int32_t chunk =
+        plan_pick_chunk_block(s_key, B, static_cast<int64_t>(s_total), p.hkv, p.nctas, s_sums);
+    for (int b = tid; b < B; b += nthr) {
+      if (s_c[b] == 1) {
+        const int32_t n = plan_num_splits(s_dlen[b], chunk, 0);
+        s_n[b] = n;
+        s_key[b] = plan_sort_key(s_dlen[b], n);
+        s_slots[b] = n;
+      } else {
+        s_n[b] = 0;
+        s_key[b] = -1;
+      }
+    }
+    __syncthreads();
+    // decode requests longest first (stable counting rank among decode requests)
+    for (int b = tid; b < B; b += nthr) {
+      if (s_c[b] != 1) continue;
+      const int32_t kb = s_key[b];
+      int r = 0;
+      for (int j = 0; j < B; ++j) {
+        const int32_t kj = s_key[j];
+        r += (s_c[j] == 1 && (kj > kb || (kj == kb && j < b))) ? 1 : 0;
+      }
+      s_order[r] = b;
+    }
+    __syncthreads();
+    const int ndb = s_ndec;
+    // the keys are consumed: s_key now holds the item counts in rank order (zero past the last)
+    for (int r = tid; r < B; r += nthr) s_key[r] = r < ndb ? s_n[s_order[r]] * p.hkv : 0;
+    __syncthreads();
+    {
+      const int32_t* in[2] = {s_key, s_slots};
+      int32_t* out[2] = {s_dioff, s_rb};
+      block_exclusive_scan_k<2>(in, out, B, s_scan);
     }
   }
-  __syncthreads();
-  // decode requests longest first (stable counting rank among decode requests)
-  for (int b = tid; b < B; b += nthr) {
-    if (s_c[b] != 1) continue;
-    const int32_t kb = s_key[b];
-    int r = 0;
-    for (int j = 0; j < B; ++j) {
-      const int32_t kj = s_key[j];
-      r += (s_c[j] == 1 && (kj > kb || (kj == kb && j < b))) ? 1 : 0;
-    }
-    s_order[r] = b;
-  }
-  __syncthreads();
   const int nd = s_ndec;
-  // the keys are consumed: s_key now holds the item counts in rank order (zero past the last)
-  for (int r = tid; r < B; r += nthr) s_key[r] = r < nd ? s_n[s_order[r]] * p.hkv : 0;
-  __syncthreads();
-  {
-    const int32_t* in[2] = {s_key, s_slots};
-    int32_t* out[2] = {s_dioff, s_rb};
-    block_exclusive_scan_k<2>(in, out, B, s_scan);
-  }
   // chunk lengths that do not add up to the packed rows of q_chunk: nothing is computed (the
   // outputs are left as they were) and the status word says why
   const bool inconsistent = s_roff[B] != T;
