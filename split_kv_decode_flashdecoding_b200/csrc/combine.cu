@@ -31,13 +31,18 @@ namespace {
 
 constexpr int kCombineWarps = 8;
 constexpr int kBatch = 8;  // splits whose loads one warp keeps in flight together
+// Calls of at least this many (row, query head) pairs (chunked prefill: every packed row of every
+// head) use a warp kernel that keeps 4 splits in flight and 48 registers a thread, for 5 CTAs
+// per multiprocessor instead of 3: their pairs have few splits each and fill several waves, so
+// more warps in flight beat more loads per warp.
+constexpr int64_t kManyPairs = 8192;
 // Above this many (row, query head) pairs every warp merges a pair of its own (eight pairs per
 // CTA); below, the eight warps of a CTA share one pair's splits.
 constexpr int64_t kWarpPerPairMin = 1024;
 
 // Online merge of splits s = first, first + step, ... < n of one (row, query head) by one warp:
 // running max m, weight sum wsum, weighted sum acc (kVec elements of D per lane).
-template <int kVec>
+template <int kVec, int kB = kBatch>
 __device__ __forceinline__ void merge_splits(const float* lse_base, int64_t lse_step,
                                              const float* o_base, int64_t o_step, int n,
                                              int first, int step, float& m, float& wsum,
@@ -46,11 +51,11 @@ __device__ __forceinline__ void merge_splits(const float* lse_base, int64_t lse_
   wsum = 0.f;
 #pragma unroll
   for (int e = 0; e < kVec; ++e) acc[e] = 0.f;
-  for (int s0 = first; s0 < n; s0 += kBatch * step) {
-    float l[kBatch];
-    float x[kBatch][kVec];
+  for (int s0 = first; s0 < n; s0 += kB * step) {
+    float l[kB];
+    float x[kB][kVec];
 #pragma unroll
-    for (int j = 0; j < kBatch; ++j) {
+    for (int j = 0; j < kB; ++j) {
       const int s = s0 + j * step;
       l[j] = -INFINITY;
 #pragma unroll
@@ -69,14 +74,14 @@ __device__ __forceinline__ void merge_splits(const float* lse_base, int64_t lse_
     }
     float mn = m;
 #pragma unroll
-    for (int j = 0; j < kBatch; ++j) mn = fmaxf(mn, l[j]);
+    for (int j = 0; j < kB; ++j) mn = fmaxf(mn, l[j]);
     if (mn == -INFINITY) continue;  // nothing visible yet
     const float scale = fast_exp2(m - mn);  // 0 while m = -inf
     wsum *= scale;
 #pragma unroll
     for (int e = 0; e < kVec; ++e) acc[e] *= scale;
 #pragma unroll
-    for (int j = 0; j < kBatch; ++j) {
+    for (int j = 0; j < kB; ++j) {
       const float w = fast_exp2(l[j] - mn);  // 0 for an empty split (l = -inf)
       wsum += w;
 #pragma unroll
@@ -157,9 +162,10 @@ __global__ void __launch_bounds__(kCombineWarps * 32) combine_cta_kernel(Combine
     p.lse[static_cast<int64_t>(v.row) * p.hq + v.hq] = W > 0.f ? (M + log2f(W)) * kLn2 : -INFINITY;
 }
 
-// One warp per (row, query head), eight pairs per CTA: every warp merges all splits of its pair.
-template <typename T, int D>
-__global__ void __launch_bounds__(kCombineWarps * 32) combine_warp_kernel(CombineParams p) {
+// One warp per (row, query head), eight pairs per CTA: every warp merges all splits of its pair,
+// kB at a time.
+template <typename T, int D, int kB, int kMinCtas>
+__global__ void __launch_bounds__(kCombineWarps * 32, kMinCtas) combine_warp_kernel(CombineParams p) {
   constexpr int kVec = D / 32;
   pdl_launch_dependents();
   pdl_wait_prerequisites();
@@ -170,7 +176,7 @@ __global__ void __launch_bounds__(kCombineWarps * 32) combine_warp_kernel(Combin
   const PairView v = pair_view<D>(p, pair, lane);
   if (v.n <= 1) return;
   float m, wsum, acc[kVec];
-  merge_splits<kVec>(v.lse_base, v.lse_step, v.o_base, v.o_step, v.n, 0, 1, m, wsum, acc);
+  merge_splits<kVec, kB>(v.lse_base, v.lse_step, v.o_base, v.o_step, v.n, 0, 1, m, wsum, acc);
   const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
 #pragma unroll
   for (int e = 0; e < kVec; ++e) write_out<T>(p, v.row, v.hq, lane * kVec + e, acc[e] * inv);
@@ -191,8 +197,9 @@ cudaError_t launch_combine_t(const CombineParams& p, int64_t pairs, cudaStream_t
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return per_warp ? cudaLaunchKernelEx(&cfg, combine_warp_kernel<T, D>, p)
-                  : cudaLaunchKernelEx(&cfg, combine_cta_kernel<T, D>, p);
+  if (!per_warp) return cudaLaunchKernelEx(&cfg, combine_cta_kernel<T, D>, p);
+  return pairs >= kManyPairs ? cudaLaunchKernelEx(&cfg, combine_warp_kernel<T, D, 4, 5>, p)
+                             : cudaLaunchKernelEx(&cfg, combine_warp_kernel<T, D, kBatch, 3>, p);
 }
 
 }  // namespace
