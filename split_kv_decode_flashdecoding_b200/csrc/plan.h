@@ -32,7 +32,7 @@ constexpr int32_t kQTile = 128;           // chunked-prefill query rows per tile
 // and merge) and leaves the mixed 512-row chunk step unchanged; 6144 and 8192 slow the chunk
 // step (fewer, longer tile items balance worse over the tile kernel's CTAs).
 constexpr int32_t kChunkKvSplit = 4096;
-constexpr int32_t kMaxPlanBatch = 4096;   // largest batch the one-CTA device planner accepts
+constexpr int32_t kMaxPlanBatch = 4096;   // largest batch the device planners accept (shared memory per CTA)
 constexpr int32_t kFusedPlanMaxBatch = 256;  // largest batch the tensor-core split kernel plans itself
 constexpr int32_t kPagedKeyAlign = 128;      // split boundaries of a paged cache: one key tile
 constexpr int32_t kTcKeyAlign = 128;         // split boundaries on the tensor-core decode path

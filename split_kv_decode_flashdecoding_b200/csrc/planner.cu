@@ -1,6 +1,7 @@
-// Device split planner: one CTA turns the device-resident lengths into the work-item list, the
-// per-row split counts and the partial-slot bases, so a call needs no host synchronisation.
-// The arithmetic is plan.h's, shared with the host planner fd_split_plan.
+// Device split planners (decode: one CTA; chunked prefill: several CTAs that derive the same
+// per-request plan and share the item stores) turn the device-resident lengths into the
+// work-item list, the per-row split counts and the partial-slot bases, so a call needs no host
+// synchronisation. The arithmetic is plan.h's, shared with the host planner fd_split_plan.
 #include "common.cuh"
 #include "internal.h"
 
