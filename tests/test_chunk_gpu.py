@@ -73,9 +73,10 @@ def test_small_chunks(case):
 CASES_D64 = [
     # (prefix_lens, chunk_lens, Hq, Hkv, cap)
     ([300], [130], 2, 2, 512),                     # two tiles, ragged second tile
-    ([1900, 10, 0], [300, 1, 1], 4, 4, 2304),      # two key splits per tile + decode rows
+    ([3900, 10, 0], [300, 1, 1], 4, 4, 4304),      # one, then two key splits per tile + decode rows
     ([1000, 77, 4000], [129, 1, 1], 16, 2, 4200),  # GQA (G = 8)
     ([3000, 5], [4, 4], 32, 8, 3072),              # verification, head-packed tiles (G = 4)
+    ([5000, 50, 2000], [300, 1, 40], 32, 4, 5400),  # 10,912 (row, head) pairs: many-pair combine
 ]
 
 

@@ -217,6 +217,18 @@ def test_cuda_graph_replay_new_lengths():
     del g
 
 
+def test_many_pairs_combine():
+    # 300 sequences x 32 query heads = 9,600 (row, head) pairs with 3 splits each: the combine's
+    # many-pair warp kernel (4 splits in flight per warp)
+    rng = np.random.default_rng(950)
+    lens = [int(x) for x in rng.integers(0, 601, size=300)]
+    inp = make_decode_inputs(300, 32, 4, 128, 600, lens, torch.bfloat16, seed=951, pad_fill=NAN)
+    out, lse = _run(inp, 3)
+    ro, rl = _oracle(inp)
+    check_out(out, ro, "many pairs out")
+    check_lse(lse, rl, "many pairs lse")
+
+
 @pytest.mark.parametrize("B", [255, 256, 257])
 def test_batch_around_in_kernel_plan_limit(B):
     # up to 256 sequences the tensor-core kernel plans the call itself; above, the planner kernel

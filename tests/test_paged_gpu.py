@@ -162,7 +162,7 @@ def test_paged_rejects_bad_layouts():
 
 
 @pytest.mark.parametrize("layout", ["head_major", "kv_pool"])
-@pytest.mark.parametrize("psz", [8, 16, 64])
+@pytest.mark.parametrize("psz", [8, 16, 32, 64])
 def test_paged_pool_layouts(layout, psz):
     # pools that are not [pages, Hkv, page_size, D] contiguous:
     # - head_major: stored [Hkv, pages, page_size, D] (a page's KV heads are not consecutive, so
