@@ -132,6 +132,10 @@ fd_status fd_decode_attention(const fd_tensor* q, const fd_tensor* k_cache,
  *                                               one (page, head) must be contiguous
  *                                               (stride[2] == D); strides multiples of 16 bytes,
  *                                               data 16-byte aligned; k and v share strides.
+ *                                               Any page stride is accepted; bf16 pages of < 128
+ *                                               keys whose heads are consecutive (stride[1] ==
+ *                                               page_size * D) are read with one copy per page,
+ *                                               other head strides with two.
  *  block_table  [B, pages_per_seq] int32 (device, contiguous rows): physical page of each
  *               logical page. Entries past a sequence's last page are never dereferenced as
  *               memory addresses (they may hold any value, e.g. -1).
