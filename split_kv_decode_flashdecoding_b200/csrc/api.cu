@@ -598,8 +598,8 @@ fd_status decode_call(const fd_tensor* q, const fd_tensor* k_cache, const fd_ten
   } else {
     // the tensor-core kernel reads whole 128-key tiles: with a bf16 cache, splits that end on a
     // tile boundary (no partly used tile in the middle of a sequence) run ~2% faster at the
-    // 70B-like shape; an E4M3 cache ran 20% slower that way (measured A/B), so it keeps
-    // unaligned splits
+    // 70B-like shape; an E4M3 cache runs ~2% slower that way (225 vs 230 us, measured A/B; 20%
+    // before the wait loop went out of line), so it keeps unaligned splits
     dp.align = (sh.use_tc && !sh.kv_fp8) ? kTcKeyAlign : 1;
   }
   // an E4M3 cache: k_scale multiplies every score, v_scale every output (both linear)
